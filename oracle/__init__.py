@@ -1,0 +1,208 @@
+"""ORACLE - test infrastructure, not part of the library.
+
+Plain CPU statement of the weight-only quantized linear (``oracle.c``), loaded
+with ctypes.  Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py`` may import this package; the library never does.
+
+Functions take and return numpy arrays in the canonical (pre-pack) layouts
+listed in ``oracle.c``.  bf16 tensors travel as uint16 bit patterns.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+FORMATS = {"int4_sym": 0, "int4_asym": 1, "int8_sym": 2, "cb4": 3, "nvfp4": 4}
+
+
+def build(force: bool = False, extra_flags=(), out_path: str | None = None,
+          src: str | None = None) -> str:
+    """Compile ``oracle.c`` with gcc.  ``src``/``out_path`` let a test build a
+    deliberately altered copy of the source elsewhere."""
+    out = out_path or _LIB_PATH
+    src = src or _SRC
+    if (not force and out_path is None and os.path.exists(out)
+            and os.path.getmtime(out) >= os.path.getmtime(_SRC)):
+        return out
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+           "-fno-fast-math", *extra_flags, "-o", tmp, src, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, out)
+    return out
+
+
+def _declare(lib):
+    i64, ptr, c_int, dbl = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_double
+    sig = {
+        "orc_bf16_to_f32": ([ctypes.c_uint16], ctypes.c_float),
+        "orc_f64_to_bf16": ([dbl], ctypes.c_uint16),
+        "orc_e2m1_value": ([c_int], dbl),
+        "orc_e2m1_encode": ([dbl], c_int),
+        "orc_e4m3_value": ([c_int], dbl),
+        "orc_e4m3_encode": ([dbl], c_int),
+        "orc_quant_int_sym": ([ptr, i64, i64, c_int, c_int, ptr, ptr], c_int),
+        "orc_quant_int4_asym": ([ptr, i64, i64, c_int, ptr, ptr, ptr], c_int),
+        "orc_lloyd_max_gaussian": ([c_int, ptr, ptr, ptr, ptr], c_int),
+        "orc_quant_cb4": ([ptr, i64, i64, ptr, ptr, ptr], c_int),
+        "orc_quant_nvfp4": ([ptr, i64, i64, ptr, ptr, ptr], c_int),
+        "orc_dequant": ([c_int, i64, i64, c_int, ptr, ptr, ptr, ptr], c_int),
+        "orc_linear": ([ptr, ptr, ptr, i64, i64, i64, ptr, ptr], c_int),
+        "orc_linear_sampled": ([c_int, i64, i64, c_int, ptr, ptr, ptr, ptr, ptr, i64, ptr, ptr,
+                                ptr, ptr], c_int),
+        "orc_threads": ([], c_int),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+
+
+def load(path: str | None = None):
+    """The oracle library (built on first use).  ``path`` loads another build."""
+    global _lib
+    if path is not None:
+        lib = ctypes.CDLL(path)
+        _declare(lib)
+        return lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB_PATH)
+            _declare(lib)
+            _lib = lib
+        return _lib
+
+
+def _p(a):
+    if a is None:
+        return None
+    assert isinstance(a, np.ndarray) and a.flags["C_CONTIGUOUS"], "contiguous numpy array expected"
+    return a.ctypes.data
+
+
+def _ok(rc, what):
+    if rc != 0:
+        raise ValueError(f"oracle {what} rejected its arguments (code {rc})")
+
+
+class Oracle:
+    """Thin numpy front end over one build of ``oracle.c``."""
+
+    def __init__(self, lib=None):
+        self.lib = lib if lib is not None else load()
+
+    # ---- scalar codecs
+    def bf16_to_f32(self, bits: int) -> float:
+        return float(self.lib.orc_bf16_to_f32(bits))
+
+    def f64_to_bf16(self, v: float) -> int:
+        return int(self.lib.orc_f64_to_bf16(v))
+
+    def e2m1_value(self, code: int) -> float:
+        return float(self.lib.orc_e2m1_value(code))
+
+    def e2m1_encode(self, r: float) -> int:
+        return int(self.lib.orc_e2m1_encode(r))
+
+    def e4m3_value(self, code: int) -> float:
+        return float(self.lib.orc_e4m3_value(code))
+
+    def e4m3_encode(self, d: float) -> int:
+        return int(self.lib.orc_e4m3_encode(d))
+
+    # ---- quantizers -> canonical layout
+    def quantize(self, fmt: str, W: np.ndarray, group_size: int = 0, centroids=None):
+        """Returns (codes, scales, aux) in the canonical layout of ``fmt``."""
+        W = np.ascontiguousarray(W, dtype=np.float32)
+        N, K = W.shape
+        G = group_size
+        if fmt in ("int4_sym", "int8_sym"):
+            bits = 4 if fmt == "int4_sym" else 8
+            codes = np.zeros((N, K // 2) if bits == 4 else (N, K),
+                             dtype=np.uint8 if bits == 4 else np.int8)
+            scales = np.zeros((N, K // G), dtype=np.uint16)
+            _ok(self.lib.orc_quant_int_sym(_p(W), N, K, G, bits, _p(codes), _p(scales)), fmt)
+            return codes, scales, None
+        if fmt == "int4_asym":
+            codes = np.zeros((N, K // 2), dtype=np.uint8)
+            scales = np.zeros((N, K // G), dtype=np.uint16)
+            zeros = np.zeros((N, K // G), dtype=np.uint8)
+            _ok(self.lib.orc_quant_int4_asym(_p(W), N, K, G, _p(codes), _p(scales), _p(zeros)), fmt)
+            return codes, scales, zeros
+        if fmt == "cb4":
+            c = self.lloyd_max(16)[1] if centroids is None else np.ascontiguousarray(
+                centroids, dtype=np.float32)
+            codes = np.zeros((N, K // 2), dtype=np.uint8)
+            norms = np.zeros((N,), dtype=np.uint16)
+            _ok(self.lib.orc_quant_cb4(_p(W), N, K, _p(c), _p(codes), _p(norms)), fmt)
+            return codes, norms, c
+        if fmt == "nvfp4":
+            codes = np.zeros((N, K // 2), dtype=np.uint8)
+            bs = np.zeros((N, K // 16), dtype=np.uint8)
+            ts = np.zeros((1,), dtype=np.float32)
+            _ok(self.lib.orc_quant_nvfp4(_p(W), N, K, _p(codes), _p(bs), _p(ts)), fmt)
+            return codes, bs, ts
+        raise ValueError(fmt)
+
+    def lloyd_max(self, levels: int = 16):
+        """(c64, c32, iterations, mse) of the Lloyd-Max quantizer of N(0,1)."""
+        c64 = np.zeros((levels,), dtype=np.float64)
+        c32 = np.zeros((levels,), dtype=np.float32)
+        it = ctypes.c_int(0)
+        mse = ctypes.c_double(0.0)
+        _ok(self.lib.orc_lloyd_max_gaussian(levels, _p(c64), _p(c32), ctypes.byref(it),
+                                            ctypes.byref(mse)), "lloyd_max")
+        return c64, c32, it.value, mse.value
+
+    # ---- dequant / linear
+    def dequant(self, fmt: str, codes, scales, aux, N: int, K: int, group_size: int = 0):
+        out = np.zeros((N, K), dtype=np.float32)
+        _ok(self.lib.orc_dequant(FORMATS[fmt], N, K, group_size, _p(codes), _p(scales), _p(aux),
+                                 _p(out)), "dequant")
+        return out
+
+    def linear(self, x_bits: np.ndarray, dq: np.ndarray, bias_bits=None):
+        """(y_bf16_bits [M,N], y_f64 [M,N]) for y = x . dq^T + bias."""
+        x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+        dq = np.ascontiguousarray(dq, dtype=np.float32)
+        M, K = x_bits.shape
+        N = dq.shape[0]
+        assert dq.shape[1] == K
+        y = np.zeros((M, N), dtype=np.uint16)
+        y64 = np.zeros((M, N), dtype=np.float64)
+        b = None if bias_bits is None else np.ascontiguousarray(bias_bits, dtype=np.uint16)
+        _ok(self.lib.orc_linear(_p(x_bits), _p(dq), _p(b), M, N, K, _p(y), _p(y64)), "linear")
+        return y, y64
+
+    def linear_sampled(self, fmt: str, codes, scales, aux, N: int, K: int, group_size: int,
+                       x_bits, bias_bits, ms, ns):
+        ms = np.ascontiguousarray(ms, dtype=np.int64)
+        ns = np.ascontiguousarray(ns, dtype=np.int64)
+        S = ms.size
+        y = np.zeros((S,), dtype=np.uint16)
+        y64 = np.zeros((S,), dtype=np.float64)
+        x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+        b = None if bias_bits is None else np.ascontiguousarray(bias_bits, dtype=np.uint16)
+        _ok(self.lib.orc_linear_sampled(FORMATS[fmt], N, K, group_size, _p(codes), _p(scales),
+                                        _p(aux), _p(x_bits), _p(b), S, _p(ms), _p(ns), _p(y),
+                                        _p(y64)), "linear_sampled")
+        return y, y64
+
+    def threads(self) -> int:
+        return int(self.lib.orc_threads())
+
+
+def bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> float32 values (exact widening)."""
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)

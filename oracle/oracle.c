@@ -1,0 +1,454 @@
+/*
+ * ORACLE - test infrastructure, not part of the library.
+ *
+ * A plain, slow CPU statement of what the weight-only quantized linear
+ * computes:  Y[M,N] = X[M,K] . dequant(Wq)[N,K]^T + bias,  X/Y/bias in bf16.
+ * Only the tests, the smoke check and the benchmark's CPU-baseline leg may
+ * load this file; the CUDA library never does, and the two share no code.
+ *
+ * Sources (the pages print no formula for any quantizer, so every format
+ * below is the plainest reading the pages support; each reading is named):
+ *  - piper-kernels README, "ConvRot INT8": group-wise INT8 weight, group 256,
+ *    weight shape [out_features, in_features].
+ *  - Mamba-2 paired-nibble state file, pack/dequant helpers: symmetric RTN
+ *    with scale = amax/qmax, clamp to +-qmax, half-precision scales, element
+ *    2i in the low nibble and 2i+1 in the high nibble, signed nibble
+ *    v = n - 16*[n > 7].
+ *  - auto-round-lib README, section 1 "Linear": INT4/INT8 weight-only GEMM,
+ *    sym and asym (zero-point) variants, per-group scales along K.
+ *  - OrbitQuant packed matmul card, "API"/"Inputs": uint8 row-major packed
+ *    codebook indices, per-row norms (bf16 on CUDA), fp32 Lloyd-Max
+ *    centroids [2**bits].
+ *  - Petit README, "Features"/"Known limitations": NVFP4 weights, positive
+ *    scales, no negative-zero codes.
+ *  - NVFP4 itself: E2M1 values, one E4M3 scale per 16 consecutive K
+ *    elements, one fp32 tensor scale (format definition).
+ *
+ * Readings taken where the pages are silent:
+ *  - rounding of w/s to an integer: round half to even;
+ *  - a scale is rounded once to bf16 and w is divided by the stored scale;
+ *  - an all-zero group / row / block gets scale 0 and code 0;
+ *  - INT4 emits [-7, 7], INT8 emits [-127, 127];
+ *  - asym INT4: lo = min(0, min w), hi = max(0, max w), s = bf16((hi-lo)/15),
+ *    z = clamp(rne(-lo/s), 0, 15), q = clamp(rne(w/s) + z, 0, 15),
+ *    dq = (q - z) * s;
+ *  - codebook: norm = bf16(||w_row||_2 / sqrt(K)), idx = argmin_j
+ *    |w/norm - c_j| with ties to the lower j, dq = fp32(c[idx] * norm);
+ *  - NVFP4: ts = fp32(amax / (6*448)), sb = E4M3_rne_satfinite(amax_b /
+ *    (6*ts)), q = E2M1_rne_sat(w / (e4m3(sb)*ts)), -0 written as +0,
+ *    dq = fp32(e2m1(q) * e4m3(sb) * ts);  the tensor scale multiplies.
+ *  - Lloyd-Max: the 2**bits-level quantizer of N(0,1), computed by the
+ *    classical fixed-point iteration (thresholds at midpoints, levels at
+ *    conditional means) from a uniform start on [-3, 3], in fp64, then cast
+ *    to fp32.
+ *  - y = sum_k x*dq accumulated in fp64 in increasing k, plus bias, rounded
+ *    once to bf16 (round to nearest even).
+ *
+ * Canonical (pre-pack) layouts, the input of the library's pack step:
+ *   int4_sym : codes u8 [N, K/2] two's complement nibbles; scales bf16 [N, K/G]
+ *   int4_asym: codes u8 [N, K/2] nibbles 0..15; scales bf16 [N, K/G];
+ *              zeros u8 [N, K/G] (one per byte, 0..15)
+ *   int8_sym : codes i8 [N, K]; scales bf16 [N, K/G]
+ *   cb4      : codes u8 [N, K/2] indices; norms bf16 [N]; centroids f32 [16]
+ *   nvfp4    : codes u8 [N, K/2] E2M1 nibbles; block scales u8 [N, K/16] E4M3;
+ *              tensor scale f32 [1]
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+enum { ORC_INT4_SYM = 0, ORC_INT4_ASYM = 1, ORC_INT8_SYM = 2, ORC_CB4 = 3, ORC_NVFP4 = 4 };
+
+/* ------------------------------------------------------------------ bf16 */
+float orc_bf16_to_f32(uint16_t h) {
+  uint32_t b = (uint32_t)h << 16;
+  float f;
+  memcpy(&f, &b, 4);
+  return f;
+}
+
+/* Round a double to the nearest bf16 (ties to even).  bf16 keeps 8 significant
+ * bits; below 2^-126 the spacing is fixed at 2^-133. */
+uint16_t orc_f64_to_bf16(double v) {
+  if (isnan(v)) return 0x7FC0;
+  int neg = signbit(v) ? 1 : 0;
+  double a = fabs(v);
+  uint16_t sign = (uint16_t)(neg << 15);
+  if (a == 0.0) return sign;
+  if (isinf(a)) return (uint16_t)(sign | 0x7F80);
+  int e;
+  frexp(a, &e);           /* a = f * 2^e, f in [0.5, 1) */
+  int E = e - 1;          /* a = 1.xxx * 2^E */
+  if (E < -126) E = -126; /* subnormal spacing */
+  double quantum = ldexp(1.0, E - 7);
+  double r = nearbyint(a / quantum) * quantum;
+  if (r >= ldexp(1.0, 128)) return (uint16_t)(sign | 0x7F80);
+  float rf = (float)r; /* exact: r has at most 8 significant bits */
+  uint32_t b;
+  memcpy(&b, &rf, 4);
+  return (uint16_t)(sign | (b >> 16));
+}
+
+/* ------------------------------------------------------------------ E2M1 */
+static const double E2M1_MAG[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+double orc_e2m1_value(int code) {
+  double m = E2M1_MAG[code & 7];
+  return (code & 8) ? -m : m;
+}
+
+/* Nearest E2M1 code (ties to the even code), saturating at +-6; a result of
+ * magnitude 0 is written as +0. */
+int orc_e2m1_encode(double r) {
+  int neg = r < 0.0;
+  double a = fabs(r);
+  int code = 7;
+  for (int i = 0; i < 7; ++i) {
+    double mid = 0.5 * (E2M1_MAG[i] + E2M1_MAG[i + 1]);
+    if (a < mid) { code = i; break; }
+    if (a == mid) { code = (i % 2 == 0) ? i : i + 1; break; }
+  }
+  if (code == 0) return 0;
+  return code | (neg ? 8 : 0);
+}
+
+/* ------------------------------------------------------------------ E4M3 */
+/* E4M3 (fn variant): 1 sign, 4 exponent (bias 7), 3 mantissa bits; exponent 0
+ * is subnormal with spacing 2^-9; 0x7F / 0xFF are NaN; no infinity. */
+double orc_e4m3_value(int code) {
+  int s = (code >> 7) & 1, e = (code >> 3) & 15, m = code & 7;
+  double v;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0) v = ldexp((double)m, -9);
+  else v = ldexp(1.0 + m / 8.0, e - 7);
+  return s ? -v : v;
+}
+
+/* Nearest non-negative finite E4M3 code (ties to the even code), saturating
+ * to 448 (0x7E).  d must be >= 0. */
+int orc_e4m3_encode(double d) {
+  if (!(d > 0.0)) return 0;
+  if (d >= 448.0) return 0x7E;
+  /* codes 0..126 are increasing in value */
+  int lo = 0, hi = 126;
+  while (hi - lo > 1) { /* invariant: value(lo) <= d < value(hi) */
+    int mid = (lo + hi) / 2;
+    if (orc_e4m3_value(mid) <= d) lo = mid; else hi = mid;
+  }
+  double vl = orc_e4m3_value(lo), vh = orc_e4m3_value(hi);
+  double half = 0.5 * (vl + vh);
+  if (d < half) return lo;
+  if (d > half) return hi;
+  return (lo % 2 == 0) ? lo : hi;
+}
+
+/* ------------------------------------------------------------- nibbles */
+static inline int get_nib(const uint8_t* row, int64_t k) {
+  uint8_t b = row[k >> 1];
+  return (k & 1) ? (b >> 4) : (b & 15);
+}
+static inline void put_nib(uint8_t* row, int64_t k, int v) {
+  uint8_t* b = &row[k >> 1];
+  if (k & 1) *b = (uint8_t)((*b & 0x0F) | ((v & 15) << 4));
+  else *b = (uint8_t)((*b & 0xF0) | (v & 15));
+}
+
+/* ---------------------------------------------------------- quantizers */
+int orc_quant_int_sym(const float* W, int64_t N, int64_t K, int G, int bits, void* codes,
+                      uint16_t* scales) {
+  if (N <= 0 || K <= 0 || G <= 0 || K % G || (bits != 4 && bits != 8)) return 1;
+  int qmax = bits == 4 ? 7 : 127;
+  int64_t ng = K / G;
+  for (int64_t n = 0; n < N; ++n) {
+    const float* w = W + n * K;
+    uint8_t* row4 = (uint8_t*)codes + n * (K / 2);
+    int8_t* row8 = (int8_t*)codes + n * K;
+    if (bits == 4) memset(row4, 0, (size_t)(K / 2));
+    for (int64_t j = 0; j < ng; ++j) {
+      double amax = 0.0;
+      for (int64_t k = j * G; k < (j + 1) * G; ++k) amax = fmax(amax, fabs((double)w[k]));
+      uint16_t sb = orc_f64_to_bf16(amax / (double)qmax);
+      scales[n * ng + j] = sb;
+      double s = (double)orc_bf16_to_f32(sb);
+      for (int64_t k = j * G; k < (j + 1) * G; ++k) {
+        int q = 0;
+        if (s != 0.0) {
+          double r = nearbyint((double)w[k] / s);
+          if (r > qmax) r = qmax;
+          if (r < -qmax) r = -qmax;
+          q = (int)r;
+        }
+        if (bits == 4) put_nib(row4, k, q & 15);
+        else row8[k] = (int8_t)q;
+      }
+    }
+  }
+  return 0;
+}
+
+int orc_quant_int4_asym(const float* W, int64_t N, int64_t K, int G, uint8_t* codes,
+                        uint16_t* scales, uint8_t* zeros) {
+  if (N <= 0 || K <= 0 || G <= 0 || K % G || K % 2) return 1;
+  int64_t ng = K / G;
+  for (int64_t n = 0; n < N; ++n) {
+    const float* w = W + n * K;
+    uint8_t* row = codes + n * (K / 2);
+    memset(row, 0, (size_t)(K / 2));
+    for (int64_t j = 0; j < ng; ++j) {
+      double lo = 0.0, hi = 0.0;
+      for (int64_t k = j * G; k < (j + 1) * G; ++k) {
+        lo = fmin(lo, (double)w[k]);
+        hi = fmax(hi, (double)w[k]);
+      }
+      uint16_t sb = orc_f64_to_bf16((hi - lo) / 15.0);
+      scales[n * ng + j] = sb;
+      double s = (double)orc_bf16_to_f32(sb);
+      int z = 0;
+      if (s != 0.0) {
+        double zr = nearbyint(-lo / s);
+        if (zr < 0) zr = 0;
+        if (zr > 15) zr = 15;
+        z = (int)zr;
+      }
+      zeros[n * ng + j] = (uint8_t)z;
+      for (int64_t k = j * G; k < (j + 1) * G; ++k) {
+        int q = 0;
+        if (s != 0.0) {
+          double r = nearbyint((double)w[k] / s) + z;
+          if (r < 0) r = 0;
+          if (r > 15) r = 15;
+          q = (int)r;
+        }
+        put_nib(row, k, q);
+      }
+    }
+  }
+  return 0;
+}
+
+/* Standard normal mass on [a, b], taking the tail form that keeps precision. */
+static double normal_mass(double a, double b) {
+  const double r2 = 1.4142135623730950488016887242097;
+  if (a >= 0.0) return 0.5 * (erfc(a / r2) - erfc(b / r2));
+  if (b <= 0.0) return 0.5 * (erfc(-b / r2) - erfc(-a / r2));
+  return 0.5 * (erf(b / r2) - erf(a / r2));
+}
+static double normal_pdf(double x) {
+  if (isinf(x)) return 0.0;
+  return exp(-0.5 * x * x) / 2.5066282746310005024157652848110;
+}
+
+/* Lloyd-Max quantizer of N(0,1) with L levels (L >= 2): alternate
+ * thresholds t_i = (c_i + c_{i+1})/2 and levels
+ * c_i = (pdf(t_{i-1}) - pdf(t_i)) / (Phi(t_i) - Phi(t_{i-1})), the mean of
+ * N(0,1) restricted to the cell, until no level moves by 1e-14. */
+int orc_lloyd_max_gaussian(int L, double* c64, float* c32, int* iters_out, double* mse_out) {
+  if (L < 2 || L > 256) return 1;
+  double* c = (double*)malloc(sizeof(double) * L);
+  double* t = (double*)malloc(sizeof(double) * (L + 1));
+  if (!c || !t) { free(c); free(t); return 2; }
+  for (int i = 0; i < L; ++i) c[i] = -3.0 + 6.0 * i / (L - 1);
+  int it = 0;
+  for (; it < 1000000; ++it) {
+    t[0] = -INFINITY;
+    t[L] = INFINITY;
+    for (int i = 1; i < L; ++i) t[i] = 0.5 * (c[i - 1] + c[i]);
+    double moved = 0.0;
+    for (int i = 0; i < L; ++i) {
+      double p = normal_mass(t[i], t[i + 1]);
+      double nc = (normal_pdf(t[i]) - normal_pdf(t[i + 1])) / p;
+      moved = fmax(moved, fabs(nc - c[i]));
+      c[i] = nc;
+    }
+    if (moved < 1e-14) { ++it; break; }
+  }
+  /* mean squared error of the final quantizer:
+   * E[(Z - c_i)^2 ; cell i] = (1 + c_i^2) P_i - 2 c_i (pdf(a) - pdf(b))
+   *                           + a pdf(a) - b pdf(b)                  */
+  for (int i = 1; i < L; ++i) t[i] = 0.5 * (c[i - 1] + c[i]);
+  double mse = 0.0;
+  for (int i = 0; i < L; ++i) {
+    double a = t[i], b = t[i + 1];
+    double p = normal_mass(a, b);
+    double pa = normal_pdf(a), pb = normal_pdf(b);
+    double apa = isinf(a) ? 0.0 : a * pa, bpb = isinf(b) ? 0.0 : b * pb;
+    mse += (1.0 + c[i] * c[i]) * p - 2.0 * c[i] * (pa - pb) + apa - bpb;
+  }
+  for (int i = 0; i < L; ++i) {
+    if (c64) c64[i] = c[i];
+    if (c32) c32[i] = (float)c[i];
+  }
+  if (iters_out) *iters_out = it;
+  if (mse_out) *mse_out = mse;
+  free(c);
+  free(t);
+  return 0;
+}
+
+int orc_quant_cb4(const float* W, int64_t N, int64_t K, const float* centroids, uint8_t* codes,
+                  uint16_t* norms) {
+  if (N <= 0 || K <= 0 || K % 2) return 1;
+  for (int64_t n = 0; n < N; ++n) {
+    const float* w = W + n * K;
+    uint8_t* row = codes + n * (K / 2);
+    memset(row, 0, (size_t)(K / 2));
+    double ss = 0.0;
+    for (int64_t k = 0; k < K; ++k) ss += (double)w[k] * (double)w[k];
+    double norm64 = sqrt(ss) / sqrt((double)K);
+    uint16_t nb = orc_f64_to_bf16(norm64);
+    norms[n] = nb;
+    double nd = (double)orc_bf16_to_f32(nb);
+    for (int64_t k = 0; k < K; ++k) {
+      int best = 0;
+      if (nd != 0.0) {
+        double r = (double)w[k] / nd;
+        double bestd = fabs(r - (double)centroids[0]);
+        for (int j = 1; j < 16; ++j) {
+          double d = fabs(r - (double)centroids[j]);
+          if (d < bestd) { bestd = d; best = j; }
+        }
+      }
+      put_nib(row, k, best);
+    }
+  }
+  return 0;
+}
+
+int orc_quant_nvfp4(const float* W, int64_t N, int64_t K, uint8_t* codes, uint8_t* bscales,
+                    float* tscale) {
+  if (N <= 0 || K <= 0 || K % 16) return 1;
+  double amax = 0.0;
+  for (int64_t e = 0; e < N * K; ++e) amax = fmax(amax, fabs((double)W[e]));
+  float ts = (float)(amax / (6.0 * 448.0));
+  *tscale = ts;
+  int64_t nb = K / 16;
+  for (int64_t n = 0; n < N; ++n) {
+    const float* w = W + n * K;
+    uint8_t* row = codes + n * (K / 2);
+    memset(row, 0, (size_t)(K / 2));
+    for (int64_t b = 0; b < nb; ++b) {
+      double ab = 0.0;
+      for (int64_t k = b * 16; k < b * 16 + 16; ++k) ab = fmax(ab, fabs((double)w[k]));
+      int sb = 0;
+      if (ts != 0.0f) sb = orc_e4m3_encode(ab / (6.0 * (double)ts));
+      bscales[n * nb + b] = (uint8_t)sb;
+      double d = orc_e4m3_value(sb) * (double)ts;
+      for (int64_t k = b * 16; k < b * 16 + 16; ++k) {
+        int q = 0;
+        if (d != 0.0) q = orc_e2m1_encode((double)w[k] / d);
+        put_nib(row, k, q);
+      }
+    }
+  }
+  return 0;
+}
+
+/* ------------------------------------------------------------- dequant */
+/* Exact dequantized value of element (n, k) from the canonical layout. */
+static float dq_one(int fmt, int64_t K, int G, const void* codes, const void* scales,
+                    const void* aux, int64_t n, int64_t k) {
+  switch (fmt) {
+    case ORC_INT4_SYM: {
+      int nib = get_nib((const uint8_t*)codes + n * (K / 2), k);
+      int v = nib > 7 ? nib - 16 : nib;
+      float s = orc_bf16_to_f32(((const uint16_t*)scales)[n * (K / G) + k / G]);
+      return (float)v * s;
+    }
+    case ORC_INT4_ASYM: {
+      int q = get_nib((const uint8_t*)codes + n * (K / 2), k);
+      int z = ((const uint8_t*)aux)[n * (K / G) + k / G];
+      float s = orc_bf16_to_f32(((const uint16_t*)scales)[n * (K / G) + k / G]);
+      return (float)(q - z) * s;
+    }
+    case ORC_INT8_SYM: {
+      int v = ((const int8_t*)codes)[n * K + k];
+      float s = orc_bf16_to_f32(((const uint16_t*)scales)[n * (K / G) + k / G]);
+      return (float)v * s;
+    }
+    case ORC_CB4: {
+      int idx = get_nib((const uint8_t*)codes + n * (K / 2), k);
+      double c = (double)((const float*)aux)[idx];
+      double nr = (double)orc_bf16_to_f32(((const uint16_t*)scales)[n]);
+      return (float)(c * nr);
+    }
+    case ORC_NVFP4: {
+      int q = get_nib((const uint8_t*)codes + n * (K / 2), k);
+      int sb = ((const uint8_t*)scales)[n * (K / 16) + k / 16];
+      double ts = (double)((const float*)aux)[0];
+      return (float)(orc_e2m1_value(q) * orc_e4m3_value(sb) * ts);
+    }
+  }
+  return NAN;
+}
+
+static int check_fmt(int fmt, int64_t N, int64_t K, int G) {
+  if (N <= 0 || K <= 0) return 1;
+  if (fmt < 0 || fmt > 4) return 1;
+  if ((fmt == ORC_INT4_SYM || fmt == ORC_INT4_ASYM || fmt == ORC_INT8_SYM) && (G <= 0 || K % G))
+    return 1;
+  if (fmt != ORC_INT8_SYM && K % 2) return 1;
+  if (fmt == ORC_NVFP4 && K % 16) return 1;
+  return 0;
+}
+
+int orc_dequant(int fmt, int64_t N, int64_t K, int G, const void* codes, const void* scales,
+                const void* aux, float* out) {
+  if (check_fmt(fmt, N, K, G)) return 1;
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k) out[n * K + k] = dq_one(fmt, K, G, codes, scales, aux, n, k);
+  return 0;
+}
+
+/* -------------------------------------------------------------- linear */
+/* y[m,n] = sum_k x[m,k] * dq[n,k] (fp64, k increasing) + bias[n]; bf16 out.
+ * Every product of a bf16 and an fp32 is exact in fp64. */
+int orc_linear(const uint16_t* x, const float* dq, const uint16_t* bias, int64_t M, int64_t N,
+               int64_t K, uint16_t* y, double* y64) {
+  if (M < 0 || N <= 0 || K <= 0) return 1;
+#pragma omp parallel for schedule(dynamic, 16)
+  for (int64_t n = 0; n < N; ++n) {
+    const float* w = dq + n * K;
+    for (int64_t m = 0; m < M; ++m) {
+      const uint16_t* xr = x + m * K;
+      double acc = 0.0;
+      for (int64_t k = 0; k < K; ++k) acc += (double)orc_bf16_to_f32(xr[k]) * (double)w[k];
+      if (bias) acc += (double)orc_bf16_to_f32(bias[n]);
+      if (y64) y64[m * N + n] = acc;
+      if (y) y[m * N + n] = orc_f64_to_bf16(acc);
+    }
+  }
+  return 0;
+}
+
+/* The same value for chosen (m, n) pairs only, dequantizing row n on the fly
+ * from the canonical layout; for workloads too large for the full product. */
+int orc_linear_sampled(int fmt, int64_t N, int64_t K, int G, const void* codes,
+                       const void* scales, const void* aux, const uint16_t* x,
+                       const uint16_t* bias, int64_t S, const int64_t* ms, const int64_t* ns,
+                       uint16_t* y, double* y64) {
+  if (check_fmt(fmt, N, K, G)) return 1;
+#pragma omp parallel for schedule(dynamic, 4)
+  for (int64_t i = 0; i < S; ++i) {
+    int64_t m = ms[i], n = ns[i];
+    const uint16_t* xr = x + m * K;
+    double acc = 0.0;
+    for (int64_t k = 0; k < K; ++k)
+      acc += (double)orc_bf16_to_f32(xr[k]) *
+             (double)dq_one(fmt, K, G, codes, scales, aux, n, k);
+    if (bias) acc += (double)orc_bf16_to_f32(bias[n]);
+    if (y64) y64[i] = acc;
+    if (y) y[i] = orc_f64_to_bf16(acc);
+  }
+  return 0;
+}
+
+/* Threads that OpenMP uses for the parallel loops above. */
+int orc_threads(void);
+#ifdef _OPENMP
+#include <omp.h>
+int orc_threads(void) { return omp_get_max_threads(); }
+#else
+int orc_threads(void) { return 1; }
+#endif

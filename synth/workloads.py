@@ -1,0 +1,111 @@
+"""The five synthetic workloads of the weight-only quantized linear.
+
+Each recipe fixes shapes, the weight format, the group size, the seed and the
+value distributions; ``make_inputs`` draws the dense inputs for one of them.
+Format names are the library's: int4_sym, int4_asym, int8_sym, cb4, nvfp4.
+
+Readings (the recipe texts leave these open):
+  * seeds other than the first workload's are 1, 2, 3, 4 in order;
+  * "0.1% of entries replaced by x20 outliers" = round(0.001*N*K) distinct
+    positions whose drawn value is multiplied by 20;
+  * "1% of channels scaled x10" = round(0.01*K) distinct input columns of X
+    multiplied by 10;
+  * a bias whose sigma is not given reuses N(0, 0.01^2); a workload that does
+    not mention a bias has none.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+
+from . import activations, bias as draw_bias, weight
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    fmt: str
+    N: int
+    K: int
+    Ms: tuple
+    group_size: int
+    seed: int
+    w_dist: str = "normal"
+    w_sigma: float = 0.02
+    w_outlier_frac: float = 0.0
+    w_outlier_mult: float = 1.0
+    x_channel_frac: float = 0.0
+    x_channel_mult: float = 1.0
+    bias_sigma: float | None = None
+    note: str = ""
+
+    @property
+    def w_outlier_count(self) -> int:
+        return int(round(self.w_outlier_frac * self.N * self.K))
+
+    @property
+    def x_channel_count(self) -> int:
+        return int(round(self.x_channel_frac * self.K))
+
+
+PR1 = Workload("pr1_int4_sym_g64", "int4_sym", N=256, K=512, Ms=(4,), group_size=64, seed=0,
+               bias_sigma=0.01, note="first slice: INT4 sym g64, M=4")
+DECODE = Workload("decode_int4_asym_g128", "int4_asym", N=4096, K=4096, Ms=(1, 2, 4, 8, 16),
+                  group_size=128, seed=1, w_outlier_frac=0.001, w_outlier_mult=20.0,
+                  note="decode sweep on a 4096x4096 layer, asym INT4 + uint4 zero-point")
+CODEBOOK = Workload("codebook4_3072", "cb4", N=3072, K=3072, Ms=(1, 16, 256), group_size=0,
+                    seed=2, bias_sigma=0.01, note="4-bit Lloyd-Max codebook with row norms")
+NVFP4 = Workload("nvfp4_28672x8192", "nvfp4", N=28672, K=8192, Ms=(1, 8, 64, 256),
+                 group_size=16, seed=3, w_dist="student5",
+                 note="NVFP4 70B-class MLP up-projection shape")
+PREFILL = Workload("prefill_int8_g256", "int8_sym", N=8192, K=8192, Ms=(1024, 2048, 4096),
+                   group_size=256, seed=4, x_channel_frac=0.01, x_channel_mult=10.0,
+                   bias_sigma=0.01, note="compute-bound prefill, INT8 sym g256")
+
+ALL = (PR1, DECODE, CODEBOOK, NVFP4, PREFILL)
+BY_NAME = {w.name: w for w in ALL}
+
+
+def make_weight(w: Workload) -> np.ndarray:
+    return weight(w.seed, w.N, w.K, dist=w.w_dist, sigma=w.w_sigma,
+                  outlier_count=w.w_outlier_count, outlier_mult=w.w_outlier_mult)
+
+
+def make_x(w: Workload, M: int) -> np.ndarray:
+    """X[M, K] bf16 bits.  Row m is the same for every M (one stream per workload)."""
+    return activations(w.seed, M, w.K, sigma=1.0, channel_count=w.x_channel_count,
+                       channel_mult=w.x_channel_mult)
+
+
+def make_bias(w: Workload):
+    if w.bias_sigma is None:
+        return None
+    return draw_bias(w.seed, w.N, sigma=w.bias_sigma)
+
+
+def algorithmic_bytes(w: Workload, M: int, N: int | None = None, K: int | None = None) -> int:
+    """Bytes the linear must move once: packed W + scales + aux + X + Y + bias."""
+    N = w.N if N is None else N
+    K = w.K if K is None else K
+    return packed_bytes(w.fmt, N, K, w.group_size) + 2 * M * K + 2 * M * N + \
+        (2 * N if w.bias_sigma is not None else 0)
+
+
+def packed_bytes(fmt: str, N: int, K: int, G: int) -> int:
+    """Weight-side bytes: codes + scales + auxiliary data, for the given format."""
+    if fmt == "int4_sym":
+        return N * K // 2 + 2 * N * (K // G)
+    if fmt == "int4_asym":
+        return N * K // 2 + 2 * N * (K // G) + N * (K // G) // 2
+    if fmt == "int8_sym":
+        return N * K + 2 * N * (K // G)
+    if fmt == "cb4":
+        return N * K // 2 + 2 * N + 64
+    if fmt == "nvfp4":
+        return N * K // 2 + N * (K // 16) + 4
+    raise ValueError(fmt)
+
+
+def flops(M: int, N: int, K: int) -> int:
+    return 2 * M * N * K

@@ -1,0 +1,207 @@
+"""Pins of the oracle's quantizers and dequantizer: closed-form round trips,
+error bounds, code ranges and nearest-neighbour properties, checked against
+numpy/scipy/torch rather than against the oracle."""
+from __future__ import annotations
+
+import os
+
+import numpy as np
+import pytest
+from scipy import integrate, stats
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+E2M1 = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def _nibbles(codes):
+    """canonical u8 [N, K/2] -> u8 [N, K]: element 2i in the low nibble."""
+    lo = codes & 0x0F
+    hi = codes >> 4
+    return np.stack([lo, hi], axis=-1).reshape(codes.shape[0], -1)
+
+
+def _bf16(bits):
+    return oracle.bits_to_f32(bits).astype(np.float64)
+
+
+def _weights(N, K, seed=0, outliers=True):
+    W = synth.weight(seed, N, K, sigma=0.02, outlier_count=(N * K) // 500 if outliers else 0,
+                     outlier_mult=20.0)
+    W[0, :] = 0.0                # an all-zero row (and groups)
+    W[1, : K // 2] = 0.0
+    return W
+
+
+# --------------------------------------------------------------- symmetric INT
+@pytest.mark.parametrize("fmt,qmax", [("int4_sym", 7), ("int8_sym", 127)])
+@pytest.mark.parametrize("G", [32, 64, 128, 256])
+def test_sym_properties(orc, fmt, qmax, G):
+    N, K = 48, 512
+    W = _weights(N, K, seed=G)
+    codes, scales, _ = orc.quantize(fmt, W, G)
+    q = _nibbles(codes).astype(np.int64) if fmt == "int4_sym" else codes.astype(np.int64)
+    if fmt == "int4_sym":
+        q = np.where(q > 7, q - 16, q)
+    s = _bf16(scales)
+    assert np.all(np.abs(q) <= qmax)
+    qg = np.abs(q).reshape(N, K // G, G).max(-1)
+    wg = np.abs(W).reshape(N, K // G, G).max(-1)
+    # the largest element of every non-zero group lands on +-qmax
+    assert np.all(qg[wg > 0] == qmax)
+    assert np.all(s[wg == 0] == 0) and np.all(qg[wg == 0] == 0)
+    # error within half a step of the stored scale
+    sk = np.repeat(s, G, axis=1)
+    err = np.abs(q * sk - W.astype(np.float64))
+    assert np.all(err <= 0.5 * sk)
+    # the stored scale is amax/qmax rounded to bf16: within half a bf16 ulp (2^-8 relative)
+    ratio = s[wg > 0] / (wg[wg > 0] / qmax)
+    assert np.all(np.abs(ratio - 1) <= 2.0 ** -8)
+    # dequant = q * s exactly
+    dq = orc.dequant(fmt, codes, scales, None, N, K, G)
+    assert np.array_equal(dq.astype(np.float64), q * sk)
+
+
+@pytest.mark.parametrize("fmt,qmax", [("int4_sym", 7), ("int8_sym", 127)])
+@pytest.mark.parametrize("sval", [1.0, 2.0 ** -7, 0.0173])
+def test_sym_round_trip_every_code(orc, fmt, qmax, sval):
+    """W = q*s for every representable q gives back q and s exactly."""
+    s = float(oracle.bits_to_f32(np.array([orc.f64_to_bf16(sval)], np.uint16))[0])
+    G = 256
+    q = np.arange(-qmax, qmax + 1)
+    row = np.resize(q, G).astype(np.float64)
+    W = (row * s).astype(np.float32)[None, :].repeat(2, 0)
+    codes, scales, _ = orc.quantize(fmt, W, G)
+    assert np.all(_bf16(scales) == s)
+    got = _nibbles(codes).astype(np.int64) if fmt == "int4_sym" else codes.astype(np.int64)
+    if fmt == "int4_sym":
+        got = np.where(got > 7, got - 16, got)
+    assert np.array_equal(got[0], row.astype(np.int64))
+
+
+# --------------------------------------------------------------- asymmetric INT4
+@pytest.mark.parametrize("G", [32, 128])
+def test_asym_properties(orc, G):
+    N, K = 48, 512
+    W = _weights(N, K, seed=100 + G)
+    W[2, :] = np.abs(W[2, :])      # groups with min > 0 (lo clamps to 0)
+    W[3, :] = -np.abs(W[3, :])     # groups with max < 0
+    codes, scales, zeros = orc.quantize("int4_asym", W, G)
+    q = _nibbles(codes).astype(np.int64)
+    s = _bf16(scales)
+    z = zeros.astype(np.int64)
+    assert q.min() >= 0 and q.max() <= 15 and z.min() >= 0 and z.max() <= 15
+    w64 = W.astype(np.float64)
+    lo = np.minimum(0, w64.reshape(N, K // G, G).min(-1))
+    hi = np.maximum(0, w64.reshape(N, K // G, G).max(-1))
+    s32 = (hi - lo) / 15.0
+    # error bound: half a step, plus the bf16 rounding of the scale for clamped codes
+    sk = np.repeat(s, G, axis=1)
+    zk = np.repeat(z, G, axis=1)
+    allow = 0.5 * sk + 15 * np.repeat(np.abs(s32 - s), G, axis=1) + 1e-12
+    dq = orc.dequant("int4_asym", codes, scales, zeros, N, K, G)
+    assert np.array_equal(dq.astype(np.float64), (q - zk) * sk)
+    assert np.all(np.abs(dq - w64) <= allow)
+    nz = hi - lo > 0
+    assert np.all(np.abs(s[nz] / s32[nz] - 1) <= 2.0 ** -8)
+    assert np.all(s[~nz] == 0)
+
+
+def test_asym_round_trip(orc):
+    """W = (q - z)*s with every q in 0..15 present gives back q, z and s."""
+    G = 64
+    rows = []
+    for z in range(16):
+        q = np.resize(np.arange(16), G)
+        rows.append((q - z) * 0.03125)
+    W = np.array(rows, dtype=np.float32)
+    codes, scales, zeros = orc.quantize("int4_asym", W, G)
+    assert np.all(_bf16(scales) == 0.03125)
+    assert np.array_equal(zeros[:, 0], np.arange(16))
+    assert np.array_equal(_nibbles(codes), np.resize(np.arange(16), (16, G)))
+
+
+# --------------------------------------------------------------- Lloyd-Max
+def _max_table():
+    levels, mse = [], None
+    with open(os.path.join(GOLDEN, "lloyd_max_gaussian16.txt")) as f:
+        for line in f:
+            if line.startswith("level"):
+                levels.append(float(line.split()[1]))
+            elif line.startswith("mse"):
+                mse = float(line.split()[1])
+    return np.array(levels), mse
+
+
+def test_lloyd_max_invariants(orc):
+    c64, c32, iters, mse = orc.lloyd_max(16)
+    assert np.all(np.diff(c64) > 0)
+    assert np.max(np.abs(c64 + c64[::-1])) < 1e-12          # symmetric
+    assert np.array_equal(c32, c64.astype(np.float32))       # fp32 = RN(fp64)
+    t = np.concatenate([[-np.inf], (c64[1:] + c64[:-1]) / 2, [np.inf]])
+    q_mse = 0.0
+    for i in range(16):
+        mass = stats.norm.cdf(t[i + 1]) - stats.norm.cdf(t[i])
+        mean, _ = integrate.quad(lambda x: x * stats.norm.pdf(x), t[i], t[i + 1],
+                                 epsabs=1e-14, epsrel=1e-12)
+        assert abs(mean / mass - c64[i]) < 1e-9               # centroid condition
+        v, _ = integrate.quad(lambda x: (x - c64[i]) ** 2 * stats.norm.pdf(x), t[i], t[i + 1],
+                              epsabs=1e-15, epsrel=1e-12)
+        q_mse += v
+    assert abs(q_mse - mse) < 1e-10
+    levels, mse_tab = _max_table()
+    assert np.max(np.abs(c64[8:] - levels)) < 1e-3
+    assert abs(mse - mse_tab) < 1e-5
+
+
+# --------------------------------------------------------------- codebook
+def test_cb4_nearest_neighbour(orc):
+    N, K = 40, 256
+    W = _weights(N, K, seed=9)
+    _, c32, _, _ = orc.lloyd_max(16)
+    codes, norms, cent = orc.quantize("cb4", W, centroids=c32)
+    idx = _nibbles(codes).astype(np.int64)
+    nrm = _bf16(norms)
+    ref_norm = np.linalg.norm(W.astype(np.float64), axis=1) / np.sqrt(K)
+    nz = ref_norm > 0
+    assert np.all(np.abs(nrm[nz] / ref_norm[nz] - 1) <= 2.0 ** -8)
+    assert np.all(nrm[~nz] == 0) and np.all(idx[~nz] == 0)
+    r = W[nz].astype(np.float64) / nrm[nz][:, None]
+    d = np.abs(r[..., None] - c32.astype(np.float64)[None, None, :])
+    best = d.argmin(-1)     # first minimum = lower index on ties
+    assert np.array_equal(idx[nz], best)
+    dq = orc.dequant("cb4", codes, norms, cent, N, K)
+    want = (c32.astype(np.float64)[idx] * nrm[:, None]).astype(np.float32)
+    assert np.array_equal(dq, want)
+
+
+# --------------------------------------------------------------- NVFP4
+def test_nvfp4_properties(orc):
+    N, K = 64, 512
+    W = (0.02 * synth.student5_stream(3, 1, 0, N * K)).astype(np.float32).reshape(N, K)
+    W[5, 32:48] = 0.0              # an all-zero block
+    codes, bs, ts = orc.quantize("nvfp4", W)
+    q = _nibbles(codes).astype(np.int64)
+    assert not np.any(q == 8)                       # no negative zero
+    assert np.all(bs < 0x7F)                        # sign clear, never NaN
+    amax = np.abs(W.astype(np.float64)).max()
+    assert ts[0] == np.float32(amax / 2688.0)
+    mag = np.array(E2M1)[q & 7]
+    sgn = np.where(q & 8, -1.0, 1.0)
+    sbv = np.array([orc.e4m3_value(int(c)) for c in range(128)])[bs.astype(np.int64)]
+    sbk = np.repeat(sbv, 16, axis=1)
+    dq_exact = sgn * mag * sbk * float(ts[0])
+    dq = orc.dequant("nvfp4", codes, bs, ts, N, K)
+    assert np.array_equal(dq, dq_exact.astype(np.float32))
+    # the largest element of every block with a normal scale encodes to +-6
+    blk_max = (q & 7).reshape(N, K // 16, 16).max(-1)
+    normal = sbv >= 2.0 ** -6
+    assert np.all(blk_max[normal] == 7)
+    assert np.all(blk_max[sbv == 0] == 0)
+    # error: at most half the E2M1 gap at the value's magnitude (gap 2 above 4)
+    a = np.abs(W.astype(np.float64)) / (sbk * float(ts[0]) + (sbk == 0))
+    gap = np.where(a <= 2, 0.5, np.where(a <= 4, 1.0, 2.0))
+    err = np.abs(W.astype(np.float64) - dq_exact) / (sbk * float(ts[0]) + (sbk == 0))
+    assert np.all(err[sbk > 0] <= 0.5 * gap[sbk > 0] + 1e-12)
