@@ -1,0 +1,438 @@
+"""Benchmark of the weight-only quantized linear on B200.
+
+A step is one pass of the hot path over one batch: for the default workload
+(the decode sweep, asymmetric INT4 g128, K = N = 4096) one ``wq_linear`` call
+for each M in {1, 2, 4, 8, 16}, each on a different resident copy of the
+packed weight so that no call finds its weight in L2 (the copies together are
+more than three times the L2 size).  ``value`` is whole-job algorithmic
+GB/s: packed weight + scales + zero-points + X + Y bytes of every call,
+divided by the device time of the K timed steps (CUDA events, max over
+ranks).  The timed steps are replayed from CUDA graphs so that host launch
+overhead does not pad the device timeline.
+
+``e2e`` repeats the K steps through the public Python API with host
+activations: each call copies X from pinned host memory, runs the linear and
+copies Y back (both copies inside the timed region).
+
+``--impl reference`` times the CPU oracle (plain fp64 C, all host cores) on a
+bounded sample of the same workload and prints the same line with
+``"impl": "reference"``.
+
+Multi-GPU (torchrun): replicas only -- every rank runs the same workload on
+its own GPU, no data-path collective; the timing barrier and the max over
+ranks use the process group.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "quantized-linear GB/s (M≤16) and TFLOPS (M≥1024), % of roofline, 1 B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100000)
+    ap.add_argument("--warmup", type=int, default=2000)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode_int4_asym_g128")
+    ap.add_argument("--ms", default="", help="comma list overriding the workload's batch sizes")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: str):
+        self.gpu = gpu_index
+        self.proc = None
+        self.tmp = None
+
+    def start(self):
+        try:
+            self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.tmp.flush()
+        self.tmp.seek(0)
+        rows = [l.strip().split(", ") for l in self.tmp.read().splitlines() if l.strip()]
+        self.tmp.close()
+        try:
+            os.unlink(self.tmp.name)
+        except OSError:
+            pass
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                smax = float(r[2])
+                for i, nm in enumerate(names):
+                    if r[5 + i].strip().lower() == "active":
+                        reasons.add(nm)
+            except (ValueError, IndexError):
+                continue
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ workload
+def build_workload(wl, Ms, device, copies_min_bytes):
+    """Packed weight copies (quantized on the GPU by the library), X per M, bias."""
+    import torch
+
+    import mixed_gemm_b200 as wq
+    import synth.workloads as W
+
+    Wd = torch.from_numpy(W.make_weight(wl)).to(device)
+    pw = wq.quantize_and_pack(Wd, wl.fmt, wl.group_size)
+    del Wd
+    torch.cuda.synchronize()
+    R = max(2, int(math.ceil(copies_min_bytes / pw.nbytes)))
+    R = min(R, 256)
+    weights = [pw] + [pw.clone() for _ in range(R - 1)]
+    xs = {}
+    xa = W.make_x(wl, max(Ms))
+    for M in Ms:
+        xs[M] = torch.from_numpy(xa[:M].view(np.int16).copy()).view(torch.bfloat16).to(device)
+    b = W.make_bias(wl)
+    bias = None if b is None else torch.from_numpy(b.view(np.int16).copy()).view(
+        torch.bfloat16).to(device)
+    outs = {M: torch.empty((M, wl.N), dtype=torch.bfloat16, device=device) for M in Ms}
+    return weights, xs, bias, outs, xa
+
+
+def source_hash(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_file: str, workload: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, or None when the kernel source changed since it was taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e:
+        return None
+    src = [os.path.join(ROOT, "mixed_gemm_b200", "csrc", x) for x in e.get("sources", [])]
+    if not src or not all(os.path.exists(s) for s in src) or source_hash(src) != e.get("hash"):
+        return None
+    return e.get("bytes_per_launch")
+
+
+def cpu_sample(wl, Ms, rows, data):
+    """One bounded oracle pass: every token of every M against `rows` output rows."""
+    orc, codes, scales, aux, xa, b = data
+    t0 = time.perf_counter()
+    for M in Ms:
+        ms = np.repeat(np.arange(M), rows)
+        ns = np.tile(np.arange(rows) * (wl.N // rows), M)
+        orc.linear_sampled(wl.fmt, codes, scales, aux, wl.N, wl.K, wl.group_size, xa[:M], b,
+                           ms, ns)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(wl, Ms, seconds, calibrate_only=False):
+    """The oracle, as it stands, on a bounded sample of the workload (dequant
+    + fp64 dot products for a subset of output rows, every token); GB/s is the
+    workload's algorithmic bytes scaled by the fraction of rows computed."""
+    import oracle
+    import synth.workloads as W
+
+    orc = oracle.Oracle()
+    Wd = W.make_weight(wl)
+    codes, scales, aux = orc.quantize(wl.fmt, Wd, wl.group_size)
+    del Wd
+    xa = W.make_x(wl, max(Ms))
+    b = W.make_bias(wl)
+    data = (orc, codes, scales, aux, xa, b)
+    total_bytes = sum(W.algorithmic_bytes(wl, M) for M in Ms)
+    rows = 16
+    t = cpu_sample(wl, Ms, rows, data)
+    rows = int(min(wl.N, max(1, rows * seconds / max(t, 1e-4))))
+    desc = (f"{rows} of {wl.N} output rows for every token of M in {list(Ms)}, "
+            f"{orc.threads()} threads")
+    bytes_per_sample = total_bytes * rows / wl.N
+    if calibrate_only:
+        return {"rows": rows, "data": data, "cores": orc.threads(), "sample_desc": desc,
+                "bytes_per_sample": bytes_per_sample}, 0.0
+    t = cpu_sample(wl, Ms, rows, data)
+    value = bytes_per_sample / t / 1e9
+    return {"value": value, "unit": "GB/s", "cores": orc.threads(), "kind": "oracle",
+            "sample": desc + f" ({t:.1f} s)"}, t
+
+
+# ------------------------------------------------------------------ main
+def main():
+    args = parse()
+    import synth.workloads as W
+
+    wl = W.BY_NAME[args.workload]
+    Ms = tuple(int(m) for m in args.ms.split(",")) if args.ms else wl.Ms
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    tflops_metric = min(Ms) >= 1024
+    unit = "TFLOP/s" if tflops_metric else "GB/s"
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        # each step: the oracle on a bounded sample, sized so that warm-up and
+        # timed steps together take about a minute of host time
+        per_step = min(12.0, max(0.05, 60.0 / max(1, args.steps + args.warmup)))
+        cb, _ = cpu_baseline(wl, Ms, per_step, calibrate_only=True)
+        rows = cb["rows"]
+        for _ in range(args.warmup):
+            cpu_sample(wl, Ms, rows, cb["data"])
+        times = [cpu_sample(wl, Ms, rows, cb["data"]) for _ in range(max(1, args.steps))]
+        t = sum(times)
+        value = len(times) * cb["bytes_per_sample"] / t / 1e9
+        desc = {"value": value, "unit": "GB/s", "cores": cb["cores"], "kind": "oracle",
+                "sample": cb["sample_desc"]}
+        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+                "n_gpus": args.gpus, "steps": len(times), "warmup": args.warmup,
+                "ms_per_step": t / len(times) * 1e3, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": wl.name, "N": wl.N, "K": wl.K, "Ms": list(Ms),
+                           "format": wl.fmt, "group_size": wl.group_size},
+                "cpu_baseline": desc,
+                "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    else:
+        torch.cuda.set_device(0)
+    device = torch.device("cuda", torch.cuda.current_device())
+
+    import mixed_gemm_b200 as wq
+
+    props = torch.cuda.get_device_properties(device)
+    l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20)
+    weights, xs, bias, outs, xa = build_workload(wl, Ms, device, 3 * l2)
+    R = len(weights)
+    launches_per_step = len(Ms)
+    step_bytes = sum(W.algorithmic_bytes(wl, M) for M in Ms)
+    step_flops = sum(W.flops(M, wl.N, wl.K) for M in Ms)
+    stream = torch.cuda.Stream(device)
+    counter = [0]
+
+    def step():
+        for M in Ms:
+            pw = weights[counter[0] % R]
+            counter[0] += 1
+            wq.wq_linear(xs[M], pw.w, pw.scales, pw.aux, bias, M, wl.N, wl.K, wl.fmt,
+                         wl.group_size, outs[M], stream)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier(device_ids=[local_rank])
+
+    # graphs of C steps each (the weight copies rotate inside the graph)
+    C = max(1, min(200, args.steps))
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            step()
+    torch.cuda.synchronize()
+
+    def capture(nsteps):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(nsteps):
+                step()
+        return g
+
+    g_main = capture(C)
+    rem = args.steps % C
+    g_rem = capture(rem) if rem else None
+    reps = args.steps // C
+
+    # warm-up: W untimed steps
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup // C):
+            g_main.replay()
+        for _ in range(args.warmup % C):
+            step()
+    torch.cuda.synchronize()
+
+    uuid = getattr(props, "uuid", None)
+    clocks = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(device.index))
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    ev0.record(stream)
+    for _ in range(reps):
+        g_main.replay()
+    if g_rem is not None:
+        g_rem.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms_total = ev0.elapsed_time(ev1)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms_total], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    sec = ms_total / 1e3
+    if tflops_metric:
+        value = world * args.steps * step_flops / sec / 1e12
+    else:
+        value = world * args.steps * step_bytes / sec / 1e9
+    per_launch_s = sec / (args.steps * launches_per_step)
+
+    # roofline of the dominant kernel (every launch in the step runs it)
+    pk, pk_kind = peaks()
+    if tflops_metric:
+        achieved = step_flops / launches_per_step / per_launch_s / 1e12
+        peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        bound, r_unit = "tensor", "TFLOP/s"
+    else:
+        achieved = step_bytes / launches_per_step / per_launch_s / 1e9
+        peak = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        bound, r_unit = "hbm", "GB/s"
+    kern_src = ["wq_decode.cu", "wq_internal.cuh"] if max(Ms) <= 16 else ["wq_prefill.cu",
+                                                                            "wq_internal.cuh"]
+    traffic = recorded_traffic(kern_src[0], wl.name)
+
+    # e2e through the public API with host activations
+    e2e = None
+    if not args.no_e2e:
+        xh = {M: torch.from_numpy(xa[:M].view(np.int16).copy()).view(torch.bfloat16).pin_memory()
+              for M in Ms}
+        yh = {M: torch.empty((M, wl.N), dtype=torch.bfloat16).pin_memory() for M in Ms}
+        e2e_steps = max(3, min(args.steps, 2000))
+        k = [0]
+
+        def e2e_step():
+            for M in Ms:
+                pw = weights[k[0] % R]
+                k[0] += 1
+                wq.linear(xh[M], pw, bias, out=yh[M])
+
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(e2e_steps):
+                e2e_step()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            import torch.distributed as dist
+            t = torch.tensor([e_ms], device=device, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        es = e_ms / 1e3
+        ev = world * e2e_steps * (step_flops / 1e12 if tflops_metric else step_bytes / 1e9) / es
+        e2e = {"value": ev, "unit": unit, "steps": e2e_steps,
+               "h2d_bytes_per_step": sum(M * wl.K * 2 for M in Ms),
+               "d2h_bytes_per_step": sum(M * wl.N * 2 for M in Ms)}
+
+    cb = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb, _ = cpu_baseline(wl, Ms, args.cpu_seconds)
+
+    if world > 1:
+        import torch.distributed as dist
+        del g_main, g_rem
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "format": wl.fmt, "group_size": wl.group_size,
+                   "N": wl.N, "K": wl.K, "Ms": list(Ms), "parallelism": f"replicas{world}",
+                   "l2": f"rotating {R} packed-weight copies ({R * weights[0].nbytes / 2**20:.0f} "
+                         f"MiB > 3x L2 {l2 / 2**20:.0f} MiB)",
+                   "timing": f"CUDA graphs of {C} steps, CUDA events on the launch stream"},
+        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": r_unit,
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": pk_kind,
+                     "kernel": "decode_kernel" if max(Ms) <= 16 else "prefill_kernel"},
+        "gpu_launches": args.steps * launches_per_step,
+        "clocks": clk,
+        "e2e": e2e,
+        "cpu_baseline": cb,
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,172 @@
+/*
+ * wq.h - C ABI of the B200 weight-only quantized linear.
+ *
+ *     Y[M,N] = X[M,K] . dequant(Wq)[N,K]^T + bias          X, Y, bias: bf16
+ *
+ * The weights stay packed in device memory and are expanded tile by tile
+ * inside the kernels, never as a full bf16 matrix.  This is the operation of
+ * the OrbitQuant packed matmul card ("API": matmul_packed_weight consumes
+ * packed indices, row norms and centroids "directly, avoiding a full BF16/FP16
+ * dequantized weight cache"), of the auto-round-lib README (section 1
+ * "Linear": woqgemm over a repacked weight blob, activation [M,K] ->
+ * output [M,N], optional bias [1,N]), of the Petit README ("Features": dense
+ * FP16/BF16 x NVFP4 GEMM) and of the piper-kernels README ("ConvRot INT8":
+ * group-wise INT8 weight used as a normal linear weight).
+ *
+ * Conventions shared by every entry point
+ *  - Every pointer named "device" is CUDA device memory owned by the caller;
+ *    the library never allocates, frees or keeps a pointer after returning.
+ *  - Every call is asynchronous on `stream` (0 = legacy default stream) unless
+ *    its comment says it synchronizes.  No entry point allocates memory.
+ *  - Arguments are checked on the host first; a failed check returns a status
+ *    other than WQ_OK and launches nothing.  A launch failure is reported as
+ *    WQ_ERR_CUDA (from cudaGetLastError).  No C++ exception crosses the ABI.
+ *  - bf16 values are IEEE bfloat16 bit patterns (uint16_t).
+ *  - Shapes: N % 16 == 0 and K % 64 == 0 for every format (the packed tile is
+ *    16 rows by 64 (4-bit) or 32 (INT8) K elements); INT formats take
+ *    group_size in {32, 64, 128, 256} with K % group_size == 0; NVFP4 has a
+ *    fixed block of 16 (group_size 16 or 0); CB4 ignores group_size.
+ *  - Every device pointer must be 16-byte aligned, except the NVFP4 tensor
+ *    scale and the CB4 centroids (4-byte aligned).
+ *
+ * Canonical (unpacked) layouts -- what wq_quantize writes and wq_pack reads.
+ * Rows are output features n (the weight is [out_features, in_features] as
+ * in the ConvRot INT8 section), groups run along K:
+ *   WQ_INT4_SYM : codes  u8 [N, K/2]  two's complement nibbles, element 2i in
+ *                                      the low nibble (the nibble order of the
+ *                                      Mamba-2 paired-nibble pack helper)
+ *                 scales bf16 [N, K/G]
+ *   WQ_INT4_ASYM: codes  u8 [N, K/2]  unsigned nibbles 0..15, same order
+ *                 scales bf16 [N, K/G];  aux = zeros u8 [N, K/G] (0..15)
+ *   WQ_INT8_SYM : codes  i8 [N, K];    scales bf16 [N, K/G]
+ *   WQ_CB4      : codes  u8 [N, K/2]  codebook indices, same nibble order
+ *                 scales = row norms bf16 [N]; aux = centroids f32 [16]
+ *   WQ_NVFP4    : codes  u8 [N, K/2]  E2M1 nibbles, same nibble order
+ *                 scales = block scales u8 [N, K/16] (E4M3)
+ *                 aux = tensor scale f32 [1]
+ * Dequantized value of element (n, k) -- what wq_dequant returns:
+ *   INT4_SYM/INT8_SYM: q * s            ASYM: (q - z) * s          (exact fp32)
+ *   CB4: fp32(c[idx] * norm[n])         NVFP4: fp32(e2m1(q) * e4m3(sb) * ts)
+ */
+#ifndef WQ_H_
+#define WQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Packed weight formats (auto-round-lib "Supported Data Types"; OrbitQuant
+ * card "Inputs"; Petit "Features"). */
+typedef enum {
+  WQ_INT4_SYM = 0,  /* symmetric INT4, bf16 scale per group                    */
+  WQ_INT4_ASYM = 1, /* asymmetric INT4, bf16 scale + uint4 zero-point per group */
+  WQ_INT8_SYM = 2,  /* symmetric INT8, bf16 scale per group                    */
+  WQ_CB4 = 3,       /* 4-bit codebook: 16 fp32 centroids, bf16 norm per row    */
+  WQ_NVFP4 = 4      /* E2M1 values, E4M3 scale per 16, fp32 tensor scale       */
+} wq_format_t;
+
+typedef enum {
+  WQ_OK = 0,
+  WQ_ERR_INVALID_ARG = 1,  /* null pointer, bad shape, bad format, bad group   */
+  WQ_ERR_UNSUPPORTED = 2,  /* valid request this build has no kernel for        */
+  WQ_ERR_ALIGNMENT = 3,    /* a pointer is not aligned as required              */
+  WQ_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed              */
+  WQ_ERR_DEVICE_CHECK = 5  /* a kernel's own check failed (bad input found)      */
+} wq_status_t;
+
+/* Human-readable name of a status; never NULL. */
+const char* wq_status_string(int status);
+
+/* Sizes in bytes of the three canonical buffers (codes, scales, aux) and of
+ * the three packed buffers of one weight; pure host arithmetic, any pointer
+ * may be NULL.  Packed and canonical buffers have the same sizes except the
+ * ASYM zero-points (two per byte once packed).
+ * Source: auto-round-lib README section 1 (repack_quantized_weight sizes the
+ * ARK blob from n, k, blocksize and the weight/scale types). */
+int wq_canonical_sizes(int format, int64_t N, int64_t K, int group_size, size_t* codes_bytes,
+                       size_t* scales_bytes, size_t* aux_bytes);
+int wq_packed_sizes(int format, int64_t N, int64_t K, int group_size, size_t* w_bytes,
+                    size_t* scales_bytes, size_t* aux_bytes);
+
+/* Offline reorder of canonical codes, scales and aux into the packed layout
+ * the kernels stream (16-row tiles whose 512-byte blocks hand every lane of a
+ * warp its tensor-core fragments in one 16-byte load; nibbles interleaved for
+ * two-at-a-time conversion; scales and zero-points grouped per tile).
+ * Source: Petit README "Techniques and performance" (weights shuffled offline,
+ * as Marlin does, to make GPU dequantization efficient); auto-round-lib
+ * README section 1 (repack_quantized_weight).
+ * All six buffers are device memory; canonical and packed must not overlap.
+ * Checks every NVFP4 block scale (sign clear, not NaN 0x7F) and every NVFP4
+ * code (no negative zero 0x8), as the Petit README "Known limitations"
+ * requires; that check synchronizes `stream` and returns
+ * WQ_ERR_DEVICE_CHECK when it fails.  Other formats do not synchronize. */
+int wq_pack(int format, int64_t N, int64_t K, int group_size, const void* codes,
+            const void* scales, const void* aux, void* packed_w, void* packed_scales,
+            void* packed_aux, void* stream);
+
+/* Inverse of wq_pack: packed (device) -> canonical (device). */
+int wq_unpack(int format, int64_t N, int64_t K, int group_size, const void* packed_w,
+              const void* packed_scales, const void* packed_aux, void* codes, void* scales,
+              void* aux, void* stream);
+
+/* Test export: out_f32[N, K] (device, row-major) = the exact dequantized
+ * weight (definitions above) read from the packed buffers.
+ * Source: auto-round-lib README section 1 (unpack_weight, "decompose back to
+ * full precision for verification"). */
+int wq_dequant(int format, int64_t N, int64_t K, int group_size, const void* packed_w,
+               const void* packed_scales, const void* packed_aux, float* out_f32, void* stream);
+
+/* The hot path.  Y[M,N] = X[M,K] . dequant(W)[N,K]^T (+ bias[N]).
+ *   x        device bf16 [M, K] row-major
+ *   packed_w device, from wq_pack
+ *   scales   device: INT formats packed group scales; CB4 row norms;
+ *            NVFP4 packed E4M3 block scales
+ *   aux      device: ASYM packed zero-points; CB4 centroids f32[16];
+ *            NVFP4 tensor scale f32[1]; NULL for INT4_SYM / INT8_SYM
+ *   bias     device bf16 [N], or NULL
+ *   out      device bf16 [M, N] row-major; must not overlap any input
+ * M == 0 is a no-op returning WQ_OK.  Asynchronous; no workspace.
+ * M <= 16 runs the decode kernel (register dequant, warp-level tensor-core
+ * fragments, split-K over warps); larger M runs the prefill kernel (TMA into
+ * shared memory, dequant to bf16 in shared memory, tcgen05 MMA into tensor
+ * memory).  Both end in the fused fold/bias/bf16 epilogue.
+ * Source: OrbitQuant card "API" (matmul_packed_weight(x, idx, row_norms,
+ * centroids, bits, out_features, in_features, bias)) and "Benchmark"
+ * (skinny batches decode-bound, larger batches GEMM-bound); auto-round-lib
+ * README section 1 (woqgemm(activation, packw, bias, n, k, groupsize, ...));
+ * Petit README "Techniques and performance" (batch below 16 vs larger). */
+int wq_linear(const void* x, const void* packed_w, const void* scales, const void* aux,
+              const void* bias, int64_t M, int64_t N, int64_t K, int format, int group_size,
+              void* out, void* stream);
+
+/* Offline round-to-nearest quantizer on the GPU: w_f32[N, K] (device) ->
+ * canonical codes / scales / aux (device), bit-identical to the CPU
+ * definitions listed above.  CB4 reads its 16 centroids from `aux`
+ * (device f32[16], left unchanged) and writes the row norms; NVFP4 writes the
+ * tensor scale into `aux`.  Synchronizes `stream` for NVFP4 (two passes).
+ * Source: piper-kernels README "ConvRot INT8" (ConvRotInt8Tensor.from_hp
+ * quantizes a dense weight, group_size=256); Mamba-2 pack helper (scale =
+ * amax/qmax, round, clamp). */
+int wq_quantize(int format, int64_t N, int64_t K, int group_size, const float* w_f32,
+                void* codes, void* scales, void* aux, void* stream);
+
+/* Host: the 2^bits-level Lloyd-Max quantizer of N(0,1) (bits 1..8), as fp32,
+ * ascending, written to centroids_out[2^bits] (host memory).  Fixed-point
+ * iteration in fp64 from a uniform start on [-3, 3] until no level moves by
+ * 1e-14.  Source: OrbitQuant card "Inputs" (fp32 Lloyd-Max centroids with
+ * shape [2**bits]). */
+int wq_lloyd_max_centroids(int bits, float* centroids_out);
+
+/* Device properties the dispatcher uses (SM count of the current device);
+ * exported for the benchmark's launch accounting.  Returns WQ_ERR_CUDA when
+ * no device is usable. */
+int wq_device_sm_count(int* sm_count);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WQ_H_ */

@@ -1,0 +1,103 @@
+"""User-facing helpers over the C ABI: a packed weight handle and ``linear``.
+
+torch provides device memory and streams only; quantization, packing and the
+linear itself run in ``libwq.so``.  This mirrors the reference APIs: a dense
+weight is quantized and repacked once (piper-kernels ``from_hp``,
+auto-round-lib ``repack_quantized_weight``), then used as a linear weight
+(``F.linear`` / ``woqgemm`` / ``matmul_packed_weight``).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+from . import (FORMATS, wq_canonical_sizes, wq_linear, wq_lloyd_max_centroids, wq_pack,
+               wq_packed_sizes, wq_quantize)
+
+
+@dataclass
+class PackedWeight:
+    """Packed buffers of one [N, K] weight, resident on a CUDA device."""
+    fmt: str
+    N: int
+    K: int
+    group_size: int
+    w: torch.Tensor        # packed codes (uint8)
+    scales: torch.Tensor   # packed scales (uint8 view of the bytes)
+    aux: torch.Tensor | None
+
+    @property
+    def nbytes(self) -> int:
+        return self.w.numel() + self.scales.numel() + (0 if self.aux is None else self.aux.numel())
+
+    def clone(self) -> "PackedWeight":
+        return PackedWeight(self.fmt, self.N, self.K, self.group_size, self.w.clone(),
+                            self.scales.clone(), None if self.aux is None else self.aux.clone())
+
+
+def _bytes(n: int, device) -> torch.Tensor:
+    # at least 16 bytes so every buffer has a valid, aligned address
+    return torch.empty((max(int(n), 16),), dtype=torch.uint8, device=device)
+
+
+def pack(fmt: str, N: int, K: int, group_size: int, codes: torch.Tensor, scales: torch.Tensor,
+         aux: torch.Tensor | None, stream=None) -> PackedWeight:
+    """Canonical device buffers -> PackedWeight (wq_pack)."""
+    dev = codes.device
+    wb, sb, ab = wq_packed_sizes(fmt, N, K, group_size)
+    pw, ps = _bytes(wb, dev), _bytes(sb, dev)
+    pa = _bytes(ab, dev) if ab else None
+    wq_pack(fmt, N, K, group_size, codes, scales, aux, pw, ps, pa, stream)
+    return PackedWeight(fmt, N, K, group_size, pw, ps, pa)
+
+
+def quantize_and_pack(w: torch.Tensor, fmt: str, group_size: int = 0, centroids=None,
+                      stream=None) -> PackedWeight:
+    """Dense fp32 [N, K] device weight -> round-to-nearest quantized PackedWeight.
+
+    For ``cb4`` the 16 centroids default to the Lloyd-Max quantizer of N(0,1).
+    """
+    assert w.is_cuda and w.dtype == torch.float32 and w.is_contiguous()
+    N, K = w.shape
+    dev = w.device
+    cb, sb, ab = wq_canonical_sizes(fmt, N, K, group_size)
+    codes, scales = _bytes(cb, dev), _bytes(sb, dev)
+    aux = _bytes(ab, dev) if ab else None
+    if fmt == "cb4":
+        c = wq_lloyd_max_centroids(4) if centroids is None else centroids
+        aux.view(torch.float32)[:16].copy_(torch.as_tensor(c, dtype=torch.float32))
+    wq_quantize(fmt, N, K, group_size, w, codes, scales, aux, stream)
+    return pack(fmt, N, K, group_size, codes, scales, aux, stream)
+
+
+def linear(x: torch.Tensor, weight: PackedWeight, bias: torch.Tensor | None = None,
+           out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y = x @ dequant(weight).T + bias, bf16.  ``x``: [..., K] bf16.
+
+    A host (CPU) ``x`` is copied to the weight's device and the result copied
+    back, so the call works end to end from host memory.
+    """
+    host = not x.is_cuda
+    dev = weight.w.device
+    lead = x.shape[:-1]
+    K = x.shape[-1]
+    assert K == weight.K and x.dtype == torch.bfloat16
+    xd = x.reshape(-1, K)
+    if host:
+        xd = xd.to(dev, non_blocking=True)
+    xd = xd.contiguous()
+    M = xd.shape[0]
+    if bias is not None and not bias.is_cuda:
+        bias = bias.to(dev, non_blocking=True)
+    y = out if (out is not None and not host) else torch.empty((M, weight.N), dtype=torch.bfloat16,
+                                                               device=dev)
+    wq_linear(xd, weight.w, weight.scales, weight.aux, bias, M, weight.N, K, weight.fmt,
+              weight.group_size, y, stream)
+    if host:
+        yh = out if out is not None else torch.empty((M, weight.N), dtype=torch.bfloat16,
+                                                      pin_memory=True)
+        yh.copy_(y, non_blocking=True)
+        torch.cuda.current_stream(dev).synchronize()
+        return yh.reshape(*lead, weight.N)
+    return y.reshape(*lead, weight.N)

@@ -1,0 +1,227 @@
+// C ABI: argument checks, dispatch and the host-side helpers declared in
+// include/wq.h.  Every check runs on the host before anything is launched;
+// nothing here allocates device memory.
+#include <math.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "wq_internal.cuh"
+
+namespace wq {
+
+namespace {
+
+bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p % a) == 0; }
+
+// Shape / format checks shared by every entry point.
+int check_shape(int f, int64_t N, int64_t K, int G) {
+  if (f < INT4_SYM || f > NVFP4) return WQ_ERR_INVALID_ARG;
+  if (N <= 0 || K <= 0) return WQ_ERR_INVALID_ARG;
+  if (N % 16 || K % 64) return WQ_ERR_INVALID_ARG;
+  if (N > (1LL << 30) || K > (1LL << 24) || N * K > (1LL << 40)) return WQ_ERR_INVALID_ARG;
+  if (is_int_fmt(f)) {
+    if (G != 32 && G != 64 && G != 128 && G != 256) return WQ_ERR_INVALID_ARG;
+    if (K % G) return WQ_ERR_INVALID_ARG;
+  } else if (f == NVFP4) {
+    if (G != 0 && G != 16) return WQ_ERR_INVALID_ARG;
+  }
+  return WQ_OK;
+}
+
+int effective_group(int f, int G) { return f == NVFP4 ? 16 : (f == CB4 ? 0 : G); }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA; }
+
+std::mutex g_sm_mutex;
+int g_sm_count[64];
+bool g_sm_known[64];
+
+}  // namespace
+
+int device_sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  std::lock_guard<std::mutex> lk(g_sm_mutex);
+  if (dev >= 0 && dev < 64 && g_sm_known[dev]) return g_sm_count[dev];
+  int n = 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 148;
+  if (dev >= 0 && dev < 64) {
+    g_sm_count[dev] = n;
+    g_sm_known[dev] = true;
+  }
+  return n;
+}
+
+}  // namespace wq
+
+using namespace wq;
+
+extern "C" {
+
+const char* wq_status_string(int s) {
+  switch (s) {
+    case WQ_OK: return "ok";
+    case WQ_ERR_INVALID_ARG: return "invalid argument";
+    case WQ_ERR_UNSUPPORTED: return "unsupported";
+    case WQ_ERR_ALIGNMENT: return "misaligned pointer";
+    case WQ_ERR_CUDA: return "CUDA error";
+    case WQ_ERR_DEVICE_CHECK: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+int wq_canonical_sizes(int f, int64_t N, int64_t K, int G, size_t* cb, size_t* sb, size_t* ab) {
+  int st = check_shape(f, N, K, G);
+  if (st) return st;
+  G = effective_group(f, G);
+  size_t c = 0, s = 0, a = 0;
+  switch (f) {
+    case INT4_SYM: c = N * K / 2; s = 2 * N * (K / G); break;
+    case INT4_ASYM: c = N * K / 2; s = 2 * N * (K / G); a = N * (K / G); break;
+    case INT8_SYM: c = N * K; s = 2 * N * (K / G); break;
+    case CB4: c = N * K / 2; s = 2 * N; a = 64; break;
+    case NVFP4: c = N * K / 2; s = N * (K / 16); a = 4; break;
+  }
+  if (cb) *cb = c;
+  if (sb) *sb = s;
+  if (ab) *ab = a;
+  return WQ_OK;
+}
+
+int wq_packed_sizes(int f, int64_t N, int64_t K, int G, size_t* wb, size_t* sb, size_t* ab) {
+  int st = wq_canonical_sizes(f, N, K, G, wb, sb, ab);
+  if (st) return st;
+  if (f == INT4_ASYM && ab) *ab = N * (K / G) / 2;
+  return WQ_OK;
+}
+
+int wq_pack(int f, int64_t N, int64_t K, int G, const void* codes, const void* scales,
+            const void* aux, void* pw, void* ps, void* pa, void* stream) {
+  int st = check_shape(f, N, K, G);
+  if (st) return st;
+  G = effective_group(f, G);
+  bool need_aux = f == INT4_ASYM || f == CB4 || f == NVFP4;
+  if (!codes || !scales || !pw || !ps || (need_aux && (!aux || !pa))) return WQ_ERR_INVALID_ARG;
+  return cuda_status(launch_pack(f, N, K, G, codes, scales, aux, pw, ps, pa, (cudaStream_t)stream));
+}
+
+int wq_unpack(int f, int64_t N, int64_t K, int G, const void* pw, const void* ps, const void* pa,
+              void* codes, void* scales, void* aux, void* stream) {
+  int st = check_shape(f, N, K, G);
+  if (st) return st;
+  G = effective_group(f, G);
+  bool need_aux = f == INT4_ASYM || f == CB4 || f == NVFP4;
+  if (!codes || !scales || !pw || !ps || (need_aux && (!aux || !pa))) return WQ_ERR_INVALID_ARG;
+  return cuda_status(launch_unpack(f, N, K, G, pw, ps, pa, codes, scales, aux, (cudaStream_t)stream));
+}
+
+int wq_dequant(int f, int64_t N, int64_t K, int G, const void* pw, const void* ps, const void* pa,
+               float* out, void* stream) {
+  int st = check_shape(f, N, K, G);
+  if (st) return st;
+  G = effective_group(f, G);
+  bool need_aux = f == INT4_ASYM || f == CB4 || f == NVFP4;
+  if (!pw || !ps || !out || (need_aux && !pa)) return WQ_ERR_INVALID_ARG;
+  return cuda_status(launch_dequant(f, N, K, G, pw, ps, pa, out, (cudaStream_t)stream));
+}
+
+int wq_quantize(int f, int64_t N, int64_t K, int G, const float* w, void* codes, void* scales,
+                void* aux, void* stream) {
+  int st = check_shape(f, N, K, G);
+  if (st) return st;
+  G = effective_group(f, G);
+  bool need_aux = f == INT4_ASYM || f == CB4 || f == NVFP4;
+  if (!w || !codes || !scales || (need_aux && !aux)) return WQ_ERR_INVALID_ARG;
+  if (!aligned(w, 4) || (aux && !aligned(aux, 4))) return WQ_ERR_ALIGNMENT;
+  return cuda_status(launch_quantize(f, N, K, G, w, codes, scales, aux, (cudaStream_t)stream));
+}
+
+int wq_linear(const void* x, const void* pw, const void* scales, const void* aux, const void* bias,
+              int64_t M, int64_t N, int64_t K, int f, int G, void* out, void* stream) {
+  int st = check_shape(f, N, K, G);
+  if (st) return st;
+  if (M < 0 || M > (1LL << 24)) return WQ_ERR_INVALID_ARG;
+  G = effective_group(f, G);
+  bool need_aux = f == INT4_ASYM || f == CB4 || f == NVFP4;
+  if (!x || !pw || !scales || !out || (need_aux && !aux)) return WQ_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(pw, 16) || !aligned(scales, 16) || !aligned(out, 16) ||
+      (bias && !aligned(bias, 16)) || (aux && !aligned(aux, (f == INT4_ASYM) ? 16 : 4)))
+    return WQ_ERR_ALIGNMENT;
+  // the output must not overlap an input
+  const uintptr_t o0 = (uintptr_t)out, o1 = o0 + (uintptr_t)(M * N * 2);
+  auto overlaps = [&](const void* p, uintptr_t bytes) {
+    uintptr_t a0 = (uintptr_t)p, a1 = a0 + bytes;
+    return p && a0 < o1 && o0 < a1;
+  };
+  size_t wb = 0, sb = 0, ab = 0;
+  wq_packed_sizes(f, N, K, G, &wb, &sb, &ab);
+  if (M > 0 && (overlaps(x, (uintptr_t)(M * K * 2)) || overlaps(pw, wb) || overlaps(scales, sb) ||
+                overlaps(aux, ab) || overlaps(bias, (uintptr_t)(N * 2))))
+    return WQ_ERR_INVALID_ARG;
+  if (M == 0) return WQ_OK;
+  LinearArgs a;
+  a.x = x;
+  a.w = pw;
+  a.scales = scales;
+  a.aux = aux;
+  a.bias = bias;
+  a.out = out;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.fmt = f;
+  a.G = G;
+  a.stream = (cudaStream_t)stream;
+  cudaError_t e;
+  if (M <= 16) {
+    e = launch_decode(a);
+  } else {
+    e = launch_prefill(a);
+  }
+  return cuda_status(e);
+}
+
+// Lloyd-Max quantizer of N(0,1): thresholds at the midpoints of adjacent
+// levels, each level the mean of N(0,1) over its cell, iterated from a
+// uniform start on [-3, 3] until no level moves by 1e-14.
+int wq_lloyd_max_centroids(int bits, float* out) {
+  if (bits < 1 || bits > 8 || !out) return WQ_ERR_INVALID_ARG;
+  const int L = 1 << bits;
+  double lev[256], edge[257];
+  const double inv_sqrt2 = 0.70710678118654752440084436210485;
+  const double inv_sqrt2pi = 0.39894228040143267793994605993438;
+  auto pdf = [&](double t) { return isinf(t) ? 0.0 : inv_sqrt2pi * exp(-0.5 * t * t); };
+  // probability of (a, b] under N(0,1), using the complementary error
+  // function on the side away from the mean to keep tail cells accurate
+  auto mass = [&](double a, double b) {
+    if (a >= 0.0) return 0.5 * (erfc(a * inv_sqrt2) - erfc(b * inv_sqrt2));
+    if (b <= 0.0) return 0.5 * (erfc(-b * inv_sqrt2) - erfc(-a * inv_sqrt2));
+    return 0.5 * (erf(b * inv_sqrt2) - erf(a * inv_sqrt2));
+  };
+  for (int i = 0; i < L; ++i) lev[i] = -3.0 + 6.0 * i / (L - 1);
+  for (int it = 0; it < 1000000; ++it) {
+    edge[0] = -INFINITY;
+    edge[L] = INFINITY;
+    for (int i = 1; i < L; ++i) edge[i] = 0.5 * (lev[i - 1] + lev[i]);
+    double moved = 0.0;
+    for (int i = 0; i < L; ++i) {
+      double nl = (pdf(edge[i]) - pdf(edge[i + 1])) / mass(edge[i], edge[i + 1]);
+      moved = fmax(moved, fabs(nl - lev[i]));
+      lev[i] = nl;
+    }
+    if (moved < 1e-14) break;
+  }
+  for (int i = 0; i < L; ++i) out[i] = (float)lev[i];
+  return WQ_OK;
+}
+
+int wq_device_sm_count(int* n) {
+  if (!n) return WQ_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return WQ_ERR_CUDA;
+  *n = device_sm_count();
+  return WQ_OK;
+}
+
+}  // extern "C"

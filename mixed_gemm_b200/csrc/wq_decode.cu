@@ -1,0 +1,367 @@
+// Decode path (M <= 16): stream the packed weight once from HBM.
+//
+// Work split.  A CTA owns RT row tiles (16 output features each) and a slice
+// of K; a cluster of CS CTAs covers all of K for those rows; the KW warps of a
+// CTA split the CTA's K slice again.  Every lane issues one 16-byte
+// no-L1-allocate load per row tile and 512-byte block, which holds exactly its
+// tensor-core A fragments for that block (layout in wq_internal.cuh), and one
+// 16-byte load of the 8 matching activations per token row.  Codes become
+// bf16 in registers (magic-number nibble conversion for INT4, fp32 magic for
+// INT8, byte-permute table lookups for CB4 and NVFP4) and feed
+// mma.sync.m16n8k16 with the W rows as the 16-row operand and the (<= 16)
+// tokens as the 8-column operand.  INT group scales are applied per 32-K
+// chunk to the fp32 chunk accumulator (so the bf16 fragments are the exact
+// integer codes); NVFP4 block scales are multiplied into the fragments (the
+// product e2m1*e4m3 is exact in bf16); the CB4 row norm and the NVFP4 tensor
+// scale are applied in the epilogue.  Partial sums are reduced across warps
+// through shared memory and across the cluster through distributed shared
+// memory (no global workspace), then rank 0 applies fold + bias, rounds to
+// bf16 and stores.
+//
+// Sources: OrbitQuant card "Benchmark" (skinny batches are decode-bound; the
+// Metal path dispatches a skinny GEMV for up to four rows with decoded weight
+// segments reused across the batch); Petit README "Techniques and
+// performance" (batches below 16 are the small-batch regime, weights shuffled
+// offline for cheap dequantization).
+#include <cooperative_groups.h>
+
+#include "wq_internal.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace wq {
+
+namespace {
+
+struct DecodeParams {
+  const uint16_t* x;
+  const uint4* w;
+  const void* scales;
+  const void* aux;
+  const uint16_t* bias;
+  uint16_t* out;
+  int M, N, K, G, cs;
+};
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ uint4 ld_nc(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t word(const uint4& v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t bsub2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+__device__ __forceinline__ uint32_t f32_to_bf16_bits(float v) {
+  return pack_bf16x2(v, 0.f) & 0xFFFFu;
+}
+
+// INT4, "magic" nibble order: fragment i = nibbles (i, i+4) as bf16 (128 + n),
+// minus the per-row offset (136 for offset-binary signed codes, 128 + z).
+__device__ __forceinline__ void frag_int4(uint32_t wd, uint32_t off_g, uint32_t off_g8,
+                                          uint32_t (&a)[4]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t t = ((wd >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
+    a[i] = bsub2(t, (i & 1) ? off_g8 : off_g);
+  }
+}
+
+// INT8 offset-binary bytes -> exact integers via the fp32 magic 2^23 + u.
+__device__ __forceinline__ float i8val(uint32_t w, int i) {
+  return __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7440u | i)) - 8388736.0f;
+}
+__device__ __forceinline__ void frag_int8(uint32_t wg, uint32_t wg8, uint32_t (&a)[4]) {
+  a[0] = pack_bf16x2(i8val(wg, 0), i8val(wg, 1));
+  a[1] = pack_bf16x2(i8val(wg8, 0), i8val(wg8, 1));
+  a[2] = pack_bf16x2(i8val(wg, 2), i8val(wg, 3));
+  a[3] = pack_bf16x2(i8val(wg8, 2), i8val(wg8, 3));
+}
+
+// 16-entry bf16 lookup ("table" nibble order): byte tables H (high bytes) and
+// L (low bytes), four entries per register.  `kSymLow` means the low-byte
+// table does not depend on the top index bit (true for E2M1).
+template <bool kSymLow>
+__device__ __forceinline__ void frag_table(uint32_t wd, const uint32_t (&H)[4],
+                                           const uint32_t (&L)[4], uint32_t (&a)[4]) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t x = h ? (wd >> 16) : wd;
+    uint32_t sel = x & 0x7777u;
+    uint32_t mask = __byte_perm(0u, 0xFFFFFFFFu, (x >> 1) & 0x4444u);
+    uint32_t hb = (__byte_perm(H[0], H[1], sel) & ~mask) | (__byte_perm(H[2], H[3], sel) & mask);
+    uint32_t lb;
+    if (kSymLow) lb = __byte_perm(L[0], L[1], sel);
+    else lb = (__byte_perm(L[0], L[1], sel) & ~mask) | (__byte_perm(L[2], L[3], sel) & mask);
+    a[2 * h] = __byte_perm(lb, hb, 0x5140u);
+    a[2 * h + 1] = __byte_perm(lb, hb, 0x7362u);
+  }
+}
+
+template <int FMT, int NT, int RT, int KW, int UB>
+__global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
+  constexpr int KB = FMT == INT8_SYM ? 32 : 64;   // K per 512-byte block
+  constexpr int CPB = FMT == INT8_SYM ? 1 : 2;    // 32-K chunks per block
+  constexpr int NV = RT * NT * 4;                  // accumulators per lane
+  constexpr bool kIntFmt = FMT == INT4_SYM || FMT == INT4_ASYM || FMT == INT8_SYM;
+
+  extern __shared__ float red[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, tq = lane & 3;
+  const int cs = p.cs;
+  const int rank = (int)(blockIdx.x % cs);
+  const int64_t tile0 = (int64_t)(blockIdx.x / cs) * RT;
+  const int64_t K = p.K;
+  const int64_t nblk = K / KB;
+  const int64_t groups = kIntFmt ? K / p.G : 0;
+
+  const int64_t cb = rank * nblk / cs, ce = (rank + 1) * nblk / cs;
+  const int64_t wb = cb + warp * (ce - cb) / KW, we = cb + (warp + 1) * (ce - cb) / KW;
+
+  // lookup tables (CB4: centroids rounded to bf16; NVFP4: E2M1 values)
+  uint32_t H[4] = {0, 0, 0, 0}, L[4] = {0, 0, 0, 0};
+  if constexpr (FMT == NVFP4) {
+    H[0] = 0x3F3F3F00u; H[1] = 0x40404040u; H[2] = 0xBFBFBF80u; H[3] = 0xC0C0C0C0u;
+    L[0] = 0xC0800000u; L[1] = 0xC0804000u; L[2] = L[0]; L[3] = L[1];
+  }
+  if constexpr (FMT == CB4) {
+    const float* cen = (const float*)p.aux;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      uint32_t b = f32_to_bf16_bits(__ldg(cen + j));
+      H[j >> 2] |= (b >> 8) << (8 * (j & 3));
+      L[j >> 2] |= (b & 0xFFu) << (8 * (j & 3));
+    }
+  }
+
+  float acc[RT][NT][4];
+#pragma unroll
+  for (int r = 0; r < RT; ++r)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[r][nt][i] = 0.f;
+
+  const uint4 zero4 = make_uint4(0, 0, 0, 0);
+  for (int64_t b0 = wb; b0 < we; b0 += UB) {
+    uint4 wv[UB][RT];
+#pragma unroll
+    for (int u = 0; u < UB; ++u)
+#pragma unroll
+      for (int r = 0; r < RT; ++r)
+        wv[u][r] = (b0 + u < we) ? ld_stream(p.w + ((tile0 + r) * nblk + b0 + u) * 32 + lane)
+                                 : zero4;
+#pragma unroll
+    for (int u = 0; u < UB; ++u) {
+      if (b0 + u >= we) break;
+      const int64_t kblk = (b0 + u) * KB;
+      uint4 xv[CPB][NT];
+#pragma unroll
+      for (int c = 0; c < CPB; ++c)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const int tok = g + 8 * nt;
+          xv[c][nt] = tok < p.M ? ld_nc(p.x + tok * K + kblk + 32 * c + 8 * tq) : zero4;
+        }
+#pragma unroll
+      for (int c = 0; c < CPB; ++c) {
+        const int64_t k0 = kblk + 32 * c;
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+          const int64_t tile = tile0 + r;
+          if constexpr (kIntFmt) {
+            const int64_t grp = k0 / p.G;
+            const uint32_t sw = __ldg((const uint32_t*)p.scales + (tile * groups + grp) * 8 + g);
+            uint32_t off_g = 0x43084308u, off_g8 = 0x43084308u;  // 136 = 128 + 8
+            if constexpr (FMT == INT4_ASYM) {
+              const uint32_t zb = __ldg((const uint8_t*)p.aux + (tile * groups + grp) * 8 + g);
+              off_g = (0x4300u + (zb & 15u)) * 0x00010001u;
+              off_g8 = (0x4300u + (zb >> 4)) * 0x00010001u;
+            }
+            float cacc[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+              for (int i = 0; i < 4; ++i) cacc[nt][i] = 0.f;
+#pragma unroll
+            for (int s = 0; s < 2; ++s) {
+              uint32_t a[4];
+              if constexpr (FMT == INT8_SYM) frag_int8(word(wv[u][r], 2 * s), word(wv[u][r], 2 * s + 1), a);
+              else frag_int4(word(wv[u][r], 2 * c + s), off_g, off_g8, a);
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt)
+                mma16816(cacc[nt], a, word(xv[c][nt], 2 * s), word(xv[c][nt], 2 * s + 1));
+            }
+            const float s_g = __uint_as_float(sw << 16), s_g8 = __uint_as_float(sw & 0xFFFF0000u);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              acc[r][nt][0] = fmaf(s_g, cacc[nt][0], acc[r][nt][0]);
+              acc[r][nt][1] = fmaf(s_g, cacc[nt][1], acc[r][nt][1]);
+              acc[r][nt][2] = fmaf(s_g8, cacc[nt][2], acc[r][nt][2]);
+              acc[r][nt][3] = fmaf(s_g8, cacc[nt][3], acc[r][nt][3]);
+            }
+          } else {
+            uint32_t sc_g = 0, sc_g8 = 0;
+            if constexpr (FMT == NVFP4) {
+              const int64_t blk = (k0 + 8 * tq) >> 4;
+              const uint32_t sb = __ldg((const uint16_t*)p.scales + (tile * (K >> 4) + blk) * 8 + g);
+              sc_g = f32_to_bf16_bits(e4m3_to_f32(sb & 0xFFu)) * 0x00010001u;
+              sc_g8 = f32_to_bf16_bits(e4m3_to_f32(sb >> 8)) * 0x00010001u;
+            }
+#pragma unroll
+            for (int s = 0; s < 2; ++s) {
+              uint32_t a[4];
+              frag_table<FMT == NVFP4>(word(wv[u][r], 2 * c + s), H, L, a);
+              if constexpr (FMT == NVFP4) {
+                a[0] = bmul2(a[0], sc_g);
+                a[1] = bmul2(a[1], sc_g8);
+                a[2] = bmul2(a[2], sc_g);
+                a[3] = bmul2(a[3], sc_g8);
+              }
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt)
+                mma16816(acc[r][nt], a, word(xv[c][nt], 2 * s), word(xv[c][nt], 2 * s + 1));
+            }
+          }
+        }
+      }
+    }
+  }
+
+  // ---- reduction: warps -> CTA partial (shared) -> cluster rank 0 (DSMEM)
+#pragma unroll
+  for (int r = 0; r < RT; ++r)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) red[(warp * NV + (r * NT + nt) * 4 + i) * 32 + lane] = acc[r][nt][i];
+  __syncthreads();
+  float* part = red + KW * NV * 32;
+  for (int idx = threadIdx.x; idx < NV * 32; idx += KW * 32) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < KW; ++w) s += red[w * NV * 32 + idx];
+    part[idx] = s;
+  }
+  if (cs > 1) cg::this_cluster().sync();
+  else __syncthreads();
+  if (rank == 0) {
+    float tsc = 1.f;
+    if constexpr (FMT == NVFP4) tsc = __ldg((const float*)p.aux);
+    for (int idx = threadIdx.x; idx < NV * 32; idx += KW * 32) {
+      float tot = part[idx];
+      for (int q = 1; q < cs; ++q) tot += cg::this_cluster().map_shared_rank(part, q)[idx];
+      const int v = idx >> 5, ln = idx & 31;
+      const int r = v / (NT * 4), nt = (v / 4) % NT, i = v & 3;
+      const int gg = ln >> 2, tt = ln & 3;
+      const int64_t n = (tile0 + r) * 16 + gg + 8 * (i >> 1);
+      const int m = nt * 8 + 2 * tt + (i & 1);
+      if (m < p.M) {
+        float fold = tsc;
+        if constexpr (FMT == CB4) fold = bf16_bits_to_f32(__ldg((const uint16_t*)p.scales + n));
+        float y = tot * fold;
+        if (p.bias) y += bf16_bits_to_f32(__ldg(p.bias + n));
+        p.out[(int64_t)m * p.N + n] = (uint16_t)f32_to_bf16_bits(y);
+      }
+    }
+  }
+  if (cs > 1) cg::this_cluster().sync();
+}
+
+template <int FMT, int NT, int RT>
+cudaError_t launch_t(const DecodeParams& p, int grid, cudaStream_t st) {
+  constexpr int KW = 4, UB = 4;
+  auto kern = decode_kernel<FMT, NT, RT, KW, UB>;
+  const size_t smem = (size_t)(KW + 1) * RT * NT * 4 * 32 * sizeof(float);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(KW * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = p.cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = p.cs > 1 ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+template <int FMT>
+cudaError_t launch_fmt(const DecodeParams& p, int nt, int rt, int grid, cudaStream_t st) {
+  if (nt == 1) return rt == 2 ? launch_t<FMT, 1, 2>(p, grid, st) : launch_t<FMT, 1, 1>(p, grid, st);
+  return rt == 2 ? launch_t<FMT, 2, 2>(p, grid, st) : launch_t<FMT, 2, 1>(p, grid, st);
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const LinearArgs& a) {
+  DecodeParams p;
+  p.x = (const uint16_t*)a.x;
+  p.w = (const uint4*)a.w;
+  p.scales = a.scales;
+  p.aux = a.aux;
+  p.bias = (const uint16_t*)a.bias;
+  p.out = (uint16_t*)a.out;
+  p.M = (int)a.M;
+  p.N = (int)a.N;
+  p.K = (int)a.K;
+  p.G = a.G;
+  const int nt = a.M <= 8 ? 1 : 2;
+  const int64_t tiles = a.N / 16;
+  const int rt = (tiles % 2 == 0) ? 2 : 1;
+  const int64_t rowgroups = tiles / rt;
+  const int64_t nblk = a.K / block_k(a.fmt);
+  const int64_t target = 2LL * device_sm_count();
+  int64_t cs = (target + rowgroups - 1) / rowgroups;
+  if (cs > 8) cs = 8;
+  if (cs > nblk / 4) cs = nblk / 4;  // keep every warp busy
+  if (cs < 1) cs = 1;
+  p.cs = (int)cs;
+  const int grid = (int)(rowgroups * cs);
+  switch (a.fmt) {
+    case INT4_SYM: return launch_fmt<INT4_SYM>(p, nt, rt, grid, a.stream);
+    case INT4_ASYM: return launch_fmt<INT4_ASYM>(p, nt, rt, grid, a.stream);
+    case INT8_SYM: return launch_fmt<INT8_SYM>(p, nt, rt, grid, a.stream);
+    case CB4: return launch_fmt<CB4>(p, nt, rt, grid, a.stream);
+    case NVFP4: return launch_fmt<NVFP4>(p, nt, rt, grid, a.stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace wq

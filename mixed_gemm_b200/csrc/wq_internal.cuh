@@ -1,0 +1,126 @@
+// Internal declarations shared by the library's translation units.
+//
+// Packed layout (written by wq_pack, read by every kernel)
+// --------------------------------------------------------
+// Rows are grouped in tiles of 16 (n = 16*tile + r, r = g + 8*hr, g = 0..7,
+// hr = 0/1).  Along K a tile is cut into blocks of 512 bytes: 64 K elements
+// for 4-bit codes, 32 for INT8.  Inside a block, lane L = 4*g + tq of a warp
+// owns 16 contiguous bytes: the codes of rows g and g+8 for K offsets
+// {32c + 8tq + 4s + e : c, s in {0,1} (4-bit) or c = 0 (INT8), e = 0..3}.
+// One 16-byte load per lane therefore yields exactly the A-operand fragments
+// of an m16n8k16 tensor-core step (W rows as the 16-row operand), with the K
+// order inside each 16-step permuted consistently for A and B, so that the
+// matching 8 activations of each lane are also contiguous (one 16-byte load).
+//
+//   4-bit word j = 2c + s holds the 8 nibbles of rows {g, g+8} x K offsets
+//   {e = 0..3}.  Two nibble orders:
+//     "magic" (INT4_SYM, INT4_ASYM):  p = 4*(e&1) + 2*(e>>1) + hr, so that
+//        (word >> 4i) & 0x000F000F yields fragment register i as two nibbles
+//        at bit 0 and bit 16;
+//     "table" (CB4, NVFP4):           p = 4*(e>>1) + 2*hr + (e&1), so that the
+//        low/high 16 bits hold registers {0,1} / {2,3} as four nibbles each,
+//        ready for byte-permute table lookups.
+//   INT4_SYM nibbles are stored offset-binary (v + 8); INT8 bytes likewise
+//   (v + 128), word j = 2s + hr, byte e.
+//
+// Scales (INT formats):  bf16 [N/16][K/G][16], entry 2g + hr (so lane g
+//   reads rows g and g+8 as one 32-bit word).
+// Zero-points (ASYM):    u8 [N/16][K/G][8], byte g = z(row g) | z(row g+8) << 4.
+// NVFP4 block scales:    u8 [N/16][K/16][16], entry 2g + hr.
+// CB4 norms, CB4 centroids and the NVFP4 tensor scale keep their canonical
+// layout.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/wq.h"
+
+namespace wq {
+
+enum Fmt { INT4_SYM = 0, INT4_ASYM = 1, INT8_SYM = 2, CB4 = 3, NVFP4 = 4 };
+
+__host__ __device__ inline bool is_int_fmt(int f) { return f == INT4_SYM || f == INT4_ASYM || f == INT8_SYM; }
+__host__ __device__ inline bool is_4bit(int f) { return f != INT8_SYM; }
+// elements of K per 512-byte block
+__host__ __device__ inline int block_k(int f) { return is_4bit(f) ? 64 : 32; }
+
+// Byte offset and bit shift of element (n, k) inside the packed weight.
+__host__ __device__ inline void packed_loc(int f, int64_t n, int64_t k, int64_t K,
+                                           int64_t* byte_off, int* shift) {
+  int64_t tile = n >> 4;
+  int r = (int)(n & 15), g = r & 7, hr = r >> 3;
+  if (is_4bit(f)) {
+    int64_t b = k >> 6;
+    int kk = (int)(k & 63), c = kk >> 5, kc = kk & 31, tq = kc >> 3, e8 = kc & 7, s = e8 >> 2,
+        e = e8 & 3;
+    int lane = 4 * g + tq, j = 2 * c + s;
+    int p = (f == CB4 || f == NVFP4) ? (4 * (e >> 1) + 2 * hr + (e & 1))
+                                     : (4 * (e & 1) + 2 * (e >> 1) + hr);
+    *byte_off = ((tile * (K >> 6) + b) * 32 + lane) * 16 + j * 4 + (p >> 1);
+    *shift = (p & 1) * 4;
+  } else {
+    int64_t b = k >> 5;
+    int kk = (int)(k & 31), tq = kk >> 3, e8 = kk & 7, s = e8 >> 2, e = e8 & 3;
+    int lane = 4 * g + tq, j = 2 * s + hr;
+    *byte_off = ((tile * (K >> 5) + b) * 32 + lane) * 16 + j * 4 + e;
+    *shift = 0;
+  }
+}
+
+// Index (in elements) of the packed group scale / NVFP4 block scale of (n, group).
+__host__ __device__ inline int64_t packed_scale_idx(int64_t n, int64_t grp, int64_t groups) {
+  int r = (int)(n & 15);
+  return ((n >> 4) * groups + grp) * 16 + 2 * (r & 7) + (r >> 3);
+}
+// Byte and shift of the packed ASYM zero-point of (n, group).
+__host__ __device__ inline int64_t packed_zero_byte(int64_t n, int64_t grp, int64_t groups,
+                                                    int* shift) {
+  int r = (int)(n & 15);
+  *shift = (r >> 3) * 4;
+  return ((n >> 4) * groups + grp) * 8 + (r & 7);
+}
+
+// ------------------------------------------------------------ device math
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t h) {
+  return __uint_as_float(((uint32_t)h) << 16);
+}
+
+// E4M3 (fn) code -> fp32, exact for all 256 codes (0x7F/0xFF -> NaN).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
+  uint32_t s = (c >> 7) & 1u, e = (c >> 3) & 15u, m = c & 7u;
+  float v;
+  if (e == 15u && m == 7u) v = __uint_as_float(0x7FC00000u);
+  else if (e == 0u) v = (float)m * 0.001953125f;  // m * 2^-9
+  else v = __uint_as_float(((e + 120u) << 23) | (m << 20));
+  return s ? -v : v;
+}
+
+// ------------------------------------------------------------- launchers
+struct LinearArgs {
+  const void* x;
+  const void* w;
+  const void* scales;
+  const void* aux;
+  const void* bias;
+  void* out;
+  int64_t M, N, K;
+  int fmt, G;
+  cudaStream_t stream;
+};
+
+cudaError_t launch_decode(const LinearArgs& a);
+cudaError_t launch_prefill(const LinearArgs& a);
+int device_sm_count();
+
+cudaError_t launch_pack(int f, int64_t N, int64_t K, int G, const void* codes, const void* scales,
+                        const void* aux, void* pw, void* ps, void* pa, cudaStream_t st);
+cudaError_t launch_unpack(int f, int64_t N, int64_t K, int G, const void* pw, const void* ps,
+                          const void* pa, void* codes, void* scales, void* aux, cudaStream_t st);
+cudaError_t launch_dequant(int f, int64_t N, int64_t K, int G, const void* pw, const void* ps,
+                           const void* pa, float* out, cudaStream_t st);
+cudaError_t launch_quantize(int f, int64_t N, int64_t K, int G, const float* w, void* codes,
+                            void* scales, void* aux, cudaStream_t st);
+
+}  // namespace wq

@@ -1,0 +1,106 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol the header
+declares, sizes buffers, and rejects bad arguments before launching anything."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "wq.h")
+
+import mixed_gemm_b200 as wqm  # noqa: E402
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(wq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_symbols_exported():
+    names = _declared()
+    assert "wq_linear" in names and "wq_pack" in names and len(names) >= 10
+    lib = ctypes.CDLL(wqm.LIB_PATH)
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings():
+    for s in range(6):
+        assert wqm.wq_status_string(s)
+    assert wqm.wq_status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("fmt,G", [("int4_sym", 64), ("int4_asym", 128), ("int8_sym", 256),
+                                   ("cb4", 0), ("nvfp4", 16)])
+def test_sizes(fmt, G):
+    import synth.workloads as W
+    N, K = 4096, 4096
+    wb, sb, ab = wqm.wq_packed_sizes(fmt, N, K, G)
+    assert wb + sb + ab == W.packed_bytes(fmt, N, K, G if G else 16)
+    cb, cs, ca = wqm.wq_canonical_sizes(fmt, N, K, G)
+    assert cb == wb and cs == sb
+    if fmt == "int4_asym":
+        assert ca == 2 * ab
+
+
+BAD_SHAPES = [
+    dict(fmt=7), dict(N=0), dict(K=0), dict(N=24), dict(K=96), dict(G=48), dict(G=512),
+    dict(fmt="nvfp4", G=32), dict(M=-1),
+]
+
+
+@pytest.mark.parametrize("bad", BAD_SHAPES, ids=[str(b) for b in BAD_SHAPES])
+def test_linear_rejects_bad_shapes(bad):
+    a = dict(fmt="int4_sym", M=4, N=256, K=512, G=64)
+    a.update(bad)
+    base = 1 << 20
+    st = wqm._lib.wq_linear(base, base * 2, base * 3, base * 4, None, a["M"], a["N"], a["K"],
+                            wqm._fmt(a["fmt"]), a["G"], base * 5, 0)
+    assert st == wqm.WQ_ERR_INVALID_ARG
+
+
+def test_linear_rejects_null_and_misaligned():
+    base = 1 << 20
+    f = wqm.FORMATS["int4_asym"]
+    # null aux for a format that needs it
+    assert wqm._lib.wq_linear(base, base * 2, base * 3, None, None, 4, 256, 512, f, 64, base * 5,
+                              0) == wqm.WQ_ERR_INVALID_ARG
+    # misaligned x
+    assert wqm._lib.wq_linear(base + 2, base * 2, base * 3, base * 4, None, 4, 256, 512, f, 64,
+                              base * 5, 0) == wqm.WQ_ERR_ALIGNMENT
+    # misaligned output
+    assert wqm._lib.wq_linear(base, base * 2, base * 3, base * 4, None, 4, 256, 512, f, 64,
+                              base * 5 + 8, 0) == wqm.WQ_ERR_ALIGNMENT
+    # output overlapping the activations
+    assert wqm._lib.wq_linear(base, base * 2, base * 3, base * 4, None, 4, 256, 512, f, 64,
+                              base + 256, 0) == wqm.WQ_ERR_INVALID_ARG
+
+
+def test_linear_empty_batch_is_noop():
+    base = 1 << 20
+    st = wqm._lib.wq_linear(base, base * 2, base * 3, None, None, 0, 256, 512,
+                            wqm.FORMATS["int4_sym"], 64, base * 5, 0)
+    assert st == wqm.WQ_OK
+
+
+def test_pack_and_quantize_reject_bad_args():
+    base = 1 << 20
+    f = wqm.FORMATS["cb4"]
+    assert wqm._lib.wq_pack(f, 256, 512, 0, base, base, None, base, base, base, 0) == \
+        wqm.WQ_ERR_INVALID_ARG
+    assert wqm._lib.wq_quantize(wqm.FORMATS["int8_sym"], 256, 500, 64, base, base, base, None, 0) \
+        == wqm.WQ_ERR_INVALID_ARG
+    assert wqm._lib.wq_dequant(f, 256, 512, 0, None, base, base, base, 0) == wqm.WQ_ERR_INVALID_ARG
+
+
+def test_lloyd_max_host_matches_oracle(orc):
+    """Two independent statements of the Lloyd-Max iteration agree in fp32."""
+    c = wqm.wq_lloyd_max_centroids(4)
+    _, c32, _, _ = orc.lloyd_max(16)
+    assert np.max(np.abs(c.view(np.int32) - c32.view(np.int32))) <= 1
+    assert np.all(np.diff(c) > 0)

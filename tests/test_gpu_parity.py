@@ -1,0 +1,156 @@
+"""GPU parity on small and ragged shapes: pack/unpack round trip, exact
+dequant, the GPU quantizer against the oracle's, and the linear against the
+oracle for every format, group size and a spread of batch sizes."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from gpu_cases import (bf16_bits, check_close, dev_bf16, dev_u8, pack_on_gpu, run_linear,
+                       small_case)
+
+pytestmark = pytest.mark.gpu
+
+FMT_G = [("int4_sym", 32), ("int4_sym", 64), ("int4_sym", 128), ("int4_sym", 256),
+         ("int4_asym", 32), ("int4_asym", 128), ("int8_sym", 32), ("int8_sym", 256),
+         ("cb4", 0), ("nvfp4", 16)]
+IDS = [f"{f}-g{g}" for f, g in FMT_G]
+
+
+@pytest.mark.parametrize("fmt,G", FMT_G, ids=IDS)
+def test_pack_unpack_round_trip(wq, orc, fmt, G):
+    N, K = 48, 768 if G == 256 else 320
+    K = K if (G == 0 or K % G == 0) else 768
+    W, (codes, scales, aux) = small_case(orc, fmt, N, K, G, seed=3)
+    pw = pack_on_gpu(wq, fmt, N, K, G, codes, scales, aux)
+    cb, cs, ca = wq.wq_canonical_sizes(fmt, N, K, G)
+    c2 = torch.zeros(cb, dtype=torch.uint8, device="cuda")
+    s2 = torch.zeros(cs, dtype=torch.uint8, device="cuda")
+    a2 = torch.zeros(max(ca, 16), dtype=torch.uint8, device="cuda") if ca else None
+    wq.wq_unpack(fmt, N, K, G, pw.w, pw.scales, pw.aux, c2, s2, a2)
+    torch.cuda.synchronize()
+    assert np.array_equal(c2.cpu().numpy(), codes.view(np.uint8).reshape(-1))
+    assert np.array_equal(s2.cpu().numpy(), scales.view(np.uint8).reshape(-1))
+    if ca:
+        assert np.array_equal(a2[:ca].cpu().numpy(), aux.view(np.uint8).reshape(-1))
+    # the packed weight is a permutation: same multiset of bytes for 8-bit codes
+    if fmt == "int8_sym":
+        got = np.sort(pw.w.cpu().numpy() ^ 0x80)
+        assert np.array_equal(got, np.sort(codes.view(np.uint8).reshape(-1)))
+
+
+@pytest.mark.parametrize("fmt,G", FMT_G, ids=IDS)
+def test_dequant_bit_exact(wq, orc, fmt, G):
+    N, K = 64, 512
+    W, (codes, scales, aux) = small_case(orc, fmt, N, K, G, seed=5)
+    pw = pack_on_gpu(wq, fmt, N, K, G, codes, scales, aux)
+    out = torch.empty((N, K), dtype=torch.float32, device="cuda")
+    wq.wq_dequant(fmt, N, K, G, pw.w, pw.scales, pw.aux, out)
+    torch.cuda.synchronize()
+    ref = orc.dequant(fmt, codes, scales, aux, N, K, G)
+    assert np.array_equal(out.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("fmt,G", FMT_G, ids=IDS)
+def test_gpu_quantizer_matches_oracle(wq, orc, fmt, G):
+    N, K = 96, 1024
+    W = synth.weight(17, N, K, dist="student5" if fmt == "nvfp4" else "normal", sigma=0.02,
+                     outlier_count=100, outlier_mult=20.0)
+    W[7, :] = 0.0
+    W[9, 64:192] = 0.0
+    codes, scales, aux = orc.quantize(fmt, W, G)
+    cb, cs, ca = wq.wq_canonical_sizes(fmt, N, K, G)
+    dc = torch.zeros(cb, dtype=torch.uint8, device="cuda")
+    ds = torch.zeros(cs, dtype=torch.uint8, device="cuda")
+    da = torch.zeros(max(ca, 16), dtype=torch.uint8, device="cuda") if ca else None
+    if fmt == "cb4":
+        da.view(torch.float32)[:16].copy_(torch.from_numpy(aux))
+    wq.wq_quantize(fmt, N, K, G, torch.from_numpy(W).cuda(), dc, ds, da)
+    torch.cuda.synchronize()
+    assert np.array_equal(dc.cpu().numpy(), codes.view(np.uint8).reshape(-1))
+    assert np.array_equal(ds.cpu().numpy(), scales.view(np.uint8).reshape(-1))
+    if ca:
+        assert np.array_equal(da[:ca].cpu().numpy(), aux.view(np.uint8).reshape(-1))
+
+
+MS = [1, 2, 3, 4, 5, 7, 8, 9, 13, 16, 17, 31, 64, 100, 129, 300]
+
+
+@pytest.mark.parametrize("fmt,G", FMT_G, ids=IDS)
+@pytest.mark.parametrize("shape", [(80, 448), (256, 1024)], ids=["ragged80x448", "256x1024"])
+def test_linear_parity(wq, orc, fmt, G, shape):
+    N, K = shape
+    if G and K % G:
+        K = 1024
+    W, (codes, scales, aux) = small_case(orc, fmt, N, K, G, seed=N + K)
+    pw = pack_on_gpu(wq, fmt, N, K, G, codes, scales, aux)
+    dq = orc.dequant(fmt, codes, scales, aux, N, K, G)
+    xa = synth.activations(31, max(MS), K)
+    b = synth.bias(31, N)
+    y_ref, _ = orc.linear(xa, dq, b)
+    for M in MS:
+        for bias in (b, None):
+            y = run_linear(wq, pw, xa[:M], bias, M)
+            ref = y_ref[:M] if bias is not None else orc.linear(xa[:M], dq, None)[0]
+            check_close(y, ref, f"{fmt} g{G} N={N} K={K} M={M} bias={bias is not None}")
+
+
+def _int_case(fmt, N, K, G, rng):
+    import test_oracle_linear as tol
+    return tol._int_case(fmt, N, K, G, rng)
+
+
+@pytest.mark.parametrize("fmt,G", [("int4_sym", 64), ("int4_asym", 32), ("int8_sym", 128),
+                                   ("cb4", 0), ("nvfp4", 16)])
+@pytest.mark.parametrize("M", [1, 5, 16, 40, 200])
+def test_linear_integer_bit_exact(wq, orc, fmt, G, M):
+    """Integer activations and unit scales: every partial sum is exact in
+    fp32, so the GPU result must equal the oracle's bit for bit."""
+    N, K = 96, 256
+    rng = np.random.default_rng(7)
+    codes, scales, aux, wval = _int_case(fmt, N, K, G, rng)
+    if fmt == "cb4":   # keep |centroids| small enough that fp32 sums stay exact
+        aux = ((np.arange(16) - 8) * 1.0).astype(np.float32)
+    pw = pack_on_gpu(wq, fmt, N, K, G, codes, scales, aux)
+    xi = rng.integers(-4, 5, size=(M, K))
+    x = synth.f64_to_bf16_bits(xi.astype(np.float64))
+    dq = orc.dequant(fmt, codes, scales, aux, N, K, G)
+    ref, ref64 = orc.linear(x, dq, None)
+    y = run_linear(wq, pw, x, None, M)
+    assert np.array_equal(y, ref), f"max diff {np.max(np.abs(y.astype(int) - ref.astype(int)))}"
+
+
+def test_linear_empty_and_api(wq, orc):
+    N, K, G = 64, 256, 64
+    W, (codes, scales, aux) = small_case(orc, "int4_sym", N, K, G, seed=1)
+    pw = pack_on_gpu(wq, "int4_sym", N, K, G, codes, scales, aux)
+    y = torch.empty((1, N), dtype=torch.bfloat16, device="cuda")
+    x = torch.zeros((1, K), dtype=torch.bfloat16, device="cuda")
+    wq.wq_linear(x, pw.w, pw.scales, pw.aux, None, 0, N, K, "int4_sym", G, y)
+    # the high-level helper, from host memory, matches the C call
+    xa = synth.activations(2, 3, K)
+    xh = torch.from_numpy(xa.view(np.int16).copy()).view(torch.bfloat16)
+    yh = wq.linear(xh, pw)
+    yd = run_linear(wq, pw, xa, None, 3)
+    assert np.array_equal(bf16_bits(yh), yd)
+    # quantize_and_pack on the GPU gives the same packed bytes as the oracle path
+    pw2 = wq.quantize_and_pack(torch.from_numpy(W).cuda(), "int4_sym", G)
+    assert torch.equal(pw2.w, pw.w) and torch.equal(pw2.scales, pw.scales)
+
+
+def test_linear_respects_stream(wq, orc):
+    N, K, G = 128, 512, 128
+    W, (codes, scales, aux) = small_case(orc, "int4_asym", N, K, G, seed=2)
+    pw = pack_on_gpu(wq, "int4_asym", N, K, G, codes, scales, aux)
+    xa = synth.activations(3, 4, K)
+    ref = run_linear(wq, pw, xa, None, 4)
+    s = torch.cuda.Stream()
+    x = dev_bf16(xa)
+    y = torch.empty((4, N), dtype=torch.bfloat16, device="cuda")
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        wq.wq_linear(x, pw.w, pw.scales, pw.aux, None, 4, N, K, "int4_asym", G, y, s)
+    s.synchronize()
+    assert np.array_equal(bf16_bits(y), ref)
