@@ -160,6 +160,15 @@ int wq_quantize(int format, int64_t N, int64_t K, int group_size, const float* w
  * shape [2**bits]). */
 int wq_lloyd_max_centroids(int bits, float* centroids_out);
 
+/* The kernels' own error word on the current device.  Every wait of the
+ * prefill kernel on a shared-memory barrier has an iteration limit; a wait that
+ * runs out sets a bit here (1 producer, 2 producer drain, 4/8 MMA waits, 16
+ * MMA drain, 32 dequant, 64 epilogue) and the thread block winds down instead
+ * of hanging, leaving the CUDA context usable.  Synchronizes the device (a
+ * symbol copy).  Writes the word to *value, clears it when `clear` is non-zero,
+ * and returns WQ_ERR_DEVICE_CHECK when it was non-zero, WQ_OK otherwise. */
+int wq_device_error(unsigned* value, int clear);
+
 /* Device properties the dispatcher uses (SM count of the current device);
  * exported for the benchmark's launch accounting.  Returns WQ_ERR_CUDA when
  * no device is usable. */

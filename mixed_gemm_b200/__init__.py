@@ -52,6 +52,7 @@ _SIGS = {
     "wq_quantize": ([_int, _i64, _i64, _int, _ptr, _ptr, _ptr, _ptr, _ptr], _int),
     "wq_lloyd_max_centroids": ([_int, ctypes.POINTER(ctypes.c_float)], _int),
     "wq_device_sm_count": ([ctypes.POINTER(ctypes.c_int)], _int),
+    "wq_device_error": ([ctypes.POINTER(ctypes.c_uint), _int], _int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -138,6 +139,15 @@ def wq_lloyd_max_centroids(bits: int = 4):
     _check(_lib.wq_lloyd_max_centroids(bits, out.ctypes.data_as(ctypes.POINTER(ctypes.c_float))),
            "wq_lloyd_max_centroids")
     return out
+
+
+def wq_device_error(clear: bool = True) -> int:
+    """The kernels' error word (0 when every bounded wait completed)."""
+    v = ctypes.c_uint(0)
+    st = _lib.wq_device_error(ctypes.byref(v), 1 if clear else 0)
+    if st not in (WQ_OK, WQ_ERR_DEVICE_CHECK):
+        raise WQError(st, "wq_device_error")
+    return v.value
 
 
 def wq_device_sm_count() -> int:

@@ -216,6 +216,12 @@ int wq_lloyd_max_centroids(int bits, float* out) {
   return WQ_OK;
 }
 
+int wq_device_error(unsigned* value, int clear) {
+  if (!value) return WQ_ERR_INVALID_ARG;
+  if (read_device_error(value, clear != 0) != cudaSuccess) return WQ_ERR_CUDA;
+  return *value ? WQ_ERR_DEVICE_CHECK : WQ_OK;
+}
+
 int wq_device_sm_count(int* n) {
   if (!n) return WQ_ERR_INVALID_ARG;
   int dev = 0;

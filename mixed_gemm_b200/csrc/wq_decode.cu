@@ -25,6 +25,7 @@
 // offline for cheap dequantization).
 #include <cooperative_groups.h>
 
+#include "wq_frag.cuh"
 #include "wq_internal.cuh"
 
 namespace cg = cooperative_groups;
@@ -59,77 +60,12 @@ __device__ __forceinline__ uint4 ld_nc(const void* p) {
   return v;
 }
 
-__device__ __forceinline__ uint32_t word(const uint4& v, int i) {
-  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
-}
-
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                          uint32_t b1) {
   asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
       "{%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t bsub2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-__device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  uint32_t d;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
-  return d;
-}
-__device__ __forceinline__ uint32_t f32_to_bf16_bits(float v) {
-  return pack_bf16x2(v, 0.f) & 0xFFFFu;
-}
-
-// INT4, "magic" nibble order: fragment i = nibbles (i, i+4) as bf16 (128 + n),
-// minus the per-row offset (136 for offset-binary signed codes, 128 + z).
-__device__ __forceinline__ void frag_int4(uint32_t wd, uint32_t off_g, uint32_t off_g8,
-                                          uint32_t (&a)[4]) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    uint32_t t = ((wd >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
-    a[i] = bsub2(t, (i & 1) ? off_g8 : off_g);
-  }
-}
-
-// INT8 offset-binary bytes -> exact integers via the fp32 magic 2^23 + u.
-__device__ __forceinline__ float i8val(uint32_t w, int i) {
-  return __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7440u | i)) - 8388736.0f;
-}
-__device__ __forceinline__ void frag_int8(uint32_t wg, uint32_t wg8, uint32_t (&a)[4]) {
-  a[0] = pack_bf16x2(i8val(wg, 0), i8val(wg, 1));
-  a[1] = pack_bf16x2(i8val(wg8, 0), i8val(wg8, 1));
-  a[2] = pack_bf16x2(i8val(wg, 2), i8val(wg, 3));
-  a[3] = pack_bf16x2(i8val(wg8, 2), i8val(wg8, 3));
-}
-
-// 16-entry bf16 lookup ("table" nibble order): byte tables H (high bytes) and
-// L (low bytes), four entries per register.  `kSymLow` means the low-byte
-// table does not depend on the top index bit (true for E2M1).
-template <bool kSymLow>
-__device__ __forceinline__ void frag_table(uint32_t wd, const uint32_t (&H)[4],
-                                           const uint32_t (&L)[4], uint32_t (&a)[4]) {
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    uint32_t x = h ? (wd >> 16) : wd;
-    uint32_t sel = x & 0x7777u;
-    uint32_t mask = __byte_perm(0u, 0xFFFFFFFFu, (x >> 1) & 0x4444u);
-    uint32_t hb = (__byte_perm(H[0], H[1], sel) & ~mask) | (__byte_perm(H[2], H[3], sel) & mask);
-    uint32_t lb;
-    if (kSymLow) lb = __byte_perm(L[0], L[1], sel);
-    else lb = (__byte_perm(L[0], L[1], sel) & ~mask) | (__byte_perm(L[2], L[3], sel) & mask);
-    a[2 * h] = __byte_perm(lb, hb, 0x5140u);
-    a[2 * h + 1] = __byte_perm(lb, hb, 0x7362u);
-  }
 }
 
 template <int FMT, int NT, int RT, int KW, int UB>

@@ -1,0 +1,80 @@
+// Register-level conversion of packed codes to bf16 tensor-core fragments,
+// shared by the decode kernel (fragments go straight into mma.sync) and the
+// prefill kernel (fragments are scaled and stored to shared memory for
+// tcgen05).  Fragment i of an m16n8k16 A operand holds two consecutive K
+// elements of one row: i = 0 row g / K 0,1;  1 row g+8 / K 0,1;
+// 2 row g / K 2,3;  3 row g+8 / K 2,3  (see the packed layout in
+// wq_internal.cuh).
+#pragma once
+
+#include <stdint.h>
+
+namespace wq {
+
+static __device__ __forceinline__ uint32_t word(const uint4& v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+static __device__ __forceinline__ uint32_t bsub2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+static __device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+static __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+static __device__ __forceinline__ uint32_t f32_to_bf16_bits(float v) {
+  return pack_bf16x2(v, 0.f) & 0xFFFFu;
+}
+
+// INT4, "magic" nibble order: fragment i = nibbles (i, i+4) as bf16 (128 + n),
+// minus the per-row offset (136 for offset-binary signed codes, 128 + z).
+static __device__ __forceinline__ void frag_int4(uint32_t wd, uint32_t off_g, uint32_t off_g8,
+                                          uint32_t (&a)[4]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t t = ((wd >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
+    a[i] = bsub2(t, (i & 1) ? off_g8 : off_g);
+  }
+}
+
+// INT8 offset-binary bytes -> exact integers via the fp32 magic 2^23 + u.
+static __device__ __forceinline__ float i8val(uint32_t w, int i) {
+  return __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7440u | i)) - 8388736.0f;
+}
+static __device__ __forceinline__ void frag_int8(uint32_t wg, uint32_t wg8, uint32_t (&a)[4]) {
+  a[0] = pack_bf16x2(i8val(wg, 0), i8val(wg, 1));
+  a[1] = pack_bf16x2(i8val(wg8, 0), i8val(wg8, 1));
+  a[2] = pack_bf16x2(i8val(wg, 2), i8val(wg, 3));
+  a[3] = pack_bf16x2(i8val(wg8, 2), i8val(wg8, 3));
+}
+
+// 16-entry bf16 lookup ("table" nibble order): byte tables H (high bytes) and
+// L (low bytes), four entries per register.  `kSymLow` means the low-byte
+// table does not depend on the top index bit (true for E2M1).
+template <bool kSymLow>
+static __device__ __forceinline__ void frag_table(uint32_t wd, const uint32_t (&H)[4],
+                                           const uint32_t (&L)[4], uint32_t (&a)[4]) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t x = h ? (wd >> 16) : wd;
+    uint32_t sel = x & 0x7777u;
+    uint32_t mask = __byte_perm(0u, 0xFFFFFFFFu, (x >> 1) & 0x4444u);
+    uint32_t hb = (__byte_perm(H[0], H[1], sel) & ~mask) | (__byte_perm(H[2], H[3], sel) & mask);
+    uint32_t lb;
+    if (kSymLow) lb = __byte_perm(L[0], L[1], sel);
+    else lb = (__byte_perm(L[0], L[1], sel) & ~mask) | (__byte_perm(L[2], L[3], sel) & mask);
+    a[2 * h] = __byte_perm(lb, hb, 0x5140u);
+    a[2 * h + 1] = __byte_perm(lb, hb, 0x7362u);
+  }
+}
+
+
+}  // namespace wq

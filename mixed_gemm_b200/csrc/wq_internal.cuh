@@ -113,6 +113,8 @@ struct LinearArgs {
 cudaError_t launch_decode(const LinearArgs& a);
 cudaError_t launch_prefill(const LinearArgs& a);
 int device_sm_count();
+// The kernels' own error word (bit per failed bounded wait); synchronous read.
+cudaError_t read_device_error(unsigned* value, bool clear);
 
 cudaError_t launch_pack(int f, int64_t N, int64_t K, int G, const void* codes, const void* scales,
                         const void* aux, void* pw, void* ps, void* pa, cudaStream_t st);

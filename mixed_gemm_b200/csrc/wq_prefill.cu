@@ -1,19 +1,490 @@
-// Prefill path (M > 16).  Placeholder that runs the decode kernel over
-// 16-token slices of X; replaced by the tcgen05 kernel.
+// Prefill path (M > 16): tcgen05 tensor cores, weights dequantized in shared
+// memory, accumulators in tensor memory.
+//
+// The product is computed transposed, D[w_row, token] = W[w_row, :] . X[token, :],
+// so that the dequantized weight tile is the 128-row A operand and the tokens
+// are the N side of the MMA (N = 32..256, chosen from M).  Per 64-wide K step:
+//   warp 0 (one lane)  TMA-loads the X tile (bf16, 128-byte swizzle, zero fill
+//                      past M) and the packed weight tile of 8 row tiles into
+//                      a ring stage and arms the stage's mbarrier;
+//   warps 2..5         convert the packed tile to bf16 in registers (the same
+//                      fragment decoders as the decode path, then the group
+//                      scale or E4M3 block scale is multiplied in, so a tile
+//                      value is the bf16 rounding of the exact dequantized
+//                      value; CB4 leaves the row norm for the epilogue) and
+//                      store it in the canonical 128-byte-swizzled K-major
+//                      layout the MMA descriptors expect;
+//   warp 1 (one lane)  issues four tcgen05.mma.kind::f16 (K = 16 each) into
+//                      the fp32 accumulator in tensor memory and commits the
+//                      stage back to the producer.
+// After the last K step warps 2..5 read the accumulator with tcgen05.ld,
+// apply the per-row fold (CB4 norm, NVFP4 tensor scale) and the bias, round
+// to bf16 and store Y.  Every mbarrier wait has an iteration limit; a wait
+// that runs out records an error word and the CTA winds down.
+//
+// Sources: Petit README "Techniques and performance" (compute-bound at larger
+// batch; offline-shuffled weights make GPU dequantization cheap); OrbitQuant
+// card "Benchmark" (larger batches are GEMM-bound, the packed path decodes
+// weights on the fly instead of materializing a dense copy).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "wq_frag.cuh"
 #include "wq_internal.cuh"
 
 namespace wq {
 
-cudaError_t launch_prefill(const LinearArgs& a) {
-  for (int64_t m0 = 0; m0 < a.M; m0 += 16) {
-    LinearArgs s = a;
-    s.M = (a.M - m0) < 16 ? (a.M - m0) : 16;
-    s.x = (const uint16_t*)a.x + m0 * a.K;
-    s.out = (uint16_t*)a.out + m0 * a.N;
-    cudaError_t e = launch_decode(s);
-    if (e != cudaSuccess) return e;
+__device__ unsigned int g_wq_device_error;
+
+namespace {
+
+constexpr int kThreads = 192;  // 6 warps
+constexpr uint32_t kWaitLimit = 1u << 22;
+
+struct PrefillParams {
+  const void* scales;
+  const void* aux;
+  const uint16_t* bias;
+  uint16_t* out;
+  int M, N, K, G;
+  int BN, stages;
+  uint32_t tmem_cols;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: false when the CTA is aborting or the limit ran out (which
+// raises the abort flag and the device error word).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+                                          unsigned code) {
+  for (uint32_t i = 0; i < kWaitLimit; ++i) {
+    if (mbar_try(bar, parity)) return true;
+    if ((i & 255u) == 255u && *abort) return false;
   }
-  return cudaSuccess;
+  *abort = 1;
+  atomicOr(&g_wq_device_error, code);
+  return false;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(map), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
+// UMMA shared-memory descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (stride byte offset), descriptor version 1.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;              // leading byte offset (unused for swizzled K-major)
+  d |= (uint64_t)(1024u >> 4) << 32;    // stride byte offset
+  d |= (uint64_t)1u << 46;              // version
+  d |= (uint64_t)2u << 61;              // SWIZZLE_128B
+  return d;
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// byte offset of 16-byte chunk j (K elements 8j..8j+7) of row R in a
+// 128-row x 64-K bf16 tile, 128-byte swizzle, 8-row groups of 1024 bytes
+__device__ __forceinline__ uint32_t swz(int R, int j) {
+  return (uint32_t)((R >> 3) * 1024 + (R & 7) * 128 + ((j ^ (R & 7)) << 4));
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                   const PrefillParams p) {
+  constexpr bool kInt = FMT == INT4_SYM || FMT == INT4_ASYM || FMT == INT8_SYM;
+  constexpr uint32_t kWpk = FMT == INT8_SYM ? 8192u : 4096u;  // packed bytes per stage
+  constexpr uint32_t kAtile = 16384u;                          // 128 x 64 bf16
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const int BN = p.BN, S = p.stages;
+  const uint32_t xbytes = (uint32_t)BN * 128u;
+  const uint32_t stage_bytes = xbytes + kAtile + kWpk;
+  uint64_t* bars = (uint64_t*)(smem + S * stage_bytes);
+  uint32_t* tmem_slot = (uint32_t*)(bars + 3 * S + 1);
+  volatile int* abort = (volatile int*)(tmem_slot + 1);
+  auto full_bar = [&](int s) { return smem_u32(bars + s); };
+  auto dq_bar = [&](int s) { return smem_u32(bars + S + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + 2 * S + s); };
+  const uint32_t acc_bar = smem_u32(bars + 3 * S);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile0 = blockIdx.x * 8;  // first 16-row tile of the CTA's 128 rows
+  const int m0 = blockIdx.y * BN;
+  const int KT = p.K / 64;
+  const int ntiles = p.N / 16;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(dq_bar(s), 4);
+      mbar_init(empty_bar(s), 1);
+    }
+    mbar_init(acc_bar, 1);
+    *abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(p.tmem_cols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int kt = 0; kt < KT; ++kt) {
+        const int s = kt % S;
+        const uint32_t ph = (uint32_t)(kt / S) & 1u;
+        if (kt >= S && !mbar_wait(empty_bar(s), ph ^ 1u, abort, 1u)) break;
+        uint8_t* st = smem + s * stage_bytes;
+        mbar_expect_tx(full_bar(s), xbytes + kWpk);
+        tma_load_2d(smem_u32(st), &tmX, kt * 64, m0, full_bar(s));
+        tma_load_2d(smem_u32(st + xbytes + kAtile), &tmW, kt * (int)(kWpk / 32u), tile0,
+                    full_bar(s));
+        ++issued;
+      }
+      // before teardown, make sure no copy into this CTA's memory is in flight
+      for (int kt = issued - S < 0 ? 0 : issued - S; kt < issued; ++kt)
+        mbar_wait(full_bar(kt % S), (uint32_t)(kt / S) & 1u, abort, 2u);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                             ((128u >> 4) << 24);
+      bool ok = true;
+      for (int kt = 0; kt < KT && ok; ++kt) {
+        const int s = kt % S;
+        const uint32_t ph = (uint32_t)(kt / S) & 1u;
+        ok = mbar_wait(full_bar(s), ph, abort, 4u) && mbar_wait(dq_bar(s), ph, abort, 8u);
+        if (!ok) break;
+        tc_fence_after();
+        uint8_t* st = smem + s * stage_bytes;
+        const uint32_t xa = smem_u32(st), aa = smem_u32(st + xbytes);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_f16(tmem, umma_desc_sw128(aa + kk * 32), umma_desc_sw128(xa + kk * 32), idesc,
+                   (kt | kk) != 0);
+        umma_commit(empty_bar(s));
+      }
+      umma_commit(acc_bar);  // also covers the abort path: wait for own MMAs
+      if (!ok) mbar_wait(acc_bar, 0u, abort, 16u);
+    }
+  } else {
+    // ------------------------------------------------------------ dequant
+    const int dw = warp - 2;  // 0..3
+    const int g = lane >> 2, tq = lane & 3;
+    const int64_t groups = kInt ? p.K / p.G : 0;
+    uint32_t H[4] = {0, 0, 0, 0}, L[4] = {0, 0, 0, 0};
+    if constexpr (FMT == NVFP4) {
+      H[0] = 0x3F3F3F00u; H[1] = 0x40404040u; H[2] = 0xBFBFBF80u; H[3] = 0xC0C0C0C0u;
+      L[0] = 0xC0800000u; L[1] = 0xC0804000u; L[2] = L[0]; L[3] = L[1];
+    }
+    if constexpr (FMT == CB4) {
+      const float* cen = (const float*)p.aux;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        uint32_t b = f32_to_bf16_bits(__ldg(cen + j));
+        H[j >> 2] |= (b >> 8) << (8 * (j & 3));
+        L[j >> 2] |= (b & 0xFFu) << (8 * (j & 3));
+      }
+    }
+    bool ok = true;
+    for (int kt = 0; kt < KT; ++kt) {
+      const int s = kt % S;
+      const uint32_t ph = (uint32_t)(kt / S) & 1u;
+      if (!mbar_wait(full_bar(s), ph, abort, 32u)) { ok = false; break; }
+      uint8_t* st = smem + s * stage_bytes;
+      const uint32_t abase = smem_u32(st + xbytes);
+      const uint8_t* wpk = st + xbytes + kAtile;
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        const int rt = 2 * dw + rr;
+        const int64_t tile = tile0 + rt;
+        const bool valid = tile < ntiles;
+        const int Rg = rt * 16 + g, Rg8 = Rg + 8;
+        if constexpr (FMT == INT8_SYM) {
+#pragma unroll
+          for (int blk = 0; blk < 2; ++blk) {
+            const uint4 ch = *(const uint4*)(wpk + rt * 1024 + blk * 512 + lane * 16);
+            uint32_t sc_g = 0, sc_g8 = 0;
+            if (valid) {
+              const int64_t grp = ((int64_t)kt * 64 + 32 * blk) / p.G;
+              const uint32_t sw = __ldg((const uint32_t*)p.scales + (tile * groups + grp) * 8 + g);
+              sc_g = (sw & 0xFFFFu) * 0x00010001u;
+              sc_g8 = (sw >> 16) * 0x00010001u;
+            }
+            uint32_t a[4], b[4];
+            frag_int8(ch.x, ch.y, a);
+            frag_int8(ch.z, ch.w, b);
+            const int j = 4 * blk + tq;
+            st_shared_v4(abase + swz(Rg, j), bmul2(a[0], sc_g), bmul2(a[2], sc_g),
+                         bmul2(b[0], sc_g), bmul2(b[2], sc_g));
+            st_shared_v4(abase + swz(Rg8, j), bmul2(a[1], sc_g8), bmul2(a[3], sc_g8),
+                         bmul2(b[1], sc_g8), bmul2(b[3], sc_g8));
+          }
+        } else {
+          const uint4 ch = *(const uint4*)(wpk + rt * 512 + lane * 16);
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const uint32_t w0 = c ? ch.z : ch.x, w1 = c ? ch.w : ch.y;
+            uint32_t a[4], b[4];
+            uint32_t sc_g = 0, sc_g8 = 0;
+            if constexpr (kInt) {
+              uint32_t off_g = 0x43084308u, off_g8 = 0x43084308u;
+              if (valid) {
+                const int64_t grp = ((int64_t)kt * 64 + 32 * c) / p.G;
+                const uint32_t sw =
+                    __ldg((const uint32_t*)p.scales + (tile * groups + grp) * 8 + g);
+                sc_g = (sw & 0xFFFFu) * 0x00010001u;
+                sc_g8 = (sw >> 16) * 0x00010001u;
+                if constexpr (FMT == INT4_ASYM) {
+                  const uint32_t zb =
+                      __ldg((const uint8_t*)p.aux + (tile * groups + grp) * 8 + g);
+                  off_g = (0x4300u + (zb & 15u)) * 0x00010001u;
+                  off_g8 = (0x4300u + (zb >> 4)) * 0x00010001u;
+                }
+              }
+              frag_int4(w0, off_g, off_g8, a);
+              frag_int4(w1, off_g, off_g8, b);
+            } else {
+              frag_table<FMT == NVFP4>(w0, H, L, a);
+              frag_table<FMT == NVFP4>(w1, H, L, b);
+              if constexpr (FMT == NVFP4) {
+                if (valid) {
+                  const int64_t b16 = ((int64_t)kt * 64 + 32 * c + 8 * tq) >> 4;
+                  const uint32_t sb =
+                      __ldg((const uint16_t*)p.scales + (tile * (p.K >> 4) + b16) * 8 + g);
+                  sc_g = f32_to_bf16_bits(e4m3_to_f32(sb & 0xFFu)) * 0x00010001u;
+                  sc_g8 = f32_to_bf16_bits(e4m3_to_f32(sb >> 8)) * 0x00010001u;
+                }
+              } else {
+                sc_g = valid ? 0x3F803F80u : 0u;  // CB4: norm applied in the epilogue
+                sc_g8 = sc_g;
+              }
+            }
+            const int j = 4 * c + tq;
+            st_shared_v4(abase + swz(Rg, j), bmul2(a[0], sc_g), bmul2(a[2], sc_g),
+                         bmul2(b[0], sc_g), bmul2(b[2], sc_g));
+            st_shared_v4(abase + swz(Rg8, j), bmul2(a[1], sc_g8), bmul2(a[3], sc_g8),
+                         bmul2(b[1], sc_g8), bmul2(b[3], sc_g8));
+          }
+        }
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dq_bar(s));
+    }
+
+    // ------------------------------------------------------------ epilogue
+    const bool have_acc = ok && mbar_wait(acc_bar, 0u, abort, 64u);
+    __syncwarp();
+    tc_fence_after();
+    const int q = warp & 3;  // tensor-memory lane quarter this warp may read
+    const int row = q * 32 + lane;
+    const int64_t n = (int64_t)tile0 * 16 + row;
+    const bool nvalid = n < p.N;
+    float fold = 1.f, bval = 0.f;
+    if (nvalid) {
+      if constexpr (FMT == CB4) fold = bf16_bits_to_f32(__ldg((const uint16_t*)p.scales + n));
+      if constexpr (FMT == NVFP4) fold = __ldg((const float*)p.aux);
+      if (p.bias) bval = bf16_bits_to_f32(__ldg(p.bias + n));
+    }
+    if (__all_sync(0xffffffffu, have_acc ? 1 : 0)) {
+      for (int c0 = 0; c0 < BN; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int m = m0 + c0 + j;
+          if (nvalid && m < p.M) {
+            const float y = __uint_as_float(v[j]) * fold + bval;
+            p.out[(int64_t)m * p.N + n] = (uint16_t)f32_to_bf16_bits(y);
+          }
+        }
+      }
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(p.tmem_cols)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (PFN_cuTensorMapEncodeTiled_v12000)f;
+  });
+  return fn;
+}
+
+template <int FMT>
+cudaError_t launch_fmt(const LinearArgs& a, int BN) {
+  constexpr uint32_t kWpk = FMT == INT8_SYM ? 8192u : 4096u;
+  auto fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  CUtensorMap tmX, tmW;
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)a.K, (cuuint64_t)a.M};
+    cuuint64_t strides[1] = {(cuuint64_t)a.K * 2};
+    cuuint32_t box[2] = {64u, (cuuint32_t)BN};
+    cuuint32_t es[2] = {1u, 1u};
+    if (fn(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.x), dims, strides, box,
+           es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t row_bytes = (uint64_t)a.K * (FMT == INT8_SYM ? 16 : 8);  // bytes per row tile
+    cuuint64_t dims[2] = {(cuuint64_t)(row_bytes / 4), (cuuint64_t)(a.N / 16)};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    cuuint32_t box[2] = {kWpk / 32u, 8u};
+    cuuint32_t es[2] = {1u, 1u};
+    if (fn(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(a.w), dims, strides, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  const uint32_t stage_bytes = (uint32_t)BN * 128u + 16384u + kWpk;
+  int S = (int)((200u * 1024u) / stage_bytes);
+  if (S > 6) S = 6;
+  if (S < 2) S = 2;
+  const size_t smem = (size_t)S * stage_bytes + 1024 + 8 * (3 * S + 1) + 16;
+  static std::once_flag attr_once;
+  cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [&] {
+    attr_err = cudaFuncSetAttribute(prefill_kernel<FMT>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  PrefillParams p;
+  p.scales = a.scales;
+  p.aux = a.aux;
+  p.bias = (const uint16_t*)a.bias;
+  p.out = (uint16_t*)a.out;
+  p.M = (int)a.M;
+  p.N = (int)a.N;
+  p.K = (int)a.K;
+  p.G = a.G;
+  p.BN = BN;
+  p.stages = S;
+  p.tmem_cols = BN <= 32 ? 32u : (uint32_t)BN;
+  dim3 grid((unsigned)((a.N + 127) / 128), (unsigned)((a.M + BN - 1) / BN));
+  prefill_kernel<FMT><<<grid, kThreads, smem, a.stream>>>(tmX, tmW, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(const LinearArgs& a) {
+  const int BN = a.M <= 32 ? 32 : a.M <= 64 ? 64 : a.M <= 128 ? 128 : 256;
+  switch (a.fmt) {
+    case INT4_SYM: return launch_fmt<INT4_SYM>(a, BN);
+    case INT4_ASYM: return launch_fmt<INT4_ASYM>(a, BN);
+    case INT8_SYM: return launch_fmt<INT8_SYM>(a, BN);
+    case CB4: return launch_fmt<CB4>(a, BN);
+    case NVFP4: return launch_fmt<NVFP4>(a, BN);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t read_device_error(unsigned* value, bool clear) {
+  cudaError_t e = cudaMemcpyFromSymbol(value, g_wq_device_error, sizeof(unsigned));
+  if (e != cudaSuccess || !clear) return e;
+  unsigned z = 0;
+  return cudaMemcpyToSymbol(g_wq_device_error, &z, sizeof(unsigned));
 }
 
 }  // namespace wq
