@@ -3,29 +3,34 @@
 //
 // The product is computed transposed, D[w_row, token] = W[w_row, :] . X[token, :],
 // so that the dequantized weight tile is the 128-row A operand and the tokens
-// are the N side of the MMA (N = 32..256, chosen from M).  Per 64-wide K step:
-//   warp 0 (one lane)  TMA-loads the X tile (bf16, 128-byte swizzle, zero fill
-//                      past M) and the packed weight tile of 8 row tiles into
-//                      a ring stage and arms the stage's mbarrier;
-//   warps 2..5         convert the packed tile to bf16 in registers (the same
-//                      fragment decoders as the decode path, then the group
-//                      scale or E4M3 block scale is multiplied in, so a tile
-//                      value is the bf16 rounding of the exact dequantized
-//                      value; CB4 leaves the row norm for the epilogue) and
-//                      store it in the canonical 128-byte-swizzled K-major
-//                      layout the MMA descriptors expect;
-//   warp 1 (one lane)  issues four tcgen05.mma.kind::f16 (K = 16 each) into
-//                      the fp32 accumulator in tensor memory and commits the
-//                      stage back to the producer.
-// After the last K step warps 2..5 read the accumulator with tcgen05.ld,
-// apply the per-row fold (CB4 norm, NVFP4 tensor scale) and the bias, round
-// to bf16 and store Y.  Every mbarrier wait has an iteration limit; a wait
-// that runs out records an error word and the CTA winds down.
+// are the N side of the MMA (N = 32..256, chosen from M).  Four warpgroups:
+//   warp 0 (one lane)   TMA-loads, per 64-wide K step, the X tile (bf16,
+//                       128-byte swizzle, zero fill past M) and the packed
+//                       tile of 8 row tiles into a ring stage;
+//   warp 1 (one lane)   issues four tcgen05.mma.kind::f16 (K = 16 each) per
+//                       stage and commits the stage back to the producer;
+//   warps 4..7          convert packed codes to bf16 in registers (the decode
+//                       path's fragment decoders) and store them in the
+//                       canonical 128-byte-swizzled K-major layout;
+//   warps 8..15         fold and epilogue.
+// INT formats with groups of 64 or more keep the tile values exact: the tile
+// holds the integer code (or code minus zero-point), each group of K is
+// accumulated into its own tensor-memory buffer (two buffers alternate), and
+// the fold warps add group_scale[row] * partial into fp32 registers -- the
+// same arithmetic as the decode path, so no bf16 rounding of q*s ever enters
+// the sum.  NVFP4 tiles hold e2m1 * e4m3 (exact in bf16); CB4 tiles hold the
+// bf16 centroid; INT groups of 32 hold the bf16 rounding of q*s.  The
+// epilogue applies the CB4 row norm / NVFP4 tensor scale and the bias, rounds
+// to bf16 and stores Y.  Registers are rebalanced per warpgroup with
+// setmaxnreg (56 / 104 / 168 / 168 of the 128 per thread launched).  Every
+// mbarrier wait has an iteration limit; a wait that runs out records an error
+// word and the CTA winds down.
 //
 // Sources: Petit README "Techniques and performance" (compute-bound at larger
 // batch; offline-shuffled weights make GPU dequantization cheap); OrbitQuant
 // card "Benchmark" (larger batches are GEMM-bound, the packed path decodes
-// weights on the fly instead of materializing a dense copy).
+// weights on the fly instead of materializing a dense copy); auto-round-lib
+// README section 1 (per-group scales along K).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -40,7 +45,7 @@ __device__ unsigned int g_wq_device_error;
 
 namespace {
 
-constexpr int kThreads = 192;  // 6 warps
+constexpr int kThreads = 512;  // 4 warpgroups: TMA+MMA, dequant, 2x fold/epilogue
 constexpr uint32_t kWaitLimit = 1u << 22;
 
 struct PrefillParams {
@@ -158,32 +163,39 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
-template <int FMT>
+template <int FMT, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                    const PrefillParams p) {
   constexpr bool kInt = FMT == INT4_SYM || FMT == INT4_ASYM || FMT == INT8_SYM;
   constexpr uint32_t kWpk = FMT == INT8_SYM ? 8192u : 4096u;  // packed bytes per stage
   constexpr uint32_t kAtile = 16384u;                          // 128 x 64 bf16
+  constexpr uint32_t kXbytes = (uint32_t)BN * 128u;
+  constexpr uint32_t kStage = kXbytes + kAtile + kWpk;
+  constexpr int kHalf = BN / 2;  // accumulator columns per fold thread
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  const int BN = p.BN, S = p.stages;
-  const uint32_t xbytes = (uint32_t)BN * 128u;
-  const uint32_t stage_bytes = xbytes + kAtile + kWpk;
-  uint64_t* bars = (uint64_t*)(smem + S * stage_bytes);
-  uint32_t* tmem_slot = (uint32_t*)(bars + 3 * S + 1);
+  const int S = p.stages;
+  uint64_t* bars = (uint64_t*)(smem + S * kStage);
+  uint32_t* tmem_slot = (uint32_t*)(bars + 3 * S + 5);
   volatile int* abort = (volatile int*)(tmem_slot + 1);
   auto full_bar = [&](int s) { return smem_u32(bars + s); };
   auto dq_bar = [&](int s) { return smem_u32(bars + S + s); };
   auto empty_bar = [&](int s) { return smem_u32(bars + 2 * S + s); };
-  const uint32_t acc_bar = smem_u32(bars + 3 * S);
+  auto gfull_bar = [&](int b) { return smem_u32(bars + 3 * S + b); };
+  auto gempty_bar = [&](int b) { return smem_u32(bars + 3 * S + 2 + b); };
+  const uint32_t drain_bar = smem_u32(bars + 3 * S + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile0 = blockIdx.x * 8;  // first 16-row tile of the CTA's 128 rows
   const int m0 = blockIdx.y * BN;
   const int KT = p.K / 64;
   const int ntiles = p.N / 16;
+  // group-scale fold: exact integer tiles, one accumulator per group
+  const bool fold = kInt && p.G >= 64;
+  const int SPG = fold ? p.G / 64 : KT;  // K stages per accumulation group
+  const int NG = KT / SPG;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -191,7 +203,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(dq_bar(s), 4);
       mbar_init(empty_bar(s), 1);
     }
-    mbar_init(acc_bar, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(gfull_bar(b), 1);
+      mbar_init(gempty_bar(b), 8);
+    }
+    mbar_init(drain_bar, 1);
     *abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -207,51 +223,64 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 56;\n" ::: "memory");
+    if (warp == 0 && lane == 0) {
+      // ---------------------------------------------------------- producer
       int issued = 0;
       for (int kt = 0; kt < KT; ++kt) {
         const int s = kt % S;
         const uint32_t ph = (uint32_t)(kt / S) & 1u;
         if (kt >= S && !mbar_wait(empty_bar(s), ph ^ 1u, abort, 1u)) break;
-        uint8_t* st = smem + s * stage_bytes;
-        mbar_expect_tx(full_bar(s), xbytes + kWpk);
+        uint8_t* st = smem + s * kStage;
+        mbar_expect_tx(full_bar(s), kXbytes + kWpk);
         tma_load_2d(smem_u32(st), &tmX, kt * 64, m0, full_bar(s));
-        tma_load_2d(smem_u32(st + xbytes + kAtile), &tmW, kt * (int)(kWpk / 32u), tile0,
+        tma_load_2d(smem_u32(st + kXbytes + kAtile), &tmW, kt * (int)(kWpk / 32u), tile0,
                     full_bar(s));
         ++issued;
       }
       // before teardown, make sure no copy into this CTA's memory is in flight
       for (int kt = issued - S < 0 ? 0 : issued - S; kt < issued; ++kt)
         mbar_wait(full_bar(kt % S), (uint32_t)(kt / S) & 1u, abort, 2u);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    } else if (warp == 1 && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
       const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                              ((128u >> 4) << 24);
       bool ok = true;
-      for (int kt = 0; kt < KT && ok; ++kt) {
-        const int s = kt % S;
-        const uint32_t ph = (uint32_t)(kt / S) & 1u;
-        ok = mbar_wait(full_bar(s), ph, abort, 4u) && mbar_wait(dq_bar(s), ph, abort, 8u);
-        if (!ok) break;
+      int kt = 0;
+      for (int g = 0; g < NG && ok; ++g) {
+        const int gb = g & 1;
+        if (g >= 2 && !mbar_wait(gempty_bar(gb), (uint32_t)((g >> 1) - 1) & 1u, abort, 4u)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        uint8_t* st = smem + s * stage_bytes;
-        const uint32_t xa = smem_u32(st), aa = smem_u32(st + xbytes);
+        const uint32_t d = tmem + (uint32_t)(gb * BN);
+        for (int sg = 0; sg < SPG; ++sg, ++kt) {
+          const int s = kt % S;
+          const uint32_t ph = (uint32_t)(kt / S) & 1u;
+          ok = mbar_wait(full_bar(s), ph, abort, 4u) && mbar_wait(dq_bar(s), ph, abort, 8u);
+          if (!ok) break;
+          tc_fence_after();
+          uint8_t* st = smem + s * kStage;
+          const uint32_t xa = smem_u32(st), aa = smem_u32(st + kXbytes);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_f16(tmem, umma_desc_sw128(aa + kk * 32), umma_desc_sw128(xa + kk * 32), idesc,
-                   (kt | kk) != 0);
-        umma_commit(empty_bar(s));
+          for (int kk = 0; kk < 4; ++kk)
+            umma_f16(d, umma_desc_sw128(aa + kk * 32), umma_desc_sw128(xa + kk * 32), idesc,
+                     (sg | kk) != 0);
+          umma_commit(empty_bar(s));
+        }
+        umma_commit(gfull_bar(gb));
       }
-      umma_commit(acc_bar);  // also covers the abort path: wait for own MMAs
-      if (!ok) mbar_wait(acc_bar, 0u, abort, 16u);
+      if (!ok) {  // wait for this thread's own MMAs before the memory goes away
+        umma_commit(drain_bar);
+        mbar_wait(drain_bar, 0u, abort, 16u);
+      }
     }
-  } else {
+  } else if (warp < 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 104;\n" ::: "memory");
     // ------------------------------------------------------------ dequant
-    const int dw = warp - 2;  // 0..3
+    const int dw = warp - 4;  // 0..3
     const int g = lane >> 2, tq = lane & 3;
     const int64_t groups = kInt ? p.K / p.G : 0;
     uint32_t H[4] = {0, 0, 0, 0}, L[4] = {0, 0, 0, 0};
@@ -268,14 +297,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         L[j >> 2] |= (b & 0xFFu) << (8 * (j & 3));
       }
     }
-    bool ok = true;
     for (int kt = 0; kt < KT; ++kt) {
       const int s = kt % S;
       const uint32_t ph = (uint32_t)(kt / S) & 1u;
-      if (!mbar_wait(full_bar(s), ph, abort, 32u)) { ok = false; break; }
-      uint8_t* st = smem + s * stage_bytes;
-      const uint32_t abase = smem_u32(st + xbytes);
-      const uint8_t* wpk = st + xbytes + kAtile;
+      if (!mbar_wait(full_bar(s), ph, abort, 32u)) break;
+      uint8_t* st = smem + s * kStage;
+      const uint32_t abase = smem_u32(st + kXbytes);
+      const uint8_t* wpk = st + kXbytes + kAtile;
 #pragma unroll
       for (int rr = 0; rr < 2; ++rr) {
         const int rt = 2 * dw + rr;
@@ -286,8 +314,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int blk = 0; blk < 2; ++blk) {
             const uint4 ch = *(const uint4*)(wpk + rt * 1024 + blk * 512 + lane * 16);
-            uint32_t sc_g = 0, sc_g8 = 0;
-            if (valid) {
+            // exact codes (fold) or codes times the group scale (group of 32)
+            uint32_t sc_g = valid ? 0x3F803F80u : 0u, sc_g8 = sc_g;
+            if (!fold && valid) {
               const int64_t grp = ((int64_t)kt * 64 + 32 * blk) / p.G;
               const uint32_t sw = __ldg((const uint32_t*)p.scales + (tile * groups + grp) * 8 + g);
               sc_g = (sw & 0xFFFFu) * 0x00010001u;
@@ -308,15 +337,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 2; ++c) {
             const uint32_t w0 = c ? ch.z : ch.x, w1 = c ? ch.w : ch.y;
             uint32_t a[4], b[4];
-            uint32_t sc_g = 0, sc_g8 = 0;
+            uint32_t sc_g = valid ? 0x3F803F80u : 0u, sc_g8 = sc_g;
             if constexpr (kInt) {
               uint32_t off_g = 0x43084308u, off_g8 = 0x43084308u;
               if (valid) {
                 const int64_t grp = ((int64_t)kt * 64 + 32 * c) / p.G;
-                const uint32_t sw =
-                    __ldg((const uint32_t*)p.scales + (tile * groups + grp) * 8 + g);
-                sc_g = (sw & 0xFFFFu) * 0x00010001u;
-                sc_g8 = (sw >> 16) * 0x00010001u;
+                if (!fold) {
+                  const uint32_t sw =
+                      __ldg((const uint32_t*)p.scales + (tile * groups + grp) * 8 + g);
+                  sc_g = (sw & 0xFFFFu) * 0x00010001u;
+                  sc_g8 = (sw >> 16) * 0x00010001u;
+                }
                 if constexpr (FMT == INT4_ASYM) {
                   const uint32_t zb =
                       __ldg((const uint8_t*)p.aux + (tile * groups + grp) * 8 + g);
@@ -337,9 +368,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                   sc_g = f32_to_bf16_bits(e4m3_to_f32(sb & 0xFFu)) * 0x00010001u;
                   sc_g8 = f32_to_bf16_bits(e4m3_to_f32(sb >> 8)) * 0x00010001u;
                 }
-              } else {
-                sc_g = valid ? 0x3F803F80u : 0u;  // CB4: norm applied in the epilogue
-                sc_g8 = sc_g;
               }
             }
             const int j = 4 * c + tq;
@@ -354,36 +382,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(dq_bar(s));
     }
-
-    // ------------------------------------------------------------ epilogue
-    const bool have_acc = ok && mbar_wait(acc_bar, 0u, abort, 64u);
-    __syncwarp();
-    tc_fence_after();
-    const int q = warp & 3;  // tensor-memory lane quarter this warp may read
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 168;\n" ::: "memory");
+    // ------------------------------------------------------------ fold + epilogue
+    const int q = warp & 3;            // tensor-memory lane quarter this warp may read
+    const int hcol = ((warp - 8) >> 2) * kHalf;
     const int row = q * 32 + lane;
     const int64_t n = (int64_t)tile0 * 16 + row;
     const bool nvalid = n < p.N;
-    float fold = 1.f, bval = 0.f;
-    if (nvalid) {
-      if constexpr (FMT == CB4) fold = bf16_bits_to_f32(__ldg((const uint16_t*)p.scales + n));
-      if constexpr (FMT == NVFP4) fold = __ldg((const float*)p.aux);
-      if (p.bias) bval = bf16_bits_to_f32(__ldg(p.bias + n));
-    }
-    if (__all_sync(0xffffffffu, have_acc ? 1 : 0)) {
-      for (int c0 = 0; c0 < BN; c0 += 16) {
-        uint32_t v[16];
-        tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
+    const int64_t groups = kInt ? p.K / p.G : 0;
+    float acc[kHalf];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int m = m0 + c0 + j;
-          if (nvalid && m < p.M) {
-            const float y = __uint_as_float(v[j]) * fold + bval;
-            p.out[(int64_t)m * p.N + n] = (uint16_t)f32_to_bf16_bits(y);
-          }
-        }
+    for (int j = 0; j < kHalf; ++j) acc[j] = 0.f;
+    bool ok = true;
+    for (int g = 0; g < NG; ++g) {
+      const int gb = g & 1;
+      ok = mbar_wait(gfull_bar(gb), (uint32_t)(g >> 1) & 1u, abort, 64u);
+      if (!__all_sync(0xffffffffu, ok ? 1 : 0)) { ok = false; break; }
+      tc_fence_after();
+      float sc = 1.f;
+      if (fold && nvalid) {
+        const int r16 = (int)(n & 15);
+        sc = bf16_bits_to_f32(__ldg((const uint16_t*)p.scales +
+                                    ((n >> 4) * groups + g) * 16 + 2 * (r16 & 7) + (r16 >> 3)));
+      }
+      const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(gb * BN + hcol);
+#pragma unroll
+      for (int c = 0; c < kHalf; c += 16) {
+        uint32_t v[16];
+        tmem_ld16(base + (uint32_t)c, v);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) acc[c + j] = fmaf(sc, __uint_as_float(v[j]), acc[c + j]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(gempty_bar(gb));
+    }
+    if (ok && nvalid) {
+      float post = 1.f, bval = 0.f;
+      if constexpr (FMT == CB4) post = bf16_bits_to_f32(__ldg((const uint16_t*)p.scales + n));
+      if constexpr (FMT == NVFP4) post = __ldg((const float*)p.aux);
+      if (p.bias) bval = bf16_bits_to_f32(__ldg(p.bias + n));
+#pragma unroll
+      for (int j = 0; j < kHalf; ++j) {
+        const int m = m0 + hcol + j;
+        if (m < p.M)
+          p.out[(int64_t)m * p.N + n] = (uint16_t)f32_to_bf16_bits(acc[j] * post + bval);
       }
     }
-    tc_fence_before();
   }
 
   __syncthreads();
@@ -410,8 +456,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-template <int FMT>
-cudaError_t launch_fmt(const LinearArgs& a, int BN) {
+template <int FMT, int BN>
+cudaError_t launch_bn(const LinearArgs& a) {
   constexpr uint32_t kWpk = FMT == INT8_SYM ? 8192u : 4096u;
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
@@ -441,11 +487,11 @@ cudaError_t launch_fmt(const LinearArgs& a, int BN) {
   int S = (int)((200u * 1024u) / stage_bytes);
   if (S > 6) S = 6;
   if (S < 2) S = 2;
-  const size_t smem = (size_t)S * stage_bytes + 1024 + 8 * (3 * S + 1) + 16;
+  const size_t smem = (size_t)S * stage_bytes + 1024 + 8 * (3 * S + 5) + 16;
   static std::once_flag attr_once;
   cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [&] {
-    attr_err = cudaFuncSetAttribute(prefill_kernel<FMT>,
+    attr_err = cudaFuncSetAttribute(prefill_kernel<FMT, BN>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
   });
   if (attr_err != cudaSuccess) return attr_err;
@@ -460,10 +506,21 @@ cudaError_t launch_fmt(const LinearArgs& a, int BN) {
   p.G = a.G;
   p.BN = BN;
   p.stages = S;
-  p.tmem_cols = BN <= 32 ? 32u : (uint32_t)BN;
+  const bool fold = is_int_fmt(FMT) && a.G >= 64 && (a.K / a.G) > 1;
+  p.tmem_cols = (uint32_t)(fold ? 2 * BN : (BN < 32 ? 32 : BN));
   dim3 grid((unsigned)((a.N + 127) / 128), (unsigned)((a.M + BN - 1) / BN));
-  prefill_kernel<FMT><<<grid, kThreads, smem, a.stream>>>(tmX, tmW, p);
+  prefill_kernel<FMT, BN><<<grid, kThreads, smem, a.stream>>>(tmX, tmW, p);
   return cudaGetLastError();
+}
+
+template <int FMT>
+cudaError_t launch_fmt(const LinearArgs& a, int BN) {
+  switch (BN) {
+    case 32: return launch_bn<FMT, 32>(a);
+    case 64: return launch_bn<FMT, 64>(a);
+    case 128: return launch_bn<FMT, 128>(a);
+    default: return launch_bn<FMT, 256>(a);
+  }
 }
 
 }  // namespace
