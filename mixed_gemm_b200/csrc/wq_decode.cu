@@ -42,6 +42,8 @@ struct DecodeParams {
   const uint16_t* bias;
   uint16_t* out;
   int M, N, K, G, cs;
+  int xs_stride;  // bytes per token row of the staged X slice
+  int xs_bytes;   // bytes of the staged X slice (M rows)
 };
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
@@ -68,6 +70,20 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
 template <int FMT, int NT, int RT, int KW, int UB>
 __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   constexpr int KB = FMT == INT8_SYM ? 32 : 64;   // K per 512-byte block
@@ -75,7 +91,7 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   constexpr int NV = RT * NT * 4;                  // accumulators per lane
   constexpr bool kIntFmt = FMT == INT4_SYM || FMT == INT4_ASYM || FMT == INT8_SYM;
 
-  extern __shared__ float red[];
+  extern __shared__ __align__(16) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, tq = lane & 3;
   const int cs = p.cs;
@@ -85,8 +101,21 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   const int64_t nblk = K / KB;
   const int64_t groups = kIntFmt ? K / p.G : 0;
 
+  // this CTA's K blocks [cb, ce), this warp's [wb, we)
   const int64_t cb = rank * nblk / cs, ce = (rank + 1) * nblk / cs;
   const int64_t wb = cb + warp * (ce - cb) / KW, we = cb + (warp + 1) * (ce - cb) / KW;
+
+  // stage the CTA's slice of X (tokens < M, K in [cb*KB, ce*KB)) in shared memory
+  const uint32_t xs = (uint32_t)__cvta_generic_to_shared(smem);
+  float* red = (float*)(smem + p.xs_bytes);
+  {
+    const int64_t kbeg = cb * KB;
+    const int cpr = (int)((ce - cb) * KB / 8);  // 16-byte chunks per token row
+    for (int i = threadIdx.x; i < p.M * cpr; i += KW * 32) {
+      const int tok = i / cpr, c = i - tok * cpr;
+      cp_async16(xs + tok * p.xs_stride + c * 16, p.x + tok * K + kbeg + c * 8);
+    }
+  }
 
   // lookup tables (CB4: centroids rounded to bf16; NVFP4: E2M1 values)
   uint32_t H[4] = {0, 0, 0, 0}, L[4] = {0, 0, 0, 0};
@@ -113,14 +142,16 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
       for (int i = 0; i < 4; ++i) acc[r][nt][i] = 0.f;
 
   const uint4 zero4 = make_uint4(0, 0, 0, 0);
-  for (int64_t b0 = wb; b0 < we; b0 += UB) {
-    uint4 wv[UB][RT];
+  auto load_batch = [&](uint4 (&wv)[UB][RT], int64_t b0) {
 #pragma unroll
     for (int u = 0; u < UB; ++u)
 #pragma unroll
       for (int r = 0; r < RT; ++r)
         wv[u][r] = (b0 + u < we) ? ld_stream(p.w + ((tile0 + r) * nblk + b0 + u) * 32 + lane)
                                  : zero4;
+  };
+
+  auto compute_batch = [&](const uint4 (&wv)[UB][RT], int64_t b0) {
 #pragma unroll
     for (int u = 0; u < UB; ++u) {
       if (b0 + u >= we) break;
@@ -131,7 +162,9 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           const int tok = g + 8 * nt;
-          xv[c][nt] = tok < p.M ? ld_nc(p.x + tok * K + kblk + 32 * c + 8 * tq) : zero4;
+          xv[c][nt] = tok < p.M ? lds128(xs + tok * p.xs_stride +
+                                         (uint32_t)((kblk - cb * KB) + 32 * c + 8 * tq) * 2u)
+                                : zero4;
         }
 #pragma unroll
       for (int c = 0; c < CPB; ++c) {
@@ -156,8 +189,10 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
 #pragma unroll
             for (int s = 0; s < 2; ++s) {
               uint32_t a[4];
-              if constexpr (FMT == INT8_SYM) frag_int8(word(wv[u][r], 2 * s), word(wv[u][r], 2 * s + 1), a);
-              else frag_int4(word(wv[u][r], 2 * c + s), off_g, off_g8, a);
+              if constexpr (FMT == INT8_SYM)
+                frag_int8(word(wv[u][r], 2 * s), word(wv[u][r], 2 * s + 1), a);
+              else
+                frag_int4(word(wv[u][r], 2 * c + s), off_g, off_g8, a);
 #pragma unroll
               for (int nt = 0; nt < NT; ++nt)
                 mma16816(cacc[nt], a, word(xv[c][nt], 2 * s), word(xv[c][nt], 2 * s + 1));
@@ -174,7 +209,8 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
             uint32_t sc_g = 0, sc_g8 = 0;
             if constexpr (FMT == NVFP4) {
               const int64_t blk = (k0 + 8 * tq) >> 4;
-              const uint32_t sb = __ldg((const uint16_t*)p.scales + (tile * (K >> 4) + blk) * 8 + g);
+              const uint32_t sb =
+                  __ldg((const uint16_t*)p.scales + (tile * (K >> 4) + blk) * 8 + g);
               sc_g = f32_to_bf16_bits(e4m3_to_f32(sb & 0xFFu)) * 0x00010001u;
               sc_g8 = f32_to_bf16_bits(e4m3_to_f32(sb >> 8)) * 0x00010001u;
             }
@@ -196,6 +232,19 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
         }
       }
     }
+  };
+
+  // two register batches in flight: while one batch is converted and
+  // multiplied, the loads of the next one are outstanding
+  uint4 wa[UB][RT], wz[UB][RT];
+  load_batch(wa, wb);
+  cp_async_wait_all();
+  __syncthreads();
+  for (int64_t b0 = wb; b0 < we; b0 += 2 * UB) {
+    load_batch(wz, b0 + UB);
+    compute_batch(wa, b0);
+    load_batch(wa, b0 + 2 * UB);
+    compute_batch(wz, b0 + UB);
   }
 
   // ---- reduction: warps -> CTA partial (shared) -> cluster rank 0 (DSMEM)
@@ -242,7 +291,14 @@ template <int FMT, int NT, int RT>
 cudaError_t launch_t(const DecodeParams& p, int grid, cudaStream_t st) {
   constexpr int KW = 4, UB = 4;
   auto kern = decode_kernel<FMT, NT, RT, KW, UB>;
-  const size_t smem = (size_t)(KW + 1) * RT * NT * 4 * 32 * sizeof(float);
+  const size_t smem = (size_t)p.xs_bytes + (size_t)(KW + 1) * RT * NT * 4 * 32 * sizeof(float);
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         227 * 1024);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(KW * 32);
@@ -282,13 +338,24 @@ cudaError_t launch_decode(const LinearArgs& a) {
   const int64_t tiles = a.N / 16;
   const int rt = (tiles % 2 == 0) ? 2 : 1;
   const int64_t rowgroups = tiles / rt;
-  const int64_t nblk = a.K / block_k(a.fmt);
+  const int kb = block_k(a.fmt);
+  const int64_t nblk = a.K / kb;
+  // split K over a cluster: enough CTAs to cover the SMs twice, and a staged
+  // X slice of at most 96 KB
   const int64_t target = 2LL * device_sm_count();
   int64_t cs = (target + rowgroups - 1) / rowgroups;
+  const int64_t x_bytes_all = a.M * a.K * 2;
+  const int64_t cs_x = (x_bytes_all + 98303) / 98304;
+  if (cs < cs_x) cs = cs_x;
   if (cs > 8) cs = 8;
   if (cs > nblk / 4) cs = nblk / 4;  // keep every warp busy
   if (cs < 1) cs = 1;
+  const int64_t max_blocks = (nblk + cs - 1) / cs;
+  const int64_t stride = ((max_blocks * kb * 2 + 127) / 128) * 128 + 64;
+  if (stride * a.M > 200 * 1024) return cudaErrorInvalidValue;  // K too large for M <= 16
   p.cs = (int)cs;
+  p.xs_stride = (int)stride;
+  p.xs_bytes = (int)(stride * a.M);
   const int grid = (int)(rowgroups * cs);
   switch (a.fmt) {
     case INT4_SYM: return launch_fmt<INT4_SYM>(p, nt, rt, grid, a.stream);

@@ -13,13 +13,14 @@
 //                       path's fragment decoders) and store them in the
 //                       canonical 128-byte-swizzled K-major layout;
 //   warps 8..15         fold and epilogue.
-// INT formats with groups of 64 or more keep the tile values exact: the tile
-// holds the integer code (or code minus zero-point), each group of K is
-// accumulated into its own tensor-memory buffer (two buffers alternate), and
-// the fold warps add group_scale[row] * partial into fp32 registers -- the
-// same arithmetic as the decode path, so no bf16 rounding of q*s ever enters
-// the sum.  NVFP4 tiles hold e2m1 * e4m3 (exact in bf16); CB4 tiles hold the
-// bf16 centroid; INT groups of 32 hold the bf16 rounding of q*s.  The
+// INT formats keep the tile values exact: the tile holds the integer code (or
+// code minus zero-point), each group of K is accumulated into its own
+// tensor-memory buffer (two buffers alternate; a group boundary may fall
+// inside a stage for groups of 32), and the fold warps add
+// group_scale[row] * partial into fp32 registers -- the same arithmetic as
+// the decode path, so no bf16 rounding of q*s ever enters the sum.  NVFP4
+// tiles hold e2m1 * e4m3 (exact in bf16); CB4 tiles hold the bf16 centroid.
+// The
 // epilogue applies the CB4 row norm / NVFP4 tensor scale and the bias, rounds
 // to bf16 and stores Y.  Registers are rebalanced per warpgroup with
 // setmaxnreg (56 / 104 / 168 / 168 of the 128 per thread launched).  Every
@@ -192,10 +193,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int m0 = blockIdx.y * BN;
   const int KT = p.K / 64;
   const int ntiles = p.N / 16;
-  // group-scale fold: exact integer tiles, one accumulator per group
-  const bool fold = kInt && p.G >= 64;
-  const int SPG = fold ? p.G / 64 : KT;  // K stages per accumulation group
-  const int NG = KT / SPG;
+  // group-scale fold: exact integer tiles, one accumulator per group of K;
+  // groups are counted in 16-wide MMA steps (two groups per stage for G = 32)
+  const int KPG = kInt ? p.G / 16 : 4 * KT;  // MMA steps per accumulation group
+  const int NG = 4 * KT / KPG;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -247,30 +248,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                              ((128u >> 4) << 24);
       bool ok = true;
-      int kt = 0;
-      for (int g = 0; g < NG && ok; ++g) {
-        const int gb = g & 1;
-        if (g >= 2 && !mbar_wait(gempty_bar(gb), (uint32_t)((g >> 1) - 1) & 1u, abort, 4u)) {
-          ok = false;
-          break;
-        }
+      int gb = 0;
+      uint32_t d = tmem;
+      for (int kt = 0; kt < KT && ok; ++kt) {
+        const int s = kt % S;
+        const uint32_t ph = (uint32_t)(kt / S) & 1u;
+        ok = mbar_wait(full_bar(s), ph, abort, 4u) && mbar_wait(dq_bar(s), ph, abort, 8u);
+        if (!ok) break;
         tc_fence_after();
-        const uint32_t d = tmem + (uint32_t)(gb * BN);
-        for (int sg = 0; sg < SPG; ++sg, ++kt) {
-          const int s = kt % S;
-          const uint32_t ph = (uint32_t)(kt / S) & 1u;
-          ok = mbar_wait(full_bar(s), ph, abort, 4u) && mbar_wait(dq_bar(s), ph, abort, 8u);
-          if (!ok) break;
-          tc_fence_after();
-          uint8_t* st = smem + s * kStage;
-          const uint32_t xa = smem_u32(st), aa = smem_u32(st + kXbytes);
+        uint8_t* st = smem + s * kStage;
+        const uint32_t xa = smem_u32(st), aa = smem_u32(st + kXbytes);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_f16(d, umma_desc_sw128(aa + kk * 32), umma_desc_sw128(xa + kk * 32), idesc,
-                     (sg | kk) != 0);
-          umma_commit(empty_bar(s));
+        for (int kk = 0; kk < 4; ++kk) {
+          const int step = kt * 4 + kk;
+          const int g = step / KPG, in_g = step - g * KPG;
+          if (in_g == 0) {
+            gb = g & 1;
+            d = tmem + (uint32_t)(gb * BN);
+            // the fold of group g-2 must have drained this buffer
+            if (g >= 2 && !mbar_wait(gempty_bar(gb), (uint32_t)((g >> 1) - 1) & 1u, abort, 4u)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          umma_f16(d, umma_desc_sw128(aa + kk * 32), umma_desc_sw128(xa + kk * 32), idesc,
+                   in_g != 0);
+          if (in_g == KPG - 1) umma_commit(gfull_bar(gb));
         }
-        umma_commit(gfull_bar(gb));
+        umma_commit(empty_bar(s));
       }
       if (!ok) {  // wait for this thread's own MMAs before the memory goes away
         umma_commit(drain_bar);
@@ -314,14 +320,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int blk = 0; blk < 2; ++blk) {
             const uint4 ch = *(const uint4*)(wpk + rt * 1024 + blk * 512 + lane * 16);
-            // exact codes (fold) or codes times the group scale (group of 32)
-            uint32_t sc_g = valid ? 0x3F803F80u : 0u, sc_g8 = sc_g;
-            if (!fold && valid) {
-              const int64_t grp = ((int64_t)kt * 64 + 32 * blk) / p.G;
-              const uint32_t sw = __ldg((const uint32_t*)p.scales + (tile * groups + grp) * 8 + g);
-              sc_g = (sw & 0xFFFFu) * 0x00010001u;
-              sc_g8 = (sw >> 16) * 0x00010001u;
-            }
+            // exact codes; the group scale is applied by the fold warps
+            const uint32_t sc_g = valid ? 0x3F803F80u : 0u, sc_g8 = sc_g;
             uint32_t a[4], b[4];
             frag_int8(ch.x, ch.y, a);
             frag_int8(ch.z, ch.w, b);
@@ -342,12 +342,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               uint32_t off_g = 0x43084308u, off_g8 = 0x43084308u;
               if (valid) {
                 const int64_t grp = ((int64_t)kt * 64 + 32 * c) / p.G;
-                if (!fold) {
-                  const uint32_t sw =
-                      __ldg((const uint32_t*)p.scales + (tile * groups + grp) * 8 + g);
-                  sc_g = (sw & 0xFFFFu) * 0x00010001u;
-                  sc_g8 = (sw >> 16) * 0x00010001u;
-                }
                 if constexpr (FMT == INT4_ASYM) {
                   const uint32_t zb =
                       __ldg((const uint8_t*)p.aux + (tile * groups + grp) * 8 + g);
@@ -401,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xffffffffu, ok ? 1 : 0)) { ok = false; break; }
       tc_fence_after();
       float sc = 1.f;
-      if (fold && nvalid) {
+      if (kInt && nvalid) {
         const int r16 = (int)(n & 15);
         sc = bf16_bits_to_f32(__ldg((const uint16_t*)p.scales +
                                     ((n >> 4) * groups + g) * 16 + 2 * (r16 & 7) + (r16 >> 3)));
@@ -506,8 +500,8 @@ cudaError_t launch_bn(const LinearArgs& a) {
   p.G = a.G;
   p.BN = BN;
   p.stages = S;
-  const bool fold = is_int_fmt(FMT) && a.G >= 64 && (a.K / a.G) > 1;
-  p.tmem_cols = (uint32_t)(fold ? 2 * BN : (BN < 32 ? 32 : BN));
+  const bool groups2 = is_int_fmt(FMT) && (a.K / a.G) > 1;  // two alternating accumulators
+  p.tmem_cols = (uint32_t)(groups2 ? 2 * BN : (BN < 32 ? 32 : BN));
   dim3 grid((unsigned)((a.N + 127) / 128), (unsigned)((a.M + BN - 1) / BN));
   prefill_kernel<FMT, BN><<<grid, kThreads, smem, a.stream>>>(tmX, tmW, p);
   return cudaGetLastError();
