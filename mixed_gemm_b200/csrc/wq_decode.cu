@@ -44,6 +44,8 @@ struct DecodeParams {
   int M, N, K, G, cs;
   int xs_stride;  // bytes per token row of the staged X slice
   int xs_bytes;   // bytes of the staged X slice (M rows)
+  int side_rows;  // per row tile: scale groups (INT) or 16-K blocks (NVFP4) staged
+  int side_bytes; // bytes of staged scales / zero-points / block scales
 };
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
@@ -73,8 +75,26 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds16(uint32_t addr) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds8(uint32_t addr) {
+  unsigned short v;
+  asm volatile("ld.shared.u8 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
 }
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
@@ -105,15 +125,47 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   const int64_t cb = rank * nblk / cs, ce = (rank + 1) * nblk / cs;
   const int64_t wb = cb + warp * (ce - cb) / KW, we = cb + (warp + 1) * (ce - cb) / KW;
 
-  // stage the CTA's slice of X (tokens < M, K in [cb*KB, ce*KB)) in shared memory
+  // Stage in shared memory, with cp.async, everything the K loop reads besides
+  // the weight stream: the CTA's slice of X (tokens < M, K in
+  // [cb*KB, ce*KB)), and the group scales + zero-points (INT) or E4M3 block
+  // scales (NVFP4) of its row tiles over that K range.
   const uint32_t xs = (uint32_t)__cvta_generic_to_shared(smem);
-  float* red = (float*)(smem + p.xs_bytes);
+  const uint32_t side = xs + (uint32_t)p.xs_bytes;
+  float* red = (float*)(smem + p.xs_bytes + p.side_bytes);
+  const int64_t kbeg = cb * KB;
+  const int64_t g_begin = kIntFmt ? kbeg / p.G : 0;   // first scale group staged
+  const int64_t b16_begin = kbeg >> 4;                // first NVFP4 16-block staged
   {
-    const int64_t kbeg = cb * KB;
     const int cpr = (int)((ce - cb) * KB / 8);  // 16-byte chunks per token row
     for (int i = threadIdx.x; i < p.M * cpr; i += KW * 32) {
       const int tok = i / cpr, c = i - tok * cpr;
       cp_async16(xs + tok * p.xs_stride + c * 16, p.x + tok * K + kbeg + c * 8);
+    }
+    if constexpr (kIntFmt) {
+      const int64_t g_end = (ce * KB - 1) / p.G + 1;
+      const int ng = (int)(g_end - g_begin);
+      // scales: 32 bytes per (tile, group) -> two 16-byte chunks
+      for (int i = threadIdx.x; i < RT * ng * 2; i += KW * 32) {
+        const int r = i / (ng * 2), rem = i - r * ng * 2, gi = rem >> 1, h = rem & 1;
+        cp_async16(side + (r * p.side_rows + gi) * 32 + h * 16,
+                   (const uint8_t*)p.scales + ((tile0 + r) * groups + g_begin + gi) * 32 + h * 16);
+      }
+      if constexpr (FMT == INT4_ASYM) {
+        const uint32_t zs = side + RT * p.side_rows * 32;
+        for (int i = threadIdx.x; i < RT * ng; i += KW * 32) {
+          const int r = i / ng, gi = i - r * ng;
+          cp_async8(zs + (r * p.side_rows + gi) * 8,
+                    (const uint8_t*)p.aux + ((tile0 + r) * groups + g_begin + gi) * 8);
+        }
+      }
+    }
+    if constexpr (FMT == NVFP4) {
+      const int nb = (int)((ce - cb) * KB / 16);
+      for (int i = threadIdx.x; i < RT * nb; i += KW * 32) {
+        const int r = i / nb, bi = i - r * nb;
+        cp_async16(side + (r * p.side_rows + bi) * 16,
+                   (const uint8_t*)p.scales + ((tile0 + r) * (K >> 4) + b16_begin + bi) * 16);
+      }
     }
   }
 
@@ -163,7 +215,7 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
         for (int nt = 0; nt < NT; ++nt) {
           const int tok = g + 8 * nt;
           xv[c][nt] = tok < p.M ? lds128(xs + tok * p.xs_stride +
-                                         (uint32_t)((kblk - cb * KB) + 32 * c + 8 * tq) * 2u)
+                                         (uint32_t)((kblk - kbeg) + 32 * c + 8 * tq) * 2u)
                                 : zero4;
         }
 #pragma unroll
@@ -173,11 +225,12 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
         for (int r = 0; r < RT; ++r) {
           const int64_t tile = tile0 + r;
           if constexpr (kIntFmt) {
-            const int64_t grp = k0 / p.G;
-            const uint32_t sw = __ldg((const uint32_t*)p.scales + (tile * groups + grp) * 8 + g);
+            const int gi = (int)(k0 / p.G - g_begin);
+            const uint32_t sw = lds32(side + (r * p.side_rows + gi) * 32 + g * 4);
             uint32_t off_g = 0x43084308u, off_g8 = 0x43084308u;  // 136 = 128 + 8
             if constexpr (FMT == INT4_ASYM) {
-              const uint32_t zb = __ldg((const uint8_t*)p.aux + (tile * groups + grp) * 8 + g);
+              const uint32_t zb =
+                  lds8(side + RT * p.side_rows * 32 + (r * p.side_rows + gi) * 8 + g);
               off_g = (0x4300u + (zb & 15u)) * 0x00010001u;
               off_g8 = (0x4300u + (zb >> 4)) * 0x00010001u;
             }
@@ -208,9 +261,8 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
           } else {
             uint32_t sc_g = 0, sc_g8 = 0;
             if constexpr (FMT == NVFP4) {
-              const int64_t blk = (k0 + 8 * tq) >> 4;
-              const uint32_t sb =
-                  __ldg((const uint16_t*)p.scales + (tile * (K >> 4) + blk) * 8 + g);
+              const int bi = (int)(((k0 + 8 * tq) >> 4) - b16_begin);
+              const uint32_t sb = lds16(side + (r * p.side_rows + bi) * 16 + g * 2);
               sc_g = f32_to_bf16_bits(e4m3_to_f32(sb & 0xFFu)) * 0x00010001u;
               sc_g8 = f32_to_bf16_bits(e4m3_to_f32(sb >> 8)) * 0x00010001u;
             }
@@ -291,7 +343,8 @@ template <int FMT, int NT, int RT>
 cudaError_t launch_t(const DecodeParams& p, int grid, cudaStream_t st) {
   constexpr int KW = 4, UB = 4;
   auto kern = decode_kernel<FMT, NT, RT, KW, UB>;
-  const size_t smem = (size_t)p.xs_bytes + (size_t)(KW + 1) * RT * NT * 4 * 32 * sizeof(float);
+  const size_t smem = (size_t)p.xs_bytes + (size_t)p.side_bytes +
+                      (size_t)(KW + 1) * RT * NT * 4 * 32 * sizeof(float);
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -356,6 +409,19 @@ cudaError_t launch_decode(const LinearArgs& a) {
   p.cs = (int)cs;
   p.xs_stride = (int)stride;
   p.xs_bytes = (int)(stride * a.M);
+  // staged side data per row tile: a K range of max_blocks*kb may touch one
+  // more group than it spans
+  if (is_int_fmt(a.fmt)) {
+    p.side_rows = (int)((max_blocks * kb + a.G - 1) / a.G + 1);
+    p.side_bytes = rt * p.side_rows * (a.fmt == INT4_ASYM ? 40 : 32);
+  } else if (a.fmt == NVFP4) {
+    p.side_rows = (int)(max_blocks * kb / 16);
+    p.side_bytes = rt * p.side_rows * 16;
+  } else {
+    p.side_rows = 0;
+    p.side_bytes = 0;
+  }
+  p.side_bytes = (p.side_bytes + 15) & ~15;
   const int grid = (int)(rowgroups * cs);
   switch (a.fmt) {
     case INT4_SYM: return launch_fmt<INT4_SYM>(p, nt, rt, grid, a.stream);
