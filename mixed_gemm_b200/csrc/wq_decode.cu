@@ -44,6 +44,7 @@ struct DecodeParams {
   int M, N, K, G, cs;
   int xs_stride;  // bytes per token row of the staged X slice
   int xs_bytes;   // bytes of the staged X slice (M rows)
+  int gshift;     // log2(group size) for INT formats
   int side_rows;  // per row tile: scale groups (INT) or 16-K blocks (NVFP4) staged
   int side_bytes; // bytes of staged scales / zero-points / block scales
 };
@@ -104,7 +105,21 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   return v;
 }
 
-template <int FMT, int NT, int RT, int KW, int UB>
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+
+// KW warps per CTA; each keeps a ring of D blocks (per row tile) of weight
+// loads in flight: after block j is consumed, the load of block j + D is
+// issued into the freed registers.
+template <int FMT, int NT, int RT, int KW, int D>
 __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   constexpr int KB = FMT == INT8_SYM ? 32 : 64;   // K per 512-byte block
   constexpr int CPB = FMT == INT8_SYM ? 1 : 2;    // 32-K chunks per block
@@ -115,15 +130,18 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, tq = lane & 3;
   const int cs = p.cs;
-  const int rank = (int)(blockIdx.x % cs);
-  const int64_t tile0 = (int64_t)(blockIdx.x / cs) * RT;
-  const int64_t K = p.K;
-  const int64_t nblk = K / KB;
-  const int64_t groups = kIntFmt ? K / p.G : 0;
+  const int rank = (int)(blockIdx.x % (unsigned)cs);
+  const int tile0 = (int)(blockIdx.x / (unsigned)cs) * RT;
+  const int K = p.K;
+  const int nblk = K / KB;
+  const int groups = kIntFmt ? K >> p.gshift : 0;
+
+  if (cs > 1) cluster_arrive_relaxed();  // matched by the wait before DSMEM writes
 
   // this CTA's K blocks [cb, ce), this warp's [wb, we)
-  const int64_t cb = rank * nblk / cs, ce = (rank + 1) * nblk / cs;
-  const int64_t wb = cb + warp * (ce - cb) / KW, we = cb + (warp + 1) * (ce - cb) / KW;
+  const int cb = (int)((int64_t)rank * nblk / cs), ce = (int)((int64_t)(rank + 1) * nblk / cs);
+  const int wb = cb + warp * (ce - cb) / KW, we = cb + (warp + 1) * (ce - cb) / KW;
+  const int nb = we - wb;
 
   // Stage in shared memory, with cp.async, everything the K loop reads besides
   // the weight stream: the CTA's slice of X (tokens < M, K in
@@ -132,42 +150,54 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   const uint32_t xs = (uint32_t)__cvta_generic_to_shared(smem);
   const uint32_t side = xs + (uint32_t)p.xs_bytes;
   float* red = (float*)(smem + p.xs_bytes + p.side_bytes);
-  const int64_t kbeg = cb * KB;
-  const int64_t g_begin = kIntFmt ? kbeg / p.G : 0;   // first scale group staged
-  const int64_t b16_begin = kbeg >> 4;                // first NVFP4 16-block staged
+  const int kbeg = cb * KB;
+  const int g_begin = kIntFmt ? kbeg >> p.gshift : 0;  // first scale group staged
+  const int b16_begin = kbeg >> 4;                      // first NVFP4 16-block staged
   {
-    const int cpr = (int)((ce - cb) * KB / 8);  // 16-byte chunks per token row
+    const int cpr = (ce - cb) * KB / 8;  // 16-byte chunks per token row
     for (int i = threadIdx.x; i < p.M * cpr; i += KW * 32) {
       const int tok = i / cpr, c = i - tok * cpr;
-      cp_async16(xs + tok * p.xs_stride + c * 16, p.x + tok * K + kbeg + c * 8);
+      cp_async16(xs + tok * p.xs_stride + c * 16, p.x + (int64_t)tok * K + kbeg + c * 8);
     }
     if constexpr (kIntFmt) {
-      const int64_t g_end = (ce * KB - 1) / p.G + 1;
-      const int ng = (int)(g_end - g_begin);
+      const int ng = ((ce * KB - 1) >> p.gshift) + 1 - g_begin;
       // scales: 32 bytes per (tile, group) -> two 16-byte chunks
       for (int i = threadIdx.x; i < RT * ng * 2; i += KW * 32) {
         const int r = i / (ng * 2), rem = i - r * ng * 2, gi = rem >> 1, h = rem & 1;
         cp_async16(side + (r * p.side_rows + gi) * 32 + h * 16,
-                   (const uint8_t*)p.scales + ((tile0 + r) * groups + g_begin + gi) * 32 + h * 16);
+                   (const uint8_t*)p.scales +
+                       ((int64_t)(tile0 + r) * groups + g_begin + gi) * 32 + h * 16);
       }
       if constexpr (FMT == INT4_ASYM) {
         const uint32_t zs = side + RT * p.side_rows * 32;
         for (int i = threadIdx.x; i < RT * ng; i += KW * 32) {
           const int r = i / ng, gi = i - r * ng;
           cp_async8(zs + (r * p.side_rows + gi) * 8,
-                    (const uint8_t*)p.aux + ((tile0 + r) * groups + g_begin + gi) * 8);
+                    (const uint8_t*)p.aux + ((int64_t)(tile0 + r) * groups + g_begin + gi) * 8);
         }
       }
     }
     if constexpr (FMT == NVFP4) {
-      const int nb = (int)((ce - cb) * KB / 16);
-      for (int i = threadIdx.x; i < RT * nb; i += KW * 32) {
-        const int r = i / nb, bi = i - r * nb;
+      const int nb16 = (ce - cb) * KB / 16;
+      for (int i = threadIdx.x; i < RT * nb16; i += KW * 32) {
+        const int r = i / nb16, bi = i - r * nb16;
         cp_async16(side + (r * p.side_rows + bi) * 16,
-                   (const uint8_t*)p.scales + ((tile0 + r) * (K >> 4) + b16_begin + bi) * 16);
+                   (const uint8_t*)p.scales +
+                       ((int64_t)(tile0 + r) * (K >> 4) + b16_begin + bi) * 16);
       }
     }
   }
+
+  // weight ring: D blocks per row tile in flight
+  const uint4* wrow[RT];
+#pragma unroll
+  for (int r = 0; r < RT; ++r) wrow[r] = p.w + (int64_t)(tile0 + r) * nblk * 32 + lane;
+  uint4 wv[D][RT];
+#pragma unroll
+  for (int j = 0; j < D; ++j)
+#pragma unroll
+    for (int r = 0; r < RT; ++r)
+      if (j < nb) wv[j][r] = ld_stream(wrow[r] + (wb + j) * 32);
 
   // lookup tables (CB4: centroids rounded to bf16; NVFP4: E2M1 values)
   uint32_t H[4] = {0, 0, 0, 0}, L[4] = {0, 0, 0, 0};
@@ -193,158 +223,147 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[r][nt][i] = 0.f;
 
-  const uint4 zero4 = make_uint4(0, 0, 0, 0);
-  auto load_batch = [&](uint4 (&wv)[UB][RT], int64_t b0) {
-#pragma unroll
-    for (int u = 0; u < UB; ++u)
-#pragma unroll
-      for (int r = 0; r < RT; ++r)
-        wv[u][r] = (b0 + u < we) ? ld_stream(p.w + ((tile0 + r) * nblk + b0 + u) * 32 + lane)
-                                 : zero4;
-  };
+  cp_async_wait_all();
+  __syncthreads();
 
-  auto compute_batch = [&](const uint4 (&wv)[UB][RT], int64_t b0) {
+  const uint4 zero4 = make_uint4(0, 0, 0, 0);
+  auto compute_block = [&](const uint4 (&wb_)[RT], int b) {
+    const int kblk = b * KB;
+    uint4 xv[CPB][NT];
 #pragma unroll
-    for (int u = 0; u < UB; ++u) {
-      if (b0 + u >= we) break;
-      const int64_t kblk = (b0 + u) * KB;
-      uint4 xv[CPB][NT];
+    for (int c = 0; c < CPB; ++c)
 #pragma unroll
-      for (int c = 0; c < CPB; ++c)
+      for (int nt = 0; nt < NT; ++nt) {
+        const int tok = g + 8 * nt;
+        xv[c][nt] = tok < p.M ? lds128(xs + tok * p.xs_stride +
+                                       (uint32_t)((kblk - kbeg) + 32 * c + 8 * tq) * 2u)
+                              : zero4;
+      }
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const int tok = g + 8 * nt;
-          xv[c][nt] = tok < p.M ? lds128(xs + tok * p.xs_stride +
-                                         (uint32_t)((kblk - kbeg) + 32 * c + 8 * tq) * 2u)
-                                : zero4;
-        }
+    for (int c = 0; c < CPB; ++c) {
+      const int k0 = kblk + 32 * c;
 #pragma unroll
-      for (int c = 0; c < CPB; ++c) {
-        const int64_t k0 = kblk + 32 * c;
+      for (int r = 0; r < RT; ++r) {
+        if constexpr (kIntFmt) {
+          const int gi = (k0 >> p.gshift) - g_begin;
+          const uint32_t sw = lds32(side + (r * p.side_rows + gi) * 32 + g * 4);
+          uint32_t off_g = 0x43084308u, off_g8 = 0x43084308u;  // 136 = 128 + 8
+          if constexpr (FMT == INT4_ASYM) {
+            const uint32_t zb = lds8(side + RT * p.side_rows * 32 + (r * p.side_rows + gi) * 8 + g);
+            off_g = (0x4300u + (zb & 15u)) * 0x00010001u;
+            off_g8 = (0x4300u + (zb >> 4)) * 0x00010001u;
+          }
+          float cacc[NT][4];
 #pragma unroll
-        for (int r = 0; r < RT; ++r) {
-          const int64_t tile = tile0 + r;
-          if constexpr (kIntFmt) {
-            const int gi = (int)(k0 / p.G - g_begin);
-            const uint32_t sw = lds32(side + (r * p.side_rows + gi) * 32 + g * 4);
-            uint32_t off_g = 0x43084308u, off_g8 = 0x43084308u;  // 136 = 128 + 8
-            if constexpr (FMT == INT4_ASYM) {
-              const uint32_t zb =
-                  lds8(side + RT * p.side_rows * 32 + (r * p.side_rows + gi) * 8 + g);
-              off_g = (0x4300u + (zb & 15u)) * 0x00010001u;
-              off_g8 = (0x4300u + (zb >> 4)) * 0x00010001u;
-            }
-            float cacc[NT][4];
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) cacc[nt][i] = 0.f;
+#pragma unroll
+          for (int s = 0; s < 2; ++s) {
+            uint32_t a[4];
+            if constexpr (FMT == INT8_SYM)
+              frag_int8(word(wb_[r], 2 * s), word(wb_[r], 2 * s + 1), a);
+            else
+              frag_int4(word(wb_[r], 2 * c + s), off_g, off_g8, a);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
+              mma16816(cacc[nt], a, word(xv[c][nt], 2 * s), word(xv[c][nt], 2 * s + 1));
+          }
+          const float s_g = __uint_as_float(sw << 16), s_g8 = __uint_as_float(sw & 0xFFFF0000u);
 #pragma unroll
-              for (int i = 0; i < 4; ++i) cacc[nt][i] = 0.f;
+          for (int nt = 0; nt < NT; ++nt) {
+            acc[r][nt][0] = fmaf(s_g, cacc[nt][0], acc[r][nt][0]);
+            acc[r][nt][1] = fmaf(s_g, cacc[nt][1], acc[r][nt][1]);
+            acc[r][nt][2] = fmaf(s_g8, cacc[nt][2], acc[r][nt][2]);
+            acc[r][nt][3] = fmaf(s_g8, cacc[nt][3], acc[r][nt][3]);
+          }
+        } else {
+          uint32_t sc_g = 0, sc_g8 = 0;
+          if constexpr (FMT == NVFP4) {
+            const int bi = ((k0 + 8 * tq) >> 4) - b16_begin;
+            const uint32_t sb = lds16(side + (r * p.side_rows + bi) * 16 + g * 2);
+            sc_g = f32_to_bf16_bits(e4m3_to_f32(sb & 0xFFu)) * 0x00010001u;
+            sc_g8 = f32_to_bf16_bits(e4m3_to_f32(sb >> 8)) * 0x00010001u;
+          }
 #pragma unroll
-            for (int s = 0; s < 2; ++s) {
-              uint32_t a[4];
-              if constexpr (FMT == INT8_SYM)
-                frag_int8(word(wv[u][r], 2 * s), word(wv[u][r], 2 * s + 1), a);
-              else
-                frag_int4(word(wv[u][r], 2 * c + s), off_g, off_g8, a);
-#pragma unroll
-              for (int nt = 0; nt < NT; ++nt)
-                mma16816(cacc[nt], a, word(xv[c][nt], 2 * s), word(xv[c][nt], 2 * s + 1));
-            }
-            const float s_g = __uint_as_float(sw << 16), s_g8 = __uint_as_float(sw & 0xFFFF0000u);
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-              acc[r][nt][0] = fmaf(s_g, cacc[nt][0], acc[r][nt][0]);
-              acc[r][nt][1] = fmaf(s_g, cacc[nt][1], acc[r][nt][1]);
-              acc[r][nt][2] = fmaf(s_g8, cacc[nt][2], acc[r][nt][2]);
-              acc[r][nt][3] = fmaf(s_g8, cacc[nt][3], acc[r][nt][3]);
-            }
-          } else {
-            uint32_t sc_g = 0, sc_g8 = 0;
+          for (int s = 0; s < 2; ++s) {
+            uint32_t a[4];
+            frag_table<FMT == NVFP4>(word(wb_[r], 2 * c + s), H, L, a);
             if constexpr (FMT == NVFP4) {
-              const int bi = (int)(((k0 + 8 * tq) >> 4) - b16_begin);
-              const uint32_t sb = lds16(side + (r * p.side_rows + bi) * 16 + g * 2);
-              sc_g = f32_to_bf16_bits(e4m3_to_f32(sb & 0xFFu)) * 0x00010001u;
-              sc_g8 = f32_to_bf16_bits(e4m3_to_f32(sb >> 8)) * 0x00010001u;
+              a[0] = bmul2(a[0], sc_g);
+              a[1] = bmul2(a[1], sc_g8);
+              a[2] = bmul2(a[2], sc_g);
+              a[3] = bmul2(a[3], sc_g8);
             }
 #pragma unroll
-            for (int s = 0; s < 2; ++s) {
-              uint32_t a[4];
-              frag_table<FMT == NVFP4>(word(wv[u][r], 2 * c + s), H, L, a);
-              if constexpr (FMT == NVFP4) {
-                a[0] = bmul2(a[0], sc_g);
-                a[1] = bmul2(a[1], sc_g8);
-                a[2] = bmul2(a[2], sc_g);
-                a[3] = bmul2(a[3], sc_g8);
-              }
-#pragma unroll
-              for (int nt = 0; nt < NT; ++nt)
-                mma16816(acc[r][nt], a, word(xv[c][nt], 2 * s), word(xv[c][nt], 2 * s + 1));
-            }
+            for (int nt = 0; nt < NT; ++nt)
+              mma16816(acc[r][nt], a, word(xv[c][nt], 2 * s), word(xv[c][nt], 2 * s + 1));
           }
         }
       }
     }
   };
 
-  // two register batches in flight: while one batch is converted and
-  // multiplied, the loads of the next one are outstanding
-  uint4 wa[UB][RT], wz[UB][RT];
-  load_batch(wa, wb);
-  cp_async_wait_all();
-  __syncthreads();
-  for (int64_t b0 = wb; b0 < we; b0 += 2 * UB) {
-    load_batch(wz, b0 + UB);
-    compute_batch(wa, b0);
-    load_batch(wa, b0 + 2 * UB);
-    compute_batch(wz, b0 + UB);
-  }
-
-  // ---- reduction: warps -> CTA partial (shared) -> cluster rank 0 (DSMEM)
+  for (int i = 0; i < nb; i += D) {
 #pragma unroll
-  for (int r = 0; r < RT; ++r)
+    for (int j = 0; j < D; ++j) {
+      if (i + j < nb) {
+        compute_block(wv[j], wb + i + j);
+        if (i + j + D < nb) {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) red[(warp * NV + (r * NT + nt) * 4 + i) * 32 + lane] = acc[r][nt][i];
-  __syncthreads();
-  float* part = red + KW * NV * 32;
-  for (int idx = threadIdx.x; idx < NV * 32; idx += KW * 32) {
-    float s = 0.f;
-#pragma unroll
-    for (int w = 0; w < KW; ++w) s += red[w * NV * 32 + idx];
-    part[idx] = s;
-  }
-  if (cs > 1) cg::this_cluster().sync();
-  else __syncthreads();
-  if (rank == 0) {
-    float tsc = 1.f;
-    if constexpr (FMT == NVFP4) tsc = __ldg((const float*)p.aux);
-    for (int idx = threadIdx.x; idx < NV * 32; idx += KW * 32) {
-      float tot = part[idx];
-      for (int q = 1; q < cs; ++q) tot += cg::this_cluster().map_shared_rank(part, q)[idx];
-      const int v = idx >> 5, ln = idx & 31;
-      const int r = v / (NT * 4), nt = (v / 4) % NT, i = v & 3;
-      const int gg = ln >> 2, tt = ln & 3;
-      const int64_t n = (tile0 + r) * 16 + gg + 8 * (i >> 1);
-      const int m = nt * 8 + 2 * tt + (i & 1);
-      if (m < p.M) {
-        float fold = tsc;
-        if constexpr (FMT == CB4) fold = bf16_bits_to_f32(__ldg((const uint16_t*)p.scales + n));
-        float y = tot * fold;
-        if (p.bias) y += bf16_bits_to_f32(__ldg(p.bias + n));
-        p.out[(int64_t)m * p.N + n] = (uint16_t)f32_to_bf16_bits(y);
+          for (int r = 0; r < RT; ++r) wv[j][r] = ld_stream(wrow[r] + (wb + i + j + D) * 32);
+        }
       }
     }
   }
-  if (cs > 1) cg::this_cluster().sync();
+
+  // ---- reduction: every warp writes its partial into cluster rank 0's
+  // shared memory (slot rank*KW + warp); one cluster barrier; rank 0 sums.
+  float* red0 = red;
+  if (cs > 1) {
+    cluster_wait();  // every CTA of the cluster has started
+    red0 = cg::this_cluster().map_shared_rank(red, 0);
+  }
+  {
+    float* dst = red0 + (size_t)(rank * KW + warp) * NV * 32 + lane;
+#pragma unroll
+    for (int r = 0; r < RT; ++r)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dst[((r * NT + nt) * 4 + i) * 32] = acc[r][nt][i];
+  }
+  if (cs > 1) cluster_sync_all();
+  else __syncthreads();
+  if (rank != 0) return;
+
+  float tsc = 1.f;
+  if constexpr (FMT == NVFP4) tsc = __ldg((const float*)p.aux);
+  const int slots = cs * KW;
+  for (int idx = threadIdx.x; idx < NV * 32; idx += KW * 32) {
+    float tot = 0.f;
+    for (int sl = 0; sl < slots; ++sl) tot += red[sl * NV * 32 + idx];
+    const int v = idx >> 5, ln = idx & 31;
+    const int r = v / (NT * 4), nt = (v / 4) % NT, i = v & 3;
+    const int gg = ln >> 2, tt = ln & 3;
+    const int n = (tile0 + r) * 16 + gg + 8 * (i >> 1);
+    const int m = nt * 8 + 2 * tt + (i & 1);
+    if (m < p.M) {
+      float fold = tsc;
+      if constexpr (FMT == CB4) fold = bf16_bits_to_f32(__ldg((const uint16_t*)p.scales + n));
+      float y = tot * fold;
+      if (p.bias) y += bf16_bits_to_f32(__ldg(p.bias + n));
+      p.out[(int64_t)m * p.N + n] = (uint16_t)f32_to_bf16_bits(y);
+    }
+  }
 }
 
 template <int FMT, int NT, int RT>
 cudaError_t launch_t(const DecodeParams& p, int grid, cudaStream_t st) {
-  constexpr int KW = 4, UB = 4;
-  auto kern = decode_kernel<FMT, NT, RT, KW, UB>;
+  constexpr int KW = 4, D = 4;
+  auto kern = decode_kernel<FMT, NT, RT, KW, D>;
   const size_t smem = (size_t)p.xs_bytes + (size_t)p.side_bytes +
-                      (size_t)(KW + 1) * RT * NT * 4 * 32 * sizeof(float);
+                      (size_t)p.cs * KW * RT * NT * 4 * 32 * sizeof(float);
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -369,8 +388,14 @@ cudaError_t launch_t(const DecodeParams& p, int grid, cudaStream_t st) {
 
 template <int FMT>
 cudaError_t launch_fmt(const DecodeParams& p, int nt, int rt, int grid, cudaStream_t st) {
-  if (nt == 1) return rt == 2 ? launch_t<FMT, 1, 2>(p, grid, st) : launch_t<FMT, 1, 1>(p, grid, st);
-  return rt == 2 ? launch_t<FMT, 2, 2>(p, grid, st) : launch_t<FMT, 2, 1>(p, grid, st);
+  if (nt == 1) {
+    if (rt == 4) return launch_t<FMT, 1, 4>(p, grid, st);
+    if (rt == 2) return launch_t<FMT, 1, 2>(p, grid, st);
+    return launch_t<FMT, 1, 1>(p, grid, st);
+  }
+  if (rt == 4) return launch_t<FMT, 2, 4>(p, grid, st);
+  if (rt == 2) return launch_t<FMT, 2, 2>(p, grid, st);
+  return launch_t<FMT, 2, 1>(p, grid, st);
 }
 
 }  // namespace
@@ -389,13 +414,15 @@ cudaError_t launch_decode(const LinearArgs& a) {
   p.G = a.G;
   const int nt = a.M <= 8 ? 1 : 2;
   const int64_t tiles = a.N / 16;
-  const int rt = (tiles % 2 == 0) ? 2 : 1;
+  // more row tiles per CTA when there are more tokens: the staged X slice is
+  // then reused across more weight rows
+  const int rt = (nt == 2 && tiles % 4 == 0) ? 4 : (tiles % 2 == 0) ? 2 : 1;
   const int64_t rowgroups = tiles / rt;
   const int kb = block_k(a.fmt);
   const int64_t nblk = a.K / kb;
-  // split K over a cluster: enough CTAs to cover the SMs twice, and a staged
-  // X slice of at most 96 KB
-  const int64_t target = 2LL * device_sm_count();
+  // split K over a cluster: about four 4-warp CTAs per SM, and a staged X
+  // slice of at most 96 KB
+  const int64_t target = 4LL * device_sm_count();
   int64_t cs = (target + rowgroups - 1) / rowgroups;
   const int64_t x_bytes_all = a.M * a.K * 2;
   const int64_t cs_x = (x_bytes_all + 98303) / 98304;
@@ -411,7 +438,9 @@ cudaError_t launch_decode(const LinearArgs& a) {
   p.xs_bytes = (int)(stride * a.M);
   // staged side data per row tile: a K range of max_blocks*kb may touch one
   // more group than it spans
+  p.gshift = 0;
   if (is_int_fmt(a.fmt)) {
+    while ((1 << p.gshift) < a.G) ++p.gshift;
     p.side_rows = (int)((max_blocks * kb + a.G - 1) / a.G + 1);
     p.side_bytes = rt * p.side_rows * (a.fmt == INT4_ASYM ? 40 : 32);
   } else if (a.fmt == NVFP4) {
@@ -422,6 +451,8 @@ cudaError_t launch_decode(const LinearArgs& a) {
     p.side_bytes = 0;
   }
   p.side_bytes = (p.side_bytes + 15) & ~15;
+  const int64_t red_bytes = cs * 4 * rt * nt * 4 * 32 * 4;
+  if (p.xs_bytes + p.side_bytes + red_bytes > 227 * 1024) return cudaErrorInvalidValue;
   const int grid = (int)(rowgroups * cs);
   switch (a.fmt) {
     case INT4_SYM: return launch_fmt<INT4_SYM>(p, nt, rt, grid, a.stream);
