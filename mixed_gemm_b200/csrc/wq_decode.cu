@@ -24,6 +24,7 @@
 // performance" (batches below 16 are the small-batch regime, weights shuffled
 // offline for cheap dequantization).
 #include <cooperative_groups.h>
+#include <stdlib.h>
 
 #include "wq_frag.cuh"
 #include "wq_internal.cuh"
@@ -47,6 +48,8 @@ struct DecodeParams {
   int gshift;     // log2(group size) for INT formats
   int side_rows;  // per row tile: scale groups (INT) or 16-K blocks (NVFP4) staged
   int side_bytes; // bytes of staged scales / zero-points / block scales
+  int red_off;    // offset of the cluster partial slots (after the larger of
+                  // the staged data and the per-warp partials)
 };
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
@@ -149,7 +152,6 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   // scales (NVFP4) of its row tiles over that K range.
   const uint32_t xs = (uint32_t)__cvta_generic_to_shared(smem);
   const uint32_t side = xs + (uint32_t)p.xs_bytes;
-  float* red = (float*)(smem + p.xs_bytes + p.side_bytes);
   const int kbeg = cb * KB;
   const int g_begin = kIntFmt ? kbeg >> p.gshift : 0;  // first scale group staged
   const int b16_begin = kbeg >> 4;                      // first NVFP4 16-block staged
@@ -317,21 +319,29 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
     }
   }
 
-  // ---- reduction: every warp writes its partial into cluster rank 0's
-  // shared memory (slot rank*KW + warp); one cluster barrier; rank 0 sums.
-  float* red0 = red;
+  // ---- reduction: warps -> CTA partial in this CTA's shared memory (the X
+  // slice region is free now); the CTA partial goes into slot `rank` of
+  // cluster rank 0's shared memory; one cluster barrier; rank 0 sums.
+  __syncthreads();  // every warp is done reading the staged slice
+  float* loc = (float*)smem;
+  float* slots = (float*)(smem + p.red_off);
+#pragma unroll
+  for (int r = 0; r < RT; ++r)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) loc[(warp * NV + (r * NT + nt) * 4 + i) * 32 + lane] = acc[r][nt][i];
+  __syncthreads();
+  float* slots0 = slots;
   if (cs > 1) {
     cluster_wait();  // every CTA of the cluster has started
-    red0 = cg::this_cluster().map_shared_rank(red, 0);
+    slots0 = cg::this_cluster().map_shared_rank(slots, 0);
   }
-  {
-    float* dst = red0 + (size_t)(rank * KW + warp) * NV * 32 + lane;
+  for (int idx = threadIdx.x; idx < NV * 32; idx += KW * 32) {
+    float sum = 0.f;
 #pragma unroll
-    for (int r = 0; r < RT; ++r)
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) dst[((r * NT + nt) * 4 + i) * 32] = acc[r][nt][i];
+    for (int w = 0; w < KW; ++w) sum += loc[w * NV * 32 + idx];
+    slots0[rank * NV * 32 + idx] = sum;
   }
   if (cs > 1) cluster_sync_all();
   else __syncthreads();
@@ -339,10 +349,9 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
 
   float tsc = 1.f;
   if constexpr (FMT == NVFP4) tsc = __ldg((const float*)p.aux);
-  const int slots = cs * KW;
   for (int idx = threadIdx.x; idx < NV * 32; idx += KW * 32) {
     float tot = 0.f;
-    for (int sl = 0; sl < slots; ++sl) tot += red[sl * NV * 32 + idx];
+    for (int q = 0; q < cs; ++q) tot += slots[q * NV * 32 + idx];
     const int v = idx >> 5, ln = idx & 31;
     const int r = v / (NT * 4), nt = (v / 4) % NT, i = v & 3;
     const int gg = ln >> 2, tt = ln & 3;
@@ -362,8 +371,7 @@ template <int FMT, int NT, int RT>
 cudaError_t launch_t(const DecodeParams& p, int grid, cudaStream_t st) {
   constexpr int KW = 4, D = 4;
   auto kern = decode_kernel<FMT, NT, RT, KW, D>;
-  const size_t smem = (size_t)p.xs_bytes + (size_t)p.side_bytes +
-                      (size_t)p.cs * KW * RT * NT * 4 * 32 * sizeof(float);
+  const size_t smem = (size_t)p.red_off + (size_t)p.cs * RT * NT * 4 * 32 * sizeof(float);
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -416,7 +424,10 @@ cudaError_t launch_decode(const LinearArgs& a) {
   const int64_t tiles = a.N / 16;
   // more row tiles per CTA when there are more tokens: the staged X slice is
   // then reused across more weight rows
-  const int rt = (nt == 2 && tiles % 4 == 0) ? 4 : (tiles % 2 == 0) ? 2 : 1;
+  int rt = (nt == 2 && tiles % 4 == 0) ? 4 : (tiles % 2 == 0) ? 2 : 1;
+#ifdef WQ_TUNING
+  if (const char* e = getenv("WQ_DECODE_RT")) rt = atoi(e);
+#endif
   const int64_t rowgroups = tiles / rt;
   const int kb = block_k(a.fmt);
   const int64_t nblk = a.K / kb;
@@ -430,6 +441,9 @@ cudaError_t launch_decode(const LinearArgs& a) {
   if (cs > 8) cs = 8;
   if (cs > nblk / 4) cs = nblk / 4;  // keep every warp busy
   if (cs < 1) cs = 1;
+#ifdef WQ_TUNING
+  if (const char* e = getenv("WQ_DECODE_CS")) cs = atoi(e);
+#endif
   const int64_t max_blocks = (nblk + cs - 1) / cs;
   const int64_t stride = ((max_blocks * kb * 2 + 127) / 128) * 128 + 64;
   if (stride * a.M > 200 * 1024) return cudaErrorInvalidValue;  // K too large for M <= 16
@@ -451,8 +465,11 @@ cudaError_t launch_decode(const LinearArgs& a) {
     p.side_bytes = 0;
   }
   p.side_bytes = (p.side_bytes + 15) & ~15;
-  const int64_t red_bytes = cs * 4 * rt * nt * 4 * 32 * 4;
-  if (p.xs_bytes + p.side_bytes + red_bytes > 227 * 1024) return cudaErrorInvalidValue;
+  const int64_t warp_partials = 4LL * rt * nt * 4 * 32 * 4;  // KW = 4 warps
+  int64_t region = p.xs_bytes + p.side_bytes;
+  if (region < warp_partials) region = warp_partials;
+  p.red_off = (int)((region + 15) & ~15LL);
+  if (p.red_off + cs * rt * nt * 4 * 32 * 4 > 227 * 1024) return cudaErrorInvalidValue;
   const int grid = (int)(rowgroups * cs);
   switch (a.fmt) {
     case INT4_SYM: return launch_fmt<INT4_SYM>(p, nt, rt, grid, a.stream);
