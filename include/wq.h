@@ -129,6 +129,12 @@ int wq_dequant(int format, int64_t N, int64_t K, int group_size, const void* pac
  *   bias     device bf16 [N], or NULL
  *   out      device bf16 [M, N] row-major; must not overlap any input
  * M == 0 is a no-op returning WQ_OK.  Asynchronous; no workspace.
+ * Launched with programmatic dependent launch: the kernel may start while
+ * the previous kernel on `stream` is finishing, requests the packed weight,
+ * scales and aux at once, and reads x / writes out only after the previous
+ * kernel has completed.  The packed buffers must therefore already be final
+ * when the previous kernel on `stream` starts (pack at load time, or put any
+ * other stream operation between wq_pack and the first wq_linear).
  * M <= 16 runs the decode kernel (register dequant, warp-level tensor-core
  * fragments, split-K over warps); larger M runs the prefill kernel (TMA into
  * shared memory, dequant to bf16 in shared memory, tcgen05 MMA into tensor

@@ -32,8 +32,10 @@ class PackedWeight:
         return self.w.numel() + self.scales.numel() + (0 if self.aux is None else self.aux.numel())
 
     def clone(self) -> "PackedWeight":
-        return PackedWeight(self.fmt, self.N, self.K, self.group_size, self.w.clone(),
-                            self.scales.clone(), None if self.aux is None else self.aux.clone())
+        c = PackedWeight(self.fmt, self.N, self.K, self.group_size, self.w.clone(),
+                         self.scales.clone(), None if self.aux is None else self.aux.clone())
+        torch.cuda.synchronize(self.w.device)  # final before any wq_linear prefetches it
+        return c
 
 
 def _bytes(n: int, device) -> torch.Tensor:
@@ -43,12 +45,16 @@ def _bytes(n: int, device) -> torch.Tensor:
 
 def pack(fmt: str, N: int, K: int, group_size: int, codes: torch.Tensor, scales: torch.Tensor,
          aux: torch.Tensor | None, stream=None) -> PackedWeight:
-    """Canonical device buffers -> PackedWeight (wq_pack)."""
+    """Canonical device buffers -> PackedWeight (wq_pack).
+
+    Offline: waits for the pack to finish, so that the packed buffers are
+    final before any wq_linear that may prefetch them (see wq.h)."""
     dev = codes.device
     wb, sb, ab = wq_packed_sizes(fmt, N, K, group_size)
     pw, ps = _bytes(wb, dev), _bytes(sb, dev)
     pa = _bytes(ab, dev) if ab else None
     wq_pack(fmt, N, K, group_size, codes, scales, aux, pw, ps, pa, stream)
+    torch.cuda.synchronize(dev)
     return PackedWeight(fmt, N, K, group_size, pw, ps, pa)
 
 

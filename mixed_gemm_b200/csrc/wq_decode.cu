@@ -156,11 +156,6 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   const int g_begin = kIntFmt ? kbeg >> p.gshift : 0;  // first scale group staged
   const int b16_begin = kbeg >> 4;                      // first NVFP4 16-block staged
   {
-    const int cpr = (ce - cb) * KB / 8;  // 16-byte chunks per token row
-    for (int i = threadIdx.x; i < p.M * cpr; i += KW * 32) {
-      const int tok = i / cpr, c = i - tok * cpr;
-      cp_async16(xs + tok * p.xs_stride + c * 16, p.x + (int64_t)tok * K + kbeg + c * 8);
-    }
     if constexpr (kIntFmt) {
       const int ng = ((ce * KB - 1) >> p.gshift) + 1 - g_begin;
       // scales: 32 bytes per (tile, group) -> two 16-byte chunks
@@ -201,6 +196,21 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
     for (int r = 0; r < RT; ++r)
       if (j < nb) wv[j][r] = ld_stream(wrow[r] + (wb + j) * 32);
 
+  // Programmatic dependent launch: the packed weight and its scales never
+  // depend on the previous kernel in the stream, so they are requested above
+  // before waiting for it; X (typically the previous kernel's output) is read
+  // and Y written only after the wait.  The next kernel may be scheduled as
+  // soon as every CTA of this one got here.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  {
+    const int cpr = (ce - cb) * KB / 8;  // 16-byte chunks per token row
+    for (int i = threadIdx.x; i < p.M * cpr; i += KW * 32) {
+      const int tok = i / cpr, c = i - tok * cpr;
+      cp_async16(xs + tok * p.xs_stride + c * 16, p.x + (int64_t)tok * K + kbeg + c * 8);
+    }
+  }
+
   // lookup tables (CB4: centroids rounded to bf16; NVFP4: E2M1 values)
   uint32_t H[4] = {0, 0, 0, 0}, L[4] = {0, 0, 0, 0};
   if constexpr (FMT == NVFP4) {
@@ -224,6 +234,16 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[r][nt][i] = 0.f;
+  // INT group state: chunk accumulator, packed scales, zero-point offsets
+  // (bf16 pairs of 128 + z; 136 = 128 + 8 for offset-binary signed codes)
+  float cacc[kIntFmt ? RT : 1][NT][4];
+  uint32_t gsw[RT], goff[RT][2];
+  const int gmask = kIntFmt ? (1 << p.gshift) - 1 : 0;
+#pragma unroll
+  for (int r = 0; r < RT; ++r) {
+    gsw[r] = 0;
+    goff[r][0] = goff[r][1] = 0x43084308u;
+  }
 
   cp_async_wait_all();
   __syncthreads();
@@ -244,40 +264,54 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
 #pragma unroll
     for (int c = 0; c < CPB; ++c) {
       const int k0 = kblk + 32 * c;
+      // INT formats: one accumulator per group of K (per row tile), scaled
+      // once when the group ends; the group's scale and zero-point are read
+      // once when it starts (a warp's range may begin or end inside a group)
+      const bool gstart = ((k0 & gmask) == 0) || (k0 == wb * KB);
+      const bool gend = (((k0 + 32) & gmask) == 0) || (k0 + 32 == we * KB);
+      if constexpr (kIntFmt) {
+        if (gstart) {
+          const int gi = (k0 >> p.gshift) - g_begin;
+#pragma unroll
+          for (int r = 0; r < RT; ++r) {
+            gsw[r] = lds32(side + (r * p.side_rows + gi) * 32 + g * 4);
+            if constexpr (FMT == INT4_ASYM) {
+              const uint32_t zb =
+                  lds8(side + RT * p.side_rows * 32 + (r * p.side_rows + gi) * 8 + g);
+              goff[r][0] = (0x4300u + (zb & 15u)) * 0x00010001u;
+              goff[r][1] = (0x4300u + (zb >> 4)) * 0x00010001u;
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+              for (int i = 0; i < 4; ++i) cacc[r][nt][i] = 0.f;
+          }
+        }
+      }
 #pragma unroll
       for (int r = 0; r < RT; ++r) {
         if constexpr (kIntFmt) {
-          const int gi = (k0 >> p.gshift) - g_begin;
-          const uint32_t sw = lds32(side + (r * p.side_rows + gi) * 32 + g * 4);
-          uint32_t off_g = 0x43084308u, off_g8 = 0x43084308u;  // 136 = 128 + 8
-          if constexpr (FMT == INT4_ASYM) {
-            const uint32_t zb = lds8(side + RT * p.side_rows * 32 + (r * p.side_rows + gi) * 8 + g);
-            off_g = (0x4300u + (zb & 15u)) * 0x00010001u;
-            off_g8 = (0x4300u + (zb >> 4)) * 0x00010001u;
-          }
-          float cacc[NT][4];
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) cacc[nt][i] = 0.f;
 #pragma unroll
           for (int s = 0; s < 2; ++s) {
             uint32_t a[4];
             if constexpr (FMT == INT8_SYM)
               frag_int8(word(wb_[r], 2 * s), word(wb_[r], 2 * s + 1), a);
             else
-              frag_int4(word(wb_[r], 2 * c + s), off_g, off_g8, a);
+              frag_int4(word(wb_[r], 2 * c + s), goff[r][0], goff[r][1], a);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
-              mma16816(cacc[nt], a, word(xv[c][nt], 2 * s), word(xv[c][nt], 2 * s + 1));
+              mma16816(cacc[r][nt], a, word(xv[c][nt], 2 * s), word(xv[c][nt], 2 * s + 1));
           }
-          const float s_g = __uint_as_float(sw << 16), s_g8 = __uint_as_float(sw & 0xFFFF0000u);
+          if (gend) {
+            const float s_g = __uint_as_float(gsw[r] << 16);
+            const float s_g8 = __uint_as_float(gsw[r] & 0xFFFF0000u);
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            acc[r][nt][0] = fmaf(s_g, cacc[nt][0], acc[r][nt][0]);
-            acc[r][nt][1] = fmaf(s_g, cacc[nt][1], acc[r][nt][1]);
-            acc[r][nt][2] = fmaf(s_g8, cacc[nt][2], acc[r][nt][2]);
-            acc[r][nt][3] = fmaf(s_g8, cacc[nt][3], acc[r][nt][3]);
+            for (int nt = 0; nt < NT; ++nt) {
+              acc[r][nt][0] = fmaf(s_g, cacc[r][nt][0], acc[r][nt][0]);
+              acc[r][nt][1] = fmaf(s_g, cacc[r][nt][1], acc[r][nt][1]);
+              acc[r][nt][2] = fmaf(s_g8, cacc[r][nt][2], acc[r][nt][2]);
+              acc[r][nt][3] = fmaf(s_g8, cacc[r][nt][3], acc[r][nt][3]);
+            }
           }
         } else {
           uint32_t sc_g = 0, sc_g8 = 0;
@@ -384,13 +418,15 @@ cudaError_t launch_t(const DecodeParams& p, int grid, cudaStream_t st) {
   cfg.blockDim = dim3(KW * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = p.cs;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = p.cs;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = p.cs > 1 ? 1 : 0;
+  cfg.numAttrs = p.cs > 1 ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
