@@ -48,8 +48,6 @@ struct DecodeParams {
   int gshift;     // log2(group size) for INT formats
   int side_rows;  // per row tile: scale groups (INT) or 16-K blocks (NVFP4) staged
   int side_bytes; // bytes of staged scales / zero-points / block scales
-  int xsum_off;   // INT4: per-(token, 32-K chunk) activation sums (fp32)
-  int xsum_cols;  // chunks per token row in that table
   int red_off;    // offset of the cluster partial slots (after the larger of
                   // the staged data and the per-warp partials)
 };
@@ -108,14 +106,6 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "r"(addr));
   return v;
-}
-
-// INT4 fragment without the offset: each bf16 is 128 + u for the stored
-// nibble u; the offset times the chunk's activation sum is removed in fp32
-// when the group is folded.
-__device__ __forceinline__ void frag_int4_raw(uint32_t wd, uint32_t (&a)[4]) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) a[i] = ((wd >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
 }
 
 __device__ __forceinline__ void cluster_arrive_relaxed() {
@@ -244,39 +234,32 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[r][nt][i] = 0.f;
-  // INT group state: chunk accumulator, packed scales, code offsets per row
-  // (128 + z for ASYM; 136 = 128 + 8 for offset-binary signed INT4)
+  // INT group state: chunk accumulator, packed scales, zero-point offsets
+  // (bf16 pairs of 128 + z; 136 = 128 + 8 for offset-binary signed codes)
   float cacc[kIntFmt ? RT : 1][NT][4];
   uint32_t gsw[RT], goff[RT][2];
-  float gxs[NT][2];  // activation sums of the group so far (tokens 2tq, 2tq+1)
   const int gmask = kIntFmt ? (1 << p.gshift) - 1 : 0;
 #pragma unroll
   for (int r = 0; r < RT; ++r) {
     gsw[r] = 0;
-    goff[r][0] = goff[r][1] = 136u;  // 128 + 8 for offset-binary signed codes
+    goff[r][0] = goff[r][1] = 0x43084308u;
   }
 
   cp_async_wait_all();
   __syncthreads();
-  constexpr bool kRawInt4 = FMT == INT4_SYM || FMT == INT4_ASYM;
-  float* xsum = (float*)(smem + p.xsum_off);
-  if constexpr (kRawInt4) {
-    const int nch = (ce - cb) * KB / 32;
-    for (int i = threadIdx.x; i < p.M * nch; i += KW * 32) {
-      const int tok = i / nch, ch = i - tok * nch;
-      const uint32_t base = xs + tok * p.xs_stride + ch * 64;
-      float t = 0.f;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 v = lds128(base + q * 16);
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          t += __uint_as_float(w4[e] << 16);
-          t += __uint_as_float(w4[e] & 0xFFFF0000u);
-        }
-      }
-      xsum[tok * p.xsum_cols + ch] = t;
+  // NVFP4: convert the staged E4M3 block scales once to bf16 (exact), so the
+  // K loop reads a (row g, row g+8) pair with one 32-bit shared load
+  const uint32_t side_bf16 = side + (uint32_t)(RT * p.side_rows * 16);
+  if constexpr (FMT == NVFP4) {
+    const int n16 = RT * ((ce - cb) * KB / 16) * 16;  // staged E4M3 bytes
+    for (int i = threadIdx.x; i < n16; i += KW * 32) {
+      const int rb = i >> 4, e = i & 15;
+      const int r = rb / ((ce - cb) * KB / 16), bi = rb - r * ((ce - cb) * KB / 16);
+      const uint32_t code = lds8(side + (r * p.side_rows + bi) * 16 + e);
+      const uint32_t bits = f32_to_bf16_bits(e4m3_to_f32(code));
+      asm volatile("st.shared.u16 [%0], %1;" ::"r"(side_bf16 + (r * p.side_rows + bi) * 32 + e * 2),
+                   "h"((unsigned short)bits)
+                   : "memory");
     }
     __syncthreads();
   }
@@ -302,19 +285,6 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
       // once when it starts (a warp's range may begin or end inside a group)
       const bool gstart = ((k0 & gmask) == 0) || (k0 == wb * KB);
       const bool gend = (((k0 + 32) & gmask) == 0) || (k0 + 32 == we * KB);
-      if constexpr (kRawInt4) {
-        if (gstart) {
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) gxs[nt][0] = gxs[nt][1] = 0.f;
-        }
-        const int ch = (k0 - kbeg) >> 5;
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const int t0 = 8 * nt + 2 * tq;
-          if (t0 < p.M) gxs[nt][0] += xsum[t0 * p.xsum_cols + ch];
-          if (t0 + 1 < p.M) gxs[nt][1] += xsum[(t0 + 1) * p.xsum_cols + ch];
-        }
-      }
       if constexpr (kIntFmt) {
         if (gstart) {
           const int gi = (k0 >> p.gshift) - g_begin;
@@ -324,8 +294,8 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
             if constexpr (FMT == INT4_ASYM) {
               const uint32_t zb =
                   lds8(side + RT * p.side_rows * 32 + (r * p.side_rows + gi) * 8 + g);
-              goff[r][0] = 128u + (zb & 15u);
-              goff[r][1] = 128u + (zb >> 4);
+              goff[r][0] = (0x4300u + (zb & 15u)) * 0x00010001u;
+              goff[r][1] = (0x4300u + (zb >> 4)) * 0x00010001u;
             }
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
@@ -343,7 +313,7 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
             if constexpr (FMT == INT8_SYM)
               frag_int8(word(wb_[r], 2 * s), word(wb_[r], 2 * s + 1), a);
             else
-              frag_int4_raw(word(wb_[r], 2 * c + s), a);
+              frag_int4(word(wb_[r], 2 * c + s), goff[r][0], goff[r][1], a);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
               mma16816(cacc[r][nt], a, word(xv[c][nt], 2 * s), word(xv[c][nt], 2 * s + 1));
@@ -351,33 +321,21 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
           if (gend) {
             const float s_g = __uint_as_float(gsw[r] << 16);
             const float s_g8 = __uint_as_float(gsw[r] & 0xFFFF0000u);
-            if constexpr (kRawInt4) {
-              // codes entered as 128 + u: subtract offset * sum(x) of the group
-              const float o_g = -(float)goff[r][0], o_g8 = -(float)goff[r][1];
 #pragma unroll
-              for (int nt = 0; nt < NT; ++nt) {
-                acc[r][nt][0] = fmaf(s_g, fmaf(o_g, gxs[nt][0], cacc[r][nt][0]), acc[r][nt][0]);
-                acc[r][nt][1] = fmaf(s_g, fmaf(o_g, gxs[nt][1], cacc[r][nt][1]), acc[r][nt][1]);
-                acc[r][nt][2] = fmaf(s_g8, fmaf(o_g8, gxs[nt][0], cacc[r][nt][2]), acc[r][nt][2]);
-                acc[r][nt][3] = fmaf(s_g8, fmaf(o_g8, gxs[nt][1], cacc[r][nt][3]), acc[r][nt][3]);
-              }
-            } else {
-#pragma unroll
-              for (int nt = 0; nt < NT; ++nt) {
-                acc[r][nt][0] = fmaf(s_g, cacc[r][nt][0], acc[r][nt][0]);
-                acc[r][nt][1] = fmaf(s_g, cacc[r][nt][1], acc[r][nt][1]);
-                acc[r][nt][2] = fmaf(s_g8, cacc[r][nt][2], acc[r][nt][2]);
-                acc[r][nt][3] = fmaf(s_g8, cacc[r][nt][3], acc[r][nt][3]);
-              }
+            for (int nt = 0; nt < NT; ++nt) {
+              acc[r][nt][0] = fmaf(s_g, cacc[r][nt][0], acc[r][nt][0]);
+              acc[r][nt][1] = fmaf(s_g, cacc[r][nt][1], acc[r][nt][1]);
+              acc[r][nt][2] = fmaf(s_g8, cacc[r][nt][2], acc[r][nt][2]);
+              acc[r][nt][3] = fmaf(s_g8, cacc[r][nt][3], acc[r][nt][3]);
             }
           }
         } else {
           uint32_t sc_g = 0, sc_g8 = 0;
           if constexpr (FMT == NVFP4) {
             const int bi = ((k0 + 8 * tq) >> 4) - b16_begin;
-            const uint32_t sb = lds16(side + (r * p.side_rows + bi) * 16 + g * 2);
-            sc_g = f32_to_bf16_bits(e4m3_to_f32(sb & 0xFFu)) * 0x00010001u;
-            sc_g8 = f32_to_bf16_bits(e4m3_to_f32(sb >> 8)) * 0x00010001u;
+            const uint32_t sb = lds32(side_bf16 + (r * p.side_rows + bi) * 32 + g * 4);
+            sc_g = __byte_perm(sb, 0u, 0x1010u);   // (row g, row g) as bf16x2
+            sc_g8 = __byte_perm(sb, 0u, 0x3232u);  // (row g+8, row g+8)
           }
 #pragma unroll
           for (int s = 0; s < 2; ++s) {
@@ -518,21 +476,20 @@ cudaError_t launch_decode(const LinearArgs& a) {
   const int64_t tiles = a.N / 16;
   // more row tiles per CTA when there are more tokens: the staged X slice is
   // then reused across more weight rows
-  int rt = (nt == 2 && tiles % 4 == 0) ? 4 : (tiles % 2 == 0) ? 2 : 1;
+  int rt = (tiles % 2 == 0) ? 2 : 1;
 #ifdef WQ_TUNING
   if (const char* e = getenv("WQ_DECODE_RT")) rt = atoi(e);
 #endif
   const int64_t rowgroups = tiles / rt;
   const int kb = block_k(a.fmt);
   const int64_t nblk = a.K / kb;
-  // split K over a cluster: about four 4-warp CTAs per SM, and a staged X
-  // slice of at most 96 KB
+  // split K over a cluster (a power of two up to 4): about four 4-warp CTAs
+  // per SM, and a staged X slice of at most 96 KB
   const int64_t target = 4LL * device_sm_count();
-  int64_t cs = (target + rowgroups - 1) / rowgroups;
+  int64_t cs = 1;
+  while (cs < 4 && rowgroups * cs < target) cs *= 2;
   const int64_t x_bytes_all = a.M * a.K * 2;
-  const int64_t cs_x = (x_bytes_all + 98303) / 98304;
-  if (cs < cs_x) cs = cs_x;
-  if (cs > 8) cs = 8;
+  while (cs < 8 && (x_bytes_all + cs - 1) / cs > 98304) ++cs;
   if (cs > nblk / 4) cs = nblk / 4;  // keep every warp busy
   if (cs < 1) cs = 1;
 #ifdef WQ_TUNING
@@ -553,18 +510,14 @@ cudaError_t launch_decode(const LinearArgs& a) {
     p.side_bytes = rt * p.side_rows * (a.fmt == INT4_ASYM ? 40 : 32);
   } else if (a.fmt == NVFP4) {
     p.side_rows = (int)(max_blocks * kb / 16);
-    p.side_bytes = rt * p.side_rows * 16;
+    p.side_bytes = rt * p.side_rows * (16 + 32);  // E4M3 bytes, then bf16 copies
   } else {
     p.side_rows = 0;
     p.side_bytes = 0;
   }
   p.side_bytes = (p.side_bytes + 15) & ~15;
-  p.xsum_cols = (int)(max_blocks * kb / 32);
-  p.xsum_off = p.xs_bytes + p.side_bytes;
-  const int64_t xsum_bytes =
-      (a.fmt == INT4_SYM || a.fmt == INT4_ASYM) ? ((a.M * p.xsum_cols * 4 + 15) & ~15LL) : 0;
   const int64_t warp_partials = 4LL * rt * nt * 4 * 32 * 4;  // KW = 4 warps
-  int64_t region = p.xs_bytes + p.side_bytes + xsum_bytes;
+  int64_t region = p.xs_bytes + p.side_bytes;
   if (region < warp_partials) region = warp_partials;
   p.red_off = (int)((region + 15) & ~15LL);
   if (p.red_off + cs * rt * nt * 4 * 32 * 4 > 227 * 1024) return cudaErrorInvalidValue;
