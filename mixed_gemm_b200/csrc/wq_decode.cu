@@ -247,22 +247,6 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
 
   cp_async_wait_all();
   __syncthreads();
-  // NVFP4: convert the staged E4M3 block scales once to bf16 (exact), so the
-  // K loop reads a (row g, row g+8) pair with one 32-bit shared load
-  const uint32_t side_bf16 = side + (uint32_t)(RT * p.side_rows * 16);
-  if constexpr (FMT == NVFP4) {
-    const int n16 = RT * ((ce - cb) * KB / 16) * 16;  // staged E4M3 bytes
-    for (int i = threadIdx.x; i < n16; i += KW * 32) {
-      const int rb = i >> 4, e = i & 15;
-      const int r = rb / ((ce - cb) * KB / 16), bi = rb - r * ((ce - cb) * KB / 16);
-      const uint32_t code = lds8(side + (r * p.side_rows + bi) * 16 + e);
-      const uint32_t bits = f32_to_bf16_bits(e4m3_to_f32(code));
-      asm volatile("st.shared.u16 [%0], %1;" ::"r"(side_bf16 + (r * p.side_rows + bi) * 32 + e * 2),
-                   "h"((unsigned short)bits)
-                   : "memory");
-    }
-    __syncthreads();
-  }
 
   const uint4 zero4 = make_uint4(0, 0, 0, 0);
   auto compute_block = [&](const uint4 (&wb_)[RT], int b) {
@@ -333,9 +317,10 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
           uint32_t sc_g = 0, sc_g8 = 0;
           if constexpr (FMT == NVFP4) {
             const int bi = ((k0 + 8 * tq) >> 4) - b16_begin;
-            const uint32_t sb = lds32(side_bf16 + (r * p.side_rows + bi) * 32 + g * 4);
-            sc_g = __byte_perm(sb, 0u, 0x1010u);   // (row g, row g) as bf16x2
-            sc_g8 = __byte_perm(sb, 0u, 0x3232u);  // (row g+8, row g+8)
+            const uint32_t sb = lds16(side + (r * p.side_rows + bi) * 16 + g * 2);
+            const float v_g = e4m3_bits_to_f32(sb), v_g8 = e4m3_bits_to_f32(sb >> 8);
+            sc_g = pack_bf16x2(v_g, v_g);     // exact: 4 significant bits
+            sc_g8 = pack_bf16x2(v_g8, v_g8);
           }
 #pragma unroll
           for (int s = 0; s < 2; ++s) {
@@ -483,13 +468,14 @@ cudaError_t launch_decode(const LinearArgs& a) {
   const int64_t rowgroups = tiles / rt;
   const int kb = block_k(a.fmt);
   const int64_t nblk = a.K / kb;
-  // split K over a cluster (a power of two up to 4): about four 4-warp CTAs
-  // per SM, and a staged X slice of at most 96 KB
+  // split K over a cluster: about four 4-warp CTAs per SM, and a staged X
+  // slice of at most 96 KB
   const int64_t target = 4LL * device_sm_count();
-  int64_t cs = 1;
-  while (cs < 4 && rowgroups * cs < target) cs *= 2;
+  int64_t cs = (target + rowgroups - 1) / rowgroups;
   const int64_t x_bytes_all = a.M * a.K * 2;
-  while (cs < 8 && (x_bytes_all + cs - 1) / cs > 98304) ++cs;
+  const int64_t cs_x = (x_bytes_all + 98303) / 98304;
+  if (cs < cs_x) cs = cs_x;
+  if (cs > 8) cs = 8;
   if (cs > nblk / 4) cs = nblk / 4;  // keep every warp busy
   if (cs < 1) cs = 1;
 #ifdef WQ_TUNING
@@ -510,7 +496,7 @@ cudaError_t launch_decode(const LinearArgs& a) {
     p.side_bytes = rt * p.side_rows * (a.fmt == INT4_ASYM ? 40 : 32);
   } else if (a.fmt == NVFP4) {
     p.side_rows = (int)(max_blocks * kb / 16);
-    p.side_bytes = rt * p.side_rows * (16 + 32);  // E4M3 bytes, then bf16 copies
+    p.side_bytes = rt * p.side_rows * 16;
   } else {
     p.side_rows = 0;
     p.side_bytes = 0;

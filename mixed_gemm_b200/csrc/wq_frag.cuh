@@ -77,4 +77,16 @@ static __device__ __forceinline__ void frag_table(uint32_t wd, const uint32_t (&
 }
 
 
+// E4M3 (low byte of `b`) -> fp32, exact and branch-free: the 7 magnitude bits
+// placed at fp32 bit 20 read as 2^(e-127)(1 + m/8) (or, for e = 0, the fp32
+// subnormal m * 2^-129), and the power-of-two factor 2^120 moves both to the
+// E4M3 values 2^(e-7)(1 + m/8) and m * 2^-9; the sign bit is copied and the
+// NaN codes (magnitude 0x7F) give NaN.
+static __device__ __forceinline__ float e4m3_bits_to_f32(uint32_t b) {
+  const uint32_t m7 = b & 0x7Fu;
+  const float mag = m7 == 0x7Fu ? __uint_as_float(0x7FC00000u)
+                                : __uint_as_float(m7 << 20) * 0x1p120f;
+  return __uint_as_float(__float_as_uint(mag) | ((b & 0x80u) << 24));
+}
+
 }  // namespace wq

@@ -359,8 +359,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const int64_t b16 = ((int64_t)kt * 64 + 32 * c + 8 * tq) >> 4;
                   const uint32_t sb =
                       __ldg((const uint16_t*)p.scales + (tile * (p.K >> 4) + b16) * 8 + g);
-                  sc_g = f32_to_bf16_bits(e4m3_to_f32(sb & 0xFFu)) * 0x00010001u;
-                  sc_g8 = f32_to_bf16_bits(e4m3_to_f32(sb >> 8)) * 0x00010001u;
+                  const float v_g = e4m3_bits_to_f32(sb), v_g8 = e4m3_bits_to_f32(sb >> 8);
+                  sc_g = pack_bf16x2(v_g, v_g);
+                  sc_g8 = pack_bf16x2(v_g8, v_g8);
                 }
               }
             }
