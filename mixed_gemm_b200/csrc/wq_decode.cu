@@ -7,13 +7,15 @@
 // tensor-core A fragments for that block (layout in wq_internal.cuh), and one
 // 16-byte load of the 8 matching activations per token row.  Codes become
 // bf16 in registers (magic-number nibble conversion for INT4, fp32 magic for
-// INT8, byte-permute table lookups for CB4 and NVFP4) and feed
-// mma.sync.m16n8k16 with the W rows as the 16-row operand and the (<= 16)
-// tokens as the 8-column operand.  INT group scales are applied per 32-K
-// chunk to the fp32 chunk accumulator (so the bf16 fragments are the exact
-// integer codes); NVFP4 block scales are multiplied into the fragments (the
-// product e2m1*e4m3 is exact in bf16); the CB4 row norm and the NVFP4 tensor
-// scale are applied in the epilogue.  Partial sums are reduced across warps
+// INT8, an integer-multiply bit construction for NVFP4, byte-permute table
+// lookups for CB4) and feed mma.sync.m16n8k16 with the W rows as the 16-row
+// operand and the (<= 16) tokens as the 8-column operand.  INT group scales
+// are applied once per group to an fp32 group accumulator (so the bf16
+// fragments are the exact integer codes); NVFP4 block scales are multiplied
+// into the fragments (the product e2m1*e4m3 is exact in bf16); the CB4 row
+// norm and the NVFP4 tensor scale are applied in the epilogue.  The weight
+// stream and its scales are requested before griddepcontrol.wait
+// (programmatic dependent launch); X is staged after it.  Partial sums are reduced across warps
 // through shared memory and across the cluster through distributed shared
 // memory (no global workspace), then rank 0 applies fold + bias, rounds to
 // bf16 and stores.
@@ -211,12 +213,8 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
     }
   }
 
-  // lookup tables (CB4: centroids rounded to bf16; NVFP4: E2M1 values)
+  // lookup table (CB4: centroids rounded to bf16)
   uint32_t H[4] = {0, 0, 0, 0}, L[4] = {0, 0, 0, 0};
-  if constexpr (FMT == NVFP4) {
-    H[0] = 0x3F3F3F00u; H[1] = 0x40404040u; H[2] = 0xBFBFBF80u; H[3] = 0xC0C0C0C0u;
-    L[0] = 0xC0800000u; L[1] = 0xC0804000u; L[2] = L[0]; L[3] = L[1];
-  }
   if constexpr (FMT == CB4) {
     const float* cen = (const float*)p.aux;
 #pragma unroll
@@ -318,20 +316,16 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
           if constexpr (FMT == NVFP4) {
             const int bi = ((k0 + 8 * tq) >> 4) - b16_begin;
             const uint32_t sb = lds16(side + (r * p.side_rows + bi) * 16 + g * 2);
-            const float v_g = e4m3_bits_to_f32(sb), v_g8 = e4m3_bits_to_f32(sb >> 8);
-            sc_g = pack_bf16x2(v_g, v_g);     // exact: 4 significant bits
-            sc_g8 = pack_bf16x2(v_g8, v_g8);
+            sc_g = nvfp4_scale_pair(sb);
+            sc_g8 = nvfp4_scale_pair(sb >> 8);
           }
 #pragma unroll
           for (int s = 0; s < 2; ++s) {
             uint32_t a[4];
-            frag_table<FMT == NVFP4>(word(wb_[r], 2 * c + s), H, L, a);
-            if constexpr (FMT == NVFP4) {
-              a[0] = bmul2(a[0], sc_g);
-              a[1] = bmul2(a[1], sc_g8);
-              a[2] = bmul2(a[2], sc_g);
-              a[3] = bmul2(a[3], sc_g8);
-            }
+            if constexpr (FMT == NVFP4)
+              frag_nvfp4(word(wb_[r], 2 * c + s), sc_g, sc_g8, a);
+            else
+              frag_table<false>(word(wb_[r], 2 * c + s), H, L, a);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
               mma16816(acc[r][nt], a, word(xv[c][nt], 2 * s), word(xv[c][nt], 2 * s + 1));
@@ -383,7 +377,7 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   if (rank != 0) return;
 
   float tsc = 1.f;
-  if constexpr (FMT == NVFP4) tsc = __ldg((const float*)p.aux);
+  if constexpr (FMT == NVFP4) tsc = __ldg((const float*)p.aux) * 128.f;  // 2^7 of frag_nvfp4
   for (int idx = threadIdx.x; idx < NV * 32; idx += KW * 32) {
     float tot = 0.f;
     for (int q = 0; q < cs; ++q) tot += slots[q * NV * 32 + idx];
@@ -474,6 +468,7 @@ cudaError_t launch_decode(const LinearArgs& a) {
   int64_t cs = (target + rowgroups - 1) / rowgroups;
   const int64_t x_bytes_all = a.M * a.K * 2;
   const int64_t cs_x = (x_bytes_all + 98303) / 98304;
+  if (nt == 2 && cs > 4) cs = 4;  // two token tiles: fewer, longer K slices
   if (cs < cs_x) cs = cs_x;
   if (cs > 8) cs = 8;
   if (cs > nblk / 4) cs = nblk / 4;  // keep every warp busy

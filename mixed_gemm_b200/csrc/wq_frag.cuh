@@ -77,6 +77,24 @@ static __device__ __forceinline__ void frag_table(uint32_t wd, const uint32_t (&
 }
 
 
+// NVFP4, "magic" nibble order: fragment i = E2M1 nibbles (i, i+4) times the
+// block scale.  With t = the two nibbles at bits 0..3 and 16..19, the product
+// t * 0x1040 is (t << 6) | (t << 12) (the fields do not overlap), and the mask
+// 0x81C081C0 keeps the magnitude bits at 6..8 and the sign bit at 15 of each
+// half: the bf16 bit pattern of +-e2m1 * 2^-126 (a subnormal for 0.5, zero for
+// 0).  Multiplying by bf16(e4m3 * 2^119) gives e2m1 * e4m3 * 2^-7 exactly (at
+// most 6 significant bits, between 2^-17 and 21); the caller multiplies the
+// result by 2^7 in fp32.  Integer multiply and bf16 multiply issue on the FMA
+// pipe, leaving the ALU pipe two logic operations per register.
+static __device__ __forceinline__ void frag_nvfp4(uint32_t wd, uint32_t sc_g, uint32_t sc_g8,
+                                                  uint32_t (&a)[4]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t t = (wd >> (4 * i)) & 0x000F000Fu;
+    a[i] = bmul2((t * 0x1040u) & 0x81C081C0u, (i & 1) ? sc_g8 : sc_g);
+  }
+}
+
 // E4M3 (low byte of `b`) -> fp32, exact and branch-free: the 7 magnitude bits
 // placed at fp32 bit 20 read as 2^(e-127)(1 + m/8) (or, for e = 0, the fp32
 // subnormal m * 2^-129), and the power-of-two factor 2^120 moves both to the
@@ -87,6 +105,12 @@ static __device__ __forceinline__ float e4m3_bits_to_f32(uint32_t b) {
   const float mag = m7 == 0x7Fu ? __uint_as_float(0x7FC00000u)
                                 : __uint_as_float(m7 << 20) * 0x1p120f;
   return __uint_as_float(__float_as_uint(mag) | ((b & 0x80u) << 24));
+}
+
+// bf16x2 (v, v) with v = e4m3(b) * 2^119 (exact), the factor frag_nvfp4 expects
+static __device__ __forceinline__ uint32_t nvfp4_scale_pair(uint32_t b) {
+  const float v = e4m3_bits_to_f32(b) * 0x1p119f;
+  return pack_bf16x2(v, v);
 }
 
 }  // namespace wq

@@ -14,10 +14,10 @@
 //
 //   4-bit word j = 2c + s holds the 8 nibbles of rows {g, g+8} x K offsets
 //   {e = 0..3}.  Two nibble orders:
-//     "magic" (INT4_SYM, INT4_ASYM):  p = 4*(e&1) + 2*(e>>1) + hr, so that
-//        (word >> 4i) & 0x000F000F yields fragment register i as two nibbles
-//        at bit 0 and bit 16;
-//     "table" (CB4, NVFP4):           p = 4*(e>>1) + 2*hr + (e&1), so that the
+//     "magic" (INT4_SYM, INT4_ASYM, NVFP4):  p = 4*(e&1) + 2*(e>>1) + hr, so
+//        that (word >> 4i) & 0x000F000F yields fragment register i as two
+//        nibbles at bit 0 and bit 16;
+//     "table" (CB4):                  p = 4*(e>>1) + 2*hr + (e&1), so that the
 //        low/high 16 bits hold registers {0,1} / {2,3} as four nibbles each,
 //        ready for byte-permute table lookups.
 //   INT4_SYM nibbles are stored offset-binary (v + 8); INT8 bytes likewise
@@ -56,8 +56,8 @@ __host__ __device__ inline void packed_loc(int f, int64_t n, int64_t k, int64_t 
     int kk = (int)(k & 63), c = kk >> 5, kc = kk & 31, tq = kc >> 3, e8 = kc & 7, s = e8 >> 2,
         e = e8 & 3;
     int lane = 4 * g + tq, j = 2 * c + s;
-    int p = (f == CB4 || f == NVFP4) ? (4 * (e >> 1) + 2 * hr + (e & 1))
-                                     : (4 * (e & 1) + 2 * (e >> 1) + hr);
+    int p = (f == CB4) ? (4 * (e >> 1) + 2 * hr + (e & 1))
+                       : (4 * (e & 1) + 2 * (e >> 1) + hr);
     *byte_off = ((tile * (K >> 6) + b) * 32 + lane) * 16 + j * 4 + (p >> 1);
     *shift = (p & 1) * 4;
   } else {

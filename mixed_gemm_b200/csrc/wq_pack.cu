@@ -59,7 +59,7 @@ __global__ void pack_w_kernel(int f, int64_t N, int64_t K, const uint8_t* __rest
       for (int h = 0; h < 2; ++h) {
         int p = 2 * q + h;
         int hr, e;
-        if (f == CB4 || f == NVFP4) { hr = (p >> 1) & 1; e = (p >> 2) * 2 + (p & 1); }
+        if (f == CB4) { hr = (p >> 1) & 1; e = (p >> 2) * 2 + (p & 1); }
         else { hr = p & 1; e = ((p >> 1) & 1) * 2 + (p >> 2); }
         int64_t n = tile * 16 + g + 8 * hr;
         int64_t k = b * 64 + c * 32 + tq * 8 + s * 4 + e;

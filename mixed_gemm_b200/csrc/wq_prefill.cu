@@ -290,10 +290,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int g = lane >> 2, tq = lane & 3;
     const int64_t groups = kInt ? p.K / p.G : 0;
     uint32_t H[4] = {0, 0, 0, 0}, L[4] = {0, 0, 0, 0};
-    if constexpr (FMT == NVFP4) {
-      H[0] = 0x3F3F3F00u; H[1] = 0x40404040u; H[2] = 0xBFBFBF80u; H[3] = 0xC0C0C0C0u;
-      L[0] = 0xC0800000u; L[1] = 0xC0804000u; L[2] = L[0]; L[3] = L[1];
-    }
     if constexpr (FMT == CB4) {
       const float* cen = (const float*)p.aux;
 #pragma unroll
@@ -352,17 +348,21 @@ __global__ void __launch_bounds__(kThreads, 1)
               frag_int4(w0, off_g, off_g8, a);
               frag_int4(w1, off_g, off_g8, b);
             } else {
-              frag_table<FMT == NVFP4>(w0, H, L, a);
-              frag_table<FMT == NVFP4>(w1, H, L, b);
               if constexpr (FMT == NVFP4) {
                 if (valid) {
                   const int64_t b16 = ((int64_t)kt * 64 + 32 * c + 8 * tq) >> 4;
                   const uint32_t sb =
                       __ldg((const uint16_t*)p.scales + (tile * (p.K >> 4) + b16) * 8 + g);
-                  const float v_g = e4m3_bits_to_f32(sb), v_g8 = e4m3_bits_to_f32(sb >> 8);
-                  sc_g = pack_bf16x2(v_g, v_g);
-                  sc_g8 = pack_bf16x2(v_g8, v_g8);
+                  sc_g = nvfp4_scale_pair(sb);
+                  sc_g8 = nvfp4_scale_pair(sb >> 8);
                 }
+                // the block scale is in the fragments already; stored as they are
+                frag_nvfp4(w0, sc_g, sc_g8, a);
+                frag_nvfp4(w1, sc_g, sc_g8, b);
+                sc_g = sc_g8 = valid ? 0x3F803F80u : 0u;
+              } else {
+                frag_table<false>(w0, H, L, a);
+                frag_table<false>(w1, H, L, b);
               }
             }
             const int j = 4 * c + tq;
@@ -416,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok && nvalid) {
       float post = 1.f, bval = 0.f;
       if constexpr (FMT == CB4) post = bf16_bits_to_f32(__ldg((const uint16_t*)p.scales + n));
-      if constexpr (FMT == NVFP4) post = __ldg((const float*)p.aux);
+      if constexpr (FMT == NVFP4) post = __ldg((const float*)p.aux) * 128.f;  // 2^7 of frag_nvfp4
       if (p.bias) bval = bf16_bits_to_f32(__ldg(p.bias + n));
 #pragma unroll
       for (int j = 0; j < kHalf; ++j) {
