@@ -213,6 +213,16 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
     }
   }
 
+  // NVFP4: a 256-entry table E4M3 code -> bf16x2 (e4m3 * 2^119) pair, the
+  // factor frag_nvfp4 expects, built once per CTA (covered by the barrier
+  // after the staging wait)
+  const uint32_t scale_tab = side + (uint32_t)(RT * p.side_rows * 16);
+  if constexpr (FMT == NVFP4) {
+    for (int c = threadIdx.x; c < 256; c += KW * 32)
+      asm volatile("st.shared.u32 [%0], %1;" ::"r"(scale_tab + c * 4), "r"(nvfp4_scale_pair(c))
+                   : "memory");
+  }
+
   // lookup table (CB4: centroids rounded to bf16)
   uint32_t H[4] = {0, 0, 0, 0}, L[4] = {0, 0, 0, 0};
   if constexpr (FMT == CB4) {
@@ -316,8 +326,8 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
           if constexpr (FMT == NVFP4) {
             const int bi = ((k0 + 8 * tq) >> 4) - b16_begin;
             const uint32_t sb = lds16(side + (r * p.side_rows + bi) * 16 + g * 2);
-            sc_g = nvfp4_scale_pair(sb);
-            sc_g8 = nvfp4_scale_pair(sb >> 8);
+            sc_g = lds32(scale_tab + (sb & 0xFFu) * 4);
+            sc_g8 = lds32(scale_tab + (sb >> 8) * 4);
           }
 #pragma unroll
           for (int s = 0; s < 2; ++s) {
@@ -491,7 +501,7 @@ cudaError_t launch_decode(const LinearArgs& a) {
     p.side_bytes = rt * p.side_rows * (a.fmt == INT4_ASYM ? 40 : 32);
   } else if (a.fmt == NVFP4) {
     p.side_rows = (int)(max_blocks * kb / 16);
-    p.side_bytes = rt * p.side_rows * 16;
+    p.side_bytes = rt * p.side_rows * 16 + 1024;  // block scales + code table
   } else {
     p.side_rows = 0;
     p.side_bytes = 0;
