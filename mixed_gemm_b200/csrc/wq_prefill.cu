@@ -6,13 +6,16 @@
 // are the N side of the MMA (N = 32..256, chosen from M).  Four warpgroups:
 //   warp 0 (one lane)   TMA-loads, per 64-wide K step, the X tile (bf16,
 //                       128-byte swizzle, zero fill past M) and the packed
-//                       tile of 8 row tiles into a ring stage;
-//   warp 1 (one lane)   issues four tcgen05.mma.kind::f16 (K = 16 each) per
-//                       stage and commits the stage back to the producer;
+//                       tile of 8 row tiles into a stage of the TMA ring;
 //   warps 4..7          convert packed codes to bf16 in registers (the decode
-//                       path's fragment decoders) and store them in the
-//                       canonical 128-byte-swizzled K-major layout;
+//                       path's fragment decoders) and store them, in the
+//                       canonical 128-byte-swizzled K-major layout, into a
+//                       stage of a separate ring of A tiles;
+//   warp 1 (one lane)   issues four tcgen05.mma.kind::f16 (K = 16 each) per
+//                       K step and commits both stages back;
 //   warps 8..15         fold and epilogue.
+// With two rings the TMA latency and the dequant time run side by side: a TMA
+// stage is refilled as soon as its X tile and packed tile have been read.
 // INT formats keep the tile values exact: the tile holds the integer code (or
 // code minus zero-point), each group of K is accumulated into its own
 // tensor-memory buffer (two buffers alternate; a group boundary may fall
@@ -55,7 +58,7 @@ struct PrefillParams {
   const uint16_t* bias;
   uint16_t* out;
   int M, N, K, G;
-  int BN, stages;
+  int BN, stages, astages;
   uint32_t tmem_cols;
 };
 
@@ -172,21 +175,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t kWpk = FMT == INT8_SYM ? 8192u : 4096u;  // packed bytes per stage
   constexpr uint32_t kAtile = 16384u;                          // 128 x 64 bf16
   constexpr uint32_t kXbytes = (uint32_t)BN * 128u;
-  constexpr uint32_t kStage = kXbytes + kAtile + kWpk;
+  constexpr uint32_t kTstage = kXbytes + kWpk;  // one TMA stage: X tile + packed tile
   constexpr int kHalf = BN / 2;  // accumulator columns per fold thread
 
+  // Two rings: TMA stages (X tile, packed tile) and dequantized A tiles.  A
+  // TMA stage is released when the MMAs have read its X tile and the dequant
+  // warps have read its packed tile; an A stage when the MMAs have read it.
+  // The TMA latency and the dequant time then overlap instead of adding up.
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  const int S = p.stages;
-  uint64_t* bars = (uint64_t*)(smem + S * kStage);
-  uint32_t* tmem_slot = (uint32_t*)(bars + 3 * S + 5);
+  const int ST = p.stages, SA = p.astages;
+  uint8_t* aring = smem + ST * kTstage;
+  uint64_t* bars = (uint64_t*)(aring + SA * kAtile);
+  uint32_t* tmem_slot = (uint32_t*)(bars + 2 * ST + 2 * SA + 5);
   volatile int* abort = (volatile int*)(tmem_slot + 1);
-  auto full_bar = [&](int s) { return smem_u32(bars + s); };
-  auto dq_bar = [&](int s) { return smem_u32(bars + S + s); };
-  auto empty_bar = [&](int s) { return smem_u32(bars + 2 * S + s); };
-  auto gfull_bar = [&](int b) { return smem_u32(bars + 3 * S + b); };
-  auto gempty_bar = [&](int b) { return smem_u32(bars + 3 * S + 2 + b); };
-  const uint32_t drain_bar = smem_u32(bars + 3 * S + 4);
+  auto tfull_bar = [&](int s) { return smem_u32(bars + s); };
+  auto tempty_bar = [&](int s) { return smem_u32(bars + ST + s); };
+  auto afull_bar = [&](int s) { return smem_u32(bars + 2 * ST + s); };
+  auto aempty_bar = [&](int s) { return smem_u32(bars + 2 * ST + SA + s); };
+  auto gfull_bar = [&](int b) { return smem_u32(bars + 2 * ST + 2 * SA + b); };
+  auto gempty_bar = [&](int b) { return smem_u32(bars + 2 * ST + 2 * SA + 2 + b); };
+  const uint32_t drain_bar = smem_u32(bars + 2 * ST + 2 * SA + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile0 = blockIdx.x * 8;  // first 16-row tile of the CTA's 128 rows
@@ -199,10 +208,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int NG = 4 * KT / KPG;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(dq_bar(s), 4);
-      mbar_init(empty_bar(s), 1);
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(tfull_bar(s), 1);
+      mbar_init(tempty_bar(s), 1 + 4);  // MMA commit + the four dequant warps
+    }
+    for (int s = 0; s < SA; ++s) {
+      mbar_init(afull_bar(s), 4);
+      mbar_init(aempty_bar(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(gfull_bar(b), 1);
@@ -230,19 +242,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------------------------------------------------- producer
       int issued = 0;
       for (int kt = 0; kt < KT; ++kt) {
-        const int s = kt % S;
-        const uint32_t ph = (uint32_t)(kt / S) & 1u;
-        if (kt >= S && !mbar_wait(empty_bar(s), ph ^ 1u, abort, 1u)) break;
-        uint8_t* st = smem + s * kStage;
-        mbar_expect_tx(full_bar(s), kXbytes + kWpk);
-        tma_load_2d(smem_u32(st), &tmX, kt * 64, m0, full_bar(s));
-        tma_load_2d(smem_u32(st + kXbytes + kAtile), &tmW, kt * (int)(kWpk / 32u), tile0,
-                    full_bar(s));
+        const int s = kt % ST;
+        const uint32_t ph = (uint32_t)(kt / ST) & 1u;
+        if (kt >= ST && !mbar_wait(tempty_bar(s), ph ^ 1u, abort, 1u)) break;
+        uint8_t* st = smem + s * kTstage;
+        mbar_expect_tx(tfull_bar(s), kXbytes + kWpk);
+        tma_load_2d(smem_u32(st), &tmX, kt * 64, m0, tfull_bar(s));
+        tma_load_2d(smem_u32(st + kXbytes), &tmW, kt * (int)(kWpk / 32u), tile0, tfull_bar(s));
         ++issued;
       }
       // before teardown, make sure no copy into this CTA's memory is in flight
-      for (int kt = issued - S < 0 ? 0 : issued - S; kt < issued; ++kt)
-        mbar_wait(full_bar(kt % S), (uint32_t)(kt / S) & 1u, abort, 2u);
+      for (int kt = issued - ST < 0 ? 0 : issued - ST; kt < issued; ++kt)
+        mbar_wait(tfull_bar(kt % ST), (uint32_t)(kt / ST) & 1u, abort, 2u);
     } else if (warp == 1 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
@@ -251,13 +262,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       int gb = 0;
       uint32_t d = tmem;
       for (int kt = 0; kt < KT && ok; ++kt) {
-        const int s = kt % S;
-        const uint32_t ph = (uint32_t)(kt / S) & 1u;
-        ok = mbar_wait(full_bar(s), ph, abort, 4u) && mbar_wait(dq_bar(s), ph, abort, 8u);
+        const int s = kt % ST, sa = kt % SA;
+        const uint32_t ph = (uint32_t)(kt / ST) & 1u, pha = (uint32_t)(kt / SA) & 1u;
+        ok = mbar_wait(tfull_bar(s), ph, abort, 4u) && mbar_wait(afull_bar(sa), pha, abort, 8u);
         if (!ok) break;
         tc_fence_after();
-        uint8_t* st = smem + s * kStage;
-        const uint32_t xa = smem_u32(st), aa = smem_u32(st + kXbytes);
+        const uint32_t xa = smem_u32(smem + s * kTstage), aa = smem_u32(aring + sa * kAtile);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const int step = kt * 4 + kk;
@@ -276,7 +286,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                    in_g != 0);
           if (in_g == KPG - 1) umma_commit(gfull_bar(gb));
         }
-        umma_commit(empty_bar(s));
+        umma_commit(tempty_bar(s));
+        umma_commit(aempty_bar(sa));
       }
       if (!ok) {  // wait for this thread's own MMAs before the memory goes away
         umma_commit(drain_bar);
@@ -300,12 +311,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     for (int kt = 0; kt < KT; ++kt) {
-      const int s = kt % S;
-      const uint32_t ph = (uint32_t)(kt / S) & 1u;
-      if (!mbar_wait(full_bar(s), ph, abort, 32u)) break;
-      uint8_t* st = smem + s * kStage;
-      const uint32_t abase = smem_u32(st + kXbytes);
-      const uint8_t* wpk = st + kXbytes + kAtile;
+      const int s = kt % ST, sa = kt % SA;
+      const uint32_t ph = (uint32_t)(kt / ST) & 1u, pha = (uint32_t)(kt / SA) & 1u;
+      if (!mbar_wait(tfull_bar(s), ph, abort, 32u)) break;
+      if (kt >= SA && !mbar_wait(aempty_bar(sa), pha ^ 1u, abort, 32u)) break;
+      const uint32_t abase = smem_u32(aring + sa * kAtile);
+      const uint8_t* wpk = smem + s * kTstage + kXbytes;
 #pragma unroll
       for (int rr = 0; rr < 2; ++rr) {
         const int rt = 2 * dw + rr;
@@ -375,7 +386,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(dq_bar(s));
+      if (lane == 0) {
+        mbar_arrive(afull_bar(sa));   // A tile written
+        mbar_arrive(tempty_bar(s));   // packed tile read (already in registers)
+      }
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 168;\n" ::: "memory");
@@ -478,11 +492,14 @@ cudaError_t launch_bn(const LinearArgs& a) {
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  const uint32_t stage_bytes = (uint32_t)BN * 128u + 16384u + kWpk;
-  int S = (int)((200u * 1024u) / stage_bytes);
-  if (S > 6) S = 6;
-  if (S < 2) S = 2;
-  const size_t smem = (size_t)S * stage_bytes + 1024 + 8 * (3 * S + 5) + 16;
+  // ring depths: three dequantized A tiles; as many TMA stages as fit
+  const uint32_t tstage = (uint32_t)BN * 128u + kWpk;
+  const int SA = 3;
+  const uint32_t budget = 225u * 1024u - (uint32_t)SA * 16384u;
+  int ST = (int)(budget / tstage);
+  if (ST > 8) ST = 8;
+  if (ST < 2) ST = 2;
+  const size_t smem = (size_t)ST * tstage + (size_t)SA * 16384u + 1024 + 8 * (2 * ST + 2 * SA + 5) + 16;
   static std::once_flag attr_once;
   cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [&] {
@@ -500,7 +517,8 @@ cudaError_t launch_bn(const LinearArgs& a) {
   p.K = (int)a.K;
   p.G = a.G;
   p.BN = BN;
-  p.stages = S;
+  p.stages = ST;
+  p.astages = SA;
   const bool groups2 = is_int_fmt(FMT) && (a.K / a.G) > 1;  // two alternating accumulators
   p.tmem_cols = (uint32_t)(groups2 ? 2 * BN : (BN < 32 ? 32 : BN));
   dim3 grid((unsigned)((a.N + 127) / 128), (unsigned)((a.M + BN - 1) / BN));
