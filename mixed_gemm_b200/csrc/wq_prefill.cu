@@ -258,20 +258,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------------------------------------------------- MMA issuer
       const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                              ((128u >> 4) << 24);
+      // descriptors of slot 0 of each ring; a slot / K step is a plain add to
+      // the start-address field (smem addresses stay below 2^18)
+      const uint64_t xdesc0 = umma_desc_sw128(smem_u32(smem));
+      const uint64_t adesc0 = umma_desc_sw128(smem_u32(aring));
       bool ok = true;
-      int gb = 0;
-      uint32_t d = tmem;
+      int s = 0, sa = 0, g = 0, in_g = 0, gb = 0;
+      uint32_t ph = 0, pha = 0, d = tmem;
       for (int kt = 0; kt < KT && ok; ++kt) {
-        const int s = kt % ST, sa = kt % SA;
-        const uint32_t ph = (uint32_t)(kt / ST) & 1u, pha = (uint32_t)(kt / SA) & 1u;
         ok = mbar_wait(tfull_bar(s), ph, abort, 4u) && mbar_wait(afull_bar(sa), pha, abort, 8u);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t xa = smem_u32(smem + s * kTstage), aa = smem_u32(aring + sa * kAtile);
+        const uint64_t xd = xdesc0 + (uint64_t)((uint32_t)s * (kTstage >> 4));
+        const uint64_t ad = adesc0 + (uint64_t)((uint32_t)sa * (kAtile >> 4));
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const int step = kt * 4 + kk;
-          const int g = step / KPG, in_g = step - g * KPG;
           if (in_g == 0) {
             gb = g & 1;
             d = tmem + (uint32_t)(gb * BN);
@@ -282,12 +283,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
           }
-          umma_f16(d, umma_desc_sw128(aa + kk * 32), umma_desc_sw128(xa + kk * 32), idesc,
-                   in_g != 0);
-          if (in_g == KPG - 1) umma_commit(gfull_bar(gb));
+          umma_f16(d, ad + 2 * kk, xd + 2 * kk, idesc, in_g != 0);  // +32 bytes per K step
+          if (++in_g == KPG) {
+            umma_commit(gfull_bar(gb));
+            in_g = 0;
+            ++g;
+          }
         }
         umma_commit(tempty_bar(s));
         umma_commit(aempty_bar(sa));
+        if (++s == ST) { s = 0; ph ^= 1u; }
+        if (++sa == SA) { sa = 0; pha ^= 1u; }
       }
       if (!ok) {  // wait for this thread's own MMAs before the memory goes away
         umma_commit(drain_bar);
