@@ -99,10 +99,10 @@ int wq_packed_sizes(int format, int64_t N, int64_t K, int group_size, size_t* w_
  * as Marlin does, to make GPU dequantization efficient); auto-round-lib
  * README section 1 (repack_quantized_weight).
  * All six buffers are device memory; canonical and packed must not overlap.
- * Checks every NVFP4 block scale (sign clear, not NaN 0x7F) and every NVFP4
- * code (no negative zero 0x8), as the Petit README "Known limitations"
- * requires; that check synchronizes `stream` and returns
- * WQ_ERR_DEVICE_CHECK when it fails.  Other formats do not synchronize. */
+ * A pure permutation: every byte pattern is accepted and round-trips through
+ * wq_unpack.  The Petit README "Known limitations" (positive scales, no
+ * negative-zero FP4 codes) needs no check here, because every E4M3 / E2M1
+ * bit pattern decodes by its definition.  Asynchronous; never synchronizes. */
 int wq_pack(int format, int64_t N, int64_t K, int group_size, const void* codes,
             const void* scales, const void* aux, void* packed_w, void* packed_scales,
             void* packed_aux, void* stream);

@@ -4,9 +4,13 @@
 // The product is computed transposed, D[w_row, token] = W[w_row, :] . X[token, :],
 // so that the dequantized weight tile is the 128-row A operand and the tokens
 // are the N side of the MMA (N = 32..256, chosen from M).  Four warpgroups:
-//   warp 0 (one lane)   TMA-loads, per 64-wide K step, the X tile (bf16,
-//                       128-byte swizzle, zero fill past M) and the packed
-//                       tile of 8 row tiles into a stage of the TMA ring;
+//   warp 0              one lane TMA-loads, per 64-wide K step, the X tile
+//                       (bf16, 128-byte swizzle, zero fill past M) and the
+//                       packed tile of 8 row tiles into a stage of the TMA
+//                       ring; the other lanes copy the stage's NVFP4 block
+//                       scales or zero-points beside it (cp.async completing
+//                       on the same barrier), so the dequant warps never wait
+//                       on global memory;
 //   warps 4..7          convert packed codes to bf16 in registers (the decode
 //                       path's fragment decoders) and store them, in the
 //                       canonical 128-byte-swizzled K-major layout, into a
@@ -99,6 +103,18 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   return false;
 }
 
+// 8- and 16-byte cp.async into shared memory; completion is reported to an
+// mbarrier by cp_async_arrive (one expected arrival per calling thread).
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
                                             uint32_t bar) {
   asm volatile(
@@ -155,10 +171,45 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// 32 consecutive columns: two x16 loads, one wait
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15}, [%16];"
+      : "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]),
+        "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]),
+        "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr + 16u));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
 // byte offset of 16-byte chunk j (K elements 8j..8j+7) of row R in a
 // 128-row x 64-K bf16 tile, 128-byte swizzle, 8-row groups of 1024 bytes
 __device__ __forceinline__ uint32_t swz(int R, int j) {
   return (uint32_t)((R >> 3) * 1024 + (R & 7) * 128 + ((j ^ (R & 7)) << 4));
+}
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds_u8(uint32_t addr) {
+  unsigned short v;
+  asm volatile("ld.shared.u8 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
@@ -176,6 +227,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t kAtile = 16384u;                          // 128 x 64 bf16
   constexpr uint32_t kXbytes = (uint32_t)BN * 128u;
   constexpr uint32_t kTstage = kXbytes + kWpk;  // one TMA stage: X tile + packed tile
+  // per-stage side data (same ring index): NVFP4 block scales of the 8 row
+  // tiles (8 x 64 bytes), ASYM zero-points (8 x up to two 8-byte groups)
+  constexpr uint32_t kSide = FMT == NVFP4 ? 512u : FMT == INT4_ASYM ? 128u : 0u;
+  constexpr bool kHasSide = kSide != 0;
   constexpr int kHalf = BN / 2;  // accumulator columns per fold thread
 
   // Two rings: TMA stages (X tile, packed tile) and dequantized A tiles.  A
@@ -186,7 +241,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int ST = p.stages, SA = p.astages;
   uint8_t* aring = smem + ST * kTstage;
-  uint64_t* bars = (uint64_t*)(aring + SA * kAtile);
+  uint8_t* sring = aring + SA * kAtile;  // side data, kSide bytes per TMA stage
+  uint64_t* bars = (uint64_t*)(sring + ST * kSide);
   uint32_t* tmem_slot = (uint32_t*)(bars + 2 * ST + 2 * SA + 5);
   volatile int* abort = (volatile int*)(tmem_slot + 1);
   auto tfull_bar = [&](int s) { return smem_u32(bars + s); };
@@ -209,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
-      mbar_init(tfull_bar(s), 1);
+      mbar_init(tfull_bar(s), kHasSide ? 1 + 32 : 1);  // + one cp.async arrival per lane
       mbar_init(tempty_bar(s), 1 + 4);  // MMA commit + the four dequant warps
     }
     for (int s = 0; s < SA; ++s) {
@@ -238,17 +294,39 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 56;\n" ::: "memory");
-    if (warp == 0 && lane == 0) {
+    if (warp == 0) {
       // ---------------------------------------------------------- producer
+      const int64_t groups = kInt ? p.K / p.G : 0;
       int issued = 0;
       for (int kt = 0; kt < KT; ++kt) {
         const int s = kt % ST;
         const uint32_t ph = (uint32_t)(kt / ST) & 1u;
         if (kt >= ST && !mbar_wait(tempty_bar(s), ph ^ 1u, abort, 1u)) break;
-        uint8_t* st = smem + s * kTstage;
-        mbar_expect_tx(tfull_bar(s), kXbytes + kWpk);
-        tma_load_2d(smem_u32(st), &tmX, kt * 64, m0, tfull_bar(s));
-        tma_load_2d(smem_u32(st + kXbytes), &tmW, kt * (int)(kWpk / 32u), tile0, tfull_bar(s));
+        if (lane == 0) {
+          uint8_t* st = smem + s * kTstage;
+          mbar_expect_tx(tfull_bar(s), kXbytes + kWpk);
+          tma_load_2d(smem_u32(st), &tmX, kt * 64, m0, tfull_bar(s));
+          tma_load_2d(smem_u32(st + kXbytes), &tmW, kt * (int)(kWpk / 32u), tile0, tfull_bar(s));
+        }
+        if constexpr (kHasSide) {
+          const uint32_t sd = smem_u32(sring + s * kSide);
+          const int rt = lane >> 2, c = lane & 3;  // row tile, 16-byte quarter
+          const int64_t tile = tile0 + rt;
+          if (tile < ntiles) {
+            if constexpr (FMT == NVFP4) {
+              // 4 blocks of 16 K x 16 rows = 64 bytes per row tile
+              cp_async16(sd + rt * 64 + c * 16,
+                         (const uint8_t*)p.scales + (tile * (p.K >> 4) + kt * 4 + c) * 16);
+            } else {
+              // the (one or two) groups of this K step: 8 bytes each
+              const int64_t g0 = ((int64_t)kt * 64) / p.G;
+              const int ng = p.G == 32 ? 2 : 1;
+              if (c < ng)
+                cp_async8(sd + rt * 16 + c * 8, (const uint8_t*)p.aux + (tile * groups + g0 + c) * 8);
+            }
+          }
+          cp_async_arrive(tfull_bar(s));
+        }
         ++issued;
       }
       // before teardown, make sure no copy into this CTA's memory is in flight
@@ -264,9 +342,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t adesc0 = umma_desc_sw128(smem_u32(aring));
       bool ok = true;
       int s = 0, sa = 0, g = 0, in_g = 0, gb = 0;
-      uint32_t ph = 0, pha = 0, d = tmem;
+      uint32_t pha = 0, d = tmem;
       for (int kt = 0; kt < KT && ok; ++kt) {
-        ok = mbar_wait(tfull_bar(s), ph, abort, 4u) && mbar_wait(afull_bar(sa), pha, abort, 8u);
+        // the dequant warps arrive on afull only after they have seen this
+        // stage's tfull, so afull alone orders the X tile too
+        ok = mbar_wait(afull_bar(sa), pha, abort, 8u);
         if (!ok) break;
         tc_fence_after();
         const uint64_t xd = xdesc0 + (uint64_t)((uint32_t)s * (kTstage >> 4));
@@ -292,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         umma_commit(tempty_bar(s));
         umma_commit(aempty_bar(sa));
-        if (++s == ST) { s = 0; ph ^= 1u; }
+        if (++s == ST) s = 0;
         if (++sa == SA) { sa = 0; pha ^= 1u; }
       }
       if (!ok) {  // wait for this thread's own MMAs before the memory goes away
@@ -305,7 +385,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ dequant
     const int dw = warp - 4;  // 0..3
     const int g = lane >> 2, tq = lane & 3;
-    const int64_t groups = kInt ? p.K / p.G : 0;
     uint32_t H[4] = {0, 0, 0, 0}, L[4] = {0, 0, 0, 0};
     if constexpr (FMT == CB4) {
       const float* cen = (const float*)p.aux;
@@ -316,6 +395,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         L[j >> 2] |= (b & 0xFFu) << (8 * (j & 3));
       }
     }
+    // NVFP4: E4M3 code -> bf16x2 pair (e4m3 * 2^119), the factor frag_nvfp4
+    // expects, as a 256-entry table shared by the four dequant warps
+    const uint32_t sctab = smem_u32(bars + 2 * ST + 2 * SA + 8);
+    if constexpr (FMT == NVFP4) {
+      for (int c = threadIdx.x - 128; c < 256; c += 128)
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(sctab + c * 4), "r"(nvfp4_scale_pair(c))
+                     : "memory");
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+    }
     for (int kt = 0; kt < KT; ++kt) {
       const int s = kt % ST, sa = kt % SA;
       const uint32_t ph = (uint32_t)(kt / ST) & 1u, pha = (uint32_t)(kt / SA) & 1u;
@@ -323,26 +411,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (kt >= SA && !mbar_wait(aempty_bar(sa), pha ^ 1u, abort, 32u)) break;
       const uint32_t abase = smem_u32(aring + sa * kAtile);
       const uint8_t* wpk = smem + s * kTstage + kXbytes;
+      const uint32_t sd = smem_u32(sring + s * kSide);
+      // Rows of tiles past N hold zero-filled codes (TMA fill) and stale side
+      // data; their accumulator rows are never stored.
 #pragma unroll
       for (int rr = 0; rr < 2; ++rr) {
         const int rt = 2 * dw + rr;
-        const int64_t tile = tile0 + rt;
-        const bool valid = tile < ntiles;
         const int Rg = rt * 16 + g, Rg8 = Rg + 8;
         if constexpr (FMT == INT8_SYM) {
 #pragma unroll
           for (int blk = 0; blk < 2; ++blk) {
             const uint4 ch = *(const uint4*)(wpk + rt * 1024 + blk * 512 + lane * 16);
             // exact codes; the group scale is applied by the fold warps
-            const uint32_t sc_g = valid ? 0x3F803F80u : 0u, sc_g8 = sc_g;
             uint32_t a[4], b[4];
             frag_int8(ch.x, ch.y, a);
             frag_int8(ch.z, ch.w, b);
             const int j = 4 * blk + tq;
-            st_shared_v4(abase + swz(Rg, j), bmul2(a[0], sc_g), bmul2(a[2], sc_g),
-                         bmul2(b[0], sc_g), bmul2(b[2], sc_g));
-            st_shared_v4(abase + swz(Rg8, j), bmul2(a[1], sc_g8), bmul2(a[3], sc_g8),
-                         bmul2(b[1], sc_g8), bmul2(b[3], sc_g8));
+            st_shared_v4(abase + swz(Rg, j), a[0], a[2], b[0], b[2]);
+            st_shared_v4(abase + swz(Rg8, j), a[1], a[3], b[1], b[3]);
           }
         } else {
           const uint4 ch = *(const uint4*)(wpk + rt * 512 + lane * 16);
@@ -350,43 +436,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 2; ++c) {
             const uint32_t w0 = c ? ch.z : ch.x, w1 = c ? ch.w : ch.y;
             uint32_t a[4], b[4];
-            uint32_t sc_g = valid ? 0x3F803F80u : 0u, sc_g8 = sc_g;
             if constexpr (kInt) {
+              // exact code (minus zero-point); the fold warps apply the scale
               uint32_t off_g = 0x43084308u, off_g8 = 0x43084308u;
-              if (valid) {
-                const int64_t grp = ((int64_t)kt * 64 + 32 * c) / p.G;
-                if constexpr (FMT == INT4_ASYM) {
-                  const uint32_t zb =
-                      __ldg((const uint8_t*)p.aux + (tile * groups + grp) * 8 + g);
-                  off_g = (0x4300u + (zb & 15u)) * 0x00010001u;
-                  off_g8 = (0x4300u + (zb >> 4)) * 0x00010001u;
-                }
+              if constexpr (FMT == INT4_ASYM) {
+                const int dg = p.G == 32 ? c : 0;  // group of this half within the step
+                const uint32_t zb = lds_u8(sd + rt * 16 + dg * 8 + g);
+                off_g = (0x4300u + (zb & 15u)) * 0x00010001u;
+                off_g8 = (0x4300u + (zb >> 4)) * 0x00010001u;
               }
               frag_int4(w0, off_g, off_g8, a);
               frag_int4(w1, off_g, off_g8, b);
+            } else if constexpr (FMT == NVFP4) {
+              // block of 16 K for this lane: 2c + (tq >> 1); rows g, g + 8
+              const uint32_t sb = lds_u16(sd + rt * 64 + (2 * c + (tq >> 1)) * 16 + 2 * g);
+              const uint32_t sc_g = lds_u32(sctab + (sb & 0xFFu) * 4);
+              const uint32_t sc_g8 = lds_u32(sctab + (sb >> 8) * 4);
+              frag_nvfp4(w0, sc_g, sc_g8, a);
+              frag_nvfp4(w1, sc_g, sc_g8, b);
             } else {
-              if constexpr (FMT == NVFP4) {
-                if (valid) {
-                  const int64_t b16 = ((int64_t)kt * 64 + 32 * c + 8 * tq) >> 4;
-                  const uint32_t sb =
-                      __ldg((const uint16_t*)p.scales + (tile * (p.K >> 4) + b16) * 8 + g);
-                  sc_g = nvfp4_scale_pair(sb);
-                  sc_g8 = nvfp4_scale_pair(sb >> 8);
-                }
-                // the block scale is in the fragments already; stored as they are
-                frag_nvfp4(w0, sc_g, sc_g8, a);
-                frag_nvfp4(w1, sc_g, sc_g8, b);
-                sc_g = sc_g8 = valid ? 0x3F803F80u : 0u;
-              } else {
-                frag_table<false>(w0, H, L, a);
-                frag_table<false>(w1, H, L, b);
-              }
+              frag_table<false>(w0, H, L, a);
+              frag_table<false>(w1, H, L, b);
             }
             const int j = 4 * c + tq;
-            st_shared_v4(abase + swz(Rg, j), bmul2(a[0], sc_g), bmul2(a[2], sc_g),
-                         bmul2(b[0], sc_g), bmul2(b[2], sc_g));
-            st_shared_v4(abase + swz(Rg8, j), bmul2(a[1], sc_g8), bmul2(a[3], sc_g8),
-                         bmul2(b[1], sc_g8), bmul2(b[3], sc_g8));
+            st_shared_v4(abase + swz(Rg, j), a[0], a[2], b[0], b[2]);
+            st_shared_v4(abase + swz(Rg8, j), a[1], a[3], b[1], b[3]);
           }
         }
       }
@@ -406,38 +480,57 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t n = (int64_t)tile0 * 16 + row;
     const bool nvalid = n < p.N;
     const int64_t groups = kInt ? p.K / p.G : 0;
+    // per-row factors, requested before the first wait: the group scales of
+    // the next two groups ride in registers ahead of the group being folded
+    const uint16_t* srow = (const uint16_t*)p.scales;
+    int64_t sidx = 0;
+    if (kInt && nvalid) {
+      const int r16 = (int)(n & 15);
+      sidx = (n >> 4) * groups * 16 + 2 * (r16 & 7) + (r16 >> 3);
+    }
+    auto group_scale = [&](int gi) -> uint32_t {
+      return (kInt && nvalid && gi < NG) ? (uint32_t)__ldg(srow + sidx + (int64_t)gi * 16) : 0u;
+    };
+    uint32_t sc0 = group_scale(0), sc1 = group_scale(1);
+    float post = 1.f, bval = 0.f;
+    if (nvalid) {
+      if constexpr (FMT == CB4) post = bf16_bits_to_f32(__ldg((const uint16_t*)p.scales + n));
+      if constexpr (FMT == NVFP4) post = __ldg((const float*)p.aux) * 128.f;  // 2^7 of frag_nvfp4
+      if (p.bias) bval = bf16_bits_to_f32(__ldg(p.bias + n));
+    }
     float acc[kHalf];
 #pragma unroll
     for (int j = 0; j < kHalf; ++j) acc[j] = 0.f;
     bool ok = true;
     for (int g = 0; g < NG; ++g) {
       const int gb = g & 1;
+      const uint32_t sc2 = group_scale(g + 2);
       ok = mbar_wait(gfull_bar(gb), (uint32_t)(g >> 1) & 1u, abort, 64u);
       if (!__all_sync(0xffffffffu, ok ? 1 : 0)) { ok = false; break; }
       tc_fence_after();
-      float sc = 1.f;
-      if (kInt && nvalid) {
-        const int r16 = (int)(n & 15);
-        sc = bf16_bits_to_f32(__ldg((const uint16_t*)p.scales +
-                                    ((n >> 4) * groups + g) * 16 + 2 * (r16 & 7) + (r16 >> 3)));
-      }
+      const float sc = kInt ? bf16_bits_to_f32((uint16_t)sc0) : 1.f;
+      sc0 = sc1;
+      sc1 = sc2;
       const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(gb * BN + hcol);
+      if constexpr (kHalf >= 32) {
 #pragma unroll
-      for (int c = 0; c < kHalf; c += 16) {
+        for (int c = 0; c < kHalf; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(base + (uint32_t)c, v);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) acc[c + j] = fmaf(sc, __uint_as_float(v[j]), acc[c + j]);
+        }
+      } else {
         uint32_t v[16];
-        tmem_ld16(base + (uint32_t)c, v);
+        tmem_ld16(base, v);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) acc[c + j] = fmaf(sc, __uint_as_float(v[j]), acc[c + j]);
+        for (int j = 0; j < 16; ++j) acc[j] = fmaf(sc, __uint_as_float(v[j]), acc[j]);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(gempty_bar(gb));
     }
     if (ok && nvalid) {
-      float post = 1.f, bval = 0.f;
-      if constexpr (FMT == CB4) post = bf16_bits_to_f32(__ldg((const uint16_t*)p.scales + n));
-      if constexpr (FMT == NVFP4) post = __ldg((const float*)p.aux) * 128.f;  // 2^7 of frag_nvfp4
-      if (p.bias) bval = bf16_bits_to_f32(__ldg(p.bias + n));
 #pragma unroll
       for (int j = 0; j < kHalf; ++j) {
         const int m = m0 + hcol + j;
@@ -499,13 +592,15 @@ cudaError_t launch_bn(const LinearArgs& a) {
       return cudaErrorInvalidValue;
   }
   // ring depths: three dequantized A tiles; as many TMA stages as fit
+  const uint32_t side = FMT == NVFP4 ? 512u : FMT == INT4_ASYM ? 128u : 0u;
   const uint32_t tstage = (uint32_t)BN * 128u + kWpk;
   const int SA = 3;
-  const uint32_t budget = 225u * 1024u - (uint32_t)SA * 16384u;
-  int ST = (int)(budget / tstage);
+  const uint32_t fixed = 1024u /* alignment */ + (uint32_t)SA * 16384u + 8u * (2 * 8 + 2 * SA + 8) +
+                         1024u /* NVFP4 scale table */;
+  int ST = (int)((227u * 1024u - fixed) / (tstage + side));
   if (ST > 8) ST = 8;
   if (ST < 2) ST = 2;
-  const size_t smem = (size_t)ST * tstage + (size_t)SA * 16384u + 1024 + 8 * (2 * ST + 2 * SA + 5) + 16;
+  const size_t smem = (size_t)ST * (tstage + side) + fixed;
   static std::once_flag attr_once;
   cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [&] {
