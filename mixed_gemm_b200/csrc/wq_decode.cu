@@ -15,10 +15,11 @@
 // into the fragments (the product e2m1*e4m3 is exact in bf16); the CB4 row
 // norm and the NVFP4 tensor scale are applied in the epilogue.  The weight
 // stream and its scales are requested before griddepcontrol.wait
-// (programmatic dependent launch); X is staged after it.  Partial sums are reduced across warps
-// through shared memory and across the cluster through distributed shared
-// memory (no global workspace), then rank 0 applies fold + bias, rounds to
-// bf16 and stores.
+// (programmatic dependent launch); after it, thread 0 stages the X slice with
+// one bulk copy (cp.async.bulk) per token row onto an mbarrier.  Partial sums
+// are reduced across warps through shared memory and across the cluster
+// through distributed shared memory (no global workspace), then rank 0
+// applies fold + bias, rounds to bf16 and stores.
 //
 // Sources: OrbitQuant card "Benchmark" (skinny batches are decode-bound; the
 // Metal path dispatches a skinny GEMV for up to four rows with decoded weight
@@ -52,19 +53,12 @@ struct DecodeParams {
   int side_bytes; // bytes of staged scales / zero-points / block scales
   int red_off;    // offset of the cluster partial slots (after the larger of
                   // the staged data and the per-warp partials)
+  int bar_off;    // offset of the mbarrier the X-slice bulk copies complete on
 };
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   uint4 v;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
-__device__ __forceinline__ uint4 ld_nc(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
   return v;
@@ -83,6 +77,30 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
 }
 __device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                         uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+// Bounded wait for phase 0 of the X-slice barrier.  The limit is far beyond
+// any copy time; a wait that runs out leaves the block's output unwritten.
+__device__ __forceinline__ bool mbar_wait0(uint32_t bar) {
+  for (uint32_t i = 0; i < (1u << 22); ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar)
+        : "memory");
+    if (ok) return true;
+  }
+  return false;
 }
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
@@ -137,6 +155,11 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   const int cs = p.cs;
   const int rank = (int)(blockIdx.x % (unsigned)cs);
   const int tile0 = (int)(blockIdx.x / (unsigned)cs) * RT;
+  const uint32_t xbar = (uint32_t)__cvta_generic_to_shared(smem) + (uint32_t)p.bar_off;
+  if (threadIdx.x == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(xbar) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
   const int K = p.K;
   const int nblk = K / KB;
   const int groups = kIntFmt ? K >> p.gshift : 0;
@@ -202,15 +225,18 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   // depend on the previous kernel in the stream, so they are requested above
   // before waiting for it; X (typically the previous kernel's output) is read
   // and Y written only after the wait.  The next kernel may be scheduled as
-  // soon as every CTA of this one got here.
+  // soon as every block of this one got here (signalling at kernel entry
+  // instead measured slower: the next kernel's blocks then compete with this
+  // one's compute).  One bulk copy per token row stages the X slice.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  {
-    const int cpr = (ce - cb) * KB / 8;  // 16-byte chunks per token row
-    for (int i = threadIdx.x; i < p.M * cpr; i += KW * 32) {
-      const int tok = i / cpr, c = i - tok * cpr;
-      cp_async16(xs + tok * p.xs_stride + c * 16, p.x + (int64_t)tok * K + kbeg + c * 8);
-    }
+  if (threadIdx.x == 0) {
+    const uint32_t xbytes = (uint32_t)((ce - cb) * KB * 2);
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(xbar),
+                 "r"(xbytes * (uint32_t)p.M)
+                 : "memory");
+    for (int tok = 0; tok < p.M; ++tok)
+      bulk_g2s(xs + tok * p.xs_stride, p.x + (int64_t)tok * K + kbeg, xbytes, xbar);
   }
 
   // NVFP4: a 256-entry table E4M3 code -> bf16x2 (e4m3 * 2^119) pair, the
@@ -235,16 +261,23 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
     }
   }
 
-  float acc[RT][NT][4];
+  // NVFP4 / CB4 with one token tile: the two 16-K steps of a chunk
+  // accumulate into separate chains (NS = 2), so consecutive tensor-core
+  // steps overlap (INT formats already alternate per group; measured faster
+  // with one chain).
+  constexpr int NS = (NT == 1 && !kIntFmt) ? 2 : 1;
+  float acc[NS][RT][NT][4];
 #pragma unroll
-  for (int r = 0; r < RT; ++r)
+  for (int q = 0; q < NS; ++q)
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+    for (int r = 0; r < RT; ++r)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[r][nt][i] = 0.f;
-  // INT group state: chunk accumulator, packed scales, zero-point offsets
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[q][r][nt][i] = 0.f;
+  // INT group state: chunk accumulators, packed scales, zero-point offsets
   // (bf16 pairs of 128 + z; 136 = 128 + 8 for offset-binary signed codes)
-  float cacc[kIntFmt ? RT : 1][NT][4];
+  float cacc[NS][kIntFmt ? RT : 1][NT][4];
   uint32_t gsw[RT], goff[RT][2];
   const int gmask = kIntFmt ? (1 << p.gshift) - 1 : 0;
 #pragma unroll
@@ -254,7 +287,8 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   }
 
   cp_async_wait_all();
-  __syncthreads();
+  __syncthreads();  // staged scales, the NVFP4 table and the barrier init are visible
+  const bool xok = mbar_wait0(xbar);  // false never in practice: then nothing is stored
 
   const uint4 zero4 = make_uint4(0, 0, 0, 0);
   auto compute_block = [&](const uint4 (&wb_)[RT], int b) {
@@ -290,9 +324,11 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
               goff[r][1] = (0x4300u + (zb >> 4)) * 0x00010001u;
             }
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
+            for (int q = 0; q < NS; ++q)
 #pragma unroll
-              for (int i = 0; i < 4; ++i) cacc[r][nt][i] = 0.f;
+              for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) cacc[q][r][nt][i] = 0.f;
           }
         }
       }
@@ -308,17 +344,22 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
               frag_int4(word(wb_[r], 2 * c + s), goff[r][0], goff[r][1], a);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
-              mma16816(cacc[r][nt], a, word(xv[c][nt], 2 * s), word(xv[c][nt], 2 * s + 1));
+              mma16816(cacc[s % NS][r][nt], a, word(xv[c][nt], 2 * s),
+                       word(xv[c][nt], 2 * s + 1));
           }
           if (gend) {
             const float s_g = __uint_as_float(gsw[r] << 16);
             const float s_g8 = __uint_as_float(gsw[r] & 0xFFFF0000u);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-              acc[r][nt][0] = fmaf(s_g, cacc[r][nt][0], acc[r][nt][0]);
-              acc[r][nt][1] = fmaf(s_g, cacc[r][nt][1], acc[r][nt][1]);
-              acc[r][nt][2] = fmaf(s_g8, cacc[r][nt][2], acc[r][nt][2]);
-              acc[r][nt][3] = fmaf(s_g8, cacc[r][nt][3], acc[r][nt][3]);
+              float c4[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                c4[i] = NS == 2 ? cacc[0][r][nt][i] + cacc[NS - 1][r][nt][i] : cacc[0][r][nt][i];
+              acc[0][r][nt][0] = fmaf(s_g, c4[0], acc[0][r][nt][0]);
+              acc[0][r][nt][1] = fmaf(s_g, c4[1], acc[0][r][nt][1]);
+              acc[0][r][nt][2] = fmaf(s_g8, c4[2], acc[0][r][nt][2]);
+              acc[0][r][nt][3] = fmaf(s_g8, c4[3], acc[0][r][nt][3]);
             }
           }
         } else {
@@ -338,7 +379,8 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
               frag_table<false>(word(wb_[r], 2 * c + s), H, L, a);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
-              mma16816(acc[r][nt], a, word(xv[c][nt], 2 * s), word(xv[c][nt], 2 * s + 1));
+              mma16816(acc[s % NS][r][nt], a, word(xv[c][nt], 2 * s),
+                       word(xv[c][nt], 2 * s + 1));
           }
         }
       }
@@ -369,7 +411,9 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) loc[(warp * NV + (r * NT + nt) * 4 + i) * 32 + lane] = acc[r][nt][i];
+      for (int i = 0; i < 4; ++i)
+        loc[(warp * NV + (r * NT + nt) * 4 + i) * 32 + lane] =
+            NS == 2 ? acc[0][r][nt][i] + acc[NS - 1][r][nt][i] : acc[0][r][nt][i];
   __syncthreads();
   float* slots0 = slots;
   if (cs > 1) {
@@ -396,7 +440,7 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
     const int gg = ln >> 2, tt = ln & 3;
     const int n = (tile0 + r) * 16 + gg + 8 * (i >> 1);
     const int m = nt * 8 + 2 * tt + (i & 1);
-    if (m < p.M) {
+    if (m < p.M && xok) {
       float fold = tsc;
       if constexpr (FMT == CB4) fold = bf16_bits_to_f32(__ldg((const uint16_t*)p.scales + n));
       float y = tot * fold;
@@ -410,7 +454,7 @@ template <int FMT, int NT, int RT>
 cudaError_t launch_t(const DecodeParams& p, int grid, cudaStream_t st) {
   constexpr int KW = 4, D = 4;
   auto kern = decode_kernel<FMT, NT, RT, KW, D>;
-  const size_t smem = (size_t)p.red_off + (size_t)p.cs * RT * NT * 4 * 32 * sizeof(float);
+  const size_t smem = (size_t)p.bar_off + 16;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -511,7 +555,8 @@ cudaError_t launch_decode(const LinearArgs& a) {
   int64_t region = p.xs_bytes + p.side_bytes;
   if (region < warp_partials) region = warp_partials;
   p.red_off = (int)((region + 15) & ~15LL);
-  if (p.red_off + cs * rt * nt * 4 * 32 * 4 > 227 * 1024) return cudaErrorInvalidValue;
+  p.bar_off = (int)(p.red_off + cs * rt * nt * 4 * 32 * 4);
+  if (p.bar_off + 16 > 227 * 1024) return cudaErrorInvalidValue;
   const int grid = (int)(rowgroups * cs);
   switch (a.fmt) {
     case INT4_SYM: return launch_fmt<INT4_SYM>(p, nt, rt, grid, a.stream);
