@@ -8,7 +8,8 @@
 // 16-byte load of the 8 matching activations per token row.  Codes become
 // bf16 in registers (magic-number nibble conversion for INT4, fp32 magic for
 // INT8, an integer-multiply bit construction for NVFP4, byte-permute table
-// lookups for CB4) and feed mma.sync.m16n8k16 with the W rows as the 16-row
+// lookups for CB4: a bf16 high part and a bf16 remainder per centroid, two
+// products) and feed mma.sync.m16n8k16 with the W rows as the 16-row
 // operand and the (<= 16) tokens as the 8-column operand.  INT group scales
 // are applied once per group to an fp32 group accumulator (so the bf16
 // fragments are the exact integer codes); NVFP4 block scales are multiplied
@@ -153,8 +154,14 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, tq = lane & 3;
   const int cs = p.cs;
-  const int rank = (int)(blockIdx.x % (unsigned)cs);
-  const int tile0 = (int)(blockIdx.x / (unsigned)cs) * RT;
+  // cluster (cs, 1, 1) over a grid of rowgroups * cs blocks: the cluster
+  // index is the row group, the rank in the cluster the K slice
+  int rank = 0, rgroup = (int)blockIdx.x;
+  if (cs > 1) {
+    asm("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
+    asm("mov.u32 %0, %%clusterid.x;" : "=r"(rgroup));
+  }
+  const int tile0 = rgroup * RT;
   const uint32_t xbar = (uint32_t)__cvta_generic_to_shared(smem) + (uint32_t)p.bar_off;
   if (threadIdx.x == 0) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(xbar) : "memory");
@@ -167,7 +174,8 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   if (cs > 1) cluster_arrive_relaxed();  // matched by the wait before DSMEM writes
 
   // this CTA's K blocks [cb, ce), this warp's [wb, we)
-  const int cb = (int)((int64_t)rank * nblk / cs), ce = (int)((int64_t)(rank + 1) * nblk / cs);
+  const int cb = (int)((unsigned)(rank * nblk) / (unsigned)cs);
+  const int ce = (int)((unsigned)((rank + 1) * nblk) / (unsigned)cs);
   const int wb = cb + warp * (ce - cb) / KW, we = cb + (warp + 1) * (ce - cb) / KW;
   const int nb = we - wb;
 
@@ -184,28 +192,29 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
     if constexpr (kIntFmt) {
       const int ng = ((ce * KB - 1) >> p.gshift) + 1 - g_begin;
       // scales: 32 bytes per (tile, group) -> two 16-byte chunks
-      for (int i = threadIdx.x; i < RT * ng * 2; i += KW * 32) {
-        const int r = i / (ng * 2), rem = i - r * ng * 2, gi = rem >> 1, h = rem & 1;
-        cp_async16(side + (r * p.side_rows + gi) * 32 + h * 16,
-                   (const uint8_t*)p.scales +
-                       ((int64_t)(tile0 + r) * groups + g_begin + gi) * 32 + h * 16);
+#pragma unroll
+      for (int r = 0; r < RT; ++r) {
+        const uint8_t* src = (const uint8_t*)p.scales + ((int64_t)(tile0 + r) * groups + g_begin) * 32;
+        for (int i = threadIdx.x; i < ng * 2; i += KW * 32)
+          cp_async16(side + (r * p.side_rows) * 32 + i * 16, src + i * 16);
       }
       if constexpr (FMT == INT4_ASYM) {
         const uint32_t zs = side + RT * p.side_rows * 32;
-        for (int i = threadIdx.x; i < RT * ng; i += KW * 32) {
-          const int r = i / ng, gi = i - r * ng;
-          cp_async8(zs + (r * p.side_rows + gi) * 8,
-                    (const uint8_t*)p.aux + ((int64_t)(tile0 + r) * groups + g_begin + gi) * 8);
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+          const uint8_t* src = (const uint8_t*)p.aux + ((int64_t)(tile0 + r) * groups + g_begin) * 8;
+          for (int i = threadIdx.x; i < ng; i += KW * 32)
+            cp_async8(zs + (r * p.side_rows + i) * 8, src + i * 8);
         }
       }
     }
     if constexpr (FMT == NVFP4) {
       const int nb16 = (ce - cb) * KB / 16;
-      for (int i = threadIdx.x; i < RT * nb16; i += KW * 32) {
-        const int r = i / nb16, bi = i - r * nb16;
-        cp_async16(side + (r * p.side_rows + bi) * 16,
-                   (const uint8_t*)p.scales +
-                       ((int64_t)(tile0 + r) * (K >> 4) + b16_begin + bi) * 16);
+#pragma unroll
+      for (int r = 0; r < RT; ++r) {
+        const uint8_t* src = (const uint8_t*)p.scales + ((int64_t)(tile0 + r) * (K >> 4) + b16_begin) * 16;
+        for (int i = threadIdx.x; i < nb16; i += KW * 32)
+          cp_async16(side + (r * p.side_rows + i) * 16, src + i * 16);
       }
     }
   }
@@ -249,15 +258,22 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
                    : "memory");
   }
 
-  // lookup table (CB4: centroids rounded to bf16)
+  // lookup tables (CB4): each fp32 centroid as a bf16 high part plus the
+  // bf16 rounding of the remainder (c - hi is exact in fp32), so the two
+  // tensor-core products carry the centroid to within 2^-18 of its value
   uint32_t H[4] = {0, 0, 0, 0}, L[4] = {0, 0, 0, 0};
+  uint32_t H2[4] = {0, 0, 0, 0}, L2[4] = {0, 0, 0, 0};
   if constexpr (FMT == CB4) {
     const float* cen = (const float*)p.aux;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
-      uint32_t b = f32_to_bf16_bits(__ldg(cen + j));
+      const float c = __ldg(cen + j);
+      const uint32_t b = f32_to_bf16_bits(c);
+      const uint32_t b2 = f32_to_bf16_bits(c - bf16_bits_to_f32((uint16_t)b));
       H[j >> 2] |= (b >> 8) << (8 * (j & 3));
       L[j >> 2] |= (b & 0xFFu) << (8 * (j & 3));
+      H2[j >> 2] |= (b2 >> 8) << (8 * (j & 3));
+      L2[j >> 2] |= (b2 & 0xFFu) << (8 * (j & 3));
     }
   }
 
@@ -381,6 +397,13 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
             for (int nt = 0; nt < NT; ++nt)
               mma16816(acc[s % NS][r][nt], a, word(xv[c][nt], 2 * s),
                        word(xv[c][nt], 2 * s + 1));
+            if constexpr (FMT == CB4) {  // the centroids' remainders
+              frag_table<false>(word(wb_[r], 2 * c + s), H2, L2, a);
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt)
+                mma16816(acc[s % NS][r][nt], a, word(xv[c][nt], 2 * s),
+                         word(xv[c][nt], 2 * s + 1));
+            }
           }
         }
       }

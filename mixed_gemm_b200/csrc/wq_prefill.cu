@@ -26,10 +26,13 @@
 // inside a stage for groups of 32), and the fold warps add
 // group_scale[row] * partial into fp32 registers -- the same arithmetic as
 // the decode path, so no bf16 rounding of q*s ever enters the sum.  NVFP4
-// tiles hold e2m1 * e4m3 (exact in bf16); CB4 tiles hold the bf16 centroid.
-// The
+// tiles hold e2m1 * e4m3 (exact in bf16); CB4 uses two tiles, the bf16 high
+// part of each centroid and the bf16 remainder (two MMAs per K step).  The
 // epilogue applies the CB4 row norm / NVFP4 tensor scale and the bias, rounds
-// to bf16 and stores Y.  Registers are rebalanced per warpgroup with
+// to bf16 and stores Y.  When the tiles would fill at most half of the SMs,
+// the K range is split over a thread-block cluster (1, 1, S) and the fp32
+// partial tiles are summed through distributed shared memory before the
+// epilogue.  Registers are rebalanced per warpgroup with
 // setmaxnreg (56 / 104 / 168 / 168 of the 128 per thread launched).  Every
 // mbarrier wait has an iteration limit; a wait that runs out records an error
 // word and the CTA winds down.
@@ -43,6 +46,7 @@
 #include <cudaTypedefs.h>
 
 #include <mutex>
+#include <stdlib.h>
 
 #include "wq_frag.cuh"
 #include "wq_internal.cuh"
@@ -63,6 +67,7 @@ struct PrefillParams {
   uint16_t* out;
   int M, N, K, G;
   int BN, stages, astages;
+  int splits;  // K split over a cluster of this many CTAs (1: no cluster)
   uint32_t tmem_cols;
 };
 
@@ -122,6 +127,22 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(map), "r"(c0), "r"(c1), "r"(bar)
       : "memory");
+}
+
+// Cluster-wide barrier (every thread of every CTA in the cluster), and the
+// distributed-shared-memory address of `addr` in cluster CTA `rank`.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t dsmem_addr(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
 }
 
 // UMMA shared-memory descriptor: K-major, 128-byte swizzle, 8-row groups
@@ -224,7 +245,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const PrefillParams p) {
   constexpr bool kInt = FMT == INT4_SYM || FMT == INT4_ASYM || FMT == INT8_SYM;
   constexpr uint32_t kWpk = FMT == INT8_SYM ? 8192u : 4096u;  // packed bytes per stage
-  constexpr uint32_t kAtile = 16384u;                          // 128 x 64 bf16
+  // A stage: one 128 x 64 bf16 tile; CB4 adds a second tile holding the
+  // bf16 remainders of its centroids (two MMAs per K step)
+  constexpr uint32_t kAsub = FMT == CB4 ? 2u : 1u;
+  constexpr uint32_t kAtile = 16384u * kAsub;
   constexpr uint32_t kXbytes = (uint32_t)BN * 128u;
   constexpr uint32_t kTstage = kXbytes + kWpk;  // one TMA stage: X tile + packed tile
   // per-stage side data (same ring index): NVFP4 block scales of the 8 row
@@ -256,7 +280,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile0 = blockIdx.x * 8;  // first 16-row tile of the CTA's 128 rows
   const int m0 = blockIdx.y * BN;
-  const int KT = p.K / 64;
+  // K split: the S CTAs of a cluster (1, 1, S) share a tile and take
+  // consecutive ranges of KT K steps each (whole scale groups); their fp32
+  // partial tiles are summed through distributed shared memory at the end
+  const int S = p.splits;
+  const int split = S > 1 ? (int)blockIdx.z : 0;
+  const int KT = p.K / 64 / S;
+  const int kt0 = split * KT;  // first K step of this CTA
   const int ntiles = p.N / 16;
   // group-scale fold: exact integer tiles, one accumulator per group of K;
   // groups are counted in 16-wide MMA steps (two groups per stage for G = 32)
@@ -305,8 +335,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
           uint8_t* st = smem + s * kTstage;
           mbar_expect_tx(tfull_bar(s), kXbytes + kWpk);
-          tma_load_2d(smem_u32(st), &tmX, kt * 64, m0, tfull_bar(s));
-          tma_load_2d(smem_u32(st + kXbytes), &tmW, kt * (int)(kWpk / 32u), tile0, tfull_bar(s));
+          tma_load_2d(smem_u32(st), &tmX, (kt0 + kt) * 64, m0, tfull_bar(s));
+          tma_load_2d(smem_u32(st + kXbytes), &tmW, (kt0 + kt) * (int)(kWpk / 32u), tile0,
+                      tfull_bar(s));
         }
         if constexpr (kHasSide) {
           const uint32_t sd = smem_u32(sring + s * kSide);
@@ -316,10 +347,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if constexpr (FMT == NVFP4) {
               // 4 blocks of 16 K x 16 rows = 64 bytes per row tile
               cp_async16(sd + rt * 64 + c * 16,
-                         (const uint8_t*)p.scales + (tile * (p.K >> 4) + kt * 4 + c) * 16);
+                         (const uint8_t*)p.scales + (tile * (p.K >> 4) + (kt0 + kt) * 4 + c) * 16);
             } else {
               // the (one or two) groups of this K step: 8 bytes each
-              const int64_t g0 = ((int64_t)kt * 64) / p.G;
+              const int64_t g0 = ((int64_t)(kt0 + kt) * 64) / p.G;
               const int ng = p.G == 32 ? 2 : 1;
               if (c < ng)
                 cp_async8(sd + rt * 16 + c * 8, (const uint8_t*)p.aux + (tile * groups + g0 + c) * 8);
@@ -364,6 +395,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
           }
           umma_f16(d, ad + 2 * kk, xd + 2 * kk, idesc, in_g != 0);  // +32 bytes per K step
+          if constexpr (FMT == CB4)  // the centroids' remainders, same X columns
+            umma_f16(d, ad + (16384u >> 4) + 2 * kk, xd + 2 * kk, idesc, 1u);
           if (++in_g == KPG) {
             umma_commit(gfull_bar(gb));
             in_g = 0;
@@ -385,14 +418,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ dequant
     const int dw = warp - 4;  // 0..3
     const int g = lane >> 2, tq = lane & 3;
+    // CB4: each fp32 centroid as a bf16 high part (tables H, L) plus the bf16
+    // rounding of the exact remainder (H2, L2)
     uint32_t H[4] = {0, 0, 0, 0}, L[4] = {0, 0, 0, 0};
+    uint32_t H2[4] = {0, 0, 0, 0}, L2[4] = {0, 0, 0, 0};
     if constexpr (FMT == CB4) {
       const float* cen = (const float*)p.aux;
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        uint32_t b = f32_to_bf16_bits(__ldg(cen + j));
+        const float cv = __ldg(cen + j);
+        const uint32_t b = f32_to_bf16_bits(cv);
+        const uint32_t b2 = f32_to_bf16_bits(cv - bf16_bits_to_f32((uint16_t)b));
         H[j >> 2] |= (b >> 8) << (8 * (j & 3));
         L[j >> 2] |= (b & 0xFFu) << (8 * (j & 3));
+        H2[j >> 2] |= (b2 >> 8) << (8 * (j & 3));
+        L2[j >> 2] |= (b2 & 0xFFu) << (8 * (j & 3));
       }
     }
     // NVFP4: E4M3 code -> bf16x2 pair (e4m3 * 2^119), the factor frag_nvfp4
@@ -457,6 +497,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
               frag_table<false>(w0, H, L, a);
               frag_table<false>(w1, H, L, b);
+              uint32_t a2[4], b2[4];  // remainder tile, 16 KB after the high tile
+              frag_table<false>(w0, H2, L2, a2);
+              frag_table<false>(w1, H2, L2, b2);
+              const int j2 = 4 * c + tq;
+              st_shared_v4(abase + 16384u + swz(Rg, j2), a2[0], a2[2], b2[0], b2[2]);
+              st_shared_v4(abase + 16384u + swz(Rg8, j2), a2[1], a2[3], b2[1], b2[3]);
             }
             const int j = 4 * c + tq;
             st_shared_v4(abase + swz(Rg, j), a[0], a[2], b[0], b[2]);
@@ -475,9 +521,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("setmaxnreg.inc.sync.aligned.u32 168;\n" ::: "memory");
     // ------------------------------------------------------------ fold + epilogue
     const int q = warp & 3;            // tensor-memory lane quarter this warp may read
+    const int frow = q * 32 + lane;    // accumulator row
     const int hcol = ((warp - 8) >> 2) * kHalf;
-    const int row = q * 32 + lane;
-    const int64_t n = (int64_t)tile0 * 16 + row;
+    const int64_t n = (int64_t)tile0 * 16 + frow;
     const bool nvalid = n < p.N;
     const int64_t groups = kInt ? p.K / p.G : 0;
     // per-row factors, requested before the first wait: the group scales of
@@ -488,8 +534,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int r16 = (int)(n & 15);
       sidx = (n >> 4) * groups * 16 + 2 * (r16 & 7) + (r16 >> 3);
     }
+    const int gfirst = kInt ? (kt0 * 64) / p.G : 0;  // first group of this CTA's K range
     auto group_scale = [&](int gi) -> uint32_t {
-      return (kInt && nvalid && gi < NG) ? (uint32_t)__ldg(srow + sidx + (int64_t)gi * 16) : 0u;
+      return (kInt && nvalid && gi < NG)
+                 ? (uint32_t)__ldg(srow + sidx + (int64_t)(gfirst + gi) * 16)
+                 : 0u;
     };
     uint32_t sc0 = group_scale(0), sc1 = group_scale(1);
     float post = 1.f, bval = 0.f;
@@ -530,16 +579,55 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(gempty_bar(gb));
     }
-    if (ok && nvalid) {
+    if (S == 1) {
+      if (ok && nvalid) {
 #pragma unroll
-      for (int j = 0; j < kHalf; ++j) {
-        const int m = m0 + hcol + j;
-        if (m < p.M)
-          p.out[(int64_t)m * p.N + n] = (uint16_t)f32_to_bf16_bits(acc[j] * post + bval);
+        for (int j = 0; j < kHalf; ++j) {
+          const int m = m0 + hcol + j;
+          if (m < p.M)
+            p.out[(int64_t)m * p.N + n] = (uint16_t)f32_to_bf16_bits(acc[j] * post + bval);
+        }
+      }
+    } else {
+      // Split-K reduction.  After the first cluster barrier the rings of
+      // every CTA in the cluster are idle (all its roles are done); CTA r
+      // owns columns [r*CW, (r+1)*CW) of the tile and receives every CTA's
+      // fp32 partial of them in slot [source][row][col] of its ring memory;
+      // after the second barrier it adds the slots in source order, folds
+      // and stores.
+      const int CW = BN / S;
+      const uint32_t slots = smem_u32(smem);
+      cluster_sync_all();
+#pragma unroll
+      for (int j = 0; j < kHalf; j += 4) {
+        const int col = hcol + j;
+        const int owner = col / CW;
+        const uint32_t off = (uint32_t)(((split * 128 + frow) * CW + (col - owner * CW)) * 4);
+        st_cluster_v4(dsmem_addr(slots + off, (uint32_t)owner), acc[j], acc[j + 1], acc[j + 2],
+                      acc[j + 3]);
+      }
+      cluster_sync_all();
+      if (ok && nvalid) {
+        // this CTA's CW columns, split between the two fold warpgroups
+        const int half = (warp - 8) >> 2;
+        const float* sl = (const float*)smem;
+        for (int c = half * (CW / 2); c < (half + 1) * (CW / 2); ++c) {
+          float tot = 0.f;
+          for (int src = 0; src < S; ++src) tot += sl[(src * 128 + frow) * CW + c];
+          const int m = m0 + split * CW + c;
+          if (m < p.M)
+            p.out[(int64_t)m * p.N + n] = (uint16_t)f32_to_bf16_bits(tot * post + bval);
+        }
       }
     }
   }
 
+  // the other roles take part in the two cluster barriers of the split-K
+  // reduction once their own work is done
+  if (S > 1 && warp < 8) {
+    cluster_sync_all();
+    cluster_sync_all();
+  }
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
@@ -595,7 +683,8 @@ cudaError_t launch_bn(const LinearArgs& a) {
   const uint32_t side = FMT == NVFP4 ? 512u : FMT == INT4_ASYM ? 128u : 0u;
   const uint32_t tstage = (uint32_t)BN * 128u + kWpk;
   const int SA = 3;
-  const uint32_t fixed = 1024u /* alignment */ + (uint32_t)SA * 16384u + 8u * (2 * 8 + 2 * SA + 8) +
+  const uint32_t fixed = 1024u /* alignment */ + (uint32_t)SA * 16384u * (FMT == CB4 ? 2u : 1u) +
+                         8u * (2 * 8 + 2 * SA + 8) +
                          1024u /* NVFP4 scale table */;
   int ST = (int)((227u * 1024u - fixed) / (tstage + side));
   if (ST > 8) ST = 8;
@@ -620,10 +709,57 @@ cudaError_t launch_bn(const LinearArgs& a) {
   p.BN = BN;
   p.stages = ST;
   p.astages = SA;
+  // K split over a cluster of S CTAs only when the tiles fill at most half
+  // of the SMs: the distributed-shared-memory reduction (every CTA sends
+  // (S-1)/S of a 128 x BN fp32 tile) costs more than a partly empty last wave
+  // (measured: the 24 tiles of a 3072-row layer at M = 256 run 1.4x faster
+  // with S = 4; the 224 or 256 tiles of larger layers run slower with any S).
+  // S is the largest power of two <= 8 with S x tiles <= SMs that splits K
+  // into whole scale groups and leaves each CTA a multiple of 4 columns.
+  {
+    const int64_t tiles = (int64_t)((a.N + 127) / 128) * ((a.M + BN - 1) / BN);
+    const int64_t KTall = a.K / 64;
+    const int64_t unit = (is_int_fmt(FMT) && a.G > 64) ? a.G / 64 : 1;
+    const int64_t sms = device_sm_count();
+    int best_s = 1;
+    if (2 * tiles <= sms) {
+      for (int sp = 8; sp >= 2; sp /= 2) {
+        if (tiles * sp <= sms && KTall % (sp * unit) == 0 && BN % (4 * sp) == 0 && KTall / sp >= 8) {
+          best_s = sp;
+          break;
+        }
+      }
+    }
+#ifdef WQ_TUNING
+    if (const char* e = getenv("WQ_PREFILL_SPLITS")) {
+      const int v = atoi(e);
+      if (v == 1 || ((v == 2 || v == 4 || v == 8) && KTall % (v * unit) == 0 && BN % (4 * v) == 0))
+        best_s = v;
+    }
+#endif
+    p.splits = best_s;
+  }
   const bool groups2 = is_int_fmt(FMT) && (a.K / a.G) > 1;  // two alternating accumulators
   p.tmem_cols = (uint32_t)(groups2 ? 2 * BN : (BN < 32 ? 32 : BN));
-  dim3 grid((unsigned)((a.N + 127) / 128), (unsigned)((a.M + BN - 1) / BN));
-  prefill_kernel<FMT, BN><<<grid, kThreads, smem, a.stream>>>(tmX, tmW, p);
+  dim3 grid((unsigned)((a.N + 127) / 128), (unsigned)((a.M + BN - 1) / BN), (unsigned)p.splits);
+  if (p.splits > 1) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = a.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = (unsigned)p.splits;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_kernel<FMT, BN>, tmX, tmW, p);
+    if (e != cudaSuccess) return e;
+  } else {
+    prefill_kernel<FMT, BN><<<grid, kThreads, smem, a.stream>>>(tmX, tmW, p);
+  }
   return cudaGetLastError();
 }
 

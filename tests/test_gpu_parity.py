@@ -154,3 +154,29 @@ def test_linear_respects_stream(wq, orc):
         wq.wq_linear(x, pw.w, pw.scales, pw.aux, None, 4, N, K, "int4_asym", G, y, s)
     s.synchronize()
     assert np.array_equal(bf16_bits(y), ref)
+
+
+EDGE = [
+    # (N, K, G, Ms): the smallest packed weight (one row tile, one 64-K block);
+    # an odd number of scale groups; a long K whose activation slice forces a
+    # six-block cluster at M = 16
+    (16, 64, 32, (1, 7, 16, 17, 40)),
+    (48, 192, 64, (3, 16, 33, 130)),
+    (32, 16384, 256, (1, 16, 20)),
+]
+
+
+@pytest.mark.parametrize("fmt", ["int4_sym", "int4_asym", "int8_sym", "cb4", "nvfp4"])
+@pytest.mark.parametrize("case", EDGE, ids=["16x64", "48x192", "32x16384"])
+def test_linear_edge_shapes(wq, orc, fmt, case):
+    N, K, G, Ms = case
+    G = 0 if fmt == "cb4" else 16 if fmt == "nvfp4" else G
+    W, (codes, scales, aux) = small_case(orc, fmt, N, K, G, seed=N * 7 + K)
+    pw = pack_on_gpu(wq, fmt, N, K, G, codes, scales, aux)
+    dq = orc.dequant(fmt, codes, scales, aux, N, K, G)
+    xa = synth.activations(41, max(Ms), K)
+    b = synth.bias(41, N)
+    for M in Ms:
+        y = run_linear(wq, pw, xa[:M], b, M)
+        ref, _ = orc.linear(xa[:M], dq, b)
+        check_close(y, ref, f"{fmt} N={N} K={K} M={M}")
