@@ -22,7 +22,7 @@ _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 _lock = threading.Lock()
 _lib = None
 
-FORMATS = {"int4_sym": 0, "int4_asym": 1, "int8_sym": 2, "cb4": 3, "nvfp4": 4}
+FORMATS = {"int4_sym": 0, "int4_asym": 1, "int8_sym": 2, "cb4": 3, "nvfp4": 4, "mxfp4": 5}
 
 
 def build(force: bool = False, extra_flags=(), out_path: str | None = None,
@@ -56,6 +56,8 @@ def _declare(lib):
         "orc_lloyd_max_gaussian": ([c_int, ptr, ptr, ptr, ptr], c_int),
         "orc_quant_cb4": ([ptr, i64, i64, ptr, ptr, ptr], c_int),
         "orc_quant_nvfp4": ([ptr, i64, i64, ptr, ptr, ptr], c_int),
+        "orc_quant_mxfp4": ([ptr, i64, i64, ptr, ptr], c_int),
+        "orc_e8m0_value": ([c_int], dbl),
         "orc_dequant": ([c_int, i64, i64, c_int, ptr, ptr, ptr, ptr], c_int),
         "orc_linear": ([ptr, ptr, ptr, i64, i64, i64, ptr, ptr], c_int),
         "orc_linear_sampled": ([c_int, i64, i64, c_int, ptr, ptr, ptr, ptr, ptr, i64, ptr, ptr,
@@ -121,6 +123,9 @@ class Oracle:
     def e4m3_encode(self, d: float) -> int:
         return int(self.lib.orc_e4m3_encode(d))
 
+    def e8m0_value(self, code: int) -> float:
+        return float(self.lib.orc_e8m0_value(code))
+
     # ---- quantizers -> canonical layout
     def quantize(self, fmt: str, W: np.ndarray, group_size: int = 0, centroids=None):
         """Returns (codes, scales, aux) in the canonical layout of ``fmt``."""
@@ -153,6 +158,11 @@ class Oracle:
             ts = np.zeros((1,), dtype=np.float32)
             _ok(self.lib.orc_quant_nvfp4(_p(W), N, K, _p(codes), _p(bs), _p(ts)), fmt)
             return codes, bs, ts
+        if fmt == "mxfp4":
+            codes = np.zeros((N, K // 2), dtype=np.uint8)
+            bs = np.zeros((N, K // 32), dtype=np.uint8)
+            _ok(self.lib.orc_quant_mxfp4(_p(W), N, K, _p(codes), _p(bs)), fmt)
+            return codes, bs, None
         raise ValueError(fmt)
 
     def lloyd_max(self, levels: int = 16):

@@ -23,6 +23,10 @@
  *    scales, no negative-zero codes.
  *  - NVFP4 itself: E2M1 values, one E4M3 scale per 16 consecutive K
  *    elements, one fp32 tensor scale (format definition).
+ *  - Petit README, "Features": MXFP4 weights beside NVFP4.  MXFP4 itself
+ *    (the OCP microscaling format definition): E2M1 values, one E8M0 scale
+ *    (a power of two, 2^(e-127), e = 255 is NaN) per 32 consecutive K
+ *    elements, no tensor scale.
  *
  * Readings taken where the pages are silent:
  *  - rounding of w/s to an integer: round half to even;
@@ -37,6 +41,12 @@
  *  - NVFP4: ts = fp32(amax / (6*448)), sb = E4M3_rne_satfinite(amax_b /
  *    (6*ts)), q = E2M1_rne_sat(w / (e4m3(sb)*ts)), -0 written as +0,
  *    dq = fp32(e2m1(q) * e4m3(sb) * ts);  the tensor scale multiplies.
+ *  - MXFP4: the microscaling recipe: shared exponent = floor(log2(amax_b))
+ *    - 2 (2 = the largest E2M1 exponent, since 6 = 1.5 * 2^2), clamped to
+ *    [-127, 127]; e = shared exponent + 127; q = E2M1_rne_sat(w / 2^(e-127))
+ *    (|w| / 2^(e-127) in [4, 8) at the block's largest element, so values
+ *    above 6 saturate), -0 written as +0; an all-zero block gets e = 0 and
+ *    codes 0; dq = fp32(e2m1(q) * 2^(e-127)) (exact).
  *  - Lloyd-Max: the 2**bits-level quantizer of N(0,1), computed by the
  *    classical fixed-point iteration (thresholds at midpoints, levels at
  *    conditional means) from a uniform start on [-3, 3], in fp64, then cast
@@ -52,13 +62,15 @@
  *   cb4      : codes u8 [N, K/2] indices; norms bf16 [N]; centroids f32 [16]
  *   nvfp4    : codes u8 [N, K/2] E2M1 nibbles; block scales u8 [N, K/16] E4M3;
  *              tensor scale f32 [1]
+ *   mxfp4    : codes u8 [N, K/2] E2M1 nibbles; block scales u8 [N, K/32] E8M0
  */
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
 
-enum { ORC_INT4_SYM = 0, ORC_INT4_ASYM = 1, ORC_INT8_SYM = 2, ORC_CB4 = 3, ORC_NVFP4 = 4 };
+enum { ORC_INT4_SYM = 0, ORC_INT4_ASYM = 1, ORC_INT8_SYM = 2, ORC_CB4 = 3, ORC_NVFP4 = 4,
+       ORC_MXFP4 = 5 };
 
 /* ------------------------------------------------------------------ bf16 */
 float orc_bf16_to_f32(uint16_t h) {
@@ -344,6 +356,41 @@ int orc_quant_nvfp4(const float* W, int64_t N, int64_t K, uint8_t* codes, uint8_
   return 0;
 }
 
+/* E8M0 (unsigned power-of-two scale): 2^(code - 127); code 255 is NaN. */
+double orc_e8m0_value(int code) {
+  if (code == 255) return NAN;
+  return ldexp(1.0, code - 127);
+}
+
+int orc_quant_mxfp4(const float* W, int64_t N, int64_t K, uint8_t* codes, uint8_t* bscales) {
+  if (N <= 0 || K <= 0 || K % 32) return 1;
+  int64_t nb = K / 32;
+  for (int64_t n = 0; n < N; ++n) {
+    const float* w = W + n * K;
+    uint8_t* row = codes + n * (K / 2);
+    memset(row, 0, (size_t)(K / 2));
+    for (int64_t b = 0; b < nb; ++b) {
+      double ab = 0.0;
+      for (int64_t k = b * 32; k < b * 32 + 32; ++k) ab = fmax(ab, fabs((double)w[k]));
+      int e = 0;
+      if (ab > 0.0) {
+        int ex;
+        frexp(ab, &ex);         /* ab = m * 2^ex, m in [0.5, 1): floor(log2 ab) = ex - 1 */
+        int se = (ex - 1) - 2;  /* minus the largest E2M1 exponent */
+        if (se < -127) se = -127;
+        if (se > 127) se = 127;
+        e = se + 127;
+      }
+      bscales[n * nb + b] = (uint8_t)e;
+      if (ab > 0.0) {
+        double d = orc_e8m0_value(e);
+        for (int64_t k = b * 32; k < b * 32 + 32; ++k) put_nib(row, k, orc_e2m1_encode((double)w[k] / d));
+      }
+    }
+  }
+  return 0;
+}
+
 /* ------------------------------------------------------------- dequant */
 /* Exact dequantized value of element (n, k) from the canonical layout. */
 static float dq_one(int fmt, int64_t K, int G, const void* codes, const void* scales,
@@ -378,17 +425,23 @@ static float dq_one(int fmt, int64_t K, int G, const void* codes, const void* sc
       double ts = (double)((const float*)aux)[0];
       return (float)(orc_e2m1_value(q) * orc_e4m3_value(sb) * ts);
     }
+    case ORC_MXFP4: {
+      int q = get_nib((const uint8_t*)codes + n * (K / 2), k);
+      int e = ((const uint8_t*)scales)[n * (K / 32) + k / 32];
+      return (float)(orc_e2m1_value(q) * orc_e8m0_value(e));
+    }
   }
   return NAN;
 }
 
 static int check_fmt(int fmt, int64_t N, int64_t K, int G) {
   if (N <= 0 || K <= 0) return 1;
-  if (fmt < 0 || fmt > 4) return 1;
+  if (fmt < 0 || fmt > 5) return 1;
   if ((fmt == ORC_INT4_SYM || fmt == ORC_INT4_ASYM || fmt == ORC_INT8_SYM) && (G <= 0 || K % G))
     return 1;
   if (fmt != ORC_INT8_SYM && K % 2) return 1;
   if (fmt == ORC_NVFP4 && K % 16) return 1;
+  if (fmt == ORC_MXFP4 && K % 32) return 1;
   return 0;
 }
 

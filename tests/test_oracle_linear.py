@@ -94,11 +94,16 @@ def _int_case(fmt, N, K, G, rng):
         bs = np.full((N, K // 16), 0x38, np.uint8)         # E4M3 1.0
         ts = np.array([1.0], np.float32)
         return _pack_nibbles(q), bs, ts, E2M1[q]
+    if fmt == "mxfp4":
+        q = rng.integers(0, 16, size=(N, K))
+        q[q == 8] = 0
+        bs = np.full((N, K // 32), 127, np.uint8)          # E8M0 1.0
+        return _pack_nibbles(q), bs, None, E2M1[q]
     raise ValueError(fmt)
 
 
 @pytest.mark.parametrize("fmt,G", [("int4_sym", 64), ("int4_asym", 32), ("int8_sym", 128),
-                                   ("cb4", 0), ("nvfp4", 16)])
+                                   ("cb4", 0), ("nvfp4", 16), ("mxfp4", 32)])
 def test_integer_special_case(orc, fmt, G):
     """Integer X, unit scales: every partial sum is exact, so y equals an
     integer matmul done by numpy -- pins layout, nibble order and orientation."""
@@ -116,7 +121,7 @@ def test_integer_special_case(orc, fmt, G):
 
 
 @pytest.mark.parametrize("fmt,G", [("int4_sym", 64), ("int4_asym", 128), ("int8_sym", 256),
-                                   ("cb4", 0), ("nvfp4", 16)])
+                                   ("cb4", 0), ("nvfp4", 16), ("mxfp4", 32)])
 def test_sampled_equals_full(orc, fmt, G):
     M, N, K = 6, 32, 512
     W = synth.weight(21, N, K, sigma=0.02)

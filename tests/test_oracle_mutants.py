@@ -44,6 +44,10 @@ MUTANTS = [
      "float ts = (float)(amax / (6.0 * 448.0));",
      "float ts = (float)(amax / 448.0);",
      lambda o: quant.test_nvfp4_properties(o)),
+    ("MXFP4 shared exponent without the E2M1 maximum exponent",
+     "int se = (ex - 1) - 2;",
+     "int se = (ex - 1);",
+     lambda o: quant.test_mxfp4_properties(o)),
     ("INT scale divided by qmax+1",
      "uint16_t sb = orc_f64_to_bf16(amax / (double)qmax);",
      "uint16_t sb = orc_f64_to_bf16(amax / (double)(qmax + 1));",

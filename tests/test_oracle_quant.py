@@ -205,3 +205,64 @@ def test_nvfp4_properties(orc):
     gap = np.where(a <= 2, 0.5, np.where(a <= 4, 1.0, 2.0))
     err = np.abs(W.astype(np.float64) - dq_exact) / (sbk * float(ts[0]) + (sbk == 0))
     assert np.all(err[sbk > 0] <= 0.5 * gap[sbk > 0] + 1e-12)
+
+
+# ------------------------------------------------------------------- MXFP4
+def test_e8m0_values(orc):
+    """E8M0: code c is 2^(c - 127); 255 is NaN (format definition)."""
+    import math
+    for c in range(255):
+        assert orc.e8m0_value(c) == math.ldexp(1.0, c - 127)
+    assert math.isnan(orc.e8m0_value(255))
+
+
+def test_mxfp4_properties(orc):
+    """Block scale = 2^(floor(log2 amax) - 2) from an independent frexp; every
+    code within half the E2M1 gap, or saturated at 6 when |w| / scale > 6;
+    exact dequant; no negative zero; all-zero blocks get code 0."""
+    import math
+    N, K = 48, 512
+    W = (0.02 * synth.student5_stream(5, 1, 0, N * K)).astype(np.float32).reshape(N, K)
+    W[3, 64:96] = 0.0                 # an all-zero block
+    W[4, 7] = 3.0e5                   # a block scale far above the others
+    codes, bs, aux = orc.quantize("mxfp4", W)
+    assert aux is None and bs.shape == (N, K // 32)
+    q = _nibbles(codes).astype(np.int64)
+    assert not np.any(q == 8)
+    W64 = W.astype(np.float64)
+    amax = np.abs(W64).reshape(N, K // 32, 32).max(-1)
+    want = np.zeros_like(bs, dtype=np.int64)
+    for (n, b), a in np.ndenumerate(amax):
+        if a > 0:
+            want[n, b] = min(max(math.frexp(a)[1] - 1 - 2, -127), 127) + 127
+    assert np.array_equal(bs.astype(np.int64), want)
+    assert bs[3, 2] == 0 and not np.any(q[3, 64:96])
+    X = np.repeat(np.ldexp(1.0, bs.astype(np.int64) - 127), 32, axis=1)
+    mag = np.array(E2M1)[q & 7]
+    dq_exact = np.where(q & 8, -1.0, 1.0) * mag * X
+    dq = orc.dequant("mxfp4", codes, bs, None, N, K)
+    assert np.array_equal(dq, dq_exact.astype(np.float32))
+    a = np.abs(W64) / X
+    gap = np.where(a <= 2, 0.5, np.where(a <= 4, 1.0, 2.0))
+    err = np.abs(W64 - dq_exact) / X
+    inside = a <= 6.0
+    assert np.all(err[inside] <= 0.5 * gap[inside] + 1e-12)
+    # above 6 the element saturates to +-6 (a block's largest is below 8)
+    assert np.all(a < 8.0)
+    assert np.all(np.abs(dq_exact[~inside]) == 6.0 * X[~inside])
+
+
+def test_mxfp4_round_trip(orc):
+    """Blocks built from E2M1 values times a power of two (each block holding
+    +-6 at its scale) quantize back to the same codes and scale."""
+    rng = np.random.default_rng(11)
+    N, K = 8, 256
+    e = rng.integers(100, 140, size=(N, K // 32))
+    q = rng.integers(0, 16, size=(N, K))
+    q[q == 8] = 0
+    q[:, ::32] = 7                    # +6 in every block
+    X = np.repeat(np.ldexp(1.0, e - 127), 32, axis=1)
+    W = (np.where(q & 8, -1.0, 1.0) * np.array(E2M1)[q & 7] * X).astype(np.float32)
+    codes, bs, _ = orc.quantize("mxfp4", W)
+    assert np.array_equal(bs.astype(np.int64), e)
+    assert np.array_equal(_nibbles(codes).astype(np.int64), q)
