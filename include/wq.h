@@ -10,7 +10,7 @@
  * dequantized weight cache"), of the auto-round-lib README (section 1
  * "Linear": woqgemm over a repacked weight blob, activation [M,K] ->
  * output [M,N], optional bias [1,N]), of the Petit README ("Features": dense
- * FP16/BF16 x NVFP4 GEMM) and of the piper-kernels README ("ConvRot INT8":
+ * FP16/BF16 x NVFP4 / MXFP4 GEMM) and of the piper-kernels README ("ConvRot INT8":
  * group-wise INT8 weight used as a normal linear weight).
  *
  * Conventions shared by every entry point
@@ -25,7 +25,8 @@
  *  - Shapes: N % 16 == 0 and K % 64 == 0 for every format (the packed tile is
  *    16 rows by 64 (4-bit) or 32 (INT8) K elements); INT formats take
  *    group_size in {32, 64, 128, 256} with K % group_size == 0; NVFP4 has a
- *    fixed block of 16 (group_size 16 or 0); CB4 ignores group_size.
+ *    fixed block of 16 (group_size 16 or 0), MXFP4 one of 32 (group_size 32
+ *    or 0); CB4 ignores group_size.
  *  - Every device pointer must be 16-byte aligned, except the NVFP4 tensor
  *    scale and the CB4 centroids (4-byte aligned).
  *
@@ -44,9 +45,14 @@
  *   WQ_NVFP4    : codes  u8 [N, K/2]  E2M1 nibbles, same nibble order
  *                 scales = block scales u8 [N, K/16] (E4M3)
  *                 aux = tensor scale f32 [1]
+ *   WQ_MXFP4    : codes  u8 [N, K/2]  E2M1 nibbles, same nibble order
+ *                 scales = block scales u8 [N, K/32] (E8M0: 2^(e-127),
+ *                 e = 255 is NaN); aux = NULL
  * Dequantized value of element (n, k) -- what wq_dequant returns:
  *   INT4_SYM/INT8_SYM: q * s            ASYM: (q - z) * s          (exact fp32)
  *   CB4: fp32(c[idx] * norm[n])         NVFP4: fp32(e2m1(q) * e4m3(sb) * ts)
+ *   MXFP4: fp32(e2m1(q) * 2^(e-127))    (exact; +-inf where the product
+ *                                          reaches 2^128, NaN for e = 255)
  */
 #ifndef WQ_H_
 #define WQ_H_
@@ -65,7 +71,8 @@ typedef enum {
   WQ_INT4_ASYM = 1, /* asymmetric INT4, bf16 scale + uint4 zero-point per group */
   WQ_INT8_SYM = 2,  /* symmetric INT8, bf16 scale per group                    */
   WQ_CB4 = 3,       /* 4-bit codebook: 16 fp32 centroids, bf16 norm per row    */
-  WQ_NVFP4 = 4      /* E2M1 values, E4M3 scale per 16, fp32 tensor scale       */
+  WQ_NVFP4 = 4,     /* E2M1 values, E4M3 scale per 16, fp32 tensor scale       */
+  WQ_MXFP4 = 5      /* E2M1 values, E8M0 power-of-two scale per 32 (OCP MX)    */
 } wq_format_t;
 
 typedef enum {
@@ -123,9 +130,9 @@ int wq_dequant(int format, int64_t N, int64_t K, int group_size, const void* pac
  *   x        device bf16 [M, K] row-major
  *   packed_w device, from wq_pack
  *   scales   device: INT formats packed group scales; CB4 row norms;
- *            NVFP4 packed E4M3 block scales
+ *            NVFP4 packed E4M3 block scales; MXFP4 packed E8M0 block scales
  *   aux      device: ASYM packed zero-points; CB4 centroids f32[16];
- *            NVFP4 tensor scale f32[1]; NULL for INT4_SYM / INT8_SYM
+ *            NVFP4 tensor scale f32[1]; NULL for INT4_SYM / INT8_SYM / MXFP4
  *   bias     device bf16 [N], or NULL
  *   out      device bf16 [M, N] row-major; must not overlap any input
  * M == 0 is a no-op returning WQ_OK.  Asynchronous; no workspace.

@@ -18,7 +18,7 @@ import os
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libwq.so")
 
-FORMATS = {"int4_sym": 0, "int4_asym": 1, "int8_sym": 2, "cb4": 3, "nvfp4": 4}
+FORMATS = {"int4_sym": 0, "int4_asym": 1, "int8_sym": 2, "cb4": 3, "nvfp4": 4, "mxfp4": 5}
 FORMAT_NAMES = {v: k for k, v in FORMATS.items()}
 
 WQ_OK = 0

@@ -16,7 +16,7 @@ bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p % a) == 0; }
 
 // Shape / format checks shared by every entry point.
 int check_shape(int f, int64_t N, int64_t K, int G) {
-  if (f < INT4_SYM || f > NVFP4) return WQ_ERR_INVALID_ARG;
+  if (f < INT4_SYM || f > MXFP4) return WQ_ERR_INVALID_ARG;
   if (N <= 0 || K <= 0) return WQ_ERR_INVALID_ARG;
   if (N % 16 || K % 64) return WQ_ERR_INVALID_ARG;
   if (N > (1LL << 30) || K > (1LL << 24) || N * K > (1LL << 40)) return WQ_ERR_INVALID_ARG;
@@ -25,11 +25,15 @@ int check_shape(int f, int64_t N, int64_t K, int G) {
     if (K % G) return WQ_ERR_INVALID_ARG;
   } else if (f == NVFP4) {
     if (G != 0 && G != 16) return WQ_ERR_INVALID_ARG;
+  } else if (f == MXFP4) {
+    if (G != 0 && G != 32) return WQ_ERR_INVALID_ARG;
   }
   return WQ_OK;
 }
 
-int effective_group(int f, int G) { return f == NVFP4 ? 16 : (f == CB4 ? 0 : G); }
+int effective_group(int f, int G) {
+  return f == NVFP4 ? 16 : f == MXFP4 ? 32 : (f == CB4 ? 0 : G);
+}
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA; }
 
@@ -82,6 +86,7 @@ int wq_canonical_sizes(int f, int64_t N, int64_t K, int G, size_t* cb, size_t* s
     case INT8_SYM: c = N * K; s = 2 * N * (K / G); break;
     case CB4: c = N * K / 2; s = 2 * N; a = 64; break;
     case NVFP4: c = N * K / 2; s = N * (K / 16); a = 4; break;
+    case MXFP4: c = N * K / 2; s = N * (K / 32); a = 0; break;
   }
   if (cb) *cb = c;
   if (sb) *sb = s;

@@ -208,12 +208,15 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
         }
       }
     }
-    if constexpr (FMT == NVFP4) {
-      const int nb16 = (ce - cb) * KB / 16;
+    if constexpr (FMT == NVFP4 || FMT == MXFP4) {
+      // block scales: one 16-byte entry per (row tile, block of 16 / 32 K)
+      constexpr int LB = FMT == NVFP4 ? 4 : 5;  // log2 of the block
+      const int nbk = ((ce - cb) * KB) >> LB;
 #pragma unroll
       for (int r = 0; r < RT; ++r) {
-        const uint8_t* src = (const uint8_t*)p.scales + ((int64_t)(tile0 + r) * (K >> 4) + b16_begin) * 16;
-        for (int i = threadIdx.x; i < nb16; i += KW * 32)
+        const uint8_t* src = (const uint8_t*)p.scales +
+                             ((int64_t)(tile0 + r) * (K >> LB) + (kbeg >> LB)) * 16;
+        for (int i = threadIdx.x; i < nbk; i += KW * 32)
           cp_async16(side + (r * p.side_rows + i) * 16, src + i * 16);
       }
     }
@@ -252,9 +255,10 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   // factor frag_nvfp4 expects, built once per CTA (covered by the barrier
   // after the staging wait)
   const uint32_t scale_tab = side + (uint32_t)(RT * p.side_rows * 16);
-  if constexpr (FMT == NVFP4) {
+  if constexpr (FMT == NVFP4 || FMT == MXFP4) {
     for (int c = threadIdx.x; c < 256; c += KW * 32)
-      asm volatile("st.shared.u32 [%0], %1;" ::"r"(scale_tab + c * 4), "r"(nvfp4_scale_pair(c))
+      asm volatile("st.shared.u32 [%0], %1;" ::"r"(scale_tab + c * 4),
+                   "r"(FMT == NVFP4 ? nvfp4_scale_pair(c) : mx_lo_pair(c))
                    : "memory");
   }
 
@@ -379,20 +383,38 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
             }
           }
         } else {
-          uint32_t sc_g = 0, sc_g8 = 0;
+          uint32_t sc_g = 0, sc_g8 = 0, eg = 0, eg8 = 0;
           if constexpr (FMT == NVFP4) {
             const int bi = ((k0 + 8 * tq) >> 4) - b16_begin;
             const uint32_t sb = lds16(side + (r * p.side_rows + bi) * 16 + g * 2);
             sc_g = lds32(scale_tab + (sb & 0xFFu) * 4);
             sc_g8 = lds32(scale_tab + (sb >> 8) * 4);
           }
+          if constexpr (FMT == MXFP4) {  // a 32-K chunk is one MXFP4 block
+            const int bi = (k0 >> 5) - (kbeg >> 5);
+            const uint32_t sb = lds16(side + (r * p.side_rows + bi) * 16 + g * 2);
+            eg = sb & 0xFFu;
+            eg8 = sb >> 8;
+            sc_g = lds32(scale_tab + eg * 4);
+            sc_g8 = lds32(scale_tab + eg8 * 4);
+          }
 #pragma unroll
           for (int s = 0; s < 2; ++s) {
             uint32_t a[4];
-            if constexpr (FMT == NVFP4)
+            if constexpr (FMT == NVFP4 || FMT == MXFP4)
               frag_nvfp4(word(wb_[r], 2 * c + s), sc_g, sc_g8, a);
             else
               frag_table<false>(word(wb_[r], 2 * c + s), H, L, a);
+            if constexpr (FMT == MXFP4) {
+              if (eg > 128u && eg != 255u) {
+                a[0] = bmul2(a[0], mx_hi_pair(eg));
+                a[2] = bmul2(a[2], mx_hi_pair(eg));
+              }
+              if (eg8 > 128u && eg8 != 255u) {
+                a[1] = bmul2(a[1], mx_hi_pair(eg8));
+                a[3] = bmul2(a[3], mx_hi_pair(eg8));
+              }
+            }
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
               mma16816(acc[s % NS][r][nt], a, word(xv[c][nt], 2 * s),
@@ -566,8 +588,8 @@ cudaError_t launch_decode(const LinearArgs& a) {
     while ((1 << p.gshift) < a.G) ++p.gshift;
     p.side_rows = (int)((max_blocks * kb + a.G - 1) / a.G + 1);
     p.side_bytes = rt * p.side_rows * (a.fmt == INT4_ASYM ? 40 : 32);
-  } else if (a.fmt == NVFP4) {
-    p.side_rows = (int)(max_blocks * kb / 16);
+  } else if (a.fmt == NVFP4 || a.fmt == MXFP4) {
+    p.side_rows = (int)(max_blocks * kb / (a.fmt == NVFP4 ? 16 : 32));
     p.side_bytes = rt * p.side_rows * 16 + 1024;  // block scales + code table
   } else {
     p.side_rows = 0;
@@ -587,6 +609,7 @@ cudaError_t launch_decode(const LinearArgs& a) {
     case INT8_SYM: return launch_fmt<INT8_SYM>(p, nt, rt, grid, a.stream);
     case CB4: return launch_fmt<CB4>(p, nt, rt, grid, a.stream);
     case NVFP4: return launch_fmt<NVFP4>(p, nt, rt, grid, a.stream);
+    case MXFP4: return launch_fmt<MXFP4>(p, nt, rt, grid, a.stream);
   }
   return cudaErrorInvalidValue;
 }

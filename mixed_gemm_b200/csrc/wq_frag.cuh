@@ -113,4 +113,18 @@ static __device__ __forceinline__ uint32_t nvfp4_scale_pair(uint32_t b) {
   return pack_bf16x2(v, v);
 }
 
+// MXFP4: E8M0 code e -> bf16x2 (s, s), s = 2^(min(e, 128) - 1) (NaN for the
+// NaN code 255).  With frag_nvfp4 (e2m1 * 2^-126 bit patterns) this gives
+// e2m1 * 2^(min(e, 128) - 127) exactly; blocks with e > 128 take one more
+// exact multiply by mx_hi_pair(e) = 2^(e - 128), so that no factor leaves the
+// bf16 range.
+static __device__ __forceinline__ uint32_t mx_lo_pair(uint32_t e) {
+  if (e == 255u) return 0x7FC07FC0u;
+  const uint32_t m = (e < 128u ? e : 128u) + 126u;  // exponent field of 2^(min(e,128) - 1)
+  return (m << 7) * 0x00010001u;
+}
+static __device__ __forceinline__ uint32_t mx_hi_pair(uint32_t e) {
+  return ((e - 128u + 127u) << 7) * 0x00010001u;  // 2^(e - 128), e in 129..254
+}
+
 }  // namespace wq

@@ -14,7 +14,7 @@
 //
 //   4-bit word j = 2c + s holds the 8 nibbles of rows {g, g+8} x K offsets
 //   {e = 0..3}.  Two nibble orders:
-//     "magic" (INT4_SYM, INT4_ASYM, NVFP4):  p = 4*(e&1) + 2*(e>>1) + hr, so
+//     "magic" (INT4_SYM, INT4_ASYM, NVFP4, MXFP4):  p = 4*(e&1) + 2*(e>>1) + hr, so
 //        that (word >> 4i) & 0x000F000F yields fragment register i as two
 //        nibbles at bit 0 and bit 16;
 //     "table" (CB4):                  p = 4*(e>>1) + 2*hr + (e&1), so that the
@@ -27,6 +27,7 @@
 //   reads rows g and g+8 as one 32-bit word).
 // Zero-points (ASYM):    u8 [N/16][K/G][8], byte g = z(row g) | z(row g+8) << 4.
 // NVFP4 block scales:    u8 [N/16][K/16][16], entry 2g + hr.
+// MXFP4 block scales:    u8 [N/16][K/32][16], entry 2g + hr.
 // CB4 norms, CB4 centroids and the NVFP4 tensor scale keep their canonical
 // layout.
 #pragma once
@@ -39,7 +40,7 @@
 
 namespace wq {
 
-enum Fmt { INT4_SYM = 0, INT4_ASYM = 1, INT8_SYM = 2, CB4 = 3, NVFP4 = 4 };
+enum Fmt { INT4_SYM = 0, INT4_ASYM = 1, INT8_SYM = 2, CB4 = 3, NVFP4 = 4, MXFP4 = 5 };
 
 __host__ __device__ inline bool is_int_fmt(int f) { return f == INT4_SYM || f == INT4_ASYM || f == INT8_SYM; }
 __host__ __device__ inline bool is_4bit(int f) { return f != INT8_SYM; }
@@ -95,6 +96,14 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
   else if (e == 0u) v = (float)m * 0.001953125f;  // m * 2^-9
   else v = __uint_as_float(((e + 120u) << 23) | (m << 20));
   return s ? -v : v;
+}
+
+// E8M0 (a power of two, 2^(c - 127)) -> fp32, exact; 255 -> NaN, 0 -> the
+// fp32 subnormal 2^-127.
+__device__ __forceinline__ float e8m0_to_f32(uint32_t c) {
+  if (c == 255u) return __uint_as_float(0x7FC00000u);
+  if (c == 0u) return __uint_as_float(0x00400000u);
+  return __uint_as_float(c << 23);
 }
 
 // ------------------------------------------------------------- launchers

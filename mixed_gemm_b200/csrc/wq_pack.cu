@@ -176,12 +176,16 @@ __global__ void dequant_kernel(int f, int64_t N, int64_t K, int G, const uint8_t
       float c = ((const float*)pa)[raw];
       float nr = bf16_bits_to_f32(((const uint16_t*)ps)[n]);
       v = __fmul_rn(c, nr);
-    } else {  // NVFP4: e2m1 * e4m3 is exact in fp32; one rounding when * ts
+    } else if (f == NVFP4) {  // e2m1 * e4m3 is exact in fp32; one rounding when * ts
       const float mag[8] = {0.f, 0.5f, 1.f, 1.5f, 2.f, 3.f, 4.f, 6.f};
       float e = (raw & 8u) ? -mag[raw & 7u] : mag[raw & 7u];
       float sb = e4m3_to_f32(((const uint8_t*)ps)[packed_scale_idx(n, k >> 4, K >> 4)]);
       float ts = ((const float*)pa)[0];
       v = __fmul_rn(__fmul_rn(e, sb), ts);
+    } else {  // MXFP4: e2m1 * 2^(e - 127), exact (or the fp32 overflow)
+      const float mag[8] = {0.f, 0.5f, 1.f, 1.5f, 2.f, 3.f, 4.f, 6.f};
+      float e = (raw & 8u) ? -mag[raw & 7u] : mag[raw & 7u];
+      v = __fmul_rn(e, e8m0_to_f32(((const uint8_t*)ps)[packed_scale_idx(n, k >> 5, K >> 5)]));
     }
     out[i] = v;
   }
@@ -201,10 +205,11 @@ cudaError_t launch_pack(int f, int64_t N, int64_t K, int G, const void* codes, c
     if (f == INT4_ASYM)
       pack_zeros_kernel<<<grid_for(N * groups / 2), kThreads, 0, st>>>(
           N, groups, (const uint8_t*)aux, (uint8_t*)pa);
-  } else if (f == NVFP4) {
-    permute_scales_kernel<uint8_t><<<grid_for(N * (K / 16)), kThreads, 0, st>>>(
-        N, K / 16, (const uint8_t*)scales, (uint8_t*)ps, true);
-    copy_bytes_kernel<<<1, 32, 0, st>>>((const uint8_t*)aux, (uint8_t*)pa, 4);
+  } else if (f == NVFP4 || f == MXFP4) {
+    const int64_t blk = f == NVFP4 ? 16 : 32;  // K per block scale
+    permute_scales_kernel<uint8_t><<<grid_for(N * (K / blk)), kThreads, 0, st>>>(
+        N, K / blk, (const uint8_t*)scales, (uint8_t*)ps, true);
+    if (f == NVFP4) copy_bytes_kernel<<<1, 32, 0, st>>>((const uint8_t*)aux, (uint8_t*)pa, 4);
   } else {  // CB4: norms and centroids keep their layout
     copy_bytes_kernel<<<grid_for(N * 2), kThreads, 0, st>>>((const uint8_t*)scales,
                                                             (uint8_t*)ps, N * 2);
@@ -225,10 +230,11 @@ cudaError_t launch_unpack(int f, int64_t N, int64_t K, int G, const void* pw, co
     if (f == INT4_ASYM)
       unpack_zeros_kernel<<<grid_for(N * groups), kThreads, 0, st>>>(
           N, groups, (const uint8_t*)pa, (uint8_t*)aux);
-  } else if (f == NVFP4) {
-    permute_scales_kernel<uint8_t><<<grid_for(N * (K / 16)), kThreads, 0, st>>>(
-        N, K / 16, (const uint8_t*)ps, (uint8_t*)scales, false);
-    copy_bytes_kernel<<<1, 32, 0, st>>>((const uint8_t*)pa, (uint8_t*)aux, 4);
+  } else if (f == NVFP4 || f == MXFP4) {
+    const int64_t blk = f == NVFP4 ? 16 : 32;
+    permute_scales_kernel<uint8_t><<<grid_for(N * (K / blk)), kThreads, 0, st>>>(
+        N, K / blk, (const uint8_t*)ps, (uint8_t*)scales, false);
+    if (f == NVFP4) copy_bytes_kernel<<<1, 32, 0, st>>>((const uint8_t*)pa, (uint8_t*)aux, 4);
   } else {
     copy_bytes_kernel<<<grid_for(N * 2), kThreads, 0, st>>>((const uint8_t*)ps,
                                                             (uint8_t*)scales, N * 2);

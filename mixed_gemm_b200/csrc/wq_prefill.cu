@@ -253,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t kTstage = kXbytes + kWpk;  // one TMA stage: X tile + packed tile
   // per-stage side data (same ring index): NVFP4 block scales of the 8 row
   // tiles (8 x 64 bytes), ASYM zero-points (8 x up to two 8-byte groups)
-  constexpr uint32_t kSide = FMT == NVFP4 ? 512u : FMT == INT4_ASYM ? 128u : 0u;
+  constexpr uint32_t kSide = FMT == NVFP4 ? 512u : FMT == MXFP4 ? 256u : FMT == INT4_ASYM ? 128u : 0u;
   constexpr bool kHasSide = kSide != 0;
   constexpr int kHalf = BN / 2;  // accumulator columns per fold thread
 
@@ -348,6 +348,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               // 4 blocks of 16 K x 16 rows = 64 bytes per row tile
               cp_async16(sd + rt * 64 + c * 16,
                          (const uint8_t*)p.scales + (tile * (p.K >> 4) + (kt0 + kt) * 4 + c) * 16);
+            } else if constexpr (FMT == MXFP4) {
+              // 2 blocks of 32 K x 16 rows = 32 bytes per row tile
+              if (c < 2)
+                cp_async16(sd + rt * 32 + c * 16,
+                           (const uint8_t*)p.scales + (tile * (p.K >> 5) + (kt0 + kt) * 2 + c) * 16);
             } else {
               // the (one or two) groups of this K step: 8 bytes each
               const int64_t g0 = ((int64_t)(kt0 + kt) * 64) / p.G;
@@ -438,9 +443,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // NVFP4: E4M3 code -> bf16x2 pair (e4m3 * 2^119), the factor frag_nvfp4
     // expects, as a 256-entry table shared by the four dequant warps
     const uint32_t sctab = smem_u32(bars + 2 * ST + 2 * SA + 8);
-    if constexpr (FMT == NVFP4) {
+    if constexpr (FMT == NVFP4 || FMT == MXFP4) {
       for (int c = threadIdx.x - 128; c < 256; c += 128)
-        asm volatile("st.shared.u32 [%0], %1;" ::"r"(sctab + c * 4), "r"(nvfp4_scale_pair(c))
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(sctab + c * 4),
+                     "r"(FMT == NVFP4 ? nvfp4_scale_pair(c) : mx_lo_pair(c))
                      : "memory");
       asm volatile("bar.sync 1, 128;" ::: "memory");
     }
@@ -494,6 +500,22 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint32_t sc_g8 = lds_u32(sctab + (sb >> 8) * 4);
               frag_nvfp4(w0, sc_g, sc_g8, a);
               frag_nvfp4(w1, sc_g, sc_g8, b);
+            } else if constexpr (FMT == MXFP4) {
+              // one E8M0 block of 32 K per half step; rows g, g + 8
+              const uint32_t sb = lds_u16(sd + rt * 32 + c * 16 + 2 * g);
+              const uint32_t eg = sb & 0xFFu, eg8 = sb >> 8;
+              frag_nvfp4(w0, lds_u32(sctab + eg * 4), lds_u32(sctab + eg8 * 4), a);
+              frag_nvfp4(w1, lds_u32(sctab + eg * 4), lds_u32(sctab + eg8 * 4), b);
+              if (eg > 128u && eg != 255u) {
+                const uint32_t h = mx_hi_pair(eg);
+                a[0] = bmul2(a[0], h); a[2] = bmul2(a[2], h);
+                b[0] = bmul2(b[0], h); b[2] = bmul2(b[2], h);
+              }
+              if (eg8 > 128u && eg8 != 255u) {
+                const uint32_t h = mx_hi_pair(eg8);
+                a[1] = bmul2(a[1], h); a[3] = bmul2(a[3], h);
+                b[1] = bmul2(b[1], h); b[3] = bmul2(b[3], h);
+              }
             } else {
               frag_table<false>(w0, H, L, a);
               frag_table<false>(w1, H, L, b);
@@ -680,12 +702,18 @@ cudaError_t launch_bn(const LinearArgs& a) {
       return cudaErrorInvalidValue;
   }
   // ring depths: three dequantized A tiles; as many TMA stages as fit
-  const uint32_t side = FMT == NVFP4 ? 512u : FMT == INT4_ASYM ? 128u : 0u;
+  const uint32_t side = FMT == NVFP4 ? 512u : FMT == MXFP4 ? 256u : FMT == INT4_ASYM ? 128u : 0u;
   const uint32_t tstage = (uint32_t)BN * 128u + kWpk;
-  const int SA = 3;
+  int SA = 3;
+#ifdef WQ_TUNING
+  if (const char* e = getenv("WQ_PREFILL_SA")) {
+    const int v = atoi(e);
+    if (v >= 2 && v <= 8) SA = v;
+  }
+#endif
   const uint32_t fixed = 1024u /* alignment */ + (uint32_t)SA * 16384u * (FMT == CB4 ? 2u : 1u) +
                          8u * (2 * 8 + 2 * SA + 8) +
-                         1024u /* NVFP4 scale table */;
+                         1024u /* NVFP4 / MXFP4 scale table */;
   int ST = (int)((227u * 1024u - fixed) / (tstage + side));
   if (ST > 8) ST = 8;
   if (ST < 2) ST = 2;
@@ -776,13 +804,20 @@ cudaError_t launch_fmt(const LinearArgs& a, int BN) {
 }  // namespace
 
 cudaError_t launch_prefill(const LinearArgs& a) {
-  const int BN = a.M <= 32 ? 32 : a.M <= 64 ? 64 : a.M <= 128 ? 128 : 256;
+  int BN = a.M <= 32 ? 32 : a.M <= 64 ? 64 : a.M <= 128 ? 128 : 256;
+#ifdef WQ_TUNING
+  if (const char* e = getenv("WQ_PREFILL_BN")) {
+    const int v = atoi(e);
+    if (v == 32 || v == 64 || v == 128 || v == 256) BN = v;
+  }
+#endif
   switch (a.fmt) {
     case INT4_SYM: return launch_fmt<INT4_SYM>(a, BN);
     case INT4_ASYM: return launch_fmt<INT4_ASYM>(a, BN);
     case INT8_SYM: return launch_fmt<INT8_SYM>(a, BN);
     case CB4: return launch_fmt<CB4>(a, BN);
     case NVFP4: return launch_fmt<NVFP4>(a, BN);
+    case MXFP4: return launch_fmt<MXFP4>(a, BN);
   }
   return cudaErrorInvalidValue;
 }

@@ -8,7 +8,8 @@
 // (ConvRotInt8Tensor.from_hp(dense_weight, group_size=256)); the Mamba-2
 // paired-nibble pack helper (scale = amax/qmax, round, clamp to +-qmax);
 // OrbitQuant card "Inputs" (row norms, Lloyd-Max centroids); Petit README
-// "Features" (NVFP4) and "Known limitations" (positive scales, no -0 codes).
+// "Features" (NVFP4, MXFP4) and "Known limitations" (positive scales, no -0
+// codes).
 #include "wq_internal.cuh"
 
 namespace wq {
@@ -231,6 +232,34 @@ __global__ void nvfp4_code_kernel(int64_t N, int64_t K, const float* __restrict_
   }
 }
 
+// MXFP4: one warp per 32-element block (one lane per element).  The block
+// exponent is floor(log2 amax) - 2 (frexp, exact), clamped to [-127, 127];
+// codes are the nearest E2M1 (ties to even, saturating at 6) of w / 2^exp,
+// the division exact; an all-zero block gets exponent code 0.
+__global__ void mxfp4_code_kernel(int64_t N, int64_t K, const float* __restrict__ w,
+                                  uint8_t* __restrict__ codes, uint8_t* __restrict__ bscales) {
+  const int64_t blocks = N * (K / 32);
+  const int lane = threadIdx.x & 31;
+  for (int64_t b = blockIdx.x * (int64_t)kWarps + (threadIdx.x >> 5); b < blocks;
+       b += (int64_t)gridDim.x * kWarps) {
+    const float v = w[b * 32 + lane];
+    double ab = fabs((double)v);
+    for (int o = 16; o; o >>= 1) ab = fmax(ab, __shfl_xor_sync(0xffffffffu, ab, o));
+    uint32_t e = 0, q = 0;
+    if (ab > 0.0) {
+      int ex;
+      frexp(ab, &ex);
+      int se = (ex - 1) - 2;
+      se = se < -127 ? -127 : (se > 127 ? 127 : se);
+      e = (uint32_t)(se + 127);
+      q = e2m1_encode_rn_sat(ldexp((double)v, -se));
+    }
+    const uint32_t q_hi = __shfl_down_sync(0xffffffffu, q, 1);
+    if ((lane & 1) == 0) codes[b * 16 + lane / 2] = (uint8_t)(q | (q_hi << 4));
+    if (lane == 0) bscales[b] = (uint8_t)e;
+  }
+}
+
 __global__ void nvfp4_tscale_kernel(float* slot) {
   double amax = (double)__uint_as_float(*(const unsigned int*)slot);
   *slot = __double2float_rn(__ddiv_rn(amax, 6.0 * 448.0));
@@ -271,6 +300,10 @@ cudaError_t launch_quantize(int f, int64_t N, int64_t K, int G, const float* w, 
       nvfp4_tscale_kernel<<<1, 1, 0, st>>>((float*)aux);
       break;
     }
+    case MXFP4:
+      mxfp4_code_kernel<<<blocks_for(N * (K / 32), kWarps), kWarps * 32, 0, st>>>(
+          N, K, w, (uint8_t*)codes, (uint8_t*)scales);
+      break;
     default:
       return cudaErrorInvalidValue;
   }

@@ -1,11 +1,12 @@
-"""The five synthetic workloads of the weight-only quantized linear.
+"""The six synthetic workloads of the weight-only quantized linear.
 
 Each recipe fixes shapes, the weight format, the group size, the seed and the
 value distributions; ``make_inputs`` draws the dense inputs for one of them.
-Format names are the library's: int4_sym, int4_asym, int8_sym, cb4, nvfp4.
+Format names are the library's: int4_sym, int4_asym, int8_sym, cb4, nvfp4, mxfp4.
 
 Readings (the recipe texts leave these open):
-  * seeds other than the first workload's are 1, 2, 3, 4 in order;
+  * seeds other than the first workload's are 1, 2, 3, 4 in order, and 5
+    for the MXFP4 twin of the NVFP4 shape (same layer, same distribution);
   * "0.1% of entries replaced by x20 outliers" = round(0.001*N*K) distinct
     positions whose drawn value is multiplied by 20;
   * "1% of channels scaled x10" = round(0.01*K) distinct input columns of X
@@ -59,11 +60,14 @@ CODEBOOK = Workload("codebook4_3072", "cb4", N=3072, K=3072, Ms=(1, 16, 256), gr
 NVFP4 = Workload("nvfp4_28672x8192", "nvfp4", N=28672, K=8192, Ms=(1, 8, 64, 256),
                  group_size=16, seed=3, w_dist="student5",
                  note="NVFP4 70B-class MLP up-projection shape")
+MXFP4 = Workload("mxfp4_28672x8192", "mxfp4", N=28672, K=8192, Ms=(1, 8, 64, 256),
+                 group_size=32, seed=5, w_dist="student5",
+                 note="MXFP4 (E8M0 scale per 32) on the NVFP4 layer shape")
 PREFILL = Workload("prefill_int8_g256", "int8_sym", N=8192, K=8192, Ms=(1024, 2048, 4096),
                    group_size=256, seed=4, x_channel_frac=0.01, x_channel_mult=10.0,
                    bias_sigma=0.01, note="compute-bound prefill, INT8 sym g256")
 
-ALL = (PR1, DECODE, CODEBOOK, NVFP4, PREFILL)
+ALL = (PR1, DECODE, CODEBOOK, NVFP4, PREFILL, MXFP4)
 BY_NAME = {w.name: w for w in ALL}
 
 
@@ -104,6 +108,8 @@ def packed_bytes(fmt: str, N: int, K: int, G: int) -> int:
         return N * K // 2 + 2 * N + 64
     if fmt == "nvfp4":
         return N * K // 2 + N * (K // 16) + 4
+    if fmt == "mxfp4":
+        return N * K // 2 + N * (K // 32)
     raise ValueError(fmt)
 
 

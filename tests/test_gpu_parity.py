@@ -7,6 +7,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
 from gpu_cases import (bf16_bits, check_close, dev_bf16, dev_u8, pack_on_gpu, run_linear,
                        small_case)
@@ -15,7 +16,7 @@ pytestmark = pytest.mark.gpu
 
 FMT_G = [("int4_sym", 32), ("int4_sym", 64), ("int4_sym", 128), ("int4_sym", 256),
          ("int4_asym", 32), ("int4_asym", 128), ("int8_sym", 32), ("int8_sym", 256),
-         ("cb4", 0), ("nvfp4", 16)]
+         ("cb4", 0), ("nvfp4", 16), ("mxfp4", 32)]
 IDS = [f"{f}-g{g}" for f, g in FMT_G]
 
 
@@ -56,7 +57,7 @@ def test_dequant_bit_exact(wq, orc, fmt, G):
 @pytest.mark.parametrize("fmt,G", FMT_G, ids=IDS)
 def test_gpu_quantizer_matches_oracle(wq, orc, fmt, G):
     N, K = 96, 1024
-    W = synth.weight(17, N, K, dist="student5" if fmt == "nvfp4" else "normal", sigma=0.02,
+    W = synth.weight(17, N, K, dist="student5" if fmt in ("nvfp4", "mxfp4") else "normal", sigma=0.02,
                      outlier_count=100, outlier_mult=20.0)
     W[7, :] = 0.0
     W[9, 64:192] = 0.0
@@ -103,7 +104,7 @@ def _int_case(fmt, N, K, G, rng):
 
 
 @pytest.mark.parametrize("fmt,G", [("int4_sym", 64), ("int4_asym", 32), ("int8_sym", 128),
-                                   ("cb4", 0), ("nvfp4", 16)])
+                                   ("cb4", 0), ("nvfp4", 16), ("mxfp4", 32)])
 @pytest.mark.parametrize("M", [1, 5, 16, 40, 200])
 def test_linear_integer_bit_exact(wq, orc, fmt, G, M):
     """Integer activations and unit scales: every partial sum is exact in
@@ -166,11 +167,11 @@ EDGE = [
 ]
 
 
-@pytest.mark.parametrize("fmt", ["int4_sym", "int4_asym", "int8_sym", "cb4", "nvfp4"])
+@pytest.mark.parametrize("fmt", ["int4_sym", "int4_asym", "int8_sym", "cb4", "nvfp4", "mxfp4"])
 @pytest.mark.parametrize("case", EDGE, ids=["16x64", "48x192", "32x16384"])
 def test_linear_edge_shapes(wq, orc, fmt, case):
     N, K, G, Ms = case
-    G = 0 if fmt == "cb4" else 16 if fmt == "nvfp4" else G
+    G = {"cb4": 0, "nvfp4": 16, "mxfp4": 32}.get(fmt, G)
     W, (codes, scales, aux) = small_case(orc, fmt, N, K, G, seed=N * 7 + K)
     pw = pack_on_gpu(wq, fmt, N, K, G, codes, scales, aux)
     dq = orc.dequant(fmt, codes, scales, aux, N, K, G)
@@ -180,3 +181,38 @@ def test_linear_edge_shapes(wq, orc, fmt, case):
         y = run_linear(wq, pw, xa[:M], b, M)
         ref, _ = orc.linear(xa[:M], dq, b)
         check_close(y, ref, f"{fmt} N={N} K={K} M={M}")
+
+
+@pytest.mark.parametrize("M", [8, 40])
+def test_mxfp4_every_scale_code(wq, orc, M):
+    """Every E8M0 code 0..254 and every E2M1 code, read through the linear with
+    one-hot activations (y[m, n] is one weight, exactly): the smallest scales
+    give bf16 subnormal weights, the largest overflow to inf, and code 255
+    (NaN) or an inf weight times a zero activation makes the whole output
+    column NaN, as in the fp64 definition."""
+    N, K = 256, 512
+    nb = K // 32
+    rng = np.random.default_rng(11)
+    q = rng.integers(0, 16, size=(N, K))
+    import test_oracle_linear as tol
+    codes = tol._pack_nibbles(q)
+    e = (np.arange(N * nb).reshape(N, nb) % 255).astype(np.uint8)
+    e[3, 5] = 255
+    pw = pack_on_gpu(wq, "mxfp4", N, K, 32, codes, e, None)
+    dq = orc.dequant("mxfp4", codes, e, None, N, K, 32)
+    ks = (np.arange(M) * 37 + 5) % K
+    xf = np.zeros((M, K))
+    xf[np.arange(M), ks] = 1.0
+    x = synth.f64_to_bf16_bits(xf)
+    ref, _ = orc.linear(x, dq, None)
+    y = run_linear(wq, pw, x, None, M)
+    yf = oracle.bits_to_f32(y)
+    rf = oracle.bits_to_f32(ref)
+    assert np.array_equal(np.isnan(yf), np.isnan(rf))
+    ok = ~np.isnan(rf)
+    assert ok.sum() > 0.7 * ok.size
+    assert np.array_equal(yf[ok], rf[ok])
+    # the finite columns hold the weight itself, subnormals included
+    w_sel = dq[:, ks].T
+    assert np.array_equal(rf[ok], w_sel.astype(np.float32)[ok])
+    assert (np.abs(w_sel[ok]) < 2.0 ** -126).any() and (np.abs(w_sel[ok]) > 2.0 ** 60).any()
