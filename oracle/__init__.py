@@ -22,7 +22,8 @@ _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 _lock = threading.Lock()
 _lib = None
 
-FORMATS = {"int4_sym": 0, "int4_asym": 1, "int8_sym": 2, "cb4": 3, "nvfp4": 4, "mxfp4": 5}
+FORMATS = {"int4_sym": 0, "int4_asym": 1, "int8_sym": 2, "cb4": 3, "nvfp4": 4, "mxfp4": 5,
+           "fp8_e4m3": 6}
 
 
 def build(force: bool = False, extra_flags=(), out_path: str | None = None,
@@ -57,6 +58,7 @@ def _declare(lib):
         "orc_quant_cb4": ([ptr, i64, i64, ptr, ptr, ptr], c_int),
         "orc_quant_nvfp4": ([ptr, i64, i64, ptr, ptr, ptr], c_int),
         "orc_quant_mxfp4": ([ptr, i64, i64, ptr, ptr], c_int),
+        "orc_quant_fp8_e4m3": ([ptr, i64, i64, c_int, ptr, ptr], c_int),
         "orc_e8m0_value": ([c_int], dbl),
         "orc_dequant": ([c_int, i64, i64, c_int, ptr, ptr, ptr, ptr], c_int),
         "orc_linear": ([ptr, ptr, ptr, i64, i64, i64, ptr, ptr], c_int),
@@ -163,6 +165,11 @@ class Oracle:
             bs = np.zeros((N, K // 32), dtype=np.uint8)
             _ok(self.lib.orc_quant_mxfp4(_p(W), N, K, _p(codes), _p(bs)), fmt)
             return codes, bs, None
+        if fmt == "fp8_e4m3":
+            codes = np.zeros((N, K), dtype=np.uint8)
+            scales = np.zeros((N, K // G), dtype=np.float32)
+            _ok(self.lib.orc_quant_fp8_e4m3(_p(W), N, K, G, _p(codes), _p(scales)), fmt)
+            return codes, scales, None
         raise ValueError(fmt)
 
     def lloyd_max(self, levels: int = 16):

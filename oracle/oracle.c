@@ -27,6 +27,9 @@
  *    (the OCP microscaling format definition): E2M1 values, one E8M0 scale
  *    (a power of two, 2^(e-127), e = 255 is NaN) per 32 consecutive K
  *    elements, no tensor scale.
+ *  - auto-round-lib README, section 1 "Supported Data Types": FP8 (E4M3)
+ *    weights with an FP32 scale, BF16 / FP32 compute (QuantLinearFP8, the
+ *    FP8 weight-only linear).
  *
  * Readings taken where the pages are silent:
  *  - rounding of w/s to an integer: round half to even;
@@ -47,6 +50,11 @@
  *    (|w| / 2^(e-127) in [4, 8) at the block's largest element, so values
  *    above 6 saturate), -0 written as +0; an all-zero block gets e = 0 and
  *    codes 0; dq = fp32(e2m1(q) * 2^(e-127)) (exact).
+ *  - FP8 E4M3: one fp32 scale per group of G along K (the grouping of the
+ *    INT formats), s = fp32(amax_g / 448) (448 = the largest finite E4M3),
+ *    q = E4M3_rne_satfinite(w / s) with the sign of w, -0 written as +0;
+ *    an all-zero group gets s = 0 and codes 0; dq = fp32(e4m3(q) * s)
+ *    (one rounding of the exact product).
  *  - Lloyd-Max: the 2**bits-level quantizer of N(0,1), computed by the
  *    classical fixed-point iteration (thresholds at midpoints, levels at
  *    conditional means) from a uniform start on [-3, 3], in fp64, then cast
@@ -63,6 +71,7 @@
  *   nvfp4    : codes u8 [N, K/2] E2M1 nibbles; block scales u8 [N, K/16] E4M3;
  *              tensor scale f32 [1]
  *   mxfp4    : codes u8 [N, K/2] E2M1 nibbles; block scales u8 [N, K/32] E8M0
+ *   fp8_e4m3 : codes u8 [N, K] E4M3; scales f32 [N, K/G]
  */
 #include <math.h>
 #include <stdint.h>
@@ -70,7 +79,7 @@
 #include <string.h>
 
 enum { ORC_INT4_SYM = 0, ORC_INT4_ASYM = 1, ORC_INT8_SYM = 2, ORC_CB4 = 3, ORC_NVFP4 = 4,
-       ORC_MXFP4 = 5 };
+       ORC_MXFP4 = 5, ORC_FP8_E4M3 = 6 };
 
 /* ------------------------------------------------------------------ bf16 */
 float orc_bf16_to_f32(uint16_t h) {
@@ -391,6 +400,33 @@ int orc_quant_mxfp4(const float* W, int64_t N, int64_t K, uint8_t* codes, uint8_
   return 0;
 }
 
+/* FP8 E4M3 weights, fp32 scale per group of G along K. */
+int orc_quant_fp8_e4m3(const float* W, int64_t N, int64_t K, int G, uint8_t* codes,
+                       float* scales) {
+  if (N <= 0 || K <= 0 || G <= 0 || K % G) return 1;
+  int64_t ng = K / G;
+  for (int64_t n = 0; n < N; ++n) {
+    const float* w = W + n * K;
+    for (int64_t j = 0; j < ng; ++j) {
+      double amax = 0.0;
+      for (int64_t k = j * G; k < (j + 1) * G; ++k) amax = fmax(amax, fabs((double)w[k]));
+      float sf = (float)(amax / 448.0);
+      scales[n * ng + j] = sf;
+      double s = (double)sf;
+      for (int64_t k = j * G; k < (j + 1) * G; ++k) {
+        int q = 0;
+        if (s != 0.0) {
+          double r = (double)w[k] / s;
+          q = orc_e4m3_encode(fabs(r));
+          if (r < 0.0 && q != 0) q |= 0x80;
+        }
+        codes[n * K + k] = (uint8_t)q;
+      }
+    }
+  }
+  return 0;
+}
+
 /* ------------------------------------------------------------- dequant */
 /* Exact dequantized value of element (n, k) from the canonical layout. */
 static float dq_one(int fmt, int64_t K, int G, const void* codes, const void* scales,
@@ -430,16 +466,22 @@ static float dq_one(int fmt, int64_t K, int G, const void* codes, const void* sc
       int e = ((const uint8_t*)scales)[n * (K / 32) + k / 32];
       return (float)(orc_e2m1_value(q) * orc_e8m0_value(e));
     }
+    case ORC_FP8_E4M3: {
+      int q = ((const uint8_t*)codes)[n * K + k];
+      double s = (double)((const float*)scales)[n * (K / G) + k / G];
+      return (float)(orc_e4m3_value(q) * s);
+    }
   }
   return NAN;
 }
 
 static int check_fmt(int fmt, int64_t N, int64_t K, int G) {
   if (N <= 0 || K <= 0) return 1;
-  if (fmt < 0 || fmt > 5) return 1;
-  if ((fmt == ORC_INT4_SYM || fmt == ORC_INT4_ASYM || fmt == ORC_INT8_SYM) && (G <= 0 || K % G))
+  if (fmt < 0 || fmt > 6) return 1;
+  if ((fmt == ORC_INT4_SYM || fmt == ORC_INT4_ASYM || fmt == ORC_INT8_SYM ||
+       fmt == ORC_FP8_E4M3) && (G <= 0 || K % G))
     return 1;
-  if (fmt != ORC_INT8_SYM && K % 2) return 1;
+  if (fmt != ORC_INT8_SYM && fmt != ORC_FP8_E4M3 && K % 2) return 1;
   if (fmt == ORC_NVFP4 && K % 16) return 1;
   if (fmt == ORC_MXFP4 && K % 32) return 1;
   return 0;

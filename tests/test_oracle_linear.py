@@ -99,11 +99,20 @@ def _int_case(fmt, N, K, G, rng):
         q[q == 8] = 0
         bs = np.full((N, K // 32), 127, np.uint8)          # E8M0 1.0
         return _pack_nibbles(q), bs, None, E2M1[q]
+    if fmt == "fp8_e4m3":
+        # E4M3 codes of the integers -16..16 (exact): 2^e (1 + m/8)
+        v = rng.integers(-16, 17, size=(N, K))
+        a = np.abs(v)
+        e = np.floor(np.log2(np.maximum(a, 1))).astype(np.int64)
+        m = (a * 8 // (1 << e)) - 8
+        code = np.where(a == 0, 0, ((e + 7) << 3) | m) | np.where(v < 0, 0x80, 0)
+        scales = np.ones((N, K // G), np.float32)
+        return code.astype(np.uint8), scales, None, v.astype(np.float64)
     raise ValueError(fmt)
 
 
 @pytest.mark.parametrize("fmt,G", [("int4_sym", 64), ("int4_asym", 32), ("int8_sym", 128),
-                                   ("cb4", 0), ("nvfp4", 16), ("mxfp4", 32)])
+                                   ("cb4", 0), ("nvfp4", 16), ("mxfp4", 32), ("fp8_e4m3", 64)])
 def test_integer_special_case(orc, fmt, G):
     """Integer X, unit scales: every partial sum is exact, so y equals an
     integer matmul done by numpy -- pins layout, nibble order and orientation."""
@@ -121,7 +130,7 @@ def test_integer_special_case(orc, fmt, G):
 
 
 @pytest.mark.parametrize("fmt,G", [("int4_sym", 64), ("int4_asym", 128), ("int8_sym", 256),
-                                   ("cb4", 0), ("nvfp4", 16), ("mxfp4", 32)])
+                                   ("cb4", 0), ("nvfp4", 16), ("mxfp4", 32), ("fp8_e4m3", 128)])
 def test_sampled_equals_full(orc, fmt, G):
     M, N, K = 6, 32, 512
     W = synth.weight(21, N, K, sigma=0.02)

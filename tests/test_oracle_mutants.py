@@ -64,6 +64,14 @@ MUTANTS = [
      "double nc = (normal_pdf(t[i]) - normal_pdf(t[i + 1])) / p;",
      "double nc = (normal_pdf(t[i]) - normal_pdf(t[i + 1])) / p * 1.001;",
      lambda o: quant.test_lloyd_max_invariants(o)),
+    ("FP8 sign dropped",
+     "if (r < 0.0 && q != 0) q |= 0x80;",
+     "if (r < 0.0 && q == 0) q |= 0x80;",
+     lambda o: quant.test_fp8_e4m3_properties(o, 32)),
+    ("FP8 scale from the wrong maximum",
+     "float sf = (float)(amax / 448.0);",
+     "float sf = (float)(amax / 240.0);",
+     lambda o: quant.test_fp8_e4m3_properties(o, 128)),
     ("E2M1 tie broken toward the odd code",
      "if (a == mid) { code = (i % 2 == 0) ? i : i + 1; break; }",
      "if (a == mid) { code = (i % 2 == 0) ? i + 1 : i; break; }",

@@ -266,3 +266,71 @@ def test_mxfp4_round_trip(orc):
     codes, bs, _ = orc.quantize("mxfp4", W)
     assert np.array_equal(bs.astype(np.int64), e)
     assert np.array_equal(_nibbles(codes).astype(np.int64), q)
+
+
+# ------------------------------------------------------------------ FP8 E4M3
+def _e4m3_table():
+    """value of every E4M3 code from torch's float8_e4m3fn (an independent decoder)."""
+    import torch
+    return torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(
+        torch.float64).numpy()
+
+
+@pytest.mark.parametrize("G", [32, 128])
+def test_fp8_e4m3_properties(orc, G):
+    """Group scale within half an fp32 ulp of amax/448; every code the nearest
+    finite E4M3 value to w/s by brute force (ties to the even code), with the
+    sign of w and +0 for zero; the group maximum at +-448; all-zero groups get
+    scale 0 and code 0; dequant = fp32 of the exact product."""
+    from fractions import Fraction
+    N, K = 24, 512
+    W = _weights(N, K, seed=9)
+    codes, scales, aux = orc.quantize("fp8_e4m3", W, G)
+    assert aux is None and codes.shape == (N, K) and scales.dtype == np.float32
+    ng = K // G
+    W64 = W.astype(np.float64)
+    amax = np.abs(W64).reshape(N, ng, G).max(-1)
+    for (n, j), a in np.ndenumerate(amax):
+        s = scales[n, j]
+        if a == 0.0:
+            assert s == 0.0 and not np.any(codes[n, j * G:(j + 1) * G])
+            continue
+        exact = Fraction(a) / 448
+        ulp = np.spacing(np.float32(s))
+        assert abs(Fraction(float(s)) - exact) <= Fraction(float(ulp)) / 2
+    tab = _e4m3_table()
+    fin = np.array([c for c in range(256) if np.isfinite(tab[c])])
+    vals = tab[fin]
+    S = np.repeat(scales.astype(np.float64), G, axis=1)
+    live = S > 0
+    r = np.where(live, W64 / np.where(live, S, 1.0), 0.0)
+    # nearest finite value; among equals the code with an even mantissa
+    d = np.abs(r[..., None] - vals[None, None, :])
+    best = d.min(-1, keepdims=True)
+    cand = d == best
+    even = (fin & 1) == 0
+    pick = np.where(cand & even[None, None, :], 1, 0) + cand
+    want = fin[np.argmax(pick, axis=-1)]
+    want = np.where(tab[want] == 0.0, 0, want)       # zero is written as +0
+    got = codes.astype(np.int64)
+    assert np.array_equal(got[live], want[live])
+    gmax = np.abs(tab[got]).reshape(N, ng, G).max(-1)
+    assert np.all(gmax[amax > 0] == 448.0)
+    dq = orc.dequant("fp8_e4m3", codes, scales, None, N, K, G)
+    assert np.array_equal(dq, (tab[got] * S).astype(np.float32))
+
+
+def test_fp8_e4m3_round_trip(orc):
+    """Groups built from E4M3 values (each holding +-448) times a power-of-two
+    scale quantize back to the same codes and scale."""
+    rng = np.random.default_rng(13)
+    N, K, G = 8, 256, 64
+    tab = _e4m3_table()
+    fin = np.array([c for c in range(256) if np.isfinite(tab[c]) and c != 0x80])
+    q = rng.choice(fin, size=(N, K))
+    q[:, ::G] = 0x7E                   # +448 in every group
+    s = np.ldexp(1.0, rng.integers(-20, -5, size=(N, K // G)))
+    W = (tab[q] * np.repeat(s, G, axis=1)).astype(np.float32)
+    codes, scales, _ = orc.quantize("fp8_e4m3", W, G)
+    assert np.array_equal(scales.astype(np.float64), s)
+    assert np.array_equal(codes.astype(np.int64), q)
