@@ -26,7 +26,7 @@
  *    16 rows by 64 (4-bit) or 32 (INT8) K elements); INT formats take
  *    group_size in {32, 64, 128, 256} with K % group_size == 0; NVFP4 has a
  *    fixed block of 16 (group_size 16 or 0), MXFP4 one of 32 (group_size 32
- *    or 0); CB4 ignores group_size.
+ *    or 0); CB4 ignores group_size; FP8_E4M3 takes the INT group sizes.
  *  - Every device pointer must be 16-byte aligned, except the NVFP4 tensor
  *    scale and the CB4 centroids (4-byte aligned).
  *
@@ -48,11 +48,17 @@
  *   WQ_MXFP4    : codes  u8 [N, K/2]  E2M1 nibbles, same nibble order
  *                 scales = block scales u8 [N, K/32] (E8M0: 2^(e-127),
  *                 e = 255 is NaN); aux = NULL
+ *   WQ_FP8_E4M3 : codes  u8 [N, K]    E4M3 (fn) bytes; scales f32 [N, K/G];
+ *                 aux = NULL
  * Dequantized value of element (n, k) -- what wq_dequant returns:
  *   INT4_SYM/INT8_SYM: q * s            ASYM: (q - z) * s          (exact fp32)
  *   CB4: fp32(c[idx] * norm[n])         NVFP4: fp32(e2m1(q) * e4m3(sb) * ts)
  *   MXFP4: fp32(e2m1(q) * 2^(e-127))    (exact; +-inf where the product
  *                                          reaches 2^128, NaN for e = 255)
+ *   FP8_E4M3: fp32(e4m3(q) * s)         (one rounding; NaN for the codes
+ *                                          0x7F / 0xFF, which wq_linear does
+ *                                          not accept as weights: its kernels
+ *                                          read them as +-480)
  */
 #ifndef WQ_H_
 #define WQ_H_
@@ -72,7 +78,8 @@ typedef enum {
   WQ_INT8_SYM = 2,  /* symmetric INT8, bf16 scale per group                    */
   WQ_CB4 = 3,       /* 4-bit codebook: 16 fp32 centroids, bf16 norm per row    */
   WQ_NVFP4 = 4,     /* E2M1 values, E4M3 scale per 16, fp32 tensor scale       */
-  WQ_MXFP4 = 5      /* E2M1 values, E8M0 power-of-two scale per 32 (OCP MX)    */
+  WQ_MXFP4 = 5,     /* E2M1 values, E8M0 power-of-two scale per 32 (OCP MX)    */
+  WQ_FP8_E4M3 = 6   /* E4M3 values, fp32 scale per group (FP8 weight-only)     */
 } wq_format_t;
 
 typedef enum {
@@ -130,9 +137,11 @@ int wq_dequant(int format, int64_t N, int64_t K, int group_size, const void* pac
  *   x        device bf16 [M, K] row-major
  *   packed_w device, from wq_pack
  *   scales   device: INT formats packed group scales; CB4 row norms;
- *            NVFP4 packed E4M3 block scales; MXFP4 packed E8M0 block scales
+ *            NVFP4 packed E4M3 block scales; MXFP4 packed E8M0 block scales;
+ *            FP8_E4M3 packed fp32 group scales
  *   aux      device: ASYM packed zero-points; CB4 centroids f32[16];
- *            NVFP4 tensor scale f32[1]; NULL for INT4_SYM / INT8_SYM / MXFP4
+ *            NVFP4 tensor scale f32[1]; NULL for INT4_SYM / INT8_SYM / MXFP4 /
+ *            FP8_E4M3
  *   bias     device bf16 [N], or NULL
  *   out      device bf16 [M, N] row-major; must not overlap any input
  * M == 0 is a no-op returning WQ_OK.  Asynchronous; no workspace.
@@ -160,6 +169,7 @@ int wq_linear(const void* x, const void* packed_w, const void* scales, const voi
  * definitions listed above.  CB4 reads its 16 centroids from `aux`
  * (device f32[16], left unchanged) and writes the row norms; NVFP4 writes the
  * tensor scale into `aux`.  Synchronizes `stream` for NVFP4 (two passes).
+ * FP8_E4M3 writes fp32 scales amax/448 per group.
  * Source: piper-kernels README "ConvRot INT8" (ConvRotInt8Tensor.from_hp
  * quantizes a dense weight, group_size=256); Mamba-2 pack helper (scale =
  * amax/qmax, round, clamp). */

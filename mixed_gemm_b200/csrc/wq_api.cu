@@ -16,11 +16,11 @@ bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p % a) == 0; }
 
 // Shape / format checks shared by every entry point.
 int check_shape(int f, int64_t N, int64_t K, int G) {
-  if (f < INT4_SYM || f > MXFP4) return WQ_ERR_INVALID_ARG;
+  if (f < INT4_SYM || f > FP8_E4M3) return WQ_ERR_INVALID_ARG;
   if (N <= 0 || K <= 0) return WQ_ERR_INVALID_ARG;
   if (N % 16 || K % 64) return WQ_ERR_INVALID_ARG;
   if (N > (1LL << 30) || K > (1LL << 24) || N * K > (1LL << 40)) return WQ_ERR_INVALID_ARG;
-  if (is_int_fmt(f)) {
+  if (is_grouped_fmt(f)) {
     if (G != 32 && G != 64 && G != 128 && G != 256) return WQ_ERR_INVALID_ARG;
     if (K % G) return WQ_ERR_INVALID_ARG;
   } else if (f == NVFP4) {
@@ -84,6 +84,7 @@ int wq_canonical_sizes(int f, int64_t N, int64_t K, int G, size_t* cb, size_t* s
     case INT4_SYM: c = N * K / 2; s = 2 * N * (K / G); break;
     case INT4_ASYM: c = N * K / 2; s = 2 * N * (K / G); a = N * (K / G); break;
     case INT8_SYM: c = N * K; s = 2 * N * (K / G); break;
+    case FP8_E4M3: c = N * K; s = 4 * N * (K / G); break;
     case CB4: c = N * K / 2; s = 2 * N; a = 64; break;
     case NVFP4: c = N * K / 2; s = N * (K / 16); a = 4; break;
     case MXFP4: c = N * K / 2; s = N * (K / 32); a = 0; break;

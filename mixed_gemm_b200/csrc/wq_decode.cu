@@ -121,6 +121,11 @@ __device__ __forceinline__ uint32_t lds8(uint32_t addr) {
   asm volatile("ld.shared.u8 %0, [%1];" : "=h"(v) : "r"(addr));
   return v;
 }
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -145,10 +150,14 @@ __device__ __forceinline__ void cluster_sync_all() {
 // issued into the freed registers.
 template <int FMT, int NT, int RT, int KW, int D>
 __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
-  constexpr int KB = FMT == INT8_SYM ? 32 : 64;   // K per 512-byte block
-  constexpr int CPB = FMT == INT8_SYM ? 1 : 2;    // 32-K chunks per block
+  constexpr bool kByte = FMT == INT8_SYM || FMT == FP8_E4M3;  // one byte per code
+  constexpr int KB = kByte ? 32 : 64;             // K per 512-byte block
+  constexpr int CPB = kByte ? 1 : 2;              // 32-K chunks per block
   constexpr int NV = RT * NT * 4;                  // accumulators per lane
-  constexpr bool kIntFmt = FMT == INT4_SYM || FMT == INT4_ASYM || FMT == INT8_SYM;
+  // one scale per group of K folded into fp32 sums (INT formats, FP8)
+  constexpr bool kIntFmt =
+      FMT == INT4_SYM || FMT == INT4_ASYM || FMT == INT8_SYM || FMT == FP8_E4M3;
+  constexpr int SB = FMT == FP8_E4M3 ? 64 : 32;   // bytes per (row tile, group) of scales
 
   extern __shared__ __align__(16) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -191,12 +200,12 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   {
     if constexpr (kIntFmt) {
       const int ng = ((ce * KB - 1) >> p.gshift) + 1 - g_begin;
-      // scales: 32 bytes per (tile, group) -> two 16-byte chunks
+      // scales: SB bytes per (tile, group) -> SB / 16 chunks of 16 bytes
 #pragma unroll
       for (int r = 0; r < RT; ++r) {
-        const uint8_t* src = (const uint8_t*)p.scales + ((int64_t)(tile0 + r) * groups + g_begin) * 32;
-        for (int i = threadIdx.x; i < ng * 2; i += KW * 32)
-          cp_async16(side + (r * p.side_rows) * 32 + i * 16, src + i * 16);
+        const uint8_t* src = (const uint8_t*)p.scales + ((int64_t)(tile0 + r) * groups + g_begin) * SB;
+        for (int i = threadIdx.x; i < ng * (SB / 16); i += KW * 32)
+          cp_async16(side + (r * p.side_rows) * SB + i * 16, src + i * 16);
       }
       if constexpr (FMT == INT4_ASYM) {
         const uint32_t zs = side + RT * p.side_rows * 32;
@@ -298,11 +307,11 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   // INT group state: chunk accumulators, packed scales, zero-point offsets
   // (bf16 pairs of 128 + z; 136 = 128 + 8 for offset-binary signed codes)
   float cacc[NS][kIntFmt ? RT : 1][NT][4];
-  uint32_t gsw[RT], goff[RT][2];
+  uint32_t gsw[RT], gsw2[RT], goff[RT][2];
   const int gmask = kIntFmt ? (1 << p.gshift) - 1 : 0;
 #pragma unroll
   for (int r = 0; r < RT; ++r) {
-    gsw[r] = 0;
+    gsw[r] = gsw2[r] = 0;
     goff[r][0] = goff[r][1] = 0x43084308u;
   }
 
@@ -336,7 +345,13 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
           const int gi = (k0 >> p.gshift) - g_begin;
 #pragma unroll
           for (int r = 0; r < RT; ++r) {
-            gsw[r] = lds32(side + (r * p.side_rows + gi) * 32 + g * 4);
+            if constexpr (FMT == FP8_E4M3) {  // fp32 scales of rows g, g + 8
+              const uint2 sv = lds64(side + (r * p.side_rows + gi) * 64 + g * 8);
+              gsw[r] = sv.x;
+              gsw2[r] = sv.y;
+            } else {
+              gsw[r] = lds32(side + (r * p.side_rows + gi) * 32 + g * 4);
+            }
             if constexpr (FMT == INT4_ASYM) {
               const uint32_t zb =
                   lds8(side + RT * p.side_rows * 32 + (r * p.side_rows + gi) * 8 + g);
@@ -360,6 +375,8 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
             uint32_t a[4];
             if constexpr (FMT == INT8_SYM)
               frag_int8(word(wb_[r], 2 * s), word(wb_[r], 2 * s + 1), a);
+            else if constexpr (FMT == FP8_E4M3)
+              frag_e4m3(word(wb_[r], 2 * s), word(wb_[r], 2 * s + 1), a);
             else
               frag_int4(word(wb_[r], 2 * c + s), goff[r][0], goff[r][1], a);
 #pragma unroll
@@ -368,8 +385,10 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
                        word(xv[c][nt], 2 * s + 1));
           }
           if (gend) {
-            const float s_g = __uint_as_float(gsw[r] << 16);
-            const float s_g8 = __uint_as_float(gsw[r] & 0xFFFF0000u);
+            const float s_g =
+                FMT == FP8_E4M3 ? __uint_as_float(gsw[r]) : __uint_as_float(gsw[r] << 16);
+            const float s_g8 = FMT == FP8_E4M3 ? __uint_as_float(gsw2[r])
+                                               : __uint_as_float(gsw[r] & 0xFFFF0000u);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
               float c4[4];
@@ -584,10 +603,10 @@ cudaError_t launch_decode(const LinearArgs& a) {
   // staged side data per row tile: a K range of max_blocks*kb may touch one
   // more group than it spans
   p.gshift = 0;
-  if (is_int_fmt(a.fmt)) {
+  if (is_grouped_fmt(a.fmt)) {
     while ((1 << p.gshift) < a.G) ++p.gshift;
     p.side_rows = (int)((max_blocks * kb + a.G - 1) / a.G + 1);
-    p.side_bytes = rt * p.side_rows * (a.fmt == INT4_ASYM ? 40 : 32);
+    p.side_bytes = rt * p.side_rows * (a.fmt == INT4_ASYM ? 40 : a.fmt == FP8_E4M3 ? 64 : 32);
   } else if (a.fmt == NVFP4 || a.fmt == MXFP4) {
     p.side_rows = (int)(max_blocks * kb / (a.fmt == NVFP4 ? 16 : 32));
     p.side_bytes = rt * p.side_rows * 16 + 1024;  // block scales + code table
@@ -610,6 +629,7 @@ cudaError_t launch_decode(const LinearArgs& a) {
     case CB4: return launch_fmt<CB4>(p, nt, rt, grid, a.stream);
     case NVFP4: return launch_fmt<NVFP4>(p, nt, rt, grid, a.stream);
     case MXFP4: return launch_fmt<MXFP4>(p, nt, rt, grid, a.stream);
+    case FP8_E4M3: return launch_fmt<FP8_E4M3>(p, nt, rt, grid, a.stream);
   }
   return cudaErrorInvalidValue;
 }

@@ -56,6 +56,23 @@ static __device__ __forceinline__ void frag_int8(uint32_t wg, uint32_t wg8, uint
   a[3] = pack_bf16x2(i8val(wg8, 2), i8val(wg8, 3));
 }
 
+// FP8 E4M3 bytes -> exact bf16 fragments.  A byte placed at bits 8..15 of a
+// 16-bit half (sign at bit 15) and its 7 magnitude bits moved to bits 4..10
+// reads as the bf16 number e4m3 * 2^-120 (for the E4M3 subnormals too, whose
+// spacing 2^-9 becomes the bf16 subnormal spacing); the exact product with
+// 2^120 restores the value.  Fragment registers as in frag_int8.  The NaN
+// codes 0x7F / 0xFF come out as +-480.
+static __device__ __forceinline__ uint32_t e4m3x2_scaled_bits(uint32_t t8) {
+  return ((t8 >> 4) & 0x07F007F0u) | (t8 & 0x80008000u);
+}
+static __device__ __forceinline__ void frag_e4m3(uint32_t wg, uint32_t wg8, uint32_t (&a)[4]) {
+  const uint32_t k120 = 0x7B807B80u;  // bf16x2 (2^120, 2^120)
+  a[0] = bmul2(e4m3x2_scaled_bits(__byte_perm(wg, 0u, 0x1404u)), k120);
+  a[1] = bmul2(e4m3x2_scaled_bits(__byte_perm(wg8, 0u, 0x1404u)), k120);
+  a[2] = bmul2(e4m3x2_scaled_bits(__byte_perm(wg, 0u, 0x3424u)), k120);
+  a[3] = bmul2(e4m3x2_scaled_bits(__byte_perm(wg8, 0u, 0x3424u)), k120);
+}
+
 // 16-entry bf16 lookup ("table" nibble order): byte tables H (high bytes) and
 // L (low bytes), four entries per register.  `kSymLow` means the low-byte
 // table does not depend on the top index bit (true for E2M1).

@@ -4,9 +4,9 @@
 // --------------------------------------------------------
 // Rows are grouped in tiles of 16 (n = 16*tile + r, r = g + 8*hr, g = 0..7,
 // hr = 0/1).  Along K a tile is cut into blocks of 512 bytes: 64 K elements
-// for 4-bit codes, 32 for INT8.  Inside a block, lane L = 4*g + tq of a warp
+// for 4-bit codes, 32 for byte codes (INT8, FP8 E4M3).  Inside a block, lane L = 4*g + tq of a warp
 // owns 16 contiguous bytes: the codes of rows g and g+8 for K offsets
-// {32c + 8tq + 4s + e : c, s in {0,1} (4-bit) or c = 0 (INT8), e = 0..3}.
+// {32c + 8tq + 4s + e : c, s in {0,1} (4-bit) or c = 0 (bytes), e = 0..3}.
 // One 16-byte load per lane therefore yields exactly the A-operand fragments
 // of an m16n8k16 tensor-core step (W rows as the 16-row operand), with the K
 // order inside each 16-step permuted consistently for A and B, so that the
@@ -21,10 +21,12 @@
 //        low/high 16 bits hold registers {0,1} / {2,3} as four nibbles each,
 //        ready for byte-permute table lookups.
 //   INT4_SYM nibbles are stored offset-binary (v + 8); INT8 bytes likewise
-//   (v + 128), word j = 2s + hr, byte e.
+//   (v + 128), word j = 2s + hr, byte e; FP8 E4M3 bytes as they are, at the
+//   INT8 positions.
 //
 // Scales (INT formats):  bf16 [N/16][K/G][16], entry 2g + hr (so lane g
 //   reads rows g and g+8 as one 32-bit word).
+// Scales (FP8 E4M3):     f32 [N/16][K/G][16], entry 2g + hr (one 64-bit word).
 // Zero-points (ASYM):    u8 [N/16][K/G][8], byte g = z(row g) | z(row g+8) << 4.
 // NVFP4 block scales:    u8 [N/16][K/16][16], entry 2g + hr.
 // MXFP4 block scales:    u8 [N/16][K/32][16], entry 2g + hr.
@@ -40,10 +42,15 @@
 
 namespace wq {
 
-enum Fmt { INT4_SYM = 0, INT4_ASYM = 1, INT8_SYM = 2, CB4 = 3, NVFP4 = 4, MXFP4 = 5 };
+enum Fmt { INT4_SYM = 0, INT4_ASYM = 1, INT8_SYM = 2, CB4 = 3, NVFP4 = 4, MXFP4 = 5,
+           FP8_E4M3 = 6 };
 
 __host__ __device__ inline bool is_int_fmt(int f) { return f == INT4_SYM || f == INT4_ASYM || f == INT8_SYM; }
-__host__ __device__ inline bool is_4bit(int f) { return f != INT8_SYM; }
+// formats with one scale per group of G along K, folded into fp32 sums
+__host__ __device__ inline bool is_grouped_fmt(int f) { return is_int_fmt(f) || f == FP8_E4M3; }
+__host__ __device__ inline bool is_4bit(int f) { return f != INT8_SYM && f != FP8_E4M3; }
+// bytes of one packed group scale
+__host__ __device__ inline int scale_bytes(int f) { return f == FP8_E4M3 ? 4 : 2; }
 // elements of K per 512-byte block
 __host__ __device__ inline int block_k(int f) { return is_4bit(f) ? 64 : 32; }
 

@@ -172,6 +172,9 @@ __global__ void dequant_kernel(int f, int64_t N, int64_t K, int G, const uint8_t
       int z = (((const uint8_t*)pa)[zb] >> zs) & 15;
       float s = bf16_bits_to_f32(((const uint16_t*)ps)[packed_scale_idx(n, k / G, K / G)]);
       v = (float)((int)raw - z) * s;
+    } else if (f == FP8_E4M3) {  // one rounding of the exact e4m3 * s
+      float s = ((const float*)ps)[packed_scale_idx(n, k / G, K / G)];
+      v = __fmul_rn(e4m3_to_f32(raw), s);
     } else if (f == CB4) {
       float c = ((const float*)pa)[raw];
       float nr = bf16_bits_to_f32(((const uint16_t*)ps)[n]);
@@ -198,7 +201,11 @@ cudaError_t launch_pack(int f, int64_t N, int64_t K, int G, const void* codes, c
   const int64_t wbytes = is_4bit(f) ? N * K / 2 : N * K;
   pack_w_kernel<<<grid_for(wbytes), kThreads, 0, st>>>(f, N, K, (const uint8_t*)codes,
                                                         (uint8_t*)pw);
-  if (is_int_fmt(f)) {
+  if (f == FP8_E4M3) {
+    int64_t groups = K / G;
+    permute_scales_kernel<uint32_t><<<grid_for(N * groups), kThreads, 0, st>>>(
+        N, groups, (const uint32_t*)scales, (uint32_t*)ps, true);
+  } else if (is_int_fmt(f)) {
     int64_t groups = K / G;
     permute_scales_kernel<uint16_t><<<grid_for(N * groups), kThreads, 0, st>>>(
         N, groups, (const uint16_t*)scales, (uint16_t*)ps, true);
@@ -223,7 +230,11 @@ cudaError_t launch_unpack(int f, int64_t N, int64_t K, int G, const void* pw, co
   const int64_t wbytes = is_4bit(f) ? N * K / 2 : N * K;
   unpack_w_kernel<<<grid_for(wbytes), kThreads, 0, st>>>(f, N, K, (const uint8_t*)pw,
                                                           (uint8_t*)codes);
-  if (is_int_fmt(f)) {
+  if (f == FP8_E4M3) {
+    int64_t groups = K / G;
+    permute_scales_kernel<uint32_t><<<grid_for(N * groups), kThreads, 0, st>>>(
+        N, groups, (const uint32_t*)ps, (uint32_t*)scales, false);
+  } else if (is_int_fmt(f)) {
     int64_t groups = K / G;
     permute_scales_kernel<uint16_t><<<grid_for(N * groups), kThreads, 0, st>>>(
         N, groups, (const uint16_t*)ps, (uint16_t*)scales, false);

@@ -243,8 +243,11 @@ template <int FMT, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                    const PrefillParams p) {
-  constexpr bool kInt = FMT == INT4_SYM || FMT == INT4_ASYM || FMT == INT8_SYM;
-  constexpr uint32_t kWpk = FMT == INT8_SYM ? 8192u : 4096u;  // packed bytes per stage
+  // one scale per group of K, folded into fp32 sums (INT formats, FP8)
+  constexpr bool kInt =
+      FMT == INT4_SYM || FMT == INT4_ASYM || FMT == INT8_SYM || FMT == FP8_E4M3;
+  constexpr bool kByte = FMT == INT8_SYM || FMT == FP8_E4M3;  // one byte per code
+  constexpr uint32_t kWpk = kByte ? 8192u : 4096u;  // packed bytes per stage
   // A stage: one 128 x 64 bf16 tile; CB4 adds a second tile holding the
   // bf16 remainders of its centroids (two MMAs per K step)
   constexpr uint32_t kAsub = FMT == CB4 ? 2u : 1u;
@@ -464,14 +467,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int rr = 0; rr < 2; ++rr) {
         const int rt = 2 * dw + rr;
         const int Rg = rt * 16 + g, Rg8 = Rg + 8;
-        if constexpr (FMT == INT8_SYM) {
+        if constexpr (kByte) {
 #pragma unroll
           for (int blk = 0; blk < 2; ++blk) {
             const uint4 ch = *(const uint4*)(wpk + rt * 1024 + blk * 512 + lane * 16);
             // exact codes; the group scale is applied by the fold warps
             uint32_t a[4], b[4];
-            frag_int8(ch.x, ch.y, a);
-            frag_int8(ch.z, ch.w, b);
+            if constexpr (FMT == FP8_E4M3) {
+              frag_e4m3(ch.x, ch.y, a);
+              frag_e4m3(ch.z, ch.w, b);
+            } else {
+              frag_int8(ch.x, ch.y, a);
+              frag_int8(ch.z, ch.w, b);
+            }
             const int j = 4 * blk + tq;
             st_shared_v4(abase + swz(Rg, j), a[0], a[2], b[0], b[2]);
             st_shared_v4(abase + swz(Rg8, j), a[1], a[3], b[1], b[3]);
@@ -550,7 +558,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t groups = kInt ? p.K / p.G : 0;
     // per-row factors, requested before the first wait: the group scales of
     // the next two groups ride in registers ahead of the group being folded
+    // group scales: bf16 (INT formats) or fp32 (FP8), same packed indexing
     const uint16_t* srow = (const uint16_t*)p.scales;
+    const uint32_t* srow32 = (const uint32_t*)p.scales;
     int64_t sidx = 0;
     if (kInt && nvalid) {
       const int r16 = (int)(n & 15);
@@ -558,9 +568,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     const int gfirst = kInt ? (kt0 * 64) / p.G : 0;  // first group of this CTA's K range
     auto group_scale = [&](int gi) -> uint32_t {
-      return (kInt && nvalid && gi < NG)
-                 ? (uint32_t)__ldg(srow + sidx + (int64_t)(gfirst + gi) * 16)
-                 : 0u;
+      if (!(kInt && nvalid && gi < NG)) return 0u;
+      if constexpr (FMT == FP8_E4M3) return __ldg(srow32 + sidx + (int64_t)(gfirst + gi) * 16);
+      return (uint32_t)__ldg(srow + sidx + (int64_t)(gfirst + gi) * 16);
     };
     uint32_t sc0 = group_scale(0), sc1 = group_scale(1);
     float post = 1.f, bval = 0.f;
@@ -579,7 +589,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = mbar_wait(gfull_bar(gb), (uint32_t)(g >> 1) & 1u, abort, 64u);
       if (!__all_sync(0xffffffffu, ok ? 1 : 0)) { ok = false; break; }
       tc_fence_after();
-      const float sc = kInt ? bf16_bits_to_f32((uint16_t)sc0) : 1.f;
+      const float sc = FMT == FP8_E4M3 ? __uint_as_float(sc0)
+                       : kInt          ? bf16_bits_to_f32((uint16_t)sc0)
+                                       : 1.f;
       sc0 = sc1;
       sc1 = sc2;
       const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(gb * BN + hcol);
@@ -676,7 +688,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 template <int FMT, int BN>
 cudaError_t launch_bn(const LinearArgs& a) {
-  constexpr uint32_t kWpk = FMT == INT8_SYM ? 8192u : 4096u;
+  constexpr uint32_t kWpk = (FMT == INT8_SYM || FMT == FP8_E4M3) ? 8192u : 4096u;
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
   CUtensorMap tmX, tmW;
@@ -691,7 +703,7 @@ cudaError_t launch_bn(const LinearArgs& a) {
       return cudaErrorInvalidValue;
   }
   {
-    const uint64_t row_bytes = (uint64_t)a.K * (FMT == INT8_SYM ? 16 : 8);  // bytes per row tile
+    const uint64_t row_bytes = (uint64_t)a.K * (is_4bit(FMT) ? 8 : 16);  // bytes per row tile
     cuuint64_t dims[2] = {(cuuint64_t)(row_bytes / 4), (cuuint64_t)(a.N / 16)};
     cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
     cuuint32_t box[2] = {kWpk / 32u, 8u};
@@ -747,7 +759,7 @@ cudaError_t launch_bn(const LinearArgs& a) {
   {
     const int64_t tiles = (int64_t)((a.N + 127) / 128) * ((a.M + BN - 1) / BN);
     const int64_t KTall = a.K / 64;
-    const int64_t unit = (is_int_fmt(FMT) && a.G > 64) ? a.G / 64 : 1;
+    const int64_t unit = (is_grouped_fmt(FMT) && a.G > 64) ? a.G / 64 : 1;
     const int64_t sms = device_sm_count();
     int best_s = 1;
     if (2 * tiles <= sms) {
@@ -767,7 +779,7 @@ cudaError_t launch_bn(const LinearArgs& a) {
 #endif
     p.splits = best_s;
   }
-  const bool groups2 = is_int_fmt(FMT) && (a.K / a.G) > 1;  // two alternating accumulators
+  const bool groups2 = is_grouped_fmt(FMT) && (a.K / a.G) > 1;  // two alternating accumulators
   p.tmem_cols = (uint32_t)(groups2 ? 2 * BN : (BN < 32 ? 32 : BN));
   dim3 grid((unsigned)((a.N + 127) / 128), (unsigned)((a.M + BN - 1) / BN), (unsigned)p.splits);
   if (p.splits > 1) {
@@ -818,6 +830,7 @@ cudaError_t launch_prefill(const LinearArgs& a) {
     case CB4: return launch_fmt<CB4>(a, BN);
     case NVFP4: return launch_fmt<NVFP4>(a, BN);
     case MXFP4: return launch_fmt<MXFP4>(a, BN);
+    case FP8_E4M3: return launch_fmt<FP8_E4M3>(a, BN);
   }
   return cudaErrorInvalidValue;
 }

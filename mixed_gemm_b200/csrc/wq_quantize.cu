@@ -106,6 +106,33 @@ __global__ void quant_sym_kernel(int bits, int64_t N, int64_t K, int G,
   }
 }
 
+// One warp per (row, group): FP8 E4M3 codes, fp32 scale = amax / 448.
+__global__ void quant_fp8_kernel(int64_t N, int64_t K, int G, const float* __restrict__ w,
+                                 uint8_t* __restrict__ codes, float* __restrict__ scales) {
+  const int lane = threadIdx.x & 31;
+  const int64_t groups = K / G;
+  for (int64_t item = blockIdx.x * (int64_t)kWarps + (threadIdx.x >> 5); item < N * groups;
+       item += (int64_t)gridDim.x * kWarps) {
+    int64_t n = item / groups, grp = item % groups;
+    const float* wg = w + n * K + grp * G;
+    double amax = 0.0;
+    for (int i = lane; i < G; i += 32) amax = fmax(amax, fabs((double)wg[i]));
+    for (int o = 16; o; o >>= 1) amax = fmax(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float sf = __double2float_rn(__ddiv_rn(amax, 448.0));
+    const double s = (double)sf;
+    if (lane == 0) scales[item] = sf;
+    for (int i = lane; i < G; i += 32) {
+      uint32_t q = 0;
+      if (s != 0.0) {
+        const double r = __ddiv_rn((double)wg[i], s);
+        q = e4m3_encode_rn_satfinite(fabs(r));
+        if (r < 0.0 && q != 0u) q |= 0x80u;
+      }
+      codes[n * K + grp * G + i] = (uint8_t)q;
+    }
+  }
+}
+
 // One warp per (row, group): asymmetric INT4 with a uint4 zero-point.
 __global__ void quant_asym_kernel(int64_t N, int64_t K, int G, const float* __restrict__ w,
                                   uint8_t* __restrict__ codes, uint16_t* __restrict__ scales,
@@ -280,6 +307,10 @@ cudaError_t launch_quantize(int f, int64_t N, int64_t K, int G, const float* w, 
     case INT8_SYM:
       quant_sym_kernel<<<blocks_for(N * (K / G), kWarps), kWarps * 32, 0, st>>>(
           f == INT4_SYM ? 4 : 8, N, K, G, w, (uint8_t*)codes, (uint16_t*)scales);
+      break;
+    case FP8_E4M3:
+      quant_fp8_kernel<<<blocks_for(N * (K / G), kWarps), kWarps * 32, 0, st>>>(
+          N, K, G, w, (uint8_t*)codes, (float*)scales);
       break;
     case INT4_ASYM:
       quant_asym_kernel<<<blocks_for(N * (K / G), kWarps), kWarps * 32, 0, st>>>(

@@ -1,12 +1,15 @@
-"""The six synthetic workloads of the weight-only quantized linear.
+"""The seven synthetic workloads of the weight-only quantized linear.
 
 Each recipe fixes shapes, the weight format, the group size, the seed and the
 value distributions; ``make_inputs`` draws the dense inputs for one of them.
-Format names are the library's: int4_sym, int4_asym, int8_sym, cb4, nvfp4, mxfp4.
+Format names are the library's: int4_sym, int4_asym, int8_sym, cb4, nvfp4, mxfp4,
+fp8_e4m3.
 
 Readings (the recipe texts leave these open):
   * seeds other than the first workload's are 1, 2, 3, 4 in order, and 5
-    for the MXFP4 twin of the NVFP4 shape (same layer, same distribution);
+    for the MXFP4 twin of the NVFP4 shape (same layer, same distribution),
+    6 for the FP8 E4M3 weight-only layer (the INT8 prefill layer's shape and
+    distribution, group 128, decode and prefill batch sizes);
   * "0.1% of entries replaced by x20 outliers" = round(0.001*N*K) distinct
     positions whose drawn value is multiplied by 20;
   * "1% of channels scaled x10" = round(0.01*K) distinct input columns of X
@@ -67,7 +70,10 @@ PREFILL = Workload("prefill_int8_g256", "int8_sym", N=8192, K=8192, Ms=(1024, 20
                    group_size=256, seed=4, x_channel_frac=0.01, x_channel_mult=10.0,
                    bias_sigma=0.01, note="compute-bound prefill, INT8 sym g256")
 
-ALL = (PR1, DECODE, CODEBOOK, NVFP4, PREFILL, MXFP4)
+FP8 = Workload("fp8_e4m3_8192", "fp8_e4m3", N=8192, K=8192, Ms=(1, 16, 1024), group_size=128,
+               seed=6, note="FP8 E4M3 weight-only, fp32 scale per 128 along K")
+
+ALL = (PR1, DECODE, CODEBOOK, NVFP4, PREFILL, MXFP4, FP8)
 BY_NAME = {w.name: w for w in ALL}
 
 
@@ -110,6 +116,8 @@ def packed_bytes(fmt: str, N: int, K: int, G: int) -> int:
         return N * K // 2 + N * (K // 16) + 4
     if fmt == "mxfp4":
         return N * K // 2 + N * (K // 32)
+    if fmt == "fp8_e4m3":
+        return N * K + 4 * N * (K // G)
     raise ValueError(fmt)
 
 

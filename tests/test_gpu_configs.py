@@ -1,4 +1,4 @@
-"""GPU parity at the six workloads' full sizes, in the launch configuration
+"""GPU parity at the seven workloads' full sizes, in the launch configuration
 the benchmark times (the same wq_linear call).  Small batches are compared
 element by element against the full oracle product; large ones on sampled
 outputs that the oracle computes one by one.  The GPU quantizer (which the
