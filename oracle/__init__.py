@@ -23,7 +23,7 @@ _lock = threading.Lock()
 _lib = None
 
 FORMATS = {"int4_sym": 0, "int4_asym": 1, "int8_sym": 2, "cb4": 3, "nvfp4": 4, "mxfp4": 5,
-           "fp8_e4m3": 6}
+           "fp8_e4m3": 6, "fp8_e5m2": 7}
 
 
 def build(force: bool = False, extra_flags=(), out_path: str | None = None,
@@ -52,6 +52,8 @@ def _declare(lib):
         "orc_e2m1_encode": ([dbl], c_int),
         "orc_e4m3_value": ([c_int], dbl),
         "orc_e4m3_encode": ([dbl], c_int),
+        "orc_e5m2_value": ([c_int], dbl),
+        "orc_e5m2_encode": ([dbl], c_int),
         "orc_quant_int_sym": ([ptr, i64, i64, c_int, c_int, ptr, ptr], c_int),
         "orc_quant_int4_asym": ([ptr, i64, i64, c_int, ptr, ptr, ptr], c_int),
         "orc_lloyd_max_gaussian": ([c_int, ptr, ptr, ptr, ptr], c_int),
@@ -59,6 +61,7 @@ def _declare(lib):
         "orc_quant_nvfp4": ([ptr, i64, i64, ptr, ptr, ptr], c_int),
         "orc_quant_mxfp4": ([ptr, i64, i64, ptr, ptr], c_int),
         "orc_quant_fp8_e4m3": ([ptr, i64, i64, c_int, ptr, ptr], c_int),
+        "orc_quant_fp8_e5m2": ([ptr, i64, i64, c_int, ptr, ptr], c_int),
         "orc_e8m0_value": ([c_int], dbl),
         "orc_dequant": ([c_int, i64, i64, c_int, ptr, ptr, ptr, ptr], c_int),
         "orc_linear": ([ptr, ptr, ptr, i64, i64, i64, ptr, ptr], c_int),
@@ -125,6 +128,12 @@ class Oracle:
     def e4m3_encode(self, d: float) -> int:
         return int(self.lib.orc_e4m3_encode(d))
 
+    def e5m2_value(self, code: int) -> float:
+        return float(self.lib.orc_e5m2_value(code))
+
+    def e5m2_encode(self, d: float) -> int:
+        return int(self.lib.orc_e5m2_encode(d))
+
     def e8m0_value(self, code: int) -> float:
         return float(self.lib.orc_e8m0_value(code))
 
@@ -165,10 +174,11 @@ class Oracle:
             bs = np.zeros((N, K // 32), dtype=np.uint8)
             _ok(self.lib.orc_quant_mxfp4(_p(W), N, K, _p(codes), _p(bs)), fmt)
             return codes, bs, None
-        if fmt == "fp8_e4m3":
+        if fmt in ("fp8_e4m3", "fp8_e5m2"):
             codes = np.zeros((N, K), dtype=np.uint8)
             scales = np.zeros((N, K // G), dtype=np.float32)
-            _ok(self.lib.orc_quant_fp8_e4m3(_p(W), N, K, G, _p(codes), _p(scales)), fmt)
+            fn = self.lib.orc_quant_fp8_e4m3 if fmt == "fp8_e4m3" else self.lib.orc_quant_fp8_e5m2
+            _ok(fn(_p(W), N, K, G, _p(codes), _p(scales)), fmt)
             return codes, scales, None
         raise ValueError(fmt)
 

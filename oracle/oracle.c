@@ -27,9 +27,9 @@
  *    (the OCP microscaling format definition): E2M1 values, one E8M0 scale
  *    (a power of two, 2^(e-127), e = 255 is NaN) per 32 consecutive K
  *    elements, no tensor scale.
- *  - auto-round-lib README, section 1 "Supported Data Types": FP8 (E4M3)
- *    weights with an FP32 scale, BF16 / FP32 compute (QuantLinearFP8, the
- *    FP8 weight-only linear).
+ *  - auto-round-lib README, section 1 "Supported Data Types": FP8 (E4M3,
+ *    E5M2) weights with an FP32 scale, BF16 / FP32 compute (QuantLinearFP8,
+ *    the FP8 weight-only linear).
  *
  * Readings taken where the pages are silent:
  *  - rounding of w/s to an integer: round half to even;
@@ -55,6 +55,8 @@
  *    q = E4M3_rne_satfinite(w / s) with the sign of w, -0 written as +0;
  *    an all-zero group gets s = 0 and codes 0; dq = fp32(e4m3(q) * s)
  *    (one rounding of the exact product).
+ *  - FP8 E5M2: the same with 57344 (the largest finite E5M2) in place of 448
+ *    and E5M2_rne_satfinite; dq = fp32(e5m2(q) * s).
  *  - Lloyd-Max: the 2**bits-level quantizer of N(0,1), computed by the
  *    classical fixed-point iteration (thresholds at midpoints, levels at
  *    conditional means) from a uniform start on [-3, 3], in fp64, then cast
@@ -72,6 +74,7 @@
  *              tensor scale f32 [1]
  *   mxfp4    : codes u8 [N, K/2] E2M1 nibbles; block scales u8 [N, K/32] E8M0
  *   fp8_e4m3 : codes u8 [N, K] E4M3; scales f32 [N, K/G]
+ *   fp8_e5m2 : codes u8 [N, K] E5M2; scales f32 [N, K/G]
  */
 #include <math.h>
 #include <stdint.h>
@@ -79,7 +82,7 @@
 #include <string.h>
 
 enum { ORC_INT4_SYM = 0, ORC_INT4_ASYM = 1, ORC_INT8_SYM = 2, ORC_CB4 = 3, ORC_NVFP4 = 4,
-       ORC_MXFP4 = 5, ORC_FP8_E4M3 = 6 };
+       ORC_MXFP4 = 5, ORC_FP8_E4M3 = 6, ORC_FP8_E5M2 = 7 };
 
 /* ------------------------------------------------------------------ bf16 */
 float orc_bf16_to_f32(uint16_t h) {
@@ -158,6 +161,36 @@ int orc_e4m3_encode(double d) {
     if (orc_e4m3_value(mid) <= d) lo = mid; else hi = mid;
   }
   double vl = orc_e4m3_value(lo), vh = orc_e4m3_value(hi);
+  double half = 0.5 * (vl + vh);
+  if (d < half) return lo;
+  if (d > half) return hi;
+  return (lo % 2 == 0) ? lo : hi;
+}
+
+/* ------------------------------------------------------------------ E5M2 */
+/* E5M2: 1 sign, 5 exponent (bias 15), 2 mantissa bits; exponent 0 is
+ * subnormal with spacing 2^-16; exponent 31 is infinity (m = 0) or NaN. */
+double orc_e5m2_value(int code) {
+  int s = (code >> 7) & 1, e = (code >> 2) & 31, m = code & 3;
+  double v;
+  if (e == 31) v = m ? NAN : INFINITY;
+  else if (e == 0) v = ldexp((double)m, -16);
+  else v = ldexp(1.0 + m / 4.0, e - 15);
+  return s ? -v : v;
+}
+
+/* Nearest non-negative finite E5M2 code (ties to the even code), saturating
+ * to 57344 (0x7B).  d must be >= 0. */
+int orc_e5m2_encode(double d) {
+  if (!(d > 0.0)) return 0;
+  if (d >= 57344.0) return 0x7B;
+  int lo = 0, hi = 0x7B; /* codes 0..0x7B are finite and increasing */
+  if (d >= orc_e5m2_value(hi)) return hi;
+  while (hi - lo > 1) {  /* invariant: value(lo) <= d < value(hi) */
+    int mid = (lo + hi) / 2;
+    if (orc_e5m2_value(mid) <= d) lo = mid; else hi = mid;
+  }
+  double vl = orc_e5m2_value(lo), vh = orc_e5m2_value(hi);
   double half = 0.5 * (vl + vh);
   if (d < half) return lo;
   if (d > half) return hi;
@@ -400,24 +433,25 @@ int orc_quant_mxfp4(const float* W, int64_t N, int64_t K, uint8_t* codes, uint8_
   return 0;
 }
 
-/* FP8 E4M3 weights, fp32 scale per group of G along K. */
-int orc_quant_fp8_e4m3(const float* W, int64_t N, int64_t K, int G, uint8_t* codes,
-                       float* scales) {
+/* FP8 weights (E4M3 or E5M2), fp32 scale per group of G along K. */
+static int quant_fp8(const float* W, int64_t N, int64_t K, int G, int e5m2, uint8_t* codes,
+                     float* scales) {
   if (N <= 0 || K <= 0 || G <= 0 || K % G) return 1;
+  const double fmax_code = e5m2 ? 57344.0 : 448.0;
   int64_t ng = K / G;
   for (int64_t n = 0; n < N; ++n) {
     const float* w = W + n * K;
     for (int64_t j = 0; j < ng; ++j) {
       double amax = 0.0;
       for (int64_t k = j * G; k < (j + 1) * G; ++k) amax = fmax(amax, fabs((double)w[k]));
-      float sf = (float)(amax / 448.0);
+      float sf = (float)(amax / fmax_code);
       scales[n * ng + j] = sf;
       double s = (double)sf;
       for (int64_t k = j * G; k < (j + 1) * G; ++k) {
         int q = 0;
         if (s != 0.0) {
           double r = (double)w[k] / s;
-          q = orc_e4m3_encode(fabs(r));
+          q = e5m2 ? orc_e5m2_encode(fabs(r)) : orc_e4m3_encode(fabs(r));
           if (r < 0.0 && q != 0) q |= 0x80;
         }
         codes[n * K + k] = (uint8_t)q;
@@ -425,6 +459,15 @@ int orc_quant_fp8_e4m3(const float* W, int64_t N, int64_t K, int G, uint8_t* cod
     }
   }
   return 0;
+}
+
+int orc_quant_fp8_e4m3(const float* W, int64_t N, int64_t K, int G, uint8_t* codes,
+                       float* scales) {
+  return quant_fp8(W, N, K, G, 0, codes, scales);
+}
+int orc_quant_fp8_e5m2(const float* W, int64_t N, int64_t K, int G, uint8_t* codes,
+                       float* scales) {
+  return quant_fp8(W, N, K, G, 1, codes, scales);
 }
 
 /* ------------------------------------------------------------- dequant */
@@ -471,17 +514,23 @@ static float dq_one(int fmt, int64_t K, int G, const void* codes, const void* sc
       double s = (double)((const float*)scales)[n * (K / G) + k / G];
       return (float)(orc_e4m3_value(q) * s);
     }
+    case ORC_FP8_E5M2: {
+      int q = ((const uint8_t*)codes)[n * K + k];
+      double s = (double)((const float*)scales)[n * (K / G) + k / G];
+      return (float)(orc_e5m2_value(q) * s);
+    }
   }
   return NAN;
 }
 
 static int check_fmt(int fmt, int64_t N, int64_t K, int G) {
   if (N <= 0 || K <= 0) return 1;
-  if (fmt < 0 || fmt > 6) return 1;
+  if (fmt < 0 || fmt > 7) return 1;
+  const int bytes = fmt == ORC_INT8_SYM || fmt == ORC_FP8_E4M3 || fmt == ORC_FP8_E5M2;
   if ((fmt == ORC_INT4_SYM || fmt == ORC_INT4_ASYM || fmt == ORC_INT8_SYM ||
-       fmt == ORC_FP8_E4M3) && (G <= 0 || K % G))
+       fmt == ORC_FP8_E4M3 || fmt == ORC_FP8_E5M2) && (G <= 0 || K % G))
     return 1;
-  if (fmt != ORC_INT8_SYM && fmt != ORC_FP8_E4M3 && K % 2) return 1;
+  if (!bytes && K % 2) return 1;
   if (fmt == ORC_NVFP4 && K % 16) return 1;
   if (fmt == ORC_MXFP4 && K % 32) return 1;
   return 0;

@@ -147,3 +147,35 @@ def test_e4m3_round_trip_and_saturation(orc):
 @pytest.mark.parametrize("code", [0x00, 0x38, 0x7E])
 def test_e4m3_named_points(orc, code):
     assert orc.e4m3_value(code) == {0x00: 0.0, 0x38: 1.0, 0x7E: 448.0}[code]
+
+
+def test_e5m2_values_match_torch(orc):
+    codes = np.arange(0, 256, dtype=np.uint8)
+    ref = torch.from_numpy(codes.copy()).view(torch.float8_e5m2).to(torch.float64).numpy()
+    got = np.array([orc.e5m2_value(int(c)) for c in codes])
+    fin = np.isfinite(ref)
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    assert np.array_equal(got[~np.isnan(ref)], ref[~np.isnan(ref)])   # +-inf included
+    assert orc.e5m2_value(0x7B) == 57344.0
+    assert orc.e5m2_value(0x01) == 2.0 ** -16
+    assert np.all(np.diff(got[:0x7C]) > 0)
+    assert fin.sum() == 248
+
+
+def test_e5m2_encode_matches_torch_in_range(orc):
+    rng = np.random.default_rng(6)
+    v = np.concatenate([rng.uniform(0, 57344, 3000), np.exp2(rng.uniform(-18, 15.8, 3000))])
+    v = v[v <= 57344].astype(np.float32).astype(np.float64)
+    ref = torch.from_numpy(v.astype(np.float32)).to(torch.float8_e5m2).view(torch.uint8).numpy()
+    got = np.array([orc.e5m2_encode(float(x)) for x in v], dtype=np.uint8)
+    assert np.array_equal(got, ref)
+
+
+def test_e5m2_round_trip_and_saturation(orc):
+    for c in range(0x7C):
+        assert orc.e5m2_encode(orc.e5m2_value(c)) == c
+    assert orc.e5m2_encode(57344.0) == 0x7B
+    assert orc.e5m2_encode(1e30) == 0x7B
+    assert orc.e5m2_encode(0.0) == 0
+    assert orc.e5m2_encode(2.0 ** -17) == 0       # tie between 0 and 2^-16: even code 0
+    assert orc.e5m2_encode(3 * 2.0 ** -17) == 2   # tie between codes 1 and 2: even

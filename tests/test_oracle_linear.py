@@ -108,11 +108,21 @@ def _int_case(fmt, N, K, G, rng):
         code = np.where(a == 0, 0, ((e + 7) << 3) | m) | np.where(v < 0, 0x80, 0)
         scales = np.ones((N, K // G), np.float32)
         return code.astype(np.uint8), scales, None, v.astype(np.float64)
+    if fmt == "fp8_e5m2":
+        # E5M2 codes of the integers -8..8 (exact): 2^e (1 + m/4)
+        v = rng.integers(-8, 9, size=(N, K))
+        a = np.abs(v)
+        e = np.floor(np.log2(np.maximum(a, 1))).astype(np.int64)
+        m = (a * 4 // (1 << e)) - 4
+        code = np.where(a == 0, 0, ((e + 15) << 2) | m) | np.where(v < 0, 0x80, 0)
+        scales = np.ones((N, K // G), np.float32)
+        return code.astype(np.uint8), scales, None, v.astype(np.float64)
     raise ValueError(fmt)
 
 
 @pytest.mark.parametrize("fmt,G", [("int4_sym", 64), ("int4_asym", 32), ("int8_sym", 128),
-                                   ("cb4", 0), ("nvfp4", 16), ("mxfp4", 32), ("fp8_e4m3", 64)])
+                                   ("cb4", 0), ("nvfp4", 16), ("mxfp4", 32), ("fp8_e4m3", 64),
+                                   ("fp8_e5m2", 32)])
 def test_integer_special_case(orc, fmt, G):
     """Integer X, unit scales: every partial sum is exact, so y equals an
     integer matmul done by numpy -- pins layout, nibble order and orientation."""
@@ -130,7 +140,8 @@ def test_integer_special_case(orc, fmt, G):
 
 
 @pytest.mark.parametrize("fmt,G", [("int4_sym", 64), ("int4_asym", 128), ("int8_sym", 256),
-                                   ("cb4", 0), ("nvfp4", 16), ("mxfp4", 32), ("fp8_e4m3", 128)])
+                                   ("cb4", 0), ("nvfp4", 16), ("mxfp4", 32), ("fp8_e4m3", 128),
+                                   ("fp8_e5m2", 64)])
 def test_sampled_equals_full(orc, fmt, G):
     M, N, K = 6, 32, 512
     W = synth.weight(21, N, K, sigma=0.02)

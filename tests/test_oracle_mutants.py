@@ -67,11 +67,15 @@ MUTANTS = [
     ("FP8 sign dropped",
      "if (r < 0.0 && q != 0) q |= 0x80;",
      "if (r < 0.0 && q == 0) q |= 0x80;",
-     lambda o: quant.test_fp8_e4m3_properties(o, 32)),
+     lambda o: quant.test_fp8_properties(o, 32, "fp8_e4m3")),
     ("FP8 scale from the wrong maximum",
-     "float sf = (float)(amax / 448.0);",
-     "float sf = (float)(amax / 240.0);",
-     lambda o: quant.test_fp8_e4m3_properties(o, 128)),
+     "const double fmax_code = e5m2 ? 57344.0 : 448.0;",
+     "const double fmax_code = e5m2 ? 57344.0 : 240.0;",
+     lambda o: quant.test_fp8_properties(o, 128, "fp8_e4m3")),
+    ("E5M2 exponent bias off by one",
+     "else v = ldexp(1.0 + m / 4.0, e - 15);",
+     "else v = ldexp(1.0 + m / 4.0, e - 16);",
+     lambda o: codecs.test_e5m2_values_match_torch(o)),
     ("E2M1 tie broken toward the odd code",
      "if (a == mid) { code = (i % 2 == 0) ? i : i + 1; break; }",
      "if (a == mid) { code = (i % 2 == 0) ? i + 1 : i; break; }",

@@ -269,23 +269,30 @@ def test_mxfp4_round_trip(orc):
 
 
 # ------------------------------------------------------------------ FP8 E4M3
-def _e4m3_table():
-    """value of every E4M3 code from torch's float8_e4m3fn (an independent decoder)."""
+FP8_MAX = {"fp8_e4m3": 448.0, "fp8_e5m2": 57344.0}
+
+
+def _e4m3_table(fmt="fp8_e4m3"):
+    """value of every code from torch's float8_e4m3fn / float8_e5m2 (an
+    independent decoder)."""
     import torch
-    return torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(
-        torch.float64).numpy()
+    dt = torch.float8_e4m3fn if fmt == "fp8_e4m3" else torch.float8_e5m2
+    return torch.arange(256, dtype=torch.uint8).view(dt).to(torch.float64).numpy()
 
 
 @pytest.mark.parametrize("G", [32, 128])
-def test_fp8_e4m3_properties(orc, G):
-    """Group scale within half an fp32 ulp of amax/448; every code the nearest
-    finite E4M3 value to w/s by brute force (ties to the even code), with the
-    sign of w and +0 for zero; the group maximum at +-448; all-zero groups get
-    scale 0 and code 0; dequant = fp32 of the exact product."""
+@pytest.mark.parametrize("fmt", ["fp8_e4m3", "fp8_e5m2"])
+def test_fp8_properties(orc, G, fmt):
+    """Group scale within half an fp32 ulp of amax/fmax (448 for E4M3, 57344
+    for E5M2); every code the nearest finite value to w/s by brute force
+    (ties to the even code), with the sign of w and +0 for zero; the group
+    maximum at +-fmax; all-zero groups get scale 0 and code 0; dequant = fp32
+    of the exact product."""
     from fractions import Fraction
     N, K = 24, 512
     W = _weights(N, K, seed=9)
-    codes, scales, aux = orc.quantize("fp8_e4m3", W, G)
+    fmax = FP8_MAX[fmt]
+    codes, scales, aux = orc.quantize(fmt, W, G)
     assert aux is None and codes.shape == (N, K) and scales.dtype == np.float32
     ng = K // G
     W64 = W.astype(np.float64)
@@ -295,10 +302,10 @@ def test_fp8_e4m3_properties(orc, G):
         if a == 0.0:
             assert s == 0.0 and not np.any(codes[n, j * G:(j + 1) * G])
             continue
-        exact = Fraction(a) / 448
+        exact = Fraction(a) / Fraction(fmax)
         ulp = np.spacing(np.float32(s))
         assert abs(Fraction(float(s)) - exact) <= Fraction(float(ulp)) / 2
-    tab = _e4m3_table()
+    tab = _e4m3_table(fmt)
     fin = np.array([c for c in range(256) if np.isfinite(tab[c])])
     vals = tab[fin]
     S = np.repeat(scales.astype(np.float64), G, axis=1)
@@ -315,8 +322,8 @@ def test_fp8_e4m3_properties(orc, G):
     got = codes.astype(np.int64)
     assert np.array_equal(got[live], want[live])
     gmax = np.abs(tab[got]).reshape(N, ng, G).max(-1)
-    assert np.all(gmax[amax > 0] == 448.0)
-    dq = orc.dequant("fp8_e4m3", codes, scales, None, N, K, G)
+    assert np.all(gmax[amax > 0] == fmax)
+    dq = orc.dequant(fmt, codes, scales, None, N, K, G)
     assert np.array_equal(dq, (tab[got] * S).astype(np.float32))
 
 
@@ -332,5 +339,21 @@ def test_fp8_e4m3_round_trip(orc):
     s = np.ldexp(1.0, rng.integers(-20, -5, size=(N, K // G)))
     W = (tab[q] * np.repeat(s, G, axis=1)).astype(np.float32)
     codes, scales, _ = orc.quantize("fp8_e4m3", W, G)
+    assert np.array_equal(scales.astype(np.float64), s)
+    assert np.array_equal(codes.astype(np.int64), q)
+
+
+def test_fp8_e5m2_round_trip(orc):
+    """Groups built from E5M2 values (each holding +-57344) times a power-of-two
+    scale quantize back to the same codes and scale."""
+    rng = np.random.default_rng(14)
+    N, K, G = 8, 256, 64
+    tab = _e4m3_table("fp8_e5m2")
+    fin = np.array([c for c in range(256) if np.isfinite(tab[c]) and c != 0x80])
+    q = rng.choice(fin, size=(N, K))
+    q[:, ::G] = 0x7B                   # +57344 in every group
+    s = np.ldexp(1.0, rng.integers(-30, -16, size=(N, K // G)))
+    W = (tab[q] * np.repeat(s, G, axis=1)).astype(np.float32)
+    codes, scales, _ = orc.quantize("fp8_e5m2", W, G)
     assert np.array_equal(scales.astype(np.float64), s)
     assert np.array_equal(codes.astype(np.int64), q)
