@@ -68,6 +68,8 @@ def _declare(lib):
         "orc_linear_sampled": ([c_int, i64, i64, c_int, ptr, ptr, ptr, ptr, ptr, i64, ptr, ptr,
                                 ptr, ptr], c_int),
         "orc_threads": ([], c_int),
+        "orc_silu": ([dbl], dbl),
+        "orc_swiglu": ([ptr, i64, i64, ptr], c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -211,6 +213,18 @@ class Oracle:
         b = None if bias_bits is None else np.ascontiguousarray(bias_bits, dtype=np.uint16)
         _ok(self.lib.orc_linear(_p(x_bits), _p(dq), _p(b), M, N, K, _p(y), _p(y64)), "linear")
         return y, y64
+
+    def silu(self, g: float) -> float:
+        return float(self.lib.orc_silu(g))
+
+    def swiglu(self, x2_bits: np.ndarray) -> np.ndarray:
+        """bf16 bits [M, K] of up * silu(gate) for an input [M, 2K] = [up | gate]."""
+        x2_bits = np.ascontiguousarray(x2_bits, dtype=np.uint16)
+        M, K2 = x2_bits.shape
+        assert K2 % 2 == 0
+        a = np.zeros((M, K2 // 2), dtype=np.uint16)
+        _ok(self.lib.orc_swiglu(_p(x2_bits), M, K2 // 2, _p(a)), "swiglu")
+        return a
 
     def linear_sampled(self, fmt: str, codes, scales, aux, N: int, K: int, group_size: int,
                        x_bits, bias_bits, ms, ns):

@@ -63,6 +63,11 @@
  *    to fp32.
  *  - y = sum_k x*dq accumulated in fp64 in increasing k, plus bias, rounded
  *    once to bf16 (round to nearest even).
+ *  - SwiGLU input (piper-kernels README, convrot_linear with
+ *    input_activation="swiglu"): the input row holds [up | gate], K values
+ *    each; the linear's activation is a = bf16(up * silu(gate)) with
+ *    silu(g) = g / (1 + e^-g) in fp64, rounded once to bf16 (the page's
+ *    materialized path: SwiGLU first, then the ordinary linear).
  *
  * Canonical (pre-pack) layouts, the input of the library's pack step:
  *   int4_sym : codes u8 [N, K/2] two's complement nibbles; scales bf16 [N, K/G]
@@ -563,6 +568,21 @@ int orc_linear(const uint16_t* x, const float* dq, const uint16_t* bias, int64_t
       if (y) y[m * N + n] = orc_f64_to_bf16(acc);
     }
   }
+  return 0;
+}
+
+/* SwiGLU input: a[m, k] = bf16(up * silu(gate)), up = x2[m, k],
+ * gate = x2[m, K + k]; x2 is bf16 [M, 2K]. */
+double orc_silu(double g) { return g / (1.0 + exp(-g)); }
+
+int orc_swiglu(const uint16_t* x2, int64_t M, int64_t K, uint16_t* a) {
+  if (M < 0 || K <= 0) return 1;
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t k = 0; k < K; ++k) {
+      double up = (double)orc_bf16_to_f32(x2[m * 2 * K + k]);
+      double gate = (double)orc_bf16_to_f32(x2[m * 2 * K + K + k]);
+      a[m * K + k] = orc_f64_to_bf16(up * orc_silu(gate));
+    }
   return 0;
 }
 

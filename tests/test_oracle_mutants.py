@@ -11,6 +11,7 @@ import oracle
 import test_oracle_codecs as codecs
 import test_oracle_linear as lin
 import test_oracle_quant as quant
+import test_oracle_swiglu as swiglu
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
 
@@ -76,6 +77,10 @@ MUTANTS = [
      "else v = ldexp(1.0 + m / 4.0, e - 15);",
      "else v = ldexp(1.0 + m / 4.0, e - 16);",
      lambda o: codecs.test_e5m2_values_match_torch(o)),
+    ("SwiGLU reads the gate half as up",
+     "double up = (double)orc_bf16_to_f32(x2[m * 2 * K + k]);",
+     "double up = (double)orc_bf16_to_f32(x2[m * 2 * K + K + k]);",
+     lambda o: swiglu.test_swiglu_layout_and_rounding(o)),
     ("E2M1 tie broken toward the odd code",
      "if (a == mid) { code = (i % 2 == 0) ? i : i + 1; break; }",
      "if (a == mid) { code = (i % 2 == 0) ? i + 1 : i; break; }",
