@@ -26,7 +26,7 @@
  *    16 rows by 64 (4-bit) or 32 (INT8) K elements); INT formats take
  *    group_size in {32, 64, 128, 256} with K % group_size == 0; NVFP4 has a
  *    fixed block of 16 (group_size 16 or 0), MXFP4 one of 32 (group_size 32
- *    or 0); CB4 ignores group_size; FP8_E4M3 takes the INT group sizes.
+ *    or 0); CB4 ignores group_size; the FP8 formats take the INT group sizes.
  *  - Every device pointer must be 16-byte aligned, except the NVFP4 tensor
  *    scale and the CB4 centroids (4-byte aligned).
  *
@@ -50,6 +50,7 @@
  *                 e = 255 is NaN); aux = NULL
  *   WQ_FP8_E4M3 : codes  u8 [N, K]    E4M3 (fn) bytes; scales f32 [N, K/G];
  *                 aux = NULL
+ *   WQ_FP8_E5M2 : codes  u8 [N, K]    E5M2 bytes; scales f32 [N, K/G]; aux = NULL
  * Dequantized value of element (n, k) -- what wq_dequant returns:
  *   INT4_SYM/INT8_SYM: q * s            ASYM: (q - z) * s          (exact fp32)
  *   CB4: fp32(c[idx] * norm[n])         NVFP4: fp32(e2m1(q) * e4m3(sb) * ts)
@@ -59,6 +60,10 @@
  *                                          0x7F / 0xFF, which wq_linear does
  *                                          not accept as weights: its kernels
  *                                          read them as +-480)
+ *   FP8_E5M2: fp32(e5m2(q) * s)         (one rounding; +-inf / NaN for the
+ *                                          exponent-31 codes, which wq_linear
+ *                                          does not accept either: its kernels
+ *                                          read them as finite values)
  */
 #ifndef WQ_H_
 #define WQ_H_
@@ -79,7 +84,8 @@ typedef enum {
   WQ_CB4 = 3,       /* 4-bit codebook: 16 fp32 centroids, bf16 norm per row    */
   WQ_NVFP4 = 4,     /* E2M1 values, E4M3 scale per 16, fp32 tensor scale       */
   WQ_MXFP4 = 5,     /* E2M1 values, E8M0 power-of-two scale per 32 (OCP MX)    */
-  WQ_FP8_E4M3 = 6   /* E4M3 values, fp32 scale per group (FP8 weight-only)     */
+  WQ_FP8_E4M3 = 6,  /* E4M3 values, fp32 scale per group (FP8 weight-only)     */
+  WQ_FP8_E5M2 = 7   /* E5M2 values, fp32 scale per group (FP8 weight-only)     */
 } wq_format_t;
 
 typedef enum {
@@ -138,10 +144,10 @@ int wq_dequant(int format, int64_t N, int64_t K, int group_size, const void* pac
  *   packed_w device, from wq_pack
  *   scales   device: INT formats packed group scales; CB4 row norms;
  *            NVFP4 packed E4M3 block scales; MXFP4 packed E8M0 block scales;
- *            FP8_E4M3 packed fp32 group scales
+ *            FP8 packed fp32 group scales
  *   aux      device: ASYM packed zero-points; CB4 centroids f32[16];
  *            NVFP4 tensor scale f32[1]; NULL for INT4_SYM / INT8_SYM / MXFP4 /
- *            FP8_E4M3
+ *            FP8
  *   bias     device bf16 [N], or NULL
  *   out      device bf16 [M, N] row-major; must not overlap any input
  * M == 0 is a no-op returning WQ_OK.  Asynchronous; no workspace.
@@ -164,12 +170,32 @@ int wq_linear(const void* x, const void* packed_w, const void* scales, const voi
               const void* bias, int64_t M, int64_t N, int64_t K, int format, int group_size,
               void* out, void* stream);
 
+/* The same linear with a SwiGLU input: x2 is bf16 [M, 2K], each row holding
+ * [up | gate] (K values each), and the activation is
+ *     a = bf16(up * silu(gate)),   silu(g) = g / (1 + e^-g)  (fp32, then RNE)
+ * so that Y = a . dequant(W)^T (+ bias).
+ *   workspace  device scratch for the materialized activation a (bf16
+ *              [M, K], 16-byte aligned, at least M*K*2 bytes, overlapping no
+ *              other buffer) when M > 16; ignored (may be NULL) when
+ *              M <= 16, where the decode kernel applies the step to its
+ *              staged activation slice.  Its contents are not preserved.
+ * Everything else as wq_linear (same checks, same kernels after the step).
+ * Source: piper-kernels README (convrot_linear(up_gate, weight, bias,
+ * input_activation="swiglu") computes up * silu(gate) before the linear;
+ * the input is [..., 2 * in_features]; other than for measured
+ * configurations the page materializes the SwiGLU activation and then runs
+ * the ordinary linear). */
+int wq_linear_swiglu(const void* x2, const void* packed_w, const void* scales, const void* aux,
+                     const void* bias, int64_t M, int64_t N, int64_t K, int format,
+                     int group_size, void* workspace, size_t workspace_bytes, void* out,
+                     void* stream);
+
 /* Offline round-to-nearest quantizer on the GPU: w_f32[N, K] (device) ->
  * canonical codes / scales / aux (device), bit-identical to the CPU
  * definitions listed above.  CB4 reads its 16 centroids from `aux`
  * (device f32[16], left unchanged) and writes the row norms; NVFP4 writes the
  * tensor scale into `aux`.  Synchronizes `stream` for NVFP4 (two passes).
- * FP8_E4M3 writes fp32 scales amax/448 per group.
+ * The FP8 formats write fp32 scales amax/448 (E4M3) or amax/57344 (E5M2).
  * Source: piper-kernels README "ConvRot INT8" (ConvRotInt8Tensor.from_hp
  * quantizes a dense weight, group_size=256); Mamba-2 pack helper (scale =
  * amax/qmax, round, clamp). */

@@ -19,7 +19,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libwq.so")
 
 FORMATS = {"int4_sym": 0, "int4_asym": 1, "int8_sym": 2, "cb4": 3, "nvfp4": 4, "mxfp4": 5,
-           "fp8_e4m3": 6}
+           "fp8_e4m3": 6, "fp8_e5m2": 7}
 FORMAT_NAMES = {v: k for k, v in FORMATS.items()}
 
 WQ_OK = 0
@@ -50,6 +50,8 @@ _SIGS = {
     "wq_unpack": ([_int, _i64, _i64, _int, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr], _int),
     "wq_dequant": ([_int, _i64, _i64, _int, _ptr, _ptr, _ptr, _ptr, _ptr], _int),
     "wq_linear": ([_ptr, _ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _int, _int, _ptr, _ptr], _int),
+    "wq_linear_swiglu": ([_ptr, _ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _int, _int, _ptr,
+                          ctypes.c_size_t, _ptr, _ptr], _int),
     "wq_quantize": ([_int, _i64, _i64, _int, _ptr, _ptr, _ptr, _ptr, _ptr], _int),
     "wq_lloyd_max_centroids": ([_int, ctypes.POINTER(ctypes.c_float)], _int),
     "wq_device_sm_count": ([ctypes.POINTER(ctypes.c_int)], _int),
@@ -129,6 +131,14 @@ def wq_linear(x, packed_w, scales, aux, bias, M, N, K, fmt, group_size, out, str
                           K, _fmt(fmt), group_size, _addr(out), _stream(stream)), "wq_linear")
 
 
+def wq_linear_swiglu(x2, packed_w, scales, aux, bias, M, N, K, fmt, group_size, workspace,
+                     workspace_bytes, out, stream=None):
+    _check(_lib.wq_linear_swiglu(_addr(x2), _addr(packed_w), _addr(scales), _addr(aux),
+                                 _addr(bias), M, N, K, _fmt(fmt), group_size, _addr(workspace),
+                                 int(workspace_bytes), _addr(out), _stream(stream)),
+           "wq_linear_swiglu")
+
+
 def wq_quantize(fmt, N, K, group_size, w_f32, codes, scales, aux, stream=None):
     _check(_lib.wq_quantize(_fmt(fmt), N, K, group_size, _addr(w_f32), _addr(codes),
                             _addr(scales), _addr(aux), _stream(stream)), "wq_quantize")
@@ -157,4 +167,4 @@ def wq_device_sm_count() -> int:
     return n.value
 
 
-from .api import PackedWeight, linear, pack, quantize_and_pack  # noqa: E402,F401
+from .api import PackedWeight, linear, linear_swiglu, pack, quantize_and_pack  # noqa: E402,F401

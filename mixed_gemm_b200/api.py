@@ -12,8 +12,8 @@ from dataclasses import dataclass
 
 import torch
 
-from . import (FORMATS, wq_canonical_sizes, wq_linear, wq_lloyd_max_centroids, wq_pack,
-               wq_packed_sizes, wq_quantize)
+from . import (FORMATS, wq_canonical_sizes, wq_linear, wq_linear_swiglu, wq_lloyd_max_centroids,
+               wq_pack, wq_packed_sizes, wq_quantize)
 
 
 @dataclass
@@ -106,4 +106,22 @@ def linear(x: torch.Tensor, weight: PackedWeight, bias: torch.Tensor | None = No
         yh.copy_(y, non_blocking=True)
         torch.cuda.current_stream(dev).synchronize()
         return yh.reshape(*lead, weight.N)
+    return y.reshape(*lead, weight.N)
+
+
+def linear_swiglu(x2: torch.Tensor, weight: PackedWeight, bias: torch.Tensor | None = None,
+                  out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y = (up * silu(gate)) @ dequant(weight).T + bias for ``x2`` = [..., 2K] =
+    [up | gate] (bf16, on the weight's device).  For more than 16 rows the
+    activation is materialized in a torch-allocated workspace."""
+    dev = weight.w.device
+    lead = x2.shape[:-1]
+    K = weight.K
+    assert x2.shape[-1] == 2 * K and x2.dtype == torch.bfloat16 and x2.is_cuda
+    xd = x2.reshape(-1, 2 * K).contiguous()
+    M = xd.shape[0]
+    y = out if out is not None else torch.empty((M, weight.N), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty((M, K), dtype=torch.bfloat16, device=dev) if M > 16 else None
+    wq_linear_swiglu(xd, weight.w, weight.scales, weight.aux, bias, M, weight.N, K, weight.fmt,
+                     weight.group_size, ws, 0 if ws is None else ws.numel() * 2, y, stream)
     return y.reshape(*lead, weight.N)

@@ -14,9 +14,16 @@ namespace {
 
 bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p % a) == 0; }
 
+// [p, p + pb) and [q, q + qb) intersect (a NULL pointer intersects nothing)
+bool overlap(const void* p, int64_t pb, const void* q, int64_t qb) {
+  if (!p || !q) return false;
+  const uintptr_t p0 = (uintptr_t)p, q0 = (uintptr_t)q;
+  return p0 < q0 + (uintptr_t)qb && q0 < p0 + (uintptr_t)pb;
+}
+
 // Shape / format checks shared by every entry point.
 int check_shape(int f, int64_t N, int64_t K, int G) {
-  if (f < INT4_SYM || f > FP8_E4M3) return WQ_ERR_INVALID_ARG;
+  if (f < INT4_SYM || f > FP8_E5M2) return WQ_ERR_INVALID_ARG;
   if (N <= 0 || K <= 0) return WQ_ERR_INVALID_ARG;
   if (N % 16 || K % 64) return WQ_ERR_INVALID_ARG;
   if (N > (1LL << 30) || K > (1LL << 24) || N * K > (1LL << 40)) return WQ_ERR_INVALID_ARG;
@@ -36,6 +43,29 @@ int effective_group(int f, int G) {
 }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA; }
+
+// Checks shared by the linear entry points; x holds x_cols bf16 values per row.
+int check_linear(const void* x, int64_t x_cols, const void* pw, const void* scales,
+                 const void* aux, const void* bias, int64_t M, int64_t N, int64_t K, int f,
+                 int& G, void* out) {
+  int st = check_shape(f, N, K, G);
+  if (st) return st;
+  if (M < 0 || M > (1LL << 24)) return WQ_ERR_INVALID_ARG;
+  G = effective_group(f, G);
+  bool need_aux = f == INT4_ASYM || f == CB4 || f == NVFP4;
+  if (!x || !pw || !scales || !out || (need_aux && !aux)) return WQ_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(pw, 16) || !aligned(scales, 16) || !aligned(out, 16) ||
+      (bias && !aligned(bias, 16)) || (aux && !aligned(aux, (f == INT4_ASYM) ? 16 : 4)))
+    return WQ_ERR_ALIGNMENT;
+  // the output must not overlap an input
+  size_t wb = 0, sb = 0, ab = 0;
+  wq_packed_sizes(f, N, K, G, &wb, &sb, &ab);
+  if (M > 0 && (overlap(out, M * N * 2, x, M * x_cols * 2) || overlap(out, M * N * 2, pw, wb) ||
+                overlap(out, M * N * 2, scales, sb) || overlap(out, M * N * 2, aux, ab) ||
+                overlap(out, M * N * 2, bias, N * 2)))
+    return WQ_ERR_INVALID_ARG;
+  return WQ_OK;
+}
 
 std::mutex g_sm_mutex;
 int g_sm_count[64];
@@ -84,7 +114,8 @@ int wq_canonical_sizes(int f, int64_t N, int64_t K, int G, size_t* cb, size_t* s
     case INT4_SYM: c = N * K / 2; s = 2 * N * (K / G); break;
     case INT4_ASYM: c = N * K / 2; s = 2 * N * (K / G); a = N * (K / G); break;
     case INT8_SYM: c = N * K; s = 2 * N * (K / G); break;
-    case FP8_E4M3: c = N * K; s = 4 * N * (K / G); break;
+    case FP8_E4M3:
+    case FP8_E5M2: c = N * K; s = 4 * N * (K / G); break;
     case CB4: c = N * K / 2; s = 2 * N; a = 64; break;
     case NVFP4: c = N * K / 2; s = N * (K / 16); a = 4; break;
     case MXFP4: c = N * K / 2; s = N * (K / 32); a = 0; break;
@@ -145,26 +176,8 @@ int wq_quantize(int f, int64_t N, int64_t K, int G, const float* w, void* codes,
 
 int wq_linear(const void* x, const void* pw, const void* scales, const void* aux, const void* bias,
               int64_t M, int64_t N, int64_t K, int f, int G, void* out, void* stream) {
-  int st = check_shape(f, N, K, G);
+  int st = check_linear(x, K, pw, scales, aux, bias, M, N, K, f, G, out);
   if (st) return st;
-  if (M < 0 || M > (1LL << 24)) return WQ_ERR_INVALID_ARG;
-  G = effective_group(f, G);
-  bool need_aux = f == INT4_ASYM || f == CB4 || f == NVFP4;
-  if (!x || !pw || !scales || !out || (need_aux && !aux)) return WQ_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(pw, 16) || !aligned(scales, 16) || !aligned(out, 16) ||
-      (bias && !aligned(bias, 16)) || (aux && !aligned(aux, (f == INT4_ASYM) ? 16 : 4)))
-    return WQ_ERR_ALIGNMENT;
-  // the output must not overlap an input
-  const uintptr_t o0 = (uintptr_t)out, o1 = o0 + (uintptr_t)(M * N * 2);
-  auto overlaps = [&](const void* p, uintptr_t bytes) {
-    uintptr_t a0 = (uintptr_t)p, a1 = a0 + bytes;
-    return p && a0 < o1 && o0 < a1;
-  };
-  size_t wb = 0, sb = 0, ab = 0;
-  wq_packed_sizes(f, N, K, G, &wb, &sb, &ab);
-  if (M > 0 && (overlaps(x, (uintptr_t)(M * K * 2)) || overlaps(pw, wb) || overlaps(scales, sb) ||
-                overlaps(aux, ab) || overlaps(bias, (uintptr_t)(N * 2))))
-    return WQ_ERR_INVALID_ARG;
   if (M == 0) return WQ_OK;
   LinearArgs a;
   a.x = x;
@@ -186,6 +199,48 @@ int wq_linear(const void* x, const void* pw, const void* scales, const void* aux
     e = launch_prefill(a);
   }
   return cuda_status(e);
+}
+
+int wq_linear_swiglu(const void* x2, const void* pw, const void* scales, const void* aux,
+                     const void* bias, int64_t M, int64_t N, int64_t K, int f, int G,
+                     void* workspace, size_t workspace_bytes, void* out, void* stream) {
+  int st = check_linear(x2, 2 * K, pw, scales, aux, bias, M, N, K, f, G, out);
+  if (st) return st;
+  const bool decode = M <= 16;
+  if (!decode) {
+    // the materialized activation [M, K] bf16 lives in the caller's workspace
+    if (!workspace || workspace_bytes < (size_t)(M * K * 2)) return WQ_ERR_INVALID_ARG;
+    if (!aligned(workspace, 16)) return WQ_ERR_ALIGNMENT;
+    size_t wb = 0, sb = 0, ab = 0;
+    wq_packed_sizes(f, N, K, G, &wb, &sb, &ab);
+    const int64_t w = M * K * 2;
+    if (overlap(workspace, w, x2, M * 2 * K * 2) || overlap(workspace, w, out, M * N * 2) ||
+        overlap(workspace, w, pw, wb) || overlap(workspace, w, scales, sb) ||
+        overlap(workspace, w, aux, ab) || overlap(workspace, w, bias, N * 2))
+      return WQ_ERR_INVALID_ARG;
+  }
+  if (M == 0) return WQ_OK;
+  LinearArgs a;
+  a.x = x2;
+  a.w = pw;
+  a.scales = scales;
+  a.aux = aux;
+  a.bias = bias;
+  a.out = out;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.fmt = f;
+  a.G = G;
+  a.stream = (cudaStream_t)stream;
+  if (decode) {
+    a.swiglu = true;
+    return cuda_status(launch_decode(a));
+  }
+  cudaError_t e = launch_swiglu(x2, M, K, workspace, a.stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  a.x = workspace;
+  return cuda_status(launch_prefill(a));
 }
 
 // Lloyd-Max quantizer of N(0,1): thresholds at the midpoints of adjacent

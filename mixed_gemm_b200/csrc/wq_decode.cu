@@ -55,6 +55,8 @@ struct DecodeParams {
   int red_off;    // offset of the cluster partial slots (after the larger of
                   // the staged data and the per-warp partials)
   int bar_off;    // offset of the mbarrier the X-slice bulk copies complete on
+  int swiglu;     // x rows are [up | gate] (2K values); the gate slice is
+                  // staged at xs_bytes past the up slice
 };
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
@@ -126,6 +128,15 @@ __device__ __forceinline__ uint2 lds64(uint32_t addr) {
   asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
   return v;
 }
+__device__ __forceinline__ void sts128(uint32_t addr, const uint4& v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ uint4 swiglu_x8(const uint4& u, const uint4& g) {
+  return make_uint4(swiglu_pair(u.x, g.x), swiglu_pair(u.y, g.y), swiglu_pair(u.z, g.z),
+                    swiglu_pair(u.w, g.w));
+}
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -150,14 +161,15 @@ __device__ __forceinline__ void cluster_sync_all() {
 // issued into the freed registers.
 template <int FMT, int NT, int RT, int KW, int D>
 __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
-  constexpr bool kByte = FMT == INT8_SYM || FMT == FP8_E4M3;  // one byte per code
+  constexpr bool kFp8 = FMT == FP8_E4M3 || FMT == FP8_E5M2;
+  constexpr bool kByte = FMT == INT8_SYM || kFp8;  // one byte per code
   constexpr int KB = kByte ? 32 : 64;             // K per 512-byte block
   constexpr int CPB = kByte ? 1 : 2;              // 32-K chunks per block
   constexpr int NV = RT * NT * 4;                  // accumulators per lane
   // one scale per group of K folded into fp32 sums (INT formats, FP8)
   constexpr bool kIntFmt =
-      FMT == INT4_SYM || FMT == INT4_ASYM || FMT == INT8_SYM || FMT == FP8_E4M3;
-  constexpr int SB = FMT == FP8_E4M3 ? 64 : 32;   // bytes per (row tile, group) of scales
+      FMT == INT4_SYM || FMT == INT4_ASYM || FMT == INT8_SYM || kFp8;
+  constexpr int SB = kFp8 ? 64 : 32;   // bytes per (row tile, group) of scales
 
   extern __shared__ __align__(16) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -193,7 +205,7 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   // [cb*KB, ce*KB)), and the group scales + zero-points (INT) or E4M3 block
   // scales (NVFP4) of its row tiles over that K range.
   const uint32_t xs = (uint32_t)__cvta_generic_to_shared(smem);
-  const uint32_t side = xs + (uint32_t)p.xs_bytes;
+  const uint32_t side = xs + (uint32_t)p.xs_bytes * (p.swiglu ? 2u : 1u);
   const int kbeg = cb * KB;
   const int g_begin = kIntFmt ? kbeg >> p.gshift : 0;  // first scale group staged
   const int b16_begin = kbeg >> 4;                      // first NVFP4 16-block staged
@@ -251,13 +263,18 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   // one's compute).  One bulk copy per token row stages the X slice.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int64_t xrow = p.swiglu ? 2 * (int64_t)K : (int64_t)K;  // elements per x row
   if (threadIdx.x == 0) {
     const uint32_t xbytes = (uint32_t)((ce - cb) * KB * 2);
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(xbar),
-                 "r"(xbytes * (uint32_t)p.M)
+                 "r"(xbytes * (uint32_t)p.M * (p.swiglu ? 2u : 1u))
                  : "memory");
-    for (int tok = 0; tok < p.M; ++tok)
-      bulk_g2s(xs + tok * p.xs_stride, p.x + (int64_t)tok * K + kbeg, xbytes, xbar);
+    for (int tok = 0; tok < p.M; ++tok) {
+      bulk_g2s(xs + tok * p.xs_stride, p.x + tok * xrow + kbeg, xbytes, xbar);
+      if (p.swiglu)
+        bulk_g2s(xs + p.xs_bytes + tok * p.xs_stride, p.x + tok * xrow + K + kbeg, xbytes,
+                 xbar);
+    }
   }
 
   // NVFP4: a 256-entry table E4M3 code -> bf16x2 (e4m3 * 2^119) pair, the
@@ -318,6 +335,17 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   cp_async_wait_all();
   __syncthreads();  // staged scales, the NVFP4 table and the barrier init are visible
   const bool xok = mbar_wait0(xbar);  // false never in practice: then nothing is stored
+  if (p.swiglu) {
+    // SwiGLU input: a = bf16(up * silu(gate)), written over the staged up slice
+    const int chunks = (ce - cb) * KB / 8;  // 16-byte chunks per token row
+    for (int i = threadIdx.x; i < p.M * chunks; i += KW * 32) {
+      const int tok = i / chunks, c = i - tok * chunks;
+      const uint32_t ua = xs + (uint32_t)(tok * p.xs_stride + c * 16);
+      const uint4 u = lds128(ua), gt = lds128(ua + (uint32_t)p.xs_bytes);
+      sts128(ua, swiglu_x8(u, gt));
+    }
+    __syncthreads();
+  }
 
   const uint4 zero4 = make_uint4(0, 0, 0, 0);
   auto compute_block = [&](const uint4 (&wb_)[RT], int b) {
@@ -345,7 +373,7 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
           const int gi = (k0 >> p.gshift) - g_begin;
 #pragma unroll
           for (int r = 0; r < RT; ++r) {
-            if constexpr (FMT == FP8_E4M3) {  // fp32 scales of rows g, g + 8
+            if constexpr (kFp8) {  // fp32 scales of rows g, g + 8
               const uint2 sv = lds64(side + (r * p.side_rows + gi) * 64 + g * 8);
               gsw[r] = sv.x;
               gsw2[r] = sv.y;
@@ -377,6 +405,8 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
               frag_int8(word(wb_[r], 2 * s), word(wb_[r], 2 * s + 1), a);
             else if constexpr (FMT == FP8_E4M3)
               frag_e4m3(word(wb_[r], 2 * s), word(wb_[r], 2 * s + 1), a);
+            else if constexpr (FMT == FP8_E5M2)
+              frag_e5m2(word(wb_[r], 2 * s), word(wb_[r], 2 * s + 1), a);
             else
               frag_int4(word(wb_[r], 2 * c + s), goff[r][0], goff[r][1], a);
 #pragma unroll
@@ -386,8 +416,8 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
           }
           if (gend) {
             const float s_g =
-                FMT == FP8_E4M3 ? __uint_as_float(gsw[r]) : __uint_as_float(gsw[r] << 16);
-            const float s_g8 = FMT == FP8_E4M3 ? __uint_as_float(gsw2[r])
+                kFp8 ? __uint_as_float(gsw[r]) : __uint_as_float(gsw[r] << 16);
+            const float s_g8 = kFp8 ? __uint_as_float(gsw2[r])
                                                : __uint_as_float(gsw[r] & 0xFFFF0000u);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
@@ -596,7 +626,8 @@ cudaError_t launch_decode(const LinearArgs& a) {
 #endif
   const int64_t max_blocks = (nblk + cs - 1) / cs;
   const int64_t stride = ((max_blocks * kb * 2 + 127) / 128) * 128 + 64;
-  if (stride * a.M > 200 * 1024) return cudaErrorInvalidValue;  // K too large for M <= 16
+  // K too large for M <= 16 (the SwiGLU input stages up and gate)
+  if (stride * a.M * (a.swiglu ? 2 : 1) > 200 * 1024) return cudaErrorInvalidValue;
   p.cs = (int)cs;
   p.xs_stride = (int)stride;
   p.xs_bytes = (int)(stride * a.M);
@@ -606,7 +637,7 @@ cudaError_t launch_decode(const LinearArgs& a) {
   if (is_grouped_fmt(a.fmt)) {
     while ((1 << p.gshift) < a.G) ++p.gshift;
     p.side_rows = (int)((max_blocks * kb + a.G - 1) / a.G + 1);
-    p.side_bytes = rt * p.side_rows * (a.fmt == INT4_ASYM ? 40 : a.fmt == FP8_E4M3 ? 64 : 32);
+    p.side_bytes = rt * p.side_rows * (a.fmt == INT4_ASYM ? 40 : is_fp8(a.fmt) ? 64 : 32);
   } else if (a.fmt == NVFP4 || a.fmt == MXFP4) {
     p.side_rows = (int)(max_blocks * kb / (a.fmt == NVFP4 ? 16 : 32));
     p.side_bytes = rt * p.side_rows * 16 + 1024;  // block scales + code table
@@ -616,7 +647,8 @@ cudaError_t launch_decode(const LinearArgs& a) {
   }
   p.side_bytes = (p.side_bytes + 15) & ~15;
   const int64_t warp_partials = 4LL * rt * nt * 4 * 32 * 4;  // KW = 4 warps
-  int64_t region = p.xs_bytes + p.side_bytes;
+  p.swiglu = a.swiglu ? 1 : 0;
+  int64_t region = (int64_t)p.xs_bytes * (a.swiglu ? 2 : 1) + p.side_bytes;
   if (region < warp_partials) region = warp_partials;
   p.red_off = (int)((region + 15) & ~15LL);
   p.bar_off = (int)(p.red_off + cs * rt * nt * 4 * 32 * 4);
@@ -630,6 +662,7 @@ cudaError_t launch_decode(const LinearArgs& a) {
     case NVFP4: return launch_fmt<NVFP4>(p, nt, rt, grid, a.stream);
     case MXFP4: return launch_fmt<MXFP4>(p, nt, rt, grid, a.stream);
     case FP8_E4M3: return launch_fmt<FP8_E4M3>(p, nt, rt, grid, a.stream);
+    case FP8_E5M2: return launch_fmt<FP8_E5M2>(p, nt, rt, grid, a.stream);
   }
   return cudaErrorInvalidValue;
 }

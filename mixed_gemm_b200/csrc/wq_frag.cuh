@@ -73,6 +73,21 @@ static __device__ __forceinline__ void frag_e4m3(uint32_t wg, uint32_t wg8, uint
   a[3] = bmul2(e4m3x2_scaled_bits(__byte_perm(wg8, 0u, 0x3424u)), k120);
 }
 
+// FP8 E5M2 bytes -> exact bf16 fragments, as frag_e4m3: the 7 magnitude bits
+// at bits 5..11 read as e5m2 * 2^-112 (subnormals included), restored by an
+// exact multiply by 2^112.  The infinity / NaN codes (exponent 31) come out
+// as finite values of magnitude 2^16 (1 + m/4).
+static __device__ __forceinline__ uint32_t e5m2x2_scaled_bits(uint32_t t8) {
+  return ((t8 >> 3) & 0x0FE00FE0u) | (t8 & 0x80008000u);
+}
+static __device__ __forceinline__ void frag_e5m2(uint32_t wg, uint32_t wg8, uint32_t (&a)[4]) {
+  const uint32_t k112 = 0x77807780u;  // bf16x2 (2^112, 2^112)
+  a[0] = bmul2(e5m2x2_scaled_bits(__byte_perm(wg, 0u, 0x1404u)), k112);
+  a[1] = bmul2(e5m2x2_scaled_bits(__byte_perm(wg8, 0u, 0x1404u)), k112);
+  a[2] = bmul2(e5m2x2_scaled_bits(__byte_perm(wg, 0u, 0x3424u)), k112);
+  a[3] = bmul2(e5m2x2_scaled_bits(__byte_perm(wg8, 0u, 0x3424u)), k112);
+}
+
 // 16-entry bf16 lookup ("table" nibble order): byte tables H (high bytes) and
 // L (low bytes), four entries per register.  `kSymLow` means the low-byte
 // table does not depend on the top index bit (true for E2M1).
@@ -142,6 +157,16 @@ static __device__ __forceinline__ uint32_t mx_lo_pair(uint32_t e) {
 }
 static __device__ __forceinline__ uint32_t mx_hi_pair(uint32_t e) {
   return ((e - 128u + 127u) << 7) * 0x00010001u;  // 2^(e - 128), e in 129..254
+}
+
+// SwiGLU input: bf16 pairs up * silu(gate), silu(g) = g / (1 + e^-g), in
+// fp32 (fast exponential; the result is rounded to bf16, nearest even)
+static __device__ __forceinline__ uint32_t swiglu_pair(uint32_t u, uint32_t g) {
+  const float u0 = __uint_as_float(u << 16), u1 = __uint_as_float(u & 0xFFFF0000u);
+  const float g0 = __uint_as_float(g << 16), g1 = __uint_as_float(g & 0xFFFF0000u);
+  const float a0 = u0 * (g0 / (1.f + __expf(-g0)));
+  const float a1 = u1 * (g1 / (1.f + __expf(-g1)));
+  return pack_bf16x2(a0, a1);
 }
 
 }  // namespace wq

@@ -4,7 +4,7 @@
 // --------------------------------------------------------
 // Rows are grouped in tiles of 16 (n = 16*tile + r, r = g + 8*hr, g = 0..7,
 // hr = 0/1).  Along K a tile is cut into blocks of 512 bytes: 64 K elements
-// for 4-bit codes, 32 for byte codes (INT8, FP8 E4M3).  Inside a block, lane L = 4*g + tq of a warp
+// for 4-bit codes, 32 for byte codes (INT8, FP8).  Inside a block, lane L = 4*g + tq of a warp
 // owns 16 contiguous bytes: the codes of rows g and g+8 for K offsets
 // {32c + 8tq + 4s + e : c, s in {0,1} (4-bit) or c = 0 (bytes), e = 0..3}.
 // One 16-byte load per lane therefore yields exactly the A-operand fragments
@@ -21,12 +21,12 @@
 //        low/high 16 bits hold registers {0,1} / {2,3} as four nibbles each,
 //        ready for byte-permute table lookups.
 //   INT4_SYM nibbles are stored offset-binary (v + 8); INT8 bytes likewise
-//   (v + 128), word j = 2s + hr, byte e; FP8 E4M3 bytes as they are, at the
-//   INT8 positions.
+//   (v + 128), word j = 2s + hr, byte e; FP8 (E4M3, E5M2) bytes as they
+//   are, at the INT8 positions.
 //
 // Scales (INT formats):  bf16 [N/16][K/G][16], entry 2g + hr (so lane g
 //   reads rows g and g+8 as one 32-bit word).
-// Scales (FP8 E4M3):     f32 [N/16][K/G][16], entry 2g + hr (one 64-bit word).
+// Scales (FP8):          f32 [N/16][K/G][16], entry 2g + hr (one 64-bit word).
 // Zero-points (ASYM):    u8 [N/16][K/G][8], byte g = z(row g) | z(row g+8) << 4.
 // NVFP4 block scales:    u8 [N/16][K/16][16], entry 2g + hr.
 // MXFP4 block scales:    u8 [N/16][K/32][16], entry 2g + hr.
@@ -43,14 +43,13 @@
 namespace wq {
 
 enum Fmt { INT4_SYM = 0, INT4_ASYM = 1, INT8_SYM = 2, CB4 = 3, NVFP4 = 4, MXFP4 = 5,
-           FP8_E4M3 = 6 };
+           FP8_E4M3 = 6, FP8_E5M2 = 7 };
 
 __host__ __device__ inline bool is_int_fmt(int f) { return f == INT4_SYM || f == INT4_ASYM || f == INT8_SYM; }
 // formats with one scale per group of G along K, folded into fp32 sums
-__host__ __device__ inline bool is_grouped_fmt(int f) { return is_int_fmt(f) || f == FP8_E4M3; }
-__host__ __device__ inline bool is_4bit(int f) { return f != INT8_SYM && f != FP8_E4M3; }
-// bytes of one packed group scale
-__host__ __device__ inline int scale_bytes(int f) { return f == FP8_E4M3 ? 4 : 2; }
+__host__ __device__ inline bool is_fp8(int f) { return f == FP8_E4M3 || f == FP8_E5M2; }
+__host__ __device__ inline bool is_grouped_fmt(int f) { return is_int_fmt(f) || is_fp8(f); }
+__host__ __device__ inline bool is_4bit(int f) { return f != INT8_SYM && !is_fp8(f); }
 // elements of K per 512-byte block
 __host__ __device__ inline int block_k(int f) { return is_4bit(f) ? 64 : 32; }
 
@@ -105,6 +104,16 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
   return s ? -v : v;
 }
 
+// E5M2 code -> fp32, exact for all 256 codes (exponent 31: +-inf, NaN).
+__device__ __forceinline__ float e5m2_to_f32(uint32_t c) {
+  uint32_t s = (c >> 7) & 1u, e = (c >> 2) & 31u, m = c & 3u;
+  float v;
+  if (e == 31u) v = m ? __uint_as_float(0x7FC00000u) : __uint_as_float(0x7F800000u);
+  else if (e == 0u) v = (float)m * 1.52587890625e-05f;  // m * 2^-16
+  else v = __uint_as_float(((e + 112u) << 23) | (m << 21));
+  return s ? -v : v;
+}
+
 // E8M0 (a power of two, 2^(c - 127)) -> fp32, exact; 255 -> NaN, 0 -> the
 // fp32 subnormal 2^-127.
 __device__ __forceinline__ float e8m0_to_f32(uint32_t c) {
@@ -124,9 +133,14 @@ struct LinearArgs {
   int64_t M, N, K;
   int fmt, G;
   cudaStream_t stream;
+  // x holds rows [up | gate] of 2K values; the activation is up * silu(gate)
+  // (decode path only: the prefill path reads a materialized activation)
+  bool swiglu = false;
 };
 
 cudaError_t launch_decode(const LinearArgs& a);
+// a[m, k] = bf16(up * silu(gate)) for x2 rows [up | gate], bf16 [M, 2K] -> [M, K]
+cudaError_t launch_swiglu(const void* x2, int64_t M, int64_t K, void* a, cudaStream_t st);
 cudaError_t launch_prefill(const LinearArgs& a);
 int device_sm_count();
 // The kernels' own error word (bit per failed bounded wait); synchronous read.

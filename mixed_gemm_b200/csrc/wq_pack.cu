@@ -172,9 +172,9 @@ __global__ void dequant_kernel(int f, int64_t N, int64_t K, int G, const uint8_t
       int z = (((const uint8_t*)pa)[zb] >> zs) & 15;
       float s = bf16_bits_to_f32(((const uint16_t*)ps)[packed_scale_idx(n, k / G, K / G)]);
       v = (float)((int)raw - z) * s;
-    } else if (f == FP8_E4M3) {  // one rounding of the exact e4m3 * s
+    } else if (is_fp8(f)) {  // one rounding of the exact fp8 * s
       float s = ((const float*)ps)[packed_scale_idx(n, k / G, K / G)];
-      v = __fmul_rn(e4m3_to_f32(raw), s);
+      v = __fmul_rn(f == FP8_E4M3 ? e4m3_to_f32(raw) : e5m2_to_f32(raw), s);
     } else if (f == CB4) {
       float c = ((const float*)pa)[raw];
       float nr = bf16_bits_to_f32(((const uint16_t*)ps)[n]);
@@ -201,7 +201,7 @@ cudaError_t launch_pack(int f, int64_t N, int64_t K, int G, const void* codes, c
   const int64_t wbytes = is_4bit(f) ? N * K / 2 : N * K;
   pack_w_kernel<<<grid_for(wbytes), kThreads, 0, st>>>(f, N, K, (const uint8_t*)codes,
                                                         (uint8_t*)pw);
-  if (f == FP8_E4M3) {
+  if (is_fp8(f)) {
     int64_t groups = K / G;
     permute_scales_kernel<uint32_t><<<grid_for(N * groups), kThreads, 0, st>>>(
         N, groups, (const uint32_t*)scales, (uint32_t*)ps, true);
@@ -230,7 +230,7 @@ cudaError_t launch_unpack(int f, int64_t N, int64_t K, int G, const void* pw, co
   const int64_t wbytes = is_4bit(f) ? N * K / 2 : N * K;
   unpack_w_kernel<<<grid_for(wbytes), kThreads, 0, st>>>(f, N, K, (const uint8_t*)pw,
                                                           (uint8_t*)codes);
-  if (f == FP8_E4M3) {
+  if (is_fp8(f)) {
     int64_t groups = K / G;
     permute_scales_kernel<uint32_t><<<grid_for(N * groups), kThreads, 0, st>>>(
         N, groups, (const uint32_t*)ps, (uint32_t*)scales, false);

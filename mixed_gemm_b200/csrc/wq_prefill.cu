@@ -245,8 +245,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const PrefillParams p) {
   // one scale per group of K, folded into fp32 sums (INT formats, FP8)
   constexpr bool kInt =
-      FMT == INT4_SYM || FMT == INT4_ASYM || FMT == INT8_SYM || FMT == FP8_E4M3;
-  constexpr bool kByte = FMT == INT8_SYM || FMT == FP8_E4M3;  // one byte per code
+      FMT == INT4_SYM || FMT == INT4_ASYM || FMT == INT8_SYM || FMT == FP8_E4M3 || FMT == FP8_E5M2;
+  constexpr bool kFp8 = FMT == FP8_E4M3 || FMT == FP8_E5M2;
+  constexpr bool kByte = FMT == INT8_SYM || kFp8;  // one byte per code
   constexpr uint32_t kWpk = kByte ? 8192u : 4096u;  // packed bytes per stage
   // A stage: one 128 x 64 bf16 tile; CB4 adds a second tile holding the
   // bf16 remainders of its centroids (two MMAs per K step)
@@ -476,6 +477,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if constexpr (FMT == FP8_E4M3) {
               frag_e4m3(ch.x, ch.y, a);
               frag_e4m3(ch.z, ch.w, b);
+            } else if constexpr (FMT == FP8_E5M2) {
+              frag_e5m2(ch.x, ch.y, a);
+              frag_e5m2(ch.z, ch.w, b);
             } else {
               frag_int8(ch.x, ch.y, a);
               frag_int8(ch.z, ch.w, b);
@@ -569,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int gfirst = kInt ? (kt0 * 64) / p.G : 0;  // first group of this CTA's K range
     auto group_scale = [&](int gi) -> uint32_t {
       if (!(kInt && nvalid && gi < NG)) return 0u;
-      if constexpr (FMT == FP8_E4M3) return __ldg(srow32 + sidx + (int64_t)(gfirst + gi) * 16);
+      if constexpr (kFp8) return __ldg(srow32 + sidx + (int64_t)(gfirst + gi) * 16);
       return (uint32_t)__ldg(srow + sidx + (int64_t)(gfirst + gi) * 16);
     };
     uint32_t sc0 = group_scale(0), sc1 = group_scale(1);
@@ -589,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = mbar_wait(gfull_bar(gb), (uint32_t)(g >> 1) & 1u, abort, 64u);
       if (!__all_sync(0xffffffffu, ok ? 1 : 0)) { ok = false; break; }
       tc_fence_after();
-      const float sc = FMT == FP8_E4M3 ? __uint_as_float(sc0)
+      const float sc = kFp8 ? __uint_as_float(sc0)
                        : kInt          ? bf16_bits_to_f32((uint16_t)sc0)
                                        : 1.f;
       sc0 = sc1;
@@ -688,7 +692,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 template <int FMT, int BN>
 cudaError_t launch_bn(const LinearArgs& a) {
-  constexpr uint32_t kWpk = (FMT == INT8_SYM || FMT == FP8_E4M3) ? 8192u : 4096u;
+  constexpr uint32_t kWpk = (FMT == INT8_SYM || FMT == FP8_E4M3 || FMT == FP8_E5M2) ? 8192u : 4096u;
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
   CUtensorMap tmX, tmW;
@@ -831,6 +835,7 @@ cudaError_t launch_prefill(const LinearArgs& a) {
     case NVFP4: return launch_fmt<NVFP4>(a, BN);
     case MXFP4: return launch_fmt<MXFP4>(a, BN);
     case FP8_E4M3: return launch_fmt<FP8_E4M3>(a, BN);
+    case FP8_E5M2: return launch_fmt<FP8_E5M2>(a, BN);
   }
   return cudaErrorInvalidValue;
 }

@@ -50,6 +50,23 @@ __device__ __forceinline__ uint32_t e4m3_encode_rn_satfinite(double d) {
   return ((uint32_t)(ev + 7) << 3) | m;
 }
 
+// nearest E5M2 code (sign clear), ties to even, saturating at 57344
+__device__ __forceinline__ uint32_t e5m2_encode_rn_satfinite(double d) {
+  if (!(d > 0.0)) return 0u;
+  if (d >= 57344.0) return 0x7Bu;
+  // quantum of the binade containing d (subnormal spacing 2^-16 below 2^-14)
+  int e = ilogb(d);
+  if (e < -14) e = -14;
+  double q = ldexp(1.0, e - 2);
+  double r = rint(d / q);  // exact division by a power of two
+  double v = r * q;        // representable candidate (may equal 2^(e+1))
+  if (v >= 57344.0) return 0x7Bu;
+  if (v < 6.103515625e-05) return (uint32_t)(v * 65536.0);  // m in 0..4 (4 == 2^-14 encodes as 0x04)
+  int ev = ilogb(v);
+  uint32_t m = (uint32_t)((v / ldexp(1.0, ev) - 1.0) * 4.0);
+  return ((uint32_t)(ev + 15) << 2) | m;
+}
+
 // nearest E2M1 code, ties to even, saturating at 6; zero is +0
 __device__ __forceinline__ uint32_t e2m1_encode_rn_sat(double r) {
   double a = fabs(r);
@@ -106,9 +123,11 @@ __global__ void quant_sym_kernel(int bits, int64_t N, int64_t K, int G,
   }
 }
 
-// One warp per (row, group): FP8 E4M3 codes, fp32 scale = amax / 448.
-__global__ void quant_fp8_kernel(int64_t N, int64_t K, int G, const float* __restrict__ w,
-                                 uint8_t* __restrict__ codes, float* __restrict__ scales) {
+// One warp per (row, group): FP8 codes, fp32 scale = amax / (largest finite
+// value: 448 for E4M3, 57344 for E5M2).
+__global__ void quant_fp8_kernel(int64_t N, int64_t K, int G, bool e5m2,
+                                 const float* __restrict__ w, uint8_t* __restrict__ codes,
+                                 float* __restrict__ scales) {
   const int lane = threadIdx.x & 31;
   const int64_t groups = K / G;
   for (int64_t item = blockIdx.x * (int64_t)kWarps + (threadIdx.x >> 5); item < N * groups;
@@ -118,14 +137,14 @@ __global__ void quant_fp8_kernel(int64_t N, int64_t K, int G, const float* __res
     double amax = 0.0;
     for (int i = lane; i < G; i += 32) amax = fmax(amax, fabs((double)wg[i]));
     for (int o = 16; o; o >>= 1) amax = fmax(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const float sf = __double2float_rn(__ddiv_rn(amax, 448.0));
+    const float sf = __double2float_rn(__ddiv_rn(amax, e5m2 ? 57344.0 : 448.0));
     const double s = (double)sf;
     if (lane == 0) scales[item] = sf;
     for (int i = lane; i < G; i += 32) {
       uint32_t q = 0;
       if (s != 0.0) {
         const double r = __ddiv_rn((double)wg[i], s);
-        q = e4m3_encode_rn_satfinite(fabs(r));
+        q = e5m2 ? e5m2_encode_rn_satfinite(fabs(r)) : e4m3_encode_rn_satfinite(fabs(r));
         if (r < 0.0 && q != 0u) q |= 0x80u;
       }
       codes[n * K + grp * G + i] = (uint8_t)q;
@@ -309,8 +328,9 @@ cudaError_t launch_quantize(int f, int64_t N, int64_t K, int G, const float* w, 
           f == INT4_SYM ? 4 : 8, N, K, G, w, (uint8_t*)codes, (uint16_t*)scales);
       break;
     case FP8_E4M3:
+    case FP8_E5M2:
       quant_fp8_kernel<<<blocks_for(N * (K / G), kWarps), kWarps * 32, 0, st>>>(
-          N, K, G, w, (uint8_t*)codes, (float*)scales);
+          N, K, G, f == FP8_E5M2, w, (uint8_t*)codes, (float*)scales);
       break;
     case INT4_ASYM:
       quant_asym_kernel<<<blocks_for(N * (K / G), kWarps), kWarps * 32, 0, st>>>(

@@ -116,7 +116,7 @@ def packed_bytes(fmt: str, N: int, K: int, G: int) -> int:
         return N * K // 2 + N * (K // 16) + 4
     if fmt == "mxfp4":
         return N * K // 2 + N * (K // 32)
-    if fmt == "fp8_e4m3":
+    if fmt in ("fp8_e4m3", "fp8_e5m2"):
         return N * K + 4 * N * (K // G)
     raise ValueError(fmt)
 

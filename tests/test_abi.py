@@ -36,7 +36,8 @@ def test_status_strings():
 
 
 @pytest.mark.parametrize("fmt,G", [("int4_sym", 64), ("int4_asym", 128), ("int8_sym", 256),
-                                   ("cb4", 0), ("nvfp4", 16), ("mxfp4", 32), ("fp8_e4m3", 128)])
+                                   ("cb4", 0), ("nvfp4", 16), ("mxfp4", 32), ("fp8_e4m3", 128),
+                                   ("fp8_e5m2", 64)])
 def test_sizes(fmt, G):
     import synth.workloads as W
     N, K = 4096, 4096
@@ -49,8 +50,9 @@ def test_sizes(fmt, G):
 
 
 BAD_SHAPES = [
-    dict(fmt=7), dict(N=0), dict(K=0), dict(N=24), dict(K=96), dict(G=48), dict(G=512),
-    dict(fmt="nvfp4", G=32), dict(fmt="mxfp4", G=16), dict(fmt=7), dict(fmt="fp8_e4m3", G=16), dict(M=-1),
+    dict(fmt=8), dict(fmt=-1), dict(N=0), dict(K=0), dict(N=24), dict(K=96), dict(G=48),
+    dict(G=512), dict(fmt="nvfp4", G=32), dict(fmt="mxfp4", G=16), dict(fmt="fp8_e4m3", G=16),
+    dict(fmt="fp8_e5m2", G=0), dict(M=-1),
 ]
 
 
@@ -104,3 +106,25 @@ def test_lloyd_max_host_matches_oracle(orc):
     _, c32, _, _ = orc.lloyd_max(16)
     assert np.max(np.abs(c.view(np.int32) - c32.view(np.int32))) <= 1
     assert np.all(np.diff(c) > 0)
+
+
+def test_linear_swiglu_rejects_bad_workspace():
+    base = 1 << 20
+    f = wqm.FORMATS["int4_sym"]
+    M, N, K, G = 64, 256, 512, 64
+    args = (base, base * 4, base * 8, None, None, M, N, K, f, G)
+    out = base * 64
+    ok_ws = base * 32
+    need = M * K * 2
+    # missing, too small, misaligned, overlapping the input or the output
+    assert wqm._lib.wq_linear_swiglu(*args, None, 0, out, 0) == wqm.WQ_ERR_INVALID_ARG
+    assert wqm._lib.wq_linear_swiglu(*args, ok_ws, need - 16, out, 0) == wqm.WQ_ERR_INVALID_ARG
+    assert wqm._lib.wq_linear_swiglu(*args, ok_ws + 8, need, out, 0) == wqm.WQ_ERR_ALIGNMENT
+    assert wqm._lib.wq_linear_swiglu(*args, base + 64, need, out, 0) == wqm.WQ_ERR_INVALID_ARG
+    assert wqm._lib.wq_linear_swiglu(*args, out - 64, need, out, 0) == wqm.WQ_ERR_INVALID_ARG
+    # the output may not overlap the [up | gate] input (2K values per row)
+    assert wqm._lib.wq_linear_swiglu(*args, ok_ws, need, base + M * K * 2, 0) == \
+        wqm.WQ_ERR_INVALID_ARG
+    # M == 0 is a no-op even without a workspace
+    assert wqm._lib.wq_linear_swiglu(base, base * 4, base * 8, None, None, 0, N, K, f, G, None, 0,
+                                     out, 0) == wqm.WQ_OK

@@ -16,7 +16,8 @@ pytestmark = pytest.mark.gpu
 
 FMT_G = [("int4_sym", 32), ("int4_sym", 64), ("int4_sym", 128), ("int4_sym", 256),
          ("int4_asym", 32), ("int4_asym", 128), ("int8_sym", 32), ("int8_sym", 256),
-         ("cb4", 0), ("nvfp4", 16), ("mxfp4", 32), ("fp8_e4m3", 32), ("fp8_e4m3", 256)]
+         ("cb4", 0), ("nvfp4", 16), ("mxfp4", 32), ("fp8_e4m3", 32), ("fp8_e4m3", 256),
+         ("fp8_e5m2", 64)]
 IDS = [f"{f}-g{g}" for f, g in FMT_G]
 
 
@@ -104,7 +105,8 @@ def _int_case(fmt, N, K, G, rng):
 
 
 @pytest.mark.parametrize("fmt,G", [("int4_sym", 64), ("int4_asym", 32), ("int8_sym", 128),
-                                   ("cb4", 0), ("nvfp4", 16), ("mxfp4", 32), ("fp8_e4m3", 64)])
+                                   ("cb4", 0), ("nvfp4", 16), ("mxfp4", 32), ("fp8_e4m3", 64),
+                                   ("fp8_e5m2", 32)])
 @pytest.mark.parametrize("M", [1, 5, 16, 40, 200])
 def test_linear_integer_bit_exact(wq, orc, fmt, G, M):
     """Integer activations and unit scales: every partial sum is exact in
@@ -168,7 +170,7 @@ EDGE = [
 
 
 @pytest.mark.parametrize("fmt", ["int4_sym", "int4_asym", "int8_sym", "cb4", "nvfp4", "mxfp4",
-                                 "fp8_e4m3"])
+                                 "fp8_e4m3", "fp8_e5m2"])
 @pytest.mark.parametrize("case", EDGE, ids=["16x64", "48x192", "32x16384"])
 def test_linear_edge_shapes(wq, orc, fmt, case):
     N, K, G, Ms = case
@@ -220,16 +222,22 @@ def test_mxfp4_every_scale_code(wq, orc, M):
 
 
 @pytest.mark.parametrize("M", [8, 40])
-def test_fp8_e4m3_every_code(wq, orc, M):
-    """Every finite E4M3 code (subnormals, +-0 and +-448 included) read through
-    the linear with one-hot activations: y[m, n] is one weight, exactly."""
+@pytest.mark.parametrize("fmt", ["fp8_e4m3", "fp8_e5m2"])
+def test_fp8_every_code(wq, orc, fmt, M):
+    """Every finite FP8 code (subnormals, +-0 and the largest value included)
+    read through the linear with one-hot activations: y[m, n] is one weight,
+    exactly (bf16 holds every E4M3 and E5M2 value)."""
     N, K, G = 256, 512, 64
     rng = np.random.default_rng(12)
-    fin = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+    if fmt == "fp8_e4m3":
+        bad = (0x7F, 0xFF)
+    else:
+        bad = tuple(c for c in range(256) if (c >> 2) & 31 == 31)
+    fin = np.array([c for c in range(256) if c not in bad], np.uint8)
     codes = fin[(np.arange(N * K) * 7 + rng.integers(0, 254)) % fin.size].reshape(N, K)
     scales = np.ldexp(1.0, rng.integers(-3, 4, size=(N, K // G))).astype(np.float32)
-    pw = pack_on_gpu(wq, "fp8_e4m3", N, K, G, codes, scales, None)
-    dq = orc.dequant("fp8_e4m3", codes, scales, None, N, K, G)
+    pw = pack_on_gpu(wq, fmt, N, K, G, codes, scales, None)
+    dq = orc.dequant(fmt, codes, scales, None, N, K, G)
     ks = (np.arange(M) * 41 + 3) % K
     xf = np.zeros((M, K))
     xf[np.arange(M), ks] = 1.0
