@@ -190,6 +190,18 @@ int wq_linear_swiglu(const void* x2, const void* packed_w, const void* scales, c
                      int group_size, void* workspace, size_t workspace_bytes, void* out,
                      void* stream);
 
+/* wq_linear_swiglu without a caller workspace: for M > 16 the activation is
+ * materialized in the library's static device scratch (16 MiB, a
+ * file-scope __device__ array reserved when the module loads), so the call
+ * allocates nothing.  M * K * 2 > 16 MiB returns WQ_ERR_UNSUPPORTED (use
+ * wq_linear_swiglu with a workspace).  The scratch is one buffer per
+ * device: calls of this entry point must not overlap in time on different
+ * streams (calls on one stream are ordered by the stream).  M <= 16 is
+ * wq_linear_swiglu itself (no scratch). */
+int wq_linear_swiglu_static(const void* x2, const void* packed_w, const void* scales,
+                            const void* aux, const void* bias, int64_t M, int64_t N, int64_t K,
+                            int format, int group_size, void* out, void* stream);
+
 /* Offline round-to-nearest quantizer on the GPU: w_f32[N, K] (device) ->
  * canonical codes / scales / aux (device), bit-identical to the CPU
  * definitions listed above.  CB4 reads its 16 centroids from `aux`

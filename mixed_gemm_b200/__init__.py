@@ -52,6 +52,8 @@ _SIGS = {
     "wq_linear": ([_ptr, _ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _int, _int, _ptr, _ptr], _int),
     "wq_linear_swiglu": ([_ptr, _ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _int, _int, _ptr,
                           ctypes.c_size_t, _ptr, _ptr], _int),
+    "wq_linear_swiglu_static": ([_ptr, _ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _int, _int, _ptr,
+                                 _ptr], _int),
     "wq_quantize": ([_int, _i64, _i64, _int, _ptr, _ptr, _ptr, _ptr, _ptr], _int),
     "wq_lloyd_max_centroids": ([_int, ctypes.POINTER(ctypes.c_float)], _int),
     "wq_device_sm_count": ([ctypes.POINTER(ctypes.c_int)], _int),
@@ -137,6 +139,13 @@ def wq_linear_swiglu(x2, packed_w, scales, aux, bias, M, N, K, fmt, group_size, 
                                  _addr(bias), M, N, K, _fmt(fmt), group_size, _addr(workspace),
                                  int(workspace_bytes), _addr(out), _stream(stream)),
            "wq_linear_swiglu")
+
+
+def wq_linear_swiglu_static(x2, packed_w, scales, aux, bias, M, N, K, fmt, group_size, out,
+                            stream=None):
+    _check(_lib.wq_linear_swiglu_static(_addr(x2), _addr(packed_w), _addr(scales), _addr(aux),
+                                        _addr(bias), M, N, K, _fmt(fmt), group_size, _addr(out),
+                                        _stream(stream)), "wq_linear_swiglu_static")
 
 
 def wq_quantize(fmt, N, K, group_size, w_f32, codes, scales, aux, stream=None):

@@ -243,6 +243,20 @@ int wq_linear_swiglu(const void* x2, const void* pw, const void* scales, const v
   return cuda_status(launch_prefill(a));
 }
 
+int wq_linear_swiglu_static(const void* x2, const void* pw, const void* scales, const void* aux,
+                            const void* bias, int64_t M, int64_t N, int64_t K, int f, int G,
+                            void* out, void* stream) {
+  if (M <= 16)
+    return wq_linear_swiglu(x2, pw, scales, aux, bias, M, N, K, f, G, nullptr, 0, out, stream);
+  int st = check_linear(x2, 2 * K, pw, scales, aux, bias, M, N, K, f, G, out);
+  if (st) return st;
+  if ((uint64_t)M * (uint64_t)K * 2u > kSwigluStaticScratchBytes) return WQ_ERR_UNSUPPORTED;
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  if (static_swiglu_scratch(&ws, &ws_bytes) != cudaSuccess) return WQ_ERR_CUDA;
+  return wq_linear_swiglu(x2, pw, scales, aux, bias, M, N, K, f, G, ws, ws_bytes, out, stream);
+}
+
 // Lloyd-Max quantizer of N(0,1): thresholds at the midpoints of adjacent
 // levels, each level the mean of N(0,1) over its cell, iterated from a
 // uniform start on [-3, 3] until no level moves by 1e-14.

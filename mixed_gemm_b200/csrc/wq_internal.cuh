@@ -141,6 +141,10 @@ struct LinearArgs {
 cudaError_t launch_decode(const LinearArgs& a);
 // a[m, k] = bf16(up * silu(gate)) for x2 rows [up | gate], bf16 [M, 2K] -> [M, K]
 cudaError_t launch_swiglu(const void* x2, int64_t M, int64_t K, void* a, cudaStream_t st);
+// address and size of the library's static device scratch for the SwiGLU
+// activation (a file-scope __device__ array; nothing is allocated)
+cudaError_t static_swiglu_scratch(void** ptr, size_t* bytes);
+constexpr size_t kSwigluStaticScratchBytes = 16u << 20;
 cudaError_t launch_prefill(const LinearArgs& a);
 int device_sm_count();
 // The kernels' own error word (bit per failed bounded wait); synchronous read.

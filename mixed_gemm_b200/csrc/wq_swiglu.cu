@@ -12,6 +12,11 @@ namespace wq {
 
 namespace {
 
+// The library's own scratch for the materialized activation of
+// wq_linear_swiglu_static: a file-scope device array (one per device,
+// reserved when the module loads), so that entry point allocates nothing.
+static __device__ __align__(256) uint8_t g_swiglu_scratch[kSwigluStaticScratchBytes];
+
 __global__ void __launch_bounds__(256) swiglu_kernel(const uint4* __restrict__ x2, int64_t M,
                                                      int64_t K8, uint4* __restrict__ a) {
   const int64_t total = M * K8;  // 16-byte chunks of the output
@@ -26,6 +31,11 @@ __global__ void __launch_bounds__(256) swiglu_kernel(const uint4* __restrict__ x
 }
 
 }  // namespace
+
+cudaError_t static_swiglu_scratch(void** ptr, size_t* bytes) {
+  *bytes = kSwigluStaticScratchBytes;
+  return cudaGetSymbolAddress(ptr, g_swiglu_scratch);
+}
 
 cudaError_t launch_swiglu(const void* x2, int64_t M, int64_t K, void* a, cudaStream_t st) {
   const int64_t K8 = K / 8;
