@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--ms", default="", help="comma list overriding the workload's batch sizes")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-context", action="store_true",
+                    help="skip the per-call percentiles and the cuBLAS bf16 context line")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle sample")
     return ap.parse_args()
@@ -171,6 +173,88 @@ def recorded_traffic(kernel_file: str, workload: str):
     if not src or not all(os.path.exists(s) for s in src) or source_hash(src) != e.get("hash"):
         return None
     return e.get("bytes_per_launch")
+
+
+def context_numbers(wl, Ms, weights, xs, bias, outs, stream, l2, device):
+    """Per batch size: per-call time over 20 replays of a 50-call graph (p50,
+    p95), one launch timed alone (median of 20), and, as a reference point
+    only, torch's bf16 F.linear (cuBLAS) on the dequantized weight held as
+    bf16, with enough copies to exceed L2."""
+    import torch
+    import torch.nn.functional as F
+
+    import mixed_gemm_b200 as wq
+    R = len(weights)
+    out = {}
+    pw0 = weights[0]
+    w32 = torch.empty((wl.N, wl.K), dtype=torch.float32, device=device)
+    wq.wq_dequant(wl.fmt, wl.N, wl.K, wl.group_size, pw0.w, pw0.scales, pw0.aux, w32, stream)
+    torch.cuda.synchronize()
+    wbf = w32.to(torch.bfloat16)
+    del w32
+    nb = wbf.numel() * 2
+    copies = max(1, min(16, -(-3 * l2 // nb)))
+    wcs = [wbf] + [wbf.clone() for _ in range(copies - 1)]
+    bias_t = None
+    if bias is not None:
+        bias_t = bias
+    for M in Ms:
+        def graph_of(fn, n):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                fn(3)
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g, stream=stream):
+                fn(n)
+            return g
+
+        def ours(n, base=[0]):
+            for i in range(n):
+                pw = weights[(base[0] + i) % R]
+                wq.wq_linear(xs[M], pw.w, pw.scales, pw.aux, bias, M, wl.N, wl.K, wl.fmt,
+                             wl.group_size, outs[M], stream)
+            base[0] += n
+
+        def ref(n, base=[0]):
+            for i in range(n):
+                F.linear(xs[M], wcs[(base[0] + i) % copies], bias_t)
+            base[0] += n
+
+        def per_call(g, n, reps):
+            ts = []
+            for _ in range(reps):
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                with torch.cuda.stream(stream):
+                    e0.record(stream)
+                    g.replay()
+                    e1.record(stream)
+                torch.cuda.synchronize()
+                ts.append(e0.elapsed_time(e1) * 1e3 / n)
+            return ts
+
+        n = 50
+        t_ours = per_call(graph_of(ours, n), n, 20)
+        singles = []
+        for _ in range(20):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                ours(1)
+                e1.record(stream)
+            torch.cuda.synchronize()
+            singles.append(e0.elapsed_time(e1) * 1e3)
+        with torch.cuda.stream(stream):
+            t_ref = per_call(graph_of(ref, n), n, 10)
+        out[str(M)] = {"per_call_us_p50": float(np.percentile(t_ours, 50)),
+                       "per_call_us_p95": float(np.percentile(t_ours, 95)),
+                       "single_launch_us": float(np.median(singles)),
+                       "cublas_bf16_linear_us": float(np.median(t_ref))}
+    del wcs, wbf
+    torch.cuda.empty_cache()
+    return {"per_M": out, "note": "cublas_bf16_linear_us: torch F.linear on the dequantized "
+                                  "weight in bf16 (a reference point, not the target)"}
 
 
 def cpu_sample(wl, Ms, rows, data):
@@ -408,6 +492,10 @@ def main():
                "h2d_bytes_per_step": sum(M * wl.K * 2 for M in Ms),
                "d2h_bytes_per_step": sum(M * wl.N * 2 for M in Ms)}
 
+    ctx = None
+    if rank == 0 and world == 1 and not args.no_context:
+        ctx = context_numbers(wl, Ms, weights, xs, bias, outs, stream, l2, device)
+
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb, _ = cpu_baseline(wl, Ms, args.cpu_seconds)
@@ -435,6 +523,7 @@ def main():
         "clocks": clk,
         "e2e": e2e,
         "cpu_baseline": cb,
+        "context": ctx,
     }
     print(json.dumps(line), flush=True)
 
