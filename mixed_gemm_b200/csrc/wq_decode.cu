@@ -544,9 +544,9 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   }
 }
 
-template <int FMT, int NT, int RT>
+template <int FMT, int NT, int RT, int KW>
 cudaError_t launch_t(const DecodeParams& p, int grid, cudaStream_t st) {
-  constexpr int KW = 4, D = 4;
+  constexpr int D = 4;
   auto kern = decode_kernel<FMT, NT, RT, KW, D>;
   const size_t smem = (size_t)p.bar_off + 16;
   static bool attr_set = false;
@@ -573,16 +573,22 @@ cudaError_t launch_t(const DecodeParams& p, int grid, cudaStream_t st) {
   return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
-template <int FMT>
-cudaError_t launch_fmt(const DecodeParams& p, int nt, int rt, int grid, cudaStream_t st) {
+template <int FMT, int KW>
+cudaError_t launch_kw(const DecodeParams& p, int nt, int rt, int grid, cudaStream_t st) {
   if (nt == 1) {
-    if (rt == 4) return launch_t<FMT, 1, 4>(p, grid, st);
-    if (rt == 2) return launch_t<FMT, 1, 2>(p, grid, st);
-    return launch_t<FMT, 1, 1>(p, grid, st);
+    if (rt == 4) return launch_t<FMT, 1, 4, KW>(p, grid, st);
+    if (rt == 2) return launch_t<FMT, 1, 2, KW>(p, grid, st);
+    return launch_t<FMT, 1, 1, KW>(p, grid, st);
   }
-  if (rt == 4) return launch_t<FMT, 2, 4>(p, grid, st);
-  if (rt == 2) return launch_t<FMT, 2, 2>(p, grid, st);
-  return launch_t<FMT, 2, 1>(p, grid, st);
+  if (rt == 4) return launch_t<FMT, 2, 4, KW>(p, grid, st);
+  if (rt == 2) return launch_t<FMT, 2, 2, KW>(p, grid, st);
+  return launch_t<FMT, 2, 1, KW>(p, grid, st);
+}
+
+template <int FMT>
+cudaError_t launch_fmt(const DecodeParams& p, int nt, int rt, int kw, int grid,
+                       cudaStream_t st) {
+  return kw == 8 ? launch_kw<FMT, 8>(p, nt, rt, grid, st) : launch_kw<FMT, 4>(p, nt, rt, grid, st);
 }
 
 }  // namespace
@@ -614,12 +620,21 @@ cudaError_t launch_decode(const LinearArgs& a) {
   // slice of at most 96 KB
   const int64_t target = 4LL * device_sm_count();
   int64_t cs = (target + rowgroups - 1) / rowgroups;
+  // eight warps per CTA when the row groups alone fill the grid (large
+  // layers, no K split across CTAs): a longer K range per CTA is then split
+  // over more warps (measured on a 28672 x 8192 layer at M = 8: 59 us
+  // against 84 with four warps, whose X slice left one CTA per SM); four
+  // otherwise (4096 x 4096: 5.9 us against 7.4 with eight)
+  int kw = rowgroups >= target ? 8 : 4;
+#ifdef WQ_TUNING
+  if (const char* e = getenv("WQ_DECODE_KW")) kw = atoi(e) == 8 ? 8 : 4;
+#endif
   const int64_t x_bytes_all = a.M * a.K * 2;
   const int64_t cs_x = (x_bytes_all + 98303) / 98304;
   if (nt == 2 && cs > 4) cs = 4;  // two token tiles: fewer, longer K slices
   if (cs < cs_x) cs = cs_x;
   if (cs > 8) cs = 8;
-  if (cs > nblk / 4) cs = nblk / 4;  // keep every warp busy
+  if (cs > nblk / kw) cs = nblk / kw;  // keep every warp busy
   if (cs < 1) cs = 1;
 #ifdef WQ_TUNING
   if (const char* e = getenv("WQ_DECODE_CS")) cs = atoi(e);
@@ -646,7 +661,7 @@ cudaError_t launch_decode(const LinearArgs& a) {
     p.side_bytes = 0;
   }
   p.side_bytes = (p.side_bytes + 15) & ~15;
-  const int64_t warp_partials = 4LL * rt * nt * 4 * 32 * 4;  // KW = 4 warps
+  const int64_t warp_partials = (int64_t)kw * rt * nt * 4 * 32 * 4;
   p.swiglu = a.swiglu ? 1 : 0;
   int64_t region = (int64_t)p.xs_bytes * (a.swiglu ? 2 : 1) + p.side_bytes;
   if (region < warp_partials) region = warp_partials;
@@ -655,14 +670,14 @@ cudaError_t launch_decode(const LinearArgs& a) {
   if (p.bar_off + 16 > 227 * 1024) return cudaErrorInvalidValue;
   const int grid = (int)(rowgroups * cs);
   switch (a.fmt) {
-    case INT4_SYM: return launch_fmt<INT4_SYM>(p, nt, rt, grid, a.stream);
-    case INT4_ASYM: return launch_fmt<INT4_ASYM>(p, nt, rt, grid, a.stream);
-    case INT8_SYM: return launch_fmt<INT8_SYM>(p, nt, rt, grid, a.stream);
-    case CB4: return launch_fmt<CB4>(p, nt, rt, grid, a.stream);
-    case NVFP4: return launch_fmt<NVFP4>(p, nt, rt, grid, a.stream);
-    case MXFP4: return launch_fmt<MXFP4>(p, nt, rt, grid, a.stream);
-    case FP8_E4M3: return launch_fmt<FP8_E4M3>(p, nt, rt, grid, a.stream);
-    case FP8_E5M2: return launch_fmt<FP8_E5M2>(p, nt, rt, grid, a.stream);
+    case INT4_SYM: return launch_fmt<INT4_SYM>(p, nt, rt, kw, grid, a.stream);
+    case INT4_ASYM: return launch_fmt<INT4_ASYM>(p, nt, rt, kw, grid, a.stream);
+    case INT8_SYM: return launch_fmt<INT8_SYM>(p, nt, rt, kw, grid, a.stream);
+    case CB4: return launch_fmt<CB4>(p, nt, rt, kw, grid, a.stream);
+    case NVFP4: return launch_fmt<NVFP4>(p, nt, rt, kw, grid, a.stream);
+    case MXFP4: return launch_fmt<MXFP4>(p, nt, rt, kw, grid, a.stream);
+    case FP8_E4M3: return launch_fmt<FP8_E4M3>(p, nt, rt, kw, grid, a.stream);
+    case FP8_E5M2: return launch_fmt<FP8_E5M2>(p, nt, rt, kw, grid, a.stream);
   }
   return cudaErrorInvalidValue;
 }

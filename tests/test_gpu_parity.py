@@ -166,12 +166,15 @@ EDGE = [
     (16, 64, 32, (1, 7, 16, 17, 40)),
     (48, 192, 64, (3, 16, 33, 130)),
     (32, 16384, 256, (1, 16, 20)),
+    # enough row groups for the eight-warp decode CTAs, with fewer K blocks
+    # (three 4-bit blocks) than warps
+    (19008, 192, 64, (1, 9, 16)),
 ]
 
 
 @pytest.mark.parametrize("fmt", ["int4_sym", "int4_asym", "int8_sym", "cb4", "nvfp4", "mxfp4",
                                  "fp8_e4m3", "fp8_e5m2"])
-@pytest.mark.parametrize("case", EDGE, ids=["16x64", "48x192", "32x16384"])
+@pytest.mark.parametrize("case", EDGE, ids=["16x64", "48x192", "32x16384", "19008x192"])
 def test_linear_edge_shapes(wq, orc, fmt, case):
     N, K, G, Ms = case
     G = {"cb4": 0, "nvfp4": 16, "mxfp4": 32}.get(fmt, G)
