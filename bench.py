@@ -461,10 +461,13 @@ def main():
         k = [0]
 
         def e2e_step():
+            # every batch of the step from pinned host memory, results copied
+            # back; one wait per step (the host may read every result after it)
             for M in Ms:
                 pw = weights[k[0] % R]
                 k[0] += 1
-                wq.linear(xh[M], pw, bias, out=yh[M])
+                wq.linear(xh[M], pw, bias, out=yh[M], sync=False)
+            stream.synchronize()
 
         with torch.cuda.stream(stream):
             for _ in range(3):

@@ -158,7 +158,8 @@ int wq_dequant(int format, int64_t N, int64_t K, int group_size, const void* pac
  * when the previous kernel on `stream` starts (pack at load time, or put any
  * other stream operation between wq_pack and the first wq_linear).
  * M <= 16 runs the decode kernel (register dequant, warp-level tensor-core
- * fragments, split-K over warps); larger M runs the prefill kernel (TMA into
+ * fragments, split-K over warps) unless K is too long for its staged
+ * activation slice; larger M (and those) run the prefill kernel (TMA into
  * shared memory, dequant to bf16 in shared memory, tcgen05 MMA into tensor
  * memory).  Both end in the fused fold/bias/bf16 epilogue.
  * Source: OrbitQuant card "API" (matmul_packed_weight(x, idx, row_norms,
@@ -176,9 +177,11 @@ int wq_linear(const void* x, const void* packed_w, const void* scales, const voi
  * so that Y = a . dequant(W)^T (+ bias).
  *   workspace  device scratch for the materialized activation a (bf16
  *              [M, K], 16-byte aligned, at least M*K*2 bytes, overlapping no
- *              other buffer) when M > 16; ignored (may be NULL) when
- *              M <= 16, where the decode kernel applies the step to its
- *              staged activation slice.  Its contents are not preserved.
+ *              other buffer) when M > 16; may be NULL when M <= 16, where
+ *              the decode kernel applies the step to its staged activation
+ *              slice (except for a K too long to stage, which then needs the
+ *              workspace and returns WQ_ERR_UNSUPPORTED without one).  Its
+ *              contents are not preserved.
  * Everything else as wq_linear (same checks, same kernels after the step).
  * Source: piper-kernels README (convrot_linear(up_gate, weight, bias,
  * input_activation="swiglu") computes up * silu(gate) before the linear;
@@ -196,8 +199,8 @@ int wq_linear_swiglu(const void* x2, const void* packed_w, const void* scales, c
  * allocates nothing.  M * K * 2 > 16 MiB returns WQ_ERR_UNSUPPORTED (use
  * wq_linear_swiglu with a workspace).  The scratch is one buffer per
  * device: calls of this entry point must not overlap in time on different
- * streams (calls on one stream are ordered by the stream).  M <= 16 is
- * wq_linear_swiglu itself (no scratch). */
+ * streams (calls on one stream are ordered by the stream).  M <= 16 uses
+ * the scratch only for a K too long for the decode kernel's staged slice. */
 int wq_linear_swiglu_static(const void* x2, const void* packed_w, const void* scales,
                             const void* aux, const void* bias, int64_t M, int64_t N, int64_t K,
                             int format, int group_size, void* out, void* stream);

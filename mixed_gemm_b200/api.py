@@ -78,11 +78,14 @@ def quantize_and_pack(w: torch.Tensor, fmt: str, group_size: int = 0, centroids=
 
 
 def linear(x: torch.Tensor, weight: PackedWeight, bias: torch.Tensor | None = None,
-           out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+           out: torch.Tensor | None = None, stream=None, sync: bool = True) -> torch.Tensor:
     """y = x @ dequant(weight).T + bias, bf16.  ``x``: [..., K] bf16.
 
     A host (CPU) ``x`` is copied to the weight's device and the result copied
-    back, so the call works end to end from host memory.
+    back, so the call works end to end from host memory.  With a host ``x``
+    and ``sync=False`` the copy back is only enqueued (into ``out``, which
+    should then be pinned host memory): synchronize the stream before reading
+    it, e.g. once after several calls.
     """
     host = not x.is_cuda
     dev = weight.w.device
@@ -104,7 +107,8 @@ def linear(x: torch.Tensor, weight: PackedWeight, bias: torch.Tensor | None = No
         yh = out if out is not None else torch.empty((M, weight.N), dtype=torch.bfloat16,
                                                       pin_memory=True)
         yh.copy_(y, non_blocking=True)
-        torch.cuda.current_stream(dev).synchronize()
+        if sync:
+            torch.cuda.current_stream(dev).synchronize()
         return yh.reshape(*lead, weight.N)
     return y.reshape(*lead, weight.N)
 

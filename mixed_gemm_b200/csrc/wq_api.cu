@@ -195,6 +195,7 @@ int wq_linear(const void* x, const void* pw, const void* scales, const void* aux
   cudaError_t e;
   if (M <= 16) {
     e = launch_decode(a);
+    if (e == cudaErrorNotSupported) e = launch_prefill(a);  // K too long to stage
   } else {
     e = launch_prefill(a);
   }
@@ -207,8 +208,8 @@ int wq_linear_swiglu(const void* x2, const void* pw, const void* scales, const v
   int st = check_linear(x2, 2 * K, pw, scales, aux, bias, M, N, K, f, G, out);
   if (st) return st;
   const bool decode = M <= 16;
-  if (!decode) {
-    // the materialized activation [M, K] bf16 lives in the caller's workspace
+  // the materialized activation [M, K] bf16 lives in the caller's workspace
+  auto check_ws = [&]() -> int {
     if (!workspace || workspace_bytes < (size_t)(M * K * 2)) return WQ_ERR_INVALID_ARG;
     if (!aligned(workspace, 16)) return WQ_ERR_ALIGNMENT;
     size_t wb = 0, sb = 0, ab = 0;
@@ -218,7 +219,9 @@ int wq_linear_swiglu(const void* x2, const void* pw, const void* scales, const v
         overlap(workspace, w, pw, wb) || overlap(workspace, w, scales, sb) ||
         overlap(workspace, w, aux, ab) || overlap(workspace, w, bias, N * 2))
       return WQ_ERR_INVALID_ARG;
-  }
+    return WQ_OK;
+  };
+  if (!decode && (st = check_ws()) != WQ_OK) return st;
   if (M == 0) return WQ_OK;
   LinearArgs a;
   a.x = x2;
@@ -235,7 +238,12 @@ int wq_linear_swiglu(const void* x2, const void* pw, const void* scales, const v
   a.stream = (cudaStream_t)stream;
   if (decode) {
     a.swiglu = true;
-    return cuda_status(launch_decode(a));
+    cudaError_t e = launch_decode(a);
+    if (e != cudaErrorNotSupported) return cuda_status(e);
+    // K too long to stage both halves: materialize, if a workspace was given
+    a.swiglu = false;
+    if (!workspace) return WQ_ERR_UNSUPPORTED;
+    if ((st = check_ws()) != WQ_OK) return st;
   }
   cudaError_t e = launch_swiglu(x2, M, K, workspace, a.stream);
   if (e != cudaSuccess) return cuda_status(e);
@@ -246,11 +254,12 @@ int wq_linear_swiglu(const void* x2, const void* pw, const void* scales, const v
 int wq_linear_swiglu_static(const void* x2, const void* pw, const void* scales, const void* aux,
                             const void* bias, int64_t M, int64_t N, int64_t K, int f, int G,
                             void* out, void* stream) {
-  if (M <= 16)
-    return wq_linear_swiglu(x2, pw, scales, aux, bias, M, N, K, f, G, nullptr, 0, out, stream);
   int st = check_linear(x2, 2 * K, pw, scales, aux, bias, M, N, K, f, G, out);
   if (st) return st;
-  if ((uint64_t)M * (uint64_t)K * 2u > kSwigluStaticScratchBytes) return WQ_ERR_UNSUPPORTED;
+  const bool fits = (uint64_t)M * (uint64_t)K * 2u <= kSwigluStaticScratchBytes;
+  if (M <= 16 && !fits)  // the decode path needs no scratch unless K is very long
+    return wq_linear_swiglu(x2, pw, scales, aux, bias, M, N, K, f, G, nullptr, 0, out, stream);
+  if (!fits) return WQ_ERR_UNSUPPORTED;
   void* ws = nullptr;
   size_t ws_bytes = 0;
   if (static_swiglu_scratch(&ws, &ws_bytes) != cudaSuccess) return WQ_ERR_CUDA;

@@ -641,8 +641,9 @@ cudaError_t launch_decode(const LinearArgs& a) {
 #endif
   const int64_t max_blocks = (nblk + cs - 1) / cs;
   const int64_t stride = ((max_blocks * kb * 2 + 127) / 128) * 128 + 64;
-  // K too large for M <= 16 (the SwiGLU input stages up and gate)
-  if (stride * a.M * (a.swiglu ? 2 : 1) > 200 * 1024) return cudaErrorInvalidValue;
+  // K too large for the staged activation slice (the SwiGLU input stages up
+  // and gate): nothing launched, the caller takes the prefill path
+  if (stride * a.M * (a.swiglu ? 2 : 1) > 200 * 1024) return cudaErrorNotSupported;
   p.cs = (int)cs;
   p.xs_stride = (int)stride;
   p.xs_bytes = (int)(stride * a.M);
@@ -667,7 +668,7 @@ cudaError_t launch_decode(const LinearArgs& a) {
   if (region < warp_partials) region = warp_partials;
   p.red_off = (int)((region + 15) & ~15LL);
   p.bar_off = (int)(p.red_off + cs * rt * nt * 4 * 32 * 4);
-  if (p.bar_off + 16 > 227 * 1024) return cudaErrorInvalidValue;
+  if (p.bar_off + 16 > 227 * 1024) return cudaErrorNotSupported;
   const int grid = (int)(rowgroups * cs);
   switch (a.fmt) {
     case INT4_SYM: return launch_fmt<INT4_SYM>(p, nt, rt, kw, grid, a.stream);

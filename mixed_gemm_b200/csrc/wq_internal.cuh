@@ -138,6 +138,8 @@ struct LinearArgs {
   bool swiglu = false;
 };
 
+// cudaErrorNotSupported (nothing launched) when the shape does not fit the
+// decode kernel's shared memory (very long K); the prefill kernel takes any M
 cudaError_t launch_decode(const LinearArgs& a);
 // a[m, k] = bf16(up * silu(gate)) for x2 rows [up | gate], bf16 [M, 2K] -> [M, K]
 cudaError_t launch_swiglu(const void* x2, int64_t M, int64_t K, void* a, cudaStream_t st);

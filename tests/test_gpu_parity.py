@@ -249,3 +249,18 @@ def test_fp8_every_code(wq, orc, fmt, M):
     y = run_linear(wq, pw, x, None, M)
     assert np.array_equal(oracle.bits_to_f32(y), oracle.bits_to_f32(ref))
     assert np.array_equal(oracle.bits_to_f32(ref), dq[:, ks].T.astype(np.float32))
+
+
+@pytest.mark.parametrize("fmt,G", [("int4_sym", 128), ("nvfp4", 16)])
+def test_long_k_small_batch_takes_prefill(wq, orc, fmt, G):
+    """K = 65536 at M = 16 does not fit the decode kernel's staged activation
+    slice; the call runs the prefill kernel instead (M = 1 still decodes)."""
+    N, K = 16, 65536
+    W, (codes, scales, aux) = small_case(orc, fmt, N, K, G, seed=19)
+    pw = pack_on_gpu(wq, fmt, N, K, G, codes, scales, aux)
+    dq = orc.dequant(fmt, codes, scales, aux, N, K, G)
+    xa = synth.activations(61, 16, K)
+    for M in (1, 16):
+        y = run_linear(wq, pw, xa[:M], None, M)
+        ref, _ = orc.linear(xa[:M], dq, None)
+        check_close(y, ref, f"{fmt} long K M={M}")

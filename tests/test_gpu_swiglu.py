@@ -20,7 +20,7 @@ def _run(wq, pw, x2_bits, bias_bits, M, ws_rows=None):
     b = dev_bf16(bias_bits) if bias_bits is not None else None
     y = torch.full((max(M, 1), pw.N), float("nan"), dtype=torch.bfloat16, device="cuda")
     ws = None
-    if M > 16:
+    if M > 16 or ws_rows:
         ws = torch.full((ws_rows or M, pw.K), float("nan"), dtype=torch.bfloat16, device="cuda")
     wq.wq_linear_swiglu(x2, pw.w, pw.scales, pw.aux, b, M, pw.N, pw.K, pw.fmt, pw.group_size,
                         ws, 0 if ws is None else ws.numel() * 2, y)
@@ -78,3 +78,23 @@ def test_swiglu_helper_and_empty(wq, orc):
                         0, out)
     torch.cuda.synchronize()
     assert torch.all(out == 7.0)
+
+
+def test_swiglu_long_k_small_batch(wq, orc):
+    """M <= 16 with a K too long to stage both halves: with a workspace the
+    activation is materialized and the prefill kernel runs; without one the
+    call is refused (nothing launched)."""
+    fmt, G, N, K = "int4_asym", 128, 16, 65536
+    W, (codes, scales, aux) = small_case(orc, fmt, N, K, G, seed=20)
+    pw = pack_on_gpu(wq, fmt, N, K, G, codes, scales, aux)
+    dq = orc.dequant(fmt, codes, scales, aux, N, K, G)
+    M = 16
+    x2 = synth.activations(62, M, 2 * K)
+    ref, _ = orc.linear(orc.swiglu(x2), dq, None)
+    y = _run(wq, pw, x2, None, M, ws_rows=M)
+    check_close(y, ref, "swiglu long K")
+    out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(wq.WQError) as ei:
+        wq.wq_linear_swiglu(dev_bf16(x2), pw.w, pw.scales, pw.aux, None, M, N, K, fmt, G, None, 0,
+                            out)
+    assert ei.value.status == wq.WQ_ERR_UNSUPPORTED
