@@ -73,6 +73,12 @@ def _int_case(fmt, N, K, G, rng):
         codes = _pack_nibbles(v & 15)
         scales = np.full((N, K // G), 0x3F80, np.uint16)   # 1.0
         return codes, scales, None, v.astype(np.float64)
+    if fmt == "int2_sym":
+        v = rng.integers(-2, 2, size=(N, K))          # every 2-bit code, -2 included
+        c = (v & 3).reshape(N, K // 4, 4)
+        codes = (c[..., 0] | (c[..., 1] << 2) | (c[..., 2] << 4) | (c[..., 3] << 6)).astype(np.uint8)
+        scales = np.full((N, K // G), 0x3F80, np.uint16)
+        return codes, scales, None, v.astype(np.float64)
     if fmt == "int4_asym":
         q = rng.integers(0, 16, size=(N, K))
         z = rng.integers(0, 16, size=(N, K // G))
@@ -122,7 +128,7 @@ def _int_case(fmt, N, K, G, rng):
 
 @pytest.mark.parametrize("fmt,G", [("int4_sym", 64), ("int4_asym", 32), ("int8_sym", 128),
                                    ("cb4", 0), ("nvfp4", 16), ("mxfp4", 32), ("fp8_e4m3", 64),
-                                   ("fp8_e5m2", 32)])
+                                   ("fp8_e5m2", 32), ("int2_sym", 64)])
 def test_integer_special_case(orc, fmt, G):
     """Integer X, unit scales: every partial sum is exact, so y equals an
     integer matmul done by numpy -- pins layout, nibble order and orientation."""
@@ -141,7 +147,7 @@ def test_integer_special_case(orc, fmt, G):
 
 @pytest.mark.parametrize("fmt,G", [("int4_sym", 64), ("int4_asym", 128), ("int8_sym", 256),
                                    ("cb4", 0), ("nvfp4", 16), ("mxfp4", 32), ("fp8_e4m3", 128),
-                                   ("fp8_e5m2", 64)])
+                                   ("fp8_e5m2", 64), ("int2_sym", 32)])
 def test_sampled_equals_full(orc, fmt, G):
     M, N, K = 6, 32, 512
     W = synth.weight(21, N, K, sigma=0.02)

@@ -81,6 +81,10 @@ MUTANTS = [
      "double up = (double)orc_bf16_to_f32(x2[m * 2 * K + k]);",
      "double up = (double)orc_bf16_to_f32(x2[m * 2 * K + K + k]);",
      lambda o: swiglu.test_swiglu_layout_and_rounding(o)),
+    ("INT2 field order reversed in the dequant",
+     "int c = (((const uint8_t*)codes)[n * (K / 4) + k / 4] >> (2 * (k & 3))) & 3;",
+     "int c = (((const uint8_t*)codes)[n * (K / 4) + k / 4] >> (6 - 2 * (k & 3))) & 3;",
+     lambda o: lin.test_integer_special_case(o, "int2_sym", 64)),
     ("E2M1 tie broken toward the odd code",
      "if (a == mid) { code = (i % 2 == 0) ? i : i + 1; break; }",
      "if (a == mid) { code = (i % 2 == 0) ? i + 1 : i; break; }",

@@ -23,6 +23,19 @@ def _nibbles(codes):
     return np.stack([lo, hi], axis=-1).reshape(codes.shape[0], -1)
 
 
+def _signed_codes(fmt, codes):
+    """canonical INT codes -> signed integers [N, K] (two's complement fields:
+    2-bit element 4i+j at bits 2j of byte i, 4-bit element 2i+j at bits 4j)."""
+    if fmt == "int8_sym":
+        return codes.astype(np.int64)
+    if fmt == "int4_sym":
+        q = _nibbles(codes).astype(np.int64)
+        return np.where(q > 7, q - 16, q)
+    c = codes.astype(np.int64)
+    q = np.stack([(c >> (2 * j)) & 3 for j in range(4)], axis=-1).reshape(codes.shape[0], -1)
+    return np.where(q > 1, q - 4, q)
+
+
 def _bf16(bits):
     return oracle.bits_to_f32(bits).astype(np.float64)
 
@@ -36,15 +49,13 @@ def _weights(N, K, seed=0, outliers=True):
 
 
 # --------------------------------------------------------------- symmetric INT
-@pytest.mark.parametrize("fmt,qmax", [("int4_sym", 7), ("int8_sym", 127)])
+@pytest.mark.parametrize("fmt,qmax", [("int2_sym", 1), ("int4_sym", 7), ("int8_sym", 127)])
 @pytest.mark.parametrize("G", [32, 64, 128, 256])
 def test_sym_properties(orc, fmt, qmax, G):
     N, K = 48, 512
     W = _weights(N, K, seed=G)
     codes, scales, _ = orc.quantize(fmt, W, G)
-    q = _nibbles(codes).astype(np.int64) if fmt == "int4_sym" else codes.astype(np.int64)
-    if fmt == "int4_sym":
-        q = np.where(q > 7, q - 16, q)
+    q = _signed_codes(fmt, codes)
     s = _bf16(scales)
     assert np.all(np.abs(q) <= qmax)
     qg = np.abs(q).reshape(N, K // G, G).max(-1)
@@ -64,7 +75,7 @@ def test_sym_properties(orc, fmt, qmax, G):
     assert np.array_equal(dq.astype(np.float64), q * sk)
 
 
-@pytest.mark.parametrize("fmt,qmax", [("int4_sym", 7), ("int8_sym", 127)])
+@pytest.mark.parametrize("fmt,qmax", [("int2_sym", 1), ("int4_sym", 7), ("int8_sym", 127)])
 @pytest.mark.parametrize("sval", [1.0, 2.0 ** -7, 0.0173])
 def test_sym_round_trip_every_code(orc, fmt, qmax, sval):
     """W = q*s for every representable q gives back q and s exactly."""
@@ -75,9 +86,7 @@ def test_sym_round_trip_every_code(orc, fmt, qmax, sval):
     W = (row * s).astype(np.float32)[None, :].repeat(2, 0)
     codes, scales, _ = orc.quantize(fmt, W, G)
     assert np.all(_bf16(scales) == s)
-    got = _nibbles(codes).astype(np.int64) if fmt == "int4_sym" else codes.astype(np.int64)
-    if fmt == "int4_sym":
-        got = np.where(got > 7, got - 16, got)
+    got = _signed_codes(fmt, codes)
     assert np.array_equal(got[0], row.astype(np.int64))
 
 
