@@ -51,8 +51,11 @@
  *   WQ_FP8_E4M3 : codes  u8 [N, K]    E4M3 (fn) bytes; scales f32 [N, K/G];
  *                 aux = NULL
  *   WQ_FP8_E5M2 : codes  u8 [N, K]    E5M2 bytes; scales f32 [N, K/G]; aux = NULL
+ *   WQ_INT2_SYM : codes  u8 [N, K/4]  two's complement 2-bit fields, element
+ *                                      4i+j at bits 2j..2j+1 of byte i
+ *                 scales bf16 [N, K/G]
  * Dequantized value of element (n, k) -- what wq_dequant returns:
- *   INT4_SYM/INT8_SYM: q * s            ASYM: (q - z) * s          (exact fp32)
+ *   INT2/INT4/INT8_SYM: q * s           ASYM: (q - z) * s          (exact fp32)
  *   CB4: fp32(c[idx] * norm[n])         NVFP4: fp32(e2m1(q) * e4m3(sb) * ts)
  *   MXFP4: fp32(e2m1(q) * 2^(e-127))    (exact; +-inf where the product
  *                                          reaches 2^128, NaN for e = 255)
@@ -85,7 +88,8 @@ typedef enum {
   WQ_NVFP4 = 4,     /* E2M1 values, E4M3 scale per 16, fp32 tensor scale       */
   WQ_MXFP4 = 5,     /* E2M1 values, E8M0 power-of-two scale per 32 (OCP MX)    */
   WQ_FP8_E4M3 = 6,  /* E4M3 values, fp32 scale per group (FP8 weight-only)     */
-  WQ_FP8_E5M2 = 7   /* E5M2 values, fp32 scale per group (FP8 weight-only)     */
+  WQ_FP8_E5M2 = 7,  /* E5M2 values, fp32 scale per group (FP8 weight-only)     */
+  WQ_INT2_SYM = 8   /* symmetric INT2, bf16 scale per group                    */
 } wq_format_t;
 
 typedef enum {
@@ -146,8 +150,8 @@ int wq_dequant(int format, int64_t N, int64_t K, int group_size, const void* pac
  *            NVFP4 packed E4M3 block scales; MXFP4 packed E8M0 block scales;
  *            FP8 packed fp32 group scales
  *   aux      device: ASYM packed zero-points; CB4 centroids f32[16];
- *            NVFP4 tensor scale f32[1]; NULL for INT4_SYM / INT8_SYM / MXFP4 /
- *            FP8
+ *            NVFP4 tensor scale f32[1]; NULL for INT2_SYM / INT4_SYM /
+ *            INT8_SYM / MXFP4 / FP8
  *   bias     device bf16 [N], or NULL
  *   out      device bf16 [M, N] row-major; must not overlap any input
  * M == 0 is a no-op returning WQ_OK.  Asynchronous; no workspace.

@@ -19,7 +19,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libwq.so")
 
 FORMATS = {"int4_sym": 0, "int4_asym": 1, "int8_sym": 2, "cb4": 3, "nvfp4": 4, "mxfp4": 5,
-           "fp8_e4m3": 6, "fp8_e5m2": 7}
+           "fp8_e4m3": 6, "fp8_e5m2": 7, "int2_sym": 8}
 FORMAT_NAMES = {v: k for k, v in FORMATS.items()}
 
 WQ_OK = 0

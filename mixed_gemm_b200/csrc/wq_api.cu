@@ -23,7 +23,7 @@ bool overlap(const void* p, int64_t pb, const void* q, int64_t qb) {
 
 // Shape / format checks shared by every entry point.
 int check_shape(int f, int64_t N, int64_t K, int G) {
-  if (f < INT4_SYM || f > FP8_E5M2) return WQ_ERR_INVALID_ARG;
+  if (f < INT4_SYM || f > INT2_SYM) return WQ_ERR_INVALID_ARG;
   if (N <= 0 || K <= 0) return WQ_ERR_INVALID_ARG;
   if (N % 16 || K % 64) return WQ_ERR_INVALID_ARG;
   if (N > (1LL << 30) || K > (1LL << 24) || N * K > (1LL << 40)) return WQ_ERR_INVALID_ARG;
@@ -114,6 +114,7 @@ int wq_canonical_sizes(int f, int64_t N, int64_t K, int G, size_t* cb, size_t* s
     case INT4_SYM: c = N * K / 2; s = 2 * N * (K / G); break;
     case INT4_ASYM: c = N * K / 2; s = 2 * N * (K / G); a = N * (K / G); break;
     case INT8_SYM: c = N * K; s = 2 * N * (K / G); break;
+    case INT2_SYM: c = N * K / 4; s = 2 * N * (K / G); break;
     case FP8_E4M3:
     case FP8_E5M2: c = N * K; s = 4 * N * (K / G); break;
     case CB4: c = N * K / 2; s = 2 * N; a = 64; break;

@@ -59,6 +59,11 @@ struct DecodeParams {
                   // staged at xs_bytes past the up slice
 };
 
+__device__ __forceinline__ uint2 ld_stream8(const uint2* p) {
+  uint2 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
+}
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   uint4 v;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -168,7 +173,7 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   constexpr int NV = RT * NT * 4;                  // accumulators per lane
   // one scale per group of K folded into fp32 sums (INT formats, FP8)
   constexpr bool kIntFmt =
-      FMT == INT4_SYM || FMT == INT4_ASYM || FMT == INT8_SYM || kFp8;
+      FMT == INT4_SYM || FMT == INT4_ASYM || FMT == INT8_SYM || FMT == INT2_SYM || kFp8;
   constexpr int SB = kFp8 ? 64 : 32;   // bytes per (row tile, group) of scales
 
   extern __shared__ __align__(16) uint8_t smem[];
@@ -247,12 +252,21 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   const uint4* wrow[RT];
 #pragma unroll
   for (int r = 0; r < RT; ++r) wrow[r] = p.w + (int64_t)(tile0 + r) * nblk * 32 + lane;
+  // INT2: 256-byte blocks, 8 bytes per lane (the words 0..1 of its uint4)
+  auto ld_block = [&](int r, int blk) -> uint4 {
+    if constexpr (FMT == INT2_SYM) {
+      const uint2 v = ld_stream8((const uint2*)p.w + ((int64_t)(tile0 + r) * nblk + blk) * 32 + lane);
+      return make_uint4(v.x, v.y, 0u, 0u);
+    } else {
+      return ld_stream(wrow[r] + blk * 32);
+    }
+  };
   uint4 wv[D][RT];
 #pragma unroll
   for (int j = 0; j < D; ++j)
 #pragma unroll
     for (int r = 0; r < RT; ++r)
-      if (j < nb) wv[j][r] = ld_stream(wrow[r] + (wb + j) * 32);
+      if (j < nb) wv[j][r] = ld_block(r, wb + j);
 
   // Programmatic dependent launch: the packed weight and its scales never
   // depend on the previous kernel in the stream, so they are requested above
@@ -408,7 +422,10 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
             else if constexpr (FMT == FP8_E5M2)
               frag_e5m2(word(wb_[r], 2 * s), word(wb_[r], 2 * s + 1), a);
             else
-              frag_int4(word(wb_[r], 2 * c + s), goff[r][0], goff[r][1], a);
+              if constexpr (FMT == INT2_SYM)
+                frag_int2(word(wb_[r], c), s, 0x43024302u, a);
+              else
+                frag_int4(word(wb_[r], 2 * c + s), goff[r][0], goff[r][1], a);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
               mma16816(cacc[s % NS][r][nt], a, word(xv[c][nt], 2 * s),
@@ -488,7 +505,7 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
         compute_block(wv[j], wb + i + j);
         if (i + j + D < nb) {
 #pragma unroll
-          for (int r = 0; r < RT; ++r) wv[j][r] = ld_stream(wrow[r] + (wb + i + j + D) * 32);
+          for (int r = 0; r < RT; ++r) wv[j][r] = ld_block(r, wb + i + j + D);
         }
       }
     }
@@ -679,6 +696,7 @@ cudaError_t launch_decode(const LinearArgs& a) {
     case MXFP4: return launch_fmt<MXFP4>(p, nt, rt, kw, grid, a.stream);
     case FP8_E4M3: return launch_fmt<FP8_E4M3>(p, nt, rt, kw, grid, a.stream);
     case FP8_E5M2: return launch_fmt<FP8_E5M2>(p, nt, rt, kw, grid, a.stream);
+    case INT2_SYM: return launch_fmt<INT2_SYM>(p, nt, rt, kw, grid, a.stream);
   }
   return cudaErrorInvalidValue;
 }

@@ -45,6 +45,17 @@ static __device__ __forceinline__ void frag_int4(uint32_t wd, uint32_t off_g, ui
   }
 }
 
+// INT2, fields (4s + i, 8 + 4s + i) of the word: fragment i of tensor-core
+// step s as bf16 (128 + c), minus the offset (130 for offset-binary codes).
+static __device__ __forceinline__ void frag_int2(uint32_t wd, int s, uint32_t off,
+                                                 uint32_t (&a)[4]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t t = ((wd >> (2 * (4 * s + i))) & 0x00030003u) | 0x43004300u;
+    a[i] = bsub2(t, off);
+  }
+}
+
 // INT8 offset-binary bytes -> exact integers via the fp32 magic 2^23 + u.
 static __device__ __forceinline__ float i8val(uint32_t w, int i) {
   return __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7440u | i)) - 8388736.0f;

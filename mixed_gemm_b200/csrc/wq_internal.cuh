@@ -20,6 +20,11 @@
 //     "table" (CB4):                  p = 4*(e>>1) + 2*hr + (e&1), so that the
 //        low/high 16 bits hold registers {0,1} / {2,3} as four nibbles each,
 //        ready for byte-permute table lookups.
+//   INT2_SYM: blocks of 256 bytes (64 K); lane L owns 8 bytes, word c (the
+//   32-K chunk c) holds the 16 two-bit fields of rows {g, g+8} x K offsets
+//   {32c + 8tq + 4s + e}, field p = 8*(e&1) + 4*s + 2*(e>>1) + hr at bit 2p,
+//   so that (word >> 2(4s + i)) & 0x00030003 yields fragment register i of
+//   step s as two fields at bit 0 and bit 16; stored offset-binary (v + 2).
 //   INT4_SYM nibbles are stored offset-binary (v + 8); INT8 bytes likewise
 //   (v + 128), word j = 2s + hr, byte e; FP8 (E4M3, E5M2) bytes as they
 //   are, at the INT8 positions.
@@ -43,22 +48,38 @@
 namespace wq {
 
 enum Fmt { INT4_SYM = 0, INT4_ASYM = 1, INT8_SYM = 2, CB4 = 3, NVFP4 = 4, MXFP4 = 5,
-           FP8_E4M3 = 6, FP8_E5M2 = 7 };
+           FP8_E4M3 = 6, FP8_E5M2 = 7, INT2_SYM = 8 };
 
-__host__ __device__ inline bool is_int_fmt(int f) { return f == INT4_SYM || f == INT4_ASYM || f == INT8_SYM; }
+__host__ __device__ inline bool is_int_fmt(int f) {
+  return f == INT4_SYM || f == INT4_ASYM || f == INT8_SYM || f == INT2_SYM;
+}
 // formats with one scale per group of G along K, folded into fp32 sums
 __host__ __device__ inline bool is_fp8(int f) { return f == FP8_E4M3 || f == FP8_E5M2; }
 __host__ __device__ inline bool is_grouped_fmt(int f) { return is_int_fmt(f) || is_fp8(f); }
-__host__ __device__ inline bool is_4bit(int f) { return f != INT8_SYM && !is_fp8(f); }
+// bits per packed code
+__host__ __device__ inline int code_bits(int f) {
+  return f == INT2_SYM ? 2 : (f == INT8_SYM || is_fp8(f)) ? 8 : 4;
+}
+__host__ __device__ inline bool is_4bit(int f) { return code_bits(f) == 4; }
+// bytes of one packed block (16 rows x block_k(f) K elements)
+__host__ __device__ inline int block_bytes(int f) { return code_bits(f) == 2 ? 256 : 512; }
 // elements of K per 512-byte block
-__host__ __device__ inline int block_k(int f) { return is_4bit(f) ? 64 : 32; }
+__host__ __device__ inline int block_k(int f) { return code_bits(f) == 8 ? 32 : 64; }
 
 // Byte offset and bit shift of element (n, k) inside the packed weight.
 __host__ __device__ inline void packed_loc(int f, int64_t n, int64_t k, int64_t K,
                                            int64_t* byte_off, int* shift) {
   int64_t tile = n >> 4;
   int r = (int)(n & 15), g = r & 7, hr = r >> 3;
-  if (is_4bit(f)) {
+  if (code_bits(f) == 2) {
+    int64_t b = k >> 6;
+    int kk = (int)(k & 63), c = kk >> 5, kc = kk & 31, tq = kc >> 3, e8 = kc & 7, s = e8 >> 2,
+        e = e8 & 3;
+    int lane = 4 * g + tq;
+    int p = 8 * (e & 1) + 4 * s + 2 * (e >> 1) + hr;
+    *byte_off = ((tile * (K >> 6) + b) * 32 + lane) * 8 + c * 4 + (p >> 2);
+    *shift = (p & 3) * 2;
+  } else if (is_4bit(f)) {
     int64_t b = k >> 6;
     int kk = (int)(k & 63), c = kk >> 5, kc = kk & 31, tq = kc >> 3, e8 = kc & 7, s = e8 >> 2,
         e = e8 & 3;

@@ -23,6 +23,7 @@ inline unsigned grid_for(int64_t n) {
 // canonical nibble/byte of element (n, k)
 __device__ __forceinline__ uint32_t canon_code(int f, const uint8_t* codes, int64_t n, int64_t k,
                                                int64_t K) {
+  if (code_bits(f) == 2) return (codes[n * (K >> 2) + (k >> 2)] >> (2 * (k & 3))) & 3u;
   if (is_4bit(f)) {
     uint8_t b = codes[n * (K >> 1) + (k >> 1)];
     return (k & 1) ? (b >> 4) : (b & 15u);
@@ -33,6 +34,7 @@ __device__ __forceinline__ uint32_t canon_code(int f, const uint8_t* codes, int6
 // canonical -> packed encoding of one code
 __device__ __forceinline__ uint32_t encode(int f, uint32_t c) {
   if (f == INT4_SYM) return c ^ 0x8u;
+  if (f == INT2_SYM) return c ^ 0x2u;
   if (f == INT8_SYM) return c ^ 0x80u;
   return c;
 }
@@ -40,9 +42,25 @@ __device__ __forceinline__ uint32_t encode(int f, uint32_t c) {
 // One thread per packed weight byte: gather the canonical code(s) it holds.
 __global__ void pack_w_kernel(int f, int64_t N, int64_t K, const uint8_t* __restrict__ codes,
                               uint8_t* __restrict__ pw) {
-  const int64_t total = is_4bit(f) ? N * K / 2 : N * K;
+  const int64_t total = N * K * code_bits(f) / 8;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
        i += (int64_t)gridDim.x * blockDim.x) {
+    if (code_bits(f) == 2) {  // 8-byte lane chunks, 256-byte blocks of 64 K
+      const int q = (int)(i & 3), c = (int)((i >> 2) & 1), lane = (int)((i >> 3) & 31);
+      const int64_t blk_global = i >> 8, nblk = K >> 6;
+      const int64_t tile = blk_global / nblk, b = blk_global % nblk;
+      const int g = lane >> 2, tq = lane & 3;
+      uint32_t out = 0;
+      for (int h = 0; h < 4; ++h) {
+        const int p = 4 * q + h;
+        const int hr = p & 1, e = ((p >> 1) & 1) * 2 + (p >> 3), s = (p >> 2) & 1;
+        const int64_t n = tile * 16 + g + 8 * hr;
+        const int64_t k = b * 64 + c * 32 + tq * 8 + s * 4 + e;
+        out |= encode(f, canon_code(f, codes, n, k, K)) << (2 * h);
+      }
+      pw[i] = (uint8_t)out;
+      continue;
+    }
     // decompose the packed byte offset
     int64_t word = i >> 2;
     int q = (int)(i & 3);
@@ -78,11 +96,19 @@ __global__ void pack_w_kernel(int f, int64_t N, int64_t K, const uint8_t* __rest
 // One thread per canonical byte: scatter back from the packed weight.
 __global__ void unpack_w_kernel(int f, int64_t N, int64_t K, const uint8_t* __restrict__ pw,
                                 uint8_t* __restrict__ codes) {
-  const int64_t total = is_4bit(f) ? N * K / 2 : N * K;
+  const int64_t total = N * K * code_bits(f) / 8;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
        i += (int64_t)gridDim.x * blockDim.x) {
     uint32_t out = 0;
-    if (is_4bit(f)) {
+    if (code_bits(f) == 2) {
+      int64_t n = i / (K >> 2), k0 = (i % (K >> 2)) * 4;
+      for (int h = 0; h < 4; ++h) {
+        int64_t off;
+        int sh;
+        packed_loc(f, n, k0 + h, K, &off, &sh);
+        out |= encode(f, (pw[off] >> sh) & 3u) << (2 * h);
+      }
+    } else if (is_4bit(f)) {
       int64_t n = i / (K >> 1), k0 = (i % (K >> 1)) * 2;
       for (int h = 0; h < 2; ++h) {
         int64_t off;
@@ -160,10 +186,10 @@ __global__ void dequant_kernel(int f, int64_t N, int64_t K, int G, const uint8_t
     int64_t off;
     int sh;
     packed_loc(f, n, k, K, &off, &sh);
-    uint32_t raw = (pw[off] >> sh) & (is_4bit(f) ? 15u : 255u);
+    uint32_t raw = (pw[off] >> sh) & ((1u << code_bits(f)) - 1u);
     float v;
-    if (f == INT4_SYM || f == INT8_SYM) {
-      int q = (int)raw - (f == INT4_SYM ? 8 : 128);
+    if (f == INT4_SYM || f == INT8_SYM || f == INT2_SYM) {
+      int q = (int)raw - (f == INT4_SYM ? 8 : f == INT2_SYM ? 2 : 128);
       float s = bf16_bits_to_f32(((const uint16_t*)ps)[packed_scale_idx(n, k / G, K / G)]);
       v = (float)q * s;
     } else if (f == INT4_ASYM) {
@@ -198,7 +224,7 @@ __global__ void dequant_kernel(int f, int64_t N, int64_t K, int G, const uint8_t
 
 cudaError_t launch_pack(int f, int64_t N, int64_t K, int G, const void* codes, const void* scales,
                         const void* aux, void* pw, void* ps, void* pa, cudaStream_t st) {
-  const int64_t wbytes = is_4bit(f) ? N * K / 2 : N * K;
+  const int64_t wbytes = N * K * code_bits(f) / 8;
   pack_w_kernel<<<grid_for(wbytes), kThreads, 0, st>>>(f, N, K, (const uint8_t*)codes,
                                                         (uint8_t*)pw);
   if (is_fp8(f)) {
@@ -227,7 +253,7 @@ cudaError_t launch_pack(int f, int64_t N, int64_t K, int G, const void* codes, c
 
 cudaError_t launch_unpack(int f, int64_t N, int64_t K, int G, const void* pw, const void* ps,
                           const void* pa, void* codes, void* scales, void* aux, cudaStream_t st) {
-  const int64_t wbytes = is_4bit(f) ? N * K / 2 : N * K;
+  const int64_t wbytes = N * K * code_bits(f) / 8;
   unpack_w_kernel<<<grid_for(wbytes), kThreads, 0, st>>>(f, N, K, (const uint8_t*)pw,
                                                           (uint8_t*)codes);
   if (is_fp8(f)) {

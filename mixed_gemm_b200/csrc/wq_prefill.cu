@@ -244,11 +244,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                    const PrefillParams p) {
   // one scale per group of K, folded into fp32 sums (INT formats, FP8)
-  constexpr bool kInt =
-      FMT == INT4_SYM || FMT == INT4_ASYM || FMT == INT8_SYM || FMT == FP8_E4M3 || FMT == FP8_E5M2;
+  constexpr bool kInt = FMT == INT4_SYM || FMT == INT4_ASYM || FMT == INT8_SYM ||
+                        FMT == INT2_SYM || FMT == FP8_E4M3 || FMT == FP8_E5M2;
   constexpr bool kFp8 = FMT == FP8_E4M3 || FMT == FP8_E5M2;
   constexpr bool kByte = FMT == INT8_SYM || kFp8;  // one byte per code
-  constexpr uint32_t kWpk = kByte ? 8192u : 4096u;  // packed bytes per stage
+  // packed bytes per stage (8 row tiles x 64 K)
+  constexpr uint32_t kWpk = kByte ? 8192u : FMT == INT2_SYM ? 2048u : 4096u;
   // A stage: one 128 x 64 bf16 tile; CB4 adds a second tile holding the
   // bf16 remainders of its centroids (two MMAs per K step)
   constexpr uint32_t kAsub = FMT == CB4 ? 2u : 1u;
@@ -488,6 +489,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             st_shared_v4(abase + swz(Rg, j), a[0], a[2], b[0], b[2]);
             st_shared_v4(abase + swz(Rg8, j), a[1], a[3], b[1], b[3]);
           }
+        } else if constexpr (FMT == INT2_SYM) {
+          // 256 bytes per row tile and K step; word c = the 32-K chunk c,
+          // both tensor-core steps of it; exact codes, scale in the fold
+          const uint2 ch = *(const uint2*)(wpk + rt * 256 + lane * 8);
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const uint32_t w = c ? ch.y : ch.x;
+            uint32_t a[4], b[4];
+            frag_int2(w, 0, 0x43024302u, a);
+            frag_int2(w, 1, 0x43024302u, b);
+            const int j = 4 * c + tq;
+            st_shared_v4(abase + swz(Rg, j), a[0], a[2], b[0], b[2]);
+            st_shared_v4(abase + swz(Rg8, j), a[1], a[3], b[1], b[3]);
+          }
         } else {
           const uint4 ch = *(const uint4*)(wpk + rt * 512 + lane * 16);
 #pragma unroll
@@ -692,7 +707,9 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 template <int FMT, int BN>
 cudaError_t launch_bn(const LinearArgs& a) {
-  constexpr uint32_t kWpk = (FMT == INT8_SYM || FMT == FP8_E4M3 || FMT == FP8_E5M2) ? 8192u : 4096u;
+  constexpr uint32_t kWpk = (FMT == INT8_SYM || FMT == FP8_E4M3 || FMT == FP8_E5M2) ? 8192u
+                            : FMT == INT2_SYM                                     ? 2048u
+                                                                                  : 4096u;
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
   CUtensorMap tmX, tmW;
@@ -707,7 +724,7 @@ cudaError_t launch_bn(const LinearArgs& a) {
       return cudaErrorInvalidValue;
   }
   {
-    const uint64_t row_bytes = (uint64_t)a.K * (is_4bit(FMT) ? 8 : 16);  // bytes per row tile
+    const uint64_t row_bytes = (uint64_t)a.K * 2 * code_bits(FMT);  // bytes per row tile
     cuuint64_t dims[2] = {(cuuint64_t)(row_bytes / 4), (cuuint64_t)(a.N / 16)};
     cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
     cuuint32_t box[2] = {kWpk / 32u, 8u};
@@ -836,6 +853,7 @@ cudaError_t launch_prefill(const LinearArgs& a) {
     case MXFP4: return launch_fmt<MXFP4>(a, BN);
     case FP8_E4M3: return launch_fmt<FP8_E4M3>(a, BN);
     case FP8_E5M2: return launch_fmt<FP8_E5M2>(a, BN);
+    case INT2_SYM: return launch_fmt<INT2_SYM>(a, BN);
   }
   return cudaErrorInvalidValue;
 }

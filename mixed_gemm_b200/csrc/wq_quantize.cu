@@ -87,13 +87,13 @@ __device__ __forceinline__ uint32_t e2m1_encode_rn_sat(double r) {
 
 constexpr int kWarps = 8;
 
-// One warp per (row, group): symmetric INT4 / INT8.
+// One warp per (row, group): symmetric INT2 / INT4 / INT8.
 __global__ void quant_sym_kernel(int bits, int64_t N, int64_t K, int G,
                                  const float* __restrict__ w, uint8_t* __restrict__ codes,
                                  uint16_t* __restrict__ scales) {
   const int lane = threadIdx.x & 31;
   const int64_t groups = K / G;
-  const int qmax = bits == 4 ? 7 : 127;
+  const int qmax = (1 << (bits - 1)) - 1;
   for (int64_t item = blockIdx.x * (int64_t)kWarps + (threadIdx.x >> 5); item < N * groups;
        item += (int64_t)gridDim.x * kWarps) {
     int64_t n = item / groups, grp = item % groups;
@@ -104,7 +104,17 @@ __global__ void quant_sym_kernel(int bits, int64_t N, int64_t K, int G,
     uint16_t sb = f64_to_bf16_rn(__ddiv_rn(amax, (double)qmax));
     double s = (double)bf16_bits_to_f32(sb);
     if (lane == 0) scales[item] = sb;
-    if (bits == 4) {
+    if (bits == 2) {
+      for (int i = 4 * lane; i < G; i += 128) {
+        uint32_t packed = 0;
+        for (int j = 0; j < 4; ++j) {
+          int q = 0;
+          if (s != 0.0) q = max(-qmax, min(qmax, __double2int_rn(__ddiv_rn((double)wg[i + j], s))));
+          packed |= (uint32_t)(q & 3) << (2 * j);
+        }
+        codes[n * (K / 4) + (grp * G + i) / 4] = (uint8_t)packed;
+      }
+    } else if (bits == 4) {
       for (int i = 2 * lane; i < G; i += 64) {
         int q0 = 0, q1 = 0;
         if (s != 0.0) {
@@ -324,8 +334,9 @@ cudaError_t launch_quantize(int f, int64_t N, int64_t K, int G, const float* w, 
   switch (f) {
     case INT4_SYM:
     case INT8_SYM:
+    case INT2_SYM:
       quant_sym_kernel<<<blocks_for(N * (K / G), kWarps), kWarps * 32, 0, st>>>(
-          f == INT4_SYM ? 4 : 8, N, K, G, w, (uint8_t*)codes, (uint16_t*)scales);
+          code_bits(f), N, K, G, w, (uint8_t*)codes, (uint16_t*)scales);
       break;
     case FP8_E4M3:
     case FP8_E5M2:

@@ -106,6 +106,8 @@ def packed_bytes(fmt: str, N: int, K: int, G: int) -> int:
     """Weight-side bytes: codes + scales + auxiliary data, for the given format."""
     if fmt == "int4_sym":
         return N * K // 2 + 2 * N * (K // G)
+    if fmt == "int2_sym":
+        return N * K // 4 + 2 * N * (K // G)
     if fmt == "int4_asym":
         return N * K // 2 + 2 * N * (K // G) + N * (K // G) // 2
     if fmt == "int8_sym":
