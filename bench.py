@@ -175,6 +175,23 @@ def recorded_traffic(kernel_file: str, workload: str):
     return e.get("bytes_per_launch")
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest value over all ranks (timings are taken as the slowest rank's)."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(world: int, steps: int, work_per_step: float, sec: float, scale: float):
+    """Units all ranks processed / the (max-over-ranks) time: every rank runs
+    the same step on its own replica."""
+    return world * steps * work_per_step / sec / scale
+
+
 def context_numbers(wl, Ms, weights, xs, bias, outs, stream, l2, device):
     """Per batch size: per-call time over 20 replays of a 50-call graph (p50,
     p95), one launch timed alone (median of 20), and, as a reference point
@@ -424,17 +441,12 @@ def main():
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
-    ms_total = ev0.elapsed_time(ev1)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms_total], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), world, device)
     sec = ms_total / 1e3
     if tflops_metric:
-        value = world * args.steps * step_flops / sec / 1e12
+        value = whole_job_value(world, args.steps, step_flops, sec, 1e12)
     else:
-        value = world * args.steps * step_bytes / sec / 1e9
+        value = whole_job_value(world, args.steps, step_bytes, sec, 1e9)
     per_launch_s = sec / (args.steps * launches_per_step)
 
     # roofline of the dominant kernel (every launch in the step runs it)
@@ -483,14 +495,9 @@ def main():
             e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            import torch.distributed as dist
-            t = torch.tensor([e_ms], device=device, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        es = e_ms / 1e3
-        ev = world * e2e_steps * (step_flops / 1e12 if tflops_metric else step_bytes / 1e9) / es
+        es = max_over_ranks(e0.elapsed_time(e1), world, device) / 1e3
+        ev = whole_job_value(world, e2e_steps, step_flops if tflops_metric else step_bytes, es,
+                             1e12 if tflops_metric else 1e9)
         e2e = {"value": ev, "unit": unit, "steps": e2e_steps,
                "h2d_bytes_per_step": sum(M * wl.K * 2 for M in Ms),
                "d2h_bytes_per_step": sum(M * wl.N * 2 for M in Ms)}
