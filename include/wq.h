@@ -23,7 +23,7 @@
  *    WQ_ERR_CUDA (from cudaGetLastError).  No C++ exception crosses the ABI.
  *  - bf16 values are IEEE bfloat16 bit patterns (uint16_t).
  *  - Shapes: N % 16 == 0 and K % 64 == 0 for every format (the packed tile is
- *    16 rows by 64 (4-bit) or 32 (INT8) K elements); INT formats take
+ *    16 rows by 64 (2- and 4-bit) or 32 (INT8, FP8) K elements); INT formats take
  *    group_size in {32, 64, 128, 256} with K % group_size == 0; NVFP4 has a
  *    fixed block of 16 (group_size 16 or 0), MXFP4 one of 32 (group_size 32
  *    or 0); CB4 ignores group_size; the FP8 formats take the INT group sizes.
