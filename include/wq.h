@@ -175,6 +175,25 @@ int wq_linear(const void* x, const void* packed_w, const void* scales, const voi
               const void* bias, int64_t M, int64_t N, int64_t K, int format, int group_size,
               void* out, void* stream);
 
+/* Grouped (mixture-of-experts) linear: E experts of one format, shape [N, K]
+ * and group size.  The rows of x (bf16 [T, K]) are sorted by expert: expert e
+ * owns rows [offsets[e], offsets[e+1]) and writes the same rows of out
+ * (bf16 [T, N]).
+ *   offsets   host int64 [E + 1], offsets[0] = 0, non-decreasing, T = offsets[E]
+ *   packed_w, scales, aux, bias
+ *             host arrays of E device pointers (expert e's buffers as for
+ *             wq_linear); aux and bias may be NULL arrays (no aux / no bias)
+ * Every expert's arguments are checked before anything is launched; each
+ * non-empty expert then runs wq_linear on its rows (the decode kernel for
+ * at most 16 rows, the prefill kernel otherwise), in expert order on `stream`.
+ * Source: Petit README "Features" (fused MoE kernels for BF16 and MXFP4
+ * workloads); auto-round-lib README (quantized experts); the per-expert
+ * token counts of a routed layer. */
+int wq_linear_grouped(const void* x, const void* const* packed_w, const void* const* scales,
+                      const void* const* aux, const void* const* bias, const int64_t* offsets,
+                      int64_t E, int64_t N, int64_t K, int format, int group_size, void* out,
+                      void* stream);
+
 /* The same linear with a SwiGLU input: x2 is bf16 [M, 2K], each row holding
  * [up | gate] (K values each), and the activation is
  *     a = bf16(up * silu(gate)),   silu(g) = g / (1 + e^-g)  (fp32, then RNE)

@@ -52,6 +52,8 @@ _SIGS = {
     "wq_linear": ([_ptr, _ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _int, _int, _ptr, _ptr], _int),
     "wq_linear_swiglu": ([_ptr, _ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _int, _int, _ptr,
                           ctypes.c_size_t, _ptr, _ptr], _int),
+    "wq_linear_grouped": ([_ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _int, _int,
+                           _ptr, _ptr], _int),
     "wq_linear_swiglu_static": ([_ptr, _ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _int, _int, _ptr,
                                  _ptr], _int),
     "wq_quantize": ([_int, _i64, _i64, _int, _ptr, _ptr, _ptr, _ptr, _ptr], _int),
@@ -141,6 +143,25 @@ def wq_linear_swiglu(x2, packed_w, scales, aux, bias, M, N, K, fmt, group_size, 
            "wq_linear_swiglu")
 
 
+def wq_linear_grouped(x, packed_w, scales, aux, bias, offsets, N, K, fmt, group_size, out,
+                      stream=None):
+    """``packed_w``, ``scales``, ``aux``, ``bias``: sequences of E device
+    tensors / addresses (``aux`` and ``bias`` may be None); ``offsets``: E + 1
+    row offsets (host integers)."""
+    E = len(packed_w)
+    arr = ctypes.c_void_p * E
+
+    def ptrs(seq):
+        if seq is None:
+            return None
+        return arr(*[_addr(t) for t in seq])
+
+    offs = (ctypes.c_int64 * (E + 1))(*[int(o) for o in offsets])
+    _check(_lib.wq_linear_grouped(_addr(x), ptrs(packed_w), ptrs(scales), ptrs(aux), ptrs(bias),
+                                  offs, E, N, K, _fmt(fmt), group_size, _addr(out),
+                                  _stream(stream)), "wq_linear_grouped")
+
+
 def wq_linear_swiglu_static(x2, packed_w, scales, aux, bias, M, N, K, fmt, group_size, out,
                             stream=None):
     _check(_lib.wq_linear_swiglu_static(_addr(x2), _addr(packed_w), _addr(scales), _addr(aux),
@@ -176,4 +197,5 @@ def wq_device_sm_count() -> int:
     return n.value
 
 
-from .api import PackedWeight, linear, linear_swiglu, pack, quantize_and_pack  # noqa: E402,F401
+from .api import (PackedWeight, linear, linear_grouped, linear_swiglu, pack,  # noqa: E402,F401
+                  quantize_and_pack)

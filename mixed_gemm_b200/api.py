@@ -12,8 +12,8 @@ from dataclasses import dataclass
 
 import torch
 
-from . import (FORMATS, wq_canonical_sizes, wq_linear, wq_linear_swiglu, wq_lloyd_max_centroids,
-               wq_pack, wq_packed_sizes, wq_quantize)
+from . import (FORMATS, wq_canonical_sizes, wq_linear, wq_linear_grouped, wq_linear_swiglu,
+               wq_lloyd_max_centroids, wq_pack, wq_packed_sizes, wq_quantize)
 
 
 @dataclass
@@ -129,3 +129,22 @@ def linear_swiglu(x2: torch.Tensor, weight: PackedWeight, bias: torch.Tensor | N
     wq_linear_swiglu(xd, weight.w, weight.scales, weight.aux, bias, M, weight.N, K, weight.fmt,
                      weight.group_size, ws, 0 if ws is None else ws.numel() * 2, y, stream)
     return y.reshape(*lead, weight.N)
+
+
+def linear_grouped(x: torch.Tensor, weights: list, offsets, bias: list | None = None,
+                   out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Mixture-of-experts linear: rows offsets[e]:offsets[e+1] of ``x`` ([T, K]
+    bf16, sorted by expert) use ``weights[e]`` (PackedWeights of one format,
+    shape and group size); ``bias`` an optional list of per-expert [N] tensors."""
+    w0 = weights[0]
+    assert all(w.fmt == w0.fmt and w.N == w0.N and w.K == w0.K and
+               w.group_size == w0.group_size for w in weights)
+    xd = x.contiguous()
+    T = int(offsets[-1])
+    assert xd.shape == (T, w0.K) and len(offsets) == len(weights) + 1
+    y = out if out is not None else torch.empty((T, w0.N), dtype=torch.bfloat16,
+                                                device=w0.w.device)
+    wq_linear_grouped(xd, [w.w for w in weights], [w.scales for w in weights],
+                      None if w0.aux is None else [w.aux for w in weights], bias,
+                      [int(o) for o in offsets], w0.N, w0.K, w0.fmt, w0.group_size, y, stream)
+    return y

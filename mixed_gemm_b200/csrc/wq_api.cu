@@ -203,6 +203,35 @@ int wq_linear(const void* x, const void* pw, const void* scales, const void* aux
   return cuda_status(e);
 }
 
+int wq_linear_grouped(const void* x, const void* const* pw, const void* const* scales,
+                      const void* const* aux, const void* const* bias, const int64_t* offsets,
+                      int64_t E, int64_t N, int64_t K, int f, int G, void* out, void* stream) {
+  if (!offsets || !pw || !scales || E <= 0 || E > (1 << 20)) return WQ_ERR_INVALID_ARG;
+  if (offsets[0] != 0) return WQ_ERR_INVALID_ARG;
+  for (int64_t e = 0; e < E; ++e)
+    if (offsets[e + 1] < offsets[e]) return WQ_ERR_INVALID_ARG;
+  const int64_t T = offsets[E];
+  // every expert's arguments are checked before anything is launched
+  for (int64_t e = 0; e < E; ++e) {
+    const int64_t m = offsets[e + 1] - offsets[e];
+    int g = G;
+    int st = check_linear(x, K, pw[e], scales[e], aux ? aux[e] : nullptr, bias ? bias[e] : nullptr,
+                          T, N, K, f, g, out);
+    if (st) return st;
+    if (m < 0) return WQ_ERR_INVALID_ARG;
+  }
+  for (int64_t e = 0; e < E; ++e) {
+    const int64_t m0 = offsets[e], m = offsets[e + 1] - m0;
+    if (m == 0) continue;
+    const uint16_t* xe = (const uint16_t*)x + m0 * K;
+    uint16_t* ye = (uint16_t*)out + m0 * N;
+    int st = wq_linear(xe, pw[e], scales[e], aux ? aux[e] : nullptr, bias ? bias[e] : nullptr, m,
+                       N, K, f, G, ye, stream);
+    if (st) return st;
+  }
+  return WQ_OK;
+}
+
 int wq_linear_swiglu(const void* x2, const void* pw, const void* scales, const void* aux,
                      const void* bias, int64_t M, int64_t N, int64_t K, int f, int G,
                      void* workspace, size_t workspace_bytes, void* out, void* stream) {

@@ -128,3 +128,23 @@ def test_linear_swiglu_rejects_bad_workspace():
     # M == 0 is a no-op even without a workspace
     assert wqm._lib.wq_linear_swiglu(base, base * 4, base * 8, None, None, 0, N, K, f, G, None, 0,
                                      out, 0) == wqm.WQ_OK
+
+
+def test_linear_grouped_rejects_bad_offsets_and_args():
+    base = 1 << 20
+    f = wqm.FORMATS["int4_sym"]
+    N, K, G = 256, 512, 64
+    E = 3
+    arr = ctypes.c_void_p * E
+    w = arr(*[base * (8 + e) for e in range(E)])
+    s = arr(*[base * (16 + e) for e in range(E)])
+
+    def call(offs, out=base * 64, g=G):
+        o = (ctypes.c_int64 * (E + 1))(*offs)
+        return wqm._lib.wq_linear_grouped(base, w, s, None, None, o, E, N, K, f, g, out, 0)
+
+    assert call([1, 2, 3, 4]) == wqm.WQ_ERR_INVALID_ARG        # offsets[0] != 0
+    assert call([0, 3, 2, 4]) == wqm.WQ_ERR_INVALID_ARG        # decreasing
+    assert call([0, 1, 2, 4], g=48) == wqm.WQ_ERR_INVALID_ARG  # bad group size
+    assert call([0, 1, 2, 4], out=base * 64 + 8) == wqm.WQ_ERR_ALIGNMENT
+    assert call([0, 0, 0, 0]) == wqm.WQ_OK                     # no rows: nothing launched
