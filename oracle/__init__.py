@@ -70,6 +70,8 @@ def _declare(lib):
         "orc_threads": ([], c_int),
         "orc_silu": ([dbl], dbl),
         "orc_swiglu": ([ptr, i64, i64, ptr], c_int),
+        "orc_addmm_requant_int8": ([ptr, ptr, i64, i64, c_int, ptr, ptr, i64, dbl, dbl, c_int,
+                                    ctypes.c_uint64], c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -224,6 +226,21 @@ class Oracle:
         a = np.zeros((M, K2 // 2), dtype=np.uint16)
         _ok(self.lib.orc_swiglu(_p(x2_bits), M, K2 // 2, _p(a)), "swiglu")
         return a
+
+    def addmm_requant_int8(self, codes, scales, G: int, mat1_bits, mat2_bits, alpha: float,
+                           beta: float, seed=None):
+        """New canonical INT8 codes after weight = beta * weight + alpha * mat1 @ mat2,
+        requantized with the unchanged scales (nearest, or stochastic with a seed)."""
+        out = np.ascontiguousarray(codes, dtype=np.int8).copy()
+        N, K = out.shape
+        m1 = np.ascontiguousarray(mat1_bits, dtype=np.uint16)
+        m2 = np.ascontiguousarray(mat2_bits, dtype=np.uint16)
+        R = m1.shape[1]
+        sc = np.ascontiguousarray(scales, dtype=np.uint16)
+        _ok(self.lib.orc_addmm_requant_int8(_p(out), _p(sc), N, K, G, _p(m1), _p(m2), R,
+                                            float(alpha), float(beta), 0 if seed is None else 1,
+                                            0 if seed is None else int(seed)), "addmm_requant")
+        return out
 
     def linear_sampled(self, fmt: str, codes, scales, aux, N: int, K: int, group_size: int,
                        x_bits, bias_bits, ms, ns):

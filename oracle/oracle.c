@@ -67,6 +67,15 @@
  *    to fp32.
  *  - y = sum_k x*dq accumulated in fp64 in increasing k, plus bias, rounded
  *    once to bf16 (round to nearest even).
+ *  - LoRA merge into an INT8 weight (piper-kernels README, Tensor.addmm_ on
+ *    a ConvRot weight): weight = beta * weight + alpha * (mat1 @ mat2),
+ *    requantized with the weight's unchanged scales.  Readings: w' =
+ *    beta * dq + alpha * sum_r mat1[n, r] * mat2[r, k] in fp64 (increasing r,
+ *    separate multiply and add); t = w' / s; nearest: q = rne(t); with a
+ *    seed: q = floor(t) + [u < t - floor(t)], u = top 53 bits of SplitMix64
+ *    output (n*K + k) for key = seed, times 2^-53 (the two adjacent codes,
+ *    each with probability proportional to the distance to the other); q
+ *    clamped to [-127, 127]; a zero scale keeps code 0.
  *  - SwiGLU input (piper-kernels README, convrot_linear with
  *    input_activation="swiglu"): the input row holds [up | gate], K values
  *    each; the linear's activation is a = bf16(up * silu(gate)) with
@@ -599,6 +608,45 @@ int orc_swiglu(const uint16_t* x2, int64_t M, int64_t K, uint16_t* a) {
       double up = (double)orc_bf16_to_f32(x2[m * 2 * K + k]);
       double gate = (double)orc_bf16_to_f32(x2[m * 2 * K + K + k]);
       a[m * K + k] = orc_f64_to_bf16(up * orc_silu(gate));
+    }
+  return 0;
+}
+
+/* SplitMix64 (Vigna): output i of the counter-based stream keyed by `key`. */
+static uint64_t orc_splitmix64(uint64_t key, uint64_t i) {
+  uint64_t z = key + (i + 1) * 0x9E3779B97F4A7C15ULL;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ULL;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBULL;
+  return z ^ (z >> 31);
+}
+
+/* LoRA merge into INT8 codes (canonical int8 [N, K], bf16 scales [N, K/G]):
+ * codes are rewritten in place; mat1 bf16 [N, R], mat2 bf16 [R, K]. */
+int orc_addmm_requant_int8(int8_t* codes, const uint16_t* scales, int64_t N, int64_t K, int G,
+                           const uint16_t* mat1, const uint16_t* mat2, int64_t R, double alpha,
+                           double beta, int stochastic, uint64_t seed) {
+  if (N <= 0 || K <= 0 || G <= 0 || K % G || R < 0) return 1;
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k) {
+      double s = (double)orc_bf16_to_f32(scales[n * (K / G) + k / G]);
+      if (s == 0.0) { codes[n * K + k] = 0; continue; }
+      double dot = 0.0;
+      for (int64_t r = 0; r < R; ++r) {
+        double p = (double)orc_bf16_to_f32(mat1[n * R + r]) * (double)orc_bf16_to_f32(mat2[r * K + k]);
+        dot = dot + p;
+      }
+      double wq = beta * ((double)codes[n * K + k] * s) + alpha * dot;
+      double t = wq / s, q;
+      if (stochastic) {
+        double f = floor(t);
+        double u = (double)(orc_splitmix64(seed, (uint64_t)(n * K + k)) >> 11) * 0x1p-53;
+        q = f + (u < t - f ? 1.0 : 0.0);
+      } else {
+        q = nearbyint(t);
+      }
+      if (q > 127.0) q = 127.0;
+      if (q < -127.0) q = -127.0;
+      codes[n * K + k] = (int8_t)q;
     }
   return 0;
 }

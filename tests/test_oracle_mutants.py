@@ -10,6 +10,7 @@ import pytest
 import oracle
 import test_oracle_codecs as codecs
 import test_oracle_linear as lin
+import test_oracle_lora as lora
 import test_oracle_quant as quant
 import test_oracle_swiglu as swiglu
 
@@ -85,6 +86,10 @@ MUTANTS = [
      "int c = (((const uint8_t*)codes)[n * (K / 4) + k / 4] >> (2 * (k & 3))) & 3;",
      "int c = (((const uint8_t*)codes)[n * (K / 4) + k / 4] >> (6 - 2 * (k & 3))) & 3;",
      lambda o: lin.test_integer_special_case(o, "int2_sym", 64)),
+    ("stochastic requantization compares the wrong way",
+     "q = f + (u < t - f ? 1.0 : 0.0);",
+     "q = f + (u > t - f ? 1.0 : 0.0);",
+     lambda o: lora.test_stochastic_rounding_is_unbiased(o)),
     ("E2M1 tie broken toward the odd code",
      "if (a == mid) { code = (i % 2 == 0) ? i : i + 1; break; }",
      "if (a == mid) { code = (i % 2 == 0) ? i + 1 : i; break; }",
