@@ -228,6 +228,28 @@ int wq_linear_swiglu_static(const void* x2, const void* packed_w, const void* sc
                             const void* aux, const void* bias, int64_t M, int64_t N, int64_t K,
                             int format, int group_size, void* out, void* stream);
 
+/* In-place LoRA merge into a packed INT8_SYM weight:
+ *     weight = beta * weight + alpha * (mat1 @ mat2)
+ * requantized with the weight's unchanged group scales.  With use_seed == 0
+ * each code is the nearest (ties to even) of w'/s; otherwise one of the two
+ * adjacent codes, the upper one with probability equal to the fractional
+ * part of w'/s (draw for element (n, k): output n*K + k of SplitMix64 keyed
+ * by `seed`, top 53 bits * 2^-53), so the same seed replays the same codes.
+ * Codes are clamped to [-127, 127]; a zero scale keeps code 0.  All
+ * arithmetic is fp64 with round-to-nearest steps in a fixed order.
+ *   packed_w       device, in/out (from wq_pack)
+ *   packed_scales  device, unchanged
+ *   mat1, mat2     device bf16 [N, rank] and [rank, K] (rank 0: no update)
+ * Other formats return WQ_ERR_UNSUPPORTED.  Offline; asynchronous.  Repeated
+ * merges are lossy (each one requantizes).
+ * Source: piper-kernels README (weight.addmm_(lora_b, lora_a, alpha=...,
+ * rounding_seed=seed): beta * weight + alpha * (mat1 @ mat2), requantized,
+ * deterministic row scales kept, stochastic choice of one of the two adjacent
+ * INT8 codes with probability proportional to distance). */
+int wq_addmm_requant(int format, int64_t N, int64_t K, int group_size, void* packed_w,
+                     const void* packed_scales, const void* mat1, const void* mat2, int64_t rank,
+                     double alpha, double beta, int use_seed, uint64_t seed, void* stream);
+
 /* Offline round-to-nearest quantizer on the GPU: w_f32[N, K] (device) ->
  * canonical codes / scales / aux (device), bit-identical to the CPU
  * definitions listed above.  CB4 reads its 16 centroids from `aux`

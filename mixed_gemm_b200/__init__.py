@@ -54,6 +54,8 @@ _SIGS = {
                           ctypes.c_size_t, _ptr, _ptr], _int),
     "wq_linear_grouped": ([_ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _int, _int,
                            _ptr, _ptr], _int),
+    "wq_addmm_requant": ([_int, _i64, _i64, _int, _ptr, _ptr, _ptr, _ptr, _i64, ctypes.c_double,
+                          ctypes.c_double, _int, ctypes.c_uint64, _ptr], _int),
     "wq_linear_swiglu_static": ([_ptr, _ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _int, _int, _ptr,
                                  _ptr], _int),
     "wq_quantize": ([_int, _i64, _i64, _int, _ptr, _ptr, _ptr, _ptr, _ptr], _int),
@@ -160,6 +162,15 @@ def wq_linear_grouped(x, packed_w, scales, aux, bias, offsets, N, K, fmt, group_
     _check(_lib.wq_linear_grouped(_addr(x), ptrs(packed_w), ptrs(scales), ptrs(aux), ptrs(bias),
                                   offs, E, N, K, _fmt(fmt), group_size, _addr(out),
                                   _stream(stream)), "wq_linear_grouped")
+
+
+def wq_addmm_requant(fmt, N, K, group_size, packed_w, packed_scales, mat1, mat2, rank, alpha,
+                     beta=1.0, seed=None, stream=None):
+    _check(_lib.wq_addmm_requant(_fmt(fmt), N, K, group_size, _addr(packed_w),
+                                 _addr(packed_scales), _addr(mat1), _addr(mat2), rank,
+                                 float(alpha), float(beta), 0 if seed is None else 1,
+                                 0 if seed is None else int(seed), _stream(stream)),
+           "wq_addmm_requant")
 
 
 def wq_linear_swiglu_static(x2, packed_w, scales, aux, bias, M, N, K, fmt, group_size, out,

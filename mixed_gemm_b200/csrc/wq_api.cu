@@ -10,6 +10,11 @@
 
 namespace wq {
 
+cudaError_t launch_addmm_requant_int8(int64_t N, int64_t K, int G, void* pw, const void* ps,
+                                      const void* mat1, const void* mat2, int64_t R,
+                                      double alpha, double beta, int use_seed, uint64_t seed,
+                                      cudaStream_t st);
+
 namespace {
 
 bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p % a) == 0; }
@@ -294,6 +299,26 @@ int wq_linear_swiglu_static(const void* x2, const void* pw, const void* scales, 
   size_t ws_bytes = 0;
   if (static_swiglu_scratch(&ws, &ws_bytes) != cudaSuccess) return WQ_ERR_CUDA;
   return wq_linear_swiglu(x2, pw, scales, aux, bias, M, N, K, f, G, ws, ws_bytes, out, stream);
+}
+
+int wq_addmm_requant(int f, int64_t N, int64_t K, int G, void* pw, const void* ps,
+                     const void* mat1, const void* mat2, int64_t rank, double alpha, double beta,
+                     int use_seed, uint64_t seed, void* stream) {
+  int st = check_shape(f, N, K, G);
+  if (st) return st;
+  if (f != INT8_SYM) return WQ_ERR_UNSUPPORTED;
+  if (rank < 0 || rank > (1 << 16)) return WQ_ERR_INVALID_ARG;
+  if (!pw || !ps || (rank > 0 && (!mat1 || !mat2))) return WQ_ERR_INVALID_ARG;
+  if (!aligned(pw, 16) || !aligned(ps, 16) || (mat1 && !aligned(mat1, 2)) ||
+      (mat2 && !aligned(mat2, 2)))
+    return WQ_ERR_ALIGNMENT;
+  size_t wb = 0, sb = 0, ab = 0;
+  wq_packed_sizes(f, N, K, G, &wb, &sb, &ab);
+  if (overlap(pw, wb, ps, sb) || overlap(pw, wb, mat1, N * rank * 2) ||
+      overlap(pw, wb, mat2, rank * K * 2))
+    return WQ_ERR_INVALID_ARG;
+  return cuda_status(launch_addmm_requant_int8(N, K, G, pw, ps, mat1, mat2, rank, alpha, beta,
+                                               use_seed, seed, (cudaStream_t)stream));
 }
 
 // Lloyd-Max quantizer of N(0,1): thresholds at the midpoints of adjacent

@@ -148,3 +148,21 @@ def test_linear_grouped_rejects_bad_offsets_and_args():
     assert call([0, 1, 2, 4], g=48) == wqm.WQ_ERR_INVALID_ARG  # bad group size
     assert call([0, 1, 2, 4], out=base * 64 + 8) == wqm.WQ_ERR_ALIGNMENT
     assert call([0, 0, 0, 0]) == wqm.WQ_OK                     # no rows: nothing launched
+
+
+def test_addmm_requant_rejections():
+    base = 1 << 20
+    i8, i4 = wqm.FORMATS["int8_sym"], wqm.FORMATS["int4_sym"]
+    N, K, G = 256, 512, 64
+    call = wqm._lib.wq_addmm_requant
+    assert call(i4, N, K, G, base, base * 8, base * 16, base * 32, 8, 1.0, 1.0, 0, 0, 0) == \
+        wqm.WQ_ERR_UNSUPPORTED
+    assert call(i8, N, K, G, base, base * 8, base * 16, base * 32, -1, 1.0, 1.0, 0, 0, 0) == \
+        wqm.WQ_ERR_INVALID_ARG
+    assert call(i8, N, K, G, base + 8, base * 8, base * 16, base * 32, 8, 1.0, 1.0, 0, 0, 0) == \
+        wqm.WQ_ERR_ALIGNMENT
+    assert call(i8, N, K, G, base, base * 8, None, base * 32, 8, 1.0, 1.0, 0, 0, 0) == \
+        wqm.WQ_ERR_INVALID_ARG
+    # the weight may not overlap the scales
+    assert call(i8, N, K, G, base, base + 64, base * 16, base * 32, 8, 1.0, 1.0, 0, 0, 0) == \
+        wqm.WQ_ERR_INVALID_ARG

@@ -5,6 +5,8 @@ refused before anything launches.  GPU: results identical to
 wq_linear_swiglu with a caller workspace, and no device memory allocated."""
 from __future__ import annotations
 
+import gc
+
 import numpy as np
 import pytest
 
@@ -47,6 +49,7 @@ def test_static_scratch_matches_workspace_and_allocates_nothing(orc):
         wqm.wq_linear_swiglu_static(x2[:M], pw.w, pw.scales, pw.aux, None, M, N, K, fmt, G,
                                     y_st)                      # warm-up: module and scratch loaded
         torch.cuda.synchronize()
+        gc.collect()                 # tensors of earlier tests may be freed meanwhile
         free0, _ = torch.cuda.mem_get_info()
         alloc0 = torch.cuda.memory_allocated()
         for _ in range(3):
@@ -54,5 +57,6 @@ def test_static_scratch_matches_workspace_and_allocates_nothing(orc):
                                         y_st)
         torch.cuda.synchronize()
         free1, _ = torch.cuda.mem_get_info()
-        assert free1 == free0 and torch.cuda.memory_allocated() == alloc0
+        # no device memory taken by the calls (torch's own count may only fall)
+        assert free1 == free0 and torch.cuda.memory_allocated() <= alloc0
         assert np.array_equal(bf16_bits(y_st), bf16_bits(y_ws)), f"M={M}"
