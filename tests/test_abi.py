@@ -166,3 +166,9 @@ def test_addmm_requant_rejections():
     # the weight may not overlap the scales
     assert call(i8, N, K, G, base, base + 64, base * 16, base * 32, 8, 1.0, 1.0, 0, 0, 0) == \
         wqm.WQ_ERR_INVALID_ARG
+
+
+def test_every_header_call_has_a_binding():
+    """The Python binding carries every C name the header declares."""
+    missing = [n for n in _declared() if not callable(getattr(wqm, n, None))]
+    assert not missing, missing
