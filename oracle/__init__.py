@@ -70,6 +70,8 @@ def _declare(lib):
         "orc_threads": ([], c_int),
         "orc_silu": ([dbl], dbl),
         "orc_swiglu": ([ptr, i64, i64, ptr], c_int),
+        "orc_quant_act_int8": ([ptr, i64, i64, ptr, ptr], c_int),
+        "orc_linear_a8": ([c_int, ptr, ptr, i64, i64, c_int, ptr, ptr, ptr, i64, ptr, ptr], c_int),
         "orc_addmm_requant_int8": ([ptr, ptr, i64, i64, c_int, ptr, ptr, i64, dbl, dbl, c_int,
                                     ctypes.c_uint64], c_int),
     }
@@ -213,6 +215,27 @@ class Oracle:
         y64 = np.zeros((M, N), dtype=np.float64)
         b = None if bias_bits is None else np.ascontiguousarray(bias_bits, dtype=np.uint16)
         _ok(self.lib.orc_linear(_p(x_bits), _p(dq), _p(b), M, N, K, _p(y), _p(y64)), "linear")
+        return y, y64
+
+    def quant_act_int8(self, x_bits: np.ndarray):
+        """Per-token INT8 activation quantization: (x_q int8 [M, K], s_x f32 [M])."""
+        x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+        M, K = x_bits.shape
+        xq = np.zeros((M, K), dtype=np.int8)
+        sx = np.zeros((M,), dtype=np.float32)
+        _ok(self.lib.orc_quant_act_int8(_p(x_bits), M, K, _p(xq), _p(sx)), "quant_act_int8")
+        return xq, sx
+
+    def linear_a8(self, fmt: str, codes, scales, N: int, K: int, G: int, x_bits, bias_bits=None):
+        """(y bf16 bits, y fp64) of the activation-quantized linear (INT4 / INT8 sym)."""
+        xq, sx = self.quant_act_int8(x_bits)
+        M = xq.shape[0]
+        y = np.zeros((M, N), dtype=np.uint16)
+        y64 = np.zeros((M, N), dtype=np.float64)
+        b = None if bias_bits is None else np.ascontiguousarray(bias_bits, dtype=np.uint16)
+        _ok(self.lib.orc_linear_a8(FORMATS[fmt], _p(np.ascontiguousarray(codes)),
+                                   _p(np.ascontiguousarray(scales, dtype=np.uint16)), N, K, G,
+                                   _p(xq), _p(sx), _p(b), M, _p(y), _p(y64)), "linear_a8")
         return y, y64
 
     def silu(self, g: float) -> float:

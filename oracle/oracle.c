@@ -76,6 +76,14 @@
  *    output (n*K + k) for key = seed, times 2^-53 (the two adjacent codes,
  *    each with probability proportional to the distance to the other); q
  *    clamped to [-127, 127]; a zero scale keeps code 0.
+ *  - Activation-quantized compute (auto-round-lib README, section 1: INT8
+ *    compute with dynamic activation quantization, low-bit weights rescaled
+ *    to INT8 and computed by an INT8 GEMM; the library does not implement it
+ *    yet): per token m, s_x = fp32(amax_k |x| / 127), x_q = clamp(rne(x /
+ *    s_x), -127, 127) (an all-zero row: s_x = 0, x_q = 0); with the INT4 /
+ *    INT8 symmetric weights' integer codes q_w and bf16 group scales s_w,
+ *    y = sum_g s_w[n,g] * s_x[m] * (integer sum_{k in g} q_w * x_q) in fp64
+ *    over increasing g, plus bias, rounded once to bf16.
  *  - SwiGLU input (piper-kernels README, convrot_linear with
  *    input_activation="swiglu"): the input row holds [up | gate], K values
  *    each; the linear's activation is a = bf16(up * silu(gate)) with
@@ -594,6 +602,57 @@ int orc_linear(const uint16_t* x, const float* dq, const uint16_t* bias, int64_t
       if (y) y[m * N + n] = orc_f64_to_bf16(acc);
     }
   }
+  return 0;
+}
+
+/* Per-token INT8 activation quantization: xq int8 [M, K], sx f32 [M]. */
+int orc_quant_act_int8(const uint16_t* x, int64_t M, int64_t K, int8_t* xq, float* sx) {
+  if (M < 0 || K <= 0) return 1;
+  for (int64_t m = 0; m < M; ++m) {
+    double amax = 0.0;
+    for (int64_t k = 0; k < K; ++k) amax = fmax(amax, fabs((double)orc_bf16_to_f32(x[m * K + k])));
+    float s = (float)(amax / 127.0);
+    sx[m] = s;
+    for (int64_t k = 0; k < K; ++k) {
+      double q = 0.0;
+      if (s != 0.0f) {
+        q = nearbyint((double)orc_bf16_to_f32(x[m * K + k]) / (double)s);
+        if (q > 127.0) q = 127.0;
+        if (q < -127.0) q = -127.0;
+      }
+      xq[m * K + k] = (int8_t)q;
+    }
+  }
+  return 0;
+}
+
+/* y = sum over groups of s_w * s_x * (integer dot of codes), for the INT4 /
+ * INT8 symmetric formats (canonical codes and bf16 group scales). */
+int orc_linear_a8(int fmt, const void* codes, const uint16_t* scales, int64_t N, int64_t K, int G,
+                  const int8_t* xq, const float* sx, const uint16_t* bias, int64_t M, uint16_t* y,
+                  double* y64) {
+  if ((fmt != ORC_INT4_SYM && fmt != ORC_INT8_SYM) || check_fmt(fmt, N, K, G) || M < 0) return 1;
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t m = 0; m < M; ++m) {
+      double acc = 0.0;
+      for (int64_t g = 0; g < K / G; ++g) {
+        int64_t isum = 0;
+        for (int64_t k = g * G; k < (g + 1) * G; ++k) {
+          int qw;
+          if (fmt == ORC_INT8_SYM) {
+            qw = ((const int8_t*)codes)[n * K + k];
+          } else {
+            int nib = get_nib((const uint8_t*)codes + n * (K / 2), k);
+            qw = nib > 7 ? nib - 16 : nib;
+          }
+          isum += (int64_t)qw * (int64_t)xq[m * K + k];
+        }
+        acc += (double)orc_bf16_to_f32(scales[n * (K / G) + g]) * (double)sx[m] * (double)isum;
+      }
+      if (bias) acc = acc + (double)orc_bf16_to_f32(bias[n]);
+      if (y64) y64[m * N + n] = acc;
+      if (y) y[m * N + n] = orc_f64_to_bf16(acc);
+    }
   return 0;
 }
 

@@ -1,0 +1,52 @@
+"""Pins of the oracle's activation-quantized linear (per-token INT8
+activations, integer dot products per weight group; auto-round-lib README:
+INT8 compute with dynamic activation quantization): the per-token scale
+against an exact rational, the quantization error bound, and the reduction to
+the weight-only linear when the activations already lie on their INT8 grid."""
+from __future__ import annotations
+
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import synth
+
+
+def test_activation_scale_and_error_bound(orc):
+    M, K = 12, 384
+    x = synth.activations(5, M, K, channel_count=4, channel_mult=10.0)
+    x[3] = 0                                              # an all-zero token
+    xq, sx = orc.quant_act_int8(x)
+    xv = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    for m in range(M):
+        amax = np.abs(xv[m]).max()
+        if amax == 0:
+            assert sx[m] == 0 and not xq[m].any()
+            continue
+        ulp = Fraction(float(np.spacing(np.float32(sx[m]))))
+        assert abs(Fraction(float(sx[m])) - Fraction(amax) / 127) <= ulp / 2
+        assert np.abs(xq[m].astype(np.int64)).max() == 127
+        err = np.abs(xv[m] - xq[m].astype(np.float64) * float(sx[m]))
+        assert np.all(err <= 0.5 * float(sx[m]) * (1 + 1e-12))
+
+
+@pytest.mark.parametrize("fmt", ["int8_sym", "int4_sym"])
+def test_grid_activations_reduce_to_weight_only_linear(orc, fmt):
+    """x = integers * 2^-e with every row reaching 127 * 2^-e: the INT8
+    activations are exact, so (one weight group per row) the result equals the
+    weight-only linear's fp64 sum exactly."""
+    N, K = 40, 256
+    W = synth.weight(8, N, K, sigma=0.02)
+    codes, scales, _ = orc.quantize(fmt, W, K)
+    rng = np.random.default_rng(4)
+    M = 6
+    ints = rng.integers(-127, 128, size=(M, K))
+    ints[:, 0] = 127
+    e = rng.integers(3, 9, size=(M, 1))
+    x = synth.f64_to_bf16_bits(ints * np.ldexp(1.0, -e))
+    b = synth.bias(8, N)
+    y8, y8_64 = orc.linear_a8(fmt, codes, scales, N, K, K, x, b)
+    dq = orc.dequant(fmt, codes, scales, None, N, K, K)
+    y, y64 = orc.linear(x, dq, b)
+    assert np.array_equal(y8_64, y64) and np.array_equal(y8, y)

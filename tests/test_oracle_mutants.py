@@ -8,6 +8,7 @@ import os
 import pytest
 
 import oracle
+import test_oracle_a8 as a8
 import test_oracle_codecs as codecs
 import test_oracle_linear as lin
 import test_oracle_lora as lora
@@ -90,6 +91,10 @@ MUTANTS = [
      "q = f + (u < t - f ? 1.0 : 0.0);",
      "q = f + (u > t - f ? 1.0 : 0.0);",
      lambda o: lora.test_stochastic_rounding_is_unbiased(o)),
+    ("activation scale from 128 instead of 127",
+     "float s = (float)(amax / 127.0);",
+     "float s = (float)(amax / 128.0);",
+     lambda o: a8.test_activation_scale_and_error_bound(o)),
     ("E2M1 tie broken toward the odd code",
      "if (a == mid) { code = (i % 2 == 0) ? i : i + 1; break; }",
      "if (a == mid) { code = (i % 2 == 0) ? i + 1 : i; break; }",
