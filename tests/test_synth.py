@@ -56,6 +56,11 @@ def test_workload_recipes():
     assert W.algorithmic_bytes(W.PR1, 4) == 76288
     assert W.algorithmic_bytes(W.DECODE, 1) == 8716288 + 16384
     assert W.algorithmic_bytes(W.NVFP4, 1) == 132120580 + 73728
+    # MXFP4: codes N*K/2 + one E8M0 byte per 32; FP8: N*K + fp32 scale per group
+    assert W.algorithmic_bytes(W.MXFP4, 1) == 28672 * 8192 // 2 + 28672 * 256 + 73728
+    assert W.algorithmic_bytes(W.FP8, 1) == 8192 * 8192 + 4 * 8192 * 64 + 2 * 8192 + 2 * 8192
+    assert W.packed_bytes("int2_sym", 256, 512, 64) == 256 * 128 + 2 * 256 * 8
+    assert len({w.seed for w in W.ALL}) == len(W.ALL)       # one stream per workload
     x1 = W.make_x(W.DECODE, 1)
     x16 = W.make_x(W.DECODE, 16)
     assert np.array_equal(x1[0], x16[0])
