@@ -23,7 +23,7 @@ _lock = threading.Lock()
 _lib = None
 
 FORMATS = {"int4_sym": 0, "int4_asym": 1, "int8_sym": 2, "cb4": 3, "nvfp4": 4, "mxfp4": 5,
-           "fp8_e4m3": 6, "fp8_e5m2": 7, "int2_sym": 8}
+           "fp8_e4m3": 6, "fp8_e5m2": 7, "int2_sym": 8, "int3_sym": 9}
 
 
 def build(force: bool = False, extra_flags=(), out_path: str | None = None,
@@ -149,8 +149,8 @@ class Oracle:
         W = np.ascontiguousarray(W, dtype=np.float32)
         N, K = W.shape
         G = group_size
-        if fmt in ("int2_sym", "int4_sym", "int8_sym"):
-            bits = {"int2_sym": 2, "int4_sym": 4, "int8_sym": 8}[fmt]
+        if fmt in ("int2_sym", "int3_sym", "int4_sym", "int8_sym"):
+            bits = {"int2_sym": 2, "int3_sym": 3, "int4_sym": 4, "int8_sym": 8}[fmt]
             codes = np.zeros((N, K * bits // 8), dtype=np.int8 if bits == 8 else np.uint8)
             scales = np.zeros((N, K // G), dtype=np.uint16)
             _ok(self.lib.orc_quant_int_sym(_p(W), N, K, G, bits, _p(codes), _p(scales)), fmt)

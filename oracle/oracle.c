@@ -37,7 +37,8 @@
  *  - rounding of w/s to an integer: round half to even;
  *  - a scale is rounded once to bf16 and w is divided by the stored scale;
  *  - an all-zero group / row / block gets scale 0 and code 0;
- *  - INT4 emits [-7, 7], INT8 emits [-127, 127], INT2 emits [-1, 1]
+ *  - INT4 emits [-7, 7], INT8 emits [-127, 127], INT2 emits [-1, 1],
+ *    INT3 emits [-3, 3]
  *    (qmax = 2^(bits-1) - 1 for every width; -2^(bits-1) decodes but is
  *    never written);
  *  - asym INT4: lo = min(0, min w), hi = max(0, max w), s = bf16((hi-lo)/15),
@@ -102,6 +103,9 @@
  *   fp8_e4m3 : codes u8 [N, K] E4M3; scales f32 [N, K/G]
  *   int2_sym : codes u8 [N, K/4] two's complement 2-bit fields, element 4i+j
  *              at bits 2j..2j+1 of byte i; scales bf16 [N, K/G]
+ *   int3_sym : codes u8 [N, 3K/8] a little-endian bit stream per row, element
+ *              k at bits 3k..3k+2 (two's complement); scales bf16 [N, K/G]
+ *              (oracle only: the library has no INT3 kernels yet)
  *   fp8_e5m2 : codes u8 [N, K] E5M2; scales f32 [N, K/G]
  */
 #include <math.h>
@@ -110,7 +114,8 @@
 #include <string.h>
 
 enum { ORC_INT4_SYM = 0, ORC_INT4_ASYM = 1, ORC_INT8_SYM = 2, ORC_CB4 = 3, ORC_NVFP4 = 4,
-       ORC_MXFP4 = 5, ORC_FP8_E4M3 = 6, ORC_FP8_E5M2 = 7, ORC_INT2_SYM = 8 };
+       ORC_MXFP4 = 5, ORC_FP8_E4M3 = 6, ORC_FP8_E5M2 = 7, ORC_INT2_SYM = 8,
+       ORC_INT3_SYM = 9 };
 
 /* ------------------------------------------------------------------ bf16 */
 float orc_bf16_to_f32(uint16_t h) {
@@ -239,8 +244,9 @@ static inline void put_nib(uint8_t* row, int64_t k, int v) {
 /* ---------------------------------------------------------- quantizers */
 int orc_quant_int_sym(const float* W, int64_t N, int64_t K, int G, int bits, void* codes,
                       uint16_t* scales) {
-  if (N <= 0 || K <= 0 || G <= 0 || K % G || (bits != 2 && bits != 4 && bits != 8)) return 1;
-  if (bits == 2 && K % 4) return 1;
+  if (N <= 0 || K <= 0 || G <= 0 || K % G || bits < 2 || bits > 8 || (bits > 4 && bits != 8))
+    return 1;
+  if ((bits == 2 && K % 4) || (bits == 3 && K % 8)) return 1;
   int qmax = (1 << (bits - 1)) - 1;
   int64_t ng = K / G;
   for (int64_t n = 0; n < N; ++n) {
@@ -250,6 +256,8 @@ int orc_quant_int_sym(const float* W, int64_t N, int64_t K, int G, int bits, voi
     uint8_t* row2 = (uint8_t*)codes + n * (K / 4);
     if (bits == 4) memset(row4, 0, (size_t)(K / 2));
     if (bits == 2) memset(row2, 0, (size_t)(K / 4));
+    uint8_t* row3 = (uint8_t*)codes + n * (K / 8 * 3);
+    if (bits == 3) memset(row3, 0, (size_t)(K / 8 * 3));
     for (int64_t j = 0; j < ng; ++j) {
       double amax = 0.0;
       for (int64_t k = j * G; k < (j + 1) * G; ++k) amax = fmax(amax, fabs((double)w[k]));
@@ -264,7 +272,10 @@ int orc_quant_int_sym(const float* W, int64_t N, int64_t K, int G, int bits, voi
           if (r < -qmax) r = -qmax;
           q = (int)r;
         }
-        if (bits == 2) row2[k >> 2] |= (uint8_t)((q & 3) << (2 * (k & 3)));
+        if (bits == 3) {
+          for (int b = 0; b < 3; ++b)
+            if ((q >> b) & 1) row3[(3 * k + b) >> 3] |= (uint8_t)(1u << ((3 * k + b) & 7));
+        } else if (bits == 2) row2[k >> 2] |= (uint8_t)((q & 3) << (2 * (k & 3)));
         else if (bits == 4) put_nib(row4, k, q & 15);
         else row8[k] = (int8_t)q;
       }
@@ -519,6 +530,14 @@ static float dq_one(int fmt, int64_t K, int G, const void* codes, const void* sc
       float s = orc_bf16_to_f32(((const uint16_t*)scales)[n * (K / G) + k / G]);
       return (float)(q - z) * s;
     }
+    case ORC_INT3_SYM: {
+      const uint8_t* row = (const uint8_t*)codes + n * (K / 8 * 3);
+      int c = 0;
+      for (int b = 0; b < 3; ++b) c |= ((row[(3 * k + b) >> 3] >> ((3 * k + b) & 7)) & 1) << b;
+      int v = c > 3 ? c - 8 : c;
+      float s = orc_bf16_to_f32(((const uint16_t*)scales)[n * (K / G) + k / G]);
+      return (float)v * s;
+    }
     case ORC_INT2_SYM: {
       int c = (((const uint8_t*)codes)[n * (K / 4) + k / 4] >> (2 * (k & 3))) & 3;
       int v = c > 1 ? c - 4 : c;
@@ -563,12 +582,14 @@ static float dq_one(int fmt, int64_t K, int G, const void* codes, const void* sc
 
 static int check_fmt(int fmt, int64_t N, int64_t K, int G) {
   if (N <= 0 || K <= 0) return 1;
-  if (fmt < 0 || fmt > 8) return 1;
+  if (fmt < 0 || fmt > 9) return 1;
   const int bytes = fmt == ORC_INT8_SYM || fmt == ORC_FP8_E4M3 || fmt == ORC_FP8_E5M2;
   if ((fmt == ORC_INT4_SYM || fmt == ORC_INT4_ASYM || fmt == ORC_INT8_SYM ||
-       fmt == ORC_FP8_E4M3 || fmt == ORC_FP8_E5M2 || fmt == ORC_INT2_SYM) && (G <= 0 || K % G))
+       fmt == ORC_FP8_E4M3 || fmt == ORC_FP8_E5M2 || fmt == ORC_INT2_SYM ||
+       fmt == ORC_INT3_SYM) && (G <= 0 || K % G))
     return 1;
   if (fmt == ORC_INT2_SYM && K % 4) return 1;
+  if (fmt == ORC_INT3_SYM && K % 8) return 1;
   if (!bytes && K % 2) return 1;
   if (fmt == ORC_NVFP4 && K % 16) return 1;
   if (fmt == ORC_MXFP4 && K % 32) return 1;

@@ -79,6 +79,12 @@ def _int_case(fmt, N, K, G, rng):
         codes = (c[..., 0] | (c[..., 1] << 2) | (c[..., 2] << 4) | (c[..., 3] << 6)).astype(np.uint8)
         scales = np.full((N, K // G), 0x3F80, np.uint16)
         return codes, scales, None, v.astype(np.float64)
+    if fmt == "int3_sym":
+        v = rng.integers(-4, 4, size=(N, K))          # every 3-bit code, -4 included
+        bits = np.stack([(v >> b) & 1 for b in range(3)], axis=-1).reshape(N, -1)
+        codes = np.packbits(bits.astype(np.uint8), axis=1, bitorder="little")
+        scales = np.full((N, K // G), 0x3F80, np.uint16)
+        return codes, scales, None, v.astype(np.float64)
     if fmt == "int4_asym":
         q = rng.integers(0, 16, size=(N, K))
         z = rng.integers(0, 16, size=(N, K // G))
@@ -128,7 +134,7 @@ def _int_case(fmt, N, K, G, rng):
 
 @pytest.mark.parametrize("fmt,G", [("int4_sym", 64), ("int4_asym", 32), ("int8_sym", 128),
                                    ("cb4", 0), ("nvfp4", 16), ("mxfp4", 32), ("fp8_e4m3", 64),
-                                   ("fp8_e5m2", 32), ("int2_sym", 64)])
+                                   ("fp8_e5m2", 32), ("int2_sym", 64), ("int3_sym", 32)])
 def test_integer_special_case(orc, fmt, G):
     """Integer X, unit scales: every partial sum is exact, so y equals an
     integer matmul done by numpy -- pins layout, nibble order and orientation."""

@@ -95,6 +95,10 @@ MUTANTS = [
      "float s = (float)(amax / 127.0);",
      "float s = (float)(amax / 128.0);",
      lambda o: a8.test_activation_scale_and_error_bound(o)),
+    ("INT3 bit stream read most-significant bit first",
+     "for (int b = 0; b < 3; ++b) c |= ((row[(3 * k + b) >> 3] >> ((3 * k + b) & 7)) & 1) << b;",
+     "for (int b = 0; b < 3; ++b) c |= ((row[(3 * k + b) >> 3] >> (7 - ((3 * k + b) & 7))) & 1) << b;",
+     lambda o: lin.test_integer_special_case(o, "int3_sym", 32)),
     ("E2M1 tie broken toward the odd code",
      "if (a == mid) { code = (i % 2 == 0) ? i : i + 1; break; }",
      "if (a == mid) { code = (i % 2 == 0) ? i + 1 : i; break; }",

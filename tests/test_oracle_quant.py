@@ -31,6 +31,11 @@ def _signed_codes(fmt, codes):
     if fmt == "int4_sym":
         q = _nibbles(codes).astype(np.int64)
         return np.where(q > 7, q - 16, q)
+    if fmt == "int3_sym":  # little-endian bit stream per row, element k at bits 3k..3k+2
+        bits = np.unpackbits(codes.astype(np.uint8), axis=1, bitorder="little").astype(np.int64)
+        bits = bits.reshape(codes.shape[0], -1, 3)
+        q = bits[..., 0] | (bits[..., 1] << 1) | (bits[..., 2] << 2)
+        return np.where(q > 3, q - 8, q)
     c = codes.astype(np.int64)
     q = np.stack([(c >> (2 * j)) & 3 for j in range(4)], axis=-1).reshape(codes.shape[0], -1)
     return np.where(q > 1, q - 4, q)
@@ -49,7 +54,8 @@ def _weights(N, K, seed=0, outliers=True):
 
 
 # --------------------------------------------------------------- symmetric INT
-@pytest.mark.parametrize("fmt,qmax", [("int2_sym", 1), ("int4_sym", 7), ("int8_sym", 127)])
+@pytest.mark.parametrize("fmt,qmax", [("int2_sym", 1), ("int3_sym", 3), ("int4_sym", 7),
+                                      ("int8_sym", 127)])
 @pytest.mark.parametrize("G", [32, 64, 128, 256])
 def test_sym_properties(orc, fmt, qmax, G):
     N, K = 48, 512
@@ -75,7 +81,8 @@ def test_sym_properties(orc, fmt, qmax, G):
     assert np.array_equal(dq.astype(np.float64), q * sk)
 
 
-@pytest.mark.parametrize("fmt,qmax", [("int2_sym", 1), ("int4_sym", 7), ("int8_sym", 127)])
+@pytest.mark.parametrize("fmt,qmax", [("int2_sym", 1), ("int3_sym", 3), ("int4_sym", 7),
+                                      ("int8_sym", 127)])
 @pytest.mark.parametrize("sval", [1.0, 2.0 ** -7, 0.0173])
 def test_sym_round_trip_every_code(orc, fmt, qmax, sval):
     """W = q*s for every representable q gives back q and s exactly."""
