@@ -316,8 +316,19 @@ def cpu_baseline(wl, Ms, seconds, calibrate_only=False):
         t += cpu_sample(wl, Ms, rows, data)
         reps += 1
     value = reps * bytes_per_sample / t / 1e9
-    return {"value": value, "unit": "GB/s", "cores": orc.threads(), "kind": "oracle",
-            "sample": desc + f", {reps} pass(es), {t:.1f} s"}, t / reps
+    cores = orc.threads()
+    # the same oracle on one thread, on a smaller sample (a few seconds)
+    orc.set_threads(1)
+    try:
+        rows1 = max(1, rows // max(1, cores) // 2)
+        t1 = cpu_sample(wl, Ms, rows1, data)
+        single = (total_bytes * rows1 / wl.N) / t1 / 1e9
+    finally:
+        orc.set_threads(cores)
+    return {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": desc + f", {reps} pass(es), {t:.1f} s",
+            "single_thread": {"value": single, "unit": "GB/s",
+                              "sample": f"{rows1} rows, 1 thread, {t1:.1f} s"}}, t / reps
 
 
 # ------------------------------------------------------------------ main

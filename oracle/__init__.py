@@ -68,6 +68,7 @@ def _declare(lib):
         "orc_linear_sampled": ([c_int, i64, i64, c_int, ptr, ptr, ptr, ptr, ptr, i64, ptr, ptr,
                                 ptr, ptr], c_int),
         "orc_threads": ([], c_int),
+        "orc_set_threads": ([c_int], None),
         "orc_silu": ([dbl], dbl),
         "orc_swiglu": ([ptr, i64, i64, ptr], c_int),
         "orc_quant_act_int8": ([ptr, i64, i64, ptr, ptr], c_int),
@@ -278,6 +279,9 @@ class Oracle:
                                         _p(aux), _p(x_bits), _p(b), S, _p(ms), _p(ns), _p(y),
                                         _p(y64)), "linear_sampled")
         return y, y64
+
+    def set_threads(self, n: int) -> None:
+        self.lib.orc_set_threads(int(n))
 
     def threads(self) -> int:
         return int(self.lib.orc_threads())

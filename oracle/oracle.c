@@ -755,9 +755,13 @@ int orc_linear_sampled(int fmt, int64_t N, int64_t K, int G, const void* codes,
 
 /* Threads that OpenMP uses for the parallel loops above. */
 int orc_threads(void);
+/* Threads the parallel loops use from now on (n >= 1). */
+void orc_set_threads(int n);
 #ifdef _OPENMP
 #include <omp.h>
 int orc_threads(void) { return omp_get_max_threads(); }
+void orc_set_threads(int n) { omp_set_num_threads(n < 1 ? 1 : n); }
 #else
 int orc_threads(void) { return 1; }
+void orc_set_threads(int n) { (void)n; }
 #endif

@@ -50,3 +50,15 @@ def test_reference_arm_other_ranks_exit_quietly():
                           "--steps", "1", "--warmup", "0"], cwd=ROOT, env=env,
                          capture_output=True, text=True, timeout=300)
     assert out.returncode == 0 and out.stdout.strip() == ""
+
+
+def test_cpu_baseline_reports_all_threads_and_one():
+    """The benchmark's oracle baseline on a small workload: a value on all
+    threads and one on a single thread, both positive, threads restored."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import oracle
+    import synth.workloads as W
+    cb, per_pass = bench.cpu_baseline(W.PR1, W.PR1.Ms, 0.5)
+    assert cb["value"] > 0 and cb["single_thread"]["value"] > 0 and per_pass > 0
+    assert cb["kind"] == "oracle" and cb["cores"] == oracle.Oracle().threads()
