@@ -295,7 +295,9 @@ def cpu_baseline(wl, Ms, seconds, calibrate_only=False):
 
     orc = oracle.Oracle()
     Wd = W.make_weight(wl)
+    tq0 = time.perf_counter()
     codes, scales, aux = orc.quantize(wl.fmt, Wd, wl.group_size)
+    quantize_s = time.perf_counter() - tq0          # the offline phase, whole weight
     del Wd
     xa = W.make_x(wl, max(Ms))
     b = W.make_bias(wl)
@@ -328,7 +330,8 @@ def cpu_baseline(wl, Ms, seconds, calibrate_only=False):
     return {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
             "sample": desc + f", {reps} pass(es), {t:.1f} s",
             "single_thread": {"value": single, "unit": "GB/s",
-                              "sample": f"{rows1} rows, 1 thread, {t1:.1f} s"}}, t / reps
+                              "sample": f"{rows1} rows, 1 thread, {t1:.1f} s"},
+            "quantize_s": quantize_s}, t / reps
 
 
 # ------------------------------------------------------------------ main

@@ -62,3 +62,4 @@ def test_cpu_baseline_reports_all_threads_and_one():
     cb, per_pass = bench.cpu_baseline(W.PR1, W.PR1.Ms, 0.5)
     assert cb["value"] > 0 and cb["single_thread"]["value"] > 0 and per_pass > 0
     assert cb["kind"] == "oracle" and cb["cores"] == oracle.Oracle().threads()
+    assert cb["quantize_s"] > 0
