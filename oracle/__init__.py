@@ -73,6 +73,7 @@ def _declare(lib):
         "orc_swiglu": ([ptr, i64, i64, ptr], c_int),
         "orc_quant_act_int8": ([ptr, i64, i64, ptr, ptr], c_int),
         "orc_linear_a8": ([c_int, ptr, ptr, i64, i64, c_int, ptr, ptr, ptr, i64, ptr, ptr], c_int),
+        "orc_round_bf16_array": ([ptr, i64, ptr], c_int),
         "orc_addmm_requant_int8": ([ptr, ptr, i64, i64, c_int, ptr, ptr, i64, dbl, dbl, c_int,
                                     ctypes.c_uint64], c_int),
     }
@@ -216,6 +217,32 @@ class Oracle:
         y64 = np.zeros((M, N), dtype=np.float64)
         b = None if bias_bits is None else np.ascontiguousarray(bias_bits, dtype=np.uint16)
         _ok(self.lib.orc_linear(_p(x_bits), _p(dq), _p(b), M, N, K, _p(y), _p(y64)), "linear")
+        return y, y64
+
+    def linear_full(self, x_bits: np.ndarray, dq: np.ndarray, bias_bits=None,
+                    rows_per_chunk: int = 4096):
+        """(y_bf16_bits [M,N], y_f64 [M,N]) for y = x . dq^T + bias, with the
+        fp64 product taken by numpy's fp64 matmul (a library primitive)
+        instead of orc_linear's loop, so that full-size outputs cost seconds.
+
+        Same definition as ``linear``: exact bf16 and fp32 operands widened
+        to fp64, one fp64 sum per output plus the bias, rounded once to bf16
+        by ``orc_round_bf16_array``.  Only the order of the fp64 additions
+        differs (fp64 error far below half a bf16 step), which the pins
+        check against ``linear``."""
+        x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+        M, K = x_bits.shape
+        N = dq.shape[0]
+        assert dq.shape[1] == K
+        xf = bits_to_f32(x_bits).astype(np.float64)
+        y64 = np.empty((M, N), dtype=np.float64)
+        for n0 in range(0, N, rows_per_chunk):
+            n1 = min(N, n0 + rows_per_chunk)
+            y64[:, n0:n1] = xf @ np.asarray(dq[n0:n1], dtype=np.float32).astype(np.float64).T
+        if bias_bits is not None:
+            y64 += bits_to_f32(np.asarray(bias_bits, dtype=np.uint16)).astype(np.float64)[None, :]
+        y = np.zeros((M, N), dtype=np.uint16)
+        _ok(self.lib.orc_round_bf16_array(_p(y64), M * N, _p(y)), "round_bf16_array")
         return y, y64
 
     def quant_act_int8(self, x_bits: np.ndarray):

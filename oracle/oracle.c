@@ -626,6 +626,16 @@ int orc_linear(const uint16_t* x, const float* dq, const uint16_t* bias, int64_t
   return 0;
 }
 
+/* y[i] = bf16(v[i]) (round to nearest even) for n values: the rounding of a
+ * full fp64 product computed elsewhere (a library fp64 matmul) to the output
+ * type, with the same rounding as orc_linear. */
+int orc_round_bf16_array(const double* v, int64_t n, uint16_t* y) {
+  if (n < 0) return 1;
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < n; ++i) y[i] = orc_f64_to_bf16(v[i]);
+  return 0;
+}
+
 /* Per-token INT8 activation quantization: xq int8 [M, K], sx f32 [M]. */
 int orc_quant_act_int8(const uint16_t* x, int64_t M, int64_t K, int8_t* xq, float* sx) {
   if (M < 0 || K <= 0) return 1;

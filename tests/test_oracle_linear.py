@@ -174,3 +174,65 @@ def test_empty_batch(orc):
     x = np.zeros((0, 8), np.uint16)
     y, y64 = orc.linear(x, dq)
     assert y.shape == (0, 4)
+
+
+@pytest.mark.parametrize("K", [1, 7, 32])
+def test_linear_full_matches_exact_rational(orc, K):
+    """The library-matmul product against exact rational sums (tiny K)."""
+    M, N = 3, 5
+    rng = np.random.default_rng(100 + K)
+    x = synth.f64_to_bf16_bits(rng.standard_normal((M, K)))
+    dq = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    b = synth.f64_to_bf16_bits(rng.standard_normal(N) * 0.01)
+    y, y64 = orc.linear_full(x, dq, b)
+    xf, bf = oracle.bits_to_f32(x), oracle.bits_to_f32(b)
+    for m in range(M):
+        for n in range(N):
+            exact = sum(Fraction(float(xf[m, k])) * Fraction(float(dq[n, k])) for k in range(K))
+            exact += Fraction(float(bf[n]))
+            absum = sum(abs(float(xf[m, k]) * float(dq[n, k])) for k in range(K)) + abs(float(bf[n]))
+            assert abs(Fraction(float(y64[m, n])) - exact) <= Fraction((K + 1) * 2.0 ** -52 * absum)
+            want = _bf16_exact_rne(exact)
+            got = Fraction(float(oracle.bits_to_f32(np.array([y[m, n]], np.uint16))[0]))
+            if got != want:
+                assert abs(exact - (got + want) / 2) <= Fraction((K + 1) * 2.0 ** -52 * absum)
+
+
+@pytest.mark.parametrize("fmt,G", [("int4_asym", 128), ("nvfp4", 16), ("int8_sym", 256)])
+def test_linear_full_equals_loop(orc, fmt, G):
+    """The library-matmul product and the increasing-k loop agree: fp64 values
+    within the summation-order bound, bf16 outputs identical (a difference
+    needs an exact value within ~1e-13 of a bf16 rounding boundary).  A
+    transposed weight, a dropped bias or another rounding would fail here.
+    The chunking over rows is exercised by a chunk smaller than N."""
+    M, N, K = 9, 272, 2048
+    W = synth.weight(33, N, K, sigma=0.02, outlier_count=N * K // 1000, outlier_mult=20.0)
+    codes, scales, aux = orc.quantize(fmt, W, G)
+    dq = orc.dequant(fmt, codes, scales, aux, N, K, G)
+    x = synth.activations(33, M, K)
+    b = synth.bias(33, N)
+    y, y64 = orc.linear(x, dq, b)
+    yf, yf64 = orc.linear_full(x, dq, b, rows_per_chunk=96)
+    absum = np.abs(oracle.bits_to_f32(x).astype(np.float64)) @ np.abs(dq.astype(np.float64)).T
+    assert np.all(np.abs(yf64 - y64) <= 2 * (K + 1) * 2.0 ** -52 * (absum + 1.0))
+    assert np.array_equal(yf, y)
+    # no bias: the same product without the bias term
+    y0, _ = orc.linear(x, dq, None)
+    yf0, _ = orc.linear_full(x, dq, None)
+    assert np.array_equal(yf0, y0)
+    assert not np.array_equal(yf0, yf)
+
+
+def test_linear_full_integer_case(orc):
+    """Integer operands: the library product is exact and equals numpy's
+    integer matmul bit for bit (orientation: y[m, n] = sum_k x[m, k] w[n, k])."""
+    M, N, K = 5, 40, 256
+    rng = np.random.default_rng(7)
+    codes, scales, aux, wval = _int_case("int4_sym", N, K, 64, rng)
+    xi = rng.integers(-4, 5, size=(M, K))
+    x = synth.f64_to_bf16_bits(xi.astype(np.float64))
+    dq = orc.dequant("int4_sym", codes, scales, aux, N, K, 64)
+    y, y64 = orc.linear_full(x, dq, None)
+    ref = (xi @ wval.astype(np.int64).T).astype(np.float64)
+    assert np.array_equal(y64, ref)
+    assert np.array_equal(y, synth.f64_to_bf16_bits(ref))
