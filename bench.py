@@ -10,6 +10,12 @@ divided by the device time of the K timed steps (CUDA events, max over
 ranks).  The timed steps are replayed from CUDA graphs so that host launch
 overhead does not pad the device timeline.
 
+With the default workload the line also carries ``prefill``: the other half
+of the metric, the compute-bound INT8 g256 8192 x 8192 layer at
+M in {1024, 2048, 4096}, timed by the same protocol (its own step count,
+``--prefill-steps`` capped by ``--steps``) and reported in TFLOP/s with its
+own roofline, e2e and CPU baseline.
+
 ``e2e`` repeats the K steps through the public Python API with host
 activations: each call copies X from pinned host memory, runs the linear and
 copies Y back (both copies inside the timed region).
@@ -58,6 +64,10 @@ def parse():
                     help="skip the per-call percentiles and the cuBLAS bf16 context line")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle sample")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="with the default decode workload, skip the prefill half of the metric")
+    ap.add_argument("--prefill-steps", type=int, default=300,
+                    help="timed steps of the prefill half (capped by --steps)")
     return ap.parse_args()
 
 
@@ -288,11 +298,14 @@ def cpu_sample(wl, Ms, rows, data):
 
 def cpu_baseline(wl, Ms, seconds, calibrate_only=False):
     """The oracle, as it stands, on a bounded sample of the workload (dequant
-    + fp64 dot products for a subset of output rows, every token); GB/s is the
-    workload's algorithmic bytes scaled by the fraction of rows computed."""
+    + fp64 dot products for a subset of output rows, every token), in the
+    workload's unit: algorithmic GB/s (decode) or TFLOP/s (prefill), scaled by
+    the fraction of rows computed."""
     import oracle
     import synth.workloads as W
 
+    tflops_metric = min(Ms) >= 1024
+    unit, scale = ("TFLOP/s", 1e12) if tflops_metric else ("GB/s", 1e9)
     orc = oracle.Oracle()
     Wd = W.make_weight(wl)
     tq0 = time.perf_counter()
@@ -302,36 +315,201 @@ def cpu_baseline(wl, Ms, seconds, calibrate_only=False):
     xa = W.make_x(wl, max(Ms))
     b = W.make_bias(wl)
     data = (orc, codes, scales, aux, xa, b)
-    total_bytes = sum(W.algorithmic_bytes(wl, M) for M in Ms)
+    if tflops_metric:
+        total_work = sum(W.flops(M, wl.N, wl.K) for M in Ms)
+    else:
+        total_work = sum(W.algorithmic_bytes(wl, M) for M in Ms)
     rows = 16
     t = cpu_sample(wl, Ms, rows, data)
     rows = int(min(wl.N, max(1, rows * seconds / max(t, 1e-4))))
     desc = (f"{rows} of {wl.N} output rows for every token of M in {list(Ms)}, "
             f"{orc.threads()} threads")
-    bytes_per_sample = total_bytes * rows / wl.N
+    work_per_sample = total_work * rows / wl.N
     if calibrate_only:
         return {"rows": rows, "data": data, "cores": orc.threads(), "sample_desc": desc,
-                "bytes_per_sample": bytes_per_sample}, 0.0
+                "work_per_sample": work_per_sample}, 0.0
     # repeat the pass (a whole-workload pass can be far shorter than the target)
     reps, t = 0, 0.0
     while reps == 0 or t < 0.8 * seconds:
         t += cpu_sample(wl, Ms, rows, data)
         reps += 1
-    value = reps * bytes_per_sample / t / 1e9
+    value = reps * work_per_sample / t / scale
     cores = orc.threads()
     # the same oracle on one thread, on a smaller sample (a few seconds)
     orc.set_threads(1)
     try:
         rows1 = max(1, rows // max(1, cores) // 2)
         t1 = cpu_sample(wl, Ms, rows1, data)
-        single = (total_bytes * rows1 / wl.N) / t1 / 1e9
+        single = (total_work * rows1 / wl.N) / t1 / scale
     finally:
         orc.set_threads(cores)
-    return {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+    return {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
             "sample": desc + f", {reps} pass(es), {t:.1f} s",
-            "single_thread": {"value": single, "unit": "GB/s",
+            "single_thread": {"value": single, "unit": unit,
                               "sample": f"{rows1} rows, 1 thread, {t1:.1f} s"},
             "quantize_s": quantize_s}, t / reps
+
+
+# ------------------------------------------------------------------ timing
+def time_workload(wl, Ms, steps, warmup, device, l2, world, local_rank, do_e2e):
+    """Device time of exactly `steps` steps of `wl` (one wq_linear per M, each
+    on the next resident weight copy), replayed from CUDA graphs, CUDA events
+    on the launch stream, max over ranks; plus the end-to-end pass through
+    the public API with host buffers.  Returns the numbers the JSON line
+    reports for this workload."""
+    import torch
+
+    import mixed_gemm_b200 as wq
+    import synth.workloads as W
+
+    tflops_metric = min(Ms) >= 1024
+    unit = "TFLOP/s" if tflops_metric else "GB/s"
+    weights, xs, bias, outs, xa = build_workload(wl, Ms, device, 3 * l2)
+    R = len(weights)
+    launches_per_step = len(Ms)
+    step_bytes = sum(W.algorithmic_bytes(wl, M) for M in Ms)
+    step_flops = sum(W.flops(M, wl.N, wl.K) for M in Ms)
+    stream = torch.cuda.Stream(device)
+    counter = [0]
+
+    def step():
+        for M in Ms:
+            pw = weights[counter[0] % R]
+            counter[0] += 1
+            wq.wq_linear(xs[M], pw.w, pw.scales, pw.aux, bias, M, wl.N, wl.K, wl.fmt,
+                         wl.group_size, outs[M], stream)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier(device_ids=[local_rank])
+
+    # graphs of C steps each (the weight copies rotate inside the graph)
+    C = max(1, min(200, steps))
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            step()
+    torch.cuda.synchronize()
+
+    def capture(nsteps):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(nsteps):
+                step()
+        return g
+
+    g_main = capture(C)
+    rem = steps % C
+    g_rem = capture(rem) if rem else None
+    reps = steps // C
+
+    # every graph is replayed once, untimed, whatever the step counts (a
+    # graph's first launch uploads it); then W untimed warm-up steps
+    with torch.cuda.stream(stream):
+        g_main.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        for _ in range(warmup // C):
+            g_main.replay()
+        for _ in range(warmup % C):
+            step()
+    torch.cuda.synchronize()
+
+    props = torch.cuda.get_device_properties(device)
+    uuid = getattr(props, "uuid", None)
+    clocks = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(device.index))
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    with torch.cuda.stream(stream):   # graphs replay on the current stream
+        ev0.record(stream)
+        for _ in range(reps):
+            g_main.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        ev1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier()
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), world, device)
+    sec = ms_total / 1e3
+    if tflops_metric:
+        value = whole_job_value(world, steps, step_flops, sec, 1e12)
+    else:
+        value = whole_job_value(world, steps, step_bytes, sec, 1e9)
+    per_launch_s = sec / (steps * launches_per_step)
+
+    # roofline of the dominant kernel (every launch in the step runs it)
+    pk, pk_kind = peaks()
+    if tflops_metric:
+        achieved = step_flops / launches_per_step / per_launch_s / 1e12
+        peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        bound, r_unit = "tensor", "TFLOP/s"
+    else:
+        achieved = step_bytes / launches_per_step / per_launch_s / 1e9
+        peak = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        bound, r_unit = "hbm", "GB/s"
+    kern_src = ["wq_decode.cu", "wq_internal.cuh"] if max(Ms) <= 16 else ["wq_prefill.cu",
+                                                                            "wq_internal.cuh"]
+    traffic = recorded_traffic(kern_src[0], wl.name)
+
+    # e2e through the public API with host activations
+    e2e = None
+    if do_e2e:
+        xh = {M: torch.from_numpy(xa[:M].view(np.int16).copy()).view(torch.bfloat16).pin_memory()
+              for M in Ms}
+        yh = {M: torch.empty((M, wl.N), dtype=torch.bfloat16).pin_memory() for M in Ms}
+        e2e_steps = max(3, min(steps, 2000))
+        k = [0]
+
+        def e2e_step():
+            # every batch of the step from pinned host memory, results copied
+            # back; one wait per step (the host may read every result after it)
+            for M in Ms:
+                pw = weights[k[0] % R]
+                k[0] += 1
+                wq.linear(xh[M], pw, bias, out=yh[M], stream=stream, sync=False)
+            stream.synchronize()
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        es = max_over_ranks(e0.elapsed_time(e1), world, device) / 1e3
+        ev = whole_job_value(world, e2e_steps, step_flops if tflops_metric else step_bytes, es,
+                             1e12 if tflops_metric else 1e9)
+        e2e = {"value": ev, "unit": unit, "steps": e2e_steps,
+               "h2d_bytes_per_step": sum(M * wl.K * 2 for M in Ms),
+               "d2h_bytes_per_step": sum(M * wl.N * 2 for M in Ms)}
+    del g_main, g_rem
+    return {
+        "value": value, "unit": unit, "steps": steps, "warmup": warmup,
+        "ms_per_step": ms_total / steps,
+        "config": {"workload": wl.name, "format": wl.fmt, "group_size": wl.group_size,
+                   "N": wl.N, "K": wl.K, "Ms": list(Ms), "parallelism": f"replicas{world}",
+                   "l2": f"rotating {R} packed-weight copies ({R * weights[0].nbytes / 2**20:.0f} "
+                         f"MiB > 3x L2 {l2 / 2**20:.0f} MiB)",
+                   "timing": f"CUDA graphs of {C} steps, each replayed once untimed before "
+                             "the warm-up; CUDA events on the launch stream"},
+        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": r_unit,
+                     "frac": achieved / peak, "traffic": traffic, "peak_source": pk_kind,
+                     "kernel": "decode_kernel" if max(Ms) <= 16 else "prefill_kernel"},
+        "gpu_launches": steps * launches_per_step,
+        "clocks": clk,
+        "e2e": e2e,
+        "_state": (weights, xs, bias, outs, stream),
+    }
 
 
 # ------------------------------------------------------------------ main
@@ -359,17 +537,18 @@ def main():
             cpu_sample(wl, Ms, rows, cb["data"])
         times = [cpu_sample(wl, Ms, rows, cb["data"]) for _ in range(max(1, args.steps))]
         t = sum(times)
-        value = len(times) * cb["bytes_per_sample"] / t / 1e9
-        desc = {"value": value, "unit": "GB/s", "cores": cb["cores"], "kind": "oracle",
+        scale = 1e12 if tflops_metric else 1e9
+        value = len(times) * cb["work_per_sample"] / t / scale
+        desc = {"value": value, "unit": unit, "cores": cb["cores"], "kind": "oracle",
                 "sample": cb["sample_desc"]}
-        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": unit,
                 "n_gpus": args.gpus, "steps": len(times), "warmup": args.warmup,
                 "ms_per_step": t / len(times) * 1e3, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f64", "data": "synthetic",
                 "config": {"workload": wl.name, "N": wl.N, "K": wl.K, "Ms": list(Ms),
                            "format": wl.fmt, "group_size": wl.group_size},
                 "cpu_baseline": desc,
-                "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return
@@ -386,169 +565,54 @@ def main():
         torch.cuda.set_device(0)
     device = torch.device("cuda", torch.cuda.current_device())
 
-    import mixed_gemm_b200 as wq
+    import mixed_gemm_b200  # noqa: F401  (fails loudly when the library is missing)
 
     props = torch.cuda.get_device_properties(device)
     l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20)
-    weights, xs, bias, outs, xa = build_workload(wl, Ms, device, 3 * l2)
-    R = len(weights)
-    launches_per_step = len(Ms)
-    step_bytes = sum(W.algorithmic_bytes(wl, M) for M in Ms)
-    step_flops = sum(W.flops(M, wl.N, wl.K) for M in Ms)
-    stream = torch.cuda.Stream(device)
-    counter = [0]
-
-    def step():
-        for M in Ms:
-            pw = weights[counter[0] % R]
-            counter[0] += 1
-            wq.wq_linear(xs[M], pw.w, pw.scales, pw.aux, bias, M, wl.N, wl.K, wl.fmt,
-                         wl.group_size, outs[M], stream)
-
-    def barrier():
-        if world > 1:
-            import torch.distributed as dist
-            dist.barrier(device_ids=[local_rank])
-
-    # graphs of C steps each (the weight copies rotate inside the graph)
-    C = max(1, min(200, args.steps))
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            step()
-    torch.cuda.synchronize()
-
-    def capture(nsteps):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for _ in range(nsteps):
-                step()
-        return g
-
-    g_main = capture(C)
-    rem = args.steps % C
-    g_rem = capture(rem) if rem else None
-    reps = args.steps // C
-
-    # warm-up: W untimed steps
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup // C):
-            g_main.replay()
-        for _ in range(args.warmup % C):
-            step()
-    torch.cuda.synchronize()
-
-    uuid = getattr(props, "uuid", None)
-    clocks = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(device.index))
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.3)
-    with torch.cuda.stream(stream):   # graphs replay on the current stream
-        ev0.record(stream)
-        for _ in range(reps):
-            g_main.replay()
-        if g_rem is not None:
-            g_rem.replay()
-        ev1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    clk = clocks.stop()
-    ms_total = max_over_ranks(ev0.elapsed_time(ev1), world, device)
-    sec = ms_total / 1e3
-    if tflops_metric:
-        value = whole_job_value(world, args.steps, step_flops, sec, 1e12)
-    else:
-        value = whole_job_value(world, args.steps, step_bytes, sec, 1e9)
-    per_launch_s = sec / (args.steps * launches_per_step)
-
-    # roofline of the dominant kernel (every launch in the step runs it)
-    pk, pk_kind = peaks()
-    if tflops_metric:
-        achieved = step_flops / launches_per_step / per_launch_s / 1e12
-        peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-        bound, r_unit = "tensor", "TFLOP/s"
-    else:
-        achieved = step_bytes / launches_per_step / per_launch_s / 1e9
-        peak = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-        bound, r_unit = "hbm", "GB/s"
-    kern_src = ["wq_decode.cu", "wq_internal.cuh"] if max(Ms) <= 16 else ["wq_prefill.cu",
-                                                                            "wq_internal.cuh"]
-    traffic = recorded_traffic(kern_src[0], wl.name)
-
-    # e2e through the public API with host activations
-    e2e = None
-    if not args.no_e2e:
-        xh = {M: torch.from_numpy(xa[:M].view(np.int16).copy()).view(torch.bfloat16).pin_memory()
-              for M in Ms}
-        yh = {M: torch.empty((M, wl.N), dtype=torch.bfloat16).pin_memory() for M in Ms}
-        e2e_steps = max(3, min(args.steps, 2000))
-        k = [0]
-
-        def e2e_step():
-            # every batch of the step from pinned host memory, results copied
-            # back; one wait per step (the host may read every result after it)
-            for M in Ms:
-                pw = weights[k[0] % R]
-                k[0] += 1
-                wq.linear(xh[M], pw, bias, out=yh[M], sync=False)
-            stream.synchronize()
-
-        with torch.cuda.stream(stream):
-            for _ in range(3):
-                e2e_step()
-        torch.cuda.synchronize()
-        barrier()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(e2e_steps):
-                e2e_step()
-            e1.record(stream)
-        torch.cuda.synchronize()
-        barrier()
-        es = max_over_ranks(e0.elapsed_time(e1), world, device) / 1e3
-        ev = whole_job_value(world, e2e_steps, step_flops if tflops_metric else step_bytes, es,
-                             1e12 if tflops_metric else 1e9)
-        e2e = {"value": ev, "unit": unit, "steps": e2e_steps,
-               "h2d_bytes_per_step": sum(M * wl.K * 2 for M in Ms),
-               "d2h_bytes_per_step": sum(M * wl.N * 2 for M in Ms)}
-
+    head = time_workload(wl, Ms, args.steps, args.warmup, device, l2, world, local_rank,
+                         not args.no_e2e)
     ctx = None
     if rank == 0 and world == 1 and not args.no_context:
-        ctx = context_numbers(wl, Ms, weights, xs, bias, outs, stream, l2, device)
+        ctx = context_numbers(wl, Ms, *head["_state"][:5], l2, device)
+    del head["_state"]
+    torch.cuda.empty_cache()
+
+    # the other half of the metric: the compute-bound prefill sweep, timed by
+    # the same protocol on its own step count (a prefill step is ~1.5 ms)
+    second = None
+    if not args.no_prefill and not tflops_metric and args.workload == W.DECODE.name:
+        pwl = W.PREFILL
+        psteps = max(1, min(args.steps, args.prefill_steps))
+        second = time_workload(pwl, pwl.Ms, psteps, max(3, min(args.warmup, psteps)), device, l2,
+                               world, local_rank, not args.no_e2e)
+        pctx = None
+        if rank == 0 and world == 1 and not args.no_context:
+            pctx = context_numbers(pwl, pwl.Ms, *second["_state"][:5], l2, device)
+        del second["_state"]
+        second["context"] = pctx
+        torch.cuda.empty_cache()
 
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb, _ = cpu_baseline(wl, Ms, args.cpu_seconds)
+        if second is not None:
+            second["cpu_baseline"], _ = cpu_baseline(W.PREFILL, W.PREFILL.Ms, args.cpu_seconds)
 
     if world > 1:
         import torch.distributed as dist
-        del g_main, g_rem
         dist.destroy_process_group()
     if rank != 0:
         return
     line = {
-        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": wl.name, "format": wl.fmt, "group_size": wl.group_size,
-                   "N": wl.N, "K": wl.K, "Ms": list(Ms), "parallelism": f"replicas{world}",
-                   "l2": f"rotating {R} packed-weight copies ({R * weights[0].nbytes / 2**20:.0f} "
-                         f"MiB > 3x L2 {l2 / 2**20:.0f} MiB)",
-                   "timing": f"CUDA graphs of {C} steps, CUDA events on the launch stream"},
-        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": r_unit,
-                     "frac": achieved / peak, "traffic": traffic,
-                     "peak_source": pk_kind,
-                     "kernel": "decode_kernel" if max(Ms) <= 16 else "prefill_kernel"},
-        "gpu_launches": args.steps * launches_per_step,
-        "clocks": clk,
-        "e2e": e2e,
-        "cpu_baseline": cb,
-        "context": ctx,
+        "metric": METRIC, "value": head["value"], "unit": unit, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": head["config"], "roofline": head["roofline"],
+        "gpu_launches": head["gpu_launches"], "clocks": head["clocks"], "e2e": head["e2e"],
+        "cpu_baseline": cb, "context": ctx,
     }
+    if second is not None:
+        line["prefill"] = second
     print(json.dumps(line), flush=True)
 
 

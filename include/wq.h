@@ -126,7 +126,11 @@ int wq_packed_sizes(int format, int64_t N, int64_t K, int group_size, size_t* w_
  * A pure permutation: every byte pattern is accepted and round-trips through
  * wq_unpack.  The Petit README "Known limitations" (positive scales, no
  * negative-zero FP4 codes) needs no check here, because every E4M3 / E2M1
- * bit pattern decodes by its definition.  Asynchronous; never synchronizes. */
+ * bit pattern decodes by its definition.  Asynchronous; never synchronizes.
+ * Ends with a 4-byte memset of a library word on `stream` (a stream operation
+ * that is not a kernel), so that a wq_linear enqueued after it on the same
+ * stream cannot start reading the packed buffers before they are written
+ * (see wq_linear on programmatic dependent launch). */
 int wq_pack(int format, int64_t N, int64_t K, int group_size, const void* codes,
             const void* scales, const void* aux, void* packed_w, void* packed_scales,
             void* packed_aux, void* stream);
@@ -159,8 +163,11 @@ int wq_dequant(int format, int64_t N, int64_t K, int group_size, const void* pac
  * the previous kernel on `stream` is finishing, requests the packed weight,
  * scales and aux at once, and reads x / writes out only after the previous
  * kernel has completed.  The packed buffers must therefore already be final
- * when the previous kernel on `stream` starts (pack at load time, or put any
- * other stream operation between wq_pack and the first wq_linear).
+ * when the previous kernel on `stream` starts.  wq_pack, wq_quantize and
+ * wq_addmm_requant end with a stream operation that is not a kernel, which
+ * satisfies this on their stream; a caller that writes packed buffers with
+ * its own kernels must do the same (any memset or memcpy on the stream after
+ * them) or synchronize before the first wq_linear that reads them.
  * M <= 16 runs the decode kernel (register dequant, warp-level tensor-core
  * fragments, split-K over warps) unless K is too long for its staged
  * activation slice; larger M (and those) run the prefill kernel (TMA into
@@ -241,7 +248,9 @@ int wq_linear_swiglu_static(const void* x2, const void* packed_w, const void* sc
  *   packed_scales  device, unchanged
  *   mat1, mat2     device bf16 [N, rank] and [rank, K] (rank 0: no update)
  * Other formats return WQ_ERR_UNSUPPORTED.  Offline; asynchronous.  Repeated
- * merges are lossy (each one requantizes).
+ * merges are lossy (each one requantizes).  Ends, like wq_pack, with a
+ * 4-byte memset of a library word on `stream`, so that a following
+ * wq_linear on the same stream reads the merged codes.
  * Source: piper-kernels README (weight.addmm_(lora_b, lora_a, alpha=...,
  * rounding_seed=seed): beta * weight + alpha * (mat1 @ mat2), requantized,
  * deterministic row scales kept, stochastic choice of one of the two adjacent
@@ -254,7 +263,8 @@ int wq_addmm_requant(int format, int64_t N, int64_t K, int group_size, void* pac
  * canonical codes / scales / aux (device), bit-identical to the CPU
  * definitions listed above.  CB4 reads its 16 centroids from `aux`
  * (device f32[16], left unchanged) and writes the row norms; NVFP4 writes the
- * tensor scale into `aux`.  Synchronizes `stream` for NVFP4 (two passes).
+ * tensor scale into `aux` (three stream-ordered passes: tensor maximum,
+ * codes, tensor scale).  Asynchronous; ends, like wq_pack, with a 4-byte memset.
  * The FP8 formats write fp32 scales amax/448 (E4M3) or amax/57344 (E5M2).
  * Source: piper-kernels README "ConvRot INT8" (ConvRotInt8Tensor.from_hp
  * quantizes a dense weight, group_size=256); Mamba-2 pack helper (scale =
@@ -272,8 +282,9 @@ int wq_lloyd_max_centroids(int bits, float* centroids_out);
 /* The kernels' own error word on the current device.  Every wait of the
  * prefill kernel on a shared-memory barrier has an iteration limit; a wait that
  * runs out sets a bit here (1 producer, 2 producer drain, 4/8 MMA waits, 16
- * MMA drain, 32 dequant, 64 epilogue) and the thread block winds down instead
- * of hanging, leaving the CUDA context usable.  Synchronizes the device (a
+ * MMA drain, 32 dequant, 64 epilogue; 128 the decode kernel's wait for its
+ * staged activation slice) and the thread block winds down instead of
+ * hanging, leaving the CUDA context usable.  Synchronizes the device (a
  * symbol copy).  Writes the word to *value, clears it when `clear` is non-zero,
  * and returns WQ_ERR_DEVICE_CHECK when it was non-zero, WQ_OK otherwise. */
 int wq_device_error(unsigned* value, int clear);

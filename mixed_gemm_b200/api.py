@@ -77,38 +77,52 @@ def quantize_and_pack(w: torch.Tensor, fmt: str, group_size: int = 0, centroids=
     return pack(fmt, N, K, group_size, codes, scales, aux, stream)
 
 
+def _torch_stream(stream, dev) -> torch.cuda.Stream:
+    """The torch stream object for ``stream`` (None: the device's current
+    stream; an integer: an existing cudaStream_t)."""
+    if stream is None:
+        return torch.cuda.current_stream(dev)
+    if isinstance(stream, int):
+        return torch.cuda.ExternalStream(stream, device=dev)
+    return stream
+
+
 def linear(x: torch.Tensor, weight: PackedWeight, bias: torch.Tensor | None = None,
            out: torch.Tensor | None = None, stream=None, sync: bool = True) -> torch.Tensor:
     """y = x @ dequant(weight).T + bias, bf16.  ``x``: [..., K] bf16.
 
     A host (CPU) ``x`` is copied to the weight's device and the result copied
-    back, so the call works end to end from host memory.  With a host ``x``
-    and ``sync=False`` the copy back is only enqueued (into ``out``, which
-    should then be pinned host memory): synchronize the stream before reading
-    it, e.g. once after several calls.
+    back, so the call works end to end from host memory; both copies and the
+    linear run in order on ``stream`` (default: the current stream).  With a
+    host ``x`` and ``sync=False`` the copy back is only enqueued (into
+    ``out``, which should then be pinned host memory): synchronize the stream
+    before reading it, e.g. once after several calls.
     """
     host = not x.is_cuda
     dev = weight.w.device
     lead = x.shape[:-1]
     K = x.shape[-1]
     assert K == weight.K and x.dtype == torch.bfloat16
-    xd = x.reshape(-1, K)
+    s = _torch_stream(stream, dev)
+    with torch.cuda.stream(s):
+        xd = x.reshape(-1, K)
+        if host:
+            xd = xd.to(dev, non_blocking=True)
+        xd = xd.contiguous()
+        M = xd.shape[0]
+        if bias is not None and not bias.is_cuda:
+            bias = bias.to(dev, non_blocking=True)
+        y = out if (out is not None and not host) else torch.empty(
+            (M, weight.N), dtype=torch.bfloat16, device=dev)
+        wq_linear(xd, weight.w, weight.scales, weight.aux, bias, M, weight.N, K, weight.fmt,
+                  weight.group_size, y, s)
+        if host:
+            yh = out if out is not None else torch.empty((M, weight.N), dtype=torch.bfloat16,
+                                                          pin_memory=True)
+            yh.copy_(y, non_blocking=True)
     if host:
-        xd = xd.to(dev, non_blocking=True)
-    xd = xd.contiguous()
-    M = xd.shape[0]
-    if bias is not None and not bias.is_cuda:
-        bias = bias.to(dev, non_blocking=True)
-    y = out if (out is not None and not host) else torch.empty((M, weight.N), dtype=torch.bfloat16,
-                                                               device=dev)
-    wq_linear(xd, weight.w, weight.scales, weight.aux, bias, M, weight.N, K, weight.fmt,
-              weight.group_size, y, stream)
-    if host:
-        yh = out if out is not None else torch.empty((M, weight.N), dtype=torch.bfloat16,
-                                                      pin_memory=True)
-        yh.copy_(y, non_blocking=True)
         if sync:
-            torch.cuda.current_stream(dev).synchronize()
+            s.synchronize()
         return yh.reshape(*lead, weight.N)
     return y.reshape(*lead, weight.N)
 

@@ -76,7 +76,55 @@ std::mutex g_sm_mutex;
 int g_sm_count[64];
 bool g_sm_known[64];
 
+// A word of device memory that only the stream fence below writes.
+__device__ unsigned g_wq_stream_fence;
+std::mutex g_fence_mutex;
+void* g_fence_ptr[64];
+
+// Kernel attributes are per device: one entry per (device, kernel) that has
+// been given the larger shared-memory limit; a failed attempt is not cached.
+std::mutex g_attr_mutex;
+struct AttrEntry {
+  int dev;
+  const void* fn;
+};
+AttrEntry g_attr_done[1024];
+int g_attr_count = 0;
+
 }  // namespace
+
+cudaError_t end_weight_write(cudaStream_t st) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  void* p = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_fence_mutex);
+    if (!g_fence_ptr[dev]) {
+      e = cudaGetSymbolAddress(&g_fence_ptr[dev], g_wq_stream_fence);
+      if (e != cudaSuccess) {
+        g_fence_ptr[dev] = nullptr;
+        return e;
+      }
+    }
+    p = g_fence_ptr[dev];
+  }
+  return cudaMemsetAsync(p, 0, sizeof(unsigned), st);
+}
+
+cudaError_t ensure_max_dynamic_smem(const void* fn, int bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(g_attr_mutex);
+  for (int i = 0; i < g_attr_count; ++i)
+    if (g_attr_done[i].dev == dev && g_attr_done[i].fn == fn) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  if (g_attr_count < 1024) g_attr_done[g_attr_count++] = AttrEntry{dev, fn};
+  return cudaSuccess;
+}
 
 int device_sm_count() {
   int dev = 0;
@@ -146,7 +194,9 @@ int wq_pack(int f, int64_t N, int64_t K, int G, const void* codes, const void* s
   G = effective_group(f, G);
   bool need_aux = f == INT4_ASYM || f == CB4 || f == NVFP4;
   if (!codes || !scales || !pw || !ps || (need_aux && (!aux || !pa))) return WQ_ERR_INVALID_ARG;
-  return cuda_status(launch_pack(f, N, K, G, codes, scales, aux, pw, ps, pa, (cudaStream_t)stream));
+  cudaError_t e = launch_pack(f, N, K, G, codes, scales, aux, pw, ps, pa, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = end_weight_write((cudaStream_t)stream);
+  return cuda_status(e);
 }
 
 int wq_unpack(int f, int64_t N, int64_t K, int G, const void* pw, const void* ps, const void* pa,
@@ -177,7 +227,9 @@ int wq_quantize(int f, int64_t N, int64_t K, int G, const float* w, void* codes,
   bool need_aux = f == INT4_ASYM || f == CB4 || f == NVFP4;
   if (!w || !codes || !scales || (need_aux && !aux)) return WQ_ERR_INVALID_ARG;
   if (!aligned(w, 4) || (aux && !aligned(aux, 4))) return WQ_ERR_ALIGNMENT;
-  return cuda_status(launch_quantize(f, N, K, G, w, codes, scales, aux, (cudaStream_t)stream));
+  cudaError_t e = launch_quantize(f, N, K, G, w, codes, scales, aux, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = end_weight_write((cudaStream_t)stream);
+  return cuda_status(e);
 }
 
 int wq_linear(const void* x, const void* pw, const void* scales, const void* aux, const void* bias,
@@ -317,8 +369,10 @@ int wq_addmm_requant(int f, int64_t N, int64_t K, int G, void* pw, const void* p
   if (overlap(pw, wb, ps, sb) || overlap(pw, wb, mat1, N * rank * 2) ||
       overlap(pw, wb, mat2, rank * K * 2))
     return WQ_ERR_INVALID_ARG;
-  return cuda_status(launch_addmm_requant_int8(N, K, G, pw, ps, mat1, mat2, rank, alpha, beta,
-                                               use_seed, seed, (cudaStream_t)stream));
+  cudaError_t e = launch_addmm_requant_int8(N, K, G, pw, ps, mat1, mat2, rank, alpha, beta,
+                                            use_seed, seed, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = end_weight_write((cudaStream_t)stream);
+  return cuda_status(e);
 }
 
 // Lloyd-Max quantizer of N(0,1): thresholds at the midpoints of adjacent
@@ -357,7 +411,10 @@ int wq_lloyd_max_centroids(int bits, float* out) {
 
 int wq_device_error(unsigned* value, int clear) {
   if (!value) return WQ_ERR_INVALID_ARG;
+  unsigned dec = 0;
   if (read_device_error(value, clear != 0) != cudaSuccess) return WQ_ERR_CUDA;
+  if (read_decode_error(&dec, clear != 0) != cudaSuccess) return WQ_ERR_CUDA;
+  *value |= dec;
   return *value ? WQ_ERR_DEVICE_CHECK : WQ_OK;
 }
 

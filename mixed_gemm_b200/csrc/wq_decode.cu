@@ -37,6 +37,10 @@ namespace cg = cooperative_groups;
 
 namespace wq {
 
+// Error word of the decode kernel: bit 128 when the wait for its staged
+// activation slice ran out (that CTA then stores nothing).
+__device__ unsigned int g_wq_decode_error;
+
 namespace {
 
 struct DecodeParams {
@@ -95,7 +99,8 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
       : "memory");
 }
 // Bounded wait for phase 0 of the X-slice barrier.  The limit is far beyond
-// any copy time; a wait that runs out leaves the block's output unwritten.
+// any copy time; a wait that runs out sets bit 128 of the decode error word
+// and leaves the block's output unwritten.
 __device__ __forceinline__ bool mbar_wait0(uint32_t bar) {
   for (uint32_t i = 0; i < (1u << 22); ++i) {
     uint32_t ok;
@@ -108,6 +113,7 @@ __device__ __forceinline__ bool mbar_wait0(uint32_t bar) {
         : "memory");
     if (ok) return true;
   }
+  atomicOr(&g_wq_decode_error, 128u);
   return false;
 }
 __device__ __forceinline__ void cp_async_wait_all() {
@@ -566,13 +572,8 @@ cudaError_t launch_t(const DecodeParams& p, int grid, cudaStream_t st) {
   constexpr int D = 4;
   auto kern = decode_kernel<FMT, NT, RT, KW, D>;
   const size_t smem = (size_t)p.bar_off + 16;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         227 * 1024);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = ensure_max_dynamic_smem((const void*)kern, 227 * 1024);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(KW * 32);
@@ -609,6 +610,13 @@ cudaError_t launch_fmt(const DecodeParams& p, int nt, int rt, int kw, int grid,
 }
 
 }  // namespace
+
+cudaError_t read_decode_error(unsigned* value, bool clear) {
+  cudaError_t e = cudaMemcpyFromSymbol(value, g_wq_decode_error, sizeof(unsigned));
+  if (e != cudaSuccess || !clear) return e;
+  unsigned z = 0;
+  return cudaMemcpyToSymbol(g_wq_decode_error, &z, sizeof(unsigned));
+}
 
 cudaError_t launch_decode(const LinearArgs& a) {
   DecodeParams p;

@@ -170,6 +170,19 @@ cudaError_t static_swiglu_scratch(void** ptr, size_t* bytes);
 constexpr size_t kSwigluStaticScratchBytes = 16u << 20;
 cudaError_t launch_prefill(const LinearArgs& a);
 int device_sm_count();
+// A 4-byte memset of a library word on `st`: a stream operation that is not a
+// kernel, appended to every call that writes packed weights (wq_pack,
+// wq_quantize, wq_addmm_requant).  The decode kernel is launched with
+// programmatic dependent launch and reads the packed weights before it waits
+// for the previous kernel; with this operation in between, the previous
+// kernel of a following wq_linear is never the one that wrote its weights.
+cudaError_t end_weight_write(cudaStream_t st);
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (device, kernel),
+// thread-safe; a failure is returned and retried on the next call.
+cudaError_t ensure_max_dynamic_smem(const void* fn, int bytes);
+// The decode kernel's own error word (bit 128: its activation-slice wait ran
+// out); synchronous read, optional clear.
+cudaError_t read_decode_error(unsigned* value, bool clear);
 // The kernels' own error word (bit per failed bounded wait); synchronous read.
 cudaError_t read_device_error(unsigned* value, bool clear);
 

@@ -751,12 +751,7 @@ cudaError_t launch_bn(const LinearArgs& a) {
   if (ST > 8) ST = 8;
   if (ST < 2) ST = 2;
   const size_t smem = (size_t)ST * (tstage + side) + fixed;
-  static std::once_flag attr_once;
-  cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [&] {
-    attr_err = cudaFuncSetAttribute(prefill_kernel<FMT, BN>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-  });
+  cudaError_t attr_err = ensure_max_dynamic_smem((const void*)prefill_kernel<FMT, BN>, 227 * 1024);
   if (attr_err != cudaSuccess) return attr_err;
   PrefillParams p;
   p.scales = a.scales;

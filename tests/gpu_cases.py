@@ -55,12 +55,39 @@ def check_close(y_bits: np.ndarray, ref_bits: np.ndarray, what: str = ""):
     return float((err / lim).max()) if err.size else 0.0
 
 
+GUARD_BEFORE = 128    # bf16 elements (256 bytes: the output stays 16-byte aligned)
+GUARD_AFTER = 4096    # bf16 elements
+GUARD_BITS = 0x7FA5   # a NaN pattern no kernel writes
+
+
+def guarded_out(M: int, N: int) -> tuple[torch.Tensor, torch.Tensor]:
+    """(buffer, out): ``out`` is an [M, N] bf16 view inside ``buffer`` with
+    canary bands before and after it; the output itself starts as NaN, so an
+    element the kernel never writes is caught as non-finite."""
+    buf = torch.full((GUARD_BEFORE + max(M, 1) * N + GUARD_AFTER,), GUARD_BITS, dtype=torch.int16,
+                     device="cuda")
+    out = buf[GUARD_BEFORE:GUARD_BEFORE + max(M, 1) * N].view(torch.bfloat16).view(max(M, 1), N)
+    out.fill_(float("nan"))
+    return buf, out
+
+
+def check_guards(buf: torch.Tensor, M: int, N: int, what: str = ""):
+    """Both canary bands around a guarded output are untouched."""
+    b = buf.cpu().numpy().view(np.uint16)
+    head, tail = b[:GUARD_BEFORE], b[GUARD_BEFORE + max(M, 1) * N:]
+    assert np.all(head == GUARD_BITS), f"{what}: write before the output ({np.sum(head != GUARD_BITS)})"
+    assert np.all(tail == GUARD_BITS), f"{what}: write past the output ({np.sum(tail != GUARD_BITS)})"
+
+
 def run_linear(wq, pw, x_bits, bias_bits, M, stream=None):
+    """One wq_linear call through the C ABI into a guarded output buffer; the
+    canaries around the output are checked before the result is returned."""
     x = dev_bf16(x_bits)
     b = dev_bf16(bias_bits) if bias_bits is not None else None
-    y = torch.full((max(M, 1), pw.N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    buf, y = guarded_out(M, pw.N)
     wq.wq_linear(x, pw.w, pw.scales, pw.aux, b, M, pw.N, pw.K, pw.fmt, pw.group_size, y, stream)
     torch.cuda.synchronize()
+    check_guards(buf, M, pw.N, f"{pw.fmt} M={M} N={pw.N} K={pw.K}")
     return bf16_bits(y[:M])
 
 

@@ -63,3 +63,15 @@ def test_cpu_baseline_reports_all_threads_and_one():
     assert cb["value"] > 0 and cb["single_thread"]["value"] > 0 and per_pass > 0
     assert cb["kind"] == "oracle" and cb["cores"] == oracle.Oracle().threads()
     assert cb["quantize_s"] > 0
+
+
+def test_cpu_baseline_prefill_unit():
+    """A TFLOP/s workload reports its CPU baseline in TFLOP/s (tiny sample)."""
+    import dataclasses
+
+    import bench
+    import synth.workloads as W
+    small = dataclasses.replace(W.PREFILL, N=64, K=512, Ms=(1024,))
+    cb, _ = bench.cpu_baseline(small, small.Ms, 0.2)
+    assert cb["unit"] == "TFLOP/s" and cb["value"] > 0
+    assert cb["single_thread"]["unit"] == "TFLOP/s"

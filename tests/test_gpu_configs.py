@@ -1,9 +1,10 @@
 """GPU parity at the seven workloads' full sizes, in the launch configuration
-the benchmark times (the same wq_linear call).  Small batches are compared
-element by element against the full oracle product; large ones on sampled
-outputs that the oracle computes one by one.  The GPU quantizer (which the
-benchmark uses to make its inputs) is checked bit for bit against the
-oracle's quantizer at full size."""
+the benchmark times (the same wq_linear call).  Every batch size of every
+workload is compared element by element against the oracle's full product
+(its fp64 library-matmul form, seconds even for the 4096 x 8192 x 8192
+prefill case), and canary bands around each output are checked untouched.
+The GPU quantizer (which the benchmark uses to make its inputs) is checked
+bit for bit against the oracle's quantizer at full size."""
 from __future__ import annotations
 
 import numpy as np
@@ -46,40 +47,14 @@ def _workload(orc, wq, wl):
     return _cache[wl.name]
 
 
-def _samples(M, N, count, seed):
-    rng = np.random.default_rng(seed)
-    ms = rng.integers(0, M, count)
-    ns = rng.integers(0, N, count)
-    # edges: first / last token and feature
-    ms = np.concatenate([ms, [0, 0, M - 1, M - 1]])
-    ns = np.concatenate([ns, [0, N - 1, 0, N - 1]])
-    return ms, ns
-
-
 @pytest.mark.parametrize("wl", W.ALL, ids=[w.name for w in W.ALL])
 def test_workload_parity(wq, orc, wl):
     codes, scales, aux, pw, xa, b, same = _workload(orc, wq, wl)
     assert same, "GPU quantizer differs from the oracle's at full size"
     G = wl.group_size
-    full_limit = 2_000_000_000  # multiply-adds the oracle does in full
-    dq = None
+    dq = orc.dequant(wl.fmt, codes, scales, aux, wl.N, wl.K, G)
     for M in wl.Ms:
         y = run_linear(wq, pw, xa[:M], b, M)
         assert y.shape == (M, wl.N)
-        assert np.all(np.isfinite(y.view(np.int16).astype(np.float32)))
-        if M * wl.N * wl.K <= full_limit:
-            if dq is None:
-                dq = orc.dequant(wl.fmt, codes, scales, aux, wl.N, wl.K, G)
-            ref, _ = orc.linear(xa[:M], dq, b)
-            check_close(y, ref, f"{wl.name} M={M}")
-        else:
-            ms, ns = _samples(M, wl.N, 1500, seed=M)
-            ref, _ = orc.linear_sampled(wl.fmt, codes, scales, aux, wl.N, wl.K, G, xa[:M], b,
-                                        ms, ns)
-            check_close(y[ms, ns], ref, f"{wl.name} M={M} (sampled)")
-            # a whole output row and a whole output column as well
-            rows = np.zeros(wl.N, np.int64) + (M // 2)
-            cols = np.arange(wl.N)
-            rref, _ = orc.linear_sampled(wl.fmt, codes, scales, aux, wl.N, wl.K, G, xa[:M], b,
-                                         rows, cols)
-            check_close(y[M // 2], rref, f"{wl.name} M={M} row {M // 2}")
+        ref, _ = orc.linear_full(xa[:M], dq, b)
+        check_close(y, ref, f"{wl.name} M={M}")

@@ -60,3 +60,48 @@ def test_static_scratch_matches_workspace_and_allocates_nothing(orc):
         # no device memory taken by the calls (torch's own count may only fall)
         assert free1 == free0 and torch.cuda.memory_allocated() <= alloc0
         assert np.array_equal(bf16_bits(y_st), bf16_bits(y_ws)), f"M={M}"
+
+
+@pytest.mark.gpu
+def test_static_scratch_on_the_decode_fallback(orc):
+    """A batch of at most 16 rows whose K is too long for the decode kernel's
+    staged slice (here 16 x 65536 with both SwiGLU halves) takes the
+    materialized path, so the static scratch is used there too: identical to
+    the caller-workspace call on two calls in a row, within the parity
+    tolerance of the oracle, and no device memory allocated."""
+    import torch
+
+    import synth
+    from gpu_cases import bf16_bits, check_close, dev_bf16, pack_on_gpu, small_case
+
+    fmt, G, N, K, M = "int4_sym", 128, 128, 65536, 16
+    W, (codes, scales, aux) = small_case(orc, fmt, N, K, G, seed=16)
+    pw = pack_on_gpu(wqm, fmt, N, K, G, codes, scales, aux)
+    x2h = synth.activations(55, M, 2 * K)
+    x2 = dev_bf16(x2h)
+    # the decode kernel refuses this shape: without a workspace the call is unsupported
+    y_none = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    st = wqm._lib.wq_linear_swiglu(x2.data_ptr(), pw.w.data_ptr(), pw.scales.data_ptr(), None,
+                                   None, M, N, K, wqm.FORMATS[fmt], G, None, 0,
+                                   y_none.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    assert st == wqm.WQ_ERR_UNSUPPORTED
+    y_ws = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    wqm.wq_linear_swiglu(x2, pw.w, pw.scales, pw.aux, None, M, N, K, fmt, G, ws, ws.numel() * 2,
+                         y_ws)
+    y_st = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    wqm.wq_linear_swiglu_static(x2, pw.w, pw.scales, pw.aux, None, M, N, K, fmt, G, y_st)
+    torch.cuda.synchronize()
+    gc.collect()
+    free0, _ = torch.cuda.mem_get_info()
+    alloc0 = torch.cuda.memory_allocated()
+    for _ in range(2):
+        y_st.fill_(float("nan"))
+        wqm.wq_linear_swiglu_static(x2, pw.w, pw.scales, pw.aux, None, M, N, K, fmt, G, y_st)
+        torch.cuda.synchronize()
+        assert np.array_equal(bf16_bits(y_st), bf16_bits(y_ws))
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0 and torch.cuda.memory_allocated() <= alloc0
+    dq = orc.dequant(fmt, codes, scales, aux, N, K, G)
+    ref, _ = orc.linear(orc.swiglu(x2h), dq, None)
+    check_close(bf16_bits(y_st), ref, "static scratch, decode fallback")
