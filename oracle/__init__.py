@@ -266,6 +266,31 @@ class Oracle:
                                    _p(xq), _p(sx), _p(b), M, _p(y), _p(y64)), "linear_a8")
         return y, y64
 
+    def linear_a8_full(self, codes, scales, N: int, K: int, G: int, x_bits, bias_bits=None):
+        """(y bf16 bits, y fp64) of the activation-quantized linear for INT8
+        sym weights, with each group's integer sum taken by numpy's fp64
+        matmul (exact: every partial sum is an integer below 2^53) instead
+        of orc_linear_a8's loop, so that full sizes cost seconds.  The codes
+        come from orc_quant_act_int8 and the fp64 accumulation over groups
+        follows orc_linear_a8 step for step ((s_w * s_x) * isum, increasing g,
+        then the bias), so the fp64 result is the same number."""
+        xq, sx = self.quant_act_int8(x_bits)
+        M = xq.shape[0]
+        wq = np.ascontiguousarray(codes, dtype=np.int8).reshape(N, K)
+        sw = bits_to_f32(np.ascontiguousarray(scales, dtype=np.uint16).reshape(N, K // G))
+        sw = sw.astype(np.float64)
+        sxd = sx.astype(np.float64)
+        y64 = np.zeros((M, N), dtype=np.float64)
+        for g in range(K // G):
+            isum = xq[:, g * G:(g + 1) * G].astype(np.float64) @ \
+                wq[:, g * G:(g + 1) * G].astype(np.float64).T
+            y64 += (sw[None, :, g] * sxd[:, None]) * isum
+        if bias_bits is not None:
+            y64 = y64 + bits_to_f32(np.asarray(bias_bits, dtype=np.uint16)).astype(np.float64)[None, :]
+        y = np.zeros((M, N), dtype=np.uint16)
+        _ok(self.lib.orc_round_bf16_array(_p(y64), M * N, _p(y)), "round_bf16_array")
+        return y, y64
+
     def silu(self, g: float) -> float:
         return float(self.lib.orc_silu(g))
 

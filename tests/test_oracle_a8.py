@@ -50,3 +50,35 @@ def test_grid_activations_reduce_to_weight_only_linear(orc, fmt):
     dq = orc.dequant(fmt, codes, scales, None, N, K, K)
     y, y64 = orc.linear(x, dq, b)
     assert np.array_equal(y8_64, y64) and np.array_equal(y8, y)
+
+
+@pytest.mark.parametrize("G", [32, 128, 256])
+def test_a8_full_equals_loop(orc, G):
+    """The matmul form of the activation-quantized linear gives the same fp64
+    numbers as the oracle's loop (exact integer group sums, the same scaling
+    and accumulation order), hence the same bf16 outputs; with and without
+    bias, on outlier channels."""
+    N, K, M = 48, 512, 7
+    W = synth.weight(9, N, K, sigma=0.02, outlier_count=20, outlier_mult=20.0)
+    codes, scales, _ = orc.quantize("int8_sym", W, G)
+    x = synth.activations(10, M, K, channel_count=5, channel_mult=10.0)
+    b = synth.bias(9, N)
+    for bias in (b, None):
+        y, y64 = orc.linear_a8("int8_sym", codes, scales, N, K, G, x, bias)
+        yf, yf64 = orc.linear_a8_full(codes, scales, N, K, G, x, bias)
+        assert np.array_equal(yf64, y64) and np.array_equal(yf, y)
+
+
+def test_a8_full_integer_case(orc):
+    """Unit scales and activations on the INT8 grid with s_x = 1 (row max 127):
+    y is the integer matmul of the codes."""
+    N, K, M, G = 24, 256, 5, 64
+    rng = np.random.default_rng(11)
+    q = rng.integers(-127, 128, size=(N, K)).astype(np.int8)
+    scales = np.full((N, K // G), 0x3F80, np.uint16)
+    xi = rng.integers(-127, 128, size=(M, K))
+    xi[:, 3] = 127
+    x = synth.f64_to_bf16_bits(xi.astype(np.float64))
+    y, y64 = orc.linear_a8_full(q, scales, N, K, G, x, None)
+    ref = (xi @ q.astype(np.int64).T).astype(np.float64)
+    assert np.array_equal(y64, ref)
