@@ -639,6 +639,7 @@ int orc_round_bf16_array(const double* v, int64_t n, uint16_t* y) {
 /* Per-token INT8 activation quantization: xq int8 [M, K], sx f32 [M]. */
 int orc_quant_act_int8(const uint16_t* x, int64_t M, int64_t K, int8_t* xq, float* sx) {
   if (M < 0 || K <= 0) return 1;
+#pragma omp parallel for schedule(static)
   for (int64_t m = 0; m < M; ++m) {
     double amax = 0.0;
     for (int64_t k = 0; k < K; ++k) amax = fmax(amax, fabs((double)orc_bf16_to_f32(x[m * K + k])));
@@ -663,6 +664,7 @@ int orc_linear_a8(int fmt, const void* codes, const uint16_t* scales, int64_t N,
                   const int8_t* xq, const float* sx, const uint16_t* bias, int64_t M, uint16_t* y,
                   double* y64) {
   if ((fmt != ORC_INT4_SYM && fmt != ORC_INT8_SYM) || check_fmt(fmt, N, K, G) || M < 0) return 1;
+#pragma omp parallel for schedule(dynamic, 4)
   for (int64_t n = 0; n < N; ++n)
     for (int64_t m = 0; m < M; ++m) {
       double acc = 0.0;
