@@ -225,6 +225,7 @@ def context_numbers(wl, Ms, weights, xs, bias, outs, stream, l2, device):
     bias_t = None
     if bias is not None:
         bias_t = bias
+    call = linear_call(wl, Ms, device)
     for M in Ms:
         def graph_of(fn, n):
             g = torch.cuda.CUDAGraph()
@@ -238,8 +239,7 @@ def context_numbers(wl, Ms, weights, xs, bias, outs, stream, l2, device):
         def ours(n, base=[0]):
             for i in range(n):
                 pw = weights[(base[0] + i) % R]
-                wq.wq_linear(xs[M], pw.w, pw.scales, pw.aux, bias, M, wl.N, wl.K, wl.fmt,
-                             wl.group_size, outs[M], stream)
+                call(xs[M], pw, bias, M, outs[M], stream)
             base[0] += n
 
         def ref(n, base=[0]):
@@ -288,6 +288,16 @@ def cpu_sample(wl, Ms, rows, data):
     """One bounded oracle pass: every token of every M against `rows` output rows."""
     orc, codes, scales, aux, xa, b = data
     t0 = time.perf_counter()
+    if wl.act_int8:
+        # the oracle's activation-quantized linear on the first `rows` rows
+        nb = codes.nbytes // wl.N
+        sb = scales.nbytes // wl.N
+        c = np.ascontiguousarray(codes.reshape(-1).view(np.uint8)[: rows * nb])
+        s = np.ascontiguousarray(scales.reshape(-1).view(np.uint8)[: rows * sb]).view(np.uint16)
+        for M in Ms:
+            orc.linear_a8(wl.fmt, c.view(np.int8), s, rows, wl.K, wl.group_size, xa[:M],
+                          None if b is None else b[:rows])
+        return time.perf_counter() - t0
     for M in Ms:
         ms = np.repeat(np.arange(M), rows)
         ns = np.tile(np.arange(rows) * (wl.N // rows), M)
@@ -306,6 +316,8 @@ def cpu_baseline(wl, Ms, seconds, calibrate_only=False):
 
     tflops_metric = min(Ms) >= 1024
     unit, scale = ("TFLOP/s", 1e12) if tflops_metric else ("GB/s", 1e9)
+    if wl.act_int8:
+        unit = "TOPS"
     orc = oracle.Oracle()
     Wd = W.make_weight(wl)
     tq0 = time.perf_counter()
@@ -351,6 +363,27 @@ def cpu_baseline(wl, Ms, seconds, calibrate_only=False):
 
 
 # ------------------------------------------------------------------ timing
+def linear_call(wl, Ms, device):
+    """The library call one batch of `wl` makes: wq_linear, or for the
+    activation-quantized workload wq_linear_a8 with a preallocated
+    workspace per batch size."""
+    import torch
+
+    import mixed_gemm_b200 as wq
+    if not wl.act_int8:
+        def call(x, pw, bias, M, out, stream):
+            wq.wq_linear(x, pw.w, pw.scales, pw.aux, bias, M, wl.N, wl.K, wl.fmt, wl.group_size,
+                         out, stream)
+        return call
+    ws = {M: torch.empty((wq.wq_linear_a8_workspace_size(M, wl.K),), dtype=torch.uint8,
+                         device=device) for M in Ms}
+
+    def call(x, pw, bias, M, out, stream):
+        wq.wq_linear_a8(x, pw.w, pw.scales, bias, M, wl.N, wl.K, wl.fmt, wl.group_size, ws[M],
+                        ws[M].numel(), out, stream)
+    return call
+
+
 def time_workload(wl, Ms, steps, warmup, device, l2, world, local_rank, do_e2e):
     """Device time of exactly `steps` steps of `wl` (one wq_linear per M, each
     on the next resident weight copy), replayed from CUDA graphs, CUDA events
@@ -363,7 +396,7 @@ def time_workload(wl, Ms, steps, warmup, device, l2, world, local_rank, do_e2e):
     import synth.workloads as W
 
     tflops_metric = min(Ms) >= 1024
-    unit = "TFLOP/s" if tflops_metric else "GB/s"
+    unit = ("TOPS" if wl.act_int8 else "TFLOP/s") if tflops_metric else "GB/s"
     weights, xs, bias, outs, xa = build_workload(wl, Ms, device, 3 * l2)
     R = len(weights)
     launches_per_step = len(Ms)
@@ -371,13 +404,15 @@ def time_workload(wl, Ms, steps, warmup, device, l2, world, local_rank, do_e2e):
     step_flops = sum(W.flops(M, wl.N, wl.K) for M in Ms)
     stream = torch.cuda.Stream(device)
     counter = [0]
+    call = linear_call(wl, Ms, device)
+    if wl.act_int8:
+        launches_per_step *= 2        # the activation quantizer, then the linear
 
     def step():
         for M in Ms:
             pw = weights[counter[0] % R]
             counter[0] += 1
-            wq.wq_linear(xs[M], pw.w, pw.scales, pw.aux, bias, M, wl.N, wl.K, wl.fmt,
-                         wl.group_size, outs[M], stream)
+            call(xs[M], pw, bias, M, outs[M], stream)
 
     def barrier():
         if world > 1:
@@ -442,9 +477,21 @@ def time_workload(wl, Ms, steps, warmup, device, l2, world, local_rank, do_e2e):
         value = whole_job_value(world, steps, step_bytes, sec, 1e9)
     per_launch_s = sec / (steps * launches_per_step)
 
-    # roofline of the dominant kernel (every launch in the step runs it)
+    # roofline of the dominant kernel (every launch in the step runs it; for
+    # the activation-quantized linear a call is the quantizer plus the
+    # tcgen05 kernel, both inside the time per call)
     pk, pk_kind = peaks()
-    if tflops_metric:
+    calls_per_step = len(Ms)
+    per_call_s = sec / (steps * calls_per_step)
+    peak_note = None
+    if tflops_metric and wl.act_int8:
+        achieved = step_flops / calls_per_step / per_call_s / 1e12
+        # dense INT8 tensor peak: the measured bf16 peak x 2 (the nominal
+        # 4.5 / 2.25 PFLOP/s ratio)
+        peak = 2.0 * pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        bound, r_unit = "tensor", "TOPS"
+        peak_note = "int8 dense = 2 x measured bf16 burst (nominal int8 / bf16 ratio)"
+    elif tflops_metric:
         achieved = step_flops / launches_per_step / per_launch_s / 1e12
         peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
         bound, r_unit = "tensor", "TFLOP/s"
@@ -464,6 +511,10 @@ def time_workload(wl, Ms, steps, warmup, device, l2, world, local_rank, do_e2e):
         yh = {M: torch.empty((M, wl.N), dtype=torch.bfloat16).pin_memory() for M in Ms}
         e2e_steps = max(3, min(steps, 2000))
         k = [0]
+        e2e_ws = None
+        if wl.act_int8:
+            e2e_ws = torch.empty((wq.wq_linear_a8_workspace_size(max(Ms), wl.K),),
+                                 dtype=torch.uint8, device=device)
 
         def e2e_step():
             # every batch of the step from pinned host memory, results copied
@@ -471,7 +522,11 @@ def time_workload(wl, Ms, steps, warmup, device, l2, world, local_rank, do_e2e):
             for M in Ms:
                 pw = weights[k[0] % R]
                 k[0] += 1
-                wq.linear(xh[M], pw, bias, out=yh[M], stream=stream, sync=False)
+                if wl.act_int8:
+                    wq.linear_a8(xh[M], pw, bias, out=yh[M], workspace=e2e_ws, stream=stream,
+                                 sync=False)
+                else:
+                    wq.linear(xh[M], pw, bias, out=yh[M], stream=stream, sync=False)
             stream.synchronize()
 
         for _ in range(3):
@@ -504,7 +559,8 @@ def time_workload(wl, Ms, steps, warmup, device, l2, world, local_rank, do_e2e):
                              "the warm-up; CUDA events on the launch stream"},
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": r_unit,
                      "frac": achieved / peak, "traffic": traffic, "peak_source": pk_kind,
-                     "kernel": "decode_kernel" if max(Ms) <= 16 else "prefill_kernel"},
+                     "kernel": "decode_kernel" if max(Ms) <= 16 else "prefill_kernel",
+                     **({"peak_note": peak_note} if peak_note else {})},
         "gpu_launches": steps * launches_per_step,
         "clocks": clk,
         "e2e": e2e,
@@ -523,7 +579,7 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     tflops_metric = min(Ms) >= 1024
-    unit = "TFLOP/s" if tflops_metric else "GB/s"
+    unit = ("TOPS" if wl.act_int8 else "TFLOP/s") if tflops_metric else "GB/s"
 
     if args.impl == "reference":
         if rank != 0:

@@ -235,6 +235,36 @@ int wq_linear_swiglu_static(const void* x2, const void* packed_w, const void* sc
                             const void* aux, const void* bias, int64_t M, int64_t N, int64_t K,
                             int format, int group_size, void* out, void* stream);
 
+/* Activation-quantized linear (W8A8): the activations are quantized per
+ * token to INT8 and multiplied with the INT8 weight codes on the integer
+ * tensor cores; each group's integer sum is scaled once:
+ *     s_x[m] = fp32(max_k |x[m,k]| / 127)  (quotient in fp64)
+ *     x_q[m,k] = clamp(round_half_even(x[m,k] / s_x[m]), -127, 127)
+ *     Y[m,n] = s_x[m] * sum_g s_w[n,g] * (sum_{k in g} x_q[m,k] * q[n,k]) + bias[n]
+ * This is a different computation from wq_linear (the activations are
+ * quantized), with its own reference; the group sums are exact integers and
+ * the scaling is fp32.
+ *   x, packed_w, scales, bias, out   as wq_linear (format WQ_INT8_SYM only)
+ *   workspace   device scratch of at least wq_linear_a8_workspace_size(M, K)
+ *               bytes, 16-byte aligned, overlapping no other buffer: the
+ *               INT8 codes [M, K] at offset 0 and the fp32 scales [M] at the
+ *               next multiple of 256 bytes; contents not preserved
+ * Other formats, or K % 128 != 0, return WQ_ERR_UNSUPPORTED.  M == 0 is a
+ * no-op.  Asynchronous: two kernels (the quantizer, then the tcgen05 kernel
+ * with tcgen05.mma.kind::i8 and s32 accumulators in tensor memory).
+ * Source: auto-round-lib README section 1 ("Key Features": INT8 compute with
+ * dynamic per-token activation quantization, low-bit weights used as INT8;
+ * the W8A8 / W4A8 backends). */
+int wq_linear_a8_workspace_size(int64_t M, int64_t K, size_t* bytes);
+int wq_linear_a8(const void* x, const void* packed_w, const void* scales, const void* bias,
+                 int64_t M, int64_t N, int64_t K, int format, int group_size, void* workspace,
+                 size_t workspace_bytes, void* out, void* stream);
+
+/* The per-token INT8 activation quantizer of wq_linear_a8 on its own (device
+ * buffers): xq int8 [M, K] (16-byte aligned), sx f32 [M]; K % 8 == 0.
+ * Source: as wq_linear_a8. */
+int wq_quantize_act_int8(const void* x, int64_t M, int64_t K, void* xq, void* sx, void* stream);
+
 /* In-place LoRA merge into a packed INT8_SYM weight:
  *     weight = beta * weight + alpha * (mat1 @ mat2)
  * requantized with the weight's unchanged group scales.  With use_seed == 0

@@ -59,6 +59,10 @@ _SIGS = {
     "wq_linear_swiglu_static": ([_ptr, _ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _int, _int, _ptr,
                                  _ptr], _int),
     "wq_quantize": ([_int, _i64, _i64, _int, _ptr, _ptr, _ptr, _ptr, _ptr], _int),
+    "wq_linear_a8_workspace_size": ([_i64, _i64, _sz], _int),
+    "wq_linear_a8": ([_ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _int, _int, _ptr, ctypes.c_size_t,
+                      _ptr, _ptr], _int),
+    "wq_quantize_act_int8": ([_ptr, _i64, _i64, _ptr, _ptr, _ptr], _int),
     "wq_lloyd_max_centroids": ([_int, ctypes.POINTER(ctypes.c_float)], _int),
     "wq_device_sm_count": ([ctypes.POINTER(ctypes.c_int)], _int),
     "wq_device_error": ([ctypes.POINTER(ctypes.c_uint), _int], _int),
@@ -185,6 +189,24 @@ def wq_quantize(fmt, N, K, group_size, w_f32, codes, scales, aux, stream=None):
                             _addr(scales), _addr(aux), _stream(stream)), "wq_quantize")
 
 
+def wq_linear_a8_workspace_size(M: int, K: int) -> int:
+    n = ctypes.c_size_t()
+    _check(_lib.wq_linear_a8_workspace_size(M, K, ctypes.byref(n)), "wq_linear_a8_workspace_size")
+    return n.value
+
+
+def wq_linear_a8(x, packed_w, scales, bias, M, N, K, fmt, group_size, workspace, workspace_bytes,
+                 out, stream=None):
+    _check(_lib.wq_linear_a8(_addr(x), _addr(packed_w), _addr(scales), _addr(bias), M, N, K,
+                             _fmt(fmt), group_size, _addr(workspace), int(workspace_bytes),
+                             _addr(out), _stream(stream)), "wq_linear_a8")
+
+
+def wq_quantize_act_int8(x, M, K, xq, sx, stream=None):
+    _check(_lib.wq_quantize_act_int8(_addr(x), M, K, _addr(xq), _addr(sx), _stream(stream)),
+           "wq_quantize_act_int8")
+
+
 def wq_lloyd_max_centroids(bits: int = 4):
     import numpy as np
     out = np.zeros((1 << bits,), dtype=np.float32)
@@ -208,5 +230,5 @@ def wq_device_sm_count() -> int:
     return n.value
 
 
-from .api import (PackedWeight, linear, linear_grouped, linear_swiglu, pack,  # noqa: E402,F401
-                  quantize_and_pack)
+from .api import (PackedWeight, linear, linear_a8, linear_grouped, linear_swiglu,  # noqa: E402,F401
+                  pack, quantize_and_pack)

@@ -12,8 +12,9 @@ from dataclasses import dataclass
 
 import torch
 
-from . import (FORMATS, wq_canonical_sizes, wq_linear, wq_linear_grouped, wq_linear_swiglu,
-               wq_lloyd_max_centroids, wq_pack, wq_packed_sizes, wq_quantize)
+from . import (FORMATS, wq_canonical_sizes, wq_linear, wq_linear_a8, wq_linear_a8_workspace_size,
+               wq_linear_grouped, wq_linear_swiglu, wq_lloyd_max_centroids, wq_pack,
+               wq_packed_sizes, wq_quantize)
 
 
 @dataclass
@@ -142,6 +143,45 @@ def linear_swiglu(x2: torch.Tensor, weight: PackedWeight, bias: torch.Tensor | N
     ws = torch.empty((M, K), dtype=torch.bfloat16, device=dev) if M > 16 else None
     wq_linear_swiglu(xd, weight.w, weight.scales, weight.aux, bias, M, weight.N, K, weight.fmt,
                      weight.group_size, ws, 0 if ws is None else ws.numel() * 2, y, stream)
+    return y.reshape(*lead, weight.N)
+
+
+def linear_a8(x: torch.Tensor, weight: PackedWeight, bias: torch.Tensor | None = None,
+              out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+              stream=None, sync: bool = True) -> torch.Tensor:
+    """Activation-quantized linear (INT8 weights): x quantized per token to
+    INT8, integer tensor-core products, group scales and the token scale
+    applied in fp32.  ``x``: [..., K] bf16.  The INT8 activations live in
+    ``workspace`` (allocated here when not given).  A host ``x`` is copied in
+    and the result copied back on ``stream``, as in ``linear``."""
+    host = not x.is_cuda
+    dev = weight.w.device
+    lead = x.shape[:-1]
+    K = weight.K
+    assert x.shape[-1] == K and x.dtype == torch.bfloat16
+    s = _torch_stream(stream, dev)
+    with torch.cuda.stream(s):
+        xd = x.reshape(-1, K)
+        if host:
+            xd = xd.to(dev, non_blocking=True)
+        xd = xd.contiguous()
+        M = xd.shape[0]
+        need = wq_linear_a8_workspace_size(M, K)
+        if workspace is None or workspace.numel() * workspace.element_size() < need:
+            workspace = torch.empty((max(need, 16),), dtype=torch.uint8, device=dev)
+        y = out if (out is not None and not host) else torch.empty(
+            (M, weight.N), dtype=torch.bfloat16, device=dev)
+        wq_linear_a8(xd, weight.w, weight.scales, bias, M, weight.N, K, weight.fmt,
+                     weight.group_size, workspace, workspace.numel() * workspace.element_size(),
+                     y, s)
+        if host:
+            yh = out if out is not None else torch.empty((M, weight.N), dtype=torch.bfloat16,
+                                                          pin_memory=True)
+            yh.copy_(y, non_blocking=True)
+    if host:
+        if sync:
+            s.synchronize()
+        return yh.reshape(*lead, weight.N)
     return y.reshape(*lead, weight.N)
 
 

@@ -353,6 +353,61 @@ int wq_linear_swiglu_static(const void* x2, const void* pw, const void* scales, 
   return wq_linear_swiglu(x2, pw, scales, aux, bias, M, N, K, f, G, ws, ws_bytes, out, stream);
 }
 
+int wq_linear_a8_workspace_size(int64_t M, int64_t K, size_t* bytes) {
+  if (!bytes || M < 0 || M > (1LL << 24) || K <= 0 || K > (1LL << 24)) return WQ_ERR_INVALID_ARG;
+  *bytes = (size_t)(((M * K + 255) & ~255LL) + 4 * M);
+  return WQ_OK;
+}
+
+int wq_quantize_act_int8(const void* x, int64_t M, int64_t K, void* xq, void* sx, void* stream) {
+  if (M < 0 || M > (1LL << 24) || K <= 0 || K > (1LL << 24) || K % 8) return WQ_ERR_INVALID_ARG;
+  if (M == 0) return WQ_OK;
+  if (!x || !xq || !sx) return WQ_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(xq, 16) || !aligned(sx, 4)) return WQ_ERR_ALIGNMENT;
+  if (overlap(xq, M * K, x, M * K * 2) || overlap(sx, M * 4, x, M * K * 2) ||
+      overlap(sx, M * 4, xq, M * K))
+    return WQ_ERR_INVALID_ARG;
+  return cuda_status(launch_quant_act_int8(x, M, K, xq, (float*)sx, (cudaStream_t)stream));
+}
+
+int wq_linear_a8(const void* x, const void* pw, const void* scales, const void* bias, int64_t M,
+                 int64_t N, int64_t K, int f, int G, void* workspace, size_t workspace_bytes,
+                 void* out, void* stream) {
+  int st = check_linear(x, K, pw, scales, nullptr, bias, M, N, K, f, G, out);
+  if (st) return st;
+  if (f != INT8_SYM || K % 128) return WQ_ERR_UNSUPPORTED;
+  size_t need = 0;
+  if ((st = wq_linear_a8_workspace_size(M, K, &need)) != WQ_OK) return st;
+  if (M == 0) return WQ_OK;
+  if (!workspace || workspace_bytes < need) return WQ_ERR_INVALID_ARG;
+  if (!aligned(workspace, 16)) return WQ_ERR_ALIGNMENT;
+  size_t wb = 0, sb = 0, ab = 0;
+  wq_packed_sizes(f, N, K, G, &wb, &sb, &ab);
+  const int64_t w = (int64_t)need;
+  if (overlap(workspace, w, x, M * K * 2) || overlap(workspace, w, out, M * N * 2) ||
+      overlap(workspace, w, pw, wb) || overlap(workspace, w, scales, sb) ||
+      overlap(workspace, w, bias, N * 2))
+    return WQ_ERR_INVALID_ARG;
+  uint8_t* xq = (uint8_t*)workspace;
+  float* sx = (float*)(xq + ((M * K + 255) & ~255LL));
+  cudaError_t e = launch_quant_act_int8(x, M, K, xq, sx, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  LinearArgs a;
+  a.x = xq;
+  a.w = pw;
+  a.scales = scales;
+  a.aux = sx;
+  a.bias = bias;
+  a.out = out;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.fmt = f;
+  a.G = G;
+  a.stream = (cudaStream_t)stream;
+  return cuda_status(launch_prefill_a8(a));
+}
+
 int wq_addmm_requant(int f, int64_t N, int64_t K, int G, void* pw, const void* ps,
                      const void* mat1, const void* mat2, int64_t rank, double alpha, double beta,
                      int use_seed, uint64_t seed, void* stream) {

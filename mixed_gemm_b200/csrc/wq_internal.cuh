@@ -169,6 +169,14 @@ cudaError_t launch_swiglu(const void* x2, int64_t M, int64_t K, void* a, cudaStr
 cudaError_t static_swiglu_scratch(void** ptr, size_t* bytes);
 constexpr size_t kSwigluStaticScratchBytes = 16u << 20;
 cudaError_t launch_prefill(const LinearArgs& a);
+// The same tcgen05 kernel on INT8 operands (kind::i8, s32 group sums): a.x is
+// the INT8 activation codes [M, K], a.aux the per-token fp32 scales [M];
+// INT8_SYM weights, K % 128 == 0 (else cudaErrorNotSupported, nothing launched)
+cudaError_t launch_prefill_a8(const LinearArgs& a);
+// Per-token INT8 quantization of bf16 x [M, K] (K % 8 == 0): codes xq [M, K],
+// scales sx [M]
+cudaError_t launch_quant_act_int8(const void* x, int64_t M, int64_t K, void* xq, float* sx,
+                                  cudaStream_t st);
 int device_sm_count();
 // A 4-byte memset of a library word on `st`: a stream operation that is not a
 // kernel, appended to every call that writes packed weights (wq_pack,

@@ -166,6 +166,22 @@ __device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t a, uint64_t b
       "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+__device__ __forceinline__ void umma_i8(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// an accumulator word read from tensor memory: fp32, or (i8 MMAs) s32,
+// exact in fp32 for the group sums (|sum| <= 256 * 127 * 127 < 2^24)
+template <bool kS32>
+__device__ __forceinline__ float tmem_val(uint32_t v) {
+  if constexpr (kS32) return (float)(int)v;
+  return __uint_as_float(v);
+}
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    bar)
@@ -233,13 +249,16 @@ __device__ __forceinline__ uint32_t lds_u8(uint32_t addr) {
   return v;
 }
 
+__device__ __forceinline__ void st_shared_v2(uint32_t addr, uint32_t a, uint32_t b) {
+  asm volatile("st.shared.v2.b32 [%0], {%1,%2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
+}
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
                : "memory");
 }
 
-template <int FMT, int BN>
+template <int FMT, int BN, bool A8>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                    const PrefillParams p) {
@@ -248,8 +267,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         FMT == INT2_SYM || FMT == FP8_E4M3 || FMT == FP8_E5M2;
   constexpr bool kFp8 = FMT == FP8_E4M3 || FMT == FP8_E5M2;
   constexpr bool kByte = FMT == INT8_SYM || kFp8;  // one byte per code
-  // packed bytes per stage (8 row tiles x 64 K)
-  constexpr uint32_t kWpk = kByte ? 8192u : FMT == INT2_SYM ? 2048u : 4096u;
+  // A8: INT8 activations x INT8 weight codes (kind::i8, s32 accumulators);
+  // a stage covers 128 K (128 bytes of each operand row), else 64 K of bf16
+  constexpr int KS = A8 ? 128 : 64;
+  static_assert(!A8 || FMT == INT8_SYM, "the i8 path takes INT8 weight codes");
+  // packed bytes per stage (8 row tiles x KS)
+  constexpr uint32_t kWpk = (kByte ? 8192u : FMT == INT2_SYM ? 2048u : 4096u) * (A8 ? 2u : 1u);
+  // elements of the packed tensor map's inner dimension per row tile and stage
+  constexpr int kWbox = (int)(kWpk / 8u / (kWpk / 8u > 1024u ? 8u : 4u));
   // A stage: one 128 x 64 bf16 tile; CB4 adds a second tile holding the
   // bf16 remainders of its centroids (two MMAs per K step)
   constexpr uint32_t kAsub = FMT == CB4 ? 2u : 1u;
@@ -290,12 +315,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   // partial tiles are summed through distributed shared memory at the end
   const int S = p.splits;
   const int split = S > 1 ? (int)blockIdx.z : 0;
-  const int KT = p.K / 64 / S;
+  const int KT = p.K / KS / S;
   const int kt0 = split * KT;  // first K step of this CTA
   const int ntiles = p.N / 16;
   // group-scale fold: exact integer tiles, one accumulator per group of K;
-  // groups are counted in 16-wide MMA steps (two groups per stage for G = 32)
-  const int KPG = kInt ? p.G / 16 : 4 * KT;  // MMA steps per accumulation group
+  // groups are counted in MMA steps of KS / 4 (16 for bf16, 32 for i8)
+  const int KPG = kInt ? p.G / (KS / 4) : 4 * KT;  // MMA steps per accumulation group
   const int NG = 4 * KT / KPG;
 
   if (threadIdx.x == 0) {
@@ -340,9 +365,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
           uint8_t* st = smem + s * kTstage;
           mbar_expect_tx(tfull_bar(s), kXbytes + kWpk);
-          tma_load_2d(smem_u32(st), &tmX, (kt0 + kt) * 64, m0, tfull_bar(s));
-          tma_load_2d(smem_u32(st + kXbytes), &tmW, (kt0 + kt) * (int)(kWpk / 32u), tile0,
-                      tfull_bar(s));
+          tma_load_2d(smem_u32(st), &tmX, (kt0 + kt) * KS, m0, tfull_bar(s));
+          tma_load_2d(smem_u32(st + kXbytes), &tmW, (kt0 + kt) * kWbox, tile0, tfull_bar(s));
         }
         if constexpr (kHasSide) {
           const uint32_t sd = smem_u32(sring + s * kSide);
@@ -375,8 +399,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(tfull_bar(kt % ST), (uint32_t)(kt / ST) & 1u, abort, 2u);
     } else if (warp == 1 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
-      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                             ((128u >> 4) << 24);
+      // instruction descriptor: D f32 (A8: s32), A and B bf16 (A8: signed
+      // 8-bit), both K-major, N = BN, M = 128
+      const uint32_t idesc = ((A8 ? 2u : 1u) << 4) | (1u << 7) | (1u << 10) |
+                             ((uint32_t)(BN >> 3) << 17) | ((128u >> 4) << 24);
       // descriptors of slot 0 of each ring; a slot / K step is a plain add to
       // the start-address field (smem addresses stay below 2^18)
       const uint64_t xdesc0 = umma_desc_sw128(smem_u32(smem));
@@ -404,7 +430,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
           }
-          umma_f16(d, ad + 2 * kk, xd + 2 * kk, idesc, in_g != 0);  // +32 bytes per K step
+          if constexpr (A8)  // +32 bytes (32 K) per step
+            umma_i8(d, ad + 2 * kk, xd + 2 * kk, idesc, in_g != 0);
+          else  // +32 bytes (16 K) per step
+            umma_f16(d, ad + 2 * kk, xd + 2 * kk, idesc, in_g != 0);
           if constexpr (FMT == CB4)  // the centroids' remainders, same X columns
             umma_f16(d, ad + (16384u >> 4) + 2 * kk, xd + 2 * kk, idesc, 1u);
           if (++in_g == KPG) {
@@ -469,7 +498,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int rr = 0; rr < 2; ++rr) {
         const int rt = 2 * dw + rr;
         const int Rg = rt * 16 + g, Rg8 = Rg + 8;
-        if constexpr (kByte) {
+        if constexpr (A8) {
+          // INT8 codes into the i8 operand tile: four 512-byte blocks of 32 K
+          // per row tile; a lane's 16 bytes hold rows g and g + 8 at K
+          // 32 blk + 8 tq + (0..3 | 4..7); offset-binary -> two's complement
+#pragma unroll
+          for (int blk = 0; blk < 4; ++blk) {
+            const uint4 ch = *(const uint4*)(wpk + rt * 2048 + blk * 512 + lane * 16);
+            const int j = 2 * blk + (tq >> 1);
+            const uint32_t half = (uint32_t)(tq & 1) * 8u;
+            st_shared_v2(abase + swz(Rg, j) + half, ch.x ^ 0x80808080u, ch.z ^ 0x80808080u);
+            st_shared_v2(abase + swz(Rg8, j) + half, ch.y ^ 0x80808080u, ch.w ^ 0x80808080u);
+          }
+        } else if constexpr (kByte) {
 #pragma unroll
           for (int blk = 0; blk < 2; ++blk) {
             const uint4 ch = *(const uint4*)(wpk + rt * 1024 + blk * 512 + lane * 16);
@@ -585,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int r16 = (int)(n & 15);
       sidx = (n >> 4) * groups * 16 + 2 * (r16 & 7) + (r16 >> 3);
     }
-    const int gfirst = kInt ? (kt0 * 64) / p.G : 0;  // first group of this CTA's K range
+    const int gfirst = kInt ? (kt0 * KS) / p.G : 0;  // first group of this CTA's K range
     auto group_scale = [&](int gi) -> uint32_t {
       if (!(kInt && nvalid && gi < NG)) return 0u;
       if constexpr (kFp8) return __ldg(srow32 + sidx + (int64_t)(gfirst + gi) * 16);
@@ -620,25 +661,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t v[32];
           tmem_ld32(base + (uint32_t)c, v);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) acc[c + j] = fmaf(sc, __uint_as_float(v[j]), acc[c + j]);
+          for (int j = 0; j < 32; ++j) acc[c + j] = fmaf(sc, tmem_val<A8>(v[j]), acc[c + j]);
         }
       } else {
         uint32_t v[16];
         tmem_ld16(base, v);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) acc[j] = fmaf(sc, __uint_as_float(v[j]), acc[j]);
+        for (int j = 0; j < 16; ++j) acc[j] = fmaf(sc, tmem_val<A8>(v[j]), acc[j]);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(gempty_bar(gb));
     }
+    // A8: the per-token activation scale multiplies each output column
+    auto colscale = [&](int m) -> float {
+      if constexpr (A8) return __ldg((const float*)p.aux + m);
+      return 1.f;
+    };
     if (S == 1) {
       if (ok && nvalid) {
 #pragma unroll
         for (int j = 0; j < kHalf; ++j) {
           const int m = m0 + hcol + j;
           if (m < p.M)
-            p.out[(int64_t)m * p.N + n] = (uint16_t)f32_to_bf16_bits(acc[j] * post + bval);
+            p.out[(int64_t)m * p.N + n] =
+                (uint16_t)f32_to_bf16_bits(acc[j] * post * colscale(m) + bval);
         }
       }
     } else {
@@ -669,7 +716,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int src = 0; src < S; ++src) tot += sl[(src * 128 + frow) * CW + c];
           const int m = m0 + split * CW + c;
           if (m < p.M)
-            p.out[(int64_t)m * p.N + n] = (uint16_t)f32_to_bf16_bits(tot * post + bval);
+            p.out[(int64_t)m * p.N + n] =
+                (uint16_t)f32_to_bf16_bits(tot * post * colscale(m) + bval);
         }
       }
     }
@@ -705,33 +753,42 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-template <int FMT, int BN>
+template <int FMT, int BN, bool A8>
 cudaError_t launch_bn(const LinearArgs& a) {
-  constexpr uint32_t kWpk = (FMT == INT8_SYM || FMT == FP8_E4M3 || FMT == FP8_E5M2) ? 8192u
-                            : FMT == INT2_SYM                                     ? 2048u
-                                                                                  : 4096u;
+  constexpr int KS = A8 ? 128 : 64;  // K per stage
+  constexpr uint32_t kWpk = ((FMT == INT8_SYM || FMT == FP8_E4M3 || FMT == FP8_E5M2) ? 8192u
+                             : FMT == INT2_SYM                                      ? 2048u
+                                                                                    : 4096u) *
+                            (A8 ? 2u : 1u);
+  // the packed tile of a row tile per stage as one box row of 4- or 8-byte
+  // elements (at most 256 per box dimension)
+  constexpr uint32_t kEsz = kWpk / 8u > 1024u ? 8u : 4u;
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
   CUtensorMap tmX, tmW;
   {
+    // X: bf16 [M, K], or (A8) the INT8 activation codes [M, K]; rows of
+    // 128 bytes per stage in the 128-byte swizzle
     cuuint64_t dims[2] = {(cuuint64_t)a.K, (cuuint64_t)a.M};
-    cuuint64_t strides[1] = {(cuuint64_t)a.K * 2};
-    cuuint32_t box[2] = {64u, (cuuint32_t)BN};
+    cuuint64_t strides[1] = {(cuuint64_t)a.K * (A8 ? 1 : 2)};
+    cuuint32_t box[2] = {(cuuint32_t)KS, (cuuint32_t)BN};
     cuuint32_t es[2] = {1u, 1u};
-    if (fn(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.x), dims, strides, box,
-           es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    if (fn(&tmX, A8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+           const_cast<void*>(a.x), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
   {
     const uint64_t row_bytes = (uint64_t)a.K * 2 * code_bits(FMT);  // bytes per row tile
-    cuuint64_t dims[2] = {(cuuint64_t)(row_bytes / 4), (cuuint64_t)(a.N / 16)};
+    cuuint64_t dims[2] = {(cuuint64_t)(row_bytes / kEsz), (cuuint64_t)(a.N / 16)};
     cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
-    cuuint32_t box[2] = {kWpk / 32u, 8u};
+    cuuint32_t box[2] = {kWpk / 8u / kEsz, 8u};
     cuuint32_t es[2] = {1u, 1u};
-    if (fn(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(a.w), dims, strides, box, es,
-           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    if (fn(&tmW, kEsz == 8u ? CU_TENSOR_MAP_DATA_TYPE_UINT64 : CU_TENSOR_MAP_DATA_TYPE_UINT32, 2,
+           const_cast<void*>(a.w), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
   // ring depths: three dequantized A tiles; as many TMA stages as fit
@@ -751,7 +808,8 @@ cudaError_t launch_bn(const LinearArgs& a) {
   if (ST > 8) ST = 8;
   if (ST < 2) ST = 2;
   const size_t smem = (size_t)ST * (tstage + side) + fixed;
-  cudaError_t attr_err = ensure_max_dynamic_smem((const void*)prefill_kernel<FMT, BN>, 227 * 1024);
+  cudaError_t attr_err =
+      ensure_max_dynamic_smem((const void*)prefill_kernel<FMT, BN, A8>, 227 * 1024);
   if (attr_err != cudaSuccess) return attr_err;
   PrefillParams p;
   p.scales = a.scales;
@@ -774,8 +832,8 @@ cudaError_t launch_bn(const LinearArgs& a) {
   // into whole scale groups and leaves each CTA a multiple of 4 columns.
   {
     const int64_t tiles = (int64_t)((a.N + 127) / 128) * ((a.M + BN - 1) / BN);
-    const int64_t KTall = a.K / 64;
-    const int64_t unit = (is_grouped_fmt(FMT) && a.G > 64) ? a.G / 64 : 1;
+    const int64_t KTall = a.K / KS;
+    const int64_t unit = (is_grouped_fmt(FMT) && a.G > KS) ? a.G / KS : 1;
     const int64_t sms = device_sm_count();
     int best_s = 1;
     if (2 * tiles <= sms) {
@@ -811,10 +869,10 @@ cudaError_t launch_bn(const LinearArgs& a) {
     attr[0].val.clusterDim.z = (unsigned)p.splits;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_kernel<FMT, BN>, tmX, tmW, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_kernel<FMT, BN, A8>, tmX, tmW, p);
     if (e != cudaSuccess) return e;
   } else {
-    prefill_kernel<FMT, BN><<<grid, kThreads, smem, a.stream>>>(tmX, tmW, p);
+    prefill_kernel<FMT, BN, A8><<<grid, kThreads, smem, a.stream>>>(tmX, tmW, p);
   }
   return cudaGetLastError();
 }
@@ -822,10 +880,10 @@ cudaError_t launch_bn(const LinearArgs& a) {
 template <int FMT>
 cudaError_t launch_fmt(const LinearArgs& a, int BN) {
   switch (BN) {
-    case 32: return launch_bn<FMT, 32>(a);
-    case 64: return launch_bn<FMT, 64>(a);
-    case 128: return launch_bn<FMT, 128>(a);
-    default: return launch_bn<FMT, 256>(a);
+    case 32: return launch_bn<FMT, 32, false>(a);
+    case 64: return launch_bn<FMT, 64, false>(a);
+    case 128: return launch_bn<FMT, 128, false>(a);
+    default: return launch_bn<FMT, 256, false>(a);
   }
 }
 
@@ -851,6 +909,17 @@ cudaError_t launch_prefill(const LinearArgs& a) {
     case INT2_SYM: return launch_fmt<INT2_SYM>(a, BN);
   }
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_prefill_a8(const LinearArgs& a) {
+  if (a.fmt != INT8_SYM || a.K % 128) return cudaErrorNotSupported;
+  const int BN = a.M <= 32 ? 32 : a.M <= 64 ? 64 : a.M <= 128 ? 128 : 256;
+  switch (BN) {
+    case 32: return launch_bn<INT8_SYM, 32, true>(a);
+    case 64: return launch_bn<INT8_SYM, 64, true>(a);
+    case 128: return launch_bn<INT8_SYM, 128, true>(a);
+    default: return launch_bn<INT8_SYM, 256, true>(a);
+  }
 }
 
 cudaError_t read_device_error(unsigned* value, bool clear) {

@@ -43,6 +43,7 @@ class Workload:
     x_channel_mult: float = 1.0
     bias_sigma: float | None = None
     note: str = ""
+    act_int8: bool = False   # activation-quantized linear (per-token INT8 x)
 
     @property
     def w_outlier_count(self) -> int:
@@ -73,8 +74,14 @@ PREFILL = Workload("prefill_int8_g256", "int8_sym", N=8192, K=8192, Ms=(1024, 20
 FP8 = Workload("fp8_e4m3_8192", "fp8_e4m3", N=8192, K=8192, Ms=(1, 16, 1024), group_size=128,
                seed=6, note="FP8 E4M3 weight-only, fp32 scale per 128 along K")
 
+# the prefill layer and inputs again, through the activation-quantized linear
+A8 = Workload("a8_int8_g256_8192", "int8_sym", N=8192, K=8192, Ms=(1024, 2048, 4096),
+              group_size=256, seed=4, x_channel_frac=0.01, x_channel_mult=10.0,
+              bias_sigma=0.01, act_int8=True,
+              note="W8A8: the prefill layer with per-token INT8 activations")
+
 ALL = (PR1, DECODE, CODEBOOK, NVFP4, PREFILL, MXFP4, FP8)
-BY_NAME = {w.name: w for w in ALL}
+BY_NAME = {w.name: w for w in ALL + (A8,)}
 
 
 def make_weight(w: Workload) -> np.ndarray:

@@ -172,3 +172,33 @@ def test_every_header_call_has_a_binding():
     """The Python binding carries every C name the header declares."""
     missing = [n for n in _declared() if not callable(getattr(wqm, n, None))]
     assert not missing, missing
+
+
+def test_linear_a8_argument_checks():
+    """The activation-quantized linear refuses what it has no kernel for and
+    bad workspaces before launching anything (fake, aligned addresses)."""
+    base = 1 << 30
+    x, w, s, out, ws = base, base * 2, base * 3, base * 4, base * 5
+    f8, f4 = wqm.FORMATS["int8_sym"], wqm.FORMATS["int4_sym"]
+    M, N, K, G = 64, 256, 1024, 128
+    need = wqm.wq_linear_a8_workspace_size(M, K)
+    assert need == ((M * K + 255) // 256) * 256 + 4 * M
+    lib = wqm._lib
+    assert lib.wq_linear_a8(x, w, s, None, M, N, K, f4, G, ws, need, out, None) == \
+        wqm.WQ_ERR_UNSUPPORTED
+    assert lib.wq_linear_a8(x, w, s, None, M, N, 1088, f8, 64, ws, need * 2, out, None) == \
+        wqm.WQ_ERR_UNSUPPORTED                                   # K % 128 != 0
+    assert lib.wq_linear_a8(x, w, s, None, M, N, K, f8, G, ws, need - 1, out, None) == \
+        wqm.WQ_ERR_INVALID_ARG                                   # workspace too small
+    assert lib.wq_linear_a8(x, w, s, None, M, N, K, f8, G, None, need, out, None) == \
+        wqm.WQ_ERR_INVALID_ARG
+    assert lib.wq_linear_a8(x, w, s, None, M, N, K, f8, G, ws + 8, need, out, None) == \
+        wqm.WQ_ERR_ALIGNMENT
+    assert lib.wq_linear_a8(x, w, s, None, M, N, K, f8, G, x, need, out, None) == \
+        wqm.WQ_ERR_INVALID_ARG                                   # workspace overlaps x
+    assert lib.wq_linear_a8(x, w, s, None, M, N, K, f8, 48, ws, need, out, None) == \
+        wqm.WQ_ERR_INVALID_ARG                                   # bad group
+    assert lib.wq_linear_a8(x, w, s, None, 0, N, K, f8, G, None, 0, out, None) == wqm.WQ_OK
+    assert lib.wq_quantize_act_int8(x, M, 1020, ws, ws + M * 1024, None) == \
+        wqm.WQ_ERR_INVALID_ARG                                   # K % 8 != 0
+    assert lib.wq_quantize_act_int8(x + 8, M, K, ws, ws + M * K, None) == wqm.WQ_ERR_ALIGNMENT
