@@ -568,16 +568,258 @@ def time_workload(wl, Ms, steps, warmup, device, l2, world, local_rank, do_e2e):
     }
 
 
+# ------------------------------------------------------------------ MoE
+def time_moe(mw, steps, warmup, device, l2, world, local_rank, do_e2e, do_cpu, cpu_seconds):
+    """One step = one single-launch grouped linear (wq_linear_grouped_dev) over
+    the layer's experts, with the routing offsets resident on the device;
+    stacked expert copies rotate past L2.  Context: the same step as one
+    wq_linear per non-empty expert (host offsets)."""
+    import torch
+
+    import mixed_gemm_b200 as wq
+    import synth.workloads as W
+
+    counts = W.moe_counts(mw)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+    experts = []
+    for e in range(mw.E):
+        wd = torch.from_numpy(W.moe_weight(mw, e)).to(device)
+        experts.append(wq.quantize_and_pack(wd, mw.fmt, mw.group_size))
+        del wd
+    stacked = wq.stack_experts(experts)
+    R = max(2, int(math.ceil(3 * l2 / stacked.nbytes)))
+    copies = [stacked] + [stacked.clone() for _ in range(R - 1)]
+    xa = W.moe_x(mw)
+    x = torch.from_numpy(xa.view(np.int16).copy()).view(torch.bfloat16).to(device)
+    off_d = torch.from_numpy(offsets).to(device)
+    y = torch.empty((mw.rows, mw.N), dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.Stream(device)
+    work_bytes = W.moe_bytes(mw, counts)
+    flops = 2.0 * mw.rows * mw.N * mw.K
+    prefill_like = mw.rows // mw.E > 64
+    counter = [0]
+
+    def step():
+        c = copies[counter[0] % R]
+        counter[0] += 1
+        wq.wq_linear_grouped_dev(x, c.w, c.scales, c.aux, None, off_d, mw.E, mw.rows, mw.N, mw.K,
+                                 mw.fmt, mw.group_size, y, stream)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier(device_ids=[local_rank])
+
+    C = max(1, min(100, steps))
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            step()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(C):
+            step()
+    rem = steps % C
+    g_rem = None
+    if rem:
+        g_rem = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_rem, stream=stream):
+            for _ in range(rem):
+                step()
+    with torch.cuda.stream(stream):
+        g.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        for _ in range(max(1, warmup // C)):
+            g.replay()
+    torch.cuda.synchronize()
+    props = torch.cuda.get_device_properties(device)
+    uuid = getattr(props, "uuid", None)
+    clocks = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(device.index))
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for _ in range(steps // C):
+            g.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        ev1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier()
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, device)
+    sec = ms / 1e3
+    pk, pk_kind = peaks()
+    if prefill_like:
+        value = whole_job_value(world, steps, flops, sec, 1e12)
+        unit, bound = "TFLOP/s", "tensor"
+        achieved = flops / (sec / steps) / 1e12
+        peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    else:
+        value = whole_job_value(world, steps, work_bytes, sec, 1e9)
+        unit, bound = "GB/s", "hbm"
+        achieved = work_bytes / (sec / steps) / 1e9
+        peak = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+
+    # context: the host loop of one launch per non-empty expert
+    loop_us = None
+    if world == 1:
+        def loop_step():
+            c = copies[counter[0] % R]
+            counter[0] += 1
+            wq.linear_grouped(x, [c_e for c_e in per_expert(c)], offsets, out=y, stream=stream)
+
+        wb, sb, ab = wq.wq_packed_sizes(mw.fmt, mw.N, mw.K, mw.group_size)
+
+        def per_expert(c):
+            return [wq.PackedWeight(mw.fmt, mw.N, mw.K, mw.group_size, c.w[e * wb:(e + 1) * wb],
+                                    c.scales[e * sb:(e + 1) * sb],
+                                    None if c.aux is None else c.aux[e * ab:(e + 1) * ab])
+                    for e in range(mw.E)]
+
+        views = [per_expert(c) for c in copies]
+        k = [0]
+
+        def loop_once():
+            v = views[k[0] % R]
+            k[0] += 1
+            wq.linear_grouped(x, v, offsets, out=y, stream=stream)
+
+        for _ in range(3):
+            loop_once()
+        torch.cuda.synchronize()
+        gl = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gl, stream=stream):
+            for _ in range(10):
+                loop_once()
+        with torch.cuda.stream(stream):
+            gl.replay()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            gl.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        loop_us = e0.elapsed_time(e1) * 1e3 / 10
+        del gl
+
+    e2e = None
+    if do_e2e:
+        xh = torch.from_numpy(xa.view(np.int16).copy()).view(torch.bfloat16).pin_memory()
+        oh = torch.from_numpy(offsets).pin_memory()
+        yh = torch.empty((mw.rows, mw.N), dtype=torch.bfloat16).pin_memory()
+        e2e_steps = max(3, min(steps, 200))
+
+        def e2e_step():
+            with torch.cuda.stream(stream):
+                x.copy_(xh, non_blocking=True)
+                off_d.copy_(oh, non_blocking=True)
+                step()
+                yh.copy_(y, non_blocking=True)
+            stream.synchronize()
+
+        for _ in range(3):
+            e2e_step()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        es = max_over_ranks(e0.elapsed_time(e1), world, device) / 1e3
+        ev = whole_job_value(world, e2e_steps, flops if prefill_like else work_bytes, es,
+                             1e12 if prefill_like else 1e9)
+        e2e = {"value": ev, "unit": unit, "steps": e2e_steps,
+               "h2d_bytes_per_step": int(xa.nbytes + offsets.nbytes),
+               "d2h_bytes_per_step": int(mw.rows * mw.N * 2)}
+
+    cb = None
+    if do_cpu:
+        cb = moe_cpu_baseline(mw, counts, offsets, xa, prefill_like, cpu_seconds)
+    del g, g_rem
+    return {
+        "value": value, "unit": unit, "steps": steps, "warmup": warmup, "ms_per_step": ms / steps,
+        "config": {"workload": mw.name, "format": mw.fmt, "group_size": mw.group_size,
+                   "experts": mw.E, "N": mw.N, "K": mw.K, "rows": mw.rows,
+                   "tokens": mw.tokens, "topk": mw.topk,
+                   "counts": {"min": int(counts.min()), "max": int(counts.max()),
+                              "empty": int((counts == 0).sum())},
+                   "parallelism": f"replicas{world}",
+                   "l2": f"rotating {R} stacked-expert copies "
+                         f"({R * stacked.nbytes / 2**20:.0f} MiB > 3x L2 {l2 / 2**20:.0f} MiB)",
+                   "timing": f"CUDA graphs of {C} steps, each replayed once untimed; CUDA "
+                             "events on the launch stream"},
+        "roofline": {"bound": bound, "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s" if prefill_like else "GB/s", "frac": achieved / peak,
+                     "traffic": None, "peak_source": pk_kind, "kernel": "prefill_kernel"},
+        "gpu_launches": steps, "clocks": clk, "e2e": e2e, "cpu_baseline": cb,
+        "context": {"host_loop_us_per_step": loop_us,
+                    "single_launch_us_per_step": ms / steps * 1e3,
+                    "note": "host loop: one wq_linear per non-empty expert from host offsets"},
+    }
+
+
+def moe_cpu_baseline(mw, counts, offsets, xa, prefill_like, seconds):
+    """The oracle on a bounded sample of the MoE step: every row of each
+    expert against a subset of that expert's output features."""
+    import oracle
+    import synth.workloads as W
+
+    orc = oracle.Oracle()
+    q = []
+    for e in range(mw.E):
+        q.append(orc.quantize(mw.fmt, W.moe_weight(mw, e), mw.group_size))
+
+    def sample(cols):
+        t0 = time.perf_counter()
+        for e in range(mw.E):
+            a, b = int(offsets[e]), int(offsets[e + 1])
+            if a == b:
+                continue
+            codes, scales, aux = q[e]
+            ms = np.repeat(np.arange(b - a), cols)
+            ns = np.tile(np.arange(cols) * (mw.N // cols), b - a)
+            orc.linear_sampled(mw.fmt, codes, scales, aux, mw.N, mw.K, mw.group_size, xa[a:b],
+                               None, ms, ns)
+        return time.perf_counter() - t0
+
+    cols = 2
+    t = sample(cols)
+    cols = int(min(mw.N, max(1, cols * seconds / max(t, 1e-4))))
+    reps, t = 0, 0.0
+    while reps == 0 or t < 0.8 * seconds:
+        t += sample(cols)
+        reps += 1
+    frac = cols / mw.N
+    if prefill_like:
+        value, unit = reps * 2.0 * mw.rows * mw.N * mw.K * frac / t / 1e12, "TFLOP/s"
+    else:
+        value, unit = reps * W.moe_bytes(mw, counts) * frac / t / 1e9, "GB/s"
+    return {"value": value, "unit": unit, "cores": orc.threads(), "kind": "oracle",
+            "sample": f"{cols} of {mw.N} output features of every routed row of every expert, "
+                      f"{orc.threads()} threads, {reps} pass(es), {t:.1f} s"}
+
+
 # ------------------------------------------------------------------ main
 def main():
     args = parse()
     import synth.workloads as W
 
-    wl = W.BY_NAME[args.workload]
-    Ms = tuple(int(m) for m in args.ms.split(",")) if args.ms else wl.Ms
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.workload in W.MOE:
+        return main_moe(args, W.MOE[args.workload], world, rank, local_rank)
+    wl = W.BY_NAME[args.workload]
+    Ms = tuple(int(m) for m in args.ms.split(",")) if args.ms else wl.Ms
     tflops_metric = min(Ms) >= 1024
     unit = ("TOPS" if wl.act_int8 else "TFLOP/s") if tflops_metric else "GB/s"
 
@@ -669,6 +911,58 @@ def main():
     }
     if second is not None:
         line["prefill"] = second
+    print(json.dumps(line), flush=True)
+
+
+def main_moe(args, mw, world, rank, local_rank):
+    """The grouped (mixture-of-experts) workloads: one JSON line, like main()."""
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        import synth.workloads as W
+        counts = W.moe_counts(mw)
+        offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+        prefill_like = mw.rows // mw.E > 64
+        per_step = min(12.0, max(0.05, 60.0 / max(1, args.steps + args.warmup)))
+        vals = [moe_cpu_baseline(mw, counts, offsets, W.moe_x(mw), prefill_like, per_step)
+                for _ in range(max(1, args.steps))]
+        v = float(np.median([c["value"] for c in vals]))
+        unit = vals[0]["unit"]
+        print(json.dumps({"impl": "reference", "metric": METRIC, "value": v, "unit": unit,
+                          "n_gpus": args.gpus, "steps": len(vals), "warmup": args.warmup,
+                          "ms_per_step": per_step * 1e3, "higher_is_better": True,
+                          "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                          "data": "synthetic", "config": {"workload": mw.name},
+                          "cpu_baseline": vals[0],
+                          "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0,
+                                  "d2h_bytes_per_step": 0}}), flush=True)
+        return
+    import torch
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    else:
+        torch.cuda.set_device(0)
+    device = torch.device("cuda", torch.cuda.current_device())
+    import mixed_gemm_b200  # noqa: F401
+    props = torch.cuda.get_device_properties(device)
+    l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20)
+    r = time_moe(mw, args.steps, args.warmup, device, l2, world, local_rank, not args.no_e2e,
+                 rank == 0 and world == 1 and not args.no_cpu_baseline, args.cpu_seconds)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {"metric": METRIC, "value": r["value"], "unit": r["unit"], "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": r["config"], "roofline": r["roofline"],
+            "gpu_launches": r["gpu_launches"], "clocks": r["clocks"], "e2e": r["e2e"],
+            "cpu_baseline": r["cpu_baseline"], "context": r["context"]}
     print(json.dumps(line), flush=True)
 
 

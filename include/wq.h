@@ -23,7 +23,7 @@
  *    WQ_ERR_CUDA (from cudaGetLastError).  No C++ exception crosses the ABI.
  *  - bf16 values are IEEE bfloat16 bit patterns (uint16_t).
  *  - Shapes: N % 16 == 0 and K % 64 == 0 for every format (the packed tile is
- *    16 rows by 64 (2- and 4-bit) or 32 (INT8, FP8) K elements); INT formats take
+ *    16 rows by 64 (2-, 3- and 4-bit) or 32 (INT8, FP8) K elements); INT formats take
  *    group_size in {32, 64, 128, 256} with K % group_size == 0; NVFP4 has a
  *    fixed block of 16 (group_size 16 or 0), MXFP4 one of 32 (group_size 32
  *    or 0); CB4 ignores group_size; the FP8 formats take the INT group sizes.
@@ -54,8 +54,12 @@
  *   WQ_INT2_SYM : codes  u8 [N, K/4]  two's complement 2-bit fields, element
  *                                      4i+j at bits 2j..2j+1 of byte i
  *                 scales bf16 [N, K/G]
+ *   WQ_INT3_SYM : codes  u8 [N, 3K/8] two's complement 3-bit fields, a
+ *                                      little-endian bit stream per row:
+ *                                      element k at bits 3k..3k+2
+ *                 scales bf16 [N, K/G]
  * Dequantized value of element (n, k) -- what wq_dequant returns:
- *   INT2/INT4/INT8_SYM: q * s           ASYM: (q - z) * s          (exact fp32)
+ *   INT2/INT3/INT4/INT8_SYM: q * s      ASYM: (q - z) * s          (exact fp32)
  *   CB4: fp32(c[idx] * norm[n])         NVFP4: fp32(e2m1(q) * e4m3(sb) * ts)
  *   MXFP4: fp32(e2m1(q) * 2^(e-127))    (exact; +-inf where the product
  *                                          reaches 2^128, NaN for e = 255)
@@ -89,7 +93,8 @@ typedef enum {
   WQ_MXFP4 = 5,     /* E2M1 values, E8M0 power-of-two scale per 32 (OCP MX)    */
   WQ_FP8_E4M3 = 6,  /* E4M3 values, fp32 scale per group (FP8 weight-only)     */
   WQ_FP8_E5M2 = 7,  /* E5M2 values, fp32 scale per group (FP8 weight-only)     */
-  WQ_INT2_SYM = 8   /* symmetric INT2, bf16 scale per group                    */
+  WQ_INT2_SYM = 8,  /* symmetric INT2, bf16 scale per group                    */
+  WQ_INT3_SYM = 9   /* symmetric INT3, bf16 scale per group                    */
 } wq_format_t;
 
 typedef enum {
@@ -200,6 +205,31 @@ int wq_linear_grouped(const void* x, const void* const* packed_w, const void* co
                       const void* const* aux, const void* const* bias, const int64_t* offsets,
                       int64_t E, int64_t N, int64_t K, int format, int group_size, void* out,
                       void* stream);
+
+/* Grouped (mixture-of-experts) linear in ONE launch, with the routing on the
+ * device: E experts of one format, shape [N, K] and group size, whose packed
+ * buffers are stacked (expert e's packed weight at packed_w + e * w_bytes,
+ * its scales at scales + e * scale_bytes, its aux at aux + e * aux_bytes,
+ * the sizes from wq_packed_sizes; bias [E, N] or NULL).  The T rows of x
+ * (bf16 [T, K]) are sorted by expert: expert e owns rows
+ * [offsets[e], offsets[e+1]) and writes the same rows of out (bf16 [T, N]).
+ *   offsets   DEVICE int64 [E + 1], read by the kernel (no host sync), so the
+ *             routing counts may come straight from a device-side router;
+ *             an expert whose offsets leave [0, T] or decrease is skipped and
+ *             sets bit 256 of wq_device_error; rows no expert owns are not
+ *             written
+ * The tcgen05 kernel builds its tile schedule on the device: experts in
+ * order, ceil(count / BN) token tiles each (BN from the mean rows per
+ * expert); the grid holds ceil(T / BN) + E token tiles per 128 output rows
+ * and the tiles past the schedule's end exit at once.  A bound above the
+ * grid limit (65535) returns WQ_ERR_UNSUPPORTED.  Asynchronous.
+ * Source: auto-round-lib README section 2 (moe_gemm(activations, weights,
+ * num_tokens_per_expert, ...): quantized experts, per-expert token counts);
+ * Petit README "Features" (fused MoE kernels). */
+int wq_linear_grouped_dev(const void* x, const void* packed_w, const void* scales,
+                          const void* aux, const void* bias, const int64_t* offsets, int64_t E,
+                          int64_t T, int64_t N, int64_t K, int format, int group_size, void* out,
+                          void* stream);
 
 /* The same linear with a SwiGLU input: x2 is bf16 [M, 2K], each row holding
  * [up | gate] (K values each), and the activation is
@@ -314,7 +344,8 @@ int wq_lloyd_max_centroids(int bits, float* centroids_out);
  * runs out sets a bit here (1 producer, 2 producer drain, 4/8 MMA waits, 16
  * MMA drain, 32 dequant, 64 epilogue; 128 the decode kernel's wait for its
  * staged activation slice) and the thread block winds down instead of
- * hanging, leaving the CUDA context usable.  Synchronizes the device (a
+ * hanging, leaving the CUDA context usable.  Bit 256 reports routing offsets
+ * of wq_linear_grouped_dev outside [0, T] or decreasing.  Synchronizes the device (a
  * symbol copy).  Writes the word to *value, clears it when `clear` is non-zero,
  * and returns WQ_ERR_DEVICE_CHECK when it was non-zero, WQ_OK otherwise. */
 int wq_device_error(unsigned* value, int clear);

@@ -19,7 +19,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libwq.so")
 
 FORMATS = {"int4_sym": 0, "int4_asym": 1, "int8_sym": 2, "cb4": 3, "nvfp4": 4, "mxfp4": 5,
-           "fp8_e4m3": 6, "fp8_e5m2": 7, "int2_sym": 8}
+           "fp8_e4m3": 6, "fp8_e5m2": 7, "int2_sym": 8, "int3_sym": 9}
 FORMAT_NAMES = {v: k for k, v in FORMATS.items()}
 
 WQ_OK = 0
@@ -50,6 +50,8 @@ _SIGS = {
     "wq_unpack": ([_int, _i64, _i64, _int, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr], _int),
     "wq_dequant": ([_int, _i64, _i64, _int, _ptr, _ptr, _ptr, _ptr, _ptr], _int),
     "wq_linear": ([_ptr, _ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _int, _int, _ptr, _ptr], _int),
+    "wq_linear_grouped_dev": ([_ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _i64, _int,
+                               _int, _ptr, _ptr], _int),
     "wq_linear_swiglu": ([_ptr, _ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _int, _int, _ptr,
                           ctypes.c_size_t, _ptr, _ptr], _int),
     "wq_linear_grouped": ([_ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _int, _int,
@@ -168,6 +170,15 @@ def wq_linear_grouped(x, packed_w, scales, aux, bias, offsets, N, K, fmt, group_
                                   _stream(stream)), "wq_linear_grouped")
 
 
+def wq_linear_grouped_dev(x, packed_w, scales, aux, bias, offsets, E, T, N, K, fmt, group_size,
+                          out, stream=None):
+    """One launch over E stacked experts; ``offsets``: device int64 [E + 1]."""
+    _check(_lib.wq_linear_grouped_dev(_addr(x), _addr(packed_w), _addr(scales), _addr(aux),
+                                      _addr(bias), _addr(offsets), E, T, N, K, _fmt(fmt),
+                                      group_size, _addr(out), _stream(stream)),
+           "wq_linear_grouped_dev")
+
+
 def wq_addmm_requant(fmt, N, K, group_size, packed_w, packed_scales, mat1, mat2, rank, alpha,
                      beta=1.0, seed=None, stream=None):
     _check(_lib.wq_addmm_requant(_fmt(fmt), N, K, group_size, _addr(packed_w),
@@ -230,5 +241,5 @@ def wq_device_sm_count() -> int:
     return n.value
 
 
-from .api import (PackedWeight, linear, linear_a8, linear_grouped, linear_swiglu,  # noqa: E402,F401
-                  pack, quantize_and_pack)
+from .api import (PackedWeight, linear, linear_a8, linear_grouped, linear_moe,  # noqa: E402,F401
+                  linear_swiglu, pack, quantize_and_pack, stack_experts)

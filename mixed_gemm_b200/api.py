@@ -13,13 +13,14 @@ from dataclasses import dataclass
 import torch
 
 from . import (FORMATS, wq_canonical_sizes, wq_linear, wq_linear_a8, wq_linear_a8_workspace_size,
-               wq_linear_grouped, wq_linear_swiglu, wq_lloyd_max_centroids, wq_pack,
-               wq_packed_sizes, wq_quantize)
+               wq_linear_grouped, wq_linear_grouped_dev, wq_linear_swiglu,
+               wq_lloyd_max_centroids, wq_pack, wq_packed_sizes, wq_quantize)
 
 
 @dataclass
 class PackedWeight:
-    """Packed buffers of one [N, K] weight, resident on a CUDA device."""
+    """Packed buffers of one [N, K] weight (or, with ``experts`` > 1, of
+    that many experts' weights stacked back to back), on a CUDA device."""
     fmt: str
     N: int
     K: int
@@ -27,6 +28,7 @@ class PackedWeight:
     w: torch.Tensor        # packed codes (uint8)
     scales: torch.Tensor   # packed scales (uint8 view of the bytes)
     aux: torch.Tensor | None
+    experts: int = 1
 
     @property
     def nbytes(self) -> int:
@@ -34,7 +36,8 @@ class PackedWeight:
 
     def clone(self) -> "PackedWeight":
         c = PackedWeight(self.fmt, self.N, self.K, self.group_size, self.w.clone(),
-                         self.scales.clone(), None if self.aux is None else self.aux.clone())
+                         self.scales.clone(), None if self.aux is None else self.aux.clone(),
+                         self.experts)
         torch.cuda.synchronize(self.w.device)  # final before any wq_linear prefetches it
         return c
 
@@ -183,6 +186,42 @@ def linear_a8(x: torch.Tensor, weight: PackedWeight, bias: torch.Tensor | None =
             s.synchronize()
         return yh.reshape(*lead, weight.N)
     return y.reshape(*lead, weight.N)
+
+
+def stack_experts(weights: list) -> PackedWeight:
+    """E PackedWeights of one format, shape and group size -> one PackedWeight
+    whose buffers hold them back to back at the packed sizes (the layout
+    ``linear_moe`` and wq_linear_grouped_dev read)."""
+    w0 = weights[0]
+    assert all(w.fmt == w0.fmt and w.N == w0.N and w.K == w0.K and
+               w.group_size == w0.group_size and w.experts == 1 for w in weights)
+    wb, sb, ab = wq_packed_sizes(w0.fmt, w0.N, w0.K, w0.group_size)
+    cat = lambda ts, n: torch.cat([t[:n] for t in ts] + [torch.zeros(16, dtype=torch.uint8,
+                                                                     device=ts[0].device)])
+    aux = cat([w.aux for w in weights], ab) if ab else None
+    return PackedWeight(w0.fmt, w0.N, w0.K, w0.group_size, cat([w.w for w in weights], wb),
+                        cat([w.scales for w in weights], sb), aux, experts=len(weights))
+
+
+def linear_moe(x: torch.Tensor, experts: PackedWeight, offsets: torch.Tensor,
+               bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """Mixture-of-experts linear in one launch with device-side routing:
+    rows offsets[e]:offsets[e+1] of ``x`` ([T, K] bf16, sorted by expert) use
+    expert e of ``experts`` (from ``stack_experts``); ``offsets`` is a device
+    int64 tensor [E + 1] (e.g. a cumulative sum of a router's counts);
+    ``bias`` an optional [E, N] bf16 tensor.  Rows no expert owns are left
+    as they are in ``out``."""
+    E = experts.experts
+    assert offsets.is_cuda and offsets.dtype == torch.int64 and offsets.numel() == E + 1
+    xd = x.contiguous()
+    T = xd.shape[0]
+    assert xd.shape == (T, experts.K)
+    y = out if out is not None else torch.zeros((T, experts.N), dtype=torch.bfloat16,
+                                                device=experts.w.device)
+    wq_linear_grouped_dev(xd, experts.w, experts.scales, experts.aux, bias, offsets.contiguous(),
+                          E, T, experts.N, experts.K, experts.fmt, experts.group_size, y, stream)
+    return y
 
 
 def linear_grouped(x: torch.Tensor, weights: list, offsets, bias: list | None = None,

@@ -28,7 +28,7 @@ bool overlap(const void* p, int64_t pb, const void* q, int64_t qb) {
 
 // Shape / format checks shared by every entry point.
 int check_shape(int f, int64_t N, int64_t K, int G) {
-  if (f < INT4_SYM || f > INT2_SYM) return WQ_ERR_INVALID_ARG;
+  if (f < INT4_SYM || f > INT3_SYM) return WQ_ERR_INVALID_ARG;
   if (N <= 0 || K <= 0) return WQ_ERR_INVALID_ARG;
   if (N % 16 || K % 64) return WQ_ERR_INVALID_ARG;
   if (N > (1LL << 30) || K > (1LL << 24) || N * K > (1LL << 40)) return WQ_ERR_INVALID_ARG;
@@ -168,6 +168,7 @@ int wq_canonical_sizes(int f, int64_t N, int64_t K, int G, size_t* cb, size_t* s
     case INT4_ASYM: c = N * K / 2; s = 2 * N * (K / G); a = N * (K / G); break;
     case INT8_SYM: c = N * K; s = 2 * N * (K / G); break;
     case INT2_SYM: c = N * K / 4; s = 2 * N * (K / G); break;
+    case INT3_SYM: c = N * K * 3 / 8; s = 2 * N * (K / G); break;
     case FP8_E4M3:
     case FP8_E5M2: c = N * K; s = 4 * N * (K / G); break;
     case CB4: c = N * K / 2; s = 2 * N; a = 64; break;
@@ -287,6 +288,49 @@ int wq_linear_grouped(const void* x, const void* const* pw, const void* const* s
     if (st) return st;
   }
   return WQ_OK;
+}
+
+int wq_linear_grouped_dev(const void* x, const void* pw, const void* scales, const void* aux,
+                          const void* bias, const int64_t* offsets, int64_t E, int64_t T,
+                          int64_t N, int64_t K, int f, int G, void* out, void* stream) {
+  int st = check_shape(f, N, K, G);
+  if (st) return st;
+  G = effective_group(f, G);
+  if (E <= 0 || E > (1 << 20) || T < 0 || T > (1LL << 24)) return WQ_ERR_INVALID_ARG;
+  const bool need_aux = f == INT4_ASYM || f == CB4 || f == NVFP4;
+  if (!x || !pw || !scales || !out || !offsets || (need_aux && !aux)) return WQ_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(pw, 16) || !aligned(scales, 16) || !aligned(out, 16) ||
+      !aligned(offsets, 8) || (bias && !aligned(bias, 16)) ||
+      (aux && !aligned(aux, (f == INT4_ASYM) ? 16 : 4)))
+    return WQ_ERR_ALIGNMENT;
+  size_t wb = 0, sb = 0, ab = 0;
+  wq_packed_sizes(f, N, K, G, &wb, &sb, &ab);
+  const int64_t ob = T * N * 2;
+  if (T > 0 && (overlap(out, ob, x, T * K * 2) || overlap(out, ob, pw, E * (int64_t)wb) ||
+                overlap(out, ob, scales, E * (int64_t)sb) ||
+                overlap(out, ob, aux, E * (int64_t)ab) || overlap(out, ob, bias, E * N * 2) ||
+                overlap(out, ob, offsets, (E + 1) * 8)))
+    return WQ_ERR_INVALID_ARG;
+  if (T == 0) return WQ_OK;
+  LinearArgs a;
+  a.x = x;
+  a.w = pw;
+  a.scales = scales;
+  a.aux = aux;
+  a.bias = bias;
+  a.out = out;
+  a.M = T;
+  a.N = N;
+  a.K = K;
+  a.fmt = f;
+  a.G = G;
+  a.stream = (cudaStream_t)stream;
+  a.offsets = offsets;
+  a.E = (int)E;
+  a.scale_stride = (int64_t)sb;
+  a.aux_stride = (int64_t)ab;
+  const cudaError_t e = launch_prefill_grouped(a);
+  return e == cudaErrorNotSupported ? WQ_ERR_UNSUPPORTED : cuda_status(e);
 }
 
 int wq_linear_swiglu(const void* x2, const void* pw, const void* scales, const void* aux,

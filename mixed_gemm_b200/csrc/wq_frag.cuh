@@ -56,6 +56,21 @@ static __device__ __forceinline__ void frag_int2(uint32_t wd, int s, uint32_t of
   }
 }
 
+// INT3, two planes: low bits as the INT2 fields of word `lo` (chunk c), the
+// high bit from the lane's high-plane word `hi` at 8 c + 4 s + i (and 16
+// above); fragment i of step s as bf16 (128 + c), minus the offset (132 for
+// offset-binary codes).
+static __device__ __forceinline__ void frag_int3(uint32_t lo, uint32_t hi, int c, int s,
+                                                 uint32_t off, uint32_t (&a)[4]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    // (the high bits move right first: the upper one may sit at bit 31)
+    const uint32_t t = ((lo >> (2 * (4 * s + i))) & 0x00030003u) |
+                       (((hi >> (8 * c + 4 * s + i)) << 2) & 0x00040004u) | 0x43004300u;
+    a[i] = bsub2(t, off);
+  }
+}
+
 // INT8 offset-binary bytes -> exact integers via the fp32 magic 2^23 + u.
 static __device__ __forceinline__ float i8val(uint32_t w, int i) {
   return __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7440u | i)) - 8388736.0f;

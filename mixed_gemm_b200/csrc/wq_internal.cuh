@@ -25,6 +25,13 @@
 //   {32c + 8tq + 4s + e}, field p = 8*(e&1) + 4*s + 2*(e>>1) + hr at bit 2p,
 //   so that (word >> 2(4s + i)) & 0x00030003 yields fragment register i of
 //   step s as two fields at bit 0 and bit 16; stored offset-binary (v + 2).
+//   INT3_SYM: blocks of 384 bytes (64 K) in two planes.  The low plane (the
+//   first 256 bytes) holds bits 0..1 of each offset-binary code (v + 4)
+//   exactly as INT2 holds its fields; the high plane (the last 128 bytes)
+//   gives lane L the word at 256 + 4 L, holding bit 2 of field p of chunk c
+//   at bit 16 (p >> 3) + 8 c + (p & 7), so that
+//   (hi >> (8 c + 4 s + i)) & 0x00010001 yields the high bits of fragment
+//   register i of step s of chunk c at bit 0 and bit 16.
 //   INT4_SYM nibbles are stored offset-binary (v + 8); INT8 bytes likewise
 //   (v + 128), word j = 2s + hr, byte e; FP8 (E4M3, E5M2) bytes as they
 //   are, at the INT8 positions.
@@ -48,21 +55,23 @@
 namespace wq {
 
 enum Fmt { INT4_SYM = 0, INT4_ASYM = 1, INT8_SYM = 2, CB4 = 3, NVFP4 = 4, MXFP4 = 5,
-           FP8_E4M3 = 6, FP8_E5M2 = 7, INT2_SYM = 8 };
+           FP8_E4M3 = 6, FP8_E5M2 = 7, INT2_SYM = 8, INT3_SYM = 9 };
 
 __host__ __device__ inline bool is_int_fmt(int f) {
-  return f == INT4_SYM || f == INT4_ASYM || f == INT8_SYM || f == INT2_SYM;
+  return f == INT4_SYM || f == INT4_ASYM || f == INT8_SYM || f == INT2_SYM || f == INT3_SYM;
 }
 // formats with one scale per group of G along K, folded into fp32 sums
 __host__ __device__ inline bool is_fp8(int f) { return f == FP8_E4M3 || f == FP8_E5M2; }
 __host__ __device__ inline bool is_grouped_fmt(int f) { return is_int_fmt(f) || is_fp8(f); }
 // bits per packed code
 __host__ __device__ inline int code_bits(int f) {
-  return f == INT2_SYM ? 2 : (f == INT8_SYM || is_fp8(f)) ? 8 : 4;
+  return f == INT2_SYM ? 2 : f == INT3_SYM ? 3 : (f == INT8_SYM || is_fp8(f)) ? 8 : 4;
 }
 __host__ __device__ inline bool is_4bit(int f) { return code_bits(f) == 4; }
 // bytes of one packed block (16 rows x block_k(f) K elements)
-__host__ __device__ inline int block_bytes(int f) { return code_bits(f) == 2 ? 256 : 512; }
+__host__ __device__ inline int block_bytes(int f) {
+  return code_bits(f) == 2 ? 256 : code_bits(f) == 3 ? 384 : 512;
+}
 // elements of K per 512-byte block
 __host__ __device__ inline int block_k(int f) { return code_bits(f) == 8 ? 32 : 64; }
 
@@ -95,6 +104,25 @@ __host__ __device__ inline void packed_loc(int f, int64_t n, int64_t k, int64_t 
     *byte_off = ((tile * (K >> 5) + b) * 32 + lane) * 16 + j * 4 + e;
     *shift = 0;
   }
+}
+
+// INT3: byte and shift of the low-plane field (bits 0..1) and of the
+// high-plane bit (bit 2) of element (n, k).
+__host__ __device__ inline void packed_loc3(int64_t n, int64_t k, int64_t K, int64_t* lo_off,
+                                            int* lo_shift, int64_t* hi_off, int* hi_shift) {
+  const int64_t tile = n >> 4;
+  const int r = (int)(n & 15), g = r & 7, hr = r >> 3;
+  const int64_t b = k >> 6;
+  const int kk = (int)(k & 63), c = kk >> 5, kc = kk & 31, tq = kc >> 3, e8 = kc & 7,
+            s = e8 >> 2, e = e8 & 3;
+  const int lane = 4 * g + tq;
+  const int p = 8 * (e & 1) + 4 * s + 2 * (e >> 1) + hr;
+  const int64_t base = (tile * (K >> 6) + b) * 384;
+  *lo_off = base + lane * 8 + c * 4 + (p >> 2);
+  *lo_shift = (p & 3) * 2;
+  const int bit = 16 * (p >> 3) + 8 * c + (p & 7);
+  *hi_off = base + 256 + lane * 4 + (bit >> 3);
+  *hi_shift = bit & 7;
 }
 
 // Index (in elements) of the packed group scale / NVFP4 block scale of (n, group).
@@ -157,6 +185,12 @@ struct LinearArgs {
   // x holds rows [up | gate] of 2K values; the activation is up * silu(gate)
   // (decode path only: the prefill path reads a materialized activation)
   bool swiglu = false;
+  // grouped launch (prefill kernel only): device row offsets [E + 1], M = T
+  // rows of x; w, scales, aux and bias are the first expert's, the others
+  // follow at the packed sizes (scale_stride / aux_stride bytes, N for bias)
+  const int64_t* offsets = nullptr;
+  int E = 1;
+  int64_t scale_stride = 0, aux_stride = 0;
 };
 
 // cudaErrorNotSupported (nothing launched) when the shape does not fit the
@@ -173,6 +207,9 @@ cudaError_t launch_prefill(const LinearArgs& a);
 // the INT8 activation codes [M, K], a.aux the per-token fp32 scales [M];
 // INT8_SYM weights, K % 128 == 0 (else cudaErrorNotSupported, nothing launched)
 cudaError_t launch_prefill_a8(const LinearArgs& a);
+// One launch over every expert of a grouped linear (a.offsets on the device);
+// cudaErrorNotSupported when the schedule's tile bound exceeds the grid limit
+cudaError_t launch_prefill_grouped(const LinearArgs& a);
 // Per-token INT8 quantization of bf16 x [M, K] (K % 8 == 0): codes xq [M, K],
 // scales sx [M]
 cudaError_t launch_quant_act_int8(const void* x, int64_t M, int64_t K, void* xq, float* sx,

@@ -24,6 +24,13 @@ inline unsigned grid_for(int64_t n) {
 __device__ __forceinline__ uint32_t canon_code(int f, const uint8_t* codes, int64_t n, int64_t k,
                                                int64_t K) {
   if (code_bits(f) == 2) return (codes[n * (K >> 2) + (k >> 2)] >> (2 * (k & 3))) & 3u;
+  if (code_bits(f) == 3) {  // bits 3k..3k+2 of the row's little-endian bit stream
+    const uint8_t* row = codes + n * (3 * K / 8);
+    const int64_t bit = 3 * k;
+    uint32_t v = row[bit >> 3];
+    if ((bit & 7) > 5) v |= (uint32_t)row[(bit >> 3) + 1] << 8;
+    return (v >> (bit & 7)) & 7u;
+  }
   if (is_4bit(f)) {
     uint8_t b = codes[n * (K >> 1) + (k >> 1)];
     return (k & 1) ? (b >> 4) : (b & 15u);
@@ -35,6 +42,7 @@ __device__ __forceinline__ uint32_t canon_code(int f, const uint8_t* codes, int6
 __device__ __forceinline__ uint32_t encode(int f, uint32_t c) {
   if (f == INT4_SYM) return c ^ 0x8u;
   if (f == INT2_SYM) return c ^ 0x2u;
+  if (f == INT3_SYM) return c ^ 0x4u;
   if (f == INT8_SYM) return c ^ 0x80u;
   return c;
 }
@@ -45,6 +53,36 @@ __global__ void pack_w_kernel(int f, int64_t N, int64_t K, const uint8_t* __rest
   const int64_t total = N * K * code_bits(f) / 8;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
        i += (int64_t)gridDim.x * blockDim.x) {
+    if (code_bits(f) == 3) {  // 384-byte blocks of 64 K: low plane, then high plane
+      const int64_t blk_global = i / 384, nblk = K >> 6;
+      const int rem = (int)(i % 384);
+      const int64_t tile = blk_global / nblk, b = blk_global % nblk;
+      uint32_t out = 0;
+      for (int h = 0; h < 8; ++h) {
+        int lane, c, p, sh;
+        if (rem < 256) {            // fields 4q .. 4q + 3 of word c, two bits each
+          if (h >= 4) break;
+          lane = rem >> 3;
+          c = (rem >> 2) & 1;
+          p = 4 * (rem & 3) + h;
+          sh = 2 * h;
+        } else {                    // bit 16 (p >> 3) + 8 c + (p & 7) of the lane's word
+          const int rr = rem - 256, bit = 8 * (rr & 3) + h;
+          lane = rr >> 2;
+          c = (bit & 15) >> 3;
+          p = 8 * (bit >> 4) + (bit & 7);
+          sh = h;
+        }
+        const int g = lane >> 2, tq = lane & 3;
+        const int hr = p & 1, e = ((p >> 1) & 1) * 2 + (p >> 3), s = (p >> 2) & 1;
+        const int64_t n = tile * 16 + g + 8 * hr;
+        const int64_t k = b * 64 + c * 32 + tq * 8 + s * 4 + e;
+        const uint32_t v = encode(f, canon_code(f, codes, n, k, K));
+        out |= (rem < 256 ? (v & 3u) : (v >> 2)) << sh;
+      }
+      pw[i] = (uint8_t)out;
+      continue;
+    }
     if (code_bits(f) == 2) {  // 8-byte lane chunks, 256-byte blocks of 64 K
       const int q = (int)(i & 3), c = (int)((i >> 2) & 1), lane = (int)((i >> 3) & 31);
       const int64_t blk_global = i >> 8, nblk = K >> 6;
@@ -90,6 +128,28 @@ __global__ void pack_w_kernel(int f, int64_t N, int64_t K, const uint8_t* __rest
       out = encode(f, canon_code(f, codes, n, k, K));
     }
     pw[i] = (uint8_t)out;
+  }
+}
+
+// INT3: one thread per 8 elements (three canonical bytes).
+__global__ void unpack_w3_kernel(int64_t N, int64_t K, const uint8_t* __restrict__ pw,
+                                 uint8_t* __restrict__ codes) {
+  const int64_t total = N * K / 8;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t n = i / (K >> 3), k0 = (i % (K >> 3)) * 8;
+    uint32_t bits = 0;
+    for (int h = 0; h < 8; ++h) {
+      int64_t lo, hi;
+      int ls, hs;
+      packed_loc3(n, k0 + h, K, &lo, &ls, &hi, &hs);
+      const uint32_t v = ((pw[lo] >> ls) & 3u) | (((pw[hi] >> hs) & 1u) << 2);
+      bits |= encode(INT3_SYM, v) << (3 * h);
+    }
+    uint8_t* dst = codes + n * (3 * K / 8) + 3 * (k0 >> 3);
+    dst[0] = (uint8_t)bits;
+    dst[1] = (uint8_t)(bits >> 8);
+    dst[2] = (uint8_t)(bits >> 16);
   }
 }
 
@@ -185,11 +245,19 @@ __global__ void dequant_kernel(int f, int64_t N, int64_t K, int G, const uint8_t
     int64_t n = i / K, k = i % K;
     int64_t off;
     int sh;
-    packed_loc(f, n, k, K, &off, &sh);
-    uint32_t raw = (pw[off] >> sh) & ((1u << code_bits(f)) - 1u);
+    uint32_t raw;
+    if (f == INT3_SYM) {
+      int64_t hi;
+      int hs;
+      packed_loc3(n, k, K, &off, &sh, &hi, &hs);
+      raw = ((pw[off] >> sh) & 3u) | (((pw[hi] >> hs) & 1u) << 2);
+    } else {
+      packed_loc(f, n, k, K, &off, &sh);
+      raw = (pw[off] >> sh) & ((1u << code_bits(f)) - 1u);
+    }
     float v;
-    if (f == INT4_SYM || f == INT8_SYM || f == INT2_SYM) {
-      int q = (int)raw - (f == INT4_SYM ? 8 : f == INT2_SYM ? 2 : 128);
+    if (f == INT4_SYM || f == INT8_SYM || f == INT2_SYM || f == INT3_SYM) {
+      int q = (int)raw - (f == INT4_SYM ? 8 : f == INT2_SYM ? 2 : f == INT3_SYM ? 4 : 128);
       float s = bf16_bits_to_f32(((const uint16_t*)ps)[packed_scale_idx(n, k / G, K / G)]);
       v = (float)q * s;
     } else if (f == INT4_ASYM) {
@@ -254,8 +322,12 @@ cudaError_t launch_pack(int f, int64_t N, int64_t K, int G, const void* codes, c
 cudaError_t launch_unpack(int f, int64_t N, int64_t K, int G, const void* pw, const void* ps,
                           const void* pa, void* codes, void* scales, void* aux, cudaStream_t st) {
   const int64_t wbytes = N * K * code_bits(f) / 8;
-  unpack_w_kernel<<<grid_for(wbytes), kThreads, 0, st>>>(f, N, K, (const uint8_t*)pw,
-                                                          (uint8_t*)codes);
+  if (f == INT3_SYM)
+    unpack_w3_kernel<<<grid_for(N * K / 8), kThreads, 0, st>>>(N, K, (const uint8_t*)pw,
+                                                               (uint8_t*)codes);
+  else
+    unpack_w_kernel<<<grid_for(wbytes), kThreads, 0, st>>>(f, N, K, (const uint8_t*)pw,
+                                                            (uint8_t*)codes);
   if (is_fp8(f)) {
     int64_t groups = K / G;
     permute_scales_kernel<uint32_t><<<grid_for(N * groups), kThreads, 0, st>>>(

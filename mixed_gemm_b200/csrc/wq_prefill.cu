@@ -58,7 +58,12 @@ __device__ unsigned int g_wq_device_error;
 namespace {
 
 constexpr int kThreads = 512;  // 4 warpgroups: TMA+MMA, dequant, 2x fold/epilogue
+#ifdef WQ_FAULT_TEST
+// test build only: short waits, and one skipped arrival (see fault_stage)
+constexpr uint32_t kWaitLimit = 1u << 16;
+#else
 constexpr uint32_t kWaitLimit = 1u << 22;
+#endif
 
 struct PrefillParams {
   const void* scales;
@@ -69,6 +74,19 @@ struct PrefillParams {
   int BN, stages, astages;
   int splits;  // K split over a cluster of this many CTAs (1: no cluster)
   uint32_t tmem_cols;
+#ifdef WQ_FAULT_TEST
+  // test build only: the first dequant warp does not arrive on the A-tile
+  // barrier of this K step (-1: never), so the MMA issuer's bounded wait
+  // runs out; no copy is skipped or altered
+  int fault_stage;
+#endif
+  // grouped (mixture-of-experts) launch: device row offsets [E + 1] of the
+  // experts (rows of x sorted by expert), T rows in x; the experts' packed
+  // weights are stacked (expert e's row tiles follow expert e - 1's) and
+  // their scales / aux / bias lie `*_stride` bytes apart.  NULL: one linear.
+  const int64_t* offsets;
+  int E, T;
+  int64_t scale_stride, aux_stride;
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -96,12 +114,15 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 // Bounded wait: false when the CTA is aborting or the limit ran out (which
-// raises the abort flag and the device error word).
+// raises the abort flag and the device error word).  Waits for this CTA's
+// own copies or MMAs in flight (teardown, drain) pass honor_abort = false:
+// they always complete, and the CTA must not release its shared or tensor
+// memory before they do.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                          unsigned code) {
+                                          unsigned code, bool honor_abort = true) {
   for (uint32_t i = 0; i < kWaitLimit; ++i) {
     if (mbar_try(bar, parity)) return true;
-    if ((i & 255u) == 255u && *abort) return false;
+    if (honor_abort && (i & 255u) == 255u && *abort) return false;
   }
   *abort = 1;
   atomicOr(&g_wq_device_error, code);
@@ -264,7 +285,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const PrefillParams p) {
   // one scale per group of K, folded into fp32 sums (INT formats, FP8)
   constexpr bool kInt = FMT == INT4_SYM || FMT == INT4_ASYM || FMT == INT8_SYM ||
-                        FMT == INT2_SYM || FMT == FP8_E4M3 || FMT == FP8_E5M2;
+                        FMT == INT2_SYM || FMT == INT3_SYM || FMT == FP8_E4M3 ||
+                        FMT == FP8_E5M2;
   constexpr bool kFp8 = FMT == FP8_E4M3 || FMT == FP8_E5M2;
   constexpr bool kByte = FMT == INT8_SYM || kFp8;  // one byte per code
   // A8: INT8 activations x INT8 weight codes (kind::i8, s32 accumulators);
@@ -272,7 +294,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int KS = A8 ? 128 : 64;
   static_assert(!A8 || FMT == INT8_SYM, "the i8 path takes INT8 weight codes");
   // packed bytes per stage (8 row tiles x KS)
-  constexpr uint32_t kWpk = (kByte ? 8192u : FMT == INT2_SYM ? 2048u : 4096u) * (A8 ? 2u : 1u);
+  constexpr uint32_t kWpk =
+      (kByte ? 8192u : FMT == INT2_SYM ? 2048u : FMT == INT3_SYM ? 3072u : 4096u) *
+      (A8 ? 2u : 1u);
   // elements of the packed tensor map's inner dimension per row tile and stage
   constexpr int kWbox = (int)(kWpk / 8u / (kWpk / 8u > 1024u ? 8u : 4u));
   // A stage: one 128 x 64 bf16 tile; CB4 adds a second tile holding the
@@ -309,7 +333,61 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile0 = blockIdx.x * 8;  // first 16-row tile of the CTA's 128 rows
-  const int m0 = blockIdx.y * BN;
+  // token rows of this CTA: [row0 + m0, row0 + min(m0 + BN, rows)) of x / out
+  int m0 = blockIdx.y * BN, row0 = 0, rows = p.M, expert = 0;
+  if (p.offsets) {
+    // Device-side tile schedule of a grouped launch: experts in order, each
+    // with ceil(count / BN) token tiles; CTA y takes tile y of that list (the
+    // grid holds an upper bound of ceil(T / BN) + E tiles, the rest exit).
+    // Offsets outside [0, T] or decreasing make an expert empty and set bit
+    // 256 of the error word.
+    int* sched = (int*)(bars + 2 * ST + 2 * SA + 6);  // 16 bytes before the scale table
+    if (warp == 0) {
+      const int target = (int)blockIdx.y;
+      int base = 0, found = 0;
+      for (int c0 = 0; c0 < p.E && !found; c0 += 32) {
+        const int ee = c0 + lane;
+        int cnt = 0, a = 0;
+        if (ee < p.E) {
+          const int64_t a64 = __ldg(p.offsets + ee), b64 = __ldg(p.offsets + ee + 1);
+          if (a64 >= 0 && a64 <= b64 && b64 <= p.T) {
+            a = (int)a64;
+            cnt = (int)(b64 - a64);
+          } else if (blockIdx.x == 0 && blockIdx.y == 0) {
+            atomicOr(&g_wq_device_error, 256u);
+          }
+        }
+        const int nt = (cnt + BN - 1) / BN;
+        int incl = nt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        const bool mine = nt > 0 && target >= base + incl - nt && target < base + incl;
+        const unsigned bal = __ballot_sync(0xffffffffu, mine);
+        if (mine) {
+          sched[0] = ee;
+          sched[1] = a;
+          sched[2] = (target - (base + incl - nt)) * BN;
+          sched[3] = cnt;
+        }
+        found = bal != 0;
+        base += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (!found && lane == 0) sched[0] = -1;
+    }
+    __syncthreads();
+    if (sched[0] < 0) return;  // past the end of the schedule: nothing to do
+    expert = sched[0];
+    row0 = sched[1];
+    m0 = sched[2];
+    rows = sched[3];
+  }
+  // this expert's (or the only) scales, aux and bias
+  const uint8_t* scales_p = (const uint8_t*)p.scales + (int64_t)expert * p.scale_stride;
+  const uint8_t* aux_p = (const uint8_t*)p.aux + (int64_t)expert * p.aux_stride;
+  const uint16_t* bias_p = p.bias ? p.bias + (int64_t)expert * p.N : nullptr;
   // K split: the S CTAs of a cluster (1, 1, S) share a tile and take
   // consecutive ranges of KT K steps each (whole scale groups); their fp32
   // partial tiles are summed through distributed shared memory at the end
@@ -365,8 +443,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
           uint8_t* st = smem + s * kTstage;
           mbar_expect_tx(tfull_bar(s), kXbytes + kWpk);
-          tma_load_2d(smem_u32(st), &tmX, (kt0 + kt) * KS, m0, tfull_bar(s));
-          tma_load_2d(smem_u32(st + kXbytes), &tmW, (kt0 + kt) * kWbox, tile0, tfull_bar(s));
+          tma_load_2d(smem_u32(st), &tmX, (kt0 + kt) * KS, row0 + m0, tfull_bar(s));
+          tma_load_2d(smem_u32(st + kXbytes), &tmW, (kt0 + kt) * kWbox, expert * ntiles + tile0,
+                      tfull_bar(s));
         }
         if constexpr (kHasSide) {
           const uint32_t sd = smem_u32(sring + s * kSide);
@@ -376,18 +455,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             if constexpr (FMT == NVFP4) {
               // 4 blocks of 16 K x 16 rows = 64 bytes per row tile
               cp_async16(sd + rt * 64 + c * 16,
-                         (const uint8_t*)p.scales + (tile * (p.K >> 4) + (kt0 + kt) * 4 + c) * 16);
+                         scales_p + (tile * (p.K >> 4) + (kt0 + kt) * 4 + c) * 16);
             } else if constexpr (FMT == MXFP4) {
               // 2 blocks of 32 K x 16 rows = 32 bytes per row tile
               if (c < 2)
                 cp_async16(sd + rt * 32 + c * 16,
-                           (const uint8_t*)p.scales + (tile * (p.K >> 5) + (kt0 + kt) * 2 + c) * 16);
+                           scales_p + (tile * (p.K >> 5) + (kt0 + kt) * 2 + c) * 16);
             } else {
               // the (one or two) groups of this K step: 8 bytes each
               const int64_t g0 = ((int64_t)(kt0 + kt) * 64) / p.G;
               const int ng = p.G == 32 ? 2 : 1;
               if (c < ng)
-                cp_async8(sd + rt * 16 + c * 8, (const uint8_t*)p.aux + (tile * groups + g0 + c) * 8);
+                cp_async8(sd + rt * 16 + c * 8, aux_p + (tile * groups + g0 + c) * 8);
             }
           }
           cp_async_arrive(tfull_bar(s));
@@ -396,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // before teardown, make sure no copy into this CTA's memory is in flight
       for (int kt = issued - ST < 0 ? 0 : issued - ST; kt < issued; ++kt)
-        mbar_wait(tfull_bar(kt % ST), (uint32_t)(kt / ST) & 1u, abort, 2u);
+        mbar_wait(tfull_bar(kt % ST), (uint32_t)(kt / ST) & 1u, abort, 2u, false);
     } else if (warp == 1 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       // instruction descriptor: D f32 (A8: s32), A and B bf16 (A8: signed
@@ -449,7 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) {  // wait for this thread's own MMAs before the memory goes away
         umma_commit(drain_bar);
-        mbar_wait(drain_bar, 0u, abort, 16u);
+        mbar_wait(drain_bar, 0u, abort, 16u, false);
       }
     }
   } else if (warp < 8) {
@@ -462,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t H[4] = {0, 0, 0, 0}, L[4] = {0, 0, 0, 0};
     uint32_t H2[4] = {0, 0, 0, 0}, L2[4] = {0, 0, 0, 0};
     if constexpr (FMT == CB4) {
-      const float* cen = (const float*)p.aux;
+      const float* cen = (const float*)aux_p;
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const float cv = __ldg(cen + j);
@@ -527,6 +606,21 @@ __global__ void __launch_bounds__(kThreads, 1)
               frag_int8(ch.z, ch.w, b);
             }
             const int j = 4 * blk + tq;
+            st_shared_v4(abase + swz(Rg, j), a[0], a[2], b[0], b[2]);
+            st_shared_v4(abase + swz(Rg8, j), a[1], a[3], b[1], b[3]);
+          }
+        } else if constexpr (FMT == INT3_SYM) {
+          // 384 bytes per row tile and K step: the INT2-ordered low plane
+          // (8 bytes per lane) and the high plane (4 bytes per lane)
+          const uint2 lo = *(const uint2*)(wpk + rt * 384 + lane * 8);
+          const uint32_t hi = *(const uint32_t*)(wpk + rt * 384 + 256 + lane * 4);
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const uint32_t w = c ? lo.y : lo.x;
+            uint32_t a[4], b[4];
+            frag_int3(w, hi, c, 0, 0x43044304u, a);
+            frag_int3(w, hi, c, 1, 0x43044304u, b);
+            const int j = 4 * c + tq;
             st_shared_v4(abase + swz(Rg, j), a[0], a[2], b[0], b[2]);
             st_shared_v4(abase + swz(Rg8, j), a[1], a[3], b[1], b[3]);
           }
@@ -603,8 +697,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_async_smem();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(afull_bar(sa));   // A tile written
-        mbar_arrive(tempty_bar(s));   // packed tile read (already in registers)
+#ifdef WQ_FAULT_TEST
+        if (!(dw == 0 && kt == p.fault_stage))
+#endif
+          mbar_arrive(afull_bar(sa));   // A tile written
+        mbar_arrive(tempty_bar(s));     // packed tile read (already in registers)
       }
     }
   } else {
@@ -619,8 +716,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // per-row factors, requested before the first wait: the group scales of
     // the next two groups ride in registers ahead of the group being folded
     // group scales: bf16 (INT formats) or fp32 (FP8), same packed indexing
-    const uint16_t* srow = (const uint16_t*)p.scales;
-    const uint32_t* srow32 = (const uint32_t*)p.scales;
+    const uint16_t* srow = (const uint16_t*)scales_p;
+    const uint32_t* srow32 = (const uint32_t*)scales_p;
     int64_t sidx = 0;
     if (kInt && nvalid) {
       const int r16 = (int)(n & 15);
@@ -635,9 +732,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t sc0 = group_scale(0), sc1 = group_scale(1);
     float post = 1.f, bval = 0.f;
     if (nvalid) {
-      if constexpr (FMT == CB4) post = bf16_bits_to_f32(__ldg((const uint16_t*)p.scales + n));
-      if constexpr (FMT == NVFP4) post = __ldg((const float*)p.aux) * 128.f;  // 2^7 of frag_nvfp4
-      if (p.bias) bval = bf16_bits_to_f32(__ldg(p.bias + n));
+      if constexpr (FMT == CB4) post = bf16_bits_to_f32(__ldg((const uint16_t*)scales_p + n));
+      if constexpr (FMT == NVFP4) post = __ldg((const float*)aux_p) * 128.f;  // 2^7 of frag_nvfp4
+      if (bias_p) bval = bf16_bits_to_f32(__ldg(bias_p + n));
     }
     float acc[kHalf];
 #pragma unroll
@@ -683,8 +780,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int j = 0; j < kHalf; ++j) {
           const int m = m0 + hcol + j;
-          if (m < p.M)
-            p.out[(int64_t)m * p.N + n] =
+          if (m < rows)
+            p.out[(int64_t)(row0 + m) * p.N + n] =
                 (uint16_t)f32_to_bf16_bits(acc[j] * post * colscale(m) + bval);
         }
       }
@@ -715,8 +812,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           float tot = 0.f;
           for (int src = 0; src < S; ++src) tot += sl[(src * 128 + frow) * CW + c];
           const int m = m0 + split * CW + c;
-          if (m < p.M)
-            p.out[(int64_t)m * p.N + n] =
+          if (m < rows)
+            p.out[(int64_t)(row0 + m) * p.N + n] =
                 (uint16_t)f32_to_bf16_bits(tot * post * colscale(m) + bval);
         }
       }
@@ -758,6 +855,7 @@ cudaError_t launch_bn(const LinearArgs& a) {
   constexpr int KS = A8 ? 128 : 64;  // K per stage
   constexpr uint32_t kWpk = ((FMT == INT8_SYM || FMT == FP8_E4M3 || FMT == FP8_E5M2) ? 8192u
                              : FMT == INT2_SYM                                      ? 2048u
+                             : FMT == INT3_SYM                                      ? 3072u
                                                                                     : 4096u) *
                             (A8 ? 2u : 1u);
   // the packed tile of a row tile per stage as one box row of 4- or 8-byte
@@ -781,7 +879,9 @@ cudaError_t launch_bn(const LinearArgs& a) {
   }
   {
     const uint64_t row_bytes = (uint64_t)a.K * 2 * code_bits(FMT);  // bytes per row tile
-    cuuint64_t dims[2] = {(cuuint64_t)(row_bytes / kEsz), (cuuint64_t)(a.N / 16)};
+    // all experts' row tiles, stacked, for a grouped launch
+    cuuint64_t dims[2] = {(cuuint64_t)(row_bytes / kEsz),
+                          (cuuint64_t)(a.N / 16) * (cuuint64_t)(a.offsets ? a.E : 1)};
     cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
     cuuint32_t box[2] = {kWpk / 8u / kEsz, 8u};
     cuuint32_t es[2] = {1u, 1u};
@@ -823,6 +923,14 @@ cudaError_t launch_bn(const LinearArgs& a) {
   p.BN = BN;
   p.stages = ST;
   p.astages = SA;
+#ifdef WQ_FAULT_TEST
+  p.fault_stage = getenv("WQ_FAULT_PREFILL_STAGE") ? atoi(getenv("WQ_FAULT_PREFILL_STAGE")) : -1;
+#endif
+  p.offsets = a.offsets;
+  p.E = a.offsets ? a.E : 1;
+  p.T = (int)a.M;
+  p.scale_stride = a.offsets ? a.scale_stride : 0;
+  p.aux_stride = a.offsets ? a.aux_stride : 0;
   // K split over a cluster of S CTAs only when the tiles fill at most half
   // of the SMs: the distributed-shared-memory reduction (every CTA sends
   // (S-1)/S of a 128 x BN fp32 tile) costs more than a partly empty last wave
@@ -836,7 +944,7 @@ cudaError_t launch_bn(const LinearArgs& a) {
     const int64_t unit = (is_grouped_fmt(FMT) && a.G > KS) ? a.G / KS : 1;
     const int64_t sms = device_sm_count();
     int best_s = 1;
-    if (2 * tiles <= sms) {
+    if (2 * tiles <= sms && !a.offsets) {  // no K split in a grouped launch
       for (int sp = 8; sp >= 2; sp /= 2) {
         if (tiles * sp <= sms && KTall % (sp * unit) == 0 && BN % (4 * sp) == 0 && KTall / sp >= 8) {
           best_s = sp;
@@ -855,7 +963,11 @@ cudaError_t launch_bn(const LinearArgs& a) {
   }
   const bool groups2 = is_grouped_fmt(FMT) && (a.K / a.G) > 1;  // two alternating accumulators
   p.tmem_cols = (uint32_t)(groups2 ? 2 * BN : (BN < 32 ? 32 : BN));
-  dim3 grid((unsigned)((a.N + 127) / 128), (unsigned)((a.M + BN - 1) / BN), (unsigned)p.splits);
+  // grouped: an upper bound on the schedule's token tiles (sum over experts
+  // of ceil(count / BN) <= ceil(T / BN) + E); the CTAs past its end exit
+  const int64_t ytiles = (a.M + BN - 1) / BN + (a.offsets ? a.E : 0);
+  if (ytiles > 65535) return cudaErrorNotSupported;
+  dim3 grid((unsigned)((a.N + 127) / 128), (unsigned)ytiles, (unsigned)p.splits);
   if (p.splits > 1) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
@@ -907,6 +1019,26 @@ cudaError_t launch_prefill(const LinearArgs& a) {
     case FP8_E4M3: return launch_fmt<FP8_E4M3>(a, BN);
     case FP8_E5M2: return launch_fmt<FP8_E5M2>(a, BN);
     case INT2_SYM: return launch_fmt<INT2_SYM>(a, BN);
+    case INT3_SYM: return launch_fmt<INT3_SYM>(a, BN);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_prefill_grouped(const LinearArgs& a) {
+  // token tile from the mean rows per expert (the counts are on the device)
+  const int64_t avg = (a.M + a.E - 1) / (a.E > 0 ? a.E : 1);
+  const int BN = avg <= 32 ? 32 : avg <= 64 ? 64 : avg <= 128 ? 128 : 256;
+  switch (a.fmt) {
+    case INT4_SYM: return launch_fmt<INT4_SYM>(a, BN);
+    case INT4_ASYM: return launch_fmt<INT4_ASYM>(a, BN);
+    case INT8_SYM: return launch_fmt<INT8_SYM>(a, BN);
+    case CB4: return launch_fmt<CB4>(a, BN);
+    case NVFP4: return launch_fmt<NVFP4>(a, BN);
+    case MXFP4: return launch_fmt<MXFP4>(a, BN);
+    case FP8_E4M3: return launch_fmt<FP8_E4M3>(a, BN);
+    case FP8_E5M2: return launch_fmt<FP8_E5M2>(a, BN);
+    case INT2_SYM: return launch_fmt<INT2_SYM>(a, BN);
+    case INT3_SYM: return launch_fmt<INT3_SYM>(a, BN);
   }
   return cudaErrorInvalidValue;
 }

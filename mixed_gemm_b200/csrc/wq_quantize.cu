@@ -114,6 +114,21 @@ __global__ void quant_sym_kernel(int bits, int64_t N, int64_t K, int G,
         }
         codes[n * (K / 4) + (grp * G + i) / 4] = (uint8_t)packed;
       }
+    } else if (bits == 3) {
+      // eight codes = three bytes of the row's bit stream (a group of G
+      // starts on a byte: 3 G / 8 bytes per group)
+      for (int i = 8 * lane; i < G; i += 256) {
+        uint32_t packed = 0;
+        for (int j = 0; j < 8; ++j) {
+          int q = 0;
+          if (s != 0.0) q = max(-qmax, min(qmax, __double2int_rn(__ddiv_rn((double)wg[i + j], s))));
+          packed |= (uint32_t)(q & 7) << (3 * j);
+        }
+        uint8_t* dst = codes + n * (3 * K / 8) + 3 * ((grp * G + i) / 8);
+        dst[0] = (uint8_t)packed;
+        dst[1] = (uint8_t)(packed >> 8);
+        dst[2] = (uint8_t)(packed >> 16);
+      }
     } else if (bits == 4) {
       for (int i = 2 * lane; i < G; i += 64) {
         int q0 = 0, q1 = 0;
@@ -335,6 +350,7 @@ cudaError_t launch_quantize(int f, int64_t N, int64_t K, int G, const float* w, 
     case INT4_SYM:
     case INT8_SYM:
     case INT2_SYM:
+    case INT3_SYM:
       quant_sym_kernel<<<blocks_for(N * (K / G), kWarps), kWarps * 32, 0, st>>>(
           code_bits(f), N, K, G, w, (uint8_t*)codes, (uint16_t*)scales);
       break;

@@ -115,6 +115,8 @@ def packed_bytes(fmt: str, N: int, K: int, G: int) -> int:
         return N * K // 2 + 2 * N * (K // G)
     if fmt == "int2_sym":
         return N * K // 4 + 2 * N * (K // G)
+    if fmt == "int3_sym":
+        return N * K * 3 // 8 + 2 * N * (K // G)
     if fmt == "int4_asym":
         return N * K // 2 + 2 * N * (K // G) + N * (K // G) // 2
     if fmt == "int8_sym":
@@ -132,3 +134,57 @@ def packed_bytes(fmt: str, N: int, K: int, G: int) -> int:
 
 def flops(M: int, N: int, K: int) -> int:
     return 2 * M * N * K
+
+
+@dataclass(frozen=True)
+class MoEWorkload:
+    """A mixture-of-experts layer: E experts of one format, each [N, K];
+    `tokens` tokens routed to `topk` experts each, so tokens * topk rows of x
+    sorted by expert, with skewed (Zipf-like) per-expert counts."""
+    name: str
+    fmt: str
+    E: int
+    N: int
+    K: int
+    tokens: int
+    topk: int
+    group_size: int
+    seed: int
+    note: str = ""
+
+    @property
+    def rows(self) -> int:
+        return self.tokens * self.topk
+
+
+MOE_DECODE = MoEWorkload("moe_int4_decode", "int4_sym", E=64, N=2048, K=2048, tokens=64, topk=8,
+                         group_size=128, seed=7,
+                         note="decode-like routing: 64 tokens x top-8 over 64 INT4 experts")
+MOE_PREFILL = MoEWorkload("moe_int4_prefill", "int4_sym", E=64, N=2048, K=2048, tokens=4096,
+                          topk=8, group_size=128, seed=8,
+                          note="prefill-like routing: 4096 tokens x top-8 over 64 INT4 experts")
+MOE = {w.name: w for w in (MOE_DECODE, MOE_PREFILL)}
+
+
+def moe_counts(w: MoEWorkload) -> np.ndarray:
+    """Rows per expert (sum = tokens * topk): a multinomial draw with Zipf(1.1)
+    expert weights in a seeded random order."""
+    rng = np.random.default_rng(w.seed)
+    p = 1.0 / np.arange(1, w.E + 1) ** 1.1
+    p = p[rng.permutation(w.E)]
+    return rng.multinomial(w.rows, p / p.sum()).astype(np.int64)
+
+
+def moe_weight(w: MoEWorkload, e: int) -> np.ndarray:
+    """Expert e's dense fp32 weight [N, K] ~ N(0, 0.02^2)."""
+    return weight(w.seed * 1000 + e, w.N, w.K, sigma=0.02)
+
+
+def moe_x(w: MoEWorkload) -> np.ndarray:
+    return activations(w.seed, w.rows, w.K)
+
+
+def moe_bytes(w: MoEWorkload, counts) -> int:
+    """Algorithmic bytes: the packed weights of every expert with rows, X, Y."""
+    used = int(np.count_nonzero(np.asarray(counts)))
+    return used * packed_bytes(w.fmt, w.N, w.K, w.group_size) + 2 * w.rows * (w.K + w.N)

@@ -37,7 +37,7 @@ def test_status_strings():
 
 @pytest.mark.parametrize("fmt,G", [("int4_sym", 64), ("int4_asym", 128), ("int8_sym", 256),
                                    ("cb4", 0), ("nvfp4", 16), ("mxfp4", 32), ("fp8_e4m3", 128),
-                                   ("fp8_e5m2", 64), ("int2_sym", 32)])
+                                   ("fp8_e5m2", 64), ("int2_sym", 32), ("int3_sym", 64)])
 def test_sizes(fmt, G):
     import synth.workloads as W
     N, K = 4096, 4096
@@ -50,7 +50,7 @@ def test_sizes(fmt, G):
 
 
 BAD_SHAPES = [
-    dict(fmt=9), dict(fmt=-1), dict(fmt="int2_sym", G=16), dict(N=0), dict(K=0), dict(N=24), dict(K=96), dict(G=48),
+    dict(fmt=10), dict(fmt=-1), dict(fmt="int2_sym", G=16), dict(fmt="int3_sym", G=16), dict(N=0), dict(K=0), dict(N=24), dict(K=96), dict(G=48),
     dict(G=512), dict(fmt="nvfp4", G=32), dict(fmt="mxfp4", G=16), dict(fmt="fp8_e4m3", G=16),
     dict(fmt="fp8_e5m2", G=0), dict(M=-1),
 ]

@@ -17,7 +17,8 @@ pytestmark = pytest.mark.gpu
 FMT_G = [("int4_sym", 32), ("int4_sym", 64), ("int4_sym", 128), ("int4_sym", 256),
          ("int4_asym", 32), ("int4_asym", 128), ("int8_sym", 32), ("int8_sym", 256),
          ("cb4", 0), ("nvfp4", 16), ("mxfp4", 32), ("fp8_e4m3", 32), ("fp8_e4m3", 256),
-         ("fp8_e5m2", 64), ("int2_sym", 32), ("int2_sym", 128)]
+         ("fp8_e5m2", 64), ("int2_sym", 32), ("int2_sym", 128), ("int3_sym", 32),
+         ("int3_sym", 128)]
 IDS = [f"{f}-g{g}" for f, g in FMT_G]
 
 
@@ -106,7 +107,7 @@ def _int_case(fmt, N, K, G, rng):
 
 @pytest.mark.parametrize("fmt,G", [("int4_sym", 64), ("int4_asym", 32), ("int8_sym", 128),
                                    ("cb4", 0), ("nvfp4", 16), ("mxfp4", 32), ("fp8_e4m3", 64),
-                                   ("fp8_e5m2", 32), ("int2_sym", 64)])
+                                   ("fp8_e5m2", 32), ("int2_sym", 64), ("int3_sym", 64)])
 @pytest.mark.parametrize("M", [1, 5, 16, 40, 200])
 def test_linear_integer_bit_exact(wq, orc, fmt, G, M):
     """Integer activations and unit scales: every partial sum is exact in
@@ -173,7 +174,7 @@ EDGE = [
 
 
 @pytest.mark.parametrize("fmt", ["int4_sym", "int4_asym", "int8_sym", "cb4", "nvfp4", "mxfp4",
-                                 "fp8_e4m3", "fp8_e5m2", "int2_sym"])
+                                 "fp8_e4m3", "fp8_e5m2", "int2_sym", "int3_sym"])
 @pytest.mark.parametrize("case", EDGE, ids=["16x64", "48x192", "32x16384", "19008x192"])
 def test_linear_edge_shapes(wq, orc, fmt, case):
     N, K, G, Ms = case
