@@ -218,11 +218,15 @@ int wq_linear_grouped(const void* x, const void* const* packed_w, const void* co
  *             an expert whose offsets leave [0, T] or decrease is skipped and
  *             sets bit 256 of wq_device_error; rows no expert owns are not
  *             written
- * The tcgen05 kernel builds its tile schedule on the device: experts in
- * order, ceil(count / BN) token tiles each (BN from the mean rows per
- * expert); the grid holds ceil(T / BN) + E token tiles per 128 output rows
- * and the tiles past the schedule's end exit at once.  A bound above the
- * grid limit (65535) returns WQ_ERR_UNSUPPORTED.  Asynchronous.
+ * The kernel builds its tile schedule on the device: experts in order,
+ * ceil(count / C) token chunks each.  With at most 16 rows per expert on
+ * average (decode-like routing) the decode kernel runs it (C = 8 or 16 rows,
+ * weights streamed once per chunk); otherwise the tcgen05 kernel (C = its
+ * token tile BN, from the mean rows per expert).  The grid holds
+ * ceil(T / C) + E chunks per column of output tiles and the chunks past the
+ * schedule's end exit at once.  A bound above the grid limit (65535)
+ * returns WQ_ERR_UNSUPPORTED.  Asynchronous; the offsets are read after the
+ * previous kernel on `stream` has completed.
  * Source: auto-round-lib README section 2 (moe_gemm(activations, weights,
  * num_tokens_per_expert, ...): quantized experts, per-expert token counts);
  * Petit README "Features" (fused MoE kernels). */
@@ -274,7 +278,9 @@ int wq_linear_swiglu_static(const void* x2, const void* packed_w, const void* sc
  * This is a different computation from wq_linear (the activations are
  * quantized), with its own reference; the group sums are exact integers and
  * the scaling is fp32.
- *   x, packed_w, scales, bias, out   as wq_linear (format WQ_INT8_SYM only)
+ *   x, packed_w, scales, bias, out   as wq_linear (formats WQ_INT8_SYM, and
+ *                                    WQ_INT4_SYM whose codes are used as INT8:
+ *                                    W4A8)
  *   workspace   device scratch of at least wq_linear_a8_workspace_size(M, K)
  *               bytes, 16-byte aligned, overlapping no other buffer: the
  *               INT8 codes [M, K] at offset 0 and the fp32 scales [M] at the

@@ -329,7 +329,12 @@ int wq_linear_grouped_dev(const void* x, const void* pw, const void* scales, con
   a.E = (int)E;
   a.scale_stride = (int64_t)sb;
   a.aux_stride = (int64_t)ab;
-  const cudaError_t e = launch_prefill_grouped(a);
+  // decode-like routing (at most 16 rows per expert on average): the decode
+  // kernel over (expert, chunk of 8 or 16 rows) tiles; otherwise, or for a K
+  // too long for its staged slice, the tcgen05 kernel's grouped mode
+  cudaError_t e = cudaErrorNotSupported;
+  if ((T + E - 1) / E <= 16) e = launch_decode(a);
+  if (e == cudaErrorNotSupported) e = launch_prefill_grouped(a);
   return e == cudaErrorNotSupported ? WQ_ERR_UNSUPPORTED : cuda_status(e);
 }
 
@@ -419,7 +424,7 @@ int wq_linear_a8(const void* x, const void* pw, const void* scales, const void* 
                  void* out, void* stream) {
   int st = check_linear(x, K, pw, scales, nullptr, bias, M, N, K, f, G, out);
   if (st) return st;
-  if (f != INT8_SYM || K % 128) return WQ_ERR_UNSUPPORTED;
+  if ((f != INT8_SYM && f != INT4_SYM) || K % 128) return WQ_ERR_UNSUPPORTED;
   size_t need = 0;
   if ((st = wq_linear_a8_workspace_size(M, K, &need)) != WQ_OK) return st;
   if (M == 0) return WQ_OK;

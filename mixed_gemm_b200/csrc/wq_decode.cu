@@ -76,14 +76,34 @@ cudaError_t launch_decode(const LinearArgs& a) {
   p.aux = a.aux;
   p.bias = (const uint16_t*)a.bias;
   p.out = (uint16_t*)a.out;
-  p.M = (int)a.M;
   p.N = (int)a.N;
   p.K = (int)a.K;
   p.G = a.G;
-  const int nt = a.M <= 8 ? 1 : 2;
+  // a grouped launch takes token chunks of up to 8 (mean rows per expert
+  // <= 8) or 16 per CTA; Mc is the rows a CTA stages
+  const int64_t Mc = a.offsets ? ((a.M + a.E - 1) / a.E <= 8 ? 8 : 16) : a.M;
+  p.M = (int)Mc;
+  p.offsets = a.offsets;
+  p.E = a.offsets ? a.E : 1;
+  p.T = (int)a.M;
+  size_t wbytes = 0, sbytes = 0, abytes = 0;
+  wq_packed_sizes(a.fmt, a.N, a.K, a.G, &wbytes, &sbytes, &abytes);
+  p.w_stride = a.offsets ? (int64_t)wbytes : 0;
+  p.scale_stride = a.offsets ? a.scale_stride : 0;
+  p.aux_stride = a.offsets ? a.aux_stride : 0;
+  const int nt = Mc <= 8 ? 1 : 2;
   const int64_t tiles = a.N / 16;
-  // more row tiles per CTA when there are more tokens: the staged X slice is
-  // then reused across more weight rows
+  // Launch shape, from a sweep of row tiles per CTA, warps per CTA, cluster
+  // size and ring depth over the 4096^2 INT4, 3072^2 codebook, 8192^2 FP8
+  // and 28672 x 8192 NVFP4 layers at M = 1..16 (graph replay, weights past
+  // L2): eight warps per CTA, two row tiles per CTA, K split over a cluster
+  // of at least two CTAs and enough of them to keep each CTA's staged
+  // activation slice near 64 KB (one 8-warp CTA per SM would otherwise be
+  // all that fits at M = 16, K = 8192), and a ring of eight blocks per row
+  // tile at M <= 8 (more weight bytes in flight; at M > 8 the second token
+  // tile's accumulators make the deeper ring spill).  Against the previous
+  // heuristic (about four 4-warp CTAs per SM) this measured 5-38% faster on
+  // every shape of the sweep.
   int rt = (tiles % 2 == 0) ? 2 : 1;
 #ifdef WQ_TUNING
   if (const char* e = getenv("WQ_DECODE_RT")) rt = atoi(e);
@@ -91,32 +111,21 @@ cudaError_t launch_decode(const LinearArgs& a) {
   const int64_t rowgroups = tiles / rt;
   const int kb = block_k(a.fmt);
   const int64_t nblk = a.K / kb;
-  // split K over a cluster: about four 4-warp CTAs per SM, and a staged X
-  // slice of at most 96 KB
-  const int64_t target = 4LL * device_sm_count();
-  int64_t cs = (target + rowgroups - 1) / rowgroups;
-  // eight warps per CTA when the row groups alone fill the grid (large
-  // layers, no K split across CTAs): a longer K range per CTA is then split
-  // over more warps (measured on a 28672 x 8192 layer at M = 8: 59 us
-  // against 84 with four warps, whose X slice left one CTA per SM); four
-  // otherwise (4096 x 4096: 5.9 us against 7.4 with eight)
-  int kw = rowgroups >= target ? 8 : 4;
+  int kw = nblk >= 16 ? 8 : 4;  // short K: fewer warps, each with some blocks
 #ifdef WQ_TUNING
   if (const char* e = getenv("WQ_DECODE_KW")) kw = atoi(e) == 8 ? 8 : 4;
 #endif
-  const int64_t x_bytes_all = a.M * a.K * 2;
-  const int64_t cs_x = (x_bytes_all + 98303) / 98304;
-  if (nt == 2 && cs > 4) cs = 4;  // two token tiles: fewer, longer K slices
-  if (cs < cs_x) cs = cs_x;
+  const int64_t x_bytes_all = Mc * a.K * 2 * (a.swiglu ? 2 : 1);
+  int64_t cs = (x_bytes_all + 65535) / 65536;
+  if (cs < 2) cs = 2;
   if (cs > 8) cs = 8;
   if (cs > nblk / kw) cs = nblk / kw;  // keep every warp busy
   if (cs < 1) cs = 1;
 #ifdef WQ_TUNING
   if (const char* e = getenv("WQ_DECODE_CS")) cs = atoi(e);
 #endif
-  // weight ring depth per row tile: 4, or 8 when that holds a warp's whole
-  // K slice (everything then requested before the dependency wait)
-  int d = 4;
+  // weight ring depth per row tile (two instantiated: 4 and 8)
+  int d = (nt == 1 && rt <= 2) ? 8 : 4;
 #ifdef WQ_TUNING
   if (const char* e = getenv("WQ_DECODE_D")) d = atoi(e) == 8 ? 8 : 4;
 #endif
@@ -124,10 +133,10 @@ cudaError_t launch_decode(const LinearArgs& a) {
   const int64_t stride = ((max_blocks * kb * 2 + 127) / 128) * 128 + 64;
   // K too large for the staged activation slice (the SwiGLU input stages up
   // and gate): nothing launched, the caller takes the prefill path
-  if (stride * a.M * (a.swiglu ? 2 : 1) > 200 * 1024) return cudaErrorNotSupported;
+  if (stride * Mc * (a.swiglu ? 2 : 1) > 200 * 1024) return cudaErrorNotSupported;
   p.cs = (int)cs;
   p.xs_stride = (int)stride;
-  p.xs_bytes = (int)(stride * a.M);
+  p.xs_bytes = (int)(stride * Mc);
   // staged side data per row tile: a K range of max_blocks*kb may touch one
   // more group than it spans
   p.gshift = 0;
@@ -152,8 +161,13 @@ cudaError_t launch_decode(const LinearArgs& a) {
   if (region < warp_partials) region = warp_partials;
   p.red_off = (int)((region + 15) & ~15LL);
   p.bar_off = (int)(p.red_off + cs * rt * nt * 4 * 32 * 4);
-  if (p.bar_off + 16 > 227 * 1024) return cudaErrorNotSupported;
+  // the X-slice barrier (8 bytes) and, grouped, the schedule entry after it
+  if (p.bar_off + 32 > 227 * 1024) return cudaErrorNotSupported;
   const int grid = (int)(rowgroups * cs);
+  // grouped: an upper bound on the schedule's chunks (ceil(T / Mc) + E)
+  const int64_t ytiles = a.offsets ? (a.M + Mc - 1) / Mc + a.E : 1;
+  if (ytiles > 65535) return cudaErrorNotSupported;
+  p.ytiles = (int)ytiles;
   unsigned* err = nullptr;
   cudaError_t e = decode_error_word(&err);
   if (e != cudaSuccess) return e;

@@ -31,6 +31,14 @@ struct DecodeParams {
   int bar_off;    // offset of the mbarrier the X-slice bulk copies complete on
   int swiglu;     // x rows are [up | gate] (2K values); the gate slice is
                   // staged at xs_bytes past the up slice
+  // grouped (mixture-of-experts) launch: device row offsets [E + 1] (rows of
+  // x sorted by expert, T rows); the y index of a CTA is a tile of the
+  // device-side schedule (experts in order, ceil(count / (8 NT)) token
+  // chunks each); expert e's packed weight, scales and aux lie e * *_stride
+  // bytes after expert 0's, its bias e * N values.  NULL: one linear.
+  const int64_t* offsets;
+  int E, T, ytiles;
+  int64_t w_stride, scale_stride, aux_stride;
 #ifdef WQ_FAULT_TEST
   int fault_skip_x;  // test build only (see the activation-slice stage)
 #endif
@@ -185,6 +193,69 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, tq = lane & 3;
   const int cs = p.cs;
+  // this call's (or, grouped, this schedule tile's) rows and buffers
+  int M = p.M;
+  const uint16_t* xg = p.x;
+  uint16_t* outg = p.out;
+  const uint4* wg = p.w;
+  const uint8_t* scales_g = (const uint8_t*)p.scales;
+  const uint8_t* aux_g = (const uint8_t*)p.aux;
+  const uint16_t* bias_g = p.bias;
+  if (p.offsets) {
+    // The routing offsets may be the previous kernel's output: wait first
+    // (no weight prefetch ahead of the dependency in this mode).  Warp 0
+    // finds this CTA's (expert, token chunk) with a warp prefix sum over
+    // the experts' chunk counts; invalid offsets make an expert empty.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    int* sched = (int*)(smem + p.bar_off + 16);
+    if (warp == 0) {
+      const int target = (int)blockIdx.y;
+      int base = 0, found = 0;
+      for (int c0 = 0; c0 < p.E && !found; c0 += 32) {
+        const int ee = c0 + lane;
+        int cnt = 0, a = 0;
+        if (ee < p.E) {
+          const int64_t a64 = p.offsets[ee], b64 = p.offsets[ee + 1];
+          if (a64 >= 0 && a64 <= b64 && b64 <= p.T) {
+            a = (int)a64;
+            cnt = (int)(b64 - a64);
+          } else if (blockIdx.x == 0 && blockIdx.y == 0) {
+            atomicOr(p.err, 256u);
+          }
+        }
+        const int nt = (cnt + 8 * NT - 1) / (8 * NT);
+        int incl = nt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        const bool mine = nt > 0 && target >= base + incl - nt && target < base + incl;
+        const unsigned bal = __ballot_sync(0xffffffffu, mine);
+        if (mine) {
+          sched[0] = ee;
+          sched[1] = a + (target - (base + incl - nt)) * 8 * NT;
+          const int left = cnt - (target - (base + incl - nt)) * 8 * NT;
+          sched[2] = left < 8 * NT ? left : 8 * NT;
+        }
+        found = bal != 0;
+        base += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (!found && lane == 0) sched[0] = -1;
+    }
+    __syncthreads();
+    if (sched[0] < 0) return;  // the whole cluster shares blockIdx.y: all return
+    const int e = sched[0];
+    M = sched[2];
+    const int64_t xrow_el = p.swiglu ? 2 * (int64_t)p.K : (int64_t)p.K;
+    xg = p.x + (int64_t)sched[1] * xrow_el;
+    outg = p.out + (int64_t)sched[1] * p.N;
+    wg = p.w + (int64_t)e * (p.w_stride / 16);
+    scales_g += (int64_t)e * p.scale_stride;
+    if (aux_g) aux_g += (int64_t)e * p.aux_stride;
+    if (bias_g) bias_g += (int64_t)e * p.N;
+    __syncthreads();  // sched read by every thread before the barrier memory is reused
+  }
   // cluster (cs, 1, 1) over a grid of rowgroups * cs blocks: the cluster
   // index is the row group, the rank in the cluster the K slice
   int rank = 0, rgroup = (int)blockIdx.x;
@@ -225,7 +296,7 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
       // scales: SB bytes per (tile, group) -> SB / 16 chunks of 16 bytes
 #pragma unroll
       for (int r = 0; r < RT; ++r) {
-        const uint8_t* src = (const uint8_t*)p.scales + ((int64_t)(tile0 + r) * groups + g_begin) * SB;
+        const uint8_t* src = scales_g + ((int64_t)(tile0 + r) * groups + g_begin) * SB;
         for (int i = threadIdx.x; i < ng * (SB / 16); i += KW * 32)
           cp_async16(side + (r * p.side_rows) * SB + i * 16, src + i * 16);
       }
@@ -233,7 +304,7 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
         const uint32_t zs = side + RT * p.side_rows * 32;
 #pragma unroll
         for (int r = 0; r < RT; ++r) {
-          const uint8_t* src = (const uint8_t*)p.aux + ((int64_t)(tile0 + r) * groups + g_begin) * 8;
+          const uint8_t* src = aux_g + ((int64_t)(tile0 + r) * groups + g_begin) * 8;
           for (int i = threadIdx.x; i < ng; i += KW * 32)
             cp_async8(zs + (r * p.side_rows + i) * 8, src + i * 8);
         }
@@ -245,7 +316,7 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
       const int nbk = ((ce - cb) * KB) >> LB;
 #pragma unroll
       for (int r = 0; r < RT; ++r) {
-        const uint8_t* src = (const uint8_t*)p.scales +
+        const uint8_t* src = scales_g +
                              ((int64_t)(tile0 + r) * (K >> LB) + (kbeg >> LB)) * 16;
         for (int i = threadIdx.x; i < nbk; i += KW * 32)
           cp_async16(side + (r * p.side_rows + i) * 16, src + i * 16);
@@ -256,17 +327,17 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   // weight ring: D blocks per row tile in flight
   const uint4* wrow[RT];
 #pragma unroll
-  for (int r = 0; r < RT; ++r) wrow[r] = p.w + (int64_t)(tile0 + r) * nblk * 32 + lane;
+  for (int r = 0; r < RT; ++r) wrow[r] = wg + (int64_t)(tile0 + r) * nblk * 32 + lane;
   // INT2: 256-byte blocks, 8 bytes per lane (the words 0..1 of its uint4)
   // INT3: 384-byte blocks, 8 low-plane bytes and 4 high-plane bytes per lane
   auto ld_block = [&](int r, int blk) -> uint4 {
     if constexpr (FMT == INT3_SYM) {
-      const uint8_t* bp = (const uint8_t*)p.w + ((int64_t)(tile0 + r) * nblk + blk) * 384;
+      const uint8_t* bp = (const uint8_t*)wg + ((int64_t)(tile0 + r) * nblk + blk) * 384;
       const uint2 lo = ld_stream8((const uint2*)(bp + lane * 8));
       const uint32_t hi = ld_stream4((const uint32_t*)(bp + 256 + lane * 4));
       return make_uint4(lo.x, lo.y, hi, 0u);
     } else if constexpr (FMT == INT2_SYM) {
-      const uint2 v = ld_stream8((const uint2*)p.w + ((int64_t)(tile0 + r) * nblk + blk) * 32 + lane);
+      const uint2 v = ld_stream8((const uint2*)wg + ((int64_t)(tile0 + r) * nblk + blk) * 32 + lane);
       return make_uint4(v.x, v.y, 0u, 0u);
     } else {
       return ld_stream(wrow[r] + blk * 32);
@@ -298,12 +369,12 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
 #endif
     const uint32_t xbytes = (uint32_t)((ce - cb) * KB * 2);
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(xbar),
-                 "r"(xbytes * (uint32_t)p.M * (p.swiglu ? 2u : 1u))
+                 "r"(xbytes * (uint32_t)M * (p.swiglu ? 2u : 1u))
                  : "memory");
-    for (int tok = 0; tok < p.M; ++tok) {
-      bulk_g2s(xs + tok * p.xs_stride, p.x + tok * xrow + kbeg, xbytes, xbar);
+    for (int tok = 0; tok < M; ++tok) {
+      bulk_g2s(xs + tok * p.xs_stride, xg + tok * xrow + kbeg, xbytes, xbar);
       if (p.swiglu)
-        bulk_g2s(xs + p.xs_bytes + tok * p.xs_stride, p.x + tok * xrow + K + kbeg, xbytes,
+        bulk_g2s(xs + p.xs_bytes + tok * p.xs_stride, xg + tok * xrow + K + kbeg, xbytes,
                  xbar);
     }
   }
@@ -325,7 +396,7 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   uint32_t H[4] = {0, 0, 0, 0}, L[4] = {0, 0, 0, 0};
   uint32_t H2[4] = {0, 0, 0, 0}, L2[4] = {0, 0, 0, 0};
   if constexpr (FMT == CB4) {
-    const float* cen = (const float*)p.aux;
+    const float* cen = (const float*)aux_g;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       const float c = __ldg(cen + j);
@@ -369,7 +440,7 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   if (p.swiglu) {
     // SwiGLU input: a = bf16(up * silu(gate)), written over the staged up slice
     const int chunks = (ce - cb) * KB / 8;  // 16-byte chunks per token row
-    for (int i = threadIdx.x; i < p.M * chunks; i += KW * 32) {
+    for (int i = threadIdx.x; i < M * chunks; i += KW * 32) {
       const int tok = i / chunks, c = i - tok * chunks;
       const uint32_t ua = xs + (uint32_t)(tok * p.xs_stride + c * 16);
       const uint4 u = lds128(ua), gt = lds128(ua + (uint32_t)p.xs_bytes);
@@ -387,7 +458,7 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int tok = g + 8 * nt;
-        xv[c][nt] = tok < p.M ? lds128(xs + tok * p.xs_stride +
+        xv[c][nt] = tok < M ? lds128(xs + tok * p.xs_stride +
                                        (uint32_t)((kblk - kbeg) + 32 * c + 8 * tq) * 2u)
                               : zero4;
       }
@@ -561,7 +632,7 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   if (rank != 0) return;
 
   float tsc = 1.f;
-  if constexpr (FMT == NVFP4) tsc = __ldg((const float*)p.aux) * 128.f;  // 2^7 of frag_nvfp4
+  if constexpr (FMT == NVFP4) tsc = __ldg((const float*)aux_g) * 128.f;  // 2^7 of frag_nvfp4
   for (int idx = threadIdx.x; idx < NV * 32; idx += KW * 32) {
     float tot = 0.f;
     for (int q = 0; q < cs; ++q) tot += slots[q * NV * 32 + idx];
@@ -570,12 +641,12 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
     const int gg = ln >> 2, tt = ln & 3;
     const int n = (tile0 + r) * 16 + gg + 8 * (i >> 1);
     const int m = nt * 8 + 2 * tt + (i & 1);
-    if (m < p.M && xok) {
+    if (m < M && xok) {
       float fold = tsc;
-      if constexpr (FMT == CB4) fold = bf16_bits_to_f32(__ldg((const uint16_t*)p.scales + n));
+      if constexpr (FMT == CB4) fold = bf16_bits_to_f32(__ldg((const uint16_t*)scales_g + n));
       float y = tot * fold;
-      if (p.bias) y += bf16_bits_to_f32(__ldg(p.bias + n));
-      p.out[(int64_t)m * p.N + n] = (uint16_t)f32_to_bf16_bits(y);
+      if (bias_g) y += bf16_bits_to_f32(__ldg(bias_g + n));
+      outg[(int64_t)m * p.N + n] = (uint16_t)f32_to_bf16_bits(y);
     }
   }
 }
@@ -583,11 +654,11 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
 template <int FMT, int NT, int RT, int KW, int D>
 cudaError_t launch_t(const DecodeParams& p, int grid, cudaStream_t st) {
   auto kern = decode_kernel<FMT, NT, RT, KW, D>;
-  const size_t smem = (size_t)p.bar_off + 16;
+  const size_t smem = (size_t)p.bar_off + 32;
   cudaError_t e = ensure_max_dynamic_smem((const void*)kern, 227 * 1024);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
+  cfg.gridDim = dim3(grid, p.ytiles);
   cfg.blockDim = dim3(KW * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;

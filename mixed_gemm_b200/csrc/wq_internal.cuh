@@ -205,7 +205,8 @@ constexpr size_t kSwigluStaticScratchBytes = 16u << 20;
 cudaError_t launch_prefill(const LinearArgs& a);
 // The same tcgen05 kernel on INT8 operands (kind::i8, s32 group sums): a.x is
 // the INT8 activation codes [M, K], a.aux the per-token fp32 scales [M];
-// INT8_SYM weights, K % 128 == 0 (else cudaErrorNotSupported, nothing launched)
+// INT8_SYM or INT4_SYM weights (the INT4 codes sign-extended to INT8 in the
+// operand tile), K % 128 == 0 (else cudaErrorNotSupported, nothing launched)
 cudaError_t launch_prefill_a8(const LinearArgs& a);
 // One launch over every expert of a grouped linear (a.offsets on the device);
 // cudaErrorNotSupported when the schedule's tile bound exceeds the grid limit

@@ -270,6 +270,15 @@ __device__ __forceinline__ uint32_t lds_u8(uint32_t addr) {
   return v;
 }
 
+// Four offset-binary INT4 codes (v + 8) in nibbles 0, 2, 4, 6 of w (the
+// K order e = 0, 2, 1, 3 of the magic nibble order) -> the four int8 values
+// v in K order: the byte permute restores the order, the XOR makes each
+// nibble the 4-bit two's complement of v, and the multiply copies its sign
+// bit into the high nibble (0x08 * 0x1E = 0xF0 stays inside its byte).
+__device__ __forceinline__ uint32_t s8_of_nibbles(uint32_t w) {
+  const uint32_t t = __byte_perm(w & 0x0F0F0F0Fu, 0u, 0x3120) ^ 0x08080808u;
+  return t | ((t & 0x08080808u) * 0x1Eu);
+}
 __device__ __forceinline__ void st_shared_v2(uint32_t addr, uint32_t a, uint32_t b) {
   asm volatile("st.shared.v2.b32 [%0], {%1,%2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
 }
@@ -292,7 +301,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // A8: INT8 activations x INT8 weight codes (kind::i8, s32 accumulators);
   // a stage covers 128 K (128 bytes of each operand row), else 64 K of bf16
   constexpr int KS = A8 ? 128 : 64;
-  static_assert(!A8 || FMT == INT8_SYM, "the i8 path takes INT8 weight codes");
+  static_assert(!A8 || FMT == INT8_SYM || FMT == INT4_SYM,
+                "the i8 path takes INT8 or INT4 weight codes");
   // packed bytes per stage (8 row tiles x KS)
   constexpr uint32_t kWpk =
       (kByte ? 8192u : FMT == INT2_SYM ? 2048u : FMT == INT3_SYM ? 3072u : 4096u) *
@@ -332,9 +342,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t drain_bar = smem_u32(bars + 2 * ST + 2 * SA + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile0 = blockIdx.x * 8;  // first 16-row tile of the CTA's 128 rows
+  // One linear: the grid is one-dimensional (times the K split) with the
+  // token tile varying fastest, so the CTAs resident at once share a few
+  // column blocks of the weight (each read by up to M / BN CTAs close in
+  // time) and the activation tiles stay in L2.  Grouped: x is the column
+  // block, y the schedule tile.
+  const int mtiles = (p.M + BN - 1) / BN;
+  const int tile0 = (p.offsets ? (int)blockIdx.x : (int)blockIdx.x / mtiles) * 8;
   // token rows of this CTA: [row0 + m0, row0 + min(m0 + BN, rows)) of x / out
-  int m0 = blockIdx.y * BN, row0 = 0, rows = p.M, expert = 0;
+  int m0 = (p.offsets ? 0 : (int)blockIdx.x % mtiles) * BN, row0 = 0, rows = p.M, expert = 0;
   if (p.offsets) {
     // Device-side tile schedule of a grouped launch: experts in order, each
     // with ceil(count / BN) token tiles; CTA y takes tile y of that list (the
@@ -577,7 +593,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int rr = 0; rr < 2; ++rr) {
         const int rt = 2 * dw + rr;
         const int Rg = rt * 16 + g, Rg8 = Rg + 8;
-        if constexpr (A8) {
+        if constexpr (A8 && FMT == INT4_SYM) {
+          // INT4 codes sign-extended into the i8 operand tile: two 512-byte
+          // blocks of 64 K per row tile; word 2c + s of a lane holds rows g
+          // (even nibbles) and g + 8 (odd nibbles) at K 64 blk + 32 c + 8 tq
+          // + 4 s + e, nibble 4 (e & 1) + 2 (e >> 1) + hr
+#pragma unroll
+          for (int blk = 0; blk < 2; ++blk) {
+            const uint4 ch = *(const uint4*)(wpk + rt * 1024 + blk * 512 + lane * 16);
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const uint32_t w0 = c ? ch.z : ch.x, w1 = c ? ch.w : ch.y;
+              const int j = 4 * blk + 2 * c + (tq >> 1);
+              const uint32_t half = (uint32_t)(tq & 1) * 8u;
+              st_shared_v2(abase + swz(Rg, j) + half, s8_of_nibbles(w0), s8_of_nibbles(w1));
+              st_shared_v2(abase + swz(Rg8, j) + half, s8_of_nibbles(w0 >> 4),
+                           s8_of_nibbles(w1 >> 4));
+            }
+          }
+        } else if constexpr (A8) {
           // INT8 codes into the i8 operand tile: four 512-byte blocks of 32 K
           // per row tile; a lane's 16 bytes hold rows g and g + 8 at K
           // 32 blk + 8 tq + (0..3 | 4..7); offset-binary -> two's complement
@@ -966,8 +1000,11 @@ cudaError_t launch_bn(const LinearArgs& a) {
   // grouped: an upper bound on the schedule's token tiles (sum over experts
   // of ceil(count / BN) <= ceil(T / BN) + E); the CTAs past its end exit
   const int64_t ytiles = (a.M + BN - 1) / BN + (a.offsets ? a.E : 0);
-  if (ytiles > 65535) return cudaErrorNotSupported;
-  dim3 grid((unsigned)((a.N + 127) / 128), (unsigned)ytiles, (unsigned)p.splits);
+  if (a.offsets && ytiles > 65535) return cudaErrorNotSupported;
+  const int64_t ncol = (a.N + 127) / 128;
+  if (!a.offsets && ncol * ytiles > 0x7FFFFFFFLL) return cudaErrorNotSupported;
+  dim3 grid = a.offsets ? dim3((unsigned)ncol, (unsigned)ytiles, (unsigned)p.splits)
+                        : dim3((unsigned)(ncol * ytiles), 1u, (unsigned)p.splits);
   if (p.splits > 1) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
@@ -1043,15 +1080,20 @@ cudaError_t launch_prefill_grouped(const LinearArgs& a) {
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_prefill_a8(const LinearArgs& a) {
-  if (a.fmt != INT8_SYM || a.K % 128) return cudaErrorNotSupported;
-  const int BN = a.M <= 32 ? 32 : a.M <= 64 ? 64 : a.M <= 128 ? 128 : 256;
+template <int FMT>
+cudaError_t launch_a8_fmt(const LinearArgs& a, int BN) {
   switch (BN) {
-    case 32: return launch_bn<INT8_SYM, 32, true>(a);
-    case 64: return launch_bn<INT8_SYM, 64, true>(a);
-    case 128: return launch_bn<INT8_SYM, 128, true>(a);
-    default: return launch_bn<INT8_SYM, 256, true>(a);
+    case 32: return launch_bn<FMT, 32, true>(a);
+    case 64: return launch_bn<FMT, 64, true>(a);
+    case 128: return launch_bn<FMT, 128, true>(a);
+    default: return launch_bn<FMT, 256, true>(a);
   }
+}
+
+cudaError_t launch_prefill_a8(const LinearArgs& a) {
+  if ((a.fmt != INT8_SYM && a.fmt != INT4_SYM) || a.K % 128) return cudaErrorNotSupported;
+  const int BN = a.M <= 32 ? 32 : a.M <= 64 ? 64 : a.M <= 128 ? 128 : 256;
+  return a.fmt == INT8_SYM ? launch_a8_fmt<INT8_SYM>(a, BN) : launch_a8_fmt<INT4_SYM>(a, BN);
 }
 
 cudaError_t read_device_error(unsigned* value, bool clear) {

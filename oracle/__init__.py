@@ -268,7 +268,7 @@ class Oracle:
 
     def linear_a8_full(self, codes, scales, N: int, K: int, G: int, x_bits, bias_bits=None):
         """(y bf16 bits, y fp64) of the activation-quantized linear for INT8
-        sym weights, with each group's integer sum taken by numpy's fp64
+        or INT4 sym weights, with each group's integer sum taken by numpy's fp64
         matmul (exact: every partial sum is an integer below 2^53) instead
         of orc_linear_a8's loop, so that full sizes cost seconds.  The codes
         come from orc_quant_act_int8 and the fp64 accumulation over groups
@@ -276,7 +276,14 @@ class Oracle:
         then the bias), so the fp64 result is the same number."""
         xq, sx = self.quant_act_int8(x_bits)
         M = xq.shape[0]
-        wq = np.ascontiguousarray(codes, dtype=np.int8).reshape(N, K)
+        if np.asarray(codes).size * 2 == N * K:      # INT4 sym: two's complement nibbles
+            c = np.ascontiguousarray(codes, dtype=np.uint8).reshape(N, K // 2)
+            nib = np.empty((N, K), dtype=np.int16)
+            nib[:, 0::2] = c & 15
+            nib[:, 1::2] = c >> 4
+            wq = (nib - 16 * (nib > 7)).astype(np.int8)
+        else:
+            wq = np.ascontiguousarray(codes, dtype=np.int8).reshape(N, K)
         sw = bits_to_f32(np.ascontiguousarray(scales, dtype=np.uint16).reshape(N, K // G))
         sw = sw.astype(np.float64)
         sxd = sx.astype(np.float64)

@@ -179,7 +179,7 @@ def test_linear_a8_argument_checks():
     bad workspaces before launching anything (fake, aligned addresses)."""
     base = 1 << 30
     x, w, s, out, ws = base, base * 2, base * 3, base * 4, base * 5
-    f8, f4 = wqm.FORMATS["int8_sym"], wqm.FORMATS["int4_sym"]
+    f8, f4 = wqm.FORMATS["int8_sym"], wqm.FORMATS["int2_sym"]
     M, N, K, G = 64, 256, 1024, 128
     need = wqm.wq_linear_a8_workspace_size(M, K)
     assert need == ((M * K + 255) // 256) * 256 + 4 * M

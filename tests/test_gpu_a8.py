@@ -44,17 +44,19 @@ def test_activation_codes_bit_exact(wq, orc, M, K):
     assert np.array_equal(xq.cpu().numpy(), xq_ref)
 
 
+@pytest.mark.parametrize("fmt", ["int8_sym", "int4_sym"])
 @pytest.mark.parametrize("G", [32, 64, 128, 256])
 @pytest.mark.parametrize("M", [1, 16, 40, 128, 200, 300])
-def test_a8_linear_matches_oracle(wq, orc, G, M):
+def test_a8_linear_matches_oracle(wq, orc, fmt, G, M):
+    """W8A8 and W4A8 (INT4 codes used as INT8) against the oracle."""
     N, K = 272, 1024
-    Wd, (codes, scales, _) = small_case(orc, "int8_sym", N, K, G, seed=71)
-    pw = pack_on_gpu(wq, "int8_sym", N, K, G, codes, scales, None)
+    Wd, (codes, scales, _) = small_case(orc, fmt, N, K, G, seed=71)
+    pw = pack_on_gpu(wq, fmt, N, K, G, codes, scales, None)
     x = synth.activations(72, M, K, channel_count=10, channel_mult=10.0)
     b = synth.bias(71, N) if M % 2 == 0 else None
     y = _run_a8(wq, pw, x, b, M)
-    ref, _ = orc.linear_a8("int8_sym", codes, scales, N, K, G, x, b)
-    check_close(y, ref, f"a8 G={G} M={M}")
+    ref, _ = orc.linear_a8(fmt, codes, scales, N, K, G, x, b)
+    check_close(y, ref, f"a8 {fmt} G={G} M={M}")
 
 
 def test_a8_split_k_cluster(wq, orc):
@@ -70,15 +72,20 @@ def test_a8_split_k_cluster(wq, orc):
     check_close(y, ref, "a8 split-K")
 
 
-def test_a8_integer_case_bit_exact(wq, orc):
+@pytest.mark.parametrize("fmt", ["int8_sym", "int4_sym"])
+def test_a8_integer_case_bit_exact(wq, orc, fmt):
     """Unit weight scales, activations on the INT8 grid with row maximum 127
     (s_x = 1): every output is an exact integer below 2^24, so the GPU result
-    equals the oracle's bit for bit."""
+    equals the oracle's bit for bit (every INT4 code, -8 included)."""
     N, K, G, M = 256, 512, 128, 70
     rng = np.random.default_rng(75)
-    q = rng.integers(-127, 128, size=(N, K)).astype(np.int8)
     scales = np.full((N, K // G), 0x3F80, np.uint16)
-    pw = pack_on_gpu(wq, "int8_sym", N, K, G, q, scales, None)
+    if fmt == "int8_sym":
+        q = rng.integers(-127, 128, size=(N, K)).astype(np.int8)
+    else:
+        v = rng.integers(-8, 8, size=(N, K))
+        q = ((v[:, 0::2] & 15) | ((v[:, 1::2] & 15) << 4)).astype(np.uint8)
+    pw = pack_on_gpu(wq, fmt, N, K, G, q, scales, None)
     xi = rng.integers(-3, 4, size=(M, K))
     xi[:, 5] = 127
     x = synth.f64_to_bf16_bits(xi.astype(np.float64))
@@ -102,16 +109,16 @@ def test_a8_full_size_prefill_layer(wq, orc):
         check_close(y, ref, f"a8 full size M={M}")
 
 
-def test_a8_refuses_int4_and_short_workspace(wq, orc):
+def test_a8_refuses_other_formats(wq, orc):
     N, K, G, M = 64, 512, 64, 20
-    Wd, (codes, scales, _) = small_case(orc, "int4_sym", N, K, G, seed=76)
-    pw = pack_on_gpu(wq, "int4_sym", N, K, G, codes, scales, None)
+    Wd, (codes, scales, _) = small_case(orc, "int2_sym", N, K, G, seed=76)
+    pw = pack_on_gpu(wq, "int2_sym", N, K, G, codes, scales, None)
     x = dev_bf16(synth.activations(77, M, K))
     y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     need = wq.wq_linear_a8_workspace_size(M, K)
     ws = torch.empty((need,), dtype=torch.uint8, device="cuda")
     with pytest.raises(wq.WQError) as ei:
-        wq.wq_linear_a8(x, pw.w, pw.scales, None, M, N, K, "int4_sym", G, ws, need, y)
+        wq.wq_linear_a8(x, pw.w, pw.scales, None, M, N, K, "int2_sym", G, ws, need, y)
     assert ei.value.status == wq.WQ_ERR_UNSUPPORTED
 
 

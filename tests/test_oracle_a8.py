@@ -82,3 +82,14 @@ def test_a8_full_integer_case(orc):
     y, y64 = orc.linear_a8_full(q, scales, N, K, G, x, None)
     ref = (xi @ q.astype(np.int64).T).astype(np.float64)
     assert np.array_equal(y64, ref)
+
+
+def test_a8_full_int4_equals_loop(orc):
+    """The matmul form with INT4 codes (two's complement nibbles) equals the loop."""
+    N, K, M, G = 32, 256, 5, 64
+    W = synth.weight(12, N, K, sigma=0.02)
+    codes, scales, _ = orc.quantize("int4_sym", W, G)
+    x = synth.activations(13, M, K)
+    y, y64 = orc.linear_a8("int4_sym", codes, scales, N, K, G, x, None)
+    yf, yf64 = orc.linear_a8_full(codes, scales, N, K, G, x, None)
+    assert np.array_equal(yf64, y64) and np.array_equal(yf, y)
