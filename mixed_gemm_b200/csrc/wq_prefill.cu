@@ -624,8 +624,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             st_shared_v2(abase + swz(Rg8, j) + half, ch.y ^ 0x80808080u, ch.w ^ 0x80808080u);
           }
         } else if constexpr (kByte) {
+          // (lanes with odd g take the two 8-K chunks in the other order, so
+          // that the eight lanes of each quarter warp store to eight different
+          // 16-byte bank groups of the swizzled tile)
 #pragma unroll
-          for (int blk = 0; blk < 2; ++blk) {
+          for (int bb = 0; bb < 2; ++bb) {
+            const int blk = bb ^ (g & 1);
             const uint4 ch = *(const uint4*)(wpk + rt * 1024 + blk * 512 + lane * 16);
             // exact codes; the group scale is applied by the fold warps
             uint32_t a[4], b[4];
@@ -649,7 +653,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint2 lo = *(const uint2*)(wpk + rt * 384 + lane * 8);
           const uint32_t hi = *(const uint32_t*)(wpk + rt * 384 + 256 + lane * 4);
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
+          for (int cc = 0; cc < 2; ++cc) {
+            const int c = cc ^ (g & 1);  // chunk order by lane, as above
             const uint32_t w = c ? lo.y : lo.x;
             uint32_t a[4], b[4];
             frag_int3(w, hi, c, 0, 0x43044304u, a);
@@ -663,7 +668,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           // both tensor-core steps of it; exact codes, scale in the fold
           const uint2 ch = *(const uint2*)(wpk + rt * 256 + lane * 8);
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
+          for (int cc = 0; cc < 2; ++cc) {
+            const int c = cc ^ (g & 1);  // chunk order by lane, as above
             const uint32_t w = c ? ch.y : ch.x;
             uint32_t a[4], b[4];
             frag_int2(w, 0, 0x43024302u, a);
@@ -675,7 +681,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           const uint4 ch = *(const uint4*)(wpk + rt * 512 + lane * 16);
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
+          for (int cc = 0; cc < 2; ++cc) {
+            const int c = cc ^ (g & 1);  // chunk order by lane, as above
             const uint32_t w0 = c ? ch.z : ch.x, w1 = c ? ch.w : ch.y;
             uint32_t a[4], b[4];
             if constexpr (kInt) {
