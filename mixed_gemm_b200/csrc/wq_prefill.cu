@@ -187,6 +187,22 @@ __device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t a, uint64_t b
       "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// the four K = 16 steps of one 64-K stage (descriptor start addresses +32
+// bytes per step); the first accumulates into D unless `accumulate` is 0
+__device__ __forceinline__ void umma_f16_x4(uint32_t tmem_d, uint64_t a, uint64_t b,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %9, 0;\n\t"
+      "setp.eq.b32 q, %9, %9;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %8, p;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %4, %8, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %6, %8, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %7, %10, %8, q;\n\t}" ::"r"(tmem_d),
+      "l"(a), "l"(b), "l"(a + 2), "l"(b + 2), "l"(a + 4), "l"(b + 4), "l"(a + 6), "r"(idesc),
+      "r"(accumulate), "l"(b + 6)
+      : "memory");
+}
 __device__ __forceinline__ void umma_i8(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
                                         uint32_t accumulate) {
   asm volatile(
@@ -513,6 +529,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint64_t xd = xdesc0 + (uint64_t)((uint32_t)s * (kTstage >> 4));
         const uint64_t ad = adesc0 + (uint64_t)((uint32_t)sa * (kAtile >> 4));
+        if constexpr (!A8 && FMT != CB4) {
+          if (KPG % 4 == 0) {
+            // a stage lies inside one accumulation group: its four MMAs in one
+            // instruction sequence (each tcgen05.mma issue costs ~200 cycles
+            // in this loop; issuing them back to back measured 2-3% faster)
+            if (in_g == 0) {
+              gb = g & 1;
+              d = tmem + (uint32_t)(gb * BN);
+              // the fold of group g-2 must have drained this buffer
+              if (g >= 2 && !mbar_wait(gempty_bar(gb), (uint32_t)((g >> 1) - 1) & 1u, abort, 4u)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            umma_f16_x4(d, ad, xd, idesc, (uint32_t)in_g);
+            in_g += 4;
+            if (in_g == KPG) {
+              umma_commit(gfull_bar(gb));
+              in_g = 0;
+              ++g;
+            }
+            umma_commit(tempty_bar(s));
+            umma_commit(aempty_bar(sa));
+            if (++s == ST) s = 0;
+            if (++sa == SA) { sa = 0; pha ^= 1u; }
+            continue;
+          }
+        }
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           if (in_g == 0) {

@@ -73,6 +73,8 @@ PREFILL = Workload("prefill_int8_g256", "int8_sym", N=8192, K=8192, Ms=(1024, 20
 
 FP8 = Workload("fp8_e4m3_8192", "fp8_e4m3", N=8192, K=8192, Ms=(1, 16, 1024), group_size=128,
                seed=6, note="FP8 E4M3 weight-only, fp32 scale per 128 along K")
+INT3 = Workload("int3_sym_g128_8192", "int3_sym", N=8192, K=8192, Ms=(1, 16, 1024),
+                group_size=128, seed=9, note="INT3 sym g128 (two-plane packed layout)")
 
 # the prefill layer and inputs again, through the activation-quantized linear
 A8 = Workload("a8_int8_g256_8192", "int8_sym", N=8192, K=8192, Ms=(1024, 2048, 4096),
@@ -80,7 +82,7 @@ A8 = Workload("a8_int8_g256_8192", "int8_sym", N=8192, K=8192, Ms=(1024, 2048, 4
               bias_sigma=0.01, act_int8=True,
               note="W8A8: the prefill layer with per-token INT8 activations")
 
-ALL = (PR1, DECODE, CODEBOOK, NVFP4, PREFILL, MXFP4, FP8)
+ALL = (PR1, DECODE, CODEBOOK, NVFP4, PREFILL, MXFP4, FP8, INT3)
 BY_NAME = {w.name: w for w in ALL + (A8,)}
 
 
