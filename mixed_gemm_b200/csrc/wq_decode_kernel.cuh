@@ -363,15 +363,19 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
 #ifdef WQ_FAULT_TEST
   // test build only: block 0 neither arrives on nor copies into its
   // activation-slice barrier, so its bounded wait runs out
-  if (threadIdx.x == 0 && !(p.fault_skip_x && blockIdx.x == 0)) {
+  if (warp == 0 && !(p.fault_skip_x && blockIdx.x == 0)) {
 #else
-  if (threadIdx.x == 0) {
+  if (warp == 0) {
 #endif
+    // lane 0 announces the bytes, then lane t copies token row t (rows
+    // issued in parallel rather than one after another)
     const uint32_t xbytes = (uint32_t)((ce - cb) * KB * 2);
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(xbar),
-                 "r"(xbytes * (uint32_t)M * (p.swiglu ? 2u : 1u))
-                 : "memory");
-    for (int tok = 0; tok < M; ++tok) {
+    if (lane == 0)
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(xbar),
+                   "r"(xbytes * (uint32_t)M * (p.swiglu ? 2u : 1u))
+                   : "memory");
+    __syncwarp();
+    for (int tok = lane; tok < M; tok += 32) {
       bulk_g2s(xs + tok * p.xs_stride, xg + tok * xrow + kbeg, xbytes, xbar);
       if (p.swiglu)
         bulk_g2s(xs + p.xs_bytes + tok * p.xs_stride, xg + tok * xrow + K + kbeg, xbytes,
