@@ -13,13 +13,16 @@
 //                       on global memory;
 //   warps 4..7          convert packed codes to bf16 in registers (the decode
 //                       path's fragment decoders) and store them, in the
-//                       canonical 128-byte-swizzled K-major layout, into a
-//                       stage of a separate ring of A tiles;
+//                       canonical 128-byte-swizzled K-major layout, into the
+//                       A tile that belongs to the same ring slot;
 //   warp 1 (one lane)   issues four tcgen05.mma.kind::f16 (K = 16 each) per
-//                       K step and commits both stages back;
+//                       K step and returns the slot with one commit;
 //   warps 8..15         fold and epilogue.
-// With two rings the TMA latency and the dequant time run side by side: a TMA
-// stage is refilled as soon as its X tile and packed tile have been read.
+// A slot (X tile, packed tile, A tile) is refilled once its MMAs complete:
+// their completion implies the dequant warps read the packed tile before, so
+// one commit per K step frees everything the slot holds.  The MMA issuer is
+// the busiest serial chain of the kernel (each tcgen05 instruction costs it
+// tens of cycles), so it carries as few barrier operations as possible.
 // INT formats keep the tile values exact: the tile holds the integer code (or
 // code minus zero-point), each group of K is accumulated into its own
 // tensor-memory buffer (two buffers alternate; a group boundary may fall
@@ -71,7 +74,7 @@ struct PrefillParams {
   const uint16_t* bias;
   uint16_t* out;
   int M, N, K, G;
-  int BN, stages, astages;
+  int BN, stages;
   int splits;  // K split over a cluster of this many CTAs (1: no cluster)
   uint32_t tmem_cols;
 #ifdef WQ_FAULT_TEST
@@ -337,25 +340,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr bool kHasSide = kSide != 0;
   constexpr int kHalf = BN / 2;  // accumulator columns per fold thread
 
-  // Two rings: TMA stages (X tile, packed tile) and dequantized A tiles.  A
-  // TMA stage is released when the MMAs have read its X tile and the dequant
-  // warps have read its packed tile; an A stage when the MMAs have read it.
-  // The TMA latency and the dequant time then overlap instead of adding up.
+  // One ring of ST slots, each a TMA stage (X tile, packed tile), an A tile
+  // and the side data.  A slot is released by the commit of its MMAs: the
+  // dequant warps have read its packed tile before they signalled its A tile.
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  const int ST = p.stages, SA = p.astages;
+  // ring of ST slots: TMA stage (X tile + packed tile), A tile, side data
+  const int ST = p.stages;
   uint8_t* aring = smem + ST * kTstage;
-  uint8_t* sring = aring + SA * kAtile;  // side data, kSide bytes per TMA stage
+  uint8_t* sring = aring + ST * kAtile;  // side data, kSide bytes per slot
   uint64_t* bars = (uint64_t*)(sring + ST * kSide);
-  uint32_t* tmem_slot = (uint32_t*)(bars + 2 * ST + 2 * SA + 5);
+  uint32_t* tmem_slot = (uint32_t*)(bars + 3 * ST + 5);
   volatile int* abort = (volatile int*)(tmem_slot + 1);
-  auto tfull_bar = [&](int s) { return smem_u32(bars + s); };
-  auto tempty_bar = [&](int s) { return smem_u32(bars + ST + s); };
-  auto afull_bar = [&](int s) { return smem_u32(bars + 2 * ST + s); };
-  auto aempty_bar = [&](int s) { return smem_u32(bars + 2 * ST + SA + s); };
-  auto gfull_bar = [&](int b) { return smem_u32(bars + 2 * ST + 2 * SA + b); };
-  auto gempty_bar = [&](int b) { return smem_u32(bars + 2 * ST + 2 * SA + 2 + b); };
-  const uint32_t drain_bar = smem_u32(bars + 2 * ST + 2 * SA + 4);
+  auto tfull_bar = [&](int s) { return smem_u32(bars + s); };       // TMA data landed
+  auto empty_bar = [&](int s) { return smem_u32(bars + ST + s); };  // slot's MMAs done
+  auto afull_bar = [&](int s) { return smem_u32(bars + 2 * ST + s); };  // A tile written
+  auto gfull_bar = [&](int b) { return smem_u32(bars + 3 * ST + b); };
+  auto gempty_bar = [&](int b) { return smem_u32(bars + 3 * ST + 2 + b); };
+  const uint32_t drain_bar = smem_u32(bars + 3 * ST + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // One linear: the grid is one-dimensional (times the K split) with the
@@ -373,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // grid holds an upper bound of ceil(T / BN) + E tiles, the rest exit).
     // Offsets outside [0, T] or decreasing make an expert empty and set bit
     // 256 of the error word.
-    int* sched = (int*)(bars + 2 * ST + 2 * SA + 6);  // 16 bytes before the scale table
+    int* sched = (int*)(bars + 3 * ST + 6);  // 16 bytes before the scale table
     if (warp == 0) {
       const int target = (int)blockIdx.y;
       int base = 0, found = 0;
@@ -436,11 +438,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
       mbar_init(tfull_bar(s), kHasSide ? 1 + 32 : 1);  // + one cp.async arrival per lane
-      mbar_init(tempty_bar(s), 1 + 4);  // MMA commit + the four dequant warps
-    }
-    for (int s = 0; s < SA; ++s) {
-      mbar_init(afull_bar(s), 4);
-      mbar_init(aempty_bar(s), 1);
+      mbar_init(empty_bar(s), 1);                       // the MMA issuer's commit
+      mbar_init(afull_bar(s), 4);                       // the four dequant warps
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(gfull_bar(b), 1);
@@ -471,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kt = 0; kt < KT; ++kt) {
         const int s = kt % ST;
         const uint32_t ph = (uint32_t)(kt / ST) & 1u;
-        if (kt >= ST && !mbar_wait(tempty_bar(s), ph ^ 1u, abort, 1u)) break;
+        if (kt >= ST && !mbar_wait(empty_bar(s), ph ^ 1u, abort, 1u)) break;
         if (lane == 0) {
           uint8_t* st = smem + s * kTstage;
           mbar_expect_tx(tfull_bar(s), kXbytes + kWpk);
@@ -514,21 +513,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       // 8-bit), both K-major, N = BN, M = 128
       const uint32_t idesc = ((A8 ? 2u : 1u) << 4) | (1u << 7) | (1u << 10) |
                              ((uint32_t)(BN >> 3) << 17) | ((128u >> 4) << 24);
-      // descriptors of slot 0 of each ring; a slot / K step is a plain add to
-      // the start-address field (smem addresses stay below 2^18)
+      // descriptors of slot 0 (X tile, A tile); a slot / K step is a plain
+      // add to the start-address field (smem addresses stay below 2^18)
       const uint64_t xdesc0 = umma_desc_sw128(smem_u32(smem));
       const uint64_t adesc0 = umma_desc_sw128(smem_u32(aring));
       bool ok = true;
-      int s = 0, sa = 0, g = 0, in_g = 0, gb = 0;
-      uint32_t pha = 0, d = tmem;
+      int s = 0, g = 0, in_g = 0, gb = 0;
+      uint32_t ph = 0, d = tmem;
       for (int kt = 0; kt < KT && ok; ++kt) {
         // the dequant warps arrive on afull only after they have seen this
-        // stage's tfull, so afull alone orders the X tile too
-        ok = mbar_wait(afull_bar(sa), pha, abort, 8u);
+        // slot's tfull, so afull alone orders the X tile too
+        ok = mbar_wait(afull_bar(s), ph, abort, 8u);
         if (!ok) break;
         tc_fence_after();
         const uint64_t xd = xdesc0 + (uint64_t)((uint32_t)s * (kTstage >> 4));
-        const uint64_t ad = adesc0 + (uint64_t)((uint32_t)sa * (kAtile >> 4));
+        const uint64_t ad = adesc0 + (uint64_t)((uint32_t)s * (kAtile >> 4));
         if constexpr (!A8 && FMT != CB4) {
           if (KPG % 4 == 0) {
             // a stage lies inside one accumulation group: its four MMAs in one
@@ -551,10 +550,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               in_g = 0;
               ++g;
             }
-            umma_commit(tempty_bar(s));
-            umma_commit(aempty_bar(sa));
-            if (++s == ST) s = 0;
-            if (++sa == SA) { sa = 0; pha ^= 1u; }
+            umma_commit(empty_bar(s));
+            if (++s == ST) { s = 0; ph ^= 1u; }
             continue;
           }
         }
@@ -582,10 +579,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++g;
           }
         }
-        umma_commit(tempty_bar(s));
-        umma_commit(aempty_bar(sa));
-        if (++s == ST) s = 0;
-        if (++sa == SA) { sa = 0; pha ^= 1u; }
+        umma_commit(empty_bar(s));
+        if (++s == ST) { s = 0; ph ^= 1u; }
       }
       if (!ok) {  // wait for this thread's own MMAs before the memory goes away
         umma_commit(drain_bar);
@@ -616,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // NVFP4: E4M3 code -> bf16x2 pair (e4m3 * 2^119), the factor frag_nvfp4
     // expects, as a 256-entry table shared by the four dequant warps
-    const uint32_t sctab = smem_u32(bars + 2 * ST + 2 * SA + 8);
+    const uint32_t sctab = smem_u32(bars + 3 * ST + 8);
     if constexpr (FMT == NVFP4 || FMT == MXFP4) {
       for (int c = threadIdx.x - 128; c < 256; c += 128)
         asm volatile("st.shared.u32 [%0], %1;" ::"r"(sctab + c * 4),
@@ -625,11 +620,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       asm volatile("bar.sync 1, 128;" ::: "memory");
     }
     for (int kt = 0; kt < KT; ++kt) {
-      const int s = kt % ST, sa = kt % SA;
-      const uint32_t ph = (uint32_t)(kt / ST) & 1u, pha = (uint32_t)(kt / SA) & 1u;
+      const int s = kt % ST;
+      const uint32_t ph = (uint32_t)(kt / ST) & 1u;
+      // The slot's previous MMAs are complete: the TMA warp waited for them
+      // (empty) before the load that completes this phase of tfull.
       if (!mbar_wait(tfull_bar(s), ph, abort, 32u)) break;
-      if (kt >= SA && !mbar_wait(aempty_bar(sa), pha ^ 1u, abort, 32u)) break;
-      const uint32_t abase = smem_u32(aring + sa * kAtile);
+      const uint32_t abase = smem_u32(aring + s * kAtile);
       const uint8_t* wpk = smem + s * kTstage + kXbytes;
       const uint32_t sd = smem_u32(sring + s * kSide);
       // Rows of tiles past N hold zero-filled codes (TMA fill) and stale side
@@ -786,8 +782,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #ifdef WQ_FAULT_TEST
         if (!(dw == 0 && kt == p.fault_stage))
 #endif
-          mbar_arrive(afull_bar(sa));   // A tile written
-        mbar_arrive(tempty_bar(s));     // packed tile read (already in registers)
+          mbar_arrive(afull_bar(s));  // A tile written (the packed tile is read)
       }
     }
   } else {
@@ -977,23 +972,15 @@ cudaError_t launch_bn(const LinearArgs& a) {
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  // ring depths: three dequantized A tiles; as many TMA stages as fit
+  // ring depth: as many slots (TMA stage + A tile + side data) as fit
   const uint32_t side = FMT == NVFP4 ? 512u : FMT == MXFP4 ? 256u : FMT == INT4_ASYM ? 128u : 0u;
-  const uint32_t tstage = (uint32_t)BN * 128u + kWpk;
-  int SA = 3;
-#ifdef WQ_TUNING
-  if (const char* e = getenv("WQ_PREFILL_SA")) {
-    const int v = atoi(e);
-    if (v >= 2 && v <= 8) SA = v;
-  }
-#endif
-  const uint32_t fixed = 1024u /* alignment */ + (uint32_t)SA * 16384u * (FMT == CB4 ? 2u : 1u) +
-                         8u * (2 * 8 + 2 * SA + 8) +
-                         1024u /* NVFP4 / MXFP4 scale table */;
-  int ST = (int)((227u * 1024u - fixed) / (tstage + side));
+  const uint32_t slot = (uint32_t)BN * 128u + kWpk + 16384u * (FMT == CB4 ? 2u : 1u) + side;
+  const uint32_t fixed = 1024u /* alignment */ + 8u * (3 * 8 + 8) /* barriers, tensor-memory slot,
+                         abort flag, grouped schedule */ + 1024u /* NVFP4 / MXFP4 scale table */;
+  int ST = (int)((227u * 1024u - fixed) / slot);
   if (ST > 8) ST = 8;
   if (ST < 2) ST = 2;
-  const size_t smem = (size_t)ST * (tstage + side) + fixed;
+  const size_t smem = (size_t)ST * slot + fixed;
   cudaError_t attr_err =
       ensure_max_dynamic_smem((const void*)prefill_kernel<FMT, BN, A8>, 227 * 1024);
   if (attr_err != cudaSuccess) return attr_err;
@@ -1008,7 +995,6 @@ cudaError_t launch_bn(const LinearArgs& a) {
   p.G = a.G;
   p.BN = BN;
   p.stages = ST;
-  p.astages = SA;
 #ifdef WQ_FAULT_TEST
   p.fault_stage = getenv("WQ_FAULT_PREFILL_STAGE") ? atoi(getenv("WQ_FAULT_PREFILL_STAGE")) : -1;
 #endif
