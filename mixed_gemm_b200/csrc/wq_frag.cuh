@@ -71,15 +71,26 @@ static __device__ __forceinline__ void frag_int3(uint32_t lo, uint32_t hi, int c
   }
 }
 
-// INT8 offset-binary bytes -> exact integers via the fp32 magic 2^23 + u.
-static __device__ __forceinline__ float i8val(uint32_t w, int i) {
-  return __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7440u | i)) - 8388736.0f;
+// INT8 offset-binary bytes u = q + 128 -> exact bf16 pairs of q, all in
+// bf16x2 integer arithmetic (no float conversion).  The byte pair (selected
+// by `sel` into the low bytes of the two halves) gives x = u per half; under
+// the exponent of 128 its low 7 bits read 128 + (u & 127), and adding -256
+// (u < 128) or -128 (u >= 128) leaves u - 128 = q, an integer in
+// [-128, 127] that bf16 holds exactly, so the addition rounds nothing.
+static __device__ __forceinline__ uint32_t badd2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+static __device__ __forceinline__ uint32_t i8pair(uint32_t w, uint32_t sel) {
+  const uint32_t x = __byte_perm(w, 0u, sel);
+  return badd2((x & 0x007F007Fu) | 0x43004300u, (x & 0x00800080u) ^ 0xC380C380u);
 }
 static __device__ __forceinline__ void frag_int8(uint32_t wg, uint32_t wg8, uint32_t (&a)[4]) {
-  a[0] = pack_bf16x2(i8val(wg, 0), i8val(wg, 1));
-  a[1] = pack_bf16x2(i8val(wg8, 0), i8val(wg8, 1));
-  a[2] = pack_bf16x2(i8val(wg, 2), i8val(wg, 3));
-  a[3] = pack_bf16x2(i8val(wg8, 2), i8val(wg8, 3));
+  a[0] = i8pair(wg, 0x4140u);   // bytes 0, 1
+  a[1] = i8pair(wg8, 0x4140u);
+  a[2] = i8pair(wg, 0x4342u);   // bytes 2, 3
+  a[3] = i8pair(wg8, 0x4342u);
 }
 
 // FP8 E4M3 bytes -> exact bf16 fragments.  A byte placed at bits 8..15 of a
