@@ -434,6 +434,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   // groups are counted in MMA steps of KS / 4 (16 for bf16, 32 for i8)
   const int KPG = kInt ? p.G / (KS / 4) : 4 * KT;  // MMA steps per accumulation group
   const int NG = 4 * KT / KPG;
+  // Persistent CTAs (one linear, no K split): the grid holds at most one CTA
+  // per SM and CTA b takes tiles b, b + gridDim.x, ... in the order above.
+  // The ring, the K-step count and the group count run on across a CTA's
+  // tiles, so the next tile's loads start while the MMAs of the current one
+  // drain, and its fold and stores overlap the next tile's main loop.  A K
+  // split or a grouped launch keeps one tile per CTA.
+  const bool persist = S == 1 && !p.offsets;
+  const int my_tiles =
+      persist ? ((p.N + 127) / 128 * mtiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x
+              : 1;
+  auto tile_at = [&](int i, int& t0, int& mm0) {
+    if (persist) {
+      const int t = (int)blockIdx.x + i * (int)gridDim.x;
+      t0 = (t / mtiles) * 8;
+      mm0 = (t % mtiles) * BN;
+    } else {
+      t0 = tile0;
+      mm0 = m0;
+    }
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
@@ -467,42 +487,50 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------------------------------------------------- producer
       const int64_t groups = kInt ? p.K / p.G : 0;
       int issued = 0;
-      for (int kt = 0; kt < KT; ++kt) {
-        const int s = kt % ST;
-        const uint32_t ph = (uint32_t)(kt / ST) & 1u;
-        if (kt >= ST && !mbar_wait(empty_bar(s), ph ^ 1u, abort, 1u)) break;
-        if (lane == 0) {
-          uint8_t* st = smem + s * kTstage;
-          mbar_expect_tx(tfull_bar(s), kXbytes + kWpk);
-          tma_load_2d(smem_u32(st), &tmX, (kt0 + kt) * KS, row0 + m0, tfull_bar(s));
-          tma_load_2d(smem_u32(st + kXbytes), &tmW, (kt0 + kt) * kWbox, expert * ntiles + tile0,
-                      tfull_bar(s));
-        }
-        if constexpr (kHasSide) {
-          const uint32_t sd = smem_u32(sring + s * kSide);
-          const int rt = lane >> 2, c = lane & 3;  // row tile, 16-byte quarter
-          const int64_t tile = tile0 + rt;
-          if (tile < ntiles) {
-            if constexpr (FMT == NVFP4) {
-              // 4 blocks of 16 K x 16 rows = 64 bytes per row tile
-              cp_async16(sd + rt * 64 + c * 16,
-                         scales_p + (tile * (p.K >> 4) + (kt0 + kt) * 4 + c) * 16);
-            } else if constexpr (FMT == MXFP4) {
-              // 2 blocks of 32 K x 16 rows = 32 bytes per row tile
-              if (c < 2)
-                cp_async16(sd + rt * 32 + c * 16,
-                           scales_p + (tile * (p.K >> 5) + (kt0 + kt) * 2 + c) * 16);
-            } else {
-              // the (one or two) groups of this K step: 8 bytes each
-              const int64_t g0 = ((int64_t)(kt0 + kt) * 64) / p.G;
-              const int ng = p.G == 32 ? 2 : 1;
-              if (c < ng)
-                cp_async8(sd + rt * 16 + c * 8, aux_p + (tile * groups + g0 + c) * 8);
-            }
+      bool run = true;
+      for (int i = 0; i < my_tiles && run; ++i) {
+        int t0, mm0;
+        tile_at(i, t0, mm0);
+        for (int kt = 0; kt < KT; ++kt) {
+          const int s = issued % ST;
+          const uint32_t ph = (uint32_t)(issued / ST) & 1u;
+          if (issued >= ST && !mbar_wait(empty_bar(s), ph ^ 1u, abort, 1u)) {
+            run = false;
+            break;
           }
-          cp_async_arrive(tfull_bar(s));
+          if (lane == 0) {
+            uint8_t* st = smem + s * kTstage;
+            mbar_expect_tx(tfull_bar(s), kXbytes + kWpk);
+            tma_load_2d(smem_u32(st), &tmX, (kt0 + kt) * KS, row0 + mm0, tfull_bar(s));
+            tma_load_2d(smem_u32(st + kXbytes), &tmW, (kt0 + kt) * kWbox, expert * ntiles + t0,
+                        tfull_bar(s));
+          }
+          if constexpr (kHasSide) {
+            const uint32_t sd = smem_u32(sring + s * kSide);
+            const int rt = lane >> 2, c = lane & 3;  // row tile, 16-byte quarter
+            const int64_t tile = t0 + rt;
+            if (tile < ntiles) {
+              if constexpr (FMT == NVFP4) {
+                // 4 blocks of 16 K x 16 rows = 64 bytes per row tile
+                cp_async16(sd + rt * 64 + c * 16,
+                           scales_p + (tile * (p.K >> 4) + (kt0 + kt) * 4 + c) * 16);
+              } else if constexpr (FMT == MXFP4) {
+                // 2 blocks of 32 K x 16 rows = 32 bytes per row tile
+                if (c < 2)
+                  cp_async16(sd + rt * 32 + c * 16,
+                             scales_p + (tile * (p.K >> 5) + (kt0 + kt) * 2 + c) * 16);
+              } else {
+                // the (one or two) groups of this K step: 8 bytes each
+                const int64_t g0 = ((int64_t)(kt0 + kt) * 64) / p.G;
+                const int ng = p.G == 32 ? 2 : 1;
+                if (c < ng)
+                  cp_async8(sd + rt * 16 + c * 8, aux_p + (tile * groups + g0 + c) * 8);
+              }
+            }
+            cp_async_arrive(tfull_bar(s));
+          }
+          ++issued;
         }
-        ++issued;
       }
       // before teardown, make sure no copy into this CTA's memory is in flight
       for (int kt = issued - ST < 0 ? 0 : issued - ST; kt < issued; ++kt)
@@ -520,7 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       int s = 0, g = 0, in_g = 0, gb = 0;
       uint32_t ph = 0, d = tmem;
-      for (int kt = 0; kt < KT && ok; ++kt) {
+      for (int kt = 0; kt < my_tiles * KT && ok; ++kt) {
         // the dequant warps arrive on afull only after they have seen this
         // slot's tfull, so afull alone orders the X tile too
         ok = mbar_wait(afull_bar(s), ph, abort, 8u);
@@ -619,7 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      : "memory");
       asm volatile("bar.sync 1, 128;" ::: "memory");
     }
-    for (int kt = 0; kt < KT; ++kt) {
+    for (int kt = 0; kt < my_tiles * KT; ++kt) {
       const int s = kt % ST;
       const uint32_t ph = (uint32_t)(kt / ST) & 1u;
       // The slot's previous MMAs are complete: the TMA warp waited for them
@@ -791,111 +819,115 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;            // tensor-memory lane quarter this warp may read
     const int frow = q * 32 + lane;    // accumulator row
     const int hcol = ((warp - 8) >> 2) * kHalf;
-    const int64_t n = (int64_t)tile0 * 16 + frow;
-    const bool nvalid = n < p.N;
     const int64_t groups = kInt ? p.K / p.G : 0;
-    // per-row factors, requested before the first wait: the group scales of
-    // the next two groups ride in registers ahead of the group being folded
     // group scales: bf16 (INT formats) or fp32 (FP8), same packed indexing
     const uint16_t* srow = (const uint16_t*)scales_p;
     const uint32_t* srow32 = (const uint32_t*)scales_p;
-    int64_t sidx = 0;
-    if (kInt && nvalid) {
-      const int r16 = (int)(n & 15);
-      sidx = (n >> 4) * groups * 16 + 2 * (r16 & 7) + (r16 >> 3);
-    }
     const int gfirst = kInt ? (kt0 * KS) / p.G : 0;  // first group of this CTA's K range
-    auto group_scale = [&](int gi) -> uint32_t {
-      if (!(kInt && nvalid && gi < NG)) return 0u;
-      if constexpr (kFp8) return __ldg(srow32 + sidx + (int64_t)(gfirst + gi) * 16);
-      return (uint32_t)__ldg(srow + sidx + (int64_t)(gfirst + gi) * 16);
-    };
-    uint32_t sc0 = group_scale(0), sc1 = group_scale(1);
-    float post = 1.f, bval = 0.f;
-    if (nvalid) {
-      if constexpr (FMT == CB4) post = bf16_bits_to_f32(__ldg((const uint16_t*)scales_p + n));
-      if constexpr (FMT == NVFP4) post = __ldg((const float*)aux_p) * 128.f;  // 2^7 of frag_nvfp4
-      if (bias_p) bval = bf16_bits_to_f32(__ldg(bias_p + n));
-    }
-    float acc[kHalf];
-#pragma unroll
-    for (int j = 0; j < kHalf; ++j) acc[j] = 0.f;
-    bool ok = true;
-    for (int g = 0; g < NG; ++g) {
-      const int gb = g & 1;
-      const uint32_t sc2 = group_scale(g + 2);
-      ok = mbar_wait(gfull_bar(gb), (uint32_t)(g >> 1) & 1u, abort, 64u);
-      if (!__all_sync(0xffffffffu, ok ? 1 : 0)) { ok = false; break; }
-      tc_fence_after();
-      const float sc = kFp8 ? __uint_as_float(sc0)
-                       : kInt          ? bf16_bits_to_f32((uint16_t)sc0)
-                                       : 1.f;
-      sc0 = sc1;
-      sc1 = sc2;
-      const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(gb * BN + hcol);
-      if constexpr (kHalf >= 32) {
-#pragma unroll
-        for (int c = 0; c < kHalf; c += 32) {
-          uint32_t v[32];
-          tmem_ld32(base + (uint32_t)c, v);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) acc[c + j] = fmaf(sc, tmem_val<A8>(v[j]), acc[c + j]);
-        }
-      } else {
-        uint32_t v[16];
-        tmem_ld16(base, v);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) acc[j] = fmaf(sc, tmem_val<A8>(v[j]), acc[j]);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(gempty_bar(gb));
-    }
     // A8: the per-token activation scale multiplies each output column
     auto colscale = [&](int m) -> float {
       if constexpr (A8) return __ldg((const float*)p.aux + m);
       return 1.f;
     };
-    if (S == 1) {
-      if (ok && nvalid) {
+    bool ok = true;
+    for (int i = 0; i < my_tiles && ok; ++i) {
+      int t0, mm0;
+      tile_at(i, t0, mm0);
+      const int64_t n = (int64_t)t0 * 16 + frow;
+      const bool nvalid = n < p.N;
+      // per-row factors, requested before the first wait: the group scales of
+      // the next two groups ride in registers ahead of the group being folded
+      int64_t sidx = 0;
+      if (kInt && nvalid) {
+        const int r16 = (int)(n & 15);
+        sidx = (n >> 4) * groups * 16 + 2 * (r16 & 7) + (r16 >> 3);
+      }
+      auto group_scale = [&](int gi) -> uint32_t {
+        if (!(kInt && nvalid && gi < NG)) return 0u;
+        if constexpr (kFp8) return __ldg(srow32 + sidx + (int64_t)(gfirst + gi) * 16);
+        return (uint32_t)__ldg(srow + sidx + (int64_t)(gfirst + gi) * 16);
+      };
+      uint32_t sc0 = group_scale(0), sc1 = group_scale(1);
+      float post = 1.f, bval = 0.f;
+      if (nvalid) {
+        if constexpr (FMT == CB4) post = bf16_bits_to_f32(__ldg((const uint16_t*)scales_p + n));
+        if constexpr (FMT == NVFP4) post = __ldg((const float*)aux_p) * 128.f;  // 2^7 of frag_nvfp4
+        if (bias_p) bval = bf16_bits_to_f32(__ldg(bias_p + n));
+      }
+      float acc[kHalf];
 #pragma unroll
-        for (int j = 0; j < kHalf; ++j) {
-          const int m = m0 + hcol + j;
-          if (m < rows)
-            p.out[(int64_t)(row0 + m) * p.N + n] =
-                (uint16_t)f32_to_bf16_bits(acc[j] * post * colscale(m) + bval);
+      for (int j = 0; j < kHalf; ++j) acc[j] = 0.f;
+      for (int g = 0; g < NG; ++g) {
+        const int gg = i * NG + g, gb = gg & 1;  // group count across this CTA's tiles
+        const uint32_t sc2 = group_scale(g + 2);
+        ok = mbar_wait(gfull_bar(gb), (uint32_t)(gg >> 1) & 1u, abort, 64u);
+        if (!__all_sync(0xffffffffu, ok ? 1 : 0)) { ok = false; break; }
+        tc_fence_after();
+        const float sc = kFp8 ? __uint_as_float(sc0)
+                         : kInt          ? bf16_bits_to_f32((uint16_t)sc0)
+                                         : 1.f;
+        sc0 = sc1;
+        sc1 = sc2;
+        const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(gb * BN + hcol);
+        if constexpr (kHalf >= 32) {
+#pragma unroll
+          for (int c = 0; c < kHalf; c += 32) {
+            uint32_t v[32];
+            tmem_ld32(base + (uint32_t)c, v);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc[c + j] = fmaf(sc, tmem_val<A8>(v[j]), acc[c + j]);
+          }
+        } else {
+          uint32_t v[16];
+          tmem_ld16(base, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) acc[j] = fmaf(sc, tmem_val<A8>(v[j]), acc[j]);
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(gempty_bar(gb));
       }
-    } else {
-      // Split-K reduction.  After the first cluster barrier the rings of
-      // every CTA in the cluster are idle (all its roles are done); CTA r
-      // owns columns [r*CW, (r+1)*CW) of the tile and receives every CTA's
-      // fp32 partial of them in slot [source][row][col] of its ring memory;
-      // after the second barrier it adds the slots in source order, folds
-      // and stores.
-      const int CW = BN / S;
-      const uint32_t slots = smem_u32(smem);
-      cluster_sync_all();
+      if (S == 1) {
+        if (ok && nvalid) {
 #pragma unroll
-      for (int j = 0; j < kHalf; j += 4) {
-        const int col = hcol + j;
-        const int owner = col / CW;
-        const uint32_t off = (uint32_t)(((split * 128 + frow) * CW + (col - owner * CW)) * 4);
-        st_cluster_v4(dsmem_addr(slots + off, (uint32_t)owner), acc[j], acc[j + 1], acc[j + 2],
-                      acc[j + 3]);
-      }
-      cluster_sync_all();
-      if (ok && nvalid) {
-        // this CTA's CW columns, split between the two fold warpgroups
-        const int half = (warp - 8) >> 2;
-        const float* sl = (const float*)smem;
-        for (int c = half * (CW / 2); c < (half + 1) * (CW / 2); ++c) {
-          float tot = 0.f;
-          for (int src = 0; src < S; ++src) tot += sl[(src * 128 + frow) * CW + c];
-          const int m = m0 + split * CW + c;
-          if (m < rows)
-            p.out[(int64_t)(row0 + m) * p.N + n] =
-                (uint16_t)f32_to_bf16_bits(tot * post * colscale(m) + bval);
+          for (int j = 0; j < kHalf; ++j) {
+            const int m = mm0 + hcol + j;
+            if (m < rows)
+              p.out[(int64_t)(row0 + m) * p.N + n] =
+                  (uint16_t)f32_to_bf16_bits(acc[j] * post * colscale(m) + bval);
+          }
+        }
+      } else {
+        // Split-K reduction.  After the first cluster barrier the rings of
+        // every CTA in the cluster are idle (all its roles are done); CTA r
+        // owns columns [r*CW, (r+1)*CW) of the tile and receives every CTA's
+        // fp32 partial of them in slot [source][row][col] of its ring memory;
+        // after the second barrier it adds the slots in source order, folds
+        // and stores.
+        const int CW = BN / S;
+        const uint32_t slots = smem_u32(smem);
+        cluster_sync_all();
+#pragma unroll
+        for (int j = 0; j < kHalf; j += 4) {
+          const int col = hcol + j;
+          const int owner = col / CW;
+          const uint32_t off = (uint32_t)(((split * 128 + frow) * CW + (col - owner * CW)) * 4);
+          st_cluster_v4(dsmem_addr(slots + off, (uint32_t)owner), acc[j], acc[j + 1], acc[j + 2],
+                        acc[j + 3]);
+        }
+        cluster_sync_all();
+        if (ok && nvalid) {
+          // this CTA's CW columns, split between the two fold warpgroups
+          const int half = (warp - 8) >> 2;
+          const float* sl = (const float*)smem;
+          for (int c = half * (CW / 2); c < (half + 1) * (CW / 2); ++c) {
+            float tot = 0.f;
+            for (int src = 0; src < S; ++src) tot += sl[(src * 128 + frow) * CW + c];
+            const int m = mm0 + split * CW + c;
+            if (m < rows)
+              p.out[(int64_t)(row0 + m) * p.N + n] =
+                  (uint16_t)f32_to_bf16_bits(tot * post * colscale(m) + bval);
+          }
         }
       }
     }
@@ -1041,8 +1073,13 @@ cudaError_t launch_bn(const LinearArgs& a) {
   if (a.offsets && ytiles > 65535) return cudaErrorNotSupported;
   const int64_t ncol = (a.N + 127) / 128;
   if (!a.offsets && ncol * ytiles > 0x7FFFFFFFLL) return cudaErrorNotSupported;
+  // one linear without a K split: persistent CTAs, at most one per SM (the
+  // shared-memory ring admits one CTA per SM), looping over the tiles
+  const int64_t tiles_total = ncol * ytiles;
+  const int64_t sms_avail = device_sm_count();
+  const int64_t ctas = (p.splits == 1 && tiles_total > sms_avail) ? sms_avail : tiles_total;
   dim3 grid = a.offsets ? dim3((unsigned)ncol, (unsigned)ytiles, (unsigned)p.splits)
-                        : dim3((unsigned)(ncol * ytiles), 1u, (unsigned)p.splits);
+                        : dim3((unsigned)ctas, 1u, (unsigned)p.splits);
   if (p.splits > 1) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
