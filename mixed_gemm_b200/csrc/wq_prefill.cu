@@ -366,62 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // time) and the activation tiles stay in L2.  Grouped: x is the column
   // block, y the schedule tile.
   const int mtiles = (p.M + BN - 1) / BN;
-  const int tile0 = (p.offsets ? (int)blockIdx.x : (int)blockIdx.x / mtiles) * 8;
-  // token rows of this CTA: [row0 + m0, row0 + min(m0 + BN, rows)) of x / out
-  int m0 = (p.offsets ? 0 : (int)blockIdx.x % mtiles) * BN, row0 = 0, rows = p.M, expert = 0;
-  if (p.offsets) {
-    // Device-side tile schedule of a grouped launch: experts in order, each
-    // with ceil(count / BN) token tiles; CTA y takes tile y of that list (the
-    // grid holds an upper bound of ceil(T / BN) + E tiles, the rest exit).
-    // Offsets outside [0, T] or decreasing make an expert empty and set bit
-    // 256 of the error word.
-    int* sched = (int*)(bars + 3 * ST + 6);  // 16 bytes before the scale table
-    if (warp == 0) {
-      const int target = (int)blockIdx.y;
-      int base = 0, found = 0;
-      for (int c0 = 0; c0 < p.E && !found; c0 += 32) {
-        const int ee = c0 + lane;
-        int cnt = 0, a = 0;
-        if (ee < p.E) {
-          const int64_t a64 = __ldg(p.offsets + ee), b64 = __ldg(p.offsets + ee + 1);
-          if (a64 >= 0 && a64 <= b64 && b64 <= p.T) {
-            a = (int)a64;
-            cnt = (int)(b64 - a64);
-          } else if (blockIdx.x == 0 && blockIdx.y == 0) {
-            atomicOr(&g_wq_device_error, 256u);
-          }
-        }
-        const int nt = (cnt + BN - 1) / BN;
-        int incl = nt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int v = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += v;
-        }
-        const bool mine = nt > 0 && target >= base + incl - nt && target < base + incl;
-        const unsigned bal = __ballot_sync(0xffffffffu, mine);
-        if (mine) {
-          sched[0] = ee;
-          sched[1] = a;
-          sched[2] = (target - (base + incl - nt)) * BN;
-          sched[3] = cnt;
-        }
-        found = bal != 0;
-        base += __shfl_sync(0xffffffffu, incl, 31);
-      }
-      if (!found && lane == 0) sched[0] = -1;
-    }
-    __syncthreads();
-    if (sched[0] < 0) return;  // past the end of the schedule: nothing to do
-    expert = sched[0];
-    row0 = sched[1];
-    m0 = sched[2];
-    rows = sched[3];
-  }
-  // this expert's (or the only) scales, aux and bias
-  const uint8_t* scales_p = (const uint8_t*)p.scales + (int64_t)expert * p.scale_stride;
-  const uint8_t* aux_p = (const uint8_t*)p.aux + (int64_t)expert * p.aux_stride;
-  const uint16_t* bias_p = p.bias ? p.bias + (int64_t)expert * p.N : nullptr;
+  const int ncolb = (p.N + 127) / 128;  // column blocks of 128 rows (8 row tiles)
   // K split: the S CTAs of a cluster (1, 1, S) share a tile and take
   // consecutive ranges of KT K steps each (whole scale groups); their fp32
   // partial tiles are summed through distributed shared memory at the end
@@ -434,26 +379,117 @@ __global__ void __launch_bounds__(kThreads, 1)
   // groups are counted in MMA steps of KS / 4 (16 for bf16, 32 for i8)
   const int KPG = kInt ? p.G / (KS / 4) : 4 * KT;  // MMA steps per accumulation group
   const int NG = 4 * KT / KPG;
-  // Persistent CTAs (one linear, no K split): the grid holds at most one CTA
-  // per SM and CTA b takes tiles b, b + gridDim.x, ... in the order above.
+
+  // Device-side tile schedule of a grouped launch: experts in order, each
+  // with ceil(count / BN) token tiles.  Offsets outside [0, T] or decreasing
+  // make an expert empty and set bit 256 of the error word.  `lookup` finds
+  // schedule tile y (a warp-collective scan over the experts; false past the
+  // end); with y < 0 it returns the number of schedule tiles in `mm0_`.
+  int* sched = (int*)(bars + 3 * ST + 6);  // 16 bytes before the scale table
+  auto lookup = [&](int y, int& e_, int& r0_, int& mm0_, int& rws_) -> bool {
+    int base = 0, found = 0;
+    for (int c0 = 0; c0 < p.E && !found; c0 += 32) {
+      const int ee = c0 + lane;
+      int cnt = 0, a = 0;
+      if (ee < p.E) {
+        const int64_t a64 = __ldg(p.offsets + ee), b64 = __ldg(p.offsets + ee + 1);
+        if (a64 >= 0 && a64 <= b64 && b64 <= p.T) {
+          a = (int)a64;
+          cnt = (int)(b64 - a64);
+        } else if (blockIdx.x == 0 && blockIdx.y == 0) {
+          atomicOr(&g_wq_device_error, 256u);
+        }
+      }
+      const int nt = (cnt + BN - 1) / BN;
+      int incl = nt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (y >= 0) {
+        const bool mine = nt > 0 && y >= base + incl - nt && y < base + incl;
+        const unsigned bal = __ballot_sync(0xffffffffu, mine);
+        if (bal) {
+          const int src = __ffs(bal) - 1;
+          e_ = __shfl_sync(0xffffffffu, ee, src);
+          r0_ = __shfl_sync(0xffffffffu, a, src);
+          mm0_ = (y - (base + __shfl_sync(0xffffffffu, incl - nt, src))) * BN;
+          rws_ = __shfl_sync(0xffffffffu, cnt, src);
+          found = 1;
+        }
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (y < 0) mm0_ = base;
+    return found != 0;
+  };
+  // Persistent CTAs (no K split; grouped launches except CB4, whose dequant
+  // tables are per expert): the grid holds at most one CTA per SM and CTA b
+  // takes tiles b, b + gridDim.x, ... (one linear: token tile fastest within
+  // a column block; grouped: column block fastest within a schedule tile).
   // The ring, the K-step count and the group count run on across a CTA's
   // tiles, so the next tile's loads start while the MMAs of the current one
-  // drain, and its fold and stores overlap the next tile's main loop.  A K
-  // split or a grouped launch keeps one tile per CTA.
-  const bool persist = S == 1 && !p.offsets;
+  // drain, and its fold and stores overlap the next tile's main loop.
+  // Otherwise one tile per CTA, from the grid coordinates.
+  const bool persist = S == 1 && !(p.offsets && FMT == CB4);
+  int ytot = mtiles;  // token tiles per column block
+  int tile0 = 0, m0 = 0, row0 = 0, rows = p.M, expert = 0;
+  if (p.offsets) {
+    if (warp == 0) {
+      int e_ = 0, r0_ = 0, mm0_ = 0, rws_ = 0;
+      const bool f = lookup(persist ? -1 : (int)blockIdx.y, e_, r0_, mm0_, rws_);
+      if (lane == 0) {
+        sched[0] = persist ? mm0_ : (f ? e_ : -1);
+        sched[1] = r0_;
+        sched[2] = mm0_;
+        sched[3] = rws_;
+      }
+    }
+    __syncthreads();
+    if (persist) {
+      ytot = sched[0];
+    } else {
+      if (sched[0] < 0) return;  // past the end of the schedule: nothing to do
+      tile0 = (int)blockIdx.x * 8;
+      expert = sched[0];
+      row0 = sched[1];
+      m0 = sched[2];
+      rows = sched[3];
+    }
+  } else if (!persist) {
+    tile0 = ((int)blockIdx.x / mtiles) * 8;
+    m0 = ((int)blockIdx.x % mtiles) * BN;
+  }
+  const int tiles_total = ncolb * ytot;
   const int my_tiles =
-      persist ? ((p.N + 127) / 128 * mtiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x
+      persist ? ((int)blockIdx.x < tiles_total
+                     ? (tiles_total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x
+                     : 0)
               : 1;
-  auto tile_at = [&](int i, int& t0, int& mm0) {
+  if (my_tiles == 0) return;  // (grouped) more CTAs than tiles: nothing to do
+  // Tile i of this CTA: first row tile, token offset, expert, x / out row base
+  // and expert rows.  Warp-collective for a persistent grouped launch.
+  struct Tile {
+    int t0, mm0, e, r0, rws;
+  };
+  auto tile_at = [&](int i) -> Tile {
+    Tile u{tile0, m0, expert, row0, rows};
     if (persist) {
       const int t = (int)blockIdx.x + i * (int)gridDim.x;
-      t0 = (t / mtiles) * 8;
-      mm0 = (t % mtiles) * BN;
-    } else {
-      t0 = tile0;
-      mm0 = m0;
+      if (p.offsets) {
+        u.t0 = (t % ncolb) * 8;
+        lookup(t / ncolb, u.e, u.r0, u.mm0, u.rws);
+      } else {
+        u.t0 = (t / mtiles) * 8;
+        u.mm0 = (t % mtiles) * BN;
+      }
     }
+    return u;
   };
+  // the first tile's expert (the dequant warps' CB4 centroids: CB4 grouped
+  // launches keep one tile per CTA)
+  const uint8_t* aux_p = (const uint8_t*)p.aux + (int64_t)expert * p.aux_stride;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
@@ -489,8 +525,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       int issued = 0;
       bool run = true;
       for (int i = 0; i < my_tiles && run; ++i) {
-        int t0, mm0;
-        tile_at(i, t0, mm0);
+        const Tile u = tile_at(i);
+        // this tile's expert: its block scales (NVFP4 / MXFP4) or zero-points
+        const uint8_t* scales_t = (const uint8_t*)p.scales + (int64_t)u.e * p.scale_stride;
+        const uint8_t* aux_t = (const uint8_t*)p.aux + (int64_t)u.e * p.aux_stride;
         for (int kt = 0; kt < KT; ++kt) {
           const int s = issued % ST;
           const uint32_t ph = (uint32_t)(issued / ST) & 1u;
@@ -501,30 +539,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) {
             uint8_t* st = smem + s * kTstage;
             mbar_expect_tx(tfull_bar(s), kXbytes + kWpk);
-            tma_load_2d(smem_u32(st), &tmX, (kt0 + kt) * KS, row0 + mm0, tfull_bar(s));
-            tma_load_2d(smem_u32(st + kXbytes), &tmW, (kt0 + kt) * kWbox, expert * ntiles + t0,
+            tma_load_2d(smem_u32(st), &tmX, (kt0 + kt) * KS, u.r0 + u.mm0, tfull_bar(s));
+            tma_load_2d(smem_u32(st + kXbytes), &tmW, (kt0 + kt) * kWbox, u.e * ntiles + u.t0,
                         tfull_bar(s));
           }
           if constexpr (kHasSide) {
             const uint32_t sd = smem_u32(sring + s * kSide);
             const int rt = lane >> 2, c = lane & 3;  // row tile, 16-byte quarter
-            const int64_t tile = t0 + rt;
+            const int64_t tile = u.t0 + rt;
             if (tile < ntiles) {
               if constexpr (FMT == NVFP4) {
                 // 4 blocks of 16 K x 16 rows = 64 bytes per row tile
                 cp_async16(sd + rt * 64 + c * 16,
-                           scales_p + (tile * (p.K >> 4) + (kt0 + kt) * 4 + c) * 16);
+                           scales_t + (tile * (p.K >> 4) + (kt0 + kt) * 4 + c) * 16);
               } else if constexpr (FMT == MXFP4) {
                 // 2 blocks of 32 K x 16 rows = 32 bytes per row tile
                 if (c < 2)
                   cp_async16(sd + rt * 32 + c * 16,
-                             scales_p + (tile * (p.K >> 5) + (kt0 + kt) * 2 + c) * 16);
+                             scales_t + (tile * (p.K >> 5) + (kt0 + kt) * 2 + c) * 16);
               } else {
                 // the (one or two) groups of this K step: 8 bytes each
                 const int64_t g0 = ((int64_t)(kt0 + kt) * 64) / p.G;
                 const int ng = p.G == 32 ? 2 : 1;
                 if (c < ng)
-                  cp_async8(sd + rt * 16 + c * 8, aux_p + (tile * groups + g0 + c) * 8);
+                  cp_async8(sd + rt * 16 + c * 8, aux_t + (tile * groups + g0 + c) * 8);
               }
             }
             cp_async_arrive(tfull_bar(s));
@@ -820,9 +858,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int frow = q * 32 + lane;    // accumulator row
     const int hcol = ((warp - 8) >> 2) * kHalf;
     const int64_t groups = kInt ? p.K / p.G : 0;
-    // group scales: bf16 (INT formats) or fp32 (FP8), same packed indexing
-    const uint16_t* srow = (const uint16_t*)scales_p;
-    const uint32_t* srow32 = (const uint32_t*)scales_p;
     const int gfirst = kInt ? (kt0 * KS) / p.G : 0;  // first group of this CTA's K range
     // A8: the per-token activation scale multiplies each output column
     auto colscale = [&](int m) -> float {
@@ -831,9 +866,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     bool ok = true;
     for (int i = 0; i < my_tiles && ok; ++i) {
-      int t0, mm0;
-      tile_at(i, t0, mm0);
-      const int64_t n = (int64_t)t0 * 16 + frow;
+      const Tile u = tile_at(i);
+      const int mm0 = u.mm0, row0 = u.r0, rows = u.rws;
+      const int64_t n = (int64_t)u.t0 * 16 + frow;
+      // this tile's expert (or the only) scales, aux and bias
+      const uint8_t* scales_p = (const uint8_t*)p.scales + (int64_t)u.e * p.scale_stride;
+      const uint8_t* aux_t = (const uint8_t*)p.aux + (int64_t)u.e * p.aux_stride;
+      const uint16_t* bias_p = p.bias ? p.bias + (int64_t)u.e * p.N : nullptr;
+      // group scales: bf16 (INT formats) or fp32 (FP8), same packed indexing
+      const uint16_t* srow = (const uint16_t*)scales_p;
+      const uint32_t* srow32 = (const uint32_t*)scales_p;
       const bool nvalid = n < p.N;
       // per-row factors, requested before the first wait: the group scales of
       // the next two groups ride in registers ahead of the group being folded
@@ -851,7 +893,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float post = 1.f, bval = 0.f;
       if (nvalid) {
         if constexpr (FMT == CB4) post = bf16_bits_to_f32(__ldg((const uint16_t*)scales_p + n));
-        if constexpr (FMT == NVFP4) post = __ldg((const float*)aux_p) * 128.f;  // 2^7 of frag_nvfp4
+        if constexpr (FMT == NVFP4) post = __ldg((const float*)aux_t) * 128.f;  // 2^7 of frag_nvfp4
         if (bias_p) bval = bf16_bits_to_f32(__ldg(bias_p + n));
       }
       float acc[kHalf];
@@ -1073,13 +1115,16 @@ cudaError_t launch_bn(const LinearArgs& a) {
   if (a.offsets && ytiles > 65535) return cudaErrorNotSupported;
   const int64_t ncol = (a.N + 127) / 128;
   if (!a.offsets && ncol * ytiles > 0x7FFFFFFFLL) return cudaErrorNotSupported;
-  // one linear without a K split: persistent CTAs, at most one per SM (the
-  // shared-memory ring admits one CTA per SM), looping over the tiles
+  // no K split (and, grouped, not CB4): persistent CTAs, at most one per SM
+  // (the shared-memory ring admits one CTA per SM), looping over the tiles
+  // (grouped: over an upper bound of them; the kernel reads the schedule)
+  const bool persist = p.splits == 1 && !(a.offsets && FMT == CB4);
   const int64_t tiles_total = ncol * ytiles;
   const int64_t sms_avail = device_sm_count();
-  const int64_t ctas = (p.splits == 1 && tiles_total > sms_avail) ? sms_avail : tiles_total;
-  dim3 grid = a.offsets ? dim3((unsigned)ncol, (unsigned)ytiles, (unsigned)p.splits)
-                        : dim3((unsigned)ctas, 1u, (unsigned)p.splits);
+  const int64_t ctas = (persist && tiles_total > sms_avail) ? sms_avail : tiles_total;
+  dim3 grid = persist ? dim3((unsigned)ctas, 1u, 1u)
+              : a.offsets ? dim3((unsigned)ncol, (unsigned)ytiles, (unsigned)p.splits)
+                          : dim3((unsigned)ctas, 1u, (unsigned)p.splits);
   if (p.splits > 1) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
