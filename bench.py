@@ -597,6 +597,9 @@ def time_moe(mw, steps, warmup, device, l2, world, local_rank, do_e2e, do_cpu, c
     work_bytes = W.moe_bytes(mw, counts)
     flops = 2.0 * mw.rows * mw.N * mw.K
     prefill_like = mw.rows // mw.E > 64
+    # the library's dispatch: the decode kernel while the mean rows per expert
+    # (rounded up) is at most 16, the tcgen05 kernel above
+    tc_path = -(-mw.rows // mw.E) > 16
     counter = [0]
 
     def step():
@@ -759,7 +762,9 @@ def time_moe(mw, steps, warmup, device, l2, world, local_rank, do_e2e, do_cpu, c
                              "events on the launch stream"},
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak,
                      "unit": "TFLOP/s" if prefill_like else "GB/s", "frac": achieved / peak,
-                     "traffic": None, "peak_source": pk_kind, "kernel": "prefill_kernel"},
+                     "traffic": recorded_traffic("wq_prefill.cu", mw.name) if tc_path else None,
+                     "peak_source": pk_kind,
+                     "kernel": "prefill_kernel" if tc_path else "decode_kernel"},
         "gpu_launches": steps, "clocks": clk, "e2e": e2e, "cpu_baseline": cb,
         "context": {"host_loop_us_per_step": loop_us,
                     "single_launch_us_per_step": ms / steps * 1e3,
