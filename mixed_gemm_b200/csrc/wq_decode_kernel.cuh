@@ -122,6 +122,28 @@ __device__ __forceinline__ bool mbar_wait0(uint32_t bar, unsigned* err) {
   atomicOr(err, 128u);
   return false;
 }
+// The same bounded wait, at cluster scope (acquire of the other ranks'
+// distributed-shared-memory writes), for phase 0 of the reduction barrier.
+__device__ __forceinline__ bool mbar_wait0_cluster(uint32_t bar, unsigned* err) {
+#ifdef WQ_FAULT_TEST
+  const uint32_t limit = 1u << 16;
+#else
+  const uint32_t limit = 1u << 22;
+#endif
+  for (uint32_t i = 0; i < limit; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], 0;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar)
+        : "memory");
+    if (ok) return true;
+  }
+  atomicOr(err, 128u);
+  return false;
+}
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
@@ -167,10 +189,6 @@ __device__ __forceinline__ void cluster_arrive_relaxed() {
 }
 __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                   : "memory");
 }
 
 // KW warps per CTA; each keeps a ring of D blocks (per row tile) of weight
@@ -265,8 +283,12 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
   }
   const int tile0 = rgroup * RT;
   const uint32_t xbar = (uint32_t)__cvta_generic_to_shared(smem) + (uint32_t)p.bar_off;
+  // rank 0's reduction barrier: one arrival per other rank of the cluster
+  const uint32_t rbar = xbar + 8u;
   if (threadIdx.x == 0) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(xbar) : "memory");
+    if (cs > 1 && rank == 0)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(rbar), "r"(cs - 1) : "memory");
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   const int K = p.K;
@@ -607,7 +629,9 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
 
   // ---- reduction: warps -> CTA partial in this CTA's shared memory (the X
   // slice region is free now); the CTA partial goes into slot `rank` of
-  // cluster rank 0's shared memory; one cluster barrier; rank 0 sums.
+  // cluster rank 0's shared memory.  The other ranks then arrive once each
+  // on rank 0's reduction barrier (release at cluster scope) and finish;
+  // rank 0 waits for their arrivals, sums the slots in rank order and stores.
   __syncthreads();  // every warp is done reading the staged slice
   float* loc = (float*)smem;
   float* slots = (float*)(smem + p.red_off);
@@ -631,9 +655,20 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
     for (int w = 0; w < KW; ++w) sum += loc[w * NV * 32 + idx];
     slots0[rank * NV * 32 + idx] = sum;
   }
-  if (cs > 1) cluster_sync_all();
-  else __syncthreads();
-  if (rank != 0) return;
+  bool rok = true;
+  if (cs > 1 && rank != 0) {
+    asm volatile("fence.acq_rel.cluster;" ::: "memory");  // this thread's slot writes
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      uint32_t rb0;
+      asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(rb0) : "r"(rbar));
+      asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(rb0)
+                   : "memory");
+    }
+    return;
+  }
+  __syncthreads();  // rank 0's own slot
+  if (cs > 1) rok = mbar_wait0_cluster(rbar, p.err);
 
   float tsc = 1.f;
   if constexpr (FMT == NVFP4) tsc = __ldg((const float*)aux_g) * 128.f;  // 2^7 of frag_nvfp4
@@ -645,7 +680,7 @@ __global__ void __launch_bounds__(KW * 32) decode_kernel(const DecodeParams p) {
     const int gg = ln >> 2, tt = ln & 3;
     const int n = (tile0 + r) * 16 + gg + 8 * (i >> 1);
     const int m = nt * 8 + 2 * tt + (i & 1);
-    if (m < M && xok) {
+    if (m < M && xok && rok) {
       float fold = tsc;
       if constexpr (FMT == CB4) fold = bf16_bits_to_f32(__ldg((const uint16_t*)scales_g + n));
       float y = tot * fold;
