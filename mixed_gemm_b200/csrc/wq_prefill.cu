@@ -35,7 +35,9 @@
 // to bf16 and stores Y.  When the tiles would fill at most half of the SMs,
 // the K range is split over a thread-block cluster (1, 1, S) and the fp32
 // partial tiles are summed through distributed shared memory before the
-// epilogue.  Registers are rebalanced per warpgroup with
+// epilogue; otherwise the CTAs are persistent (at most one per SM, each
+// looping over tiles with its pipelines running on from one tile to the
+// next).  Registers are rebalanced per warpgroup with
 // setmaxnreg (56 / 104 / 168 / 168 of the 128 per thread launched).  Every
 // mbarrier wait has an iteration limit; a wait that runs out records an error
 // word and the CTA winds down.
@@ -360,11 +362,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t drain_bar = smem_u32(bars + 3 * ST + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // One linear: the grid is one-dimensional (times the K split) with the
-  // token tile varying fastest, so the CTAs resident at once share a few
-  // column blocks of the weight (each read by up to M / BN CTAs close in
-  // time) and the activation tiles stay in L2.  Grouped: x is the column
-  // block, y the schedule tile.
+  // Tile order.  One linear: the token tile varies fastest, so the CTAs
+  // resident at once share a few column blocks of the weight (each read by up
+  // to M / BN CTAs close in time) and the activation tiles stay in L2.
+  // Grouped: the column block varies fastest within a schedule tile.
   const int mtiles = (p.M + BN - 1) / BN;
   const int ncolb = (p.N + 127) / 128;  // column blocks of 128 rows (8 row tiles)
   // K split: the S CTAs of a cluster (1, 1, S) share a tile and take
