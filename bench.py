@@ -762,7 +762,8 @@ def time_moe(mw, steps, warmup, device, l2, world, local_rank, do_e2e, do_cpu, c
                              "events on the launch stream"},
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak,
                      "unit": "TFLOP/s" if prefill_like else "GB/s", "frac": achieved / peak,
-                     "traffic": recorded_traffic("wq_prefill.cu", mw.name) if tc_path else None,
+                     "traffic": recorded_traffic("wq_prefill.cu" if tc_path else "wq_decode_kernel.cuh",
+                                                 mw.name),
                      "peak_source": pk_kind,
                      "kernel": "prefill_kernel" if tc_path else "decode_kernel"},
         "gpu_launches": steps, "clocks": clk, "e2e": e2e, "cpu_baseline": cb,
